@@ -1,0 +1,133 @@
+"""float64 CPU oracle for Lightning Attention — TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The product library never calls it and
+shares no code with it.
+
+The arithmetic lives in ``lightning_oracle.c`` (three forms of the same
+result: F1 definition, F2 token recurrence, F3 blockwise, plus one decode
+step; see that file's header for the formulas and their sources on the
+"MINIMAX SIGNAL LAB · M1" page, §03 Lightning Attention). This module only
+marshals numpy arrays into it.
+
+Inputs are numpy arrays: float32, or uint16 holding bfloat16 bit patterns.
+Outputs are float64.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build as _build
+
+_F32, _BF16 = 0, 1
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(_build())
+        vp, ip, fp, dp = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
+        for name in ("la_oracle_definition", "la_oracle_recurrence"):
+            fn = getattr(lib, name)
+            fn.argtypes = [vp, vp, vp, ip, fp, ip, ip, ip, ip, fp, dp, dp]
+            fn.restype = ctypes.c_int
+        lib.la_oracle_blockwise.argtypes = [vp, vp, vp, ip, fp, ip, ip, ip, ip, ip, fp, dp, dp]
+        lib.la_oracle_blockwise.restype = ctypes.c_int
+        lib.la_oracle_decode.argtypes = [vp, vp, vp, ip, fp, ip, ip, ip, dp, dp]
+        lib.la_oracle_decode.restype = ctypes.c_int
+        lib.la_oracle_max_threads.restype = ctypes.c_int
+        lib.la_oracle_set_threads.argtypes = [ip]
+        _lib = lib
+    return _lib
+
+
+def threads() -> int:
+    """Number of OpenMP threads the oracle uses."""
+    return _load().la_oracle_max_threads()
+
+
+def set_threads(n: int) -> None:
+    _load().la_oracle_set_threads(int(n))
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return _F32
+    if a.dtype == np.uint16:
+        return _BF16
+    raise TypeError("oracle inputs must be float32 or uint16 (bfloat16 bits), got %s" % a.dtype)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _prepare(q, k, v, slopes, state_in):
+    q, k, v = (np.ascontiguousarray(x) for x in (q, k, v))
+    if not (q.shape == k.shape == v.shape) or q.ndim != 4:
+        raise ValueError("q, k, v must share one [batch, heads, seq, dim] shape")
+    code = _dtype_code(q)
+    if _dtype_code(k) != code or _dtype_code(v) != code:
+        raise TypeError("q, k, v must share a dtype")
+    b, h, L, d = q.shape
+    slopes = np.ascontiguousarray(slopes, dtype=np.float32)
+    if slopes.shape != (h,):
+        raise ValueError("slopes must have shape [heads]")
+    if state_in is not None:
+        state_in = np.ascontiguousarray(state_in, dtype=np.float32)
+        if state_in.shape != (b, h, d, d):
+            raise ValueError("state_in must have shape [batch, heads, dim, dim]")
+    return q, k, v, code, slopes, state_in, (b, h, L, d)
+
+
+def prefill(q, k, v, slopes, state_in=None, form="recurrence", block=None):
+    """Return (o, state_out) in float64 for one prefill.
+
+    form: "definition" (F1), "recurrence" (F2) or "blockwise" (F3, needs block).
+    """
+    q, k, v, code, slopes, state_in, (b, h, L, d) = _prepare(q, k, v, slopes, state_in)
+    o = np.empty((b, h, L, d), dtype=np.float64)
+    s_out = np.empty((b, h, d, d), dtype=np.float64)
+    lib = _load()
+    args_head = (_ptr(q), _ptr(k), _ptr(v), code, _ptr(slopes), b, h, L, d)
+    if form == "definition":
+        rc = lib.la_oracle_definition(*args_head, _ptr(state_in), _ptr(o), _ptr(s_out))
+    elif form == "recurrence":
+        rc = lib.la_oracle_recurrence(*args_head, _ptr(state_in), _ptr(o), _ptr(s_out))
+    elif form == "blockwise":
+        if block is None or int(block) <= 0:
+            raise ValueError("the blockwise form needs a positive block size")
+        rc = lib.la_oracle_blockwise(*args_head, int(block), _ptr(state_in), _ptr(o), _ptr(s_out))
+    else:
+        raise ValueError("unknown form %r" % (form,))
+    if rc != 0:
+        raise RuntimeError("oracle %s failed (rc=%d)" % (form, rc))
+    return o, s_out
+
+
+def decode(q, k, v, slopes, state):
+    """One decode step. q, k, v: [batch, heads, dim]; state: [batch, heads, dim, dim].
+
+    Returns (o float64 [batch, heads, dim], new state float64)."""
+    q, k, v = (np.ascontiguousarray(x) for x in (q, k, v))
+    if not (q.shape == k.shape == v.shape) or q.ndim != 3:
+        raise ValueError("q, k, v must share one [batch, heads, dim] shape")
+    code = _dtype_code(q)
+    b, h, d = q.shape
+    slopes = np.ascontiguousarray(slopes, dtype=np.float32)
+    S = np.array(state, dtype=np.float64, copy=True, order="C")
+    if S.shape != (b, h, d, d):
+        raise ValueError("state must have shape [batch, heads, dim, dim]")
+    o = np.empty((b, h, d), dtype=np.float64)
+    rc = _load().la_oracle_decode(_ptr(q), _ptr(k), _ptr(v), code, _ptr(slopes), b, h, d,
+                                  _ptr(S), _ptr(o))
+    if rc != 0:
+        raise RuntimeError("oracle decode failed (rc=%d)" % rc)
+    return o, S
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Widen bfloat16 bit patterns (uint16) to float64 exactly."""
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

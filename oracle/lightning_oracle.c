@@ -1,0 +1,282 @@
+/*
+ * Lightning Attention oracle: plain, slow, float64 CPU reference.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path links, loads or
+ * calls this file; only the test suite, the smoke check and the bench's
+ * CPU-baseline leg do. It shares no code, header or constant with the CUDA
+ * library, and it reads its inputs exactly as the GPU does: bf16 bit
+ * patterns or float32 values are widened to double without rounding, and
+ * the per-head slopes are the same float32 numbers, widened.
+ *
+ * What is computed (per batch b, head h with decay slope s, length L):
+ *
+ *   o_i   = sum_{j<=i} e^{-s(i-j)} (q_i . k_j) v_j  +  e^{-s(i+1)} q_i S_in
+ *   S_out = e^{-sL} S_in + sum_{j<L} e^{-s(L-1-j)} k_j^T v_j
+ *
+ * S_in is the carried-in state, read as the state "one position before the
+ * first token". Source: "MINIMAX SIGNAL LAB · M1" (ailearn.mscapital.top),
+ * §03 Lightning Attention: the intra-block term O_intra = [(Q K^T) ⊙ D] V
+ * with D_ij = e^{-s_h(i-j)} 1[i>=j], the inter-block term
+ * O_inter = (Q ⊙ d_q) S_{t-1}, the state update
+ * S_t = e^{-s_h B} S_{t-1} + (K ⊙ d_k)^T V, the recursive fixed-size KV
+ * state of the same section, and the last-short-block rule (a final block
+ * of m < B tokens uses m). The pages print no values for d_q and d_k; the
+ * readings used here are d_q[i] = e^{-s(i+1)}, d_k[j] = e^{-s(m-1-j)} and a
+ * block decay of e^{-s m}: the only exponents for which the blockwise form
+ * equals the token-level definition above (the tests check that equality
+ * for every block size).
+ *
+ * Three forms, each written straight from its definition:
+ *   F1 la_oracle_definition : the quadratic sum above, O(L^2 d) per head.
+ *   F2 la_oracle_recurrence : token recurrence S_i = e^{-s} S_{i-1} + k_i^T v_i,
+ *                             o_i = q_i S_i  (the "cumsum" form of naive
+ *                             linear attention, fishai.com.cn article on
+ *                             M1), O(L d^2) per head; the full-size oracle.
+ *   F3 la_oracle_blockwise  : the block formulas of §03 for a given B.
+ * plus la_oracle_decode, one recurrent step for a single new token.
+ *
+ * Layouts: q, k, v, o are [batch][heads][seq][dim] contiguous (o for decode
+ * is [batch][heads][dim]); states are [batch][heads][dim(k)][dim(v)].
+ * Parallelism: OpenMP over (batch, head) only; the arithmetic inside one
+ * head is a plain sequential loop.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+
+/* Widen one stored element to double. bf16 is the top half of a float32. */
+static double widen(const void *base, int dtype, size_t idx) {
+    if (dtype == ORACLE_BF16) {
+        uint32_t bits = (uint32_t)((const uint16_t *)base)[idx] << 16;
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    return (double)((const float *)base)[idx];
+}
+
+/* Copy one head's [seq][dim] slice into a double buffer. */
+static void widen_head(const void *src, int dtype, size_t offset, size_t count, double *dst) {
+    for (size_t n = 0; n < count; ++n) dst[n] = widen(src, dtype, offset + n);
+}
+
+static int check_args(const void *q, const void *k, const void *v, int dtype, const float *slopes,
+                      int batch, int heads, int seq, int dim) {
+    if (!q || !k || !v || !slopes) return 1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16) return 1;
+    if (batch < 0 || heads <= 0 || seq < 0 || dim <= 0) return 1;
+    return 0;
+}
+
+int la_oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void la_oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* F1: the definition, term by term. */
+int la_oracle_definition(const void *q, const void *k, const void *v, int dtype,
+                         const float *slopes, int batch, int heads, int seq, int dim,
+                         const float *state_in, double *o, double *state_out) {
+    if (check_args(q, k, v, dtype, slopes, batch, heads, seq, dim) || !o) return 1;
+    const long BH = (long)batch * heads;
+    const size_t L = (size_t)seq, d = (size_t)dim;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        const int h = (int)(bh % heads);
+        const double s = (double)slopes[h];
+        double *Q = malloc(sizeof(double) * L * d + 1);
+        double *K = malloc(sizeof(double) * L * d + 1);
+        double *V = malloc(sizeof(double) * L * d + 1);
+        double *S0 = malloc(sizeof(double) * d * d);
+        if (!Q || !K || !V || !S0) {
+            fail = 1;
+            free(Q); free(K); free(V); free(S0);
+            continue;
+        }
+        widen_head(q, dtype, (size_t)bh * L * d, L * d, Q);
+        widen_head(k, dtype, (size_t)bh * L * d, L * d, K);
+        widen_head(v, dtype, (size_t)bh * L * d, L * d, V);
+        for (size_t n = 0; n < d * d; ++n)
+            S0[n] = state_in ? (double)state_in[(size_t)bh * d * d + n] : 0.0;
+        double *O = o + (size_t)bh * L * d;
+        for (size_t i = 0; i < L; ++i) {
+            for (size_t c = 0; c < d; ++c) O[i * d + c] = 0.0;
+            for (size_t j = 0; j <= i; ++j) {
+                double qk = 0.0;
+                for (size_t c = 0; c < d; ++c) qk += Q[i * d + c] * K[j * d + c];
+                const double w = exp(-s * (double)(i - j)) * qk;
+                for (size_t c = 0; c < d; ++c) O[i * d + c] += w * V[j * d + c];
+            }
+            /* carried-in state, seen from position i: i+1 steps of decay */
+            const double dq = exp(-s * (double)(i + 1));
+            for (size_t c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (size_t r = 0; r < d; ++r) acc += Q[i * d + r] * S0[r * d + c];
+                O[i * d + c] += dq * acc;
+            }
+        }
+        if (state_out) {
+            double *S = state_out + (size_t)bh * d * d;
+            const double dL = exp(-s * (double)L);
+            for (size_t n = 0; n < d * d; ++n) S[n] = dL * S0[n];
+            for (size_t j = 0; j < L; ++j) {
+                const double w = exp(-s * (double)(L - 1 - j));
+                for (size_t r = 0; r < d; ++r)
+                    for (size_t c = 0; c < d; ++c) S[r * d + c] += w * K[j * d + r] * V[j * d + c];
+            }
+        }
+        free(Q); free(K); free(V); free(S0);
+    }
+    return fail;
+}
+
+/* F2: token recurrence. S_i = e^{-s} S_{i-1} + k_i^T v_i ; o_i = q_i S_i. */
+int la_oracle_recurrence(const void *q, const void *k, const void *v, int dtype,
+                         const float *slopes, int batch, int heads, int seq, int dim,
+                         const float *state_in, double *o, double *state_out) {
+    if (check_args(q, k, v, dtype, slopes, batch, heads, seq, dim) || !o) return 1;
+    const long BH = (long)batch * heads;
+    const size_t L = (size_t)seq, d = (size_t)dim;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        const int h = (int)(bh % heads);
+        const double decay = exp(-(double)slopes[h]);
+        double *S = malloc(sizeof(double) * d * d);
+        double *qi = malloc(sizeof(double) * d), *ki = malloc(sizeof(double) * d),
+               *vi = malloc(sizeof(double) * d);
+        if (!S || !qi || !ki || !vi) {
+            fail = 1;
+            free(S); free(qi); free(ki); free(vi);
+            continue;
+        }
+        for (size_t n = 0; n < d * d; ++n)
+            S[n] = state_in ? (double)state_in[(size_t)bh * d * d + n] : 0.0;
+        const size_t base = (size_t)bh * L * d;
+        for (size_t i = 0; i < L; ++i) {
+            widen_head(q, dtype, base + i * d, d, qi);
+            widen_head(k, dtype, base + i * d, d, ki);
+            widen_head(v, dtype, base + i * d, d, vi);
+            for (size_t r = 0; r < d; ++r)
+                for (size_t c = 0; c < d; ++c) S[r * d + c] = decay * S[r * d + c] + ki[r] * vi[c];
+            double *oi = o + base + i * d;
+            for (size_t c = 0; c < d; ++c) oi[c] = 0.0;
+            for (size_t r = 0; r < d; ++r)
+                for (size_t c = 0; c < d; ++c) oi[c] += qi[r] * S[r * d + c];
+        }
+        if (state_out) memcpy(state_out + (size_t)bh * d * d, S, sizeof(double) * d * d);
+        free(S); free(qi); free(ki); free(vi);
+    }
+    return fail;
+}
+
+/* F3: the blockwise method, block by block, as the block formulas state it. */
+int la_oracle_blockwise(const void *q, const void *k, const void *v, int dtype,
+                        const float *slopes, int batch, int heads, int seq, int dim, int block,
+                        const float *state_in, double *o, double *state_out) {
+    if (check_args(q, k, v, dtype, slopes, batch, heads, seq, dim) || !o || block <= 0) return 1;
+    const long BH = (long)batch * heads;
+    const size_t L = (size_t)seq, d = (size_t)dim, B = (size_t)block;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        const int h = (int)(bh % heads);
+        const double s = (double)slopes[h];
+        double *S = malloc(sizeof(double) * d * d);     /* S_{t-1} */
+        double *Sn = malloc(sizeof(double) * d * d);    /* S_t     */
+        double *Qt = malloc(sizeof(double) * B * d), *Kt = malloc(sizeof(double) * B * d),
+               *Vt = malloc(sizeof(double) * B * d), *P = malloc(sizeof(double) * B * B);
+        if (!S || !Sn || !Qt || !Kt || !Vt || !P) {
+            fail = 1;
+            free(S); free(Sn); free(Qt); free(Kt); free(Vt); free(P);
+            continue;
+        }
+        for (size_t n = 0; n < d * d; ++n)
+            S[n] = state_in ? (double)state_in[(size_t)bh * d * d + n] : 0.0;
+        const size_t base = (size_t)bh * L * d;
+        for (size_t t0 = 0; t0 < L; t0 += B) {
+            const size_t m = (L - t0 < B) ? (L - t0) : B; /* last block: actual length m */
+            widen_head(q, dtype, base + t0 * d, m * d, Qt);
+            widen_head(k, dtype, base + t0 * d, m * d, Kt);
+            widen_head(v, dtype, base + t0 * d, m * d, Vt);
+            /* P = (Q_t K_t^T) ⊙ D,  D_ij = e^{-s(i-j)} 1[i>=j] */
+            for (size_t i = 0; i < m; ++i)
+                for (size_t j = 0; j < m; ++j) {
+                    double qk = 0.0;
+                    for (size_t c = 0; c < d; ++c) qk += Qt[i * d + c] * Kt[j * d + c];
+                    const double D = (i >= j) ? exp(-s * (double)(i - j)) : 0.0;
+                    P[i * B + j] = qk * D;
+                }
+            double *Ot = o + base + t0 * d;
+            for (size_t i = 0; i < m; ++i) {
+                const double dq = exp(-s * (double)(i + 1)); /* query decay d_q[i] */
+                for (size_t c = 0; c < d; ++c) {
+                    double intra = 0.0, inter = 0.0;
+                    for (size_t j = 0; j < m; ++j) intra += P[i * B + j] * Vt[j * d + c];
+                    for (size_t r = 0; r < d; ++r) inter += (Qt[i * d + r] * dq) * S[r * d + c];
+                    Ot[i * d + c] = intra + inter;
+                }
+            }
+            /* S_t = e^{-s m} S_{t-1} + (K_t ⊙ d_k)^T V_t,  d_k[j] = e^{-s(m-1-j)} */
+            const double dblock = exp(-s * (double)m);
+            for (size_t r = 0; r < d; ++r)
+                for (size_t c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    for (size_t j = 0; j < m; ++j)
+                        acc += (Kt[j * d + r] * exp(-s * (double)(m - 1 - j))) * Vt[j * d + c];
+                    Sn[r * d + c] = dblock * S[r * d + c] + acc;
+                }
+            double *tmp = S; S = Sn; Sn = tmp;
+        }
+        if (state_out) memcpy(state_out + (size_t)bh * d * d, S, sizeof(double) * d * d);
+        free(S); free(Sn); free(Qt); free(Kt); free(Vt); free(P);
+    }
+    return fail;
+}
+
+/* One recurrent step for a single new token per (batch, head):
+ * S <- e^{-s} S + k^T v, then o = q S (the new token is seen with e^0 = 1).
+ * q, k, v: [batch][heads][dim]; state: [batch][heads][dim][dim] float64, in/out. */
+int la_oracle_decode(const void *q, const void *k, const void *v, int dtype, const float *slopes,
+                     int batch, int heads, int dim, double *state, double *o) {
+    if (check_args(q, k, v, dtype, slopes, batch, heads, 1, dim) || !state || !o) return 1;
+    const long BH = (long)batch * heads;
+    const size_t d = (size_t)dim;
+#pragma omp parallel for schedule(static)
+    for (long bh = 0; bh < BH; ++bh) {
+        const int h = (int)(bh % heads);
+        const double decay = exp(-(double)slopes[h]);
+        double *S = state + (size_t)bh * d * d;
+        const size_t base = (size_t)bh * d;
+        for (size_t r = 0; r < d; ++r) {
+            const double kr = widen(k, dtype, base + r);
+            for (size_t c = 0; c < d; ++c)
+                S[r * d + c] = decay * S[r * d + c] + kr * widen(v, dtype, base + c);
+        }
+        double *oi = o + base;
+        for (size_t c = 0; c < d; ++c) oi[c] = 0.0;
+        for (size_t r = 0; r < d; ++r) {
+            const double qr = widen(q, dtype, base + r);
+            for (size_t c = 0; c < d; ++c) oi[c] += qr * S[r * d + c];
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,233 @@
+"""Pins for the float64 CPU oracle (runs without a GPU).
+
+Each test ties the oracle to something other than itself: a hand-worked
+example, a closed form, a special case that reduces to a numpy routine, or an
+invariant of the method ("MINIMAX SIGNAL LAB · M1", §03 Lightning Attention).
+A wrong sign, a dropped term, a transposed state or an off-by-one exponent in
+any of the three forms fails at least one of these.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal(shape) * scale).astype(np.float32)
+
+
+def _to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (nearest even) and return the bit patterns."""
+    u = x.astype(np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def _close(a, b, rtol):
+    scale = max(np.max(np.abs(b)), 1e-300)
+    assert np.max(np.abs(a - b)) <= rtol * scale, np.max(np.abs(a - b)) / scale
+
+
+SLOPES_MIX = np.array([0.0, 0.05, 0.9, 3.0], dtype=np.float32)
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_three_forms_agree_for_every_block(with_state):
+    b, h, L, d = 2, 4, 13, 5
+    q, k, v = (_rand((b, h, L, d), s, 0.5) for s in (1, 2, 3))
+    s0 = _rand((b, h, d, d), 4, 0.3) if with_state else None
+    o1, s1 = oracle.prefill(q, k, v, SLOPES_MIX, s0, form="definition")
+    o2, s2 = oracle.prefill(q, k, v, SLOPES_MIX, s0, form="recurrence")
+    _close(o2, o1, 1e-12)
+    _close(s2, s1, 1e-12)
+    for B in range(1, L + 3):
+        o3, s3 = oracle.prefill(q, k, v, SLOPES_MIX, s0, form="blockwise", block=B)
+        _close(o3, o1, 1e-12)
+        _close(s3, s1, 1e-12)
+
+
+def test_bf16_inputs_are_widened_exactly():
+    b, h, L, d = 1, 4, 9, 6
+    qf, kf, vf = (_rand((b, h, L, d), s) for s in (5, 6, 7))
+    qb, kb, vb = (_to_bf16_bits(x) for x in (qf, kf, vf))
+    # the same values handed over as float32 must give the identical result
+    widen = lambda bits: oracle.bf16_bits_to_f64(bits).astype(np.float32)
+    o_b, s_b = oracle.prefill(qb, kb, vb, SLOPES_MIX)
+    o_f, s_f = oracle.prefill(widen(qb), widen(kb), widen(vb), SLOPES_MIX)
+    assert np.array_equal(o_b, o_f) and np.array_equal(s_b, s_f)
+    # and the widening itself is exact: bf16 bits -> float64 -> bits round trip
+    back = _to_bf16_bits(oracle.bf16_bits_to_f64(qb).astype(np.float32))
+    assert np.array_equal(back, qb)
+
+
+def test_hand_worked_example():
+    rows = {}
+    with open(os.path.join(GOLDEN, "hand_example_d1.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            name, *vals = line.split()
+            rows[name] = np.array([float(x) for x in vals])
+    shape = (1, 1, 3, 1)
+    q, k, v = (rows[n].astype(np.float32).reshape(shape) for n in ("q", "k", "v"))
+    slope = np.array([math.log(2.0)], dtype=np.float32)
+    for form, blk in (("definition", None), ("recurrence", None), ("blockwise", 2)):
+        o, s = oracle.prefill(q, k, v, slope, form=form, block=blk)
+        np.testing.assert_allclose(o.ravel(), rows["o"], rtol=1e-7)
+        np.testing.assert_allclose(s.ravel(), rows["state_out"], rtol=1e-7)
+
+
+@pytest.mark.parametrize("s", [0.01, 0.3, 1.7])
+def test_closed_form_constant_inputs(s):
+    # q_i = q, k_j = k, v_j = v:  o_i = (q.k) v (1 - e^{-s(i+1)}) / (1 - e^{-s}),
+    # S_L = (1 - e^{-sL}) / (1 - e^{-s}) k^T v  (geometric series).
+    L, d = 40, 3
+    qv = np.array([0.5, -1.0, 0.25], np.float32)
+    kv = np.array([1.0, 0.5, -0.75], np.float32)
+    vv = np.array([2.0, -0.5, 1.5], np.float32)
+    q = np.broadcast_to(qv, (1, 1, L, d)).copy()
+    k = np.broadcast_to(kv, (1, 1, L, d)).copy()
+    v = np.broadcast_to(vv, (1, 1, L, d)).copy()
+    sl = np.array([s], np.float32)
+    sd = float(sl[0])
+    r = math.exp(-sd)
+    i = np.arange(L)
+    expect_o = (float(qv.astype(np.float64) @ kv.astype(np.float64))
+                * ((1 - r ** (i + 1)) / (1 - r))[:, None] * vv.astype(np.float64)[None, :])
+    expect_s = (1 - r ** L) / (1 - r) * np.outer(kv.astype(np.float64), vv.astype(np.float64))
+    for form, blk in (("definition", None), ("recurrence", None), ("blockwise", 16)):
+        o, st = oracle.prefill(q, k, v, sl, form=form, block=blk)
+        _close(o[0, 0], expect_o, 1e-12)
+        _close(st[0, 0], expect_s, 1e-12)
+
+
+def test_zero_slope_is_plain_causal_linear_attention():
+    # s = 0: o_i = q_i (S_in + sum_{j<=i} k_j^T v_j), a prefix sum (numpy cumsum).
+    b, h, L, d = 1, 2, 11, 4
+    q, k, v = (_rand((b, h, L, d), s) for s in (8, 9, 10))
+    s0 = _rand((b, h, d, d), 11)
+    sl = np.zeros(h, np.float32)
+    K, V, Q = (x.astype(np.float64) for x in (k, v, q))
+    outer = np.einsum("bhjr,bhjc->bhjrc", K, V)
+    pref = np.cumsum(outer, axis=2) + s0.astype(np.float64)[:, :, None]
+    expect = np.einsum("bhir,bhirc->bhic", Q, pref)
+    for form, blk in (("definition", None), ("recurrence", None), ("blockwise", 4)):
+        o, st = oracle.prefill(q, k, v, sl, s0, form=form, block=blk)
+        _close(o, expect, 1e-12)
+        _close(st, pref[:, :, -1], 1e-12)
+
+
+def test_large_slope_keeps_only_the_diagonal():
+    # e^{-s} underflows to 0: o_i = (q_i . k_i) v_i and S_out = k_{L-1}^T v_{L-1}.
+    b, h, L, d = 1, 1, 7, 4
+    q, k, v = (_rand((b, h, L, d), s) for s in (12, 13, 14))
+    s0 = _rand((b, h, d, d), 15)
+    sl = np.array([1.0e4], np.float32)
+    Q, K, V = (x.astype(np.float64)[0, 0] for x in (q, k, v))
+    expect = np.sum(Q * K, axis=1)[:, None] * V
+    for form, blk in (("definition", None), ("recurrence", None), ("blockwise", 3)):
+        o, st = oracle.prefill(q, k, v, sl, s0, form=form, block=blk)
+        _close(o[0, 0], expect, 1e-14)
+        _close(st[0, 0], np.outer(K[-1], V[-1]), 1e-14)
+
+
+def test_single_block_is_one_masked_matmul():
+    # L <= B: O = ((Q K^T) ⊙ D) V + diag(d_q) Q S_in, written with numpy matmuls.
+    L, d = 9, 6
+    q, k, v = (_rand((1, 1, L, d), s) for s in (16, 17, 18))
+    s0 = _rand((1, 1, d, d), 19)
+    s = np.float32(0.37)
+    Q, K, V = (x.astype(np.float64)[0, 0] for x in (q, k, v))
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    D = np.where(i >= j, np.exp(-float(s) * (i - j)), 0.0)
+    dq = np.exp(-float(s) * (np.arange(L) + 1.0))
+    expect = ((Q @ K.T) * D) @ V + dq[:, None] * (Q @ s0.astype(np.float64)[0, 0])
+    for form, blk in (("definition", None), ("recurrence", None), ("blockwise", 16)):
+        o, _ = oracle.prefill(q, k, v, np.array([s]), s0, form=form, block=blk)
+        _close(o[0, 0], expect, 1e-12)
+
+
+def test_linearity_in_v_and_state():
+    b, h, L, d = 1, 3, 10, 4
+    q, k, v1, v2 = (_rand((b, h, L, d), s) for s in (20, 21, 22, 23))
+    sa, sb = _rand((b, h, d, d), 24), _rand((b, h, d, d), 25)
+    sl = SLOPES_MIX[:3]
+    a, c = 0.75, -1.5
+    o1, t1 = oracle.prefill(q, k, v1, sl, sa)
+    o2, t2 = oracle.prefill(q, k, v2, sl, sb)
+    o12, t12 = oracle.prefill(q, k, (a * v1 + c * v2).astype(np.float32), sl,
+                              (a * sa + c * sb).astype(np.float32))
+    # inputs were rounded to float32 once, so compare against the rounded combination
+    va = (a * v1 + c * v2).astype(np.float32)
+    assert np.all(np.isfinite(va))
+    _close(o12, a * o1 + c * o2, 1e-6)
+    _close(t12, a * t1 + c * t2, 1e-6)
+
+
+def test_chunked_prefill_and_decode_continue_the_sequence():
+    b, h, L, d = 2, 4, 17, 5
+    q, k, v = (_rand((b, h, L + 1, d), s) for s in (26, 27, 28))
+    s0 = _rand((b, h, d, d), 29)
+    o_full, s_full = oracle.prefill(q, k, v, SLOPES_MIX, s0)
+    for cut in (1, 6, 16):
+        oa, sa = oracle.prefill(q[:, :, :cut], k[:, :, :cut], v[:, :, :cut], SLOPES_MIX, s0)
+        ob, sb = oracle.prefill(q[:, :, cut:], k[:, :, cut:], v[:, :, cut:], SLOPES_MIX,
+                                sa.astype(np.float32))
+        # the carried state is rounded to float32 between the two calls, as on the GPU
+        _close(np.concatenate([oa, ob], axis=2), o_full, 1e-6)
+        _close(sb, s_full, 1e-6)
+    # decode of token L after a prefill of L tokens == prefill of L+1 tokens
+    op, sp = oracle.prefill(q[:, :, :L], k[:, :, :L], v[:, :, :L], SLOPES_MIX, s0)
+    od, sd = oracle.decode(q[:, :, L], k[:, :, L], v[:, :, L], SLOPES_MIX, sp)
+    _close(od, o_full[:, :, L], 1e-12)
+    _close(sd, s_full, 1e-12)
+
+
+def test_carried_state_is_forgotten_at_the_slope_rate():
+    # the state's share of o_i is e^{-s(i+1)} q_i S_in, so |share| <= e^{-s(i+1)} |q_i| |S_in|
+    b, h, L, d = 1, 4, 30, 4
+    q, k, v = (_rand((b, h, L, d), s) for s in (30, 31, 32))
+    s0 = _rand((b, h, d, d), 33, 5.0)
+    with_s, _ = oracle.prefill(q, k, v, SLOPES_MIX, s0)
+    without, _ = oracle.prefill(q, k, v, SLOPES_MIX, None)
+    share = with_s - without
+    for hh, s in enumerate(SLOPES_MIX.astype(np.float64)):
+        qn = np.linalg.norm(q[0, hh].astype(np.float64), axis=1)
+        sn = np.linalg.norm(s0[0, hh].astype(np.float64), 2)
+        bound = np.exp(-s * (np.arange(L) + 1)) * qn * sn
+        # subtracting two float64 results leaves rounding noise of ~1e-16 |o|
+        noise = 1e-13 * np.max(np.abs(without[0, hh]))
+        assert np.all(np.linalg.norm(share[0, hh], axis=1) <= bound * (1 + 1e-12) + noise)
+
+
+def test_empty_sequence_decays_nothing_and_returns_the_state():
+    b, h, d = 1, 2, 3
+    z = np.zeros((b, h, 0, d), np.float32)
+    s0 = _rand((b, h, d, d), 34)
+    for form, blk in (("definition", None), ("recurrence", None), ("blockwise", 4)):
+        o, st = oracle.prefill(z, z, z, SLOPES_MIX[:2], s0, form=form, block=blk)
+        assert o.shape == (b, h, 0, d)
+        np.testing.assert_array_equal(st, s0.astype(np.float64))
+
+
+def test_state_size_matches_the_printed_m1_figure():
+    vals = {}
+    with open(os.path.join(GOLDEN, "state_size_m1.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            key, val = line.split()
+            vals[key] = float(val)
+    H, d = int(vals["heads"]), int(vals["dim"])
+    z = np.zeros((1, H, 1, d), np.float32)
+    _, st = oracle.prefill(z, z, z, np.ones(H, np.float32))
+    per_layer = st.astype(np.float32).nbytes
+    total_mb = vals["layers"] * per_layer / 1e6
+    assert abs(total_mb - vals["printed_megabytes"]) < 0.01
