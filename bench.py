@@ -1,0 +1,447 @@
+"""Benchmark of the Lightning Attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one lightning_prefill call over the long-context workload
+(batch 1, 64 heads, 131072 tokens, head dim 128, block 256, bf16 q/k/v/o,
+fp32 state), inputs resident in HBM. The same run also times the decode
+workload (64 sequences x 64 heads x 128, fp32 states, 1000 consecutive
+single-token steps) and the end-to-end path with host buffers. Rank 0 prints
+one JSON line. With --gpus N (under torchrun) every rank runs an independent
+replica of the workload ("replicas only": the path has no exchange step);
+times are the max over ranks.
+
+`--impl reference` times the float64 CPU oracle on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+PREFILL_WORKLOAD = "m1_prefill_128k"
+DECODE_WORKLOAD = "batched_decode"
+METRIC = "prefill tokens/s & TFLOP/s (% bf16 peak); decode state GB/s (% HBM peak)"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------- arithmetic
+
+def prefill_flops(batch, heads, seq, dim, block):
+    """Algorithmic FLOPs of one prefill, two conventions, per (token, head):
+    formula 4Bd + 4d^2 (dense masked BxB products as the block formula writes
+    them, plus the inter and state products); causal 2(B+1)d + 4d^2."""
+    units = batch * heads * seq
+    return {"formula": units * (4 * block * dim + 4 * dim * dim),
+            "causal": units * (2 * (block + 1) * dim + 4 * dim * dim)}
+
+
+def prefill_bytes(batch, heads, seq, dim, elem_bytes=2, state_in=False, state_out=True):
+    """Algorithmic HBM bytes of one prefill: q, k, v read and o written once,
+    plus the fp32 states read / written once."""
+    tok = 4 * batch * heads * seq * dim * elem_bytes
+    st = batch * heads * dim * dim * 4
+    return tok + (st if state_in else 0) + (st if state_out else 0)
+
+
+def decode_bytes(batch, heads, dim, elem_bytes=2):
+    """Algorithmic HBM bytes of one decode step: the fp32 state read and
+    written once, q, k, v read and o written once."""
+    return batch * heads * (2 * dim * dim * 4 + 4 * dim * elem_bytes)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def roofline(bound, achieved, peak, unit, traffic=None):
+    return {"bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic}
+
+
+def summarize_clocks(rows):
+    """rows: list of dicts from nvidia-smi samples; returns the clocks object."""
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["not sampled"]}
+    loaded = [r for r in rows if r.get("power_w", 0) > 200] or rows
+    sm = statistics.median(r["sm_mhz"] for r in loaded)
+    reasons = set()
+    for r in loaded:
+        for key in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"):
+            if r.get(key) == "Active":
+                reasons.add(key)
+    return {"sm_mhz": sm, "sm_max_mhz": max(r["sm_max_mhz"] for r in rows),
+            "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                self.rows.append({"sm_mhz": float(parts[0]), "sm_max_mhz": float(parts[1]),
+                                  "power_w": float(parts[2]), "hw_slowdown": parts[3],
+                                  "hw_thermal_slowdown": parts[4], "sw_thermal_slowdown": parts[5],
+                                  "sw_power_cap": parts[6]})
+            except ValueError:
+                continue
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=5)
+        return False
+
+    def summary(self):
+        return summarize_clocks(self.rows)
+
+
+# ---------------------------------------------------------------- ranks
+
+def dist_setup(n_gpus):
+    """Returns (rank, world, local_rank). Initialises torch.distributed when launched by torchrun."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        return dist.get_rank(), world, int(os.environ.get("LOCAL_RANK", "0"))
+    return 0, 1, 0
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world, device="cpu"):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, tokens, heads, threads=None):
+    """Time the float64 oracle (token recurrence) on `heads` heads x `tokens`
+    tokens of the workload's distribution; returns (seconds, token-heads)."""
+    import numpy as np
+    import oracle
+    from linear_attention_lightning_b200 import inputs
+    if threads:
+        oracle.set_threads(threads)
+    inp = inputs.prefill_inputs(1, heads, tokens, w.dim, w.dtype, w.state_in, seed=w.seed)
+    conv = inputs.to_oracle
+    sl = inputs.slopes(w.heads)[:heads].numpy()
+    args = (conv(inp["q"]), conv(inp["k"]), conv(inp["v"]), sl, None)
+    t0 = time.perf_counter()
+    oracle.prefill(*args, form="recurrence")
+    return time.perf_counter() - t0, tokens * heads
+
+
+def cpu_baseline(w, budget_s=15.0):
+    import oracle
+    cores = oracle.threads()
+    heads = min(w.heads, max(1, cores))
+    tokens = 2048
+    sec, units = oracle_sample(w, tokens, heads)
+    # grow the sample toward the time budget
+    scale = max(1.0, min(32.0, budget_s / max(sec, 1e-3) * 0.8))
+    tokens = int(min(w.seq, tokens * scale))
+    sec, units = oracle_sample(w, tokens, heads)
+    tok_per_s = units / w.heads / sec  # a token covers every head
+    return {"value": round(tok_per_s, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "float64 token recurrence, %d of %d heads x %d tokens of the %s workload, %.1f s"
+                      % (heads, w.heads, tokens, w.name, sec)}
+
+
+def run_reference(args):
+    # rank 0 alone runs the CPU oracle; the other ranks exit without work
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from linear_attention_lightning_b200 import inputs
+    w = inputs.WORKLOADS[PREFILL_WORKLOAD]
+    import oracle
+    cores = oracle.threads()
+    heads = min(w.heads, max(1, cores))
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    sec, units = oracle_sample(w, 1024, heads)
+    tokens = int(min(w.seq, max(1024, 1024 * budget / max(sec, 1e-3) * 0.7)))
+    for _ in range(args.warmup):
+        oracle_sample(w, min(tokens, 1024), heads)
+    times = []
+    for _ in range(args.steps):
+        sec, units = oracle_sample(w, tokens, heads)
+        times.append(sec)
+    tot = sum(times)
+    value = args.steps * units / w.heads / tot
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1000 * tot / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": w.seq,
+                       "dim": w.dim, "block": w.block, "inputs": "bf16 q,k,v widened to float64"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": "%d of %d heads x %d tokens per step" % (heads, w.heads, tokens)},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU path
+
+def run_ours(args):
+    import torch
+    import linear_attention_lightning_b200 as la
+    from linear_attention_lightning_b200 import abi, inputs
+
+    rank, world, local_rank = dist_setup(args.gpus)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = load_peaks()
+    w = inputs.WORKLOADS[args.workload]
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+
+    inp = inputs.workload_inputs(w, dev)
+    q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
+    o = torch.empty_like(q)
+    s_out = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32, device=dev)
+    variant = la.prefill_variant(w.dtype, w.batch, w.heads, w.seq, w.dim, w.block)
+    vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05}[variant]
+    dcode = abi.LA_DTYPE_BF16 if w.dtype == torch.bfloat16 else abi.LA_DTYPE_F32
+
+    def step():
+        abi.check(abi.lightning_prefill_ex(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads,
+            w.seq, w.dim, w.block, None if s0 is None else s0.data_ptr(), o.data_ptr(),
+            s_out.data_ptr(), None, 0, sp, vcode))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    per_launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms = max_over_ranks(total_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+    tokens = w.batch * w.seq
+    value = world * tokens * args.steps / (total_ms / 1e3)
+
+    fl = prefill_flops(w.batch, w.heads, w.seq, w.dim, w.block)
+    by = prefill_bytes(w.batch, w.heads, w.seq, w.dim, 2 if w.dtype == torch.bfloat16 else 4,
+                       state_in=s0 is not None, state_out=True)
+    avg_launch_s = statistics.mean(per_launch_ms) / 1e3
+    gbs = by / avg_launch_s / 1e9
+    tflops = {kk: vv / avg_launch_s / 1e12 for kk, vv in fl.items()}
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get("%s/%s" % (w.name, variant))
+
+    # decode: 1000 consecutive single-token steps over fp32 states
+    dw = inputs.WORKLOADS[DECODE_WORKLOAD]
+    dec = run_decode(dw, dev, stream, peaks, args)
+
+    # end to end: host buffers, copies inside the timed region
+    e2e = run_e2e(w, dev, stream, inp, variant, args, world)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": w.seq,
+                   "dim": w.dim, "block": w.block, "kernel": variant,
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (%.1f GB per step)" % (by / 1e9)},
+        "tflops": {"formula": round(tflops["formula"], 2), "causal": round(tflops["causal"], 2),
+                   "peak_bf16": peaks["bf16_tflops"],
+                   "frac_formula": round(tflops["formula"] / peaks["bf16_tflops"], 4),
+                   "frac_causal": round(tflops["causal"] / peaks["bf16_tflops"], 4),
+                   "peak_source": peaks["source"]},
+        "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s", traffic),
+        "decode": dec,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_decode(dw, dev, stream, peaks, args):
+    import torch
+    from linear_attention_lightning_b200 import abi, inputs
+    steps = args.decode_steps
+    inp = inputs.workload_inputs(dw, dev, steps=steps)
+    state = inp["state"]
+    qs, ks, vs, sl = inp["q"], inp["k"], inp["v"], inp["slopes"]
+    o = torch.empty((dw.batch, dw.heads, dw.dim), dtype=dw.dtype, device=dev)
+    sp = stream.cuda_stream
+    dcode = abi.LA_DTYPE_BF16
+    tok = dw.batch * dw.heads * dw.dim
+
+    def one(t):
+        abi.check(abi.lightning_decode(qs[t].data_ptr(), ks[t].data_ptr(), vs[t].data_ptr(), dcode,
+                                       sl.data_ptr(), dw.batch, dw.heads, dw.dim, state.data_ptr(),
+                                       o.data_ptr(), sp))
+
+    for t in range(3):
+        one(t)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(steps):
+        one(t)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    by = decode_bytes(dw.batch, dw.heads, dw.dim)
+    gbs = by * steps / (ms / 1e3) / 1e9
+    del tok
+    return {"workload": dw.name, "steps": steps, "us_per_step": round(1e3 * ms / steps, 3),
+            "value": round(gbs, 1), "unit": "GB/s (state + token bytes)",
+            "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s"),
+            "l2": "state 268 MB > L2; consecutive steps, no flush"}
+
+
+def run_e2e(w, dev, stream, inp, variant, args, world):
+    """Same prefill through the public API with host buffers: every step copies
+    q, k, v from pinned host memory and reads o and the state back."""
+    import torch
+    import linear_attention_lightning_b200 as la
+    steps = args.e2e_steps
+    hq = inp["q"].cpu().pin_memory()
+    hk = inp["k"].cpu().pin_memory()
+    hv = inp["v"].cpu().pin_memory()
+    ho = torch.empty_like(hq).pin_memory()
+    hs = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32).pin_memory()
+    dq, dk, dv = (torch.empty_like(inp["q"]) for _ in range(3))
+    h2d = 3 * hq.numel() * hq.element_size()
+    d2h = ho.numel() * ho.element_size() + hs.numel() * 4
+
+    def one():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        o, s = la.prefill(dq, dk, dv, inp["slopes"], w.block, inp["state_in"], variant=variant)
+        ho.copy_(o, non_blocking=True)
+        hs.copy_(s, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    value = world * w.batch * w.seq * steps / (ms / 1e3)
+    return {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=PREFILL_WORKLOAD)
+    p.add_argument("--decode-steps", type=int, default=1000)
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be at least 3")
+    return a
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,155 @@
+/*
+ * lightning.h — C ABI of liblightning.so, MiniMax-M1 Lightning Attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation ("MINIMAX SIGNAL LAB · M1", §03 Lightning Attention): causal
+ * linear attention with a per-head exponential decay, computed in blocks of B
+ * tokens. For block t of one (batch, head) with slope s:
+ *
+ *   intra  O_intra = [(Q_t K_t^T) ⊙ D] V_t,   D_ij = e^{-s(i-j)} 1[i >= j]
+ *   inter  O_inter = (Q_t ⊙ d_q) S_{t-1},     d_q[i] = e^{-s(i+1)}
+ *   state  S_t     = e^{-s m} S_{t-1} + (K_t ⊙ d_k)^T V_t,  d_k[j] = e^{-s(m-1-j)}
+ *   out    O_t     = O_intra + O_inter
+ *
+ * where m is the block's length (B, or fewer for the last block, as the same
+ * section states) and S_{-1} is the carried-in state. Equivalently, token by
+ * token: o_i = sum_{j<=i} e^{-s(i-j)} (q_i . k_j) v_j + e^{-s(i+1)} q_i S_in.
+ * The pages print no d_q / d_k exponents; the ones above are the readings for
+ * which the block form equals the token form.
+ *
+ * Decode (same section: the recursive, fixed-size KV state; §04: the state
+ * does not grow with context): for one new token,
+ *   S <- e^{-s} S + k^T v,   o = q S.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or retains them.
+ *   - q, k, v, o are contiguous [batch][heads][seq][dim] (decode: seq = 1,
+ *     i.e. [batch][heads][dim]); element type given by `dtype`; o has the
+ *     input dtype. Pointers must be 16-byte aligned.
+ *   - States are float32, contiguous [batch][heads][dim][dim], row index =
+ *     key dimension, column index = value dimension.
+ *   - slopes is a device float32 array of `heads` decay slopes s_h >= 0.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Every call is asynchronous on that stream.
+ *   - Argument errors are detected on the host and returned before anything
+ *     is launched; launch failures return LA_ERR_CUDA. No device-side trap
+ *     or abort is ever used: a device-side wait that runs out of its
+ *     iteration budget records LA_ERR_TIMEOUT in a device status word, read
+ *     back by lightning_device_status().
+ *   - A human-readable reason for the last failure on the calling thread is
+ *     returned by lightning_last_error_message().
+ */
+#ifndef LIGHTNING_H
+#define LIGHTNING_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum la_status {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,   /* bad pointer, shape, alignment or aliasing        */
+    LA_ERR_UNSUPPORTED = 2,   /* valid request the library has no kernel for      */
+    LA_ERR_CUDA = 3,          /* CUDA runtime error while launching               */
+    LA_ERR_TIMEOUT = 4        /* a device-side bounded wait gave up               */
+} la_status;
+
+typedef enum la_dtype {
+    LA_DTYPE_F32 = 0,
+    LA_DTYPE_BF16 = 1
+} la_dtype;
+
+/* Kernel selection for lightning_prefill_ex. AUTO picks the tensor-core
+ * kernel whenever it supports the request (bf16, dim 128, block 128 or 256)
+ * and the CUDA-core kernel otherwise. */
+typedef enum la_variant {
+    LA_VARIANT_AUTO = 0,
+    LA_VARIANT_SIMT = 1,      /* CUDA-core kernel, fp32 arithmetic, any dtype    */
+    LA_VARIANT_TCGEN05 = 2    /* tcgen05/TMEM/TMA kernel, bf16, dim 128          */
+} la_variant;
+
+/* Version of this ABI; bumps on any incompatible change. */
+int lightning_abi_version(void);
+
+/*
+ * Blockwise prefill of `seq` tokens for every (batch, head).
+ * Source: "MINIMAX SIGNAL LAB · M1", §03 Lightning Attention (intra-block,
+ * inter-block and state-update formulas; last short block uses its length).
+ *
+ *   q, k, v    [batch][heads][seq][dim], dtype; read only.
+ *   dtype      LA_DTYPE_F32 or LA_DTYPE_BF16.
+ *   slopes     [heads] float32.
+ *   batch      >= 0 (0: nothing to do).  heads >= 1.  seq >= 0.
+ *   dim        64 or 128.
+ *   block      block length B >= 1 (tensor-core kernel: 128 or 256).
+ *   state_in   [batch][heads][dim][dim] float32 carried-in state, or NULL for
+ *              zeros.
+ *   o          [batch][heads][seq][dim], dtype; written. Must not overlap
+ *              q, k, v, slopes or either state.
+ *   state_out  [batch][heads][dim][dim] float32 state after the last token, or
+ *              NULL to skip. May be the same pointer as state_in (in-place
+ *              carry); any other overlap is rejected.
+ *   workspace, workspace_bytes
+ *              scratch; the current kernels need none
+ *              (lightning_prefill_workspace_size returns 0), so NULL/0 is fine.
+ *   stream     cudaStream_t as void*.
+ * seq == 0 writes state_out = state_in (or zeros) and nothing else.
+ */
+la_status lightning_prefill(const void *q, const void *k, const void *v, la_dtype dtype,
+                            const float *slopes, int batch, int heads, int seq, int dim,
+                            int block, const float *state_in, void *o, float *state_out,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same as lightning_prefill with an explicit kernel choice (la_variant).
+ * Requesting LA_VARIANT_TCGEN05 for an unsupported shape returns
+ * LA_ERR_UNSUPPORTED. */
+la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_dtype dtype,
+                               const float *slopes, int batch, int heads, int seq, int dim,
+                               int block, const float *state_in, void *o, float *state_out,
+                               void *workspace, size_t workspace_bytes, void *stream,
+                               int variant);
+
+/* Kernel lightning_prefill_ex would run for these arguments (la_variant, never
+ * AUTO), or -1 if the request is invalid or unsupported. Host only. */
+int lightning_prefill_selected_variant(la_dtype dtype, int batch, int heads, int seq, int dim,
+                                       int block, int variant);
+
+/* Bytes of workspace lightning_prefill needs for these sizes (currently 0). */
+size_t lightning_prefill_workspace_size(int batch, int heads, int seq, int dim, int block);
+
+/*
+ * One decode step for a single new token of every (batch, head), updating the
+ * state in place. Source: "MINIMAX SIGNAL LAB · M1", §03 (recursive KV state)
+ * and §04 (fixed-size FP32 state per head).
+ *
+ *   q, k, v  [batch][heads][dim], dtype; read only.
+ *   slopes   [heads] float32.
+ *   dim      64 or 128.
+ *   state    [batch][heads][dim][dim] float32; read and overwritten with
+ *            e^{-s} state + k^T v.
+ *   o        [batch][heads][dim], dtype; written: q (updated state).
+ *            Must not overlap any input or the state.
+ */
+la_status lightning_decode(const void *q, const void *k, const void *v, la_dtype dtype,
+                           const float *slopes, int batch, int heads, int dim, float *state,
+                           void *o, void *stream);
+
+/* Synchronises `stream`, returns the device status word (LA_OK or
+ * LA_ERR_TIMEOUT) recorded by kernels since the last call, and clears it. */
+la_status lightning_device_status(void *stream);
+
+/* Static description of a status code. */
+const char *lightning_status_string(int status);
+
+/* Reason for the most recent failure returned on the calling thread ("" if
+ * none). The pointer stays valid until the next call on that thread. */
+const char *lightning_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGHTNING_H */

@@ -1,0 +1,10 @@
+"""MiniMax-M1 Lightning Attention for NVIDIA B200 (sm_100a).
+
+The compute lives in liblightning.so (hand-written CUDA behind a C ABI, see
+include/lightning.h). This package adds a thin torch-facing layer that only
+marshals tensors into that ABI: torch provides device memory and streams.
+"""
+from . import abi
+from .api import decode, prefill, prefill_variant
+
+__all__ = ["abi", "prefill", "decode", "prefill_variant"]

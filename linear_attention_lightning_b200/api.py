@@ -1,0 +1,91 @@
+"""torch-facing wrappers over the C ABI: argument marshalling only.
+
+Tensors must be CUDA, contiguous, on the current device. Outputs are
+allocated with torch when not supplied. Nothing here computes anything of
+the method; a missing library raises instead of falling back.
+"""
+from typing import Optional, Tuple
+
+import torch
+
+from . import abi
+
+_DTYPES = {torch.float32: abi.LA_DTYPE_F32, torch.bfloat16: abi.LA_DTYPE_BF16}
+_VARIANTS = {"auto": abi.LA_VARIANT_AUTO, "simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need_cuda(name, t, dtype=None):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor, block: int,
+            state_in: Optional[torch.Tensor] = None, o: Optional[torch.Tensor] = None,
+            state_out: Optional[torch.Tensor] = None, want_state: bool = True,
+            variant: str = "auto", stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """lightning_prefill on [batch, heads, seq, dim] tensors; returns (o, state_out)."""
+    if q.dtype not in _DTYPES:
+        raise ValueError("q must be float32 or bfloat16")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [batch, heads, seq, dim] shape")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, q.dtype)
+    b, h, L, d = q.shape
+    _need_cuda("slopes", slopes, torch.float32)
+    if state_in is not None:
+        _need_cuda("state_in", state_in, torch.float32)
+        if tuple(state_in.shape) != (b, h, d, d):
+            raise ValueError("state_in must be [batch, heads, dim, dim]")
+    if o is None:
+        o = torch.empty_like(q)
+    if state_out is None and want_state:
+        state_out = torch.empty((b, h, d, d), dtype=torch.float32, device=q.device)
+    abi.check(abi.lightning_prefill_ex(
+        _ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(slopes), b, h, L, d, int(block),
+        _ptr(state_in), _ptr(o), _ptr(state_out), None, 0, _stream(stream), _VARIANTS[variant]))
+    return o, state_out
+
+
+def prefill_variant(dtype: torch.dtype, batch: int, heads: int, seq: int, dim: int, block: int,
+                    variant: str = "auto") -> str:
+    """Which kernel lightning_prefill would run: "simt" or "tcgen05"."""
+    r = abi.lightning_prefill_selected_variant(_DTYPES[dtype], batch, heads, seq, dim, block,
+                                               _VARIANTS[variant])
+    if r < 0:
+        raise ValueError(abi.last_error_message() or "unsupported request")
+    return {abi.LA_VARIANT_SIMT: "simt", abi.LA_VARIANT_TCGEN05: "tcgen05"}[r]
+
+
+def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor,
+           state: torch.Tensor, o: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """lightning_decode on [batch, heads, dim] tensors; updates `state` in place, returns o."""
+    if q.dtype not in _DTYPES:
+        raise ValueError("q must be float32 or bfloat16")
+    if q.dim() != 3 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [batch, heads, dim] shape")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, q.dtype)
+    b, h, d = q.shape
+    _need_cuda("slopes", slopes, torch.float32)
+    _need_cuda("state", state, torch.float32)
+    if tuple(state.shape) != (b, h, d, d):
+        raise ValueError("state must be [batch, heads, dim, dim]")
+    if o is None:
+        o = torch.empty_like(q)
+    abi.check(abi.lightning_decode(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(slopes), b, h, d,
+                                   _ptr(state), _ptr(o), _stream(stream)))
+    return o

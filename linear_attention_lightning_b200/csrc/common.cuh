@@ -1,0 +1,28 @@
+// Shared device helpers for the Lightning Attention kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace la {
+
+// Device status word: kernels set LA_ERR_TIMEOUT here when a bounded wait
+// gives up. Read and cleared by lightning_device_status().
+__device__ unsigned int g_device_status;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// e^{-s * n} for n >= 0 through exp2f; s is the per-head slope.
+__device__ __forceinline__ float decay_pow(float s, float n) { return exp2f(-s * kLog2e * n); }
+
+}  // namespace la

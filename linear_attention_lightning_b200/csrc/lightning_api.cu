@@ -1,0 +1,271 @@
+// liblightning.so: host side of the C ABI declared in include/lightning.h.
+//
+// Argument checking happens here, before any launch; every check failure
+// returns a status and records a message for lightning_last_error_message().
+// The library allocates nothing: all tensors, and the (currently unused)
+// workspace, belong to the caller.
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include "../../include/lightning.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_simt.cuh"
+#include "prefill_tc.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+la_status fail(la_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+la_status ok() {
+    g_last_error.clear();
+    return LA_OK;
+}
+
+la_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(LA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+
+Range range_of(const void *p, size_t bytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return {a, a + bytes};
+}
+
+bool overlaps(Range a, Range b) {
+    return a.lo < a.hi && b.lo < b.hi && a.lo < b.hi && b.lo < a.hi;
+}
+
+size_t elem_bytes(la_dtype dt) { return dt == LA_DTYPE_BF16 ? 2 : 4; }
+
+struct PrefillArgs {
+    const void *q, *k, *v;
+    la_dtype dtype;
+    const float *slopes;
+    int batch, heads, seq, dim, block;
+    const float *state_in;
+    void *o;
+    float *state_out;
+};
+
+// Shape / dtype checks shared by the launcher and the variant query.
+la_status check_prefill_shape(la_dtype dtype, int batch, int heads, int seq, int dim, int block) {
+    if (dtype != LA_DTYPE_F32 && dtype != LA_DTYPE_BF16)
+        return fail(LA_ERR_INVALID_ARG, "dtype %d is neither LA_DTYPE_F32 nor LA_DTYPE_BF16", (int)dtype);
+    if (batch < 0 || heads < 1 || seq < 0)
+        return fail(LA_ERR_INVALID_ARG, "need batch >= 0, heads >= 1, seq >= 0 (got %d, %d, %d)",
+                    batch, heads, seq);
+    if (block < 1) return fail(LA_ERR_INVALID_ARG, "block must be >= 1 (got %d)", block);
+    if (dim != 64 && dim != 128)
+        return fail(LA_ERR_UNSUPPORTED, "dim %d unsupported (64 or 128)", dim);
+    if ((long long)batch * heads > (1ll << 28))
+        return fail(LA_ERR_UNSUPPORTED, "batch*heads too large (at most 2^28)");
+    return LA_OK;
+}
+
+int choose_variant(la_dtype dtype, int dim, int block, int requested) {
+    const bool tc_ok = la::tc_supports(dtype == LA_DTYPE_BF16, dim, block);
+    switch (requested) {
+        case LA_VARIANT_AUTO: return tc_ok ? LA_VARIANT_TCGEN05 : LA_VARIANT_SIMT;
+        case LA_VARIANT_SIMT: return LA_VARIANT_SIMT;
+        case LA_VARIANT_TCGEN05: return tc_ok ? LA_VARIANT_TCGEN05 : -1;
+        default: return -1;
+    }
+}
+
+la_status check_prefill_pointers(const PrefillArgs &a) {
+    const size_t eb = elem_bytes(a.dtype);
+    const size_t n_tok = (size_t)a.batch * a.heads * a.seq * a.dim;
+    const size_t n_state = (size_t)a.batch * a.heads * a.dim * a.dim;
+    if (a.seq > 0 && (!a.q || !a.k || !a.v || !a.o))
+        return fail(LA_ERR_INVALID_ARG, "q, k, v and o must be non-NULL when seq > 0");
+    if (!a.slopes) return fail(LA_ERR_INVALID_ARG, "slopes must be non-NULL");
+    const void *ptrs[] = {a.q, a.k, a.v, a.o, a.slopes, a.state_in, a.state_out};
+    const char *names[] = {"q", "k", "v", "o", "slopes", "state_in", "state_out"};
+    for (int i = 0; i < 7; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i]))
+            return fail(LA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+    const Range ro = range_of(a.o, a.seq > 0 ? n_tok * eb : 0);
+    const Range rin[] = {range_of(a.q, n_tok * eb), range_of(a.k, n_tok * eb),
+                         range_of(a.v, n_tok * eb), range_of(a.slopes, sizeof(float) * a.heads),
+                         range_of(a.state_in, a.state_in ? n_state * 4 : 0),
+                         range_of(a.state_out, a.state_out ? n_state * 4 : 0)};
+    for (const Range &r : rin)
+        if (overlaps(ro, r)) return fail(LA_ERR_INVALID_ARG, "o overlaps an input or a state");
+    if (a.state_out) {
+        const Range rs = range_of(a.state_out, n_state * 4);
+        for (int i = 0; i < 4; ++i)
+            if (overlaps(rs, rin[i])) return fail(LA_ERR_INVALID_ARG, "state_out overlaps an input");
+        if (a.state_in && a.state_in != a.state_out && overlaps(rs, rin[4]))
+            return fail(LA_ERR_INVALID_ARG, "state_out partially overlaps state_in");
+    }
+    return LA_OK;
+}
+
+template <typename T, int D>
+la_status launch_simt(const PrefillArgs &a, cudaStream_t stream) {
+    auto kern = la::prefill_simt_kernel<T, D>;
+    const size_t smem = la::simt_smem_bytes<D>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_simt)");
+    dim3 grid((unsigned)((size_t)a.batch * a.heads * (D / la::kSimtCols)));
+    kern<<<grid, la::kSimtThreads, smem, stream>>>(
+        static_cast<const T *>(a.q), static_cast<const T *>(a.k), static_cast<const T *>(a.v),
+        a.slopes, a.heads, a.seq, a.block, a.state_in, static_cast<T *>(a.o), a.state_out);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "prefill_simt launch");
+    return ok();
+}
+
+la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
+    if (a.batch == 0) return ok();
+    if (a.seq == 0) {
+        if (!a.state_out) return ok();
+        const size_t n = (size_t)a.batch * a.heads * a.dim * a.dim;
+        la::state_passthrough_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0,
+                                       stream>>>(a.state_in, a.state_out, n);
+        cudaError_t e = cudaGetLastError();
+        return e == cudaSuccess ? ok() : cuda_fail(e, "state passthrough launch");
+    }
+    if (variant == LA_VARIANT_TCGEN05) return la::launch_tc(a.q, a.k, a.v, a.slopes, a.batch, a.heads,
+                                                           a.seq, a.block, a.state_in, a.o, a.state_out,
+                                                           stream, &g_last_error);
+    if (a.dtype == LA_DTYPE_BF16)
+        return a.dim == 64 ? launch_simt<__nv_bfloat16, 64>(a, stream)
+                           : launch_simt<__nv_bfloat16, 128>(a, stream);
+    return a.dim == 64 ? launch_simt<float, 64>(a, stream) : launch_simt<float, 128>(a, stream);
+}
+
+template <typename T, int D>
+la_status launch_decode(const void *q, const void *k, const void *v, const float *slopes, int batch,
+                        int heads, float *state, void *o, cudaStream_t stream) {
+    la::decode_kernel<T, D><<<(unsigned)((size_t)batch * heads), la::kDecodeThreads, 0, stream>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), slopes, heads,
+        state, static_cast<T *>(o));
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "decode launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int lightning_abi_version(void) { return 1; }
+
+la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_dtype dtype,
+                               const float *slopes, int batch, int heads, int seq, int dim, int block,
+                               const float *state_in, void *o, float *state_out, void *workspace,
+                               size_t workspace_bytes, void *stream, int variant) {
+    (void)workspace;
+    (void)workspace_bytes;
+    la_status st = check_prefill_shape(dtype, batch, heads, seq, dim, block);
+    if (st != LA_OK) return st;
+    const int chosen = choose_variant(dtype, dim, block, variant);
+    if (chosen < 0) {
+        if (variant < LA_VARIANT_AUTO || variant > LA_VARIANT_TCGEN05)
+            return fail(LA_ERR_INVALID_ARG, "unknown variant %d", variant);
+        return fail(LA_ERR_UNSUPPORTED,
+                    "the tcgen05 kernel needs bf16, dim 128 and block 128 or 256 (got dtype %d, dim %d, block %d)",
+                    (int)dtype, dim, block);
+    }
+    PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out};
+    st = check_prefill_pointers(a);
+    if (st != LA_OK) return st;
+    return run_prefill(a, static_cast<cudaStream_t>(stream), chosen);
+}
+
+la_status lightning_prefill(const void *q, const void *k, const void *v, la_dtype dtype,
+                            const float *slopes, int batch, int heads, int seq, int dim, int block,
+                            const float *state_in, void *o, float *state_out, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    return lightning_prefill_ex(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o,
+                                state_out, workspace, workspace_bytes, stream, LA_VARIANT_AUTO);
+}
+
+int lightning_prefill_selected_variant(la_dtype dtype, int batch, int heads, int seq, int dim, int block,
+                                       int variant) {
+    if (check_prefill_shape(dtype, batch, heads, seq, dim, block) != LA_OK) return -1;
+    return choose_variant(dtype, dim, block, variant);
+}
+
+size_t lightning_prefill_workspace_size(int batch, int heads, int seq, int dim, int block) {
+    (void)batch; (void)heads; (void)seq; (void)dim; (void)block;
+    return 0;
+}
+
+la_status lightning_decode(const void *q, const void *k, const void *v, la_dtype dtype, const float *slopes,
+                           int batch, int heads, int dim, float *state, void *o, void *stream) {
+    if (dtype != LA_DTYPE_F32 && dtype != LA_DTYPE_BF16)
+        return fail(LA_ERR_INVALID_ARG, "dtype %d is neither LA_DTYPE_F32 nor LA_DTYPE_BF16", (int)dtype);
+    if (batch < 0 || heads < 1)
+        return fail(LA_ERR_INVALID_ARG, "need batch >= 0 and heads >= 1 (got %d, %d)", batch, heads);
+    if (dim != 64 && dim != 128) return fail(LA_ERR_UNSUPPORTED, "dim %d unsupported (64 or 128)", dim);
+    if ((long long)batch * heads > (1ll << 31) - 1) return fail(LA_ERR_UNSUPPORTED, "batch*heads too large");
+    if (batch == 0) return ok();
+    if (!q || !k || !v || !slopes || !state || !o)
+        return fail(LA_ERR_INVALID_ARG, "q, k, v, slopes, state and o must be non-NULL");
+    const void *ptrs[] = {q, k, v, slopes, state, o};
+    const char *names[] = {"q", "k", "v", "slopes", "state", "o"};
+    for (int i = 0; i < 6; ++i)
+        if (!aligned16(ptrs[i])) return fail(LA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+    const size_t eb = elem_bytes(dtype);
+    const size_t n_tok = (size_t)batch * heads * dim;
+    const Range ro = range_of(o, n_tok * eb), rs = range_of(state, n_tok * dim * 4);
+    const Range rin[] = {range_of(q, n_tok * eb), range_of(k, n_tok * eb), range_of(v, n_tok * eb),
+                         range_of(slopes, sizeof(float) * heads)};
+    if (overlaps(ro, rs)) return fail(LA_ERR_INVALID_ARG, "o overlaps the state");
+    for (const Range &r : rin) {
+        if (overlaps(ro, r)) return fail(LA_ERR_INVALID_ARG, "o overlaps an input");
+        if (overlaps(rs, r)) return fail(LA_ERR_INVALID_ARG, "state overlaps an input");
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == LA_DTYPE_BF16)
+        return dim == 64 ? launch_decode<__nv_bfloat16, 64>(q, k, v, slopes, batch, heads, state, o, s)
+                         : launch_decode<__nv_bfloat16, 128>(q, k, v, slopes, batch, heads, state, o, s);
+    return dim == 64 ? launch_decode<float, 64>(q, k, v, slopes, batch, heads, state, o, s)
+                     : launch_decode<float, 128>(q, k, v, slopes, batch, heads, state, o, s);
+}
+
+la_status lightning_device_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int word = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&word, la::g_device_status, sizeof word);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    e = cudaMemcpyToSymbol(la::g_device_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    if (word != 0) return fail(LA_ERR_TIMEOUT, "a device-side wait gave up (status word 0x%x)", word);
+    return ok();
+}
+
+const char *lightning_status_string(int status) {
+    switch (status) {
+        case LA_OK: return "LA_OK: success";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: no kernel for this request";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA runtime error";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT: a device-side wait gave up";
+        default: return "unknown status";
+    }
+}
+
+const char *lightning_last_error_message(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,114 @@
+"""Host-only checks of the C ABI: the library loads, exports everything the
+header declares, and rejects bad arguments before launching anything.
+
+No call here reaches a kernel launch, so these run without a GPU.
+"""
+import ctypes
+
+import pytest
+
+from linear_attention_lightning_b200 import abi
+from linear_attention_lightning_b200.build import build
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build()
+    abi.load()
+
+
+def test_every_declared_function_is_exported():
+    lib = ctypes.CDLL(abi.LIBRARY)
+    declared = abi.declared_functions()
+    assert "lightning_prefill" in declared and "lightning_decode" in declared
+    for name in declared:
+        assert hasattr(lib, name), name
+        assert name in abi._SIGNATURES, "binding lacks " + name
+
+
+def test_version_and_status_strings():
+    assert abi.lightning_abi_version() == 1
+    for st in range(5):
+        assert abi.status_string(st).startswith("LA_")
+    assert abi.status_string(99) == "unknown status"
+
+
+def test_workspace_is_zero():
+    assert abi.lightning_prefill_workspace_size(16, 64, 4096, 128, 256) == 0
+
+
+# Fake, well-aligned, non-overlapping "device" addresses: every call below must
+# be rejected (or finish trivially) before any CUDA call is made.
+Q, K, V, O, SL, S0, S1 = (0x10000000 * (i + 1) for i in range(7))
+GOOD = dict(q=Q, k=K, v=V, dtype=abi.LA_DTYPE_BF16, slopes=SL, batch=1, heads=2, seq=16, dim=128,
+            block=256, state_in=S0, o=O, state_out=S1)
+
+
+def _prefill(variant=abi.LA_VARIANT_AUTO, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return abi.lightning_prefill_ex(a["q"], a["k"], a["v"], a["dtype"], a["slopes"], a["batch"],
+                                    a["heads"], a["seq"], a["dim"], a["block"], a["state_in"], a["o"],
+                                    a["state_out"], None, 0, None, variant)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype=7), abi.LA_ERR_INVALID_ARG),
+    (dict(batch=-1), abi.LA_ERR_INVALID_ARG),
+    (dict(heads=0), abi.LA_ERR_INVALID_ARG),
+    (dict(seq=-3), abi.LA_ERR_INVALID_ARG),
+    (dict(block=0), abi.LA_ERR_INVALID_ARG),
+    (dict(dim=96), abi.LA_ERR_UNSUPPORTED),
+    (dict(q=None), abi.LA_ERR_INVALID_ARG),
+    (dict(o=None), abi.LA_ERR_INVALID_ARG),
+    (dict(slopes=None), abi.LA_ERR_INVALID_ARG),
+    (dict(k=K + 8), abi.LA_ERR_INVALID_ARG),            # misaligned
+    (dict(state_out=S1 + 4), abi.LA_ERR_INVALID_ARG),   # misaligned
+    (dict(o=Q + 256), abi.LA_ERR_INVALID_ARG),          # o overlaps q
+    (dict(state_out=V), abi.LA_ERR_INVALID_ARG),        # state overlaps v
+    (dict(state_out=S0 + 4096), abi.LA_ERR_INVALID_ARG),  # partial overlap with state_in
+])
+def test_prefill_argument_errors(kw, status):
+    assert _prefill(**kw) == status
+    assert abi.last_error_message() != ""
+
+
+def test_prefill_trivial_calls_need_no_gpu():
+    assert _prefill(batch=0) == abi.LA_OK
+    assert _prefill(seq=0, state_out=None) == abi.LA_OK
+
+
+def test_unknown_variant_and_unsupported_tensor_core_requests():
+    assert _prefill(variant=9) == abi.LA_ERR_INVALID_ARG
+    assert _prefill(variant=abi.LA_VARIANT_TCGEN05, dtype=abi.LA_DTYPE_F32) == abi.LA_ERR_UNSUPPORTED
+    assert _prefill(variant=abi.LA_VARIANT_TCGEN05, dim=64) == abi.LA_ERR_UNSUPPORTED
+    assert _prefill(variant=abi.LA_VARIANT_TCGEN05, block=192) == abi.LA_ERR_UNSUPPORTED
+
+
+def test_variant_selection():
+    sel = abi.lightning_prefill_selected_variant
+    assert sel(abi.LA_DTYPE_F32, 1, 2, 256, 64, 64, abi.LA_VARIANT_AUTO) == abi.LA_VARIANT_SIMT
+    assert sel(abi.LA_DTYPE_BF16, 1, 64, 8192, 128, 256, abi.LA_VARIANT_SIMT) == abi.LA_VARIANT_SIMT
+    assert sel(abi.LA_DTYPE_BF16, 1, 64, 8192, 96, 256, abi.LA_VARIANT_AUTO) == -1
+    tc = sel(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_AUTO)
+    assert tc in (abi.LA_VARIANT_TCGEN05, abi.LA_VARIANT_SIMT)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype=5), abi.LA_ERR_INVALID_ARG),
+    (dict(dim=32), abi.LA_ERR_UNSUPPORTED),
+    (dict(state=None), abi.LA_ERR_INVALID_ARG),
+    (dict(o=S1 + 8), abi.LA_ERR_INVALID_ARG),
+    (dict(o=S1 + 1024), abi.LA_ERR_INVALID_ARG),   # o inside the state
+    (dict(state=Q), abi.LA_ERR_INVALID_ARG),       # state overlaps q
+])
+def test_decode_argument_errors(kw, status):
+    a = dict(q=Q, k=K, v=V, dtype=abi.LA_DTYPE_BF16, slopes=SL, batch=2, heads=4, dim=128, state=S1, o=O)
+    a.update(kw)
+    st = abi.lightning_decode(a["q"], a["k"], a["v"], a["dtype"], a["slopes"], a["batch"], a["heads"],
+                              a["dim"], a["state"], a["o"], None)
+    assert st == status
+
+
+def test_decode_empty_batch_is_a_no_op():
+    assert abi.lightning_decode(Q, K, V, abi.LA_DTYPE_BF16, SL, 0, 4, 128, S1, O, None) == abi.LA_OK
