@@ -1,11 +1,625 @@
-// placeholder, replaced by the tcgen05 kernel
+// Blockwise Lightning Attention prefill on the sm_100a tensor cores
+// (tcgen05 MMA with TMEM accumulators, operands staged by TMA).
+//
+// The method ("MINIMAX SIGNAL LAB · M1", §03 Lightning Attention), per block t
+// of B = 128 * NSUB tokens of one (batch, head) with slope s:
+//   O_t = [(Q_t K_t^T) ⊙ D] V_t + (Q_t ⊙ d_q) S_{t-1}
+//   S_t = e^{-s m} S_{t-1} + (K_t ⊙ d_k)^T V_t
+// D_ij = e^{-s(i-j)} 1[i>=j], d_q[i] = e^{-s(i+1)}, d_k[j] = e^{-s(m-1-j)}.
+//
+// Work split. Output columns are independent (o[:, c] needs only v[:, c] and
+// S[:, c]), so each CTA owns one (batch, head) and one half of the value
+// columns: 2 CTAs per head, each carrying S[:, half] (128 x 64 fp32) across
+// the whole sequence. The two halves recompute Q K^T; L2 serves the second
+// read of Q and K. A block of 256 rows is handled as two 128-row sub-tiles
+// a, b: P_aa = Q_a K_a^T, P_ba = Q_b K_a^T, P_bb = Q_b K_b^T (the all-zero
+// upper-right tile is skipped).
+//
+// Per block, with bf16 operands and fp32 accumulation:
+//   QK   (SS MMA, M128 N128 K128)  P tiles -> TMEM (fp32)
+//   conv (warpgroup 1)            P ⊙ D -> bf16 back into TMEM, and
+//                                 Qd = Q ⊙ d_q (bf16) next to it in TMEM
+//   PV   (TS MMA, M128 N64)       O  = P V        (A = P from TMEM)
+//   QS   (TS MMA, M128 N64)       O += Qd S_{t-1} (A = Qd from TMEM, B = bf16 S in smem)
+//   epi  (warpgroup 2)            O (TMEM) -> bf16 -> global
+//   Vd   (warpgroup 3)            V rows scaled by d_k in place (bf16)
+//   dS   (SS MMA, M128 N64 K256)  dS = K^T Vd -> TMEM
+//   state(warpgroup 3)            S = e^{-s m} S + dS in fp32 registers, bf16 copy -> smem
+// Warp roles: warp 0 issues TMA, warp 1 issues MMAs, warp 2 owns TMEM,
+// warps 4-7 / 8-11 / 12-15 are warpgroups 1 / 2 / 3. All hand-offs are
+// mbarriers; every wait is bounded (see tc_ptx.cuh).
+//
+// Shared memory (1024-aligned, 128B-swizzled tiles as TMA writes them):
+//   5 x 32 KB Q/K sub-tiles (128 rows x 128 dims), 3 x 16 KB V sub-tiles
+//   (128 rows x 64 value columns), 16 KB bf16 state operand, barriers.
+// TMEM (512 columns x 128 lanes of 32 bit):
+//   [0,128) P_aa   [128,256) P_ba   [256,384) P_bb (its upper half [320,384)
+//   doubles as dS once P_bb is in bf16)   [384,448) O_a   [448,512) O_b
 #pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <string>
-#include "common.cuh"
+
 #include "../../include/lightning.h"
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
 namespace la {
-inline bool tc_supports(bool bf16, int dim, int block) { (void)bf16; (void)dim; (void)block; return false; }
-inline la_status launch_tc(const void*, const void*, const void*, const float*, int, int, int, int,
-                           const float*, void*, float*, cudaStream_t, std::string* err) {
-    *err = "tcgen05 kernel not built"; return LA_ERR_UNSUPPORTED; }
+namespace tc {
+
+constexpr int kThreads = 512;
+constexpr int kDim = 128;
+constexpr int kRows = 128;
+constexpr int kQKSlots = 5;
+constexpr int kVSlots = 3;
+constexpr uint32_t kBoxBytes = 16384;                    // 128 rows x 64 bf16 (128 B rows)
+constexpr uint32_t kQKSlotBytes = 2 * kBoxBytes;
+constexpr uint32_t kVSlotBytes = kBoxBytes;
+constexpr uint32_t kOffQK = 0;
+constexpr uint32_t kOffV = kOffQK + kQKSlots * kQKSlotBytes;
+constexpr uint32_t kOffS = kOffV + kVSlots * kVSlotBytes;
+constexpr uint32_t kOffBar = kOffS + kBoxBytes;
+constexpr int kNumBars = 36;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;   // + slack to align the base to 1024
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColP0 = 0, kColP1 = 128, kColP2 = 256, kColDS = 320, kColO0 = 384, kColO1 = 448;
+
+// barrier indices
+constexpr int FULL_QK = 0, EMPTY_QK = 5, FULL_V = 10, EMPTY_V = 13, P_FULL = 16, P_CONV = 19,
+              P_FREE = 22, O_FULL = 25, O_FREE = 27, PV_DONE = 29, VD_READY = 30, DS_FULL = 31,
+              DS_FREE = 32, S_READY = 33, DRAIN = 34;
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulate, M x N.
+__host__ __device__ constexpr uint32_t idesc(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+constexpr uint32_t kIdescQK = idesc(128, 128, false, false);  // Q (K-major) x K (K-major)
+constexpr uint32_t kIdescPV = idesc(128, 64, false, true);    // P/Qd (TMEM) x V/S (MN-major)
+constexpr uint32_t kIdescDS = idesc(128, 64, true, true);     // K^T (MN-major) x Vd (MN-major)
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// K-major operand (rows of 128 dims = two 64-dim boxes): k-step k of 16 dims
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int k) {
+    return sdesc(tile + (uint32_t)(k >> 2) * kBoxBytes + (uint32_t)(k & 3) * 32u, 16u, 1024u);
+}
+// MN-major operand (rows = the K dimension, 128 B per row): k-step of 16 rows
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int k) {
+    return sdesc(tile + (uint32_t)k * 2048u, kBoxBytes, 1024u);
+}
+
+// Rotation of the five Q/K sub-tile slots between blocks. Slots are reused in
+// the order they are released: Q slots free early (after their P tiles are
+// converted), K slots only after the block's state MMA.
+template <int NSUB>
+struct SlotMap {
+    int k0, q0, k1, q1, f, t;
+    __device__ __forceinline__ void init() {
+        t = 0;
+        k0 = 0; q0 = 1; k1 = 2; q1 = 3; f = 4;
+    }
+    __device__ __forceinline__ void advance() {
+        ++t;
+        if (NSUB == 2) {
+            const int nk0 = f, nq0 = q0, nq1 = q1, nk1 = k0, nf = k1;
+            k0 = nk0; q0 = nq0; q1 = nq1; k1 = nk1; f = nf;
+        } else {
+            k0 = (2 * t) % kQKSlots;
+            q0 = (2 * t + 1) % kQKSlots;
+        }
+    }
+    __device__ __forceinline__ uint32_t used_mask() const {
+        return NSUB == 2 ? ((1u << k0) | (1u << q0) | (1u << k1) | (1u << q1)) : ((1u << k0) | (1u << q0));
+    }
+};
+
+struct Ctx {
+    uint8_t *smem;
+    uint32_t sbase;       // shared address of smem
+    uint64_t *bars;
+    volatile int *abort;
+    uint32_t tmem;
+};
+
+__device__ __forceinline__ bool wait_bar(const Ctx &c, int idx, uint32_t parity) {
+    return ptx::mbar_wait(&c.bars[idx], parity, c.abort);
+}
+
+// Warpgroup-wide wait: thread 0 of the group polls the mbarrier, the named
+// barrier hands its verdict to all 128 threads, so every thread of the group
+// takes the same path (no thread is left behind at a later named barrier).
+__device__ __forceinline__ bool wg_wait(const Ctx &c, int idx, uint32_t parity, int r, int bar_id) {
+    const bool ok = (r == 0) ? wait_bar(c, idx, parity) : true;
+    return ptx::named_bar_and(bar_id, 128, ok);
+}
+
+template <int NSUB>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ slopes, int heads,
+                  int seq, const float *state_in, __nv_bfloat16 *o, float *state_out) {
+    constexpr int B = kRows * NSUB;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+    const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+    Ctx c;
+    c.smem = smem_raw + pad;
+    c.sbase = raw_addr + pad;
+    c.bars = reinterpret_cast<uint64_t *>(c.smem + kOffBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c.smem + kOffMisc);
+    c.abort = reinterpret_cast<volatile int *>(c.smem + kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x >> 1, half = blockIdx.x & 1;
+    const float s = slopes[bh % heads];
+    const float sl2 = s * kLog2e;  // e^{-s n} = 2^{-sl2 n}
+    const int nblk = (seq + B - 1) / B;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(&c.bars[i], 1);
+        *c.abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tensormap(&tm_q);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+    }
+    if (warp == 2) {
+        ptx::tmem_alloc(tmem_slot, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    c.tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t qk_par = 0, qk_issued = 0, v_issued = 0;
+            int vtile = 0;
+            SlotMap<NSUB> sm;
+            sm.init();
+            bool ok = true;
+            auto load_qk = [&](int slot, const CUtensorMap *map, int row) -> bool {
+                if (!wait_bar(c, EMPTY_QK + slot, ((qk_par >> slot) & 1u) ^ 1u)) return false;
+                qk_par ^= 1u << slot;
+                qk_issued |= 1u << slot;
+                uint8_t *dst = c.smem + kOffQK + slot * kQKSlotBytes;
+                ptx::mbar_arrive_expect_tx(&c.bars[FULL_QK + slot], kQKSlotBytes);
+                ptx::tma_load_3d(dst, map, &c.bars[FULL_QK + slot], 0, row, bh);
+                ptx::tma_load_3d(dst + kBoxBytes, map, &c.bars[FULL_QK + slot], 64, row, bh);
+                return true;
+            };
+            auto load_v = [&](int n, int row) -> bool {
+                const int slot = n % kVSlots;
+                if (!wait_bar(c, EMPTY_V + slot, ((uint32_t)(n / kVSlots) & 1u) ^ 1u)) return false;
+                v_issued |= 1u << slot;
+                ptx::mbar_arrive_expect_tx(&c.bars[FULL_V + slot], kVSlotBytes);
+                ptx::tma_load_3d(c.smem + kOffV + slot * kVSlotBytes, &tm_v, &c.bars[FULL_V + slot],
+                                 64 * half, row, bh);
+                return true;
+            };
+            for (int t = 0; t < nblk && ok; ++t) {
+                const int row0 = t * B;
+                ok = ok && load_qk(sm.k0, &tm_k, row0);
+                ok = ok && load_qk(sm.q0, &tm_q, row0);
+                ok = ok && load_v(vtile, row0);
+                if (NSUB == 2) {
+                    ok = ok && load_qk(sm.q1, &tm_q, row0 + kRows);
+                    ok = ok && load_qk(sm.k1, &tm_k, row0 + kRows);
+                    ok = ok && load_v(vtile + 1, row0 + kRows);
+                }
+                vtile += NSUB;
+                sm.advance();
+            }
+            {
+                // let every copy issued land before the CTA exits (already true
+                // unless some role gave up early)
+                for (int sl = 0; sl < kQKSlots; ++sl)
+                    if (qk_issued & (1u << sl)) {
+                        volatile int never = 0;
+                        ptx::mbar_wait(&c.bars[FULL_QK + sl], ((qk_par >> sl) & 1u) ^ 1u, &never);
+                    }
+                for (int sl = 0; sl < kVSlots; ++sl)
+                    if (v_issued & (1u << sl)) {
+                        volatile int never = 0;
+                        int last = -1;
+                        for (int n = 0; n < vtile; ++n)
+                            if (n % kVSlots == sl) last = n;
+                        if (last >= 0) ptx::mbar_wait(&c.bars[FULL_V + sl], (uint32_t)(last / kVSlots) & 1u, &never);
+                    }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t qk_par = 0;
+            int vtile = 0;
+            SlotMap<NSUB> sm;
+            sm.init();
+            const uint32_t tm = c.tmem;
+            const uint32_t s_tile = c.sbase + kOffS;
+            auto qk_tile = [&](int slot) { return c.sbase + kOffQK + (uint32_t)slot * kQKSlotBytes; };
+            auto v_tile = [&](int n) { return c.sbase + kOffV + (uint32_t)(n % kVSlots) * kVSlotBytes; };
+            auto wait_qk = [&](int slot) -> bool {
+                const bool r = wait_bar(c, FULL_QK + slot, (qk_par >> slot) & 1u);
+                qk_par ^= 1u << slot;
+                return r;
+            };
+            auto issue_qk = [&](uint32_t dcol, int qslot, int kslot) {
+                for (int k = 0; k < 8; ++k)
+                    ptx::mma_ss(tm + dcol, desc_kmajor(qk_tile(qslot), k), desc_kmajor(qk_tile(kslot), k),
+                                kIdescQK, k > 0);
+            };
+            auto issue_pv = [&](uint32_t dcol, uint32_t acol, uint32_t vt, bool acc) {
+                for (int k = 0; k < 8; ++k)
+                    ptx::mma_ts(tm + dcol, tm + acol + 8u * k, desc_mnmajor(vt, k), kIdescPV, acc || k > 0);
+            };
+            auto issue_ds = [&](uint32_t kt, uint32_t vt, bool acc) {
+                for (int k = 0; k < 8; ++k)
+                    ptx::mma_ss(tm + kColDS, desc_mnmajor(kt, k), desc_mnmajor(vt, k), kIdescDS, acc || k > 0);
+            };
+            bool ok = true;
+            for (int t = 0; t < nblk && ok; ++t) {
+                const uint32_t par = t & 1, fpar = par ^ 1u;
+                const int va = vtile, vb = vtile + 1;
+                // P_aa = Q_a K_a^T
+                ok = wait_qk(sm.k0) && wait_qk(sm.q0) && wait_bar(c, P_FREE + 0, fpar);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                issue_qk(kColP0, sm.q0, sm.k0);
+                ptx::mma_commit(&c.bars[P_FULL + 0]);
+                if (NSUB == 2) {
+                    // P_ba = Q_b K_a^T
+                    ok = wait_qk(sm.q1) && wait_bar(c, P_FREE + 1, fpar);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    issue_qk(kColP1, sm.q1, sm.k0);
+                    ptx::mma_commit(&c.bars[P_FULL + 1]);
+                }
+                // O_a = P_aa V_a + Qd_a S_{t-1}
+                ok = wait_bar(c, FULL_V + va % kVSlots, (uint32_t)(va / kVSlots) & 1u) &&
+                     wait_bar(c, P_CONV + 0, par) && wait_bar(c, O_FREE + 0, fpar) &&
+                     wait_bar(c, S_READY, par);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                issue_pv(kColO0, kColP0, v_tile(va), false);
+                issue_pv(kColO0, kColP0 + 64, s_tile, true);
+                ptx::mma_commit(&c.bars[P_FREE + 0]);
+                ptx::mma_commit(&c.bars[O_FULL + 0]);
+                if (NSUB == 2) {
+                    // O_b = P_ba V_a + Qd_b S_{t-1} + P_bb V_b
+                    ok = wait_bar(c, P_CONV + 1, par) && wait_bar(c, O_FREE + 1, fpar);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    issue_pv(kColO1, kColP1, v_tile(va), false);
+                    issue_pv(kColO1, kColP1 + 64, s_tile, true);
+                    ptx::mma_commit(&c.bars[P_FREE + 1]);
+                    // P_bb = Q_b K_b^T (its upper half is the dS region: wait until dS_{t-1} was read)
+                    ok = wait_qk(sm.k1) && wait_bar(c, P_FREE + 2, fpar) && wait_bar(c, DS_FREE, fpar);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    issue_qk(kColP2, sm.q1, sm.k1);
+                    ptx::mma_commit(&c.bars[P_FULL + 2]);
+                    ok = wait_bar(c, FULL_V + vb % kVSlots, (uint32_t)(vb / kVSlots) & 1u) &&
+                         wait_bar(c, P_CONV + 2, par);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    issue_pv(kColO1, kColP2, v_tile(vb), true);
+                    ptx::mma_commit(&c.bars[P_FREE + 2]);
+                    ptx::mma_commit(&c.bars[O_FULL + 1]);
+                }
+                ptx::mma_commit(&c.bars[PV_DONE]);
+                // dS = K^T (d_k ⊙ V)
+                ok = wait_bar(c, VD_READY, par) && (NSUB == 2 || wait_bar(c, DS_FREE, fpar));
+                if (!ok) break;
+                ptx::tc_fence_after();
+                issue_ds(qk_tile(sm.k0), v_tile(va), false);
+                if (NSUB == 2) issue_ds(qk_tile(sm.k1), v_tile(vb), true);
+                ptx::mma_commit(&c.bars[DS_FULL]);
+                ptx::mma_commit(&c.bars[EMPTY_QK + sm.k0]);
+                ptx::mma_commit(&c.bars[EMPTY_V + va % kVSlots]);
+                if (NSUB == 2) {
+                    ptx::mma_commit(&c.bars[EMPTY_QK + sm.k1]);
+                    ptx::mma_commit(&c.bars[EMPTY_V + vb % kVSlots]);
+                }
+                vtile += NSUB;
+                sm.advance();
+            }
+            // drain: every MMA issued has completed before TMEM is released
+            ptx::mma_commit(&c.bars[DRAIN]);
+            volatile int never = 0;
+            ptx::mbar_wait(&c.bars[DRAIN], 0, &never);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ warpgroup 1: P conversion
+        const int r = threadIdx.x - 128;
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        const float step = ptx::ex2(-sl2);  // e^{-s}
+        uint32_t qk_par = 0;
+        SlotMap<NSUB> sm;
+        sm.init();
+        for (int t = 0; t < nblk; ++t) {
+            const uint32_t par = t & 1;
+            for (int tile = 0; tile < 2 * NSUB - 1; ++tile) {
+                // tile 0: P_aa (rows a, keys a, Qd_a); 1: P_ba (rows b, keys a, Qd_b); 2: P_bb
+                const uint32_t col = tile == 0 ? kColP0 : (tile == 1 ? kColP1 : kColP2);
+                const int i = (tile == 0 ? 0 : kRows) + r;
+                const int j0 = tile == 2 ? kRows : 0;
+                if (!wg_wait(c, P_FULL + tile, par, r, 1)) goto wg1_done;
+                ptx::tc_fence_after();
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t v[32], out[16];
+                    ptx::tmem_ld32(c.tmem + lane_off + col + 32 * ch, v);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        const int jb = j0 + 32 * ch + 16 * g;
+                        const int dlast = i - (jb + 15);
+                        float p[16];
+                        if (dlast >= 0) {
+                            float w = ptx::ex2(-sl2 * (float)dlast);
+#pragma unroll
+                            for (int u = 15; u >= 0; --u) {
+                                p[u] = __uint_as_float(v[16 * g + u]) * w;
+                                w *= step;
+                            }
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 16; ++u) {
+                                const int dd = i - (jb + u);
+                                p[u] = dd >= 0 ? __uint_as_float(v[16 * g + u]) * ptx::ex2(-sl2 * (float)dd) : 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) out[8 * g + u] = ptx::pack_bf16(p[2 * u], p[2 * u + 1]);
+                    }
+                    __syncwarp();
+                    ptx::tmem_st16(c.tmem + lane_off + col + 16 * ch, out);
+                }
+                if (tile < 2) {
+                    // Qd = Q ⊙ d_q for this row, from the swizzled Q sub-tile
+                    const int qslot = tile == 0 ? sm.q0 : sm.q1;
+                    if (!wg_wait(c, FULL_QK + qslot, (qk_par >> qslot) & 1u, r, 1)) goto wg1_done;
+                    const float dq = ptx::ex2(-sl2 * (float)(i + 1));
+                    const uint8_t *qrow = c.smem + kOffQK + qslot * kQKSlotBytes + r * 128;
+#pragma unroll
+                    for (int hb = 0; hb < 4; ++hb) {  // 4 x 16 output words = 2 boxes x 8 chunks
+                        uint32_t out[16];
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int chunk = (hb & 1) * 4 + cc;
+                            const uint8_t *src = qrow + (hb >> 1) * kBoxBytes + ((chunk ^ (r & 7)) << 4);
+                            const uint4 w = *reinterpret_cast<const uint4 *>(src);
+                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                out[4 * cc + e] = ptx::pack_bf16(ptx::bf16_lo(ws[e]) * dq, ptx::bf16_hi(ws[e]) * dq);
+                        }
+                        ptx::tmem_st16(c.tmem + lane_off + col + 64 + 16 * hb, out);
+                    }
+                }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                ptx::named_bar_sync(1, 128);
+                if (r == 0) {
+                    ptx::mbar_arrive(&c.bars[P_CONV + tile]);
+                    // Q_a is done after P_aa; Q_b after P_bb (or after P_aa when B = 128)
+                    if (tile == 0) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q0]);
+                    if (tile == 2) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q1]);
+                }
+            }
+            qk_par ^= sm.used_mask();
+            sm.advance();
+        }
+    wg1_done:;
+    } else if (warp >= 8 && warp < 12) {
+        // ------------------------------------------------------------ warpgroup 2: epilogue
+        const int r = threadIdx.x - 256;
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        for (int t = 0; t < nblk; ++t) {
+            const uint32_t par = t & 1;
+            for (int sub = 0; sub < NSUB; ++sub) {
+                if (!wg_wait(c, O_FULL + sub, par, r, 2)) goto wg2_done;
+                ptx::tc_fence_after();
+                uint32_t a[32], b[32];
+                const uint32_t col = sub == 0 ? kColO0 : kColO1;
+                ptx::tmem_ld32(c.tmem + lane_off + col, a);
+                ptx::tmem_ld32(c.tmem + lane_off + col + 32, b);
+                ptx::tmem_ld_wait();
+                ptx::tc_fence_before();
+                ptx::named_bar_sync(2, 128);
+                if (r == 0) ptx::mbar_arrive(&c.bars[O_FREE + sub]);
+                const int row = t * B + sub * kRows + r;
+                if (row < seq) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)bh * seq + row) * kDim + 64 * half);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(ptx::pack_bf16(__uint_as_float(a[8 * q + 0]), __uint_as_float(a[8 * q + 1])),
+                                            ptx::pack_bf16(__uint_as_float(a[8 * q + 2]), __uint_as_float(a[8 * q + 3])),
+                                            ptx::pack_bf16(__uint_as_float(a[8 * q + 4]), __uint_as_float(a[8 * q + 5])),
+                                            ptx::pack_bf16(__uint_as_float(a[8 * q + 6]), __uint_as_float(a[8 * q + 7])));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[4 + q] = make_uint4(ptx::pack_bf16(__uint_as_float(b[8 * q + 0]), __uint_as_float(b[8 * q + 1])),
+                                                ptx::pack_bf16(__uint_as_float(b[8 * q + 2]), __uint_as_float(b[8 * q + 3])),
+                                                ptx::pack_bf16(__uint_as_float(b[8 * q + 4]), __uint_as_float(b[8 * q + 5])),
+                                                ptx::pack_bf16(__uint_as_float(b[8 * q + 6]), __uint_as_float(b[8 * q + 7])));
+                }
+            }
+        }
+    wg2_done:;
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------ warpgroup 3: state carry
+        const int r = threadIdx.x - 384;  // key-dimension row of S owned by this thread
+        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        float S[64];
+        const size_t sbase = (size_t)bh * kDim * kDim + (size_t)r * kDim + 64 * half;
+        if (state_in) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const float4 x = *reinterpret_cast<const float4 *>(state_in + sbase + 4 * q);
+                S[4 * q] = x.x; S[4 * q + 1] = x.y; S[4 * q + 2] = x.z; S[4 * q + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 64; ++q) S[q] = 0.f;
+        }
+        uint8_t *srow = c.smem + kOffS + r * 128;
+        auto write_state_operand = [&]() {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint4 w;
+                w.x = ptx::pack_bf16(S[8 * ch + 0], S[8 * ch + 1]);
+                w.y = ptx::pack_bf16(S[8 * ch + 2], S[8 * ch + 3]);
+                w.z = ptx::pack_bf16(S[8 * ch + 4], S[8 * ch + 5]);
+                w.w = ptx::pack_bf16(S[8 * ch + 6], S[8 * ch + 7]);
+                *reinterpret_cast<uint4 *>(srow + ((ch ^ (r & 7)) << 4)) = w;
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::named_bar_sync(3, 128);
+            if (r == 0) ptx::mbar_arrive(&c.bars[S_READY]);
+        };
+        write_state_operand();
+        int vtile = 0;
+        for (int t = 0; t < nblk; ++t) {
+            const uint32_t par = t & 1;
+            const int m = min(B, seq - t * B);
+            if (!wg_wait(c, PV_DONE, par, r, 3)) goto wg3_done;
+            for (int sub = 0; sub < NSUB; ++sub) {
+                const int n = vtile + sub;
+                if (!wg_wait(c, FULL_V + n % kVSlots, (uint32_t)(n / kVSlots) & 1u, r, 3)) goto wg3_done;
+                const int j = sub * kRows + r;
+                const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
+                uint8_t *vrow = c.smem + kOffV + (n % kVSlots) * kVSlotBytes + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint4 *p = reinterpret_cast<uint4 *>(vrow + (ch << 4));
+                    uint4 w = *p;
+                    w.x = ptx::pack_bf16(ptx::bf16_lo(w.x) * dk, ptx::bf16_hi(w.x) * dk);
+                    w.y = ptx::pack_bf16(ptx::bf16_lo(w.y) * dk, ptx::bf16_hi(w.y) * dk);
+                    w.z = ptx::pack_bf16(ptx::bf16_lo(w.z) * dk, ptx::bf16_hi(w.z) * dk);
+                    w.w = ptx::pack_bf16(ptx::bf16_lo(w.w) * dk, ptx::bf16_hi(w.w) * dk);
+                    *p = w;
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::named_bar_sync(3, 128);
+            if (r == 0) ptx::mbar_arrive(&c.bars[VD_READY]);
+
+            if (!wg_wait(c, DS_FULL, par, r, 3)) goto wg3_done;
+            ptx::tc_fence_after();
+            const float dblock = ptx::ex2(-sl2 * (float)m);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t d[32];
+                ptx::tmem_ld32(c.tmem + lane_off + kColDS + 32 * hh, d);
+                ptx::tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) S[32 * hh + q] = fmaf(dblock, S[32 * hh + q], __uint_as_float(d[q]));
+            }
+            ptx::tc_fence_before();
+            ptx::named_bar_sync(3, 128);
+            if (r == 0) ptx::mbar_arrive(&c.bars[DS_FREE]);
+            write_state_operand();
+            vtile += NSUB;
+        }
+        if (state_out) {
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                *reinterpret_cast<float4 *>(state_out + sbase + 4 * q) =
+                    make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+        }
+    wg3_done:;
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(c.tmem, kTmemCols);
+    }
+}
+
+}  // namespace tc
+
+// The tensor-core kernel covers bf16 inputs, head dim 128 and blocks of 128 or 256.
+inline bool tc_supports(bool bf16, int dim, int block) {
+    return bf16 && dim == 128 && (block == 128 || block == 256);
+}
+
+namespace tc {
+
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn(std::string *err) {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) {
+            *err = "cuTensorMapEncodeTiled is not available from the driver";
+            return nullptr;
+        }
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// [batch*heads][seq][128] bf16 viewed as a 3-D tensor; boxes of 64 dims x 128 rows,
+// 128-byte swizzle; rows past seq read as zeros.
+inline bool make_map(CUtensorMap *map, const void *base, int seq, long long bh, std::string *err) {
+    auto fn = encode_fn(err);
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kDim, (cuuint64_t)seq, (cuuint64_t)bh};
+    cuuint64_t strides[2] = {(cuuint64_t)kDim * 2, (cuuint64_t)seq * kDim * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)kRows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *err = "cuTensorMapEncodeTiled failed (CUresult " + std::to_string((int)r) + ")";
+        return false;
+    }
+    return true;
+}
+
+}  // namespace tc
+
+inline la_status launch_tc(const void *q, const void *k, const void *v, const float *slopes, int batch,
+                           int heads, int seq, int block, const float *state_in, void *o, float *state_out,
+                           cudaStream_t stream, std::string *err) {
+    const long long bh = (long long)batch * heads;
+    CUtensorMap mq, mk, mv;
+    if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
+        !tc::make_map(&mv, v, seq, bh, err))
+        return LA_ERR_CUDA;
+    auto kern = block == 256 ? tc::prefill_tc_kernel<2> : tc::prefill_tc_kernel<1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
+    if (e != cudaSuccess) {
+        *err = std::string("cudaFuncSetAttribute(prefill_tc): ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    kern<<<(unsigned)(bh * 2), tc::kThreads, tc::kSmemBytes, stream>>>(
+        mq, mk, mv, slopes, heads, seq, state_in, static_cast<__nv_bfloat16 *>(o), state_out);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        *err = std::string("prefill_tc launch: ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    err->clear();
+    return LA_OK;
+}
+
+}  // namespace la
