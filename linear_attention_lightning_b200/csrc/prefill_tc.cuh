@@ -15,26 +15,33 @@
 // a, b: P_aa = Q_a K_a^T, P_ba = Q_b K_a^T, P_bb = Q_b K_b^T (the all-zero
 // upper-right tile is skipped).
 //
-// Per block, with bf16 operands and fp32 accumulation:
-//   QK   (SS MMA, M128 N128 K128)  P tiles -> TMEM (fp32)
-//   conv (warpgroup 1)            P ⊙ D -> bf16 back into TMEM, and
-//                                 Qd = Q ⊙ d_q (bf16) next to it in TMEM
-//   PV   (TS MMA, M128 N64)       O  = P V        (A = P from TMEM)
-//   QS   (TS MMA, M128 N64)       O += Qd S_{t-1} (A = Qd from TMEM, B = bf16 S in smem)
-//   epi  (warpgroup 2)            O (TMEM) -> bf16 -> global
-//   Vd   (warpgroup 3)            V rows scaled by d_k in place (bf16)
-//   dS   (SS MMA, M128 N64 K256)  dS = K^T Vd -> TMEM
-//   state(warpgroup 3)            S = e^{-s m} S + dS in fp32 registers, bf16 copy -> smem
+// Precision. Q K^T runs on the bf16 inputs. Every operand the kernel itself
+// produces — P ⊙ D, Q ⊙ d_q, the carried state S and K ⊙ d_k — is rounded to
+// fp16 (11 significant bits) rather than bf16 (8): these values are bounded
+// (|D|, d_q, d_k <= 1) and an fp16 operand carries an 8x smaller rounding
+// error. V is converted bf16 -> fp16 exactly. All accumulation is fp32 and
+// the state is carried in fp32.
+//
+// Per block:
+//   QK    (SS MMA bf16, M128 N128 K128)  P tiles -> TMEM (fp32)
+//   conv  (warps 4-11)                   P ⊙ D -> fp16 back into TMEM, and
+//                                        Qd = Q ⊙ d_q (fp16) next to it
+//   PV    (TS MMA f16, M128 N64)         O  = P V          (A = P from TMEM)
+//   dS    (SS MMA f16, M128 N64 K256)    dS = (K ⊙ d_k)^T V
+//   QS    (TS MMA f16, M128 N64)         O += Qd S_{t-1}   (B = fp16 S in smem)
+//   warpgroup 3: converts V to fp16 and K to fp16 K ⊙ d_k in place, carries
+//                S = e^{-s m} S + dS in fp32 registers (fp16 copy -> smem),
+//                and writes O (TMEM -> bf16 -> global).
 // Warp roles: warp 0 issues TMA, warp 1 issues MMAs, warp 2 owns TMEM,
-// warps 4-7 / 8-11 / 12-15 are warpgroups 1 / 2 / 3. All hand-offs are
-// mbarriers; every wait is bounded (see tc_ptx.cuh).
+// warps 4-11 convert P (each warpgroup one half of the columns), warps 12-15
+// are warpgroup 3. All hand-offs are mbarriers; every wait is bounded.
 //
 // Shared memory (1024-aligned, 128B-swizzled tiles as TMA writes them):
 //   5 x 32 KB Q/K sub-tiles (128 rows x 128 dims), 3 x 16 KB V sub-tiles
-//   (128 rows x 64 value columns), 16 KB bf16 state operand, barriers.
+//   (128 rows x 64 value columns), 16 KB fp16 state operand, barriers.
 // TMEM (512 columns x 128 lanes of 32 bit):
-//   [0,128) P_aa   [128,256) P_ba   [256,384) P_bb (its upper half [320,384)
-//   doubles as dS once P_bb is in bf16)   [384,448) O_a   [448,512) O_b
+//   [0,128) P_aa | Qd_a   [128,256) P_ba | Qd_b   [256,384) P_bb | dS
+//   [384,448) O_a   [448,512) O_b
 #pragma once
 
 #include <cuda.h>
@@ -54,7 +61,7 @@ constexpr int kDim = 128;
 constexpr int kRows = 128;
 constexpr int kQKSlots = 5;
 constexpr int kVSlots = 3;
-constexpr uint32_t kBoxBytes = 16384;                    // 128 rows x 64 bf16 (128 B rows)
+constexpr uint32_t kBoxBytes = 16384;                    // 128 rows x 64 16-bit (128 B rows)
 constexpr uint32_t kQKSlotBytes = 2 * kBoxBytes;
 constexpr uint32_t kVSlotBytes = kBoxBytes;
 constexpr uint32_t kOffQK = 0;
@@ -66,21 +73,27 @@ constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;   // + slack to align the base to 1024
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColP0 = 0, kColP1 = 128, kColP2 = 256, kColDS = 320, kColO0 = 384, kColO1 = 448;
+constexpr uint32_t kColP0 = 0, kColP1 = 128, kColP2 = 256;
+constexpr uint32_t kColDS = 320, kColO0 = 384, kColO1 = 448;
+
+__device__ __forceinline__ uint32_t p_col(int tile) { return tile == 0 ? kColP0 : (tile == 1 ? kColP1 : kColP2); }
 
 // barrier indices
 constexpr int FULL_QK = 0, EMPTY_QK = 5, FULL_V = 10, EMPTY_V = 13, P_FULL = 16, P_CONV = 19,
-              P_FREE = 22, O_FULL = 25, O_FREE = 27, PV_DONE = 29, VD_READY = 30, DS_FULL = 31,
-              DS_FREE = 32, S_READY = 33, DRAIN = 34;
+              P_FREE = 22, O_FULL = 25, O_FREE = 27, V_CONV = 29, KD_READY = 31, DS_FULL = 32,
+              DS_FREE = 33, S_READY = 34, DRAIN = 35;
 
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulate, M x N.
-__host__ __device__ constexpr uint32_t idesc(int M, int N, bool a_mn_major, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+// named barriers: 1 = the 256 conversion threads, 2 = warpgroup 3
+constexpr int kBarConv = 1, kBarWG3 = 2;
+
+// Instruction descriptor, kind::f16, fp32 accumulate, M x N; fmt 0 = f16, 1 = bf16.
+__host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) |
            ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr uint32_t kIdescQK = idesc(128, 128, false, false);  // Q (K-major) x K (K-major)
-constexpr uint32_t kIdescPV = idesc(128, 64, false, true);    // P/Qd (TMEM) x V/S (MN-major)
-constexpr uint32_t kIdescDS = idesc(128, 64, true, true);     // K^T (MN-major) x Vd (MN-major)
+constexpr uint32_t kIdescQK = idesc(128, 128, 1, false, false);  // Q x K^T, bf16, both K-major
+constexpr uint32_t kIdescPV = idesc(128, 64, 0, false, true);    // P/Qd (TMEM) x V/S (MN-major), f16
+constexpr uint32_t kIdescDS = idesc(128, 64, 0, true, true);     // Kd^T (MN-major) x V (MN-major), f16
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -133,12 +146,18 @@ __device__ __forceinline__ bool wait_bar(const Ctx &c, int idx, uint32_t parity)
     return ptx::mbar_wait(&c.bars[idx], parity, c.abort);
 }
 
-// Warpgroup-wide wait: thread 0 of the group polls the mbarrier, the named
-// barrier hands its verdict to all 128 threads, so every thread of the group
-// takes the same path (no thread is left behind at a later named barrier).
-__device__ __forceinline__ bool wg_wait(const Ctx &c, int idx, uint32_t parity, int r, int bar_id) {
-    const bool ok = (r == 0) ? wait_bar(c, idx, parity) : true;
-    return ptx::named_bar_and(bar_id, 128, ok);
+// Group-wide wait: the group's first thread polls the mbarrier, the named
+// barrier hands its verdict to every thread of the group, so all of them take
+// the same path (none is left behind at a later named barrier).
+__device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parity, bool leader, int bar_id,
+                                           int threads) {
+    const bool ok = leader ? wait_bar(c, idx, parity) : true;
+    return ptx::named_bar_and(bar_id, threads, ok);
+}
+
+// bf16x2 word -> f16x2 word of the values times `scale`
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
+    return ptx::pack_f16(ptx::bf16_lo(w) * scale, ptx::bf16_hi(w) * scale);
 }
 
 template <int NSUB>
@@ -147,6 +166,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ slopes, int heads,
                   int seq, const float *state_in, __nv_bfloat16 *o, float *state_out) {
     constexpr int B = kRows * NSUB;
+    constexpr int kLastTile = 2 * NSUB - 2;  // index of the block's last P tile
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_addr(smem_raw);
     const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -185,8 +205,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t qk_par = 0, qk_issued = 0, v_issued = 0;
-            int vtile = 0;
+            uint32_t qk_par = 0, qk_issued = 0;
+            int vtile = 0, vissued = 0;
             SlotMap<NSUB> sm;
             sm.init();
             bool ok = true;
@@ -203,10 +223,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             auto load_v = [&](int n, int row) -> bool {
                 const int slot = n % kVSlots;
                 if (!wait_bar(c, EMPTY_V + slot, ((uint32_t)(n / kVSlots) & 1u) ^ 1u)) return false;
-                v_issued |= 1u << slot;
                 ptx::mbar_arrive_expect_tx(&c.bars[FULL_V + slot], kVSlotBytes);
                 ptx::tma_load_3d(c.smem + kOffV + slot * kVSlotBytes, &tm_v, &c.bars[FULL_V + slot],
                                  64 * half, row, bh);
+                vissued = n + 1;
                 return true;
             };
             for (int t = 0; t < nblk && ok; ++t) {
@@ -222,23 +242,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 vtile += NSUB;
                 sm.advance();
             }
-            {
-                // let every copy issued land before the CTA exits (already true
-                // unless some role gave up early)
-                for (int sl = 0; sl < kQKSlots; ++sl)
-                    if (qk_issued & (1u << sl)) {
-                        volatile int never = 0;
-                        ptx::mbar_wait(&c.bars[FULL_QK + sl], ((qk_par >> sl) & 1u) ^ 1u, &never);
-                    }
-                for (int sl = 0; sl < kVSlots; ++sl)
-                    if (v_issued & (1u << sl)) {
-                        volatile int never = 0;
-                        int last = -1;
-                        for (int n = 0; n < vtile; ++n)
-                            if (n % kVSlots == sl) last = n;
-                        if (last >= 0) ptx::mbar_wait(&c.bars[FULL_V + sl], (uint32_t)(last / kVSlots) & 1u, &never);
-                    }
-            }
+            // every copy issued lands before the CTA exits (already true unless
+            // some role gave up early)
+            volatile int never = 0;
+            for (int sl = 0; sl < kQKSlots; ++sl)
+                if (qk_issued & (1u << sl))
+                    ptx::mbar_wait(&c.bars[FULL_QK + sl], ((qk_par >> sl) & 1u) ^ 1u, &never);
+            for (int n = vissued > kVSlots ? vissued - kVSlots : 0; n < vissued; ++n)
+                ptx::mbar_wait(&c.bars[FULL_V + n % kVSlots], (uint32_t)(n / kVSlots) & 1u, &never);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -261,9 +272,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     ptx::mma_ss(tm + dcol, desc_kmajor(qk_tile(qslot), k), desc_kmajor(qk_tile(kslot), k),
                                 kIdescQK, k > 0);
             };
-            auto issue_pv = [&](uint32_t dcol, uint32_t acol, uint32_t vt, bool acc) {
+            auto issue_ts = [&](uint32_t dcol, uint32_t acol, uint32_t bt, bool acc) {
                 for (int k = 0; k < 8; ++k)
-                    ptx::mma_ts(tm + dcol, tm + acol + 8u * k, desc_mnmajor(vt, k), kIdescPV, acc || k > 0);
+                    ptx::mma_ts(tm + dcol, tm + acol + 8u * k, desc_mnmajor(bt, k), kIdescPV, acc || k > 0);
             };
             auto issue_ds = [&](uint32_t kt, uint32_t vt, bool acc) {
                 for (int k = 0; k < 8; ++k)
@@ -286,46 +297,49 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     ptx::tc_fence_after();
                     issue_qk(kColP1, sm.q1, sm.k0);
                     ptx::mma_commit(&c.bars[P_FULL + 1]);
-                }
-                // O_a = P_aa V_a + Qd_a S_{t-1}
-                ok = wait_bar(c, FULL_V + va % kVSlots, (uint32_t)(va / kVSlots) & 1u) &&
-                     wait_bar(c, P_CONV + 0, par) && wait_bar(c, O_FREE + 0, fpar) &&
-                     wait_bar(c, S_READY, par);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                issue_pv(kColO0, kColP0, v_tile(va), false);
-                issue_pv(kColO0, kColP0 + 64, s_tile, true);
-                ptx::mma_commit(&c.bars[P_FREE + 0]);
-                ptx::mma_commit(&c.bars[O_FULL + 0]);
-                if (NSUB == 2) {
-                    // O_b = P_ba V_a + Qd_b S_{t-1} + P_bb V_b
-                    ok = wait_bar(c, P_CONV + 1, par) && wait_bar(c, O_FREE + 1, fpar);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                    issue_pv(kColO1, kColP1, v_tile(va), false);
-                    issue_pv(kColO1, kColP1 + 64, s_tile, true);
-                    ptx::mma_commit(&c.bars[P_FREE + 1]);
-                    // P_bb = Q_b K_b^T (its upper half is the dS region: wait until dS_{t-1} was read)
+                    // P_bb = Q_b K_b^T; its upper half is the dS region of the previous block
                     ok = wait_qk(sm.k1) && wait_bar(c, P_FREE + 2, fpar) && wait_bar(c, DS_FREE, fpar);
                     if (!ok) break;
                     ptx::tc_fence_after();
                     issue_qk(kColP2, sm.q1, sm.k1);
                     ptx::mma_commit(&c.bars[P_FULL + 2]);
-                    ok = wait_bar(c, FULL_V + vb % kVSlots, (uint32_t)(vb / kVSlots) & 1u) &&
-                         wait_bar(c, P_CONV + 2, par);
+                }
+                // O_a = P_aa V_a
+                ok = wait_bar(c, V_CONV + 0, par) && wait_bar(c, P_CONV + 0, par) && wait_bar(c, O_FREE + 0, fpar);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                issue_ts(kColO0, kColP0, v_tile(va), false);
+                if (NSUB == 2) {
+                    // O_b = P_ba V_a + P_bb V_b
+                    ok = wait_bar(c, P_CONV + 1, par) && wait_bar(c, O_FREE + 1, fpar);
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    issue_pv(kColO1, kColP2, v_tile(vb), true);
+                    issue_ts(kColO1, kColP1, v_tile(va), false);
+                    ok = wait_bar(c, V_CONV + 1, par) && wait_bar(c, P_CONV + 2, par);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    issue_ts(kColO1, kColP2, v_tile(vb), true);
                     ptx::mma_commit(&c.bars[P_FREE + 2]);
-                    ptx::mma_commit(&c.bars[O_FULL + 1]);
                 }
-                ptx::mma_commit(&c.bars[PV_DONE]);
-                // dS = K^T (d_k ⊙ V)
-                ok = wait_bar(c, VD_READY, par) && (NSUB == 2 || wait_bar(c, DS_FREE, fpar));
+                // dS = (K ⊙ d_k)^T V (for B = 128 the previous dS must have been read first)
+                ok = wait_bar(c, KD_READY, par) && (NSUB == 2 || wait_bar(c, DS_FREE, fpar));
                 if (!ok) break;
                 ptx::tc_fence_after();
                 issue_ds(qk_tile(sm.k0), v_tile(va), false);
                 if (NSUB == 2) issue_ds(qk_tile(sm.k1), v_tile(vb), true);
+                // O += Qd S_{t-1}
+                ok = wait_bar(c, S_READY, par);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                issue_ts(kColO0, kColP0 + 64, s_tile, true);
+                if (NSUB == 2) issue_ts(kColO1, kColP1 + 64, s_tile, true);
+                ptx::mma_commit(&c.bars[P_FREE + 0]);
+                ptx::mma_commit(&c.bars[O_FULL + 0]);
+                if (NSUB == 2) {
+                    ptx::mma_commit(&c.bars[P_FREE + 1]);
+                    ptx::mma_commit(&c.bars[O_FULL + 1]);
+                }
+                // dS is ready and S_{t-1} is no longer read: the state may move on
                 ptx::mma_commit(&c.bars[DS_FULL]);
                 ptx::mma_commit(&c.bars[EMPTY_QK + sm.k0]);
                 ptx::mma_commit(&c.bars[EMPTY_V + va % kVSlots]);
@@ -341,9 +355,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             volatile int never = 0;
             ptx::mbar_wait(&c.bars[DRAIN], 0, &never);
         }
-    } else if (warp >= 4 && warp < 8) {
-        // ------------------------------------------------------------ warpgroup 1: P conversion
-        const int r = threadIdx.x - 128;
+    } else if (warp >= 4 && warp < 12) {
+        // ------------------------------------------------------------ P conversion (256 threads)
+        // thread (w, r): TMEM lane r = row of the sub-tile, column half w of the P tile
+        const int cr = threadIdx.x - 128;
+        const int w = cr >> 7, r = cr & 127;
+        const bool leader = cr == 0;
         const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
         const float step = ptx::ex2(-sl2);  // e^{-s}
         uint32_t qk_par = 0;
@@ -351,29 +368,34 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         sm.init();
         for (int t = 0; t < nblk; ++t) {
             const uint32_t par = t & 1;
-            for (int tile = 0; tile < 2 * NSUB - 1; ++tile) {
+            for (int tile = 0; tile <= kLastTile; ++tile) {
                 // tile 0: P_aa (rows a, keys a, Qd_a); 1: P_ba (rows b, keys a, Qd_b); 2: P_bb
-                const uint32_t col = tile == 0 ? kColP0 : (tile == 1 ? kColP1 : kColP2);
+                const uint32_t col = p_col(tile);
                 const int i = (tile == 0 ? 0 : kRows) + r;
-                const int j0 = tile == 2 ? kRows : 0;
-                if (!wg_wait(c, P_FULL + tile, par, r, 1)) goto wg1_done;
+                const int j0 = (tile == 2 ? kRows : 0) + 64 * w;
+                if (!group_wait(c, P_FULL + tile, par, leader, kBarConv, 256)) goto conv_done;
                 ptx::tc_fence_after();
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t v[32], out[16];
-                    ptx::tmem_ld32(c.tmem + lane_off + col + 32 * ch, v);
-                    ptx::tmem_ld_wait();
+                uint32_t va[32], vb[32];
+                ptx::tmem_ld32(c.tmem + lane_off + col + 64 * w, va);
+                ptx::tmem_ld32(c.tmem + lane_off + col + 64 * w + 32, vb);
+                ptx::tmem_ld_wait();
+                // both column halves are in registers before anything is written back
+                ptx::named_bar_sync(kBarConv, 256);
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    const uint32_t *v = hb == 0 ? va : vb;
+                    uint32_t out[16];
 #pragma unroll
                     for (int g = 0; g < 2; ++g) {
-                        const int jb = j0 + 32 * ch + 16 * g;
+                        const int jb = j0 + 32 * hb + 16 * g;
                         const int dlast = i - (jb + 15);
                         float p[16];
                         if (dlast >= 0) {
-                            float w = ptx::ex2(-sl2 * (float)dlast);
+                            float wgt = ptx::ex2(-sl2 * (float)dlast);
 #pragma unroll
                             for (int u = 15; u >= 0; --u) {
-                                p[u] = __uint_as_float(v[16 * g + u]) * w;
-                                w *= step;
+                                p[u] = __uint_as_float(v[16 * g + u]) * wgt;
+                                wgt *= step;
                             }
                         } else {
 #pragma unroll
@@ -383,86 +405,52 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             }
                         }
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) out[8 * g + u] = ptx::pack_bf16(p[2 * u], p[2 * u + 1]);
+                        for (int u = 0; u < 8; ++u) out[8 * g + u] = ptx::pack_f16(p[2 * u], p[2 * u + 1]);
                     }
                     __syncwarp();
-                    ptx::tmem_st16(c.tmem + lane_off + col + 16 * ch, out);
+                    ptx::tmem_st16(c.tmem + lane_off + col + 32 * w + 16 * hb, out);
                 }
                 if (tile < 2) {
-                    // Qd = Q ⊙ d_q for this row, from the swizzled Q sub-tile
+                    // Qd = Q ⊙ d_q for dims [64w, 64w+64) of this row, from the swizzled Q sub-tile
                     const int qslot = tile == 0 ? sm.q0 : sm.q1;
-                    if (!wg_wait(c, FULL_QK + qslot, (qk_par >> qslot) & 1u, r, 1)) goto wg1_done;
+                    if (!group_wait(c, FULL_QK + qslot, (qk_par >> qslot) & 1u, leader, kBarConv, 256))
+                        goto conv_done;
                     const float dq = ptx::ex2(-sl2 * (float)(i + 1));
-                    const uint8_t *qrow = c.smem + kOffQK + qslot * kQKSlotBytes + r * 128;
+                    const uint8_t *qrow = c.smem + kOffQK + qslot * kQKSlotBytes + w * kBoxBytes + r * 128;
 #pragma unroll
-                    for (int hb = 0; hb < 4; ++hb) {  // 4 x 16 output words = 2 boxes x 8 chunks
+                    for (int hb = 0; hb < 2; ++hb) {
                         uint32_t out[16];
 #pragma unroll
                         for (int cc = 0; cc < 4; ++cc) {
-                            const int chunk = (hb & 1) * 4 + cc;
-                            const uint8_t *src = qrow + (hb >> 1) * kBoxBytes + ((chunk ^ (r & 7)) << 4);
-                            const uint4 w = *reinterpret_cast<const uint4 *>(src);
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                out[4 * cc + e] = ptx::pack_bf16(ptx::bf16_lo(ws[e]) * dq, ptx::bf16_hi(ws[e]) * dq);
+                            const int chunk = 4 * hb + cc;
+                            const uint4 q4 = *reinterpret_cast<const uint4 *>(qrow + ((chunk ^ (r & 7)) << 4));
+                            out[4 * cc + 0] = bf16x2_to_f16x2(q4.x, dq);
+                            out[4 * cc + 1] = bf16x2_to_f16x2(q4.y, dq);
+                            out[4 * cc + 2] = bf16x2_to_f16x2(q4.z, dq);
+                            out[4 * cc + 3] = bf16x2_to_f16x2(q4.w, dq);
                         }
-                        ptx::tmem_st16(c.tmem + lane_off + col + 64 + 16 * hb, out);
+                        __syncwarp();
+                        ptx::tmem_st16(c.tmem + lane_off + col + 64 + 32 * w + 16 * hb, out);
                     }
                 }
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
-                ptx::named_bar_sync(1, 128);
-                if (r == 0) {
+                ptx::named_bar_sync(kBarConv, 256);
+                if (leader) {
                     ptx::mbar_arrive(&c.bars[P_CONV + tile]);
-                    // Q_a is done after P_aa; Q_b after P_bb (or after P_aa when B = 128)
+                    // Q_a is done after P_aa; Q_b after P_bb
                     if (tile == 0) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q0]);
-                    if (tile == 2) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q1]);
+                    if (NSUB == 2 && tile == 2) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q1]);
                 }
             }
             qk_par ^= sm.used_mask();
             sm.advance();
         }
-    wg1_done:;
-    } else if (warp >= 8 && warp < 12) {
-        // ------------------------------------------------------------ warpgroup 2: epilogue
-        const int r = threadIdx.x - 256;
-        const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-        for (int t = 0; t < nblk; ++t) {
-            const uint32_t par = t & 1;
-            for (int sub = 0; sub < NSUB; ++sub) {
-                if (!wg_wait(c, O_FULL + sub, par, r, 2)) goto wg2_done;
-                ptx::tc_fence_after();
-                uint32_t a[32], b[32];
-                const uint32_t col = sub == 0 ? kColO0 : kColO1;
-                ptx::tmem_ld32(c.tmem + lane_off + col, a);
-                ptx::tmem_ld32(c.tmem + lane_off + col + 32, b);
-                ptx::tmem_ld_wait();
-                ptx::tc_fence_before();
-                ptx::named_bar_sync(2, 128);
-                if (r == 0) ptx::mbar_arrive(&c.bars[O_FREE + sub]);
-                const int row = t * B + sub * kRows + r;
-                if (row < seq) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)bh * seq + row) * kDim + 64 * half);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(ptx::pack_bf16(__uint_as_float(a[8 * q + 0]), __uint_as_float(a[8 * q + 1])),
-                                            ptx::pack_bf16(__uint_as_float(a[8 * q + 2]), __uint_as_float(a[8 * q + 3])),
-                                            ptx::pack_bf16(__uint_as_float(a[8 * q + 4]), __uint_as_float(a[8 * q + 5])),
-                                            ptx::pack_bf16(__uint_as_float(a[8 * q + 6]), __uint_as_float(a[8 * q + 7])));
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[4 + q] = make_uint4(ptx::pack_bf16(__uint_as_float(b[8 * q + 0]), __uint_as_float(b[8 * q + 1])),
-                                                ptx::pack_bf16(__uint_as_float(b[8 * q + 2]), __uint_as_float(b[8 * q + 3])),
-                                                ptx::pack_bf16(__uint_as_float(b[8 * q + 4]), __uint_as_float(b[8 * q + 5])),
-                                                ptx::pack_bf16(__uint_as_float(b[8 * q + 6]), __uint_as_float(b[8 * q + 7])));
-                }
-            }
-        }
-    wg2_done:;
+    conv_done:;
     } else if (warp >= 12) {
-        // ------------------------------------------------------------ warpgroup 3: state carry
-        const int r = threadIdx.x - 384;  // key-dimension row of S owned by this thread
+        // ------------------------------------------------------------ warpgroup 3
+        const int r = threadIdx.x - 384;  // row of V / K sub-tiles, key-dim row of S, output row
+        const bool leader = r == 0;
         const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
         float S[64];
         const size_t sbase = (size_t)bh * kDim * kDim + (size_t)r * kDim + 64 * half;
@@ -480,59 +468,114 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         auto write_state_operand = [&]() {
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch) {
-                uint4 w;
-                w.x = ptx::pack_bf16(S[8 * ch + 0], S[8 * ch + 1]);
-                w.y = ptx::pack_bf16(S[8 * ch + 2], S[8 * ch + 3]);
-                w.z = ptx::pack_bf16(S[8 * ch + 4], S[8 * ch + 5]);
-                w.w = ptx::pack_bf16(S[8 * ch + 6], S[8 * ch + 7]);
-                *reinterpret_cast<uint4 *>(srow + ((ch ^ (r & 7)) << 4)) = w;
+                uint4 wv;
+                wv.x = ptx::pack_f16(S[8 * ch + 0], S[8 * ch + 1]);
+                wv.y = ptx::pack_f16(S[8 * ch + 2], S[8 * ch + 3]);
+                wv.z = ptx::pack_f16(S[8 * ch + 4], S[8 * ch + 5]);
+                wv.w = ptx::pack_f16(S[8 * ch + 6], S[8 * ch + 7]);
+                *reinterpret_cast<uint4 *>(srow + ((ch ^ (r & 7)) << 4)) = wv;
             }
             ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(3, 128);
-            if (r == 0) ptx::mbar_arrive(&c.bars[S_READY]);
+            ptx::named_bar_sync(kBarWG3, 128);
+            if (leader) ptx::mbar_arrive(&c.bars[S_READY]);
         };
         write_state_operand();
+        uint32_t qk_par = 0;
+        SlotMap<NSUB> sm;
+        sm.init();
         int vtile = 0;
         for (int t = 0; t < nblk; ++t) {
             const uint32_t par = t & 1;
             const int m = min(B, seq - t * B);
-            if (!wg_wait(c, PV_DONE, par, r, 3)) goto wg3_done;
+            // V sub-tiles: bf16 -> fp16 in place
             for (int sub = 0; sub < NSUB; ++sub) {
                 const int n = vtile + sub;
-                if (!wg_wait(c, FULL_V + n % kVSlots, (uint32_t)(n / kVSlots) & 1u, r, 3)) goto wg3_done;
-                const int j = sub * kRows + r;
-                const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
+                if (!group_wait(c, FULL_V + n % kVSlots, (uint32_t)(n / kVSlots) & 1u, leader, kBarWG3, 128))
+                    goto wg3_done;
                 uint8_t *vrow = c.smem + kOffV + (n % kVSlots) * kVSlotBytes + r * 128;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    uint4 *p = reinterpret_cast<uint4 *>(vrow + (ch << 4));
-                    uint4 w = *p;
-                    w.x = ptx::pack_bf16(ptx::bf16_lo(w.x) * dk, ptx::bf16_hi(w.x) * dk);
-                    w.y = ptx::pack_bf16(ptx::bf16_lo(w.y) * dk, ptx::bf16_hi(w.y) * dk);
-                    w.z = ptx::pack_bf16(ptx::bf16_lo(w.z) * dk, ptx::bf16_hi(w.z) * dk);
-                    w.w = ptx::pack_bf16(ptx::bf16_lo(w.w) * dk, ptx::bf16_hi(w.w) * dk);
-                    *p = w;
+                    uint4 *pv = reinterpret_cast<uint4 *>(vrow + (ch << 4));
+                    uint4 x = *pv;
+                    x.x = bf16x2_to_f16x2(x.x, 1.f); x.y = bf16x2_to_f16x2(x.y, 1.f);
+                    x.z = bf16x2_to_f16x2(x.z, 1.f); x.w = bf16x2_to_f16x2(x.w, 1.f);
+                    *pv = x;
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_sync(kBarWG3, 128);
+                if (leader) ptx::mbar_arrive(&c.bars[V_CONV + sub]);
+            }
+            // K sub-tiles: bf16 -> fp16 K ⊙ d_k in place, once the block's Q K^T is done
+            if (!group_wait(c, P_FULL + kLastTile, par, leader, kBarWG3, 128)) goto wg3_done;
+            for (int sub = 0; sub < NSUB; ++sub) {
+                const int kslot = sub == 0 ? sm.k0 : sm.k1;
+                // full-barrier wait: makes the TMA bytes visible to these threads
+                if (!group_wait(c, FULL_QK + kslot, (qk_par >> kslot) & 1u, leader, kBarWG3, 128)) goto wg3_done;
+                const int j = sub * kRows + r;
+                const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
+                uint8_t *krow = c.smem + kOffQK + kslot * kQKSlotBytes + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < 16; ++ch) {
+                    uint4 *pk = reinterpret_cast<uint4 *>(krow + (ch >> 3) * kBoxBytes + ((ch & 7) << 4));
+                    uint4 x = *pk;
+                    x.x = bf16x2_to_f16x2(x.x, dk); x.y = bf16x2_to_f16x2(x.y, dk);
+                    x.z = bf16x2_to_f16x2(x.z, dk); x.w = bf16x2_to_f16x2(x.w, dk);
+                    *pk = x;
                 }
             }
             ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(3, 128);
-            if (r == 0) ptx::mbar_arrive(&c.bars[VD_READY]);
+            ptx::named_bar_sync(kBarWG3, 128);
+            if (leader) ptx::mbar_arrive(&c.bars[KD_READY]);
 
-            if (!wg_wait(c, DS_FULL, par, r, 3)) goto wg3_done;
+            // state: S_t = e^{-s m} S_{t-1} + dS
+            if (!group_wait(c, DS_FULL, par, leader, kBarWG3, 128)) goto wg3_done;
             ptx::tc_fence_after();
-            const float dblock = ptx::ex2(-sl2 * (float)m);
+            {
+                const float dblock = ptx::ex2(-sl2 * (float)m);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t d[32];
-                ptx::tmem_ld32(c.tmem + lane_off + kColDS + 32 * hh, d);
-                ptx::tmem_ld_wait();
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t d[32];
+                    ptx::tmem_ld32(c.tmem + lane_off + kColDS + 32 * hh, d);
+                    ptx::tmem_ld_wait();
 #pragma unroll
-                for (int q = 0; q < 32; ++q) S[32 * hh + q] = fmaf(dblock, S[32 * hh + q], __uint_as_float(d[q]));
+                    for (int q = 0; q < 32; ++q) S[32 * hh + q] = fmaf(dblock, S[32 * hh + q], __uint_as_float(d[q]));
+                }
             }
             ptx::tc_fence_before();
-            ptx::named_bar_sync(3, 128);
-            if (r == 0) ptx::mbar_arrive(&c.bars[DS_FREE]);
+            ptx::named_bar_sync(kBarWG3, 128);
+            if (leader) ptx::mbar_arrive(&c.bars[DS_FREE]);
             write_state_operand();
+
+            // outputs of this block: O (TMEM, fp32) -> bf16 -> global, 32 columns at a time
+            for (int sub = 0; sub < NSUB; ++sub) {
+                if (!group_wait(c, O_FULL + sub, par, leader, kBarWG3, 128)) goto wg3_done;
+                ptx::tc_fence_after();
+                const uint32_t col = sub == 0 ? kColO0 : kColO1;
+                const int row = t * B + sub * kRows + r;
+                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)bh * seq + row) * kDim + 64 * half);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t a[32];
+                    ptx::tmem_ld32(c.tmem + lane_off + col + 32 * hh, a);
+                    ptx::tmem_ld_wait();
+                    if (hh == 1) {
+                        ptx::tc_fence_before();
+                        ptx::named_bar_sync(kBarWG3, 128);
+                        if (leader) ptx::mbar_arrive(&c.bars[O_FREE + sub]);
+                    }
+                    if (row < seq) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[4 * hh + q] = make_uint4(
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 0]), __uint_as_float(a[8 * q + 1])),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 2]), __uint_as_float(a[8 * q + 3])),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 4]), __uint_as_float(a[8 * q + 5])),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 6]), __uint_as_float(a[8 * q + 7])));
+                    }
+                }
+            }
+            qk_par ^= sm.used_mask();
+            sm.advance();
             vtile += NSUB;
         }
         if (state_out) {
