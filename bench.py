@@ -311,10 +311,10 @@ def run_ours(args):
 
     # decode: 1000 consecutive single-token steps over fp32 states
     dw = inputs.WORKLOADS[DECODE_WORKLOAD]
-    dec = run_decode(dw, dev, stream, peaks, args)
+    dec = run_decode(dw, dev, stream, peaks, args) if args.decode_steps > 0 else None
 
     # end to end: host buffers, copies inside the timed region
-    e2e = run_e2e(w, dev, stream, inp, variant, args, world)
+    e2e = run_e2e(w, dev, stream, inp, variant, args, world) if args.e2e_steps > 0 else None
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

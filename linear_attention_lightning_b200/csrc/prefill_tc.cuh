@@ -24,17 +24,18 @@
 //
 // Per block:
 //   QK    (SS MMA bf16, M128 N128 K128)  P tiles -> TMEM (fp32)
-//   conv  (warps 4-11)                   P ⊙ D -> fp16 back into TMEM, and
+//   conv  (warps 4-11, one tile each)    P ⊙ D -> fp16 back into TMEM, and
 //                                        Qd = Q ⊙ d_q (fp16) next to it
 //   PV    (TS MMA f16, M128 N64)         O  = P V          (A = P from TMEM)
 //   dS    (SS MMA f16, M128 N64 K256)    dS = (K ⊙ d_k)^T V
 //   QS    (TS MMA f16, M128 N64)         O += Qd S_{t-1}   (B = fp16 S in smem)
-//   warpgroup 3: converts V to fp16 and K to fp16 K ⊙ d_k in place, carries
+//   K ⊙ d_k: the P_ba warpgroup converts K to fp16 K ⊙ d_k in place.
+//   warpgroup 3: converts V to fp16 in place, carries
 //                S = e^{-s m} S + dS in fp32 registers (fp16 copy -> smem),
 //                and writes O (TMEM -> bf16 -> global).
 // Warp roles: warp 0 issues TMA, warp 1 issues MMAs, warp 2 owns TMEM,
-// warps 4-11 convert P (each warpgroup one half of the columns), warps 12-15
-// are warpgroup 3. All hand-offs are mbarriers; every wait is bounded.
+// warps 4-7 and 8-11 convert P tiles (P_aa and P_bb / P_ba, then K ⊙ d_k),
+// warps 12-15 are warpgroup 3. All hand-offs are mbarriers; every wait is bounded.
 //
 // Shared memory (1024-aligned, 128B-swizzled tiles as TMA writes them):
 //   5 x 32 KB Q/K sub-tiles (128 rows x 128 dims), 3 x 16 KB V sub-tiles
@@ -83,8 +84,8 @@ constexpr int FULL_QK = 0, EMPTY_QK = 5, FULL_V = 10, EMPTY_V = 13, P_FULL = 16,
               P_FREE = 22, O_FULL = 25, O_FREE = 27, V_CONV = 29, KD_READY = 31, DS_FULL = 32,
               DS_FREE = 33, S_READY = 34, DRAIN = 35;
 
-// named barriers: 1 = the 256 conversion threads, 2 = warpgroup 3
-constexpr int kBarConv = 1, kBarWG3 = 2;
+// named barriers: 1 / 3 = the two conversion warpgroups, 2 = warpgroup 3
+constexpr int kBarConv = 1, kBarWG3 = 2, kBarConv2 = 3;
 
 // Instruction descriptor, kind::f16, fp32 accumulate, M x N; fmt 0 = f16, 1 = bf16.
 __host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool a_mn_major, bool b_mn_major) {
@@ -259,26 +260,41 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             SlotMap<NSUB> sm;
             sm.init();
             const uint32_t tm = c.tmem;
-            const uint32_t s_tile = c.sbase + kOffS;
-            auto qk_tile = [&](int slot) { return c.sbase + kOffQK + (uint32_t)slot * kQKSlotBytes; };
-            auto v_tile = [&](int n) { return c.sbase + kOffV + (uint32_t)(n % kVSlots) * kVSlotBytes; };
+            // Descriptors are built once; per MMA only the start-address field
+            // moves (a plain add on the low bits: shared addresses stay < 2^18).
+            const uint64_t qk_kmaj = sdesc(c.sbase + kOffQK, 16u, 1024u);
+            const uint64_t qk_mnmaj = sdesc(c.sbase + kOffQK, kBoxBytes, 1024u);
+            const uint64_t v_mnmaj = sdesc(c.sbase + kOffV, kBoxBytes, 1024u);
+            const uint64_t s_mnmaj = sdesc(c.sbase + kOffS, kBoxBytes, 1024u);
+            auto qk_off = [](int slot) { return (uint64_t)((uint32_t)slot * (kQKSlotBytes >> 4)); };
+            auto v_off = [](int n) { return (uint64_t)((uint32_t)(n % kVSlots) * (kVSlotBytes >> 4)); };
             auto wait_qk = [&](int slot) -> bool {
                 const bool r = wait_bar(c, FULL_QK + slot, (qk_par >> slot) & 1u);
                 qk_par ^= 1u << slot;
                 return r;
             };
             auto issue_qk = [&](uint32_t dcol, int qslot, int kslot) {
-                for (int k = 0; k < 8; ++k)
-                    ptx::mma_ss(tm + dcol, desc_kmajor(qk_tile(qslot), k), desc_kmajor(qk_tile(kslot), k),
-                                kIdescQK, k > 0);
+                const uint64_t a0 = qk_kmaj + qk_off(qslot), b0 = qk_kmaj + qk_off(kslot);
+                const uint32_t d = tm + dcol;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
+                    ptx::mma_ss(d, a0 + koff, b0 + koff, kIdescQK, k > 0);
+                }
             };
-            auto issue_ts = [&](uint32_t dcol, uint32_t acol, uint32_t bt, bool acc) {
+            auto issue_ts = [&](uint32_t dcol, uint32_t acol, uint64_t b0, bool acc) {
+                const uint32_t d = tm + dcol, a = tm + acol;
+#pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    ptx::mma_ts(tm + dcol, tm + acol + 8u * k, desc_mnmajor(bt, k), kIdescPV, acc || k > 0);
+                    ptx::mma_ts(d, a + 8u * k, b0 + (uint64_t)(k * (2048 >> 4)), kIdescPV, acc || k > 0);
             };
-            auto issue_ds = [&](uint32_t kt, uint32_t vt, bool acc) {
+            auto issue_ds = [&](int kslot, int vn, bool acc) {
+                const uint64_t a0 = qk_mnmaj + qk_off(kslot), b0 = v_mnmaj + v_off(vn);
+                const uint32_t d = tm + kColDS;
+#pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    ptx::mma_ss(tm + kColDS, desc_mnmajor(kt, k), desc_mnmajor(vt, k), kIdescDS, acc || k > 0);
+                    ptx::mma_ss(d, a0 + (uint64_t)(k * (2048 >> 4)), b0 + (uint64_t)(k * (2048 >> 4)), kIdescDS,
+                                acc || k > 0);
             };
             bool ok = true;
             for (int t = 0; t < nblk && ok; ++t) {
@@ -308,31 +324,31 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 ok = wait_bar(c, V_CONV + 0, par) && wait_bar(c, P_CONV + 0, par) && wait_bar(c, O_FREE + 0, fpar);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                issue_ts(kColO0, kColP0, v_tile(va), false);
+                issue_ts(kColO0, kColP0, v_mnmaj + v_off(va), false);
                 if (NSUB == 2) {
                     // O_b = P_ba V_a + P_bb V_b
                     ok = wait_bar(c, P_CONV + 1, par) && wait_bar(c, O_FREE + 1, fpar);
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    issue_ts(kColO1, kColP1, v_tile(va), false);
+                    issue_ts(kColO1, kColP1, v_mnmaj + v_off(va), false);
                     ok = wait_bar(c, V_CONV + 1, par) && wait_bar(c, P_CONV + 2, par);
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    issue_ts(kColO1, kColP2, v_tile(vb), true);
+                    issue_ts(kColO1, kColP2, v_mnmaj + v_off(vb), true);
                     ptx::mma_commit(&c.bars[P_FREE + 2]);
                 }
                 // dS = (K ⊙ d_k)^T V (for B = 128 the previous dS must have been read first)
                 ok = wait_bar(c, KD_READY, par) && (NSUB == 2 || wait_bar(c, DS_FREE, fpar));
                 if (!ok) break;
                 ptx::tc_fence_after();
-                issue_ds(qk_tile(sm.k0), v_tile(va), false);
-                if (NSUB == 2) issue_ds(qk_tile(sm.k1), v_tile(vb), true);
+                issue_ds(sm.k0, va, false);
+                if (NSUB == 2) issue_ds(sm.k1, vb, true);
                 // O += Qd S_{t-1}
                 ok = wait_bar(c, S_READY, par);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                issue_ts(kColO0, kColP0 + 64, s_tile, true);
-                if (NSUB == 2) issue_ts(kColO1, kColP1 + 64, s_tile, true);
+                issue_ts(kColO0, kColP0 + 64, s_mnmaj, true);
+                if (NSUB == 2) issue_ts(kColO1, kColP1 + 64, s_mnmaj, true);
                 ptx::mma_commit(&c.bars[P_FREE + 0]);
                 ptx::mma_commit(&c.bars[O_FULL + 0]);
                 if (NSUB == 2) {
@@ -356,92 +372,136 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             ptx::mbar_wait(&c.bars[DRAIN], 0, &never);
         }
     } else if (warp >= 4 && warp < 12) {
-        // ------------------------------------------------------------ P conversion (256 threads)
-        // thread (w, r): TMEM lane r = row of the sub-tile, column half w of the P tile
-        const int cr = threadIdx.x - 128;
-        const int w = cr >> 7, r = cr & 127;
-        const bool leader = cr == 0;
+        // ------------------------------------------------------------ P conversion
+        // Two warpgroups, each converting whole P tiles: group 0 takes P_aa (and
+        // P_bb), group 1 takes P_ba. Thread r owns TMEM lane r = row r of the tile.
+        const int grp = (warp - 4) >> 2;
+        const int r = threadIdx.x - 128 - 128 * grp;
+        const bool leader = r == 0;
+        const int bar_id = grp == 0 ? kBarConv : kBarConv2;
         const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+        // tab[u] = e^{-s(15-u)}: decay inside a group of 16 keys, relative to its last key
         const float step = ptx::ex2(-sl2);  // e^{-s}
+        float tab[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) tab[u] = ptx::ex2(-sl2 * (float)(15 - u));
         uint32_t qk_par = 0;
         SlotMap<NSUB> sm;
         sm.init();
         for (int t = 0; t < nblk; ++t) {
             const uint32_t par = t & 1;
-            for (int tile = 0; tile <= kLastTile; ++tile) {
+            for (int tile = grp; tile <= kLastTile; tile += 2) {
                 // tile 0: P_aa (rows a, keys a, Qd_a); 1: P_ba (rows b, keys a, Qd_b); 2: P_bb
                 const uint32_t col = p_col(tile);
                 const int i = (tile == 0 ? 0 : kRows) + r;
-                const int j0 = (tile == 2 ? kRows : 0) + 64 * w;
-                if (!group_wait(c, P_FULL + tile, par, leader, kBarConv, 256)) goto conv_done;
+                const int j0 = tile == 2 ? kRows : 0;
+                if (!group_wait(c, P_FULL + tile, par, leader, bar_id, 128)) goto conv_done;
                 ptx::tc_fence_after();
-                uint32_t va[32], vb[32];
-                ptx::tmem_ld32(c.tmem + lane_off + col + 64 * w, va);
-                ptx::tmem_ld32(c.tmem + lane_off + col + 64 * w + 32, vb);
-                ptx::tmem_ld_wait();
-                // both column halves are in registers before anything is written back
-                ptx::named_bar_sync(kBarConv, 256);
-#pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    const uint32_t *v = hb == 0 ? va : vb;
-                    uint32_t out[16];
-#pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        const int jb = j0 + 32 * hb + 16 * g;
-                        const int dlast = i - (jb + 15);
-                        float p[16];
-                        if (dlast >= 0) {
-                            float wgt = ptx::ex2(-sl2 * (float)dlast);
-#pragma unroll
-                            for (int u = 15; u >= 0; --u) {
-                                p[u] = __uint_as_float(v[16 * g + u]) * wgt;
-                                wgt *= step;
-                            }
-                        } else {
-#pragma unroll
-                            for (int u = 0; u < 16; ++u) {
-                                const int dd = i - (jb + u);
-                                p[u] = dd >= 0 ? __uint_as_float(v[16 * g + u]) * ptx::ex2(-sl2 * (float)dd) : 0.f;
-                            }
-                        }
-#pragma unroll
-                        for (int u = 0; u < 8; ++u) out[8 * g + u] = ptx::pack_f16(p[2 * u], p[2 * u + 1]);
-                    }
-                    __syncwarp();
-                    ptx::tmem_st16(c.tmem + lane_off + col + 32 * w + 16 * hb, out);
-                }
-                if (tile < 2) {
-                    // Qd = Q ⊙ d_q for dims [64w, 64w+64) of this row, from the swizzled Q sub-tile
-                    const int qslot = tile == 0 ? sm.q0 : sm.q1;
-                    if (!group_wait(c, FULL_QK + qslot, (qk_par >> qslot) & 1u, leader, kBarConv, 256))
-                        goto conv_done;
-                    const float dq = ptx::ex2(-sl2 * (float)(i + 1));
-                    const uint8_t *qrow = c.smem + kOffQK + qslot * kQKSlotBytes + w * kBoxBytes + r * 128;
+#pragma unroll 1
+                for (int pass = 0; pass < 2; ++pass) {
+                    // fp32 columns [64 pass, 64 pass + 64) -> fp16 pairs in [32 pass, 32 pass + 32);
+                    // the destination was read by this same thread in an earlier pass
+                    uint32_t va[32], vb[32];
+                    ptx::tmem_ld32(c.tmem + lane_off + col + 64 * pass, va);
+                    ptx::tmem_ld32(c.tmem + lane_off + col + 64 * pass + 32, vb);
+                    ptx::tmem_ld_wait();
 #pragma unroll
                     for (int hb = 0; hb < 2; ++hb) {
                         uint32_t out[16];
 #pragma unroll
+                        for (int g = 0; g < 2; ++g) {
+                            const uint32_t *v = (hb == 0 ? va : vb) + 16 * g;
+                            const int jb = j0 + 64 * pass + 32 * hb + 16 * g;
+                            const int dlast = i - (jb + 15);
+                            float p[16];
+                            if (dlast >= 0) {
+                                const float wb = ptx::ex2(-sl2 * (float)dlast);
+#pragma unroll
+                                for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[u]) * tab[u]) * wb;
+                            } else if (i < jb) {
+                                // every key of the group is after row i: masked
+#pragma unroll
+                                for (int u = 0; u < 16; ++u) p[u] = 0.f;
+                            } else {
+                                // the group holds the diagonal key jb + d0: walk down from it
+                                const int d0 = i - jb;
+                                float w = 1.f;
+#pragma unroll
+                                for (int u = 15; u >= 0; --u) {
+                                    const bool live = u <= d0;
+                                    p[u] = live ? __uint_as_float(v[u]) * w : 0.f;
+                                    w = live ? w * step : w;
+                                }
+                            }
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) out[8 * g + u] = ptx::pack_f16(p[2 * u], p[2 * u + 1]);
+                        }
+                        __syncwarp();
+                        ptx::tmem_st16(c.tmem + lane_off + col + 32 * pass + 16 * hb, out);
+                    }
+                }
+                if (tile < 2) {
+                    // Qd = Q ⊙ d_q for this row, from the swizzled Q sub-tile, into columns [64, 128)
+                    const int qslot = tile == 0 ? sm.q0 : sm.q1;
+                    if (!group_wait(c, FULL_QK + qslot, (qk_par >> qslot) & 1u, leader, bar_id, 128))
+                        goto conv_done;
+                    const float dq = ptx::ex2(-sl2 * (float)(i + 1));
+                    const uint8_t *qrow = c.smem + kOffQK + qslot * kQKSlotBytes + r * 128;
+#pragma unroll
+                    for (int hb = 0; hb < 4; ++hb) {
+                        uint32_t out[16];
+#pragma unroll
                         for (int cc = 0; cc < 4; ++cc) {
-                            const int chunk = 4 * hb + cc;
-                            const uint4 q4 = *reinterpret_cast<const uint4 *>(qrow + ((chunk ^ (r & 7)) << 4));
+                            const int chunk = 4 * (hb & 1) + cc;
+                            const uint4 q4 = *reinterpret_cast<const uint4 *>(
+                                qrow + (hb >> 1) * kBoxBytes + ((chunk ^ (r & 7)) << 4));
                             out[4 * cc + 0] = bf16x2_to_f16x2(q4.x, dq);
                             out[4 * cc + 1] = bf16x2_to_f16x2(q4.y, dq);
                             out[4 * cc + 2] = bf16x2_to_f16x2(q4.z, dq);
                             out[4 * cc + 3] = bf16x2_to_f16x2(q4.w, dq);
                         }
                         __syncwarp();
-                        ptx::tmem_st16(c.tmem + lane_off + col + 64 + 32 * w + 16 * hb, out);
+                        ptx::tmem_st16(c.tmem + lane_off + col + 64 + 16 * hb, out);
                     }
                 }
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
-                ptx::named_bar_sync(kBarConv, 256);
-                if (leader) {
-                    ptx::mbar_arrive(&c.bars[P_CONV + tile]);
-                    // Q_a is done after P_aa; Q_b after P_bb
-                    if (tile == 0) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q0]);
-                    if (NSUB == 2 && tile == 2) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q1]);
+                ptx::named_bar_sync(bar_id, 128);
+                if (leader) ptx::mbar_arrive(&c.bars[P_CONV + tile]);
+                if (tile == 0 && leader) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q0]);  // Q_a done
+                if (tile == 2) {
+                    // Q_b is done once P_bb's Q K^T has run (it has: P_bb was full) and
+                    // the other group has built Qd_b
+                    if (!group_wait(c, P_CONV + 1, par, leader, bar_id, 128)) goto conv_done;
+                    if (leader) ptx::mbar_arrive(&c.bars[EMPTY_QK + sm.q1]);
                 }
+            }
+            if (grp == NSUB - 1) {
+                // K sub-tiles: bf16 -> fp16 K ⊙ d_k in place, once the block's Q K^T is done
+                const int m = min(B, seq - t * B);
+                if (!group_wait(c, P_FULL + kLastTile, par, leader, bar_id, 128)) goto conv_done;
+                for (int sub = 0; sub < NSUB; ++sub) {
+                    const int kslot = sub == 0 ? sm.k0 : sm.k1;
+                    // full-barrier wait: makes the TMA bytes visible to these threads
+                    if (!group_wait(c, FULL_QK + kslot, (qk_par >> kslot) & 1u, leader, bar_id, 128)) goto conv_done;
+                    const int j = sub * kRows + r;
+                    const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
+                    uint8_t *krow = c.smem + kOffQK + kslot * kQKSlotBytes + r * 128;
+                    uint4 x[16];
+#pragma unroll
+                    for (int ch = 0; ch < 16; ++ch)
+                        x[ch] = *reinterpret_cast<const uint4 *>(krow + (ch >> 3) * kBoxBytes + (((ch & 7) ^ (r & 7)) << 4));
+#pragma unroll
+                    for (int ch = 0; ch < 16; ++ch) {
+                        uint4 y;
+                        y.x = bf16x2_to_f16x2(x[ch].x, dk); y.y = bf16x2_to_f16x2(x[ch].y, dk);
+                        y.z = bf16x2_to_f16x2(x[ch].z, dk); y.w = bf16x2_to_f16x2(x[ch].w, dk);
+                        *reinterpret_cast<uint4 *>(krow + (ch >> 3) * kBoxBytes + (((ch & 7) ^ (r & 7)) << 4)) = y;
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_sync(bar_id, 128);
+                if (leader) ptx::mbar_arrive(&c.bars[KD_READY]);
             }
             qk_par ^= sm.used_mask();
             sm.advance();
@@ -495,7 +555,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 uint8_t *vrow = c.smem + kOffV + (n % kVSlots) * kVSlotBytes + r * 128;
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
-                    uint4 *pv = reinterpret_cast<uint4 *>(vrow + (ch << 4));
+                    // walk the row in its swizzled chunk order: the 32 rows of a warp
+                    // then hit 8 different bank groups instead of one
+                    uint4 *pv = reinterpret_cast<uint4 *>(vrow + ((ch ^ (r & 7)) << 4));
                     uint4 x = *pv;
                     x.x = bf16x2_to_f16x2(x.x, 1.f); x.y = bf16x2_to_f16x2(x.y, 1.f);
                     x.z = bf16x2_to_f16x2(x.z, 1.f); x.w = bf16x2_to_f16x2(x.w, 1.f);
@@ -505,28 +567,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 ptx::named_bar_sync(kBarWG3, 128);
                 if (leader) ptx::mbar_arrive(&c.bars[V_CONV + sub]);
             }
-            // K sub-tiles: bf16 -> fp16 K ⊙ d_k in place, once the block's Q K^T is done
-            if (!group_wait(c, P_FULL + kLastTile, par, leader, kBarWG3, 128)) goto wg3_done;
-            for (int sub = 0; sub < NSUB; ++sub) {
-                const int kslot = sub == 0 ? sm.k0 : sm.k1;
-                // full-barrier wait: makes the TMA bytes visible to these threads
-                if (!group_wait(c, FULL_QK + kslot, (qk_par >> kslot) & 1u, leader, kBarWG3, 128)) goto wg3_done;
-                const int j = sub * kRows + r;
-                const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
-                uint8_t *krow = c.smem + kOffQK + kslot * kQKSlotBytes + r * 128;
-#pragma unroll
-                for (int ch = 0; ch < 16; ++ch) {
-                    uint4 *pk = reinterpret_cast<uint4 *>(krow + (ch >> 3) * kBoxBytes + ((ch & 7) << 4));
-                    uint4 x = *pk;
-                    x.x = bf16x2_to_f16x2(x.x, dk); x.y = bf16x2_to_f16x2(x.y, dk);
-                    x.z = bf16x2_to_f16x2(x.z, dk); x.w = bf16x2_to_f16x2(x.w, dk);
-                    *pk = x;
-                }
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(kBarWG3, 128);
-            if (leader) ptx::mbar_arrive(&c.bars[KD_READY]);
-
             // state: S_t = e^{-s m} S_{t-1} + dS
             if (!group_wait(c, DS_FULL, par, leader, kBarWG3, 128)) goto wg3_done;
             ptx::tc_fence_after();
