@@ -77,6 +77,33 @@ def roofline(bound, achieved, peak, unit, traffic=None):
             "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic}
 
 
+def kernel_source_digest():
+    """Digest of the CUDA sources, to tell whether stored ncu counters still
+    describe the kernels being timed."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_lightning_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload, variant):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernels changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_digest") != kernel_source_digest():
+        return None
+    entry = t.get("launches", {}).get("%s/%s" % (workload, variant))
+    return None if entry is None else entry.get("dram_bytes_per_launch")
+
+
 def summarize_clocks(rows):
     """rows: list of dicts from nvidia-smi samples; returns the clocks object."""
     if not rows:
@@ -303,11 +330,7 @@ def run_ours(args):
     avg_launch_s = statistics.mean(per_launch_ms) / 1e3
     gbs = by / avg_launch_s / 1e9
     tflops = {kk: vv / avg_launch_s / 1e12 for kk, vv in fl.items()}
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            traffic = json.load(f).get("%s/%s" % (w.name, variant))
+    traffic = measured_traffic(w.name, variant)
 
     # decode: 1000 consecutive single-token steps over fp32 states
     dw = inputs.WORKLOADS[DECODE_WORKLOAD]

@@ -1,0 +1,102 @@
+"""Host-side logic of bench.py (no GPU): the algorithmic FLOP / byte counts
+the roofline divides by, the clock summary, the JSON contract's guards, and
+the max-over-ranks reduction on a 2-rank gloo group."""
+import json
+import multiprocessing as mp
+import os
+import socket
+
+import pytest
+
+import bench
+
+
+def test_prefill_work_matches_the_stated_figures():
+    # 4Bd + 4d^2 = 196,608 FLOPs per (token, head) at B=256, d=128
+    f = bench.prefill_flops(1, 1, 1, 128, 256)
+    assert f["formula"] == 196608
+    assert f["causal"] == 2 * 257 * 128 + 4 * 128 * 128
+    big = bench.prefill_flops(1, 64, 131072, 128, 256)
+    assert abs(big["formula"] - 1.649e12) / 1.649e12 < 1e-3
+    # q, k, v, o in bf16 + fp32 state out: 8.594 GB for the long-context case
+    by = bench.prefill_bytes(1, 64, 131072, 128, 2, state_in=False, state_out=True)
+    assert abs(by - 8.594e9) / 8.594e9 < 1e-3
+
+
+def test_decode_bytes():
+    # state read + written (2 * 4 * d^2) plus four bf16 vectors per (seq, head)
+    assert bench.decode_bytes(1, 1, 128) == 2 * 4 * 128 * 128 + 4 * 128 * 2
+    assert abs(bench.decode_bytes(64, 64, 128) - 541.1e6) / 541.1e6 < 1e-3
+
+
+def test_roofline_fraction():
+    r = bench.roofline("hbm", 3260.1, 6520.2, "GB/s", None)
+    assert r["frac"] == 0.5 and r["bound"] == "hbm" and r["traffic"] is None
+
+
+def test_clock_summary_flags_throttling():
+    rows = [{"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "power_w": 800.0, "hw_slowdown": "Not Active",
+             "hw_thermal_slowdown": "Not Active", "sw_thermal_slowdown": "Not Active",
+             "sw_power_cap": "Active"},
+            {"sm_mhz": 1800.0, "sm_max_mhz": 1965.0, "power_w": 900.0, "hw_slowdown": "Not Active",
+             "hw_thermal_slowdown": "Active", "sw_thermal_slowdown": "Not Active",
+             "sw_power_cap": "Not Active"},
+            {"sm_mhz": 300.0, "sm_max_mhz": 1965.0, "power_w": 90.0, "hw_slowdown": "Not Active",
+             "hw_thermal_slowdown": "Not Active", "sw_thermal_slowdown": "Not Active",
+             "sw_power_cap": "Not Active"}]
+    c = bench.summarize_clocks(rows)
+    assert c["sm_mhz"] == 1850.0            # idle sample excluded
+    assert c["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert bench.summarize_clocks([])["sm_mhz"] is None
+
+
+def test_warmup_floor():
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--warmup", "2"])
+    a = bench.parse_args([])
+    assert a.gpus == 1 and a.warmup >= 3 and a.impl == "ours"
+
+
+def test_stored_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    digest = bench.kernel_source_digest()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "traffic.json").write_text(json.dumps({
+        "kernel_source_digest": digest,
+        "launches": {"w/tcgen05": {"dram_bytes_per_launch": 123}}}))
+    csrc = os.path.join(bench.ROOT, "linear_attention_lightning_b200", "csrc")
+    pkg = tmp_path / "linear_attention_lightning_b200"
+    pkg.mkdir()
+    os.symlink(csrc, pkg / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("w", "tcgen05") == 123
+    (prof / "traffic.json").write_text(json.dumps({
+        "kernel_source_digest": "stale", "launches": {"w/tcgen05": {"dram_bytes_per_launch": 123}}}))
+    assert bench.measured_traffic("w", "tcgen05") is None
+
+
+def _rank_main(rank, port, q):
+    os.environ.update(RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    r, world, _ = bench.dist_setup(2)
+    bench.barrier(world)
+    got = bench.max_over_ranks(10.0 + r, world)
+    q.put((r, world, got))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_on_two_gloo_ranks():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert out == [(0, 2, 11.0), (1, 2, 11.0)]
