@@ -295,7 +295,8 @@ def run_ours(args):
     o = torch.empty_like(q)
     s_out = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32, device=dev)
     variant = la.prefill_variant(w.dtype, w.batch, w.heads, w.seq, w.dim, w.block)
-    vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05}[variant]
+    vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05,
+             "pair": abi.LA_VARIANT_TCGEN05_PAIR}[variant]
     dcode = abi.LA_DTYPE_BF16 if w.dtype == torch.bfloat16 else abi.LA_DTYPE_F32
 
     def step():

@@ -62,13 +62,16 @@ typedef enum la_dtype {
     LA_DTYPE_BF16 = 1
 } la_dtype;
 
-/* Kernel selection for lightning_prefill_ex. AUTO picks the tensor-core
- * kernel whenever it supports the request (bf16, dim 128, block 128 or 256)
- * and the CUDA-core kernel otherwise. */
+/* Kernel selection for lightning_prefill_ex. AUTO picks the CTA-pair kernel
+ * for bf16, dim 128, block 256; the single-CTA tensor-core kernel for bf16,
+ * dim 128, block 128; and the CUDA-core kernel otherwise. */
 typedef enum la_variant {
     LA_VARIANT_AUTO = 0,
-    LA_VARIANT_SIMT = 1,      /* CUDA-core kernel, fp32 arithmetic, any dtype    */
-    LA_VARIANT_TCGEN05 = 2    /* tcgen05/TMEM/TMA kernel, bf16, dim 128          */
+    LA_VARIANT_SIMT = 1,          /* CUDA-core kernel, fp32 arithmetic, any dtype          */
+    LA_VARIANT_TCGEN05 = 2,       /* tcgen05/TMEM/TMA, one CTA per (head, value half),
+                                     bf16, dim 128, block 128 or 256                      */
+    LA_VARIANT_TCGEN05_PAIR = 3   /* tcgen05 on a CTA pair (cta_group::2) per head,
+                                     bf16, dim 128, block 256                             */
 } la_variant;
 
 /* Version of this ABI; bumps on any incompatible change. */
@@ -84,7 +87,7 @@ int lightning_abi_version(void);
  *   slopes     [heads] float32.
  *   batch      >= 0 (0: nothing to do).  heads >= 1.  seq >= 0.
  *   dim        64 or 128.
- *   block      block length B >= 1 (tensor-core kernel: 128 or 256).
+ *   block      block length B >= 1 (tensor-core kernels: 128 or 256).
  *   state_in   [batch][heads][dim][dim] float32 carried-in state, or NULL for
  *              zeros.
  *   o          [batch][heads][seq][dim], dtype; written. Must not overlap
@@ -104,7 +107,7 @@ la_status lightning_prefill(const void *q, const void *k, const void *v, la_dtyp
                             void *workspace, size_t workspace_bytes, void *stream);
 
 /* Same as lightning_prefill with an explicit kernel choice (la_variant).
- * Requesting LA_VARIANT_TCGEN05 for an unsupported shape returns
+ * Requesting a tensor-core variant for a shape it does not take returns
  * LA_ERR_UNSUPPORTED. */
 la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_dtype dtype,
                                const float *slopes, int batch, int heads, int seq, int dim,

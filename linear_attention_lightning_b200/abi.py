@@ -16,7 +16,7 @@ HEADER = os.path.join(os.path.dirname(PKG), "include", "lightning.h")
 
 LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT = range(5)
 LA_DTYPE_F32, LA_DTYPE_BF16 = 0, 1
-LA_VARIANT_AUTO, LA_VARIANT_SIMT, LA_VARIANT_TCGEN05 = 0, 1, 2
+LA_VARIANT_AUTO, LA_VARIANT_SIMT, LA_VARIANT_TCGEN05, LA_VARIANT_TCGEN05_PAIR = 0, 1, 2, 3
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 

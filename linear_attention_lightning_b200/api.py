@@ -11,7 +11,8 @@ import torch
 from . import abi
 
 _DTYPES = {torch.float32: abi.LA_DTYPE_F32, torch.bfloat16: abi.LA_DTYPE_BF16}
-_VARIANTS = {"auto": abi.LA_VARIANT_AUTO, "simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05}
+_VARIANTS = {"auto": abi.LA_VARIANT_AUTO, "simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05,
+             "pair": abi.LA_VARIANT_TCGEN05_PAIR}
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -62,12 +63,13 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Ten
 
 def prefill_variant(dtype: torch.dtype, batch: int, heads: int, seq: int, dim: int, block: int,
                     variant: str = "auto") -> str:
-    """Which kernel lightning_prefill would run: "simt" or "tcgen05"."""
+    """Which kernel lightning_prefill would run: "simt", "tcgen05" or "pair"."""
     r = abi.lightning_prefill_selected_variant(_DTYPES[dtype], batch, heads, seq, dim, block,
                                                _VARIANTS[variant])
     if r < 0:
         raise ValueError(abi.last_error_message() or "unsupported request")
-    return {abi.LA_VARIANT_SIMT: "simt", abi.LA_VARIANT_TCGEN05: "tcgen05"}[r]
+    return {abi.LA_VARIANT_SIMT: "simt", abi.LA_VARIANT_TCGEN05: "tcgen05",
+            abi.LA_VARIANT_TCGEN05_PAIR: "pair"}[r]
 
 
 def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor,

@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_simt.cuh"
+#include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
 
 namespace {
@@ -81,11 +82,15 @@ la_status check_prefill_shape(la_dtype dtype, int batch, int heads, int seq, int
 }
 
 int choose_variant(la_dtype dtype, int dim, int block, int requested) {
-    const bool tc_ok = la::tc_supports(dtype == LA_DTYPE_BF16, dim, block);
+    const bool bf16 = dtype == LA_DTYPE_BF16;
+    const bool tc_ok = la::tc_supports(bf16, dim, block);
+    const bool pair_ok = la::pair_supports(bf16, dim, block);
     switch (requested) {
-        case LA_VARIANT_AUTO: return tc_ok ? LA_VARIANT_TCGEN05 : LA_VARIANT_SIMT;
+        case LA_VARIANT_AUTO:
+            return pair_ok ? LA_VARIANT_TCGEN05_PAIR : (tc_ok ? LA_VARIANT_TCGEN05 : LA_VARIANT_SIMT);
         case LA_VARIANT_SIMT: return LA_VARIANT_SIMT;
         case LA_VARIANT_TCGEN05: return tc_ok ? LA_VARIANT_TCGEN05 : -1;
+        case LA_VARIANT_TCGEN05_PAIR: return pair_ok ? LA_VARIANT_TCGEN05_PAIR : -1;
         default: return -1;
     }
 }
@@ -144,6 +149,9 @@ la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
         cudaError_t e = cudaGetLastError();
         return e == cudaSuccess ? ok() : cuda_fail(e, "state passthrough launch");
     }
+    if (variant == LA_VARIANT_TCGEN05_PAIR)
+        return la::launch_pair(a.q, a.k, a.v, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.o, a.state_out,
+                               stream, &g_last_error);
     if (variant == LA_VARIANT_TCGEN05) return la::launch_tc(a.q, a.k, a.v, a.slopes, a.batch, a.heads,
                                                            a.seq, a.block, a.state_in, a.o, a.state_out,
                                                            stream, &g_last_error);
@@ -179,10 +187,11 @@ la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_d
     if (st != LA_OK) return st;
     const int chosen = choose_variant(dtype, dim, block, variant);
     if (chosen < 0) {
-        if (variant < LA_VARIANT_AUTO || variant > LA_VARIANT_TCGEN05)
+        if (variant < LA_VARIANT_AUTO || variant > LA_VARIANT_TCGEN05_PAIR)
             return fail(LA_ERR_INVALID_ARG, "unknown variant %d", variant);
         return fail(LA_ERR_UNSUPPORTED,
-                    "the tcgen05 kernel needs bf16, dim 128 and block 128 or 256 (got dtype %d, dim %d, block %d)",
+                    "the tcgen05 kernels need bf16 and dim 128, with block 128 or 256 (single CTA) or block 256 "
+                    "(CTA pair) (got dtype %d, dim %d, block %d)",
                     (int)dtype, dim, block);
     }
     PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out};

@@ -1,0 +1,598 @@
+// Blockwise Lightning Attention prefill on a CTA pair (cta_group::2): block 256,
+// bf16 inputs, head dim 128.
+//
+// The method ("MINIMAX SIGNAL LAB · M1", §03 Lightning Attention), per block t
+// of 256 tokens of one (batch, head) with slope s:
+//   O_t = [(Q_t K_t^T) ⊙ D] V_t + (Q_t ⊙ d_q) S_{t-1}
+//   S_t = e^{-s m} S_{t-1} + (K_t ⊙ d_k)^T V_t
+// D_ij = e^{-s(i-j)} 1[i>=j], d_q[i] = e^{-s(i+1)}, d_k[j] = e^{-s(m-1-j)}.
+//
+// One cluster of two CTAs works on one (batch, head). The even CTA issues
+// every MMA for both SMs with M = 256: A operands are split by rows across
+// the pair and B operands by columns, so no product is computed twice.
+// CTA c owns
+//   - rows 128c .. 128c+127 of every block (its Q and K sub-tile),
+//   - value columns 64c .. 64c+63 (its half of V, of the state and of the
+//     state operand), and
+//   - the key-dimension half 64c .. 64c+63 of K ⊙ d_k for the state MMA.
+// Per block:
+//   QK   SS, M256 N256 K128, bf16      P (128 rows x 256 keys per SM, fp32 in TMEM)
+//   QS   TS, M256 N128 K128, f16       O  = Qd S_{t-1}   (Qd = Q ⊙ d_q, fp16 in TMEM)
+//   dS   SS, M128 N128 K256, f16       dS^T = V^T (K ⊙ d_k) (each SM: its 64 value
+//                                      columns x all 128 key dims)
+//   PV   TS, M256 N128 K256, f16       O += P V          (P ⊙ D, fp16 in TMEM)
+// Precision as in the single-CTA kernel: Q K^T on the bf16 inputs; P ⊙ D,
+// Q ⊙ d_q, S and K ⊙ d_k rounded to fp16; V widened to fp16 exactly; fp32
+// accumulation; the fp32 state stays in registers for the whole sequence.
+//
+// Warp roles (per CTA): warp 0 TMA, warp 1 MMA (even CTA only), warp 2 TMEM,
+// warp 3 forwards "Q/K landed" to the even CTA; warpgroup A (warps 4-7) turns
+// keys 0..127 of P into fp16 P ⊙ D and writes K ⊙ d_k; warpgroup B (warps
+// 8-11) does keys 128..255 and Qd; warpgroup 3 (warps 12-15) widens V,
+// carries the state and writes O. Hand-offs to the even CTA's MMA thread are
+// remote mbarrier arrivals; MMA completions reach both CTAs through
+// multicast commits. Every wait is bounded. A barrier that counts arrivals
+// from several groups is safe only if no group can arrive for block t+1
+// before the barrier's phase for block t has completed; each group's
+// per-block sequence below is ordered so that this holds.
+//
+// Shared memory per CTA (1024-aligned, 128B-swizzled):
+//   Q sub-tile 32 KB, K sub-tile 32 KB,
+//   2 stages x (V half for 256 keys 32 KB + K half-dims for 256 keys 32 KB),
+//   fp16 state operand 16 KB (rows = this CTA's 64 value columns).
+// TMEM per CTA: [0,256) P fp32 -> fp16 keys 0..127 in [0,64), keys 128..255
+// in [128,192); [256,384) O; [384,448) dS^T; [448,512) Qd.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <string>
+
+#include "../../include/lightning.h"
+#include "common.cuh"
+#include "prefill_tc.cuh"
+#include "tc_ptx.cuh"
+
+namespace la {
+namespace pair {
+
+constexpr int kThreads = 512;
+constexpr int kDim = 128;
+constexpr int kRows = 128;     // rows per CTA per block
+constexpr int kBlock = 256;    // tokens per block
+constexpr uint32_t kBoxBytes = 16384;   // 128 rows x 64 16-bit values (128 B rows)
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + 2 * kBoxBytes;
+constexpr uint32_t kOffStage = kOffK + 2 * kBoxBytes;          // 2 stages
+constexpr uint32_t kStageBytes = 4 * kBoxBytes;                // V (2 boxes) + Kd (2 boxes)
+constexpr uint32_t kOffS = kOffStage + 2 * kStageBytes;
+constexpr uint32_t kSBytes = 2 * 8192;                         // 2 boxes of 64 rows x 128 B
+constexpr uint32_t kOffBar = kOffS + kSBytes;
+constexpr int kNumBars = 24;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColP = 0, kColPHi = 128, kColO = 256, kColDS = 384, kColQd = 448;
+
+// barriers: local ones first, then the ones only the even CTA's MMA thread waits on
+constexpr int QK_LOADED = 0, VK_LOADED = 1 /* 2 */, P_FULL = 3, QK_DONE = 4, O_FULL = 5, DS_FULL = 6,
+              VK_EMPTY = 7 /* 2 */, P_FREE = 9, QD_LOCAL = 10, QK_FULL = 11, QD_READY = 12, S_READY = 13,
+              O_FREE = 14, VK_READY = 15, DS_FREE = 16, P_CONV = 17, DRAIN = 18;
+
+constexpr int kBarA = 1, kBarB = 3, kBarW3 = 2;  // named barriers of the three warpgroups
+
+__host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool a_mn, bool b_mn) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+constexpr uint32_t kIdescQK = idesc(256, 256, 1, false, false);  // Q (K-major) x K (K-major), bf16
+constexpr uint32_t kIdescQS = idesc(256, 128, 0, false, false);  // Qd (TMEM) x S (K-major), f16
+constexpr uint32_t kIdescPV = idesc(256, 128, 0, false, true);   // P (TMEM) x V (MN-major), f16
+constexpr uint32_t kIdescDS = idesc(128, 128, 0, true, true);    // V^T (MN-major) x Kd (MN-major), f16
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the same shared-memory location in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(ptx::smem_addr(p)), "r"(rank));
+    return out;
+}
+// arrive on the even CTA's copy of barrier `bar`
+__device__ __forceinline__ void arrive_leader(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(map_to_rank(bar, 0))
+                 : "memory");
+}
+
+struct Ctx {
+    uint8_t *smem;
+    uint32_t sbase;
+    uint64_t *bars;
+    volatile int *abort;
+    uint32_t tmem;
+};
+
+__device__ __forceinline__ bool wait_bar(const Ctx &c, int idx, uint32_t parity) {
+    return ptx::mbar_wait(&c.bars[idx], parity, c.abort);
+}
+// waits of the even CTA's MMA thread on barriers both CTAs arrive on
+__device__ __forceinline__ bool wait_pair(const Ctx &c, int idx, uint32_t parity) {
+    return ptx::mbar_wait_cluster(&c.bars[idx], parity, c.abort);
+}
+__device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parity, bool leader, int bar_id) {
+    const bool ok = leader ? wait_bar(c, idx, parity) : true;
+    return ptx::named_bar_and(bar_id, 128, ok);
+}
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
+    return ptx::pack_f16(ptx::bf16_lo(w) * scale, ptx::bf16_hi(w) * scale);
+}
+
+// fp32 P columns [col0, col0 + 128) of this thread's row -> fp16 P ⊙ D in
+// [dst0, dst0 + 64), two passes of 64 keys. Row i (block position) against
+// keys j0 .. j0+127. Every destination column was read by this thread first.
+__device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uint32_t dst0, int i, int j0,
+                                          float sl2, float step, const float (&tab)[16]) {
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        uint32_t va[32], vb[32];
+        ptx::tmem_ld32(taddr_row + col0 + 64 * pass, va);
+        ptx::tmem_ld32(taddr_row + col0 + 64 * pass + 32, vb);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+            uint32_t out[16];
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                const uint32_t *v = (hb == 0 ? va : vb) + 16 * g;
+                const int jb = j0 + 64 * pass + 32 * hb + 16 * g;
+                const int dlast = i - (jb + 15);
+                float p[16];
+                if (dlast >= 0) {
+                    const float wb = ptx::ex2(-sl2 * (float)dlast);
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[u]) * tab[u]) * wb;
+                } else if (i < jb) {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) p[u] = 0.f;
+                } else {
+                    const int d0 = i - jb;
+                    float w = 1.f;
+#pragma unroll
+                    for (int u = 15; u >= 0; --u) {
+                        const bool live = u <= d0;
+                        p[u] = live ? __uint_as_float(v[u]) * w : 0.f;
+                        w = live ? w * step : w;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) out[8 * g + u] = ptx::pack_f16(p[2 * u], p[2 * u + 1]);
+            }
+            __syncwarp();
+            ptx::tmem_st16(taddr_row + dst0 + 32 * pass + 16 * hb, out);
+        }
+    }
+}
+
+// scale one 128-byte swizzled row (64 16-bit values) in place: bf16 -> fp16 x scale
+__device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scale) {
+    uint4 x[8];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) x[ch] = *reinterpret_cast<const uint4 *>(row + ((ch ^ (r & 7)) << 4));
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        uint4 y;
+        y.x = bf16x2_to_f16x2(x[ch].x, scale); y.y = bf16x2_to_f16x2(x[ch].y, scale);
+        y.z = bf16x2_to_f16x2(x[ch].z, scale); y.w = bf16x2_to_f16x2(x[ch].w, scale);
+        *reinterpret_cast<uint4 *>(row + ((ch ^ (r & 7)) << 4)) = y;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ slopes, int heads,
+                    int seq, const float *state_in, __nv_bfloat16 *o, float *state_out) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+    const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+    Ctx c;
+    c.smem = smem_raw + pad;
+    c.sbase = raw_addr + pad;
+    c.bars = reinterpret_cast<uint64_t *>(c.smem + kOffBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c.smem + kOffMisc);
+    c.abort = reinterpret_cast<volatile int *>(c.smem + kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int bh = blockIdx.x >> 1;
+    const float s = slopes[bh % heads];
+    const float sl2 = s * kLog2e;
+    const int nblk = (seq + kBlock - 1) / kBlock;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(&c.bars[i], 1);
+        // the even CTA's MMA thread collects arrivals from both CTAs
+        ptx::mbar_init(&c.bars[QK_FULL], 2);
+        ptx::mbar_init(&c.bars[QD_READY], 2);
+        ptx::mbar_init(&c.bars[S_READY], 2);
+        ptx::mbar_init(&c.bars[O_FREE], 2);
+        ptx::mbar_init(&c.bars[VK_READY], 4);
+        ptx::mbar_init(&c.bars[DS_FREE], 2);
+        ptx::mbar_init(&c.bars[P_CONV], 4);
+        *c.abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tensormap(&tm_q);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         ptx::smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated on both SMs
+    ptx::tc_fence_after();
+    c.tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer (each CTA)
+        if (lane == 0) {
+            bool ok = true;
+            int vk_issued = 0, qk_issued = 0;
+            auto load_vk = [&](int t) -> bool {
+                const int st = t & 1;
+                if (!wait_bar(c, VK_EMPTY + st, ((uint32_t)(t >> 1) & 1u) ^ 1u)) return false;
+                uint8_t *dst = c.smem + kOffStage + st * kStageBytes;
+                uint64_t *bar = &c.bars[VK_LOADED + st];
+                ptx::mbar_arrive_expect_tx(bar, kStageBytes);
+                const int row0 = t * kBlock;
+                ptx::tma_load_3d(dst, &tm_v, bar, 64 * rank, row0, bh);                      // V keys 0..127
+                ptx::tma_load_3d(dst + kBoxBytes, &tm_v, bar, 64 * rank, row0 + kRows, bh);  // V keys 128..255
+                ptx::tma_load_3d(dst + 2 * kBoxBytes, &tm_k, bar, 64 * rank, row0, bh);      // K dims half, keys 0..127
+                ptx::tma_load_3d(dst + 3 * kBoxBytes, &tm_k, bar, 64 * rank, row0 + kRows, bh);
+                vk_issued = t + 1;
+                return true;
+            };
+            ok = load_vk(0);
+            for (int t = 0; t < nblk && ok; ++t) {
+                // Q and K sub-tiles of block t, once block t-1's Q K^T ran and its Qd was built
+                if (t > 0) ok = wait_bar(c, QK_DONE, (uint32_t)(t - 1) & 1u) && wait_bar(c, QD_LOCAL, (uint32_t)(t - 1) & 1u);
+                if (!ok) break;
+                const int row = t * kBlock + kRows * (int)rank;
+                ptx::mbar_arrive_expect_tx(&c.bars[QK_LOADED], 4 * kBoxBytes);
+                ptx::tma_load_3d(c.smem + kOffQ, &tm_q, &c.bars[QK_LOADED], 0, row, bh);
+                ptx::tma_load_3d(c.smem + kOffQ + kBoxBytes, &tm_q, &c.bars[QK_LOADED], 64, row, bh);
+                ptx::tma_load_3d(c.smem + kOffK, &tm_k, &c.bars[QK_LOADED], 0, row, bh);
+                ptx::tma_load_3d(c.smem + kOffK + kBoxBytes, &tm_k, &c.bars[QK_LOADED], 64, row, bh);
+                qk_issued = t + 1;
+                if (t + 1 < nblk) ok = load_vk(t + 1);
+            }
+            // let every copy issued land before the CTA may exit
+            volatile int never = 0;
+            if (qk_issued > 0) ptx::mbar_wait(&c.bars[QK_LOADED], (uint32_t)(qk_issued - 1) & 1u, &never);
+            for (int t = vk_issued > 2 ? vk_issued - 2 : 0; t < vk_issued; ++t)
+                ptx::mbar_wait(&c.bars[VK_LOADED + (t & 1)], (uint32_t)(t >> 1) & 1u, &never);
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------ forwarder (each CTA)
+        if (lane == 0) {
+            for (int t = 0; t < nblk; ++t) {
+                if (!wait_bar(c, QK_LOADED, (uint32_t)t & 1u)) break;
+                arrive_leader(&c.bars[QK_FULL]);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (lane == 0 && rank == 0) {
+            const uint32_t tm = c.tmem;
+            const uint64_t dq = sdesc(c.sbase + kOffQ, 16u, 1024u);
+            const uint64_t dk = sdesc(c.sbase + kOffK, 16u, 1024u);
+            const uint64_t ds = sdesc(c.sbase + kOffS, 16u, 1024u);
+            const uint64_t dstage = sdesc(c.sbase + kOffStage, kBoxBytes, 1024u);
+            bool ok = true;
+            for (int t = 0; t < nblk && ok; ++t) {
+                const uint32_t par = t & 1, fpar = par ^ 1u;
+                const uint64_t vdesc = dstage + (uint64_t)((uint32_t)(t & 1) * (kStageBytes >> 4));
+                const uint64_t kddesc = vdesc + (uint64_t)((2 * kBoxBytes) >> 4);
+                // P = Q K^T (256 x 256)
+                ok = wait_pair(c, QK_FULL, par) && wait_bar(c, P_FREE, fpar);
+                if (!ok) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
+                    ptx::mma_ss_2(tm + kColP, dq + koff, dk + koff, kIdescQK, k > 0);
+                }
+                ptx::mma_commit_2_mc(&c.bars[P_FULL], 0x3);
+                ptx::mma_commit_2_mc(&c.bars[QK_DONE], 0x3);
+                // O = Qd S_{t-1}
+                ok = wait_pair(c, QD_READY, par) && wait_pair(c, S_READY, par) && wait_pair(c, O_FREE, fpar);
+                if (!ok) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t koff = (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4);
+                    ptx::mma_ts_2(tm + kColO, tm + kColQd + 8u * k, ds + koff, kIdescQS, k > 0);
+                }
+                // dS^T = V^T (K ⊙ d_k)
+                ok = wait_pair(c, VK_READY, par) && wait_pair(c, DS_FREE, fpar);
+                if (!ok) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const uint64_t koff = (uint64_t)(k * (2048 >> 4));
+                    ptx::mma_ss_2(tm + kColDS, vdesc + koff, kddesc + koff, kIdescDS, k > 0);
+                }
+                // dS is complete and S_{t-1} is no longer read
+                ptx::mma_commit_2_mc(&c.bars[DS_FULL], 0x3);
+                // O += P V
+                ok = wait_pair(c, P_CONV, par);
+                if (!ok) break;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const uint32_t acol = k < 8 ? kColP + 8u * k : kColPHi + 8u * (k - 8);
+                    ptx::mma_ts_2(tm + kColO, tm + acol, vdesc + (uint64_t)(k * (2048 >> 4)), kIdescPV, 1);
+                }
+                ptx::mma_commit_2_mc(&c.bars[P_FREE], 0x3);
+                ptx::mma_commit_2_mc(&c.bars[O_FULL], 0x3);
+                ptx::mma_commit_2_mc(&c.bars[VK_EMPTY + (t & 1)], 0x3);
+            }
+            ptx::mma_commit_2_mc(&c.bars[DRAIN], 0x1);
+            volatile int never = 0;
+            ptx::mbar_wait(&c.bars[DRAIN], 0, &never);
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // ------------------------------------------------------------ warpgroups A and B
+        const int grp = (warp - 4) >> 2;           // 0: keys 0..127 (+ K ⊙ d_k), 1: keys 128..255 (+ Qd)
+        const int r = (threadIdx.x & 127);         // TMEM lane = row of this CTA's sub-tile
+        const bool leader = r == 0;
+        const int bar_id = grp == 0 ? kBarA : kBarB;
+        const uint32_t trow = c.tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const int i = kRows * (int)rank + r;       // row position inside the block
+        const float step = ptx::ex2(-sl2);
+        float tab[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) tab[u] = ptx::ex2(-sl2 * (float)(15 - u));
+        for (int t = 0; t < nblk; ++t) {
+            const uint32_t par = t & 1;
+            const int m = min(kBlock, seq - t * kBlock);
+            if (grp == 0) {
+                // K ⊙ d_k (fp16) for this CTA's key-dim half, keys r and 128 + r. The
+                // wait on the previous block's dS keeps this group from arriving on
+                // VK_READY for block t before that barrier's phase t-1 completed
+                // (VK_READY counts arrivals from both CTAs' groups).
+                if (t > 0 && !group_wait(c, DS_FULL, (uint32_t)(t - 1) & 1u, leader, bar_id)) goto ab_done;
+                if (!group_wait(c, VK_LOADED + (t & 1), (uint32_t)(t >> 1) & 1u, leader, bar_id)) goto ab_done;
+                uint8_t *kd = c.smem + kOffStage + (t & 1) * kStageBytes + 2 * kBoxBytes;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    const int j = kRows * h + r;
+                    const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
+                    scale_row_to_f16(kd + h * kBoxBytes + r * 128, r, dk);
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_sync(bar_id, 128);
+                if (leader) arrive_leader(&c.bars[VK_READY]);
+            } else {
+                // Qd = Q ⊙ d_q (fp16) into TMEM [448, 512), once the previous block's
+                // Qd S MMA (which precedes its dS MMA) has read the region
+                if (t > 0 && !group_wait(c, DS_FULL, (uint32_t)(t - 1) & 1u, leader, bar_id)) goto ab_done;
+                if (!group_wait(c, QK_LOADED, par, leader, bar_id)) goto ab_done;
+                const float dq = ptx::ex2(-sl2 * (float)(i + 1));
+                const uint8_t *qrow = c.smem + kOffQ + r * 128;
+#pragma unroll
+                for (int hb = 0; hb < 4; ++hb) {
+                    uint32_t out[16];
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        const int chunk = 4 * (hb & 1) + cc;
+                        const uint4 q4 = *reinterpret_cast<const uint4 *>(qrow + (hb >> 1) * kBoxBytes +
+                                                                          ((chunk ^ (r & 7)) << 4));
+                        out[4 * cc + 0] = bf16x2_to_f16x2(q4.x, dq);
+                        out[4 * cc + 1] = bf16x2_to_f16x2(q4.y, dq);
+                        out[4 * cc + 2] = bf16x2_to_f16x2(q4.z, dq);
+                        out[4 * cc + 3] = bf16x2_to_f16x2(q4.w, dq);
+                    }
+                    __syncwarp();
+                    ptx::tmem_st16(trow + kColQd + 16 * hb, out);
+                }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                ptx::named_bar_sync(bar_id, 128);
+                if (leader) {
+                    ptx::mbar_arrive(&c.bars[QD_LOCAL]);
+                    arrive_leader(&c.bars[QD_READY]);
+                }
+            }
+            // P ⊙ D -> fp16 for keys [128 grp, 128 grp + 128)
+            if (!group_wait(c, P_FULL, par, leader, bar_id)) goto ab_done;
+            ptx::tc_fence_after();
+            if (grp == 1 && rank == 0) {
+                // rows 0..127 against keys 128..255: every entry is masked
+                uint32_t zero[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) zero[u] = 0u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) ptx::tmem_st16(trow + kColPHi + 16 * q, zero);
+            } else {
+                convert_p(trow, grp == 0 ? kColP : kColPHi, grp == 0 ? kColP : kColPHi, i, kRows * grp, sl2,
+                          step, tab);
+            }
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            ptx::named_bar_sync(bar_id, 128);
+            if (leader) arrive_leader(&c.bars[P_CONV]);
+        }
+    ab_done:;
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------ warpgroup 3
+        // lane l of TMEM = this thread: value column 64*rank + (l & 63), key-dim half (l >> 6)
+        const int l = threadIdx.x - 384;
+        const bool leader = l == 0;
+        const uint32_t trow = c.tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const int vcol = 64 * (int)rank + (l & 63);
+        const int khalf = l >> 6;
+        float S[64];  // S[64 khalf + q][vcol], q = 0..63
+        const size_t sb = (size_t)bh * kDim * kDim;
+        if (state_in) {
+#pragma unroll
+            for (int q = 0; q < 64; ++q) S[q] = state_in[sb + (size_t)(64 * khalf + q) * kDim + vcol];
+        } else {
+#pragma unroll
+            for (int q = 0; q < 64; ++q) S[q] = 0.f;
+        }
+        // fp16 state operand: K-major rows = value column (l & 63), 64 key dims per box
+        uint8_t *srow = c.smem + kOffS + khalf * 8192 + (l & 63) * 128;
+        auto write_state_operand = [&]() {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                uint4 wv;
+                wv.x = ptx::pack_f16(S[8 * ch + 0], S[8 * ch + 1]);
+                wv.y = ptx::pack_f16(S[8 * ch + 2], S[8 * ch + 3]);
+                wv.z = ptx::pack_f16(S[8 * ch + 4], S[8 * ch + 5]);
+                wv.w = ptx::pack_f16(S[8 * ch + 6], S[8 * ch + 7]);
+                *reinterpret_cast<uint4 *>(srow + ((ch ^ (l & 7)) << 4)) = wv;
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::named_bar_sync(kBarW3, 128);
+            if (leader) arrive_leader(&c.bars[S_READY]);
+        };
+        write_state_operand();
+        for (int t = 0; t < nblk; ++t) {
+            const uint32_t par = t & 1;
+            const int m = min(kBlock, seq - t * kBlock);
+            // V half (256 keys x 64 value columns): bf16 -> fp16 in place
+            if (!group_wait(c, VK_LOADED + (t & 1), (uint32_t)(t >> 1) & 1u, leader, kBarW3)) goto w3_done;
+            {
+                uint8_t *vt = c.smem + kOffStage + (t & 1) * kStageBytes;
+                const int rr = l & 127;
+                scale_row_to_f16(vt + rr * 128, rr, 1.f);
+                scale_row_to_f16(vt + kBoxBytes + rr * 128, rr, 1.f);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::named_bar_sync(kBarW3, 128);
+            if (leader) arrive_leader(&c.bars[VK_READY]);
+            // state: S_t = e^{-s m} S_{t-1} + dS
+            if (!group_wait(c, DS_FULL, par, leader, kBarW3)) goto w3_done;
+            ptx::tc_fence_after();
+            {
+                const float dblock = ptx::ex2(-sl2 * (float)m);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t d[32];
+                    ptx::tmem_ld32(trow + kColDS + 32 * hh, d);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) S[32 * hh + q] = fmaf(dblock, S[32 * hh + q], __uint_as_float(d[q]));
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::named_bar_sync(kBarW3, 128);
+            if (leader) arrive_leader(&c.bars[DS_FREE]);
+            write_state_operand();
+            // O rows of this CTA: TMEM (fp32) -> bf16 -> global, 32 columns at a time
+            if (!group_wait(c, O_FULL, par, leader, kBarW3)) goto w3_done;
+            ptx::tc_fence_after();
+            {
+                const int row = t * kBlock + kRows * (int)rank + l;
+                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)bh * seq + row) * kDim);
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t a[32];
+                    ptx::tmem_ld32(trow + kColO + 32 * cb, a);
+                    ptx::tmem_ld_wait();
+                    if (cb == 3) {
+                        ptx::tc_fence_before();
+                        ptx::named_bar_sync(kBarW3, 128);
+                        if (leader) arrive_leader(&c.bars[O_FREE]);
+                    }
+                    if (row < seq) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[4 * cb + q] = make_uint4(
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 0]), __uint_as_float(a[8 * q + 1])),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 2]), __uint_as_float(a[8 * q + 3])),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 4]), __uint_as_float(a[8 * q + 5])),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 6]), __uint_as_float(a[8 * q + 7])));
+                    }
+                }
+            }
+        }
+        if (state_out) {
+#pragma unroll
+            for (int q = 0; q < 64; ++q) state_out[sb + (size_t)(64 * khalf + q) * kDim + vcol] = S[q];
+        }
+    w3_done:;
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the even CTA's MMAs, which read this CTA's memory, are done
+    if (warp == 2) {
+        ptx::tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(c.tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace pair
+
+// The CTA-pair kernel covers bf16 inputs, head dim 128 and blocks of 256.
+inline bool pair_supports(bool bf16, int dim, int block) { return bf16 && dim == 128 && block == 256; }
+
+inline la_status launch_pair(const void *q, const void *k, const void *v, const float *slopes, int batch,
+                             int heads, int seq, const float *state_in, void *o, float *state_out,
+                             cudaStream_t stream, std::string *err) {
+    const long long bh = (long long)batch * heads;
+    CUtensorMap mq, mk, mv;
+    if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
+        !tc::make_map(&mv, v, seq, bh, err))
+        return LA_ERR_CUDA;
+    cudaError_t e = cudaFuncSetAttribute(pair::prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)pair::kSmemBytes);
+    if (e != cudaSuccess) {
+        *err = std::string("cudaFuncSetAttribute(prefill_pair): ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(bh * 2));
+    cfg.blockDim = dim3(pair::kThreads);
+    cfg.dynamicSmemBytes = pair::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, pair::prefill_pair_kernel, mq, mk, mv, slopes, heads, seq, state_in,
+                           static_cast<__nv_bfloat16 *>(o), state_out);
+    if (e != cudaSuccess) {
+        *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    err->clear();
+    return LA_OK;
+}
+
+}  // namespace la

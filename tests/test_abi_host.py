@@ -83,6 +83,7 @@ def test_unknown_variant_and_unsupported_tensor_core_requests():
     assert _prefill(variant=abi.LA_VARIANT_TCGEN05, dtype=abi.LA_DTYPE_F32) == abi.LA_ERR_UNSUPPORTED
     assert _prefill(variant=abi.LA_VARIANT_TCGEN05, dim=64) == abi.LA_ERR_UNSUPPORTED
     assert _prefill(variant=abi.LA_VARIANT_TCGEN05, block=192) == abi.LA_ERR_UNSUPPORTED
+    assert _prefill(variant=abi.LA_VARIANT_TCGEN05_PAIR, block=128) == abi.LA_ERR_UNSUPPORTED
 
 
 def test_variant_selection():
@@ -90,8 +91,10 @@ def test_variant_selection():
     assert sel(abi.LA_DTYPE_F32, 1, 2, 256, 64, 64, abi.LA_VARIANT_AUTO) == abi.LA_VARIANT_SIMT
     assert sel(abi.LA_DTYPE_BF16, 1, 64, 8192, 128, 256, abi.LA_VARIANT_SIMT) == abi.LA_VARIANT_SIMT
     assert sel(abi.LA_DTYPE_BF16, 1, 64, 8192, 96, 256, abi.LA_VARIANT_AUTO) == -1
-    tc = sel(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_AUTO)
-    assert tc in (abi.LA_VARIANT_TCGEN05, abi.LA_VARIANT_SIMT)
+    assert sel(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_AUTO) == abi.LA_VARIANT_TCGEN05_PAIR
+    assert sel(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 128, abi.LA_VARIANT_AUTO) == abi.LA_VARIANT_TCGEN05
+    assert sel(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 128, abi.LA_VARIANT_TCGEN05_PAIR) == -1
+    assert sel(abi.LA_DTYPE_BF16, 1, 64, 4096, 128, 256, abi.LA_VARIANT_TCGEN05) == abi.LA_VARIANT_TCGEN05
 
 
 @pytest.mark.parametrize("kw,status", [
