@@ -18,18 +18,18 @@
 // Per block:
 //   QK   SS, M256 N256 K128, bf16      P (128 rows x 256 keys per SM, fp32 in TMEM)
 //   QS   TS, M256 N128 K128, f16       O  = Qd S_{t-1}   (Qd = Q ⊙ d_q, fp16 in TMEM)
-//   dS   SS, M128 N128 K256, f16       dS^T = V^T (K ⊙ d_k) (each SM: its 64 value
-//                                      columns x all 128 key dims)
+//   dS   SS, M128 N128 K256, f16       S^T += V^T (K ⊙ d_k) onto e^{-s m} S^T (each
+//                                      SM: its 64 value columns x all 128 key dims)
 //   PV   TS, M256 N128 K256, f16       O += P V          (P ⊙ D, fp16 in TMEM)
 // Precision as in the single-CTA kernel: Q K^T on the bf16 inputs; P ⊙ D,
 // Q ⊙ d_q, S and K ⊙ d_k rounded to fp16; V widened to fp16 exactly; fp32
 // accumulation; the fp32 state stays in registers for the whole sequence.
 //
 // Warp roles (per CTA): warp 0 TMA, warp 1 MMA (even CTA only), warp 2 TMEM,
-// warp 3 forwards "Q/K landed" to the even CTA; warpgroup A (warps 4-7) turns
-// keys 0..127 of P into fp16 P ⊙ D and writes K ⊙ d_k; warpgroup B (warps
-// 8-11) does keys 128..255 and Qd; warpgroup 3 (warps 12-15) widens V,
-// carries the state and writes O. Hand-offs to the even CTA's MMA thread are
+// warp 3 forwards "Q/K landed" to the even CTA; warpgroup A (warps 4-7) writes
+// K ⊙ d_k and widens V, then turns keys 0..127 of P into fp16 P ⊙ D;
+// warpgroup B (warps 8-11) builds Qd, then does keys 128..255 of P;
+// warpgroup 3 (warps 12-15) carries the state (fp32, in TMEM) and writes O. Hand-offs to the even CTA's MMA thread are
 // remote mbarrier arrivals; MMA completions reach both CTAs through
 // multicast commits. Every wait is bounded. A barrier that counts arrivals
 // from several groups is safe only if no group can arrive for block t+1
@@ -39,9 +39,10 @@
 // Shared memory per CTA (1024-aligned, 128B-swizzled):
 //   Q sub-tile 32 KB, K sub-tile 32 KB,
 //   2 stages x (V half for 256 keys 32 KB + K half-dims for 256 keys 32 KB),
-//   fp16 state operand 16 KB (rows = this CTA's 64 value columns).
+//   fp16 state operand 16 KB (rows = this CTA's 64 value columns),
+//   output staging 16 KB (half a row block of O, written out by TMA).
 // TMEM per CTA: [0,256) P fp32 -> fp16 keys 0..127 in [0,64), keys 128..255
-// in [128,192); [256,384) O; [384,448) dS^T; [448,512) Qd.
+// in [128,192); [256,384) O; [384,448) the fp32 state S^T; [448,512) Qd.
 #pragma once
 
 #include <cuda.h>
@@ -68,7 +69,8 @@ constexpr uint32_t kOffStage = kOffK + 2 * kBoxBytes;          // 2 stages
 constexpr uint32_t kStageBytes = 4 * kBoxBytes;                // V (2 boxes) + Kd (2 boxes)
 constexpr uint32_t kOffS = kOffStage + 2 * kStageBytes;
 constexpr uint32_t kSBytes = 2 * 8192;                         // 2 boxes of 64 rows x 128 B
-constexpr uint32_t kOffBar = kOffS + kSBytes;
+constexpr uint32_t kOffE = kOffS + kSBytes;                    // output staging: 128 rows x 64 bf16
+constexpr uint32_t kOffBar = kOffE + kBoxBytes;
 constexpr int kNumBars = 24;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
@@ -202,8 +204,9 @@ __device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scal
 
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ slopes, int heads,
-                    int seq, const float *state_in, __nv_bfloat16 *o, float *state_out) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const float *__restrict__ slopes, int heads, int seq, const float *state_in,
+                    float *state_out) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_addr(smem_raw);
     const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -228,7 +231,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::mbar_init(&c.bars[QD_READY], 2);
         ptx::mbar_init(&c.bars[S_READY], 2);
         ptx::mbar_init(&c.bars[O_FREE], 2);
-        ptx::mbar_init(&c.bars[VK_READY], 4);
+        ptx::mbar_init(&c.bars[VK_READY], 2);
         ptx::mbar_init(&c.bars[DS_FREE], 2);
         ptx::mbar_init(&c.bars[P_CONV], 4);
         *c.abort = 0;
@@ -238,6 +241,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::prefetch_tensormap(&tm_q);
         ptx::prefetch_tensormap(&tm_k);
         ptx::prefetch_tensormap(&tm_v);
+        ptx::prefetch_tensormap(&tm_o);
     }
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -332,16 +336,16 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const uint64_t koff = (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4);
                     ptx::mma_ts_2(tm + kColO, tm + kColQd + 8u * k, ds + koff, kIdescQS, k > 0);
                 }
-                // dS^T = V^T (K ⊙ d_k)
-                ok = wait_pair(c, VK_READY, par) && wait_pair(c, DS_FREE, fpar);
+                // S^T += V^T (K ⊙ d_k), onto e^{-s m} S^T prepared in TMEM
+                ok = wait_pair(c, VK_READY, par) && wait_pair(c, DS_FREE, par);
                 if (!ok) break;
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const uint64_t koff = (uint64_t)(k * (2048 >> 4));
-                    ptx::mma_ss_2(tm + kColDS, vdesc + koff, kddesc + koff, kIdescDS, k > 0);
+                    ptx::mma_ss_2(tm + kColDS, vdesc + koff, kddesc + koff, kIdescDS, 1);
                 }
-                // dS is complete and S_{t-1} is no longer read
+                // S_t is complete and S_{t-1} (the operand copy) is no longer read
                 ptx::mma_commit_2_mc(&c.bars[DS_FULL], 0x3);
                 // O += P V
                 ok = wait_pair(c, P_CONV, par);
@@ -376,18 +380,21 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const uint32_t par = t & 1;
             const int m = min(kBlock, seq - t * kBlock);
             if (grp == 0) {
-                // K ⊙ d_k (fp16) for this CTA's key-dim half, keys r and 128 + r. The
+                // K ⊙ d_k (fp16) for this CTA's key-dim half and V widened to fp16, keys r
+                // and 128 + r. The
                 // wait on the previous block's dS keeps this group from arriving on
                 // VK_READY for block t before that barrier's phase t-1 completed
                 // (VK_READY counts arrivals from both CTAs' groups).
                 if (t > 0 && !group_wait(c, DS_FULL, (uint32_t)(t - 1) & 1u, leader, bar_id)) goto ab_done;
                 if (!group_wait(c, VK_LOADED + (t & 1), (uint32_t)(t >> 1) & 1u, leader, bar_id)) goto ab_done;
-                uint8_t *kd = c.smem + kOffStage + (t & 1) * kStageBytes + 2 * kBoxBytes;
+                uint8_t *vt = c.smem + kOffStage + (t & 1) * kStageBytes;
+                uint8_t *kd = vt + 2 * kBoxBytes;
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
                     const int j = kRows * h + r;
                     const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
                     scale_row_to_f16(kd + h * kBoxBytes + r * 128, r, dk);
+                    scale_row_to_f16(vt + h * kBoxBytes + r * 128, r, 1.f);  // V: bf16 -> fp16
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::named_bar_sync(bar_id, 128);
@@ -445,103 +452,130 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     ab_done:;
     } else if (warp >= 12) {
         // ------------------------------------------------------------ warpgroup 3
-        // lane l of TMEM = this thread: value column 64*rank + (l & 63), key-dim half (l >> 6)
+        // The fp32 state S^T lives in TMEM [384, 448) in the 2x2 layout of the
+        // M=128 pair MMA: lane l holds S[64 (l >> 6) + q][64 rank + (l & 63)],
+        // q = 0..63. Before each block's state MMA this group leaves e^{-s m} S
+        // there, and the MMA adds (K ⊙ d_k)^T V on top.
         const int l = threadIdx.x - 384;
         const bool leader = l == 0;
         const uint32_t trow = c.tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         const int vcol = 64 * (int)rank + (l & 63);
         const int khalf = l >> 6;
-        float S[64];  // S[64 khalf + q][vcol], q = 0..63
         const size_t sb = (size_t)bh * kDim * kDim;
-        if (state_in) {
-#pragma unroll
-            for (int q = 0; q < 64; ++q) S[q] = state_in[sb + (size_t)(64 * khalf + q) * kDim + vcol];
-        } else {
-#pragma unroll
-            for (int q = 0; q < 64; ++q) S[q] = 0.f;
-        }
         // fp16 state operand: K-major rows = value column (l & 63), 64 key dims per box
         uint8_t *srow = c.smem + kOffS + khalf * 8192 + (l & 63) * 128;
-        auto write_state_operand = [&]() {
+        // one 32-value half of this thread's state row: operand copy, optional
+        // state_out, then the decayed value back into TMEM for the next MMA
+        auto carry_half = [&](const float (&sv)[32], int hh, float dnext, bool last) {
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
+            for (int cq = 0; cq < 4; ++cq) {
+                const int ch = 4 * hh + cq;
                 uint4 wv;
-                wv.x = ptx::pack_f16(S[8 * ch + 0], S[8 * ch + 1]);
-                wv.y = ptx::pack_f16(S[8 * ch + 2], S[8 * ch + 3]);
-                wv.z = ptx::pack_f16(S[8 * ch + 4], S[8 * ch + 5]);
-                wv.w = ptx::pack_f16(S[8 * ch + 6], S[8 * ch + 7]);
+                wv.x = ptx::pack_f16(sv[8 * cq + 0], sv[8 * cq + 1]);
+                wv.y = ptx::pack_f16(sv[8 * cq + 2], sv[8 * cq + 3]);
+                wv.z = ptx::pack_f16(sv[8 * cq + 4], sv[8 * cq + 5]);
+                wv.w = ptx::pack_f16(sv[8 * cq + 6], sv[8 * cq + 7]);
                 *reinterpret_cast<uint4 *>(srow + ((ch ^ (l & 7)) << 4)) = wv;
             }
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(kBarW3, 128);
-            if (leader) arrive_leader(&c.bars[S_READY]);
+            if (last) {
+                if (state_out) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) state_out[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q];
+                }
+            } else {
+                uint32_t lo[16], hi[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    lo[q] = __float_as_uint(sv[q] * dnext);
+                    hi[q] = __float_as_uint(sv[16 + q] * dnext);
+                }
+                __syncwarp();
+                ptx::tmem_st16(trow + kColDS + 32 * hh, lo);
+                ptx::tmem_st16(trow + kColDS + 32 * hh + 16, hi);
+            }
         };
-        write_state_operand();
+        auto publish = [&](bool last) {
+            if (!last) ptx::tmem_st_wait();
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            ptx::named_bar_sync(kBarW3, 128);
+            if (leader) {
+                arrive_leader(&c.bars[S_READY]);   // operand copy of S ready
+                arrive_leader(&c.bars[DS_FREE]);   // e^{-s m} S ready for the next state MMA
+            }
+        };
+        {
+            const float d0 = ptx::ex2(-sl2 * (float)min(kBlock, seq));
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                float sv[32];
+#pragma unroll
+                for (int q = 0; q < 32; ++q)
+                    sv[q] = state_in ? state_in[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] : 0.f;
+                carry_half(sv, hh, d0, false);
+            }
+            publish(false);
+        }
         for (int t = 0; t < nblk; ++t) {
             const uint32_t par = t & 1;
-            const int m = min(kBlock, seq - t * kBlock);
-            // V half (256 keys x 64 value columns): bf16 -> fp16 in place
-            if (!group_wait(c, VK_LOADED + (t & 1), (uint32_t)(t >> 1) & 1u, leader, kBarW3)) goto w3_done;
-            {
-                uint8_t *vt = c.smem + kOffStage + (t & 1) * kStageBytes;
-                const int rr = l & 127;
-                scale_row_to_f16(vt + rr * 128, rr, 1.f);
-                scale_row_to_f16(vt + kBoxBytes + rr * 128, rr, 1.f);
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(kBarW3, 128);
-            if (leader) arrive_leader(&c.bars[VK_READY]);
-            // state: S_t = e^{-s m} S_{t-1} + dS
+            const bool last = t + 1 == nblk;
+            // S_t is in TMEM once the state MMA is done
             if (!group_wait(c, DS_FULL, par, leader, kBarW3)) goto w3_done;
             ptx::tc_fence_after();
             {
-                const float dblock = ptx::ex2(-sl2 * (float)m);
-#pragma unroll
+                const float dnext = last ? 0.f : ptx::ex2(-sl2 * (float)min(kBlock, seq - (t + 1) * kBlock));
+#pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t d[32];
                     ptx::tmem_ld32(trow + kColDS + 32 * hh, d);
                     ptx::tmem_ld_wait();
+                    float sv[32];
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) S[32 * hh + q] = fmaf(dblock, S[32 * hh + q], __uint_as_float(d[q]));
+                    for (int q = 0; q < 32; ++q) sv[q] = __uint_as_float(d[q]);
+                    carry_half(sv, hh, dnext, last);
                 }
+                publish(last);
             }
-            ptx::tc_fence_before();
-            ptx::named_bar_sync(kBarW3, 128);
-            if (leader) arrive_leader(&c.bars[DS_FREE]);
-            write_state_operand();
-            // O rows of this CTA: TMEM (fp32) -> bf16 -> global, 32 columns at a time
+            // O rows of this CTA: TMEM (fp32) -> bf16 -> staging (128B-swizzled) -> TMA
+            // store, 64 value columns at a time; rows past seq are clipped by TMA
             if (!group_wait(c, O_FULL, par, leader, kBarW3)) goto w3_done;
             ptx::tc_fence_after();
             {
-                const int row = t * kBlock + kRows * (int)rank + l;
-                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)bh * seq + row) * kDim);
-#pragma unroll 1
+                uint32_t pk[64];  // the whole output row as bf16 pairs
+#pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {
                     uint32_t a[32];
                     ptx::tmem_ld32(trow + kColO + 32 * cb, a);
                     ptx::tmem_ld_wait();
-                    if (cb == 3) {
-                        ptx::tc_fence_before();
-                        ptx::named_bar_sync(kBarW3, 128);
-                        if (leader) arrive_leader(&c.bars[O_FREE]);
-                    }
-                    if (row < seq) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[4 * cb + q] = make_uint4(
-                                ptx::pack_bf16(__uint_as_float(a[8 * q + 0]), __uint_as_float(a[8 * q + 1])),
-                                ptx::pack_bf16(__uint_as_float(a[8 * q + 2]), __uint_as_float(a[8 * q + 3])),
-                                ptx::pack_bf16(__uint_as_float(a[8 * q + 4]), __uint_as_float(a[8 * q + 5])),
-                                ptx::pack_bf16(__uint_as_float(a[8 * q + 6]), __uint_as_float(a[8 * q + 7])));
+                    for (int u = 0; u < 16; ++u)
+                        pk[16 * cb + u] = ptx::pack_bf16(__uint_as_float(a[2 * u]), __uint_as_float(a[2 * u + 1]));
+                }
+                ptx::tc_fence_before();
+                ptx::named_bar_sync(kBarW3, 128);
+                if (leader) arrive_leader(&c.bars[O_FREE]);
+                uint8_t *erow = c.smem + kOffE + l * 128;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    // the previous store must have finished reading the staging buffer
+                    if (leader) ptx::bulk_wait_read();
+                    ptx::named_bar_sync(kBarW3, 128);
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        *reinterpret_cast<uint4 *>(erow + ((ch ^ (l & 7)) << 4)) =
+                            make_uint4(pk[32 * hh + 4 * ch], pk[32 * hh + 4 * ch + 1], pk[32 * hh + 4 * ch + 2],
+                                       pk[32 * hh + 4 * ch + 3]);
+                    ptx::fence_proxy_async_smem();
+                    ptx::named_bar_sync(kBarW3, 128);
+                    if (leader) {
+                        ptx::tma_store_3d(&tm_o, c.smem + kOffE, 64 * hh, t * kBlock + kRows * (int)rank, bh);
+                        ptx::bulk_commit();
                     }
                 }
             }
         }
-        if (state_out) {
-#pragma unroll
-            for (int q = 0; q < 64; ++q) state_out[sb + (size_t)(64 * khalf + q) * kDim + vcol] = S[q];
-        }
     w3_done:;
+        if (leader) ptx::bulk_wait_all();  // output stores complete before the CTA exits
     }
 
     ptx::tc_fence_before();
@@ -563,9 +597,9 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
                              int heads, int seq, const float *state_in, void *o, float *state_out,
                              cudaStream_t stream, std::string *err) {
     const long long bh = (long long)batch * heads;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
-        !tc::make_map(&mv, v, seq, bh, err))
+        !tc::make_map(&mv, v, seq, bh, err) || !tc::make_map(&mo, o, seq, bh, err))
         return LA_ERR_CUDA;
     cudaError_t e = cudaFuncSetAttribute(pair::prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)pair::kSmemBytes);
@@ -585,8 +619,8 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, pair::prefill_pair_kernel, mq, mk, mv, slopes, heads, seq, state_in,
-                           static_cast<__nv_bfloat16 *>(o), state_out);
+    e = cudaLaunchKernelEx(&cfg, pair::prefill_pair_kernel, mq, mk, mv, mo, slopes, heads, seq, state_in,
+                           state_out);
     if (e != cudaSuccess) {
         *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
         return LA_ERR_CUDA;
