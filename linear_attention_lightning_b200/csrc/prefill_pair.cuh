@@ -11,16 +11,22 @@
 // every MMA for both SMs with M = 256: A operands are split by rows across
 // the pair and B operands by columns, so no product is computed twice.
 // CTA c owns
-//   - rows 128c .. 128c+127 of every block (its Q and K sub-tile),
+//   - rows 128c .. 128c+127 of every block (its Q sub-tile) and the keys
+//     64c .. 64c+63 and 128+64c .. 128+64c+63 (its K sub-tile: its share of
+//     each key half's B operand),
 //   - value columns 64c .. 64c+63 (its half of V, of the state and of the
 //     state operand), and
 //   - the key-dimension half 64c .. 64c+63 of K ⊙ d_k for the state MMA.
 // Per block:
-//   QK   SS, M256 N256 K128, bf16      P (128 rows x 256 keys per SM, fp32 in TMEM)
+//   QK   SS, M256 N128 K128, bf16, twice: keys 0..127 and 128..255
+//                                      P (128 rows x 256 keys per SM, fp32 in TMEM)
 //   QS   TS, M256 N128 K128, f16       O  = Qd S_{t-1}   (Qd = Q ⊙ d_q, fp16 in TMEM)
 //   dS   SS, M128 N128 K256, f16       S^T += V^T (K ⊙ d_k) onto e^{-s m} S^T (each
 //                                      SM: its 64 value columns x all 128 key dims)
-//   PV   TS, M256 N128 K256, f16       O += P V          (P ⊙ D, fp16 in TMEM)
+//   PV   TS, M256 N128 K128, f16, twice: O += P V per key half (P ⊙ D, fp16)
+// Splitting P by key halves pipelines the chain Q K^T -> P ⊙ D -> P V: one
+// half is converted while the tensor core works on the other, and the next
+// block's first half of Q K^T runs as soon as this block's first P V is done.
 // Precision as in the single-CTA kernel: Q K^T on the bf16 inputs; P ⊙ D,
 // Q ⊙ d_q, S and K ⊙ d_k rounded to fp16; V widened to fp16 exactly; fp32
 // accumulation; the fp32 state stays in registers for the whole sequence.
@@ -37,7 +43,8 @@
 // per-block sequence below is ordered so that this holds.
 //
 // Shared memory per CTA (1024-aligned, 128B-swizzled):
-//   Q sub-tile 32 KB, K sub-tile 32 KB,
+//   Q sub-tile 32 KB, K sub-tile 32 KB (per 64-dim box: rows 0..63 keys
+//   64c.., rows 64..127 keys 128+64c..),
 //   2 stages x (V half for 256 keys 32 KB + K half-dims for 256 keys 32 KB),
 //   fp16 state operand 16 KB (rows = this CTA's 64 value columns),
 //   output staging 16 KB (half a row block of O, written out by TMA).
@@ -79,9 +86,11 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColP = 0, kColPHi = 128, kColO = 256, kColDS = 384, kColQd = 448;
 
 // barriers: local ones first, then the ones only the even CTA's MMA thread waits on
-constexpr int QK_LOADED = 0, VK_LOADED = 1 /* 2 */, P_FULL = 3, QK_DONE = 4, O_FULL = 5, DS_FULL = 6,
-              VK_EMPTY = 7 /* 2 */, P_FREE = 9, QD_LOCAL = 10, QK_FULL = 11, QD_READY = 12, S_READY = 13,
-              O_FREE = 14, VK_READY = 15, DS_FREE = 16, P_CONV = 17, DRAIN = 18;
+// (P_FULL, P_CONV, P_FREE: one per key half, index + half)
+constexpr int QK_LOADED = 0, VK_LOADED = 1 /* 2 */, P_FULL = 3 /* 2 */, QK_DONE = 5, O_FULL = 6,
+              DS_FULL = 7, VK_EMPTY = 8 /* 2 */, P_FREE = 10 /* 2 */, QD_LOCAL = 12, QK_FULL = 13,
+              QD_READY = 14, S_READY = 15, O_FREE = 16, VK_READY = 17, DS_FREE = 18, P_CONV = 19 /* 2 */,
+              DRAIN = 21;
 
 constexpr int kBarA = 1, kBarB = 3, kBarW3 = 2;  // named barriers of the three warpgroups
 
@@ -89,7 +98,7 @@ __host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool a_
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr uint32_t kIdescQK = idesc(256, 256, 1, false, false);  // Q (K-major) x K (K-major), bf16
+constexpr uint32_t kIdescQK = idesc(256, 128, 1, false, false);  // Q (K-major) x K (K-major), bf16
 constexpr uint32_t kIdescQS = idesc(256, 128, 0, false, false);  // Qd (TMEM) x S (K-major), f16
 constexpr uint32_t kIdescPV = idesc(256, 128, 0, false, true);   // P (TMEM) x V (MN-major), f16
 constexpr uint32_t kIdescDS = idesc(128, 128, 0, true, true);    // V^T (MN-major) x Kd (MN-major), f16
@@ -113,10 +122,14 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(ptx::smem_addr(p)), "r"(rank));
     return out;
 }
-// arrive on the even CTA's copy of barrier `bar`
+// Arrive on the even CTA's copy of barrier `bar`. Every hand-off to the MMA
+// thread concerns data in the arriving CTA's own shared memory or TMEM, made
+// visible to the tensor core by the async-proxy or tcgen05 fence that precedes
+// the arrival, so the default CTA-scope release suffices. A cluster-scope
+// release would also drain this thread's outstanding global traffic (the
+// output stores), which costs thousands of cycles per hand-off.
 __device__ __forceinline__ void arrive_leader(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(map_to_rank(bar, 0))
-                 : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(map_to_rank(bar, 0)) : "memory");
 }
 
 struct Ctx {
@@ -132,7 +145,7 @@ __device__ __forceinline__ bool wait_bar(const Ctx &c, int idx, uint32_t parity)
 }
 // waits of the even CTA's MMA thread on barriers both CTAs arrive on
 __device__ __forceinline__ bool wait_pair(const Ctx &c, int idx, uint32_t parity) {
-    return ptx::mbar_wait_cluster(&c.bars[idx], parity, c.abort);
+    return ptx::mbar_wait(&c.bars[idx], parity, c.abort);
 }
 __device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parity, bool leader, int bar_id) {
     const bool ok = leader ? wait_bar(c, idx, parity) : true;
@@ -143,48 +156,44 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
 }
 
 // fp32 P columns [col0, col0 + 128) of this thread's row -> fp16 P ⊙ D in
-// [dst0, dst0 + 64), two passes of 64 keys. Row i (block position) against
-// keys j0 .. j0+127. Every destination column was read by this thread first.
+// [dst0, dst0 + 64). Row i (block position) against keys j0 .. j0+127.
 __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uint32_t dst0, int i, int j0,
                                           float sl2, float step, const float (&tab)[16]) {
+    // 32 fp32 columns per iteration -> 16 fp16 pair columns; the destination
+    // [dst0 + 16 q, dst0 + 16 q + 16) lies inside columns already read
 #pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-        uint32_t va[32], vb[32];
-        ptx::tmem_ld32(taddr_row + col0 + 64 * pass, va);
-        ptx::tmem_ld32(taddr_row + col0 + 64 * pass + 32, vb);
+    for (int q = 0; q < 4; ++q) {
+        uint32_t v[32];
+        ptx::tmem_ld32(taddr_row + col0 + 32 * q, v);
         ptx::tmem_ld_wait();
+        uint32_t out[16];
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-            uint32_t out[16];
+        for (int g = 0; g < 2; ++g) {
+            const int jb = j0 + 32 * q + 16 * g;
+            const int dlast = i - (jb + 15);
+            float p[16];
+            if (dlast >= 0) {
+                const float wb = ptx::ex2(-sl2 * (float)dlast);
 #pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                const uint32_t *v = (hb == 0 ? va : vb) + 16 * g;
-                const int jb = j0 + 64 * pass + 32 * hb + 16 * g;
-                const int dlast = i - (jb + 15);
-                float p[16];
-                if (dlast >= 0) {
-                    const float wb = ptx::ex2(-sl2 * (float)dlast);
+                for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[16 * g + u]) * tab[u]) * wb;
+            } else if (i < jb) {
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[u]) * tab[u]) * wb;
-                } else if (i < jb) {
+                for (int u = 0; u < 16; ++u) p[u] = 0.f;
+            } else {
+                const int d0 = i - jb;
+                float w = 1.f;
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) p[u] = 0.f;
-                } else {
-                    const int d0 = i - jb;
-                    float w = 1.f;
-#pragma unroll
-                    for (int u = 15; u >= 0; --u) {
-                        const bool live = u <= d0;
-                        p[u] = live ? __uint_as_float(v[u]) * w : 0.f;
-                        w = live ? w * step : w;
-                    }
+                for (int u = 15; u >= 0; --u) {
+                    const bool live = u <= d0;
+                    p[u] = live ? __uint_as_float(v[16 * g + u]) * w : 0.f;
+                    w = live ? w * step : w;
                 }
-#pragma unroll
-                for (int u = 0; u < 8; ++u) out[8 * g + u] = ptx::pack_f16(p[2 * u], p[2 * u + 1]);
             }
-            __syncwarp();
-            ptx::tmem_st16(taddr_row + dst0 + 32 * pass + 16 * hb, out);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) out[8 * g + u] = ptx::pack_f16(p[2 * u], p[2 * u + 1]);
         }
+        __syncwarp();
+        ptx::tmem_st16(taddr_row + dst0 + 16 * q, out);
     }
 }
 
@@ -204,7 +213,8 @@ __device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scal
 
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_o,
                     const float *__restrict__ slopes, int heads, int seq, const float *state_in,
                     float *state_out) {
     extern __shared__ uint8_t smem_raw[];
@@ -233,13 +243,15 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::mbar_init(&c.bars[O_FREE], 2);
         ptx::mbar_init(&c.bars[VK_READY], 2);
         ptx::mbar_init(&c.bars[DS_FREE], 2);
-        ptx::mbar_init(&c.bars[P_CONV], 4);
+        ptx::mbar_init(&c.bars[P_CONV], 2);
+        ptx::mbar_init(&c.bars[P_CONV + 1], 2);
         *c.abort = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
         ptx::prefetch_tensormap(&tm_q);
         ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_k64);
         ptx::prefetch_tensormap(&tm_v);
         ptx::prefetch_tensormap(&tm_o);
     }
@@ -281,11 +293,17 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (t > 0) ok = wait_bar(c, QK_DONE, (uint32_t)(t - 1) & 1u) && wait_bar(c, QD_LOCAL, (uint32_t)(t - 1) & 1u);
                 if (!ok) break;
                 const int row = t * kBlock + kRows * (int)rank;
-                ptx::mbar_arrive_expect_tx(&c.bars[QK_LOADED], 4 * kBoxBytes);
-                ptx::tma_load_3d(c.smem + kOffQ, &tm_q, &c.bars[QK_LOADED], 0, row, bh);
-                ptx::tma_load_3d(c.smem + kOffQ + kBoxBytes, &tm_q, &c.bars[QK_LOADED], 64, row, bh);
-                ptx::tma_load_3d(c.smem + kOffK, &tm_k, &c.bars[QK_LOADED], 0, row, bh);
-                ptx::tma_load_3d(c.smem + kOffK + kBoxBytes, &tm_k, &c.bars[QK_LOADED], 64, row, bh);
+                const int krow = t * kBlock + 64 * (int)rank;
+                uint64_t *qkbar = &c.bars[QK_LOADED];
+                ptx::mbar_arrive_expect_tx(qkbar, 4 * kBoxBytes);
+                ptx::tma_load_3d(c.smem + kOffQ, &tm_q, qkbar, 0, row, bh);
+                ptx::tma_load_3d(c.smem + kOffQ + kBoxBytes, &tm_q, qkbar, 64, row, bh);
+#pragma unroll 1
+                for (int x = 0; x < 2; ++x) {
+                    uint8_t *kdst = c.smem + kOffK + x * kBoxBytes;
+                    ptx::tma_load_3d(kdst, &tm_k64, qkbar, 64 * x, krow, bh);                  // keys 64c..
+                    ptx::tma_load_3d(kdst + kBoxBytes / 2, &tm_k64, qkbar, 64 * x, krow + kRows, bh);  // 128+64c..
+                }
                 qk_issued = t + 1;
                 if (t + 1 < nblk) ok = load_vk(t + 1);
             }
@@ -316,16 +334,22 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t par = t & 1, fpar = par ^ 1u;
                 const uint64_t vdesc = dstage + (uint64_t)((uint32_t)(t & 1) * (kStageBytes >> 4));
                 const uint64_t kddesc = vdesc + (uint64_t)((2 * kBoxBytes) >> 4);
-                // P = Q K^T (256 x 256)
-                ok = wait_pair(c, QK_FULL, par) && wait_bar(c, P_FREE, fpar);
-                if (!ok) break;
-                ptx::tc_fence_after();
+                // P = Q K^T, one key half at a time, each once the previous
+                // block's P V for that half has read its columns
+#pragma unroll 1
+                for (int h = 0; h < 2 && ok; ++h) {
+                    ok = (h > 0 || wait_pair(c, QK_FULL, par)) && wait_bar(c, P_FREE + h, fpar);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const uint64_t dkh = dk + (uint64_t)(h * (kBoxBytes / 2) >> 4);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
-                    ptx::mma_ss_2(tm + kColP, dq + koff, dk + koff, kIdescQK, k > 0);
+                    for (int k = 0; k < 8; ++k) {
+                        const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
+                        ptx::mma_ss_2(tm + kColP + kColPHi * h, dq + koff, dkh + koff, kIdescQK, k > 0);
+                    }
+                    ptx::mma_commit_2_mc(&c.bars[P_FULL + h], 0x3);
                 }
-                ptx::mma_commit_2_mc(&c.bars[P_FULL], 0x3);
+                if (!ok) break;
                 ptx::mma_commit_2_mc(&c.bars[QK_DONE], 0x3);
                 // O = Qd S_{t-1}
                 ok = wait_pair(c, QD_READY, par) && wait_pair(c, S_READY, par) && wait_pair(c, O_FREE, fpar);
@@ -347,16 +371,19 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 // S_t is complete and S_{t-1} (the operand copy) is no longer read
                 ptx::mma_commit_2_mc(&c.bars[DS_FULL], 0x3);
-                // O += P V
-                ok = wait_pair(c, P_CONV, par);
-                if (!ok) break;
-                ptx::tc_fence_after();
+                // O += P V, one key half at a time
+#pragma unroll 1
+                for (int h = 0; h < 2 && ok; ++h) {
+                    ok = wait_pair(c, P_CONV + h, par);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const uint32_t acol = k < 8 ? kColP + 8u * k : kColPHi + 8u * (k - 8);
-                    ptx::mma_ts_2(tm + kColO, tm + acol, vdesc + (uint64_t)(k * (2048 >> 4)), kIdescPV, 1);
+                    for (int k = 0; k < 8; ++k)
+                        ptx::mma_ts_2(tm + kColO, tm + kColPHi * h + 8u * k,
+                                      vdesc + (uint64_t)((8 * h + k) * (2048 >> 4)), kIdescPV, 1);
+                    ptx::mma_commit_2_mc(&c.bars[P_FREE + h], 0x3);
                 }
-                ptx::mma_commit_2_mc(&c.bars[P_FREE], 0x3);
+                if (!ok) break;
                 ptx::mma_commit_2_mc(&c.bars[O_FULL], 0x3);
                 ptx::mma_commit_2_mc(&c.bars[VK_EMPTY + (t & 1)], 0x3);
             }
@@ -406,7 +433,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (!group_wait(c, QK_LOADED, par, leader, bar_id)) goto ab_done;
                 const float dq = ptx::ex2(-sl2 * (float)(i + 1));
                 const uint8_t *qrow = c.smem + kOffQ + r * 128;
-#pragma unroll
+#pragma unroll 1
                 for (int hb = 0; hb < 4; ++hb) {
                     uint32_t out[16];
 #pragma unroll
@@ -431,7 +458,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             // P ⊙ D -> fp16 for keys [128 grp, 128 grp + 128)
-            if (!group_wait(c, P_FULL, par, leader, bar_id)) goto ab_done;
+            if (!group_wait(c, P_FULL + grp, par, leader, bar_id)) goto ab_done;
             ptx::tc_fence_after();
             if (grp == 1 && rank == 0) {
                 // rows 0..127 against keys 128..255: every entry is masked
@@ -447,7 +474,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
             ptx::named_bar_sync(bar_id, 128);
-            if (leader) arrive_leader(&c.bars[P_CONV]);
+            if (leader) arrive_leader(&c.bars[P_CONV + grp]);
         }
     ab_done:;
     } else if (warp >= 12) {
@@ -597,9 +624,10 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
                              int heads, int seq, const float *state_in, void *o, float *state_out,
                              cudaStream_t stream, std::string *err) {
     const long long bh = (long long)batch * heads;
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mk64, mv, mo;
     if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
-        !tc::make_map(&mv, v, seq, bh, err) || !tc::make_map(&mo, o, seq, bh, err))
+        !tc::make_map(&mk64, k, seq, bh, err, 64) || !tc::make_map(&mv, v, seq, bh, err) ||
+        !tc::make_map(&mo, o, seq, bh, err))
         return LA_ERR_CUDA;
     cudaError_t e = cudaFuncSetAttribute(pair::prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)pair::kSmemBytes);
@@ -619,7 +647,7 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, pair::prefill_pair_kernel, mq, mk, mv, mo, slopes, heads, seq, state_in,
+    e = cudaLaunchKernelEx(&cfg, pair::prefill_pair_kernel, mq, mk, mk64, mv, mo, slopes, heads, seq, state_in,
                            state_out);
     if (e != cudaSuccess) {
         *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
