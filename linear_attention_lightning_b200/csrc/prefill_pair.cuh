@@ -417,11 +417,11 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 uint8_t *vt = c.smem + kOffStage + (t & 1) * kStageBytes;
                 uint8_t *kd = vt + 2 * kBoxBytes;
 #pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    const int j = kRows * h + r;
-                    const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
-                    scale_row_to_f16(kd + h * kBoxBytes + r * 128, r, dk);
-                    scale_row_to_f16(vt + h * kBoxBytes + r * 128, r, 1.f);  // V: bf16 -> fp16
+                for (int u = 0; u < 4; ++u) {
+                    // u = 0, 1: K rows r and 128 + r scaled by d_k; u = 2, 3: V rows widened
+                    const int h = u & 1, j = kRows * h + r;
+                    const float sc = u >= 2 ? 1.f : (j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f);
+                    scale_row_to_f16((u >= 2 ? vt : kd) + h * kBoxBytes + r * 128, r, sc);
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::named_bar_sync(bar_id, 128);
@@ -531,38 +531,36 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 arrive_leader(&c.bars[DS_FREE]);   // e^{-s m} S ready for the next state MMA
             }
         };
-        {
-            const float d0 = ptx::ex2(-sl2 * (float)min(kBlock, seq));
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                float sv[32];
-#pragma unroll
-                for (int q = 0; q < 32; ++q)
-                    sv[q] = state_in ? state_in[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] : 0.f;
-                carry_half(sv, hh, d0, false);
-            }
-            publish(false);
-        }
-        for (int t = 0; t < nblk; ++t) {
+        // t = -1 takes the carried-in state; block t >= 0 takes S_t from TMEM
+        for (int t = -1; t < nblk; ++t) {
             const uint32_t par = t & 1;
             const bool last = t + 1 == nblk;
             // S_t is in TMEM once the state MMA is done
-            if (!group_wait(c, DS_FULL, par, leader, kBarW3)) goto w3_done;
-            ptx::tc_fence_after();
+            if (t >= 0) {
+                if (!group_wait(c, DS_FULL, par, leader, kBarW3)) goto w3_done;
+                ptx::tc_fence_after();
+            }
             {
                 const float dnext = last ? 0.f : ptx::ex2(-sl2 * (float)min(kBlock, seq - (t + 1) * kBlock));
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t d[32];
-                    ptx::tmem_ld32(trow + kColDS + 32 * hh, d);
-                    ptx::tmem_ld_wait();
                     float sv[32];
+                    if (t >= 0) {
+                        uint32_t d[32];
+                        ptx::tmem_ld32(trow + kColDS + 32 * hh, d);
+                        ptx::tmem_ld_wait();
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) sv[q] = __uint_as_float(d[q]);
+                        for (int q = 0; q < 32; ++q) sv[q] = __uint_as_float(d[q]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            sv[q] = state_in ? state_in[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] : 0.f;
+                    }
                     carry_half(sv, hh, dnext, last);
                 }
                 publish(last);
             }
+            if (t < 0) continue;
             // O rows of this CTA: TMEM (fp32) -> bf16 -> staging (128B-swizzled) -> TMA
             // store, 64 value columns at a time; rows past seq are clipped by TMA
             if (!group_wait(c, O_FULL, par, leader, kBarW3)) goto w3_done;
@@ -570,13 +568,17 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             {
                 uint32_t pk[64];  // the whole output row as bf16 pairs
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    uint32_t a[32];
-                    ptx::tmem_ld32(trow + kColO + 32 * cb, a);
+                for (int cb = 0; cb < 4; cb += 2) {
+                    // two loads in flight per wait: O_FREE is on the path to the next block's first MMA
+                    uint32_t a0[32], a1[32];
+                    ptx::tmem_ld32(trow + kColO + 32 * cb, a0);
+                    ptx::tmem_ld32(trow + kColO + 32 * cb + 32, a1);
                     ptx::tmem_ld_wait();
 #pragma unroll
-                    for (int u = 0; u < 16; ++u)
-                        pk[16 * cb + u] = ptx::pack_bf16(__uint_as_float(a[2 * u]), __uint_as_float(a[2 * u + 1]));
+                    for (int u = 0; u < 16; ++u) {
+                        pk[16 * cb + u] = ptx::pack_bf16(__uint_as_float(a0[2 * u]), __uint_as_float(a0[2 * u + 1]));
+                        pk[16 * cb + 16 + u] = ptx::pack_bf16(__uint_as_float(a1[2 * u]), __uint_as_float(a1[2 * u + 1]));
+                    }
                 }
                 ptx::tc_fence_before();
                 ptx::named_bar_sync(kBarW3, 128);
