@@ -29,7 +29,7 @@
 // block's first half of Q K^T runs as soon as this block's first P V is done.
 // Precision as in the single-CTA kernel: Q K^T on the bf16 inputs; P ⊙ D,
 // Q ⊙ d_q, S and K ⊙ d_k rounded to fp16; V widened to fp16 exactly; fp32
-// accumulation; the fp32 state stays in registers for the whole sequence.
+// accumulation; the fp32 state stays in TMEM for the whole sequence.
 //
 // Warp roles (per CTA): warp 0 TMA, warp 1 MMA (even CTA only), warp 2 TMEM,
 // warp 3 forwards "Q/K landed" to the even CTA; warpgroup A (warps 4-7) writes
