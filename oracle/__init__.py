@@ -6,8 +6,9 @@ shares no code with it.
 
 The arithmetic lives in ``lightning_oracle.c`` (three forms of the same
 result: F1 definition, F2 token recurrence, F3 blockwise, plus one decode
-step; see that file's header for the formulas and their sources on the
-"MINIMAX SIGNAL LAB · M1" page, §03 Lightning Attention). This module only
+step and the state snapshots of a prefix cache; see that file's header for
+the formulas and their sources on the "MINIMAX SIGNAL LAB · M1" page, §03
+Lightning Attention). This module only
 marshals numpy arrays into it.
 
 Inputs are numpy arrays: float32, or uint16 holding bfloat16 bit patterns.
@@ -37,6 +38,8 @@ def _load():
         lib.la_oracle_blockwise.restype = ctypes.c_int
         lib.la_oracle_decode.argtypes = [vp, vp, vp, ip, fp, ip, ip, ip, dp, dp]
         lib.la_oracle_decode.restype = ctypes.c_int
+        lib.la_oracle_snapshots.argtypes = [vp, vp, ip, fp, ip, ip, ip, ip, fp, ip, dp]
+        lib.la_oracle_snapshots.restype = ctypes.c_int
         lib.la_oracle_max_threads.restype = ctypes.c_int
         lib.la_oracle_set_threads.argtypes = [ip]
         _lib = lib
@@ -105,6 +108,24 @@ def prefill(q, k, v, slopes, state_in=None, form="recurrence", block=None):
     if rc != 0:
         raise RuntimeError("oracle %s failed (rc=%d)" % (form, rc))
     return o, s_out
+
+
+def snapshots(k, v, slopes, interval, state_in=None):
+    """States after the first (n+1)*interval tokens, n = 0 .. seq//interval - 1.
+
+    Returns float64 [batch, heads, seq//interval, dim, dim] (token recurrence)."""
+    k, v, _, code, slopes, state_in, (b, h, L, d) = _prepare(k, v, v, slopes, state_in)
+    interval = int(interval)
+    if interval <= 0:
+        raise ValueError("interval must be positive")
+    out = np.empty((b, h, L // interval, d, d), dtype=np.float64)
+    if out.size == 0:
+        return out
+    rc = _load().la_oracle_snapshots(_ptr(k), _ptr(v), code, _ptr(slopes), b, h, L, d, _ptr(state_in),
+                                     interval, _ptr(out))
+    if rc != 0:
+        raise RuntimeError("oracle snapshots failed (rc=%d)" % rc)
+    return out
 
 
 def decode(q, k, v, slopes, state):

@@ -33,7 +33,8 @@
  *                             linear attention, fishai.com.cn article on
  *                             M1), O(L d^2) per head; the full-size oracle.
  *   F3 la_oracle_blockwise  : the block formulas of §03 for a given B.
- * plus la_oracle_decode, one recurrent step for a single new token.
+ * plus la_oracle_decode, one recurrent step for a single new token, and
+ * la_oracle_snapshots, the state after every `interval` tokens (F2's state).
  *
  * Layouts: q, k, v, o are [batch][heads][seq][dim] contiguous (o for decode
  * is [batch][heads][dim]); states are [batch][heads][dim(k)][dim(v)].
@@ -184,6 +185,51 @@ int la_oracle_recurrence(const void *q, const void *k, const void *v, int dtype,
         }
         if (state_out) memcpy(state_out + (size_t)bh * d * d, S, sizeof(double) * d * d);
         free(S); free(qi); free(ki); free(vi);
+    }
+    return fail;
+}
+
+/* State snapshots: the state after the first (n+1)*interval tokens, for
+ * n = 0 .. seq/interval - 1, by the same token recurrence as F2
+ * (S_i = e^{-s} S_{i-1} + k_i^T v_i, starting from S_in). These are the
+ * states a prefix cache stores ("MINIMAX SIGNAL LAB · M1", §03 Lightning
+ * Attention: the recursive fixed-size state, and the page's note on prefix
+ * caching and speculative decoding with such states).
+ * snapshots: [batch][heads][seq/interval][dim][dim] float64. */
+int la_oracle_snapshots(const void *k, const void *v, int dtype, const float *slopes, int batch,
+                        int heads, int seq, int dim, const float *state_in, int interval,
+                        double *snapshots) {
+    if (!k || !v || !slopes || !snapshots) return 1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16) return 1;
+    if (batch < 0 || heads <= 0 || seq < 0 || dim <= 0 || interval <= 0) return 1;
+    const long BH = (long)batch * heads;
+    const size_t L = (size_t)seq, d = (size_t)dim, count = (size_t)(seq / interval);
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        const int h = (int)(bh % heads);
+        const double decay = exp(-(double)slopes[h]);
+        double *S = malloc(sizeof(double) * d * d);
+        double *ki = malloc(sizeof(double) * d), *vi = malloc(sizeof(double) * d);
+        if (!S || !ki || !vi) {
+            fail = 1;
+            free(S); free(ki); free(vi);
+            continue;
+        }
+        for (size_t n = 0; n < d * d; ++n)
+            S[n] = state_in ? (double)state_in[(size_t)bh * d * d + n] : 0.0;
+        const size_t base = (size_t)bh * L * d;
+        for (size_t i = 0; i < L; ++i) {
+            widen_head(k, dtype, base + i * d, d, ki);
+            widen_head(v, dtype, base + i * d, d, vi);
+            for (size_t r = 0; r < d; ++r)
+                for (size_t c = 0; c < d; ++c) S[r * d + c] = decay * S[r * d + c] + ki[r] * vi[c];
+            if ((i + 1) % (size_t)interval == 0) {
+                const size_t n = (i + 1) / (size_t)interval - 1;
+                memcpy(snapshots + ((size_t)bh * count + n) * d * d, S, sizeof(double) * d * d);
+            }
+        }
+        free(S); free(ki); free(vi);
     }
     return fail;
 }

@@ -231,3 +231,23 @@ def test_state_size_matches_the_printed_m1_figure():
     per_layer = st.astype(np.float32).nbytes
     total_mb = vals["layers"] * per_layer / 1e6
     assert abs(total_mb - vals["printed_megabytes"]) < 0.01
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_snapshots_are_the_states_of_the_prefixes(with_state):
+    # snapshot n is the state a prefill of the first (n+1)*interval tokens leaves behind,
+    # taken here from the quadratic definition (F1), an independent form
+    b, h, L, d, interval = 2, 4, 23, 5, 4
+    q, k, v = (_rand((b, h, L, d), s) for s in (40, 41, 42))
+    s0 = _rand((b, h, d, d), 43) if with_state else None
+    snaps = oracle.snapshots(k, v, SLOPES_MIX, interval, s0)
+    assert snaps.shape == (b, h, L // interval, d, d)
+    for n in range(L // interval):
+        n_tok = (n + 1) * interval
+        _, s_prefix = oracle.prefill(q[:, :, :n_tok], k[:, :, :n_tok], v[:, :, :n_tok], SLOPES_MIX, s0,
+                                     form="definition")
+        _close(snaps[:, :, n], s_prefix, 1e-12)
+    # an interval longer than the sequence takes no snapshot; interval == L takes state_out
+    assert oracle.snapshots(k, v, SLOPES_MIX, L + 1, s0).shape == (b, h, 0, d, d)
+    _, s_out = oracle.prefill(q, k, v, SLOPES_MIX, s0, form="definition")
+    _close(oracle.snapshots(k, v, SLOPES_MIX, L, s0)[:, :, 0], s_out, 1e-12)
