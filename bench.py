@@ -340,6 +340,10 @@ def run_ours(args):
     # end to end: host buffers, copies inside the timed region
     e2e = run_e2e(w, dev, stream, inp, variant, args, world) if args.e2e_steps > 0 else None
 
+    # the same prefill keeping prefix-cache snapshots of the state
+    snaps = (run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, ms_per_step)
+             if args.snapshot_interval > 0 and w.seq >= args.snapshot_interval else None)
+
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -357,6 +361,7 @@ def run_ours(args):
         "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s", traffic),
         "decode": dec,
         "e2e": e2e,
+        "snapshots": snaps,
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
     }
@@ -403,6 +408,42 @@ def run_decode(dw, dev, stream, peaks, args):
             "value": round(gbs, 1), "unit": "GB/s (state + token bytes)",
             "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s"),
             "l2": "state 268 MB > L2; consecutive steps, no flush"}
+
+
+def run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, plain_ms):
+    """The prefill step through lightning_prefill_snapshots: a state snapshot
+    every args.snapshot_interval tokens, timed like the main leg."""
+    import torch
+    from linear_attention_lightning_b200 import abi
+    q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
+    interval = args.snapshot_interval
+    n = abi.lightning_prefill_snapshot_count(w.seq, interval)
+    o = torch.empty_like(q)
+    s_out = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32, device=dev)
+    snaps = torch.empty((w.batch, w.heads, n, w.dim, w.dim), dtype=torch.float32, device=dev)
+    sp = stream.cuda_stream
+
+    def step():
+        abi.check(abi.lightning_prefill_snapshots(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads, w.seq, w.dim,
+            w.block, None if s0 is None else s0.data_ptr(), o.data_ptr(), s_out.data_ptr(), interval,
+            snaps.data_ptr(), sp, vcode))
+
+    for _ in range(args.warmup):
+        step()
+    steps = max(1, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    return {"interval": interval, "count": n, "steps": steps, "ms_per_step": round(ms, 4),
+            "overhead_vs_plain_pct": round(100.0 * (ms / plain_ms - 1.0), 2),
+            "snapshot_bytes_per_step": int(snaps.numel() * 4)}
 
 
 def run_e2e(w, dev, stream, inp, variant, args, world):
@@ -453,6 +494,8 @@ def parse_args(argv=None):
     p.add_argument("--decode-steps", type=int, default=1000)
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--snapshot-interval", type=int, default=16384,
+                   help="tokens between prefix-cache state snapshots in the snapshot leg (0 skips it)")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be at least 3")

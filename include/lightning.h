@@ -124,6 +124,33 @@ int lightning_prefill_selected_variant(la_dtype dtype, int batch, int heads, int
 size_t lightning_prefill_workspace_size(int batch, int heads, int seq, int dim, int block);
 
 /*
+ * Prefill that also keeps prefix-cache snapshots of the state. Source:
+ * "MINIMAX SIGNAL LAB · M1", §03 Lightning Attention (the recursive fixed-size
+ * state S_t; the page's note that prefix caching and speculative decoding are
+ * where such states are hard to serve) and §04 (the fp32 state per head).
+ *
+ * Same arguments and results as lightning_prefill_ex (workspace: none), plus
+ *   interval   snapshot spacing in tokens: a positive multiple of `block`.
+ *   snapshots  [batch][heads][n][dim][dim] float32, n = seq / interval
+ *              (lightning_prefill_snapshot_count); snapshot i is the state after
+ *              the first (i+1)*interval tokens, i.e. what lightning_prefill on
+ *              that prefix returns as state_out (it includes state_in, decayed).
+ *              Device pointer, caller-owned, 16-byte aligned, overlapping nothing
+ *              else; may be NULL when n == 0.
+ * `o` and `state_out` are bit-identical to lightning_prefill_ex's for the same
+ * variant. A bad interval or snapshot buffer returns LA_ERR_INVALID_ARG before
+ * any launch.
+ */
+la_status lightning_prefill_snapshots(const void *q, const void *k, const void *v, la_dtype dtype,
+                                      const float *slopes, int batch, int heads, int seq, int dim,
+                                      int block, const float *state_in, void *o, float *state_out,
+                                      int interval, float *snapshots, void *stream, int variant);
+
+/* Number of snapshots lightning_prefill_snapshots writes per (batch, head):
+ * seq / interval, or -1 if seq < 0 or interval < 1. Host only. */
+int lightning_prefill_snapshot_count(int seq, int interval);
+
+/*
  * One decode step for a single new token of every (batch, head), updating the
  * state in place. Source: "MINIMAX SIGNAL LAB · M1", §03 (recursive KV state)
  * and §04 (fixed-size FP32 state per head).

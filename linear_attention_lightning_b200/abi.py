@@ -27,6 +27,9 @@ _SIGNATURES = {
                               _i], _i),
     "lightning_prefill_selected_variant": ([_i, _i, _i, _i, _i, _i, _i], _i),
     "lightning_prefill_workspace_size": ([_i, _i, _i, _i, _i], _sz),
+    "lightning_prefill_snapshots": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp,
+                                     _i], _i),
+    "lightning_prefill_snapshot_count": ([_i, _i], _i),
     "lightning_decode": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp], _i),
     "lightning_device_status": ([_vp], _i),
     "lightning_status_string": ([_i], ctypes.c_char_p),
@@ -102,6 +105,16 @@ def lightning_prefill_selected_variant(dtype, batch, heads, seq, dim, block, var
 
 def lightning_prefill_workspace_size(batch, heads, seq, dim, block):
     return load().lightning_prefill_workspace_size(batch, heads, seq, dim, block)
+
+
+def lightning_prefill_snapshots(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out,
+                                interval, snapshots, stream, variant):
+    return load().lightning_prefill_snapshots(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in,
+                                              o, state_out, interval, snapshots, stream, variant)
+
+
+def lightning_prefill_snapshot_count(seq, interval):
+    return load().lightning_prefill_snapshot_count(seq, interval)
 
 
 def lightning_decode(q, k, v, dtype, slopes, batch, heads, dim, state, o, stream):

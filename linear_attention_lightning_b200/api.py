@@ -61,6 +61,46 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Ten
     return o, state_out
 
 
+def prefill_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor, block: int,
+                      interval: int, state_in: Optional[torch.Tensor] = None, o: Optional[torch.Tensor] = None,
+                      state_out: Optional[torch.Tensor] = None, snapshots: Optional[torch.Tensor] = None,
+                      want_state: bool = True, variant: str = "auto",
+                      stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor], torch.Tensor]:
+    """lightning_prefill_snapshots: returns (o, state_out, snapshots); snapshots is
+    [batch, heads, seq // interval, dim, dim] float32, the state after each
+    interval tokens."""
+    if q.dtype not in _DTYPES:
+        raise ValueError("q must be float32 or bfloat16")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [batch, heads, seq, dim] shape")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, q.dtype)
+    b, h, L, d = q.shape
+    _need_cuda("slopes", slopes, torch.float32)
+    if state_in is not None:
+        _need_cuda("state_in", state_in, torch.float32)
+        if tuple(state_in.shape) != (b, h, d, d):
+            raise ValueError("state_in must be [batch, heads, dim, dim]")
+    n = abi.lightning_prefill_snapshot_count(L, int(interval))
+    if n < 0:
+        raise ValueError("interval must be >= 1")
+    if o is None:
+        o = torch.empty_like(q)
+    if state_out is None and want_state:
+        state_out = torch.empty((b, h, d, d), dtype=torch.float32, device=q.device)
+    if snapshots is None:
+        snapshots = torch.empty((b, h, n, d, d), dtype=torch.float32, device=q.device)
+    else:
+        _need_cuda("snapshots", snapshots, torch.float32)
+        if tuple(snapshots.shape) != (b, h, n, d, d):
+            raise ValueError("snapshots must be [batch, heads, seq // interval, dim, dim]")
+    abi.check(abi.lightning_prefill_snapshots(
+        _ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(slopes), b, h, L, d, int(block),
+        _ptr(state_in), _ptr(o), _ptr(state_out), int(interval), _ptr(snapshots) if n > 0 else None,
+        _stream(stream), _VARIANTS[variant]))
+    return o, state_out, snapshots
+
+
 def prefill_variant(dtype: torch.dtype, batch: int, heads: int, seq: int, dim: int, block: int,
                     variant: str = "auto") -> str:
     """Which kernel lightning_prefill would run: "simt", "tcgen05" or "pair"."""

@@ -25,4 +25,22 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // e^{-s * n} for n >= 0 through exp2f; s is the per-head slope.
 __device__ __forceinline__ float decay_pow(float s, float n) { return exp2f(-s * kLog2e * n); }
 
+// State snapshots for a prefix cache: the fp32 state after every `interval`
+// tokens (a multiple of the block), `count` = seq / interval of them per
+// (batch, head), laid out [batch*heads][count][dim][dim]. ptr == nullptr: none.
+struct Snapshots {
+    float *ptr;
+    int interval;
+    int count;
+};
+
+// Where the state after the first `tokens_done` tokens of (batch*heads index)
+// bh goes, or nullptr when that position takes no snapshot.
+__device__ __forceinline__ float *snapshot_at(const Snapshots &sn, size_t bh, int tokens_done, int dim) {
+    if (sn.ptr == nullptr || tokens_done <= 0 || tokens_done % sn.interval != 0) return nullptr;
+    const int n = tokens_done / sn.interval - 1;
+    if (n >= sn.count) return nullptr;
+    return sn.ptr + ((size_t)bh * sn.count + n) * dim * dim;
+}
+
 }  // namespace la

@@ -64,6 +64,7 @@ struct PrefillArgs {
     const float *state_in;
     void *o;
     float *state_out;
+    la::Snapshots sn;  // prefix-cache snapshots; sn.ptr == nullptr: none
 };
 
 // Shape / dtype checks shared by the launcher and the variant query.
@@ -124,6 +125,27 @@ la_status check_prefill_pointers(const PrefillArgs &a) {
     return LA_OK;
 }
 
+// Snapshot interval and buffer: checked after check_prefill_pointers.
+la_status check_snapshots(const PrefillArgs &a) {
+    if (a.sn.interval < a.block || a.sn.interval % a.block != 0)
+        return fail(LA_ERR_INVALID_ARG, "snapshot interval %d must be a positive multiple of block %d",
+                    a.sn.interval, a.block);
+    if (a.sn.count == 0) return LA_OK;
+    if (!a.sn.ptr) return fail(LA_ERR_INVALID_ARG, "snapshots must be non-NULL when seq / interval > 0");
+    if (!aligned16(a.sn.ptr)) return fail(LA_ERR_INVALID_ARG, "snapshots is not 16-byte aligned");
+    const size_t eb = elem_bytes(a.dtype);
+    const size_t n_tok = (size_t)a.batch * a.heads * a.seq * a.dim;
+    const size_t n_state = (size_t)a.batch * a.heads * a.dim * a.dim;
+    const Range rs = range_of(a.sn.ptr, n_state * (size_t)a.sn.count * sizeof(float));
+    const Range others[] = {range_of(a.q, n_tok * eb), range_of(a.k, n_tok * eb), range_of(a.v, n_tok * eb),
+                            range_of(a.o, n_tok * eb), range_of(a.slopes, sizeof(float) * a.heads),
+                            range_of(a.state_in, a.state_in ? n_state * 4 : 0),
+                            range_of(a.state_out, a.state_out ? n_state * 4 : 0)};
+    for (const Range &r : others)
+        if (overlaps(rs, r)) return fail(LA_ERR_INVALID_ARG, "snapshots overlaps an input, o or a state");
+    return LA_OK;
+}
+
 template <typename T, int D>
 la_status launch_simt(const PrefillArgs &a, cudaStream_t stream) {
     auto kern = la::prefill_simt_kernel<T, D>;
@@ -133,7 +155,7 @@ la_status launch_simt(const PrefillArgs &a, cudaStream_t stream) {
     dim3 grid((unsigned)((size_t)a.batch * a.heads * (D / la::kSimtCols)));
     kern<<<grid, la::kSimtThreads, smem, stream>>>(
         static_cast<const T *>(a.q), static_cast<const T *>(a.k), static_cast<const T *>(a.v),
-        a.slopes, a.heads, a.seq, a.block, a.state_in, static_cast<T *>(a.o), a.state_out);
+        a.slopes, a.heads, a.seq, a.block, a.state_in, static_cast<T *>(a.o), a.state_out, a.sn);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prefill_simt launch");
     return ok();
@@ -151,10 +173,10 @@ la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
     }
     if (variant == LA_VARIANT_TCGEN05_PAIR)
         return la::launch_pair(a.q, a.k, a.v, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.o, a.state_out,
-                               stream, &g_last_error);
+                               a.sn, stream, &g_last_error);
     if (variant == LA_VARIANT_TCGEN05) return la::launch_tc(a.q, a.k, a.v, a.slopes, a.batch, a.heads,
                                                            a.seq, a.block, a.state_in, a.o, a.state_out,
-                                                           stream, &g_last_error);
+                                                           a.sn, stream, &g_last_error);
     if (a.dtype == LA_DTYPE_BF16)
         return a.dim == 64 ? launch_simt<__nv_bfloat16, 64>(a, stream)
                            : launch_simt<__nv_bfloat16, 128>(a, stream);
@@ -177,13 +199,15 @@ extern "C" {
 
 int lightning_abi_version(void) { return 1; }
 
-la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_dtype dtype,
-                               const float *slopes, int batch, int heads, int seq, int dim, int block,
-                               const float *state_in, void *o, float *state_out, void *workspace,
-                               size_t workspace_bytes, void *stream, int variant) {
-    (void)workspace;
-    (void)workspace_bytes;
-    la_status st = check_prefill_shape(dtype, batch, heads, seq, dim, block);
+}  // extern "C"
+
+namespace {
+
+// Shared path of every prefill entry point: shape, variant, pointers, launch.
+la_status prefill_entry(const PrefillArgs &a, void *stream, int variant, bool with_snapshots) {
+    const la_dtype dtype = a.dtype;
+    const int dim = a.dim, block = a.block;
+    la_status st = check_prefill_shape(dtype, a.batch, a.heads, a.seq, dim, block);
     if (st != LA_OK) return st;
     const int chosen = choose_variant(dtype, dim, block, variant);
     if (chosen < 0) {
@@ -194,10 +218,43 @@ la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_d
                     "(CTA pair) (got dtype %d, dim %d, block %d)",
                     (int)dtype, dim, block);
     }
-    PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out};
     st = check_prefill_pointers(a);
     if (st != LA_OK) return st;
+    if (with_snapshots) {
+        st = check_snapshots(a);
+        if (st != LA_OK) return st;
+    }
     return run_prefill(a, static_cast<cudaStream_t>(stream), chosen);
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_dtype dtype,
+                               const float *slopes, int batch, int heads, int seq, int dim, int block,
+                               const float *state_in, void *o, float *state_out, void *workspace,
+                               size_t workspace_bytes, void *stream, int variant) {
+    (void)workspace;
+    (void)workspace_bytes;
+    const PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out,
+                        la::Snapshots{nullptr, 0, 0}};
+    return prefill_entry(a, stream, variant, false);
+}
+
+int lightning_prefill_snapshot_count(int seq, int interval) {
+    if (seq < 0 || interval < 1) return -1;
+    return seq / interval;
+}
+
+la_status lightning_prefill_snapshots(const void *q, const void *k, const void *v, la_dtype dtype,
+                                      const float *slopes, int batch, int heads, int seq, int dim, int block,
+                                      const float *state_in, void *o, float *state_out, int interval,
+                                      float *snapshots, void *stream, int variant) {
+    const int count = interval > 0 && seq >= 0 ? seq / interval : 0;
+    const PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out,
+                        la::Snapshots{count > 0 ? snapshots : nullptr, interval, count}};
+    return prefill_entry(a, stream, variant, true);
 }
 
 la_status lightning_prefill(const void *q, const void *k, const void *v, la_dtype dtype,

@@ -216,7 +216,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_o,
                     const float *__restrict__ slopes, int heads, int seq, const float *state_in,
-                    float *state_out) {
+                    float *state_out, Snapshots sn) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_addr(smem_raw);
     const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -492,8 +492,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // fp16 state operand: K-major rows = value column (l & 63), 64 key dims per box
         uint8_t *srow = c.smem + kOffS + khalf * 8192 + (l & 63) * 128;
         // one 32-value half of this thread's state row: operand copy, optional
-        // state_out, then the decayed value back into TMEM for the next MMA
-        auto carry_half = [&](const float (&sv)[32], int hh, float dnext, bool last) {
+        // prefix-cache snapshot and state_out, then the decayed value back into
+        // TMEM for the next MMA
+        auto carry_half = [&](const float (&sv)[32], int hh, float dnext, bool last, float *snap) {
 #pragma unroll
             for (int cq = 0; cq < 4; ++cq) {
                 const int ch = 4 * hh + cq;
@@ -503,6 +504,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 wv.z = ptx::pack_f16(sv[8 * cq + 4], sv[8 * cq + 5]);
                 wv.w = ptx::pack_f16(sv[8 * cq + 6], sv[8 * cq + 7]);
                 *reinterpret_cast<uint4 *>(srow + ((ch ^ (l & 7)) << 4)) = wv;
+            }
+            if (snap) {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) snap[(size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q];
             }
             if (last) {
                 if (state_out) {
@@ -542,6 +547,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             {
                 const float dnext = last ? 0.f : ptx::ex2(-sl2 * (float)min(kBlock, seq - (t + 1) * kBlock));
+                float *snap = t >= 0 ? snapshot_at(sn, bh, t * kBlock + min(kBlock, seq - t * kBlock), kDim) : nullptr;
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     float sv[32];
@@ -556,7 +562,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         for (int q = 0; q < 32; ++q)
                             sv[q] = state_in ? state_in[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] : 0.f;
                     }
-                    carry_half(sv, hh, dnext, last);
+                    carry_half(sv, hh, dnext, last, snap);
                 }
                 publish(last);
             }
@@ -623,7 +629,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 inline bool pair_supports(bool bf16, int dim, int block) { return bf16 && dim == 128 && block == 256; }
 
 inline la_status launch_pair(const void *q, const void *k, const void *v, const float *slopes, int batch,
-                             int heads, int seq, const float *state_in, void *o, float *state_out,
+                             int heads, int seq, const float *state_in, void *o, float *state_out, Snapshots sn,
                              cudaStream_t stream, std::string *err) {
     const long long bh = (long long)batch * heads;
     CUtensorMap mq, mk, mk64, mv, mo;
@@ -650,7 +656,7 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, pair::prefill_pair_kernel, mq, mk, mk64, mv, mo, slopes, heads, seq, state_in,
-                           state_out);
+                           state_out, sn);
     if (e != cudaSuccess) {
         *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
         return LA_ERR_CUDA;

@@ -44,7 +44,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kSimtThreads)
 prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                     const float *__restrict__ slopes, int heads, int seq, int block,
-                    const float *state_in, T *__restrict__ o, float *state_out) {
+                    const float *state_in, T *__restrict__ o, float *state_out, Snapshots sn) {
     extern __shared__ float smem[];
     float *S = smem;                               // [D][32]
     float *Qs = S + D * kSimtCols;                 // [32][D+1]
@@ -151,6 +151,13 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
             }
         }
         __syncthreads();
+        // prefix-cache snapshot of S after the first t0 + m tokens
+        if (float *snap = snapshot_at(sn, bh, t0 + m, D)) {
+            for (int e = tid; e < D * kSimtCols; e += kSimtThreads) {
+                const int x = e / kSimtCols, c = e % kSimtCols;
+                snap[(size_t)x * D + col0 + c] = S[e];
+            }
+        }
     }
 
     if (state_out) {

@@ -165,7 +165,7 @@ template <int NSUB>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ slopes, int heads,
-                  int seq, const float *state_in, __nv_bfloat16 *o, float *state_out) {
+                  int seq, const float *state_in, __nv_bfloat16 *o, float *state_out, Snapshots sn) {
     constexpr int B = kRows * NSUB;
     constexpr int kLastTile = 2 * NSUB - 2;  // index of the block's last P tile
     extern __shared__ uint8_t smem_raw[];
@@ -585,6 +585,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             ptx::named_bar_sync(kBarWG3, 128);
             if (leader) ptx::mbar_arrive(&c.bars[DS_FREE]);
             write_state_operand();
+            // prefix-cache snapshot of S_t (this thread's key-dim row, its value half)
+            if (float *snap = snapshot_at(sn, bh, t * B + m, kDim)) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    *reinterpret_cast<float4 *>(snap + (size_t)r * kDim + 64 * half + 4 * q) =
+                        make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+            }
 
             // outputs of this block: O (TMEM, fp32) -> bf16 -> global, 32 columns at a time
             for (int sub = 0; sub < NSUB; ++sub) {
@@ -684,7 +691,7 @@ inline bool make_map(CUtensorMap *map, const void *base, int seq, long long bh, 
 
 inline la_status launch_tc(const void *q, const void *k, const void *v, const float *slopes, int batch,
                            int heads, int seq, int block, const float *state_in, void *o, float *state_out,
-                           cudaStream_t stream, std::string *err) {
+                           Snapshots sn, cudaStream_t stream, std::string *err) {
     const long long bh = (long long)batch * heads;
     CUtensorMap mq, mk, mv;
     if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
@@ -697,7 +704,7 @@ inline la_status launch_tc(const void *q, const void *k, const void *v, const fl
         return LA_ERR_CUDA;
     }
     kern<<<(unsigned)(bh * 2), tc::kThreads, tc::kSmemBytes, stream>>>(
-        mq, mk, mv, slopes, heads, seq, state_in, static_cast<__nv_bfloat16 *>(o), state_out);
+        mq, mk, mv, slopes, heads, seq, state_in, static_cast<__nv_bfloat16 *>(o), state_out, sn);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         *err = std::string("prefill_tc launch: ") + cudaGetErrorString(e);

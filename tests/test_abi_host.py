@@ -115,3 +115,47 @@ def test_decode_argument_errors(kw, status):
 
 def test_decode_empty_batch_is_a_no_op():
     assert abi.lightning_decode(Q, K, V, abi.LA_DTYPE_BF16, SL, 0, 4, 128, S1, O, None) == abi.LA_OK
+
+
+SN = 0x10000000 * 9  # fake snapshot buffer address, clear of the others
+
+
+def _prefill_snapshots(interval=256, snapshots=SN, variant=abi.LA_VARIANT_AUTO, **kw):
+    a = dict(GOOD, seq=1024)
+    a.update(kw)
+    return abi.lightning_prefill_snapshots(a["q"], a["k"], a["v"], a["dtype"], a["slopes"], a["batch"],
+                                           a["heads"], a["seq"], a["dim"], a["block"], a["state_in"], a["o"],
+                                           a["state_out"], interval, snapshots, None, variant)
+
+
+def test_snapshot_count():
+    assert abi.lightning_prefill_snapshot_count(1024, 256) == 4
+    assert abi.lightning_prefill_snapshot_count(1000, 256) == 3
+    assert abi.lightning_prefill_snapshot_count(100, 256) == 0
+    assert abi.lightning_prefill_snapshot_count(0, 256) == 0
+    assert abi.lightning_prefill_snapshot_count(-1, 256) == -1
+    assert abi.lightning_prefill_snapshot_count(16, 0) == -1
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(interval=0), abi.LA_ERR_INVALID_ARG),
+    (dict(interval=-256), abi.LA_ERR_INVALID_ARG),
+    (dict(interval=128), abi.LA_ERR_INVALID_ARG),           # shorter than the block
+    (dict(interval=384), abi.LA_ERR_INVALID_ARG),           # not a multiple of the block
+    (dict(snapshots=None), abi.LA_ERR_INVALID_ARG),         # 4 snapshots but no buffer
+    (dict(snapshots=SN + 8), abi.LA_ERR_INVALID_ARG),       # misaligned
+    (dict(snapshots=Q + 4096), abi.LA_ERR_INVALID_ARG),     # overlaps q
+    (dict(snapshots=O), abi.LA_ERR_INVALID_ARG),            # overlaps o
+    (dict(snapshots=S1 - 4096), abi.LA_ERR_INVALID_ARG),    # runs into state_out
+    (dict(dim=96), abi.LA_ERR_UNSUPPORTED),
+    (dict(variant=abi.LA_VARIANT_TCGEN05_PAIR, block=128, interval=128), abi.LA_ERR_UNSUPPORTED),
+])
+def test_snapshot_argument_errors(kw, status):
+    assert _prefill_snapshots(**kw) == status
+    assert abi.last_error_message() != ""
+
+
+def test_snapshot_trivial_calls_need_no_gpu():
+    assert _prefill_snapshots(batch=0) == abi.LA_OK
+    # an empty sequence takes no snapshot, so the buffer may be NULL
+    assert _prefill_snapshots(seq=0, state_out=None, snapshots=None) == abi.LA_OK
