@@ -6,7 +6,8 @@ shares no code with it.
 
 The arithmetic lives in ``lightning_oracle.c`` (three forms of the same
 result: F1 definition, F2 token recurrence, F3 blockwise, plus one decode
-step and the state snapshots of a prefix cache; see that file's header for
+step, the state snapshots of a prefix cache and the gradients of one
+prefill; see that file's header for
 the formulas and their sources on the "MINIMAX SIGNAL LAB · M1" page, §03
 Lightning Attention). This module only
 marshals numpy arrays into it.
@@ -40,6 +41,8 @@ def _load():
         lib.la_oracle_decode.restype = ctypes.c_int
         lib.la_oracle_snapshots.argtypes = [vp, vp, ip, fp, ip, ip, ip, ip, fp, ip, dp]
         lib.la_oracle_snapshots.restype = ctypes.c_int
+        lib.la_oracle_backward.argtypes = [vp, vp, vp, vp, ip, fp, ip, ip, ip, ip, fp, fp, dp, dp, dp, dp]
+        lib.la_oracle_backward.restype = ctypes.c_int
         lib.la_oracle_max_threads.restype = ctypes.c_int
         lib.la_oracle_set_threads.argtypes = [ip]
         _lib = lib
@@ -126,6 +129,28 @@ def snapshots(k, v, slopes, interval, state_in=None):
     if rc != 0:
         raise RuntimeError("oracle snapshots failed (rc=%d)" % rc)
     return out
+
+
+def backward(q, k, v, d_o, slopes, state_in=None, d_state_out=None):
+    """Gradients of one prefill for the loss sum(d_o * o) + sum(d_state_out * state_out).
+
+    Returns float64 (dq, dk, dv, d_state_in)."""
+    q, k, v, code, slopes, state_in, (b, h, L, d) = _prepare(q, k, v, slopes, state_in)
+    d_o = np.ascontiguousarray(d_o)
+    if d_o.shape != q.shape or _dtype_code(d_o) != code:
+        raise ValueError("d_o must match q in shape and dtype")
+    if d_state_out is not None:
+        d_state_out = np.ascontiguousarray(d_state_out, dtype=np.float32)
+        if d_state_out.shape != (b, h, d, d):
+            raise ValueError("d_state_out must have shape [batch, heads, dim, dim]")
+    dq, dk, dv = (np.empty((b, h, L, d), dtype=np.float64) for _ in range(3))
+    ds_in = np.empty((b, h, d, d), dtype=np.float64)
+    rc = _load().la_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(d_o), code, _ptr(slopes), b, h, L, d,
+                                    _ptr(state_in), _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv),
+                                    _ptr(ds_in))
+    if rc != 0:
+        raise RuntimeError("oracle backward failed (rc=%d)" % rc)
+    return dq, dk, dv, ds_in
 
 
 def decode(q, k, v, slopes, state):

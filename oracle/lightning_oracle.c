@@ -33,8 +33,9 @@
  *                             linear attention, fishai.com.cn article on
  *                             M1), O(L d^2) per head; the full-size oracle.
  *   F3 la_oracle_blockwise  : the block formulas of §03 for a given B.
- * plus la_oracle_decode, one recurrent step for a single new token, and
- * la_oracle_snapshots, the state after every `interval` tokens (F2's state).
+ * plus la_oracle_decode, one recurrent step for a single new token,
+ * la_oracle_snapshots, the state after every `interval` tokens (F2's state),
+ * and la_oracle_backward, the gradients of one prefill.
  *
  * Layouts: q, k, v, o are [batch][heads][seq][dim] contiguous (o for decode
  * is [batch][heads][dim]); states are [batch][heads][dim(k)][dim(v)].
@@ -230,6 +231,87 @@ int la_oracle_snapshots(const void *k, const void *v, int dtype, const float *sl
             }
         }
         free(S); free(ki); free(vi);
+    }
+    return fail;
+}
+
+/* Gradients of one prefill, for training through the layer. With the loss
+ * l = sum_i dO_i . o_i + sum dS_out * S_out, and S_i the state after token i
+ * (S_i = e^{-s} S_{i-1} + k_i^T v_i from S_{-1} = S_in, so o_i = q_i S_i and
+ * S_out = S_{L-1}):
+ *   dq_i = dO_i S_i^T
+ *   R_j  = q_j^T dO_j + e^{-s} R_{j+1},  R_{L-1} = q_{L-1}^T dO_{L-1} + dS_out
+ *          (R_j = d l / d S_j: everything token j's outer product k_j^T v_j
+ *          feeds, each later token i seen with e^{-s(i-j)})
+ *   dk_j = R_j v_j,  dv_j = R_j^T k_j
+ *   dS_in = e^{-s} R_0  (= dS_out when L = 0)
+ * Derived from the token-level definition of the forward result
+ * ("MINIMAX SIGNAL LAB · M1", §03 Lightning Attention); the pages print no
+ * backward pass. d_o has the dtype of q, k, v; d_state_out (may be NULL:
+ * zero) and state_in (NULL: zero) are float32; outputs are float64, and
+ * d_state_in may be NULL. */
+int la_oracle_backward(const void *q, const void *k, const void *v, const void *d_o, int dtype,
+                       const float *slopes, int batch, int heads, int seq, int dim,
+                       const float *state_in, const float *d_state_out, double *dq, double *dk,
+                       double *dv, double *d_state_in) {
+    if (check_args(q, k, v, dtype, slopes, batch, heads, seq, dim)) return 1;
+    if (!d_o || !dq || !dk || !dv) return 1;
+    const long BH = (long)batch * heads;
+    const size_t L = (size_t)seq, d = (size_t)dim;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        const int h = (int)(bh % heads);
+        const double decay = exp(-(double)slopes[h]);
+        double *S = malloc(sizeof(double) * d * d);
+        double *R = malloc(sizeof(double) * d * d);
+        double *Q = malloc(sizeof(double) * L * d + 1), *K = malloc(sizeof(double) * L * d + 1);
+        double *V = malloc(sizeof(double) * L * d + 1), *G = malloc(sizeof(double) * L * d + 1);
+        if (!S || !R || !Q || !K || !V || !G) {
+            fail = 1;
+            free(S); free(R); free(Q); free(K); free(V); free(G);
+            continue;
+        }
+        const size_t base = (size_t)bh * L * d;
+        widen_head(q, dtype, base, L * d, Q);
+        widen_head(k, dtype, base, L * d, K);
+        widen_head(v, dtype, base, L * d, V);
+        widen_head(d_o, dtype, base, L * d, G);
+        /* forward sweep: S_i, then dq_i = dO_i S_i^T */
+        for (size_t n = 0; n < d * d; ++n)
+            S[n] = state_in ? (double)state_in[(size_t)bh * d * d + n] : 0.0;
+        for (size_t i = 0; i < L; ++i) {
+            for (size_t r = 0; r < d; ++r)
+                for (size_t c = 0; c < d; ++c) S[r * d + c] = decay * S[r * d + c] + K[i * d + r] * V[i * d + c];
+            for (size_t r = 0; r < d; ++r) {
+                double acc = 0.0;
+                for (size_t c = 0; c < d; ++c) acc += G[i * d + c] * S[r * d + c];
+                dq[base + i * d + r] = acc;
+            }
+        }
+        /* backward sweep: R_j, then dk_j = R_j v_j and dv_j = R_j^T k_j */
+        for (size_t n = 0; n < d * d; ++n)
+            R[n] = d_state_out ? (double)d_state_out[(size_t)bh * d * d + n] : 0.0;
+        for (size_t jj = L; jj-- > 0;) {
+            const double carry = (jj + 1 == L) ? 1.0 : decay;  /* dS_out joins at the last token */
+            for (size_t r = 0; r < d; ++r)
+                for (size_t c = 0; c < d; ++c) R[r * d + c] = carry * R[r * d + c] + Q[jj * d + r] * G[jj * d + c];
+            for (size_t r = 0; r < d; ++r) {
+                double acc = 0.0;
+                for (size_t c = 0; c < d; ++c) acc += R[r * d + c] * V[jj * d + c];
+                dk[base + jj * d + r] = acc;
+            }
+            for (size_t c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (size_t r = 0; r < d; ++r) acc += K[jj * d + r] * R[r * d + c];
+                dv[base + jj * d + c] = acc;
+            }
+        }
+        if (d_state_in) {
+            const double f = L > 0 ? decay : 1.0;
+            for (size_t n = 0; n < d * d; ++n) d_state_in[(size_t)bh * d * d + n] = f * R[n];
+        }
+        free(S); free(R); free(Q); free(K); free(V); free(G);
     }
     return fail;
 }

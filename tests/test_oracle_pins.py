@@ -251,3 +251,47 @@ def test_snapshots_are_the_states_of_the_prefixes(with_state):
     assert oracle.snapshots(k, v, SLOPES_MIX, L + 1, s0).shape == (b, h, 0, d, d)
     _, s_out = oracle.prefill(q, k, v, SLOPES_MIX, s0, form="definition")
     _close(oracle.snapshots(k, v, SLOPES_MIX, L, s0)[:, :, 0], s_out, 1e-12)
+
+
+def _exact_grid(shape, seed, lo=-2.0, hi=2.0):
+    # values on a 1/64 grid: x +- 2^-12 stays exact in float32
+    rng = np.random.default_rng(seed)
+    return (np.round(rng.uniform(lo, hi, shape) * 64) / 64).astype(np.float32)
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_backward_matches_finite_differences_of_the_definition(with_state):
+    # The loss sum(dO * o) + sum(dS_out * S_out) is linear in every single input
+    # element, so a central difference of the definition (F1) is its exact derivative.
+    b, h, L, d = 1, 2, 6, 3
+    sl = np.array([0.25, 1.5], np.float32)
+    q, k, v = (_exact_grid((b, h, L, d), s) for s in (50, 51, 52))
+    s0 = _exact_grid((b, h, d, d), 53) if with_state else None
+    d_o = _rand((b, h, L, d), 54)
+    ds_out = _rand((b, h, d, d), 55)
+    dq, dk, dv, ds_in = oracle.backward(q, k, v, d_o, sl, s0, ds_out)
+
+    def loss(qq, kk, vv, ss):
+        o, st = oracle.prefill(qq, kk, vv, sl, ss, form="definition")
+        return float(np.sum(d_o.astype(np.float64) * o) + np.sum(ds_out.astype(np.float64) * st))
+
+    eps = 2.0 ** -12
+    for name, grad in (("q", dq), ("k", dk), ("v", dv), ("s", ds_in)):
+        for idx in np.ndindex(*grad.shape):
+            args = {"q": q, "k": k, "v": v, "s": s0 if s0 is not None else np.zeros((b, h, d, d), np.float32)}
+            plus = {n: a.copy() for n, a in args.items()}
+            minus = {n: a.copy() for n, a in args.items()}
+            plus[name][idx] += eps
+            minus[name][idx] -= eps
+            fd = (loss(plus["q"], plus["k"], plus["v"], plus["s"]) -
+                  loss(minus["q"], minus["k"], minus["v"], minus["s"])) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-9 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+
+
+def test_backward_of_an_empty_sequence_passes_the_state_gradient():
+    b, h, d = 1, 2, 3
+    z = np.zeros((b, h, 0, d), np.float32)
+    ds_out = _rand((b, h, d, d), 56)
+    dq, dk, dv, ds_in = oracle.backward(z, z, z, z, SLOPES_MIX[:2], None, ds_out)
+    assert dq.shape == (b, h, 0, d)
+    np.testing.assert_array_equal(ds_in, ds_out.astype(np.float64))
