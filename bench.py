@@ -344,6 +344,9 @@ def run_ours(args):
     snaps = (run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, ms_per_step)
              if args.snapshot_interval > 0 and w.seq >= args.snapshot_interval else None)
 
+    # gradients of the same prefill (dq, dk, dv, d state_in)
+    bwd = run_backward_leg(w, dev, stream, inp, dcode, args, world) if args.backward_steps > 0 else None
+
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -362,6 +365,7 @@ def run_ours(args):
         "decode": dec,
         "e2e": e2e,
         "snapshots": snaps,
+        "backward": bwd,
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
     }
@@ -446,6 +450,53 @@ def run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, plain_ms):
             "snapshot_bytes_per_step": int(snaps.numel() * 4)}
 
 
+def fp32_cuda_core_peak_tflops(sm_mhz=1965.0):
+    """fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP per clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def run_backward_leg(w, dev, stream, inp, dcode, args, world):
+    """lightning_prefill_backward on the workload, timed like the main leg:
+    three CUDA-core passes of the block recurrence (dQ forward in time, dV and
+    dK backward), fp32 arithmetic."""
+    import torch
+    from linear_attention_lightning_b200 import abi
+    q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
+    g = torch.Generator(device=dev).manual_seed(w.seed + 1000)
+    d_o = torch.randn(q.shape, generator=g, device=dev).to(q.dtype)
+    d_so = torch.randn((w.batch, w.heads, w.dim, w.dim), generator=g, device=dev) * 0.1
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ds_in = torch.empty_like(d_so)
+    sp = stream.cuda_stream
+
+    def step():
+        abi.check(abi.lightning_prefill_backward(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), d_o.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads,
+            w.seq, w.dim, w.block, None if s0 is None else s0.data_ptr(), d_so.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), ds_in.data_ptr(), sp))
+
+    for _ in range(args.warmup):
+        step()
+    steps = args.backward_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    # each pass is one prefill recurrence: 4Bd + 4d^2 FLOPs per (token, head), formula convention
+    flops = 3 * prefill_flops(w.batch, w.heads, w.seq, w.dim, w.block)["formula"]
+    peak = fp32_cuda_core_peak_tflops()
+    tf = flops / (ms / 1e3) / 1e12
+    return {"kernel": "simt (3 passes)", "steps": steps, "ms_per_step": round(ms, 3),
+            "tokens_per_s": round(world * w.batch * w.seq / (ms / 1e3), 1),
+            "roofline": roofline("alu", tf, round(peak, 1), "TFLOP/s"),
+            "note": "fp32 CUDA-core peak derived as 148 SMs x 128 lanes x 2 FLOP x 1965 MHz"}
+
+
 def run_e2e(w, dev, stream, inp, variant, args, world):
     """Same prefill through the public API with host buffers: every step copies
     q, k, v from pinned host memory and reads o and the state back."""
@@ -494,6 +545,8 @@ def parse_args(argv=None):
     p.add_argument("--decode-steps", type=int, default=1000)
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--backward-steps", type=int, default=2,
+                   help="timed steps of the gradient leg (0 skips it)")
     p.add_argument("--snapshot-interval", type=int, default=16384,
                    help="tokens between prefix-cache state snapshots in the snapshot leg (0 skips it)")
     a = p.parse_args(argv)

@@ -146,6 +146,35 @@ la_status lightning_prefill_snapshots(const void *q, const void *k, const void *
                                       int block, const float *state_in, void *o, float *state_out,
                                       int interval, float *snapshots, void *stream, int variant);
 
+/*
+ * Gradients of one prefill, for training through the layer. The pages print
+ * no backward pass; this is the derivative of the operation defined in
+ * "MINIMAX SIGNAL LAB · M1", §03 Lightning Attention (the token-level result
+ * above). For the loss  sum_i dO_i . o_i + sum dS_out * S_out, with S_i the
+ * state after token i (o_i = q_i S_i):
+ *   dq_i  = dO_i S_i^T
+ *   R_j   = sum_{i>=j} e^{-s(i-j)} q_i^T dO_i + e^{-s(L-1-j)} dS_out
+ *   dk_j  = R_j v_j,   dv_j = R_j^T k_j,   dS_in = e^{-s} R_0 (dS_out if L = 0)
+ * computed blockwise as three passes of the prefill recurrence on permuted
+ * operands: dQ forward in time on (dO, V, K) with state S^T; dV and dK
+ * backward in time on (K, Q, dO) and (V, dO, Q) with state R. CUDA cores,
+ * fp32 arithmetic, any block, dim 64 or 128.
+ *
+ *   q, k, v, d_o  [batch][heads][seq][dim], dtype; read only.
+ *   state_in      as for lightning_prefill (NULL: zeros).
+ *   d_state_out   [batch][heads][dim][dim] float32 gradient of state_out, or
+ *                 NULL for zeros.
+ *   dq, dk, dv    [batch][heads][seq][dim], dtype; written.
+ *   d_state_in    [batch][heads][dim][dim] float32, or NULL to skip.
+ * All device pointers, caller-owned, 16-byte aligned. No output may overlap
+ * an input or another output (LA_ERR_INVALID_ARG). Shape rules as for
+ * lightning_prefill.
+ */
+la_status lightning_prefill_backward(const void *q, const void *k, const void *v, const void *d_o,
+                                     la_dtype dtype, const float *slopes, int batch, int heads, int seq,
+                                     int dim, int block, const float *state_in, const float *d_state_out,
+                                     void *dq, void *dk, void *dv, float *d_state_in, void *stream);
+
 /* Number of snapshots lightning_prefill_snapshots writes per (batch, head):
  * seq / interval, or -1 if seq < 0 or interval < 1. Host only. */
 int lightning_prefill_snapshot_count(int seq, int interval);

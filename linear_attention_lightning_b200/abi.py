@@ -30,6 +30,8 @@ _SIGNATURES = {
     "lightning_prefill_snapshots": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp,
                                      _i], _i),
     "lightning_prefill_snapshot_count": ([_i, _i], _i),
+    "lightning_prefill_backward": ([_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                                    _vp, _vp], _i),
     "lightning_decode": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp], _i),
     "lightning_device_status": ([_vp], _i),
     "lightning_status_string": ([_i], ctypes.c_char_p),
@@ -111,6 +113,12 @@ def lightning_prefill_snapshots(q, k, v, dtype, slopes, batch, heads, seq, dim, 
                                 interval, snapshots, stream, variant):
     return load().lightning_prefill_snapshots(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in,
                                               o, state_out, interval, snapshots, stream, variant)
+
+
+def lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in,
+                               d_state_out, dq, dk, dv, d_state_in, stream):
+    return load().lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block,
+                                             state_in, d_state_out, dq, dk, dv, d_state_in, stream)
 
 
 def lightning_prefill_snapshot_count(seq, interval):

@@ -101,6 +101,33 @@ def prefill_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes:
     return o, state_out, snapshots
 
 
+def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, d_o: torch.Tensor, slopes: torch.Tensor,
+                     block: int, state_in: Optional[torch.Tensor] = None,
+                     d_state_out: Optional[torch.Tensor] = None, want_state_grad: bool = True,
+                     stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """lightning_prefill_backward: returns (dq, dk, dv, d_state_in) for the loss
+    sum(d_o * o) + sum(d_state_out * state_out)."""
+    if q.dtype not in _DTYPES:
+        raise ValueError("q must be float32 or bfloat16")
+    if q.dim() != 4 or any(t.shape != q.shape for t in (k, v, d_o)):
+        raise ValueError("q, k, v, d_o must share one [batch, heads, seq, dim] shape")
+    for name, t in (("q", q), ("k", k), ("v", v), ("d_o", d_o)):
+        _need_cuda(name, t, q.dtype)
+    b, h, L, d = q.shape
+    _need_cuda("slopes", slopes, torch.float32)
+    for name, t in (("state_in", state_in), ("d_state_out", d_state_out)):
+        if t is not None:
+            _need_cuda(name, t, torch.float32)
+            if tuple(t.shape) != (b, h, d, d):
+                raise ValueError("%s must be [batch, heads, dim, dim]" % name)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ds_in = torch.empty((b, h, d, d), dtype=torch.float32, device=q.device) if want_state_grad else None
+    abi.check(abi.lightning_prefill_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(d_o), _DTYPES[q.dtype], _ptr(slopes), b, h, L, d, int(block),
+        _ptr(state_in), _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds_in), _stream(stream)))
+    return dq, dk, dv, ds_in
+
+
 def prefill_variant(dtype: torch.dtype, batch: int, heads: int, seq: int, dim: int, block: int,
                     variant: str = "auto") -> str:
     """Which kernel lightning_prefill would run: "simt", "tcgen05" or "pair"."""

@@ -155,10 +155,102 @@ la_status launch_simt(const PrefillArgs &a, cudaStream_t stream) {
     dim3 grid((unsigned)((size_t)a.batch * a.heads * (D / la::kSimtCols)));
     kern<<<grid, la::kSimtThreads, smem, stream>>>(
         static_cast<const T *>(a.q), static_cast<const T *>(a.k), static_cast<const T *>(a.v),
-        a.slopes, a.heads, a.seq, a.block, a.state_in, static_cast<T *>(a.o), a.state_out, a.sn);
+        a.slopes, a.heads, a.seq, a.block, a.state_in, static_cast<T *>(a.o), a.state_out, a.sn,
+        la::SimtPass{0, 0, 0, 0});
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prefill_simt launch");
     return ok();
+}
+
+// One launch of the CUDA-core kernel as a pass of the backward computation.
+template <typename T, int D>
+la_status launch_simt_pass(const void *q, const void *k, const void *v, const float *slopes, int batch,
+                           int heads, int seq, int block, const float *state_in, void *o, float *state_out,
+                           la::SimtPass pass, cudaStream_t stream) {
+    auto kern = la::prefill_simt_kernel<T, D, true>;
+    const size_t smem = la::simt_smem_bytes<D>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_simt pass)");
+    dim3 grid((unsigned)((size_t)batch * heads * (D / la::kSimtCols)));
+    kern<<<grid, la::kSimtThreads, smem, stream>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), slopes, heads, seq,
+        block, state_in, static_cast<T *>(o), state_out, la::Snapshots{nullptr, 0, 0}, pass);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "prefill_simt pass launch");
+    return ok();
+}
+
+struct BackwardArgs {
+    const void *q, *k, *v, *d_o;
+    la_dtype dtype;
+    const float *slopes;
+    int batch, heads, seq, dim, block;
+    const float *state_in, *d_state_out;
+    void *dq, *dk, *dv;
+    float *d_state_in;
+};
+
+la_status check_backward_pointers(const BackwardArgs &a) {
+    const size_t eb = elem_bytes(a.dtype);
+    const size_t n_tok = (size_t)a.batch * a.heads * a.seq * a.dim;
+    const size_t n_state = (size_t)a.batch * a.heads * a.dim * a.dim;
+    if (a.seq > 0 && (!a.q || !a.k || !a.v || !a.d_o || !a.dq || !a.dk || !a.dv))
+        return fail(LA_ERR_INVALID_ARG, "q, k, v, d_o, dq, dk and dv must be non-NULL when seq > 0");
+    if (!a.slopes) return fail(LA_ERR_INVALID_ARG, "slopes must be non-NULL");
+    const void *ptrs[] = {a.q, a.k, a.v, a.d_o, a.slopes, a.state_in, a.d_state_out, a.dq, a.dk, a.dv,
+                          a.d_state_in};
+    const char *names[] = {"q", "k", "v", "d_o", "slopes", "state_in", "d_state_out", "dq", "dk", "dv",
+                           "d_state_in"};
+    for (int i = 0; i < 11; ++i)
+        if (ptrs[i] && !aligned16(ptrs[i])) return fail(LA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+    const size_t tok = a.seq > 0 ? n_tok * eb : 0;
+    const Range in[] = {range_of(a.q, tok), range_of(a.k, tok), range_of(a.v, tok), range_of(a.d_o, tok),
+                        range_of(a.slopes, sizeof(float) * a.heads),
+                        range_of(a.state_in, a.state_in ? n_state * 4 : 0),
+                        range_of(a.d_state_out, a.d_state_out ? n_state * 4 : 0)};
+    const Range out[] = {range_of(a.dq, tok), range_of(a.dk, tok), range_of(a.dv, tok),
+                         range_of(a.d_state_in, a.d_state_in ? n_state * 4 : 0)};
+    for (int i = 0; i < 4; ++i) {
+        for (const Range &r : in)
+            if (overlaps(out[i], r)) return fail(LA_ERR_INVALID_ARG, "a gradient output overlaps an input");
+        for (int j = i + 1; j < 4; ++j)
+            if (overlaps(out[i], out[j])) return fail(LA_ERR_INVALID_ARG, "two gradient outputs overlap");
+    }
+    return LA_OK;
+}
+
+// The gradients as three passes of the block recurrence (see lightning.h):
+//   dQ: forward in time, (q, k, v) <- (dO, V, K), carried state S_in^T;
+//   dV: backward in time, (q, k, v) <- (K, Q, dO), carried state dS_out seen
+//       from the last token on, final state times e^{-s} = dS_in;
+//   dK: backward in time, (q, k, v) <- (V, dO, Q), carried state dS_out^T.
+template <typename T, int D>
+la_status run_backward_typed(const BackwardArgs &a, cudaStream_t stream) {
+    la_status st = launch_simt_pass<T, D>(a.d_o, a.v, a.k, a.slopes, a.batch, a.heads, a.seq, a.block, a.state_in,
+                                          a.dq, nullptr, la::SimtPass{0, 1, 0, 0}, stream);
+    if (st != LA_OK) return st;
+    st = launch_simt_pass<T, D>(a.k, a.q, a.d_o, a.slopes, a.batch, a.heads, a.seq, a.block, a.d_state_out,
+                                a.dv, a.d_state_in, la::SimtPass{1, 0, 1, 1}, stream);
+    if (st != LA_OK) return st;
+    return launch_simt_pass<T, D>(a.v, a.d_o, a.q, a.slopes, a.batch, a.heads, a.seq, a.block, a.d_state_out,
+                                  a.dk, nullptr, la::SimtPass{1, 1, 1, 0}, stream);
+}
+
+la_status run_backward(const BackwardArgs &a, cudaStream_t stream) {
+    if (a.batch == 0) return ok();
+    if (a.seq == 0) {
+        // no token: the state passes through, and so does its gradient
+        if (!a.d_state_in) return ok();
+        const size_t n = (size_t)a.batch * a.heads * a.dim * a.dim;
+        la::state_passthrough_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0,
+                                       stream>>>(a.d_state_out, a.d_state_in, n);
+        cudaError_t e = cudaGetLastError();
+        return e == cudaSuccess ? ok() : cuda_fail(e, "state gradient passthrough launch");
+    }
+    if (a.dtype == LA_DTYPE_BF16)
+        return a.dim == 64 ? run_backward_typed<__nv_bfloat16, 64>(a, stream)
+                           : run_backward_typed<__nv_bfloat16, 128>(a, stream);
+    return a.dim == 64 ? run_backward_typed<float, 64>(a, stream) : run_backward_typed<float, 128>(a, stream);
 }
 
 la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
@@ -240,6 +332,19 @@ la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_d
     const PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out,
                         la::Snapshots{nullptr, 0, 0}};
     return prefill_entry(a, stream, variant, false);
+}
+
+la_status lightning_prefill_backward(const void *q, const void *k, const void *v, const void *d_o,
+                                     la_dtype dtype, const float *slopes, int batch, int heads, int seq,
+                                     int dim, int block, const float *state_in, const float *d_state_out,
+                                     void *dq, void *dk, void *dv, float *d_state_in, void *stream) {
+    la_status st = check_prefill_shape(dtype, batch, heads, seq, dim, block);
+    if (st != LA_OK) return st;
+    const BackwardArgs a{q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in, d_state_out,
+                         dq, dk, dv, d_state_in};
+    st = check_backward_pointers(a);
+    if (st != LA_OK) return st;
+    return run_backward(a, static_cast<cudaStream_t>(stream));
 }
 
 int lightning_prefill_snapshot_count(int seq, int interval) {

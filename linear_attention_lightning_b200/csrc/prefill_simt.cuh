@@ -30,21 +30,35 @@ constexpr size_t simt_smem_bytes() {
                             + kSimtRows * (kSimtRows + 1));  // P chunk
 }
 
+// How one launch maps its tokens and states. The forward prefill is the
+// identity pass. The gradients of a prefill are the same block recurrence on
+// permuted operands (lightning_api.cu): the dQ pass runs forward with the
+// carried state transposed, the dK and dV passes run backward in time with
+// the state gradient seen from the last token on.
+struct SimtPass {
+    int reverse;         // 1: visit tokens from the last to the first
+    int state_in_t;      // 1: state_in holds the transpose of the carried state
+    int state_shift;     // 1: the first visited token sees the carried state with e^0, not e^{-s}
+    int state_out_step;  // 1: write e^{-s} times the final state
+};
+
 // Copy `rows` rows (zero-filled up to kSimtRows) of a [*, D] row-major tensor
-// into shared memory with padded row stride D+1.
+// into shared memory with padded row stride D+1; source row r is at
+// src + r * stride (stride -D walks backward).
 template <typename T, int D>
-__device__ __forceinline__ void simt_load_rows(float *dst, const T *src, int rows) {
+__device__ __forceinline__ void simt_load_rows(float *dst, const T *src, int rows, long stride = D) {
     for (int e = threadIdx.x; e < kSimtRows * D; e += kSimtThreads) {
         const int r = e / D, c = e % D;
-        dst[r * (D + 1) + c] = (r < rows) ? to_f32(src[(size_t)r * D + c]) : 0.f;
+        dst[r * (D + 1) + c] = (r < rows) ? to_f32(src[(long)r * stride + c]) : 0.f;
     }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kGeneral = false>
 __global__ void __launch_bounds__(kSimtThreads)
 prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                     const float *__restrict__ slopes, int heads, int seq, int block,
-                    const float *state_in, T *__restrict__ o, float *state_out, Snapshots sn) {
+                    const float *state_in, T *__restrict__ o, float *state_out, Snapshots sn,
+                    SimtPass pass) {
     extern __shared__ float smem[];
     float *S = smem;                               // [D][32]
     float *Qs = S + D * kSimtCols;                 // [32][D+1]
@@ -61,6 +75,12 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
     const T *vh = v + bh * seq * D;
     T *oh = o + bh * seq * D;
 
+    // token x of the visiting order lives in row prow(x) of the tensors
+    const bool rev = kGeneral && pass.reverse;
+    auto prow = [&](int x) -> long { return rev ? (long)seq - 1 - x : (long)x; };
+    const long rstride = rev ? -(long)D : (long)D;
+    const float shift = kGeneral ? (float)pass.state_shift : 0.f;
+
     const int tid = threadIdx.x;
     // output / P mapping: row r, four adjacent columns starting at c4
     const int r = tid / 8, c4 = (tid % 8) * 4;
@@ -69,7 +89,8 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
 
     for (int e = tid; e < D * kSimtCols; e += kSimtThreads) {
         const int x = e / kSimtCols, c = e % kSimtCols;
-        S[e] = state_in ? state_in[bh * D * D + (size_t)x * D + col0 + c] : 0.f;
+        const size_t at = (kGeneral && pass.state_in_t) ? (size_t)(col0 + c) * D + x : (size_t)x * D + col0 + c;
+        S[e] = state_in ? state_in[bh * D * D + at] : 0.f;
     }
     __syncthreads();
 
@@ -77,7 +98,7 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
         const int m = min(block, seq - t0);
         for (int i0 = 0; i0 < m; i0 += kSimtRows) {
             const int rows_q = min(kSimtRows, m - i0);
-            simt_load_rows<T, D>(Qs, qh + (size_t)(t0 + i0) * D, rows_q);
+            simt_load_rows<T, D>(Qs, qh + prow(t0 + i0) * D, rows_q, rstride);
             __syncthreads();
 
             // inter-block term: (q_i ⊙ d_q) S_{t-1}
@@ -87,7 +108,7 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
                 const float4 sv = *reinterpret_cast<const float4 *>(&S[x * kSimtCols + c4]);
                 acc[0] += qv * sv.x; acc[1] += qv * sv.y; acc[2] += qv * sv.z; acc[3] += qv * sv.w;
             }
-            const float dq = decay_pow(s, (float)(i0 + r + 1));
+            const float dq = decay_pow(s, (float)(i0 + r + 1) - (t0 == 0 ? shift : 0.f));
             for (int u = 0; u < 4; ++u) acc[u] *= dq;
 
             // intra-block term over key chunks j0 <= last query row of this chunk
@@ -95,10 +116,10 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
             for (int j0 = 0; j0 <= last_i; j0 += kSimtRows) {
                 const int rows_k = min(kSimtRows, m - j0);
                 __syncthreads();  // previous users of Ks / Vs / Ps are done
-                simt_load_rows<T, D>(Ks, kh + (size_t)(t0 + j0) * D, rows_k);
+                simt_load_rows<T, D>(Ks, kh + prow(t0 + j0) * D, rows_k, rstride);
                 for (int e = tid; e < kSimtRows * kSimtCols; e += kSimtThreads) {
                     const int jr = e / kSimtCols, c = e % kSimtCols;
-                    Vs[e] = (jr < rows_k) ? to_f32(vh[(size_t)(t0 + j0 + jr) * D + col0 + c]) : 0.f;
+                    Vs[e] = (jr < rows_k) ? to_f32(vh[prow(t0 + j0 + jr) * D + col0 + c]) : 0.f;
                 }
                 __syncthreads();
                 // P[r][j] = (q_i . k_j) e^{-s(i-j)} 1[i>=j], four keys per thread
@@ -118,14 +139,14 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
                 }
             }
             if (r < rows_q) {
-                T *dst = oh + (size_t)(t0 + i0 + r) * D + col0 + c4;
+                T *dst = oh + prow(t0 + i0 + r) * D + col0 + c4;
                 for (int u = 0; u < 4; ++u) dst[u] = from_f32<T>(acc[u]);
             }
             __syncthreads();
         }
 
         // state update: S_t = e^{-s m} S_{t-1} + (K_t ⊙ d_k)^T V_t
-        const float dblock = decay_pow(s, (float)m);
+        const float dblock = decay_pow(s, (float)m - (t0 == 0 ? shift : 0.f));
         for (int u = 0; u < kStateRowsPerThread; ++u) {
             const int x = tid / 8 + 32 * u;
             for (int c = 0; c < 4; ++c) S[x * kSimtCols + c4 + c] *= dblock;
@@ -133,10 +154,10 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
         for (int j0 = 0; j0 < m; j0 += kSimtRows) {
             const int rows_k = min(kSimtRows, m - j0);
             __syncthreads();
-            simt_load_rows<T, D>(Ks, kh + (size_t)(t0 + j0) * D, rows_k);
+            simt_load_rows<T, D>(Ks, kh + prow(t0 + j0) * D, rows_k, rstride);
             for (int e = tid; e < kSimtRows * kSimtCols; e += kSimtThreads) {
                 const int jr = e / kSimtCols, c = e % kSimtCols;
-                Vs[e] = (jr < rows_k) ? to_f32(vh[(size_t)(t0 + j0 + jr) * D + col0 + c]) : 0.f;
+                Vs[e] = (jr < rows_k) ? to_f32(vh[prow(t0 + j0 + jr) * D + col0 + c]) : 0.f;
             }
             __syncthreads();
             for (int jj = 0; jj < rows_k; ++jj) {
@@ -161,9 +182,10 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
     }
 
     if (state_out) {
+        const float fo = (kGeneral && pass.state_out_step) ? decay_pow(s, 1.f) : 1.f;
         for (int e = tid; e < D * kSimtCols; e += kSimtThreads) {
             const int x = e / kSimtCols, c = e % kSimtCols;
-            state_out[bh * D * D + (size_t)x * D + col0 + c] = S[e];
+            state_out[bh * D * D + (size_t)x * D + col0 + c] = fo * S[e];
         }
     }
 }

@@ -159,3 +159,38 @@ def test_snapshot_trivial_calls_need_no_gpu():
     assert _prefill_snapshots(batch=0) == abi.LA_OK
     # an empty sequence takes no snapshot, so the buffer may be NULL
     assert _prefill_snapshots(seq=0, state_out=None, snapshots=None) == abi.LA_OK
+
+
+DO, DQ, DK, DV, DSI, DSO = (0x10000000 * (i + 10) for i in range(6))
+
+
+def _backward(**kw):
+    a = dict(GOOD, d_o=DO, d_state_out=DSO, dq=DQ, dk=DK, dv=DV, d_state_in=DSI)
+    a.update(kw)
+    return abi.lightning_prefill_backward(a["q"], a["k"], a["v"], a["d_o"], a["dtype"], a["slopes"], a["batch"],
+                                          a["heads"], a["seq"], a["dim"], a["block"], a["state_in"],
+                                          a["d_state_out"], a["dq"], a["dk"], a["dv"], a["d_state_in"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype=5), abi.LA_ERR_INVALID_ARG),
+    (dict(block=0), abi.LA_ERR_INVALID_ARG),
+    (dict(dim=48), abi.LA_ERR_UNSUPPORTED),
+    (dict(d_o=None), abi.LA_ERR_INVALID_ARG),
+    (dict(dk=None), abi.LA_ERR_INVALID_ARG),
+    (dict(slopes=None), abi.LA_ERR_INVALID_ARG),
+    (dict(dv=DV + 4), abi.LA_ERR_INVALID_ARG),           # misaligned
+    (dict(dq=Q + 512), abi.LA_ERR_INVALID_ARG),          # output overlaps q
+    (dict(dk=DO), abi.LA_ERR_INVALID_ARG),               # output overlaps d_o
+    (dict(dv=DQ + 1024), abi.LA_ERR_INVALID_ARG),        # two outputs overlap
+    (dict(d_state_in=DSO), abi.LA_ERR_INVALID_ARG),      # overlaps d_state_out
+    (dict(d_state_in=S0 + 16), abi.LA_ERR_INVALID_ARG),  # overlaps state_in
+])
+def test_backward_argument_errors(kw, status):
+    assert _backward(**kw) == status
+    assert abi.last_error_message() != ""
+
+
+def test_backward_trivial_calls_need_no_gpu():
+    assert _backward(batch=0) == abi.LA_OK
+    assert _backward(seq=0, d_state_in=None) == abi.LA_OK
