@@ -450,15 +450,10 @@ def run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, plain_ms):
             "snapshot_bytes_per_step": int(snaps.numel() * 4)}
 
 
-def fp32_cuda_core_peak_tflops(sm_mhz=1965.0):
-    """fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP per clock."""
-    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
-
-
 def run_backward_leg(w, dev, stream, inp, dcode, args, world):
-    """lightning_prefill_backward on the workload, timed like the main leg:
-    three CUDA-core passes of the block recurrence (dQ forward in time, dV and
-    dK backward), fp32 arithmetic."""
+    """lightning_prefill_backward on the workload (AUTO: the CTA-pair tensor-core
+    kernels where they apply), timed like the main leg: dQ on (dO, V, K), dV and
+    dK on token-reversed copies, plus the reversals."""
     import torch
     from linear_attention_lightning_b200 import abi
     q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
@@ -467,13 +462,16 @@ def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     d_so = torch.randn((w.batch, w.heads, w.dim, w.dim), generator=g, device=dev) * 0.1
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     ds_in = torch.empty_like(d_so)
+    variant = abi.LA_VARIANT_AUTO
+    need = abi.lightning_prefill_backward_workspace_size(dcode, w.batch, w.heads, w.seq, w.dim, w.block, variant)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     sp = stream.cuda_stream
 
     def step():
         abi.check(abi.lightning_prefill_backward(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), d_o.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads,
             w.seq, w.dim, w.block, None if s0 is None else s0.data_ptr(), d_so.data_ptr(), dq.data_ptr(),
-            dk.data_ptr(), dv.data_ptr(), ds_in.data_ptr(), sp))
+            dk.data_ptr(), dv.data_ptr(), ds_in.data_ptr(), ws.data_ptr(), need, sp, variant))
 
     for _ in range(args.warmup):
         step()
@@ -487,14 +485,22 @@ def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
-    # each pass is one prefill recurrence: 4Bd + 4d^2 FLOPs per (token, head), formula convention
-    flops = 3 * prefill_flops(w.batch, w.heads, w.seq, w.dim, w.block)["formula"]
-    peak = fp32_cuda_core_peak_tflops()
-    tf = flops / (ms / 1e3) / 1e12
-    return {"kernel": "simt (3 passes)", "steps": steps, "ms_per_step": round(ms, 3),
+    peaks = load_peaks()
+    eb = 2 if q.dtype == torch.bfloat16 else 4
+    # algorithmic bytes: q, k, v, dO read and dq, dk, dv written once, plus the
+    # fp32 states (state_in, d_state_out read, d_state_in written)
+    units = w.batch * w.heads * w.seq
+    by = 7 * units * w.dim * eb + 3 * w.batch * w.heads * w.dim * w.dim * 4
+    gbs = by / (ms / 1e3) / 1e9
+    # three passes of the block recurrence: 3 x (4Bd + 4d^2) per (token, head)
+    tf = 3 * prefill_flops(w.batch, w.heads, w.seq, w.dim, w.block)["formula"] / (ms / 1e3) / 1e12
+    kernel = "pair (3 passes + token reversals)" if need > 0 else "simt (3 passes)"
+    return {"kernel": kernel, "steps": steps, "ms_per_step": round(ms, 3),
             "tokens_per_s": round(world * w.batch * w.seq / (ms / 1e3), 1),
-            "roofline": roofline("alu", tf, round(peak, 1), "TFLOP/s"),
-            "note": "fp32 CUDA-core peak derived as 148 SMs x 128 lanes x 2 FLOP x 1965 MHz"}
+            "workspace_bytes": need,
+            "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s"),
+            "tflops_formula": round(tf, 2),
+            "frac_bf16_peak_formula": round(tf / peaks["bf16_tflops"], 4)}
 
 
 def run_e2e(w, dev, stream, inp, variant, args, world):
@@ -545,7 +551,7 @@ def parse_args(argv=None):
     p.add_argument("--decode-steps", type=int, default=1000)
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--backward-steps", type=int, default=2,
+    p.add_argument("--backward-steps", type=int, default=10,
                    help="timed steps of the gradient leg (0 skips it)")
     p.add_argument("--snapshot-interval", type=int, default=16384,
                    help="tokens between prefix-cache state snapshots in the snapshot leg (0 skips it)")

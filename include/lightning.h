@@ -157,8 +157,13 @@ la_status lightning_prefill_snapshots(const void *q, const void *k, const void *
  *   dk_j  = R_j v_j,   dv_j = R_j^T k_j,   dS_in = e^{-s} R_0 (dS_out if L = 0)
  * computed blockwise as three passes of the prefill recurrence on permuted
  * operands: dQ forward in time on (dO, V, K) with state S^T; dV and dK
- * backward in time on (K, Q, dO) and (V, dO, Q) with state R. CUDA cores,
- * fp32 arithmetic, any block, dim 64 or 128.
+ * backward in time on (K, Q, dO) and (V, dO, Q) with state R.
+ * Kernels (variant): LA_VARIANT_TCGEN05_PAIR runs the passes on the CTA-pair
+ * tensor-core kernel (bf16, dim 128, block 256; the backward-in-time passes
+ * read token-reversed operand copies kept in the workspace);
+ * LA_VARIANT_SIMT runs them on CUDA cores in fp32 (any dtype, dim 64 or 128,
+ * any block, no workspace); LA_VARIANT_AUTO takes the tensor-core kernels
+ * where they apply. LA_VARIANT_TCGEN05 is not a backward variant.
  *
  *   q, k, v, d_o  [batch][heads][seq][dim], dtype; read only.
  *   state_in      as for lightning_prefill (NULL: zeros).
@@ -166,14 +171,25 @@ la_status lightning_prefill_snapshots(const void *q, const void *k, const void *
  *                 NULL for zeros.
  *   dq, dk, dv    [batch][heads][seq][dim], dtype; written.
  *   d_state_in    [batch][heads][dim][dim] float32, or NULL to skip.
+ *   workspace, workspace_bytes
+ *                 scratch of at least lightning_prefill_backward_workspace_size
+ *                 bytes (0 for the CUDA-core kernels), 16-byte aligned,
+ *                 overlapping nothing else; contents undefined afterwards.
  * All device pointers, caller-owned, 16-byte aligned. No output may overlap
- * an input or another output (LA_ERR_INVALID_ARG). Shape rules as for
- * lightning_prefill.
+ * an input or another output; a short or overlapping workspace is rejected
+ * (all LA_ERR_INVALID_ARG). Shape rules as for lightning_prefill.
  */
 la_status lightning_prefill_backward(const void *q, const void *k, const void *v, const void *d_o,
                                      la_dtype dtype, const float *slopes, int batch, int heads, int seq,
                                      int dim, int block, const float *state_in, const float *d_state_out,
-                                     void *dq, void *dk, void *dv, float *d_state_in, void *stream);
+                                     void *dq, void *dk, void *dv, float *d_state_in, void *workspace,
+                                     size_t workspace_bytes, void *stream, int variant);
+
+/* Bytes of workspace lightning_prefill_backward needs for these arguments
+ * (three copies of a [batch][heads][seq][dim] tensor for the tensor-core
+ * kernels, 0 for the CUDA-core ones or an invalid request). Host only. */
+size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int heads, int seq, int dim,
+                                                 int block, int variant);
 
 /* Number of snapshots lightning_prefill_snapshots writes per (batch, head):
  * seq / interval, or -1 if seq < 0 or interval < 1. Host only. */

@@ -31,7 +31,8 @@ _SIGNATURES = {
                                      _i], _i),
     "lightning_prefill_snapshot_count": ([_i, _i], _i),
     "lightning_prefill_backward": ([_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
-                                    _vp, _vp], _i),
+                                    _vp, _vp, _sz, _vp, _i], _i),
+    "lightning_prefill_backward_workspace_size": ([_i, _i, _i, _i, _i, _i, _i], _sz),
     "lightning_decode": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp], _i),
     "lightning_device_status": ([_vp], _i),
     "lightning_status_string": ([_i], ctypes.c_char_p),
@@ -116,9 +117,14 @@ def lightning_prefill_snapshots(q, k, v, dtype, slopes, batch, heads, seq, dim, 
 
 
 def lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in,
-                               d_state_out, dq, dk, dv, d_state_in, stream):
+                               d_state_out, dq, dk, dv, d_state_in, workspace, workspace_bytes, stream, variant):
     return load().lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block,
-                                             state_in, d_state_out, dq, dk, dv, d_state_in, stream)
+                                             state_in, d_state_out, dq, dk, dv, d_state_in, workspace,
+                                             workspace_bytes, stream, variant)
+
+
+def lightning_prefill_backward_workspace_size(dtype, batch, heads, seq, dim, block, variant):
+    return load().lightning_prefill_backward_workspace_size(dtype, batch, heads, seq, dim, block, variant)
 
 
 def lightning_prefill_snapshot_count(seq, interval):

@@ -104,13 +104,17 @@ def prefill_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes:
 def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, d_o: torch.Tensor, slopes: torch.Tensor,
                      block: int, state_in: Optional[torch.Tensor] = None,
                      d_state_out: Optional[torch.Tensor] = None, want_state_grad: bool = True,
+                     variant: str = "auto", workspace: Optional[torch.Tensor] = None,
                      stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
     """lightning_prefill_backward: returns (dq, dk, dv, d_state_in) for the loss
-    sum(d_o * o) + sum(d_state_out * state_out)."""
+    sum(d_o * o) + sum(d_state_out * state_out). The workspace the tensor-core
+    kernels need is allocated with torch unless a uint8 tensor is passed."""
     if q.dtype not in _DTYPES:
         raise ValueError("q must be float32 or bfloat16")
     if q.dim() != 4 or any(t.shape != q.shape for t in (k, v, d_o)):
         raise ValueError("q, k, v, d_o must share one [batch, heads, seq, dim] shape")
+    if variant not in ("auto", "simt", "pair"):
+        raise ValueError("backward variant must be auto, simt or pair")
     for name, t in (("q", q), ("k", k), ("v", v), ("d_o", d_o)):
         _need_cuda(name, t, q.dtype)
     b, h, L, d = q.shape
@@ -120,11 +124,17 @@ def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, d_o: tor
             _need_cuda(name, t, torch.float32)
             if tuple(t.shape) != (b, h, d, d):
                 raise ValueError("%s must be [batch, heads, dim, dim]" % name)
+    need = abi.lightning_prefill_backward_workspace_size(_DTYPES[q.dtype], b, h, L, d, int(block),
+                                                          _VARIANTS[variant])
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     ds_in = torch.empty((b, h, d, d), dtype=torch.float32, device=q.device) if want_state_grad else None
     abi.check(abi.lightning_prefill_backward(
         _ptr(q), _ptr(k), _ptr(v), _ptr(d_o), _DTYPES[q.dtype], _ptr(slopes), b, h, L, d, int(block),
-        _ptr(state_in), _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds_in), _stream(stream)))
+        _ptr(state_in), _ptr(d_state_out), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds_in), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream),
+        _VARIANTS[variant]))
     return dq, dk, dv, ds_in
 
 

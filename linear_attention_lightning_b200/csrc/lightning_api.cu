@@ -14,6 +14,7 @@
 #include "decode.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_pair.cuh"
+#include "reverse_rows.cuh"
 #include "prefill_tc.cuh"
 
 namespace {
@@ -188,7 +189,26 @@ struct BackwardArgs {
     const float *state_in, *d_state_out;
     void *dq, *dk, *dv;
     float *d_state_in;
+    void *workspace;
+    size_t workspace_bytes;
 };
+
+// Which kernels a backward request runs (LA_VARIANT_SIMT or _TCGEN05_PAIR), or -1.
+int choose_backward_variant(la_dtype dtype, int dim, int block, int requested) {
+    const bool pair_ok = la::pair_supports(dtype == LA_DTYPE_BF16, dim, block);
+    switch (requested) {
+        case LA_VARIANT_AUTO: return pair_ok ? LA_VARIANT_TCGEN05_PAIR : LA_VARIANT_SIMT;
+        case LA_VARIANT_SIMT: return LA_VARIANT_SIMT;
+        case LA_VARIANT_TCGEN05_PAIR: return pair_ok ? LA_VARIANT_TCGEN05_PAIR : -1;
+        default: return -1;
+    }
+}
+
+// Workspace of the tensor-core backward: three token-reversed operand copies.
+size_t backward_workspace_bytes(la_dtype dtype, int batch, int heads, int seq, int dim, int variant) {
+    if (variant != LA_VARIANT_TCGEN05_PAIR) return 0;
+    return 3 * (size_t)batch * heads * seq * dim * elem_bytes(dtype);
+}
 
 la_status check_backward_pointers(const BackwardArgs &a) {
     const size_t eb = elem_bytes(a.dtype);
@@ -219,6 +239,67 @@ la_status check_backward_pointers(const BackwardArgs &a) {
     return LA_OK;
 }
 
+la_status check_backward_workspace(const BackwardArgs &a, size_t need) {
+    if (need == 0 || a.seq == 0 || a.batch == 0) return LA_OK;
+    if (!a.workspace || a.workspace_bytes < need)
+        return fail(LA_ERR_INVALID_ARG, "the tensor-core backward needs %zu bytes of workspace (got %zu)", need,
+                    a.workspace ? a.workspace_bytes : (size_t)0);
+    if (!aligned16(a.workspace)) return fail(LA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    const size_t eb = elem_bytes(a.dtype);
+    const size_t n_tok = (size_t)a.batch * a.heads * a.seq * a.dim;
+    const size_t n_state = (size_t)a.batch * a.heads * a.dim * a.dim;
+    const Range rw = range_of(a.workspace, need);
+    const Range others[] = {range_of(a.q, n_tok * eb), range_of(a.k, n_tok * eb), range_of(a.v, n_tok * eb),
+                            range_of(a.d_o, n_tok * eb), range_of(a.dq, n_tok * eb), range_of(a.dk, n_tok * eb),
+                            range_of(a.dv, n_tok * eb), range_of(a.slopes, sizeof(float) * a.heads),
+                            range_of(a.state_in, a.state_in ? n_state * 4 : 0),
+                            range_of(a.d_state_out, a.d_state_out ? n_state * 4 : 0),
+                            range_of(a.d_state_in, a.d_state_in ? n_state * 4 : 0)};
+    for (const Range &r : others)
+        if (overlaps(rw, r)) return fail(LA_ERR_INVALID_ARG, "workspace overlaps an input or an output");
+    return LA_OK;
+}
+
+la_status launch_reverse(const void *src, void *dst, long long bh, int seq, int row_bytes, cudaStream_t stream) {
+    const int row_words = row_bytes / 16;
+    const int blocks = 148 * la::kRevBlocksPerSm;
+    if (dst) {
+        la::reverse_rows_kernel<<<blocks, la::kRevThreads, 0, stream>>>(
+            static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), bh * seq, seq, row_words);
+    } else {
+        la::reverse_rows_inplace_kernel<<<blocks, la::kRevThreads, 0, stream>>>(
+            static_cast<uint4 *>(const_cast<void *>(src)), bh, seq, row_words);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "token reversal launch");
+}
+
+// The tensor-core backward: the dQ pass runs the CTA-pair prefill kernel
+// forward on (dO, V, K); the dV and dK passes run it on token-reversed copies
+// (in the workspace) and put their outputs back in order.
+la_status run_backward_pair(const BackwardArgs &a, cudaStream_t stream) {
+    const long long bh = (long long)a.batch * a.heads;
+    const size_t bytes = (size_t)bh * a.seq * a.dim * 2;
+    const int row_bytes = a.dim * 2;
+    uint8_t *w0 = static_cast<uint8_t *>(a.workspace), *w1 = w0 + bytes, *w2 = w1 + bytes;
+    const la::Snapshots none{nullptr, 0, 0};
+    la_status st = la::launch_pair(a.d_o, a.v, a.k, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.dq, nullptr,
+                                   none, la::pair::PairPass{1, 0, 0}, stream, &g_last_error);
+    if (st != LA_OK) return st;
+    if ((st = launch_reverse(a.k, w0, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
+    if ((st = launch_reverse(a.q, w1, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
+    if ((st = launch_reverse(a.d_o, w2, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
+    st = la::launch_pair(w0, w1, w2, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dv, a.d_state_in, none,
+                         la::pair::PairPass{0, 1, 1}, stream, &g_last_error);
+    if (st != LA_OK) return st;
+    if ((st = launch_reverse(a.dv, nullptr, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
+    if ((st = launch_reverse(a.v, w0, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
+    st = la::launch_pair(w0, w2, w1, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dk, nullptr, none,
+                         la::pair::PairPass{1, 1, 0}, stream, &g_last_error);
+    if (st != LA_OK) return st;
+    return launch_reverse(a.dk, nullptr, bh, a.seq, row_bytes, stream);
+}
+
 // The gradients as three passes of the block recurrence (see lightning.h):
 //   dQ: forward in time, (q, k, v) <- (dO, V, K), carried state S_in^T;
 //   dV: backward in time, (q, k, v) <- (K, Q, dO), carried state dS_out seen
@@ -236,7 +317,7 @@ la_status run_backward_typed(const BackwardArgs &a, cudaStream_t stream) {
                                   a.dk, nullptr, la::SimtPass{1, 1, 1, 0}, stream);
 }
 
-la_status run_backward(const BackwardArgs &a, cudaStream_t stream) {
+la_status run_backward(const BackwardArgs &a, cudaStream_t stream, int variant) {
     if (a.batch == 0) return ok();
     if (a.seq == 0) {
         // no token: the state passes through, and so does its gradient
@@ -247,6 +328,7 @@ la_status run_backward(const BackwardArgs &a, cudaStream_t stream) {
         cudaError_t e = cudaGetLastError();
         return e == cudaSuccess ? ok() : cuda_fail(e, "state gradient passthrough launch");
     }
+    if (variant == LA_VARIANT_TCGEN05_PAIR) return run_backward_pair(a, stream);
     if (a.dtype == LA_DTYPE_BF16)
         return a.dim == 64 ? run_backward_typed<__nv_bfloat16, 64>(a, stream)
                            : run_backward_typed<__nv_bfloat16, 128>(a, stream);
@@ -265,7 +347,7 @@ la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
     }
     if (variant == LA_VARIANT_TCGEN05_PAIR)
         return la::launch_pair(a.q, a.k, a.v, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.o, a.state_out,
-                               a.sn, stream, &g_last_error);
+                               a.sn, la::pair::PairPass{0, 0, 0}, stream, &g_last_error);
     if (variant == LA_VARIANT_TCGEN05) return la::launch_tc(a.q, a.k, a.v, a.slopes, a.batch, a.heads,
                                                            a.seq, a.block, a.state_in, a.o, a.state_out,
                                                            a.sn, stream, &g_last_error);
@@ -337,14 +419,31 @@ la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_d
 la_status lightning_prefill_backward(const void *q, const void *k, const void *v, const void *d_o,
                                      la_dtype dtype, const float *slopes, int batch, int heads, int seq,
                                      int dim, int block, const float *state_in, const float *d_state_out,
-                                     void *dq, void *dk, void *dv, float *d_state_in, void *stream) {
+                                     void *dq, void *dk, void *dv, float *d_state_in, void *workspace,
+                                     size_t workspace_bytes, void *stream, int variant) {
     la_status st = check_prefill_shape(dtype, batch, heads, seq, dim, block);
     if (st != LA_OK) return st;
+    const int chosen = choose_backward_variant(dtype, dim, block, variant);
+    if (chosen < 0) {
+        if (variant < LA_VARIANT_AUTO || variant > LA_VARIANT_TCGEN05_PAIR || variant == LA_VARIANT_TCGEN05)
+            return fail(LA_ERR_INVALID_ARG, "variant %d is not a backward variant (AUTO, SIMT or TCGEN05_PAIR)",
+                        variant);
+        return fail(LA_ERR_UNSUPPORTED, "the tensor-core backward needs bf16, dim 128 and block 256");
+    }
     const BackwardArgs a{q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in, d_state_out,
-                         dq, dk, dv, d_state_in};
+                         dq, dk, dv, d_state_in, workspace, workspace_bytes};
     st = check_backward_pointers(a);
     if (st != LA_OK) return st;
-    return run_backward(a, static_cast<cudaStream_t>(stream));
+    st = check_backward_workspace(a, backward_workspace_bytes(dtype, batch, heads, seq, dim, chosen));
+    if (st != LA_OK) return st;
+    return run_backward(a, static_cast<cudaStream_t>(stream), chosen);
+}
+
+size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int heads, int seq, int dim,
+                                                 int block, int variant) {
+    if (check_prefill_shape(dtype, batch, heads, seq, dim, block) != LA_OK) return 0;
+    const int chosen = choose_backward_variant(dtype, dim, block, variant);
+    return chosen < 0 ? 0 : backward_workspace_bytes(dtype, batch, heads, seq, dim, chosen);
 }
 
 int lightning_prefill_snapshot_count(int seq, int interval) {

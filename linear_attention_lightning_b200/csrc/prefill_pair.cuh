@@ -211,12 +211,22 @@ __device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scal
     }
 }
 
+// How one launch treats its states. The forward prefill is {0, 0, 0}; the
+// passes of the backward computation (lightning_api.cu) read the carried
+// state transposed, let the first token see it with e^0 instead of e^{-s},
+// or write the final state one decay step further on.
+struct PairPass {
+    int state_in_t;      // 1: state_in holds the transpose of the carried state
+    int state_shift;     // 1: block 0 sees the carried state one step closer
+    int state_out_step;  // 1: state_out = e^{-s} times the final state
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_o,
                     const float *__restrict__ slopes, int heads, int seq, const float *state_in,
-                    float *state_out, Snapshots sn) {
+                    float *state_out, Snapshots sn, PairPass pp) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_addr(smem_raw);
     const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -431,7 +441,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // Qd S MMA (which precedes its dS MMA) has read the region
                 if (t > 0 && !group_wait(c, DS_FULL, (uint32_t)(t - 1) & 1u, leader, bar_id)) goto ab_done;
                 if (!group_wait(c, QK_LOADED, par, leader, bar_id)) goto ab_done;
-                const float dq = ptx::ex2(-sl2 * (float)(i + 1));
+                const float dq = ptx::ex2(-sl2 * (float)(i + 1 - (t == 0 ? pp.state_shift : 0)));
                 const uint8_t *qrow = c.smem + kOffQ + r * 128;
 #pragma unroll 1
                 for (int hb = 0; hb < 4; ++hb) {
@@ -489,6 +499,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int vcol = 64 * (int)rank + (l & 63);
         const int khalf = l >> 6;
         const size_t sb = (size_t)bh * kDim * kDim;
+        const float fout = pp.state_out_step ? ptx::ex2(-sl2) : 1.f;
         // fp16 state operand: K-major rows = value column (l & 63), 64 key dims per box
         uint8_t *srow = c.smem + kOffS + khalf * 8192 + (l & 63) * 128;
         // one 32-value half of this thread's state row: operand copy, optional
@@ -512,7 +523,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (last) {
                 if (state_out) {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) state_out[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q];
+                    for (int q = 0; q < 32; ++q)
+                        state_out[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q] * fout;
                 }
             } else {
                 uint32_t lo[16], hi[16];
@@ -546,7 +558,11 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::tc_fence_after();
             }
             {
-                const float dnext = last ? 0.f : ptx::ex2(-sl2 * (float)min(kBlock, seq - (t + 1) * kBlock));
+                // decay from block t's end to block t+1's end (from the carried state's
+                // position to block 0's end when t = -1)
+                const float dnext =
+                    last ? 0.f
+                         : ptx::ex2(-sl2 * (float)(min(kBlock, seq - (t + 1) * kBlock) - (t < 0 ? pp.state_shift : 0)));
                 float *snap = t >= 0 ? snapshot_at(sn, bh, t * kBlock + min(kBlock, seq - t * kBlock), kDim) : nullptr;
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
@@ -560,7 +576,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     } else {
 #pragma unroll
                         for (int q = 0; q < 32; ++q)
-                            sv[q] = state_in ? state_in[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] : 0.f;
+                            sv[q] = state_in ? state_in[sb + (pp.state_in_t
+                                                                  ? (size_t)vcol * kDim + (64 * khalf + 32 * hh + q)
+                                                                  : (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol)]
+                                             : 0.f;
                     }
                     carry_half(sv, hh, dnext, last, snap);
                 }
@@ -630,6 +649,7 @@ inline bool pair_supports(bool bf16, int dim, int block) { return bf16 && dim ==
 
 inline la_status launch_pair(const void *q, const void *k, const void *v, const float *slopes, int batch,
                              int heads, int seq, const float *state_in, void *o, float *state_out, Snapshots sn,
+                             pair::PairPass pp,
                              cudaStream_t stream, std::string *err) {
     const long long bh = (long long)batch * heads;
     CUtensorMap mq, mk, mk64, mv, mo;
@@ -656,7 +676,7 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, pair::prefill_pair_kernel, mq, mk, mk64, mv, mo, slopes, heads, seq, state_in,
-                           state_out, sn);
+                           state_out, sn, pp);
     if (e != cudaSuccess) {
         *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
         return LA_ERR_CUDA;

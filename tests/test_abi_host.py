@@ -161,15 +161,17 @@ def test_snapshot_trivial_calls_need_no_gpu():
     assert _prefill_snapshots(seq=0, state_out=None, snapshots=None) == abi.LA_OK
 
 
-DO, DQ, DK, DV, DSI, DSO = (0x10000000 * (i + 10) for i in range(6))
+DO, DQ, DK, DV, DSI, DSO, WS = (0x10000000 * (i + 10) for i in range(7))
+WS_BYTES = 1 << 26
 
 
-def _backward(**kw):
-    a = dict(GOOD, d_o=DO, d_state_out=DSO, dq=DQ, dk=DK, dv=DV, d_state_in=DSI)
+def _backward(variant=abi.LA_VARIANT_AUTO, **kw):
+    a = dict(GOOD, d_o=DO, d_state_out=DSO, dq=DQ, dk=DK, dv=DV, d_state_in=DSI, ws=WS, ws_bytes=WS_BYTES)
     a.update(kw)
     return abi.lightning_prefill_backward(a["q"], a["k"], a["v"], a["d_o"], a["dtype"], a["slopes"], a["batch"],
                                           a["heads"], a["seq"], a["dim"], a["block"], a["state_in"],
-                                          a["d_state_out"], a["dq"], a["dk"], a["dv"], a["d_state_in"], None)
+                                          a["d_state_out"], a["dq"], a["dk"], a["dv"], a["d_state_in"],
+                                          a["ws"], a["ws_bytes"], None, variant)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -185,10 +187,28 @@ def _backward(**kw):
     (dict(dv=DQ + 1024), abi.LA_ERR_INVALID_ARG),        # two outputs overlap
     (dict(d_state_in=DSO), abi.LA_ERR_INVALID_ARG),      # overlaps d_state_out
     (dict(d_state_in=S0 + 16), abi.LA_ERR_INVALID_ARG),  # overlaps state_in
+    (dict(ws=None), abi.LA_ERR_INVALID_ARG),              # the tensor-core kernels need a workspace
+    (dict(ws_bytes=1024), abi.LA_ERR_INVALID_ARG),        # too short
+    (dict(ws=WS + 8), abi.LA_ERR_INVALID_ARG),            # misaligned
+    (dict(ws=DQ), abi.LA_ERR_INVALID_ARG),                # overlaps an output
+    (dict(variant=abi.LA_VARIANT_TCGEN05), abi.LA_ERR_INVALID_ARG),
+    (dict(variant=7), abi.LA_ERR_INVALID_ARG),
+    (dict(variant=abi.LA_VARIANT_TCGEN05_PAIR, block=128), abi.LA_ERR_UNSUPPORTED),
 ])
 def test_backward_argument_errors(kw, status):
     assert _backward(**kw) == status
     assert abi.last_error_message() != ""
+
+
+def test_backward_workspace_size():
+    ws = abi.lightning_prefill_backward_workspace_size
+    # three token-reversed bf16 copies for the tensor-core kernels, nothing for the CUDA cores
+    assert ws(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_AUTO) == 3 * 64 * 131072 * 128 * 2
+    assert ws(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_SIMT) == 0
+    assert ws(abi.LA_DTYPE_F32, 1, 2, 100, 64, 64, abi.LA_VARIANT_AUTO) == 0
+    assert ws(abi.LA_DTYPE_BF16, 1, 2, 100, 128, 128, abi.LA_VARIANT_TCGEN05_PAIR) == 0  # unsupported
+    # a CUDA-core request needs no workspace at all
+    assert _backward(variant=abi.LA_VARIANT_SIMT, ws=None, ws_bytes=0, batch=0) == abi.LA_OK
 
 
 def test_backward_trivial_calls_need_no_gpu():

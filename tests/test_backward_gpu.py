@@ -41,45 +41,54 @@ def _check(got, ref, dtype):
         assert e <= TOL[dtype], "%s error %.3g rms > %.3g" % (name, e, TOL[dtype])
 
 
-# (batch, heads, seq, dim, block, dtype, with_state, with_dstate)
+# (batch, heads, seq, dim, block, dtype, with_state, with_dstate, variant)
 CASES = [
-    (1, 2, 256, 64, 64, torch.float32, False, False),
-    (2, 3, 300, 64, 100, torch.float32, True, True),
-    (1, 2, 129, 128, 1, torch.float32, True, False),
-    (1, 2, 513, 128, 256, torch.float32, False, True),
-    (1, 4, 1000, 128, 256, torch.bfloat16, True, True),
-    (2, 2, 640, 128, 128, torch.bfloat16, False, False),
-    (1, 1, 1, 128, 256, torch.bfloat16, True, True),
+    (1, 2, 256, 64, 64, torch.float32, False, False, "simt"),
+    (2, 3, 300, 64, 100, torch.float32, True, True, "simt"),
+    (1, 2, 129, 128, 1, torch.float32, True, False, "simt"),
+    (1, 2, 513, 128, 256, torch.float32, False, True, "simt"),
+    (1, 4, 1000, 128, 256, torch.bfloat16, True, True, "simt"),
+    (2, 2, 640, 128, 128, torch.bfloat16, False, False, "simt"),
+    (1, 1, 1, 128, 256, torch.bfloat16, True, True, "simt"),
+    (1, 4, 1000, 128, 256, torch.bfloat16, True, True, "pair"),
+    (2, 3, 512, 128, 256, torch.bfloat16, False, False, "pair"),
+    (1, 2, 1300, 128, 256, torch.bfloat16, False, True, "pair"),
+    (1, 2, 257, 128, 256, torch.bfloat16, True, False, "pair"),
+    (1, 1, 1, 128, 256, torch.bfloat16, True, True, "pair"),
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: "b%d_h%d_L%d_d%d_B%d_%s_%s_%s" % (
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "b%d_h%d_L%d_d%d_B%d_%s_%s_%s_%s" % (
     c[0], c[1], c[2], c[3], c[4], "bf16" if c[5] == torch.bfloat16 else "f32",
-    "state" if c[6] else "zero", "dstate" if c[7] else "nodstate"))
+    "state" if c[6] else "zero", "dstate" if c[7] else "nodstate", c[8]))
 def test_backward_matches_the_oracle(case):
-    b, h, L, d, block, dtype, with_state, with_dstate = case
+    b, h, L, d, block, dtype, with_state, with_dstate, variant = case
     inp = _grads_inputs(b, h, L, d, dtype, with_state, with_dstate, seed=31)
     got = la.prefill_backward(inp["q"], inp["k"], inp["v"], inp["d_o"], inp["slopes"], block, inp["state_in"],
-                              inp["d_state_out"])
+                              inp["d_state_out"], variant=variant)
     torch.cuda.synchronize()
     _check(got, _oracle_backward(inp), dtype)
 
 
-def test_backward_writes_only_its_outputs():
-    b, h, L, d, block = 1, 2, 300, 128, 64
+@pytest.mark.parametrize("variant,block", [(abi.LA_VARIANT_SIMT, 64), (abi.LA_VARIANT_TCGEN05_PAIR, 256)])
+def test_backward_writes_only_its_outputs(variant, block):
+    b, h, L, d = 1, 2, 300, 128
     inp = _grads_inputs(b, h, L, d, torch.bfloat16, True, True, seed=32)
     outs = [guarded_empty((b, h, L, d), torch.bfloat16, DEV) for _ in range(3)]
     ds, ds_back = guarded_empty((b, h, d, d), torch.float32, DEV)
+    need = abi.lightning_prefill_backward_workspace_size(abi.LA_DTYPE_BF16, b, h, L, d, block, variant)
+    ws, ws_back = guarded_empty((max(need, 4) // 4,), torch.float32, DEV)  # need is a multiple of 4
     st = abi.lightning_prefill_backward(
         inp["q"].data_ptr(), inp["k"].data_ptr(), inp["v"].data_ptr(), inp["d_o"].data_ptr(), abi.LA_DTYPE_BF16,
         inp["slopes"].data_ptr(), b, h, L, d, block, inp["state_in"].data_ptr(), inp["d_state_out"].data_ptr(),
-        outs[0][0].data_ptr(), outs[1][0].data_ptr(), outs[2][0].data_ptr(), ds.data_ptr(),
-        torch.cuda.current_stream().cuda_stream)
+        outs[0][0].data_ptr(), outs[1][0].data_ptr(), outs[2][0].data_ptr(), ds.data_ptr(), ws.data_ptr(), need,
+        torch.cuda.current_stream().cuda_stream, variant)
     assert st == abi.LA_OK, abi.last_error_message()
     torch.cuda.synchronize()
     for view, back in outs:
         assert guards_intact(back, view.numel())
     assert guards_intact(ds_back, ds.numel())
+    assert guards_intact(ws_back, ws.numel())
     _check([outs[0][0], outs[1][0], outs[2][0], ds], _oracle_backward(inp), torch.bfloat16)
 
 
@@ -92,11 +101,12 @@ def test_backward_of_an_empty_sequence_passes_the_state_gradient():
     assert torch.equal(ds_in, dso)
 
 
-def test_m1_prefill_8k_backward_sampled_heads():
+@pytest.mark.parametrize("variant", ["simt", "pair"])
+def test_m1_prefill_8k_backward_sampled_heads(variant):
     w = inputs.WORKLOADS["m1_prefill_8k"]
     inp = _grads_inputs(w.batch, w.heads, w.seq, w.dim, w.dtype, w.state_in, True, seed=w.seed)
     got = la.prefill_backward(inp["q"], inp["k"], inp["v"], inp["d_o"], inp["slopes"], w.block, inp["state_in"],
-                              inp["d_state_out"])
+                              inp["d_state_out"], variant=variant)
     torch.cuda.synchronize()
     heads = [0, 40, 63]
     _check([t[:, heads] for t in got], _oracle_backward(inp, heads_idx=heads), w.dtype)
