@@ -185,6 +185,26 @@ la_status lightning_prefill_backward(const void *q, const void *k, const void *v
                                      void *dq, void *dk, void *dv, float *d_state_in, void *workspace,
                                      size_t workspace_bytes, void *stream, int variant);
 
+/*
+ * lightning_prefill_backward without a workspace argument. The pages have no
+ * counterpart to this entry point; it is a convenience of this library. It
+ * takes its scratch from a fixed device array inside the library (its size:
+ * lightning_prefill_backward_noalloc_capacity(), 64 MiB) and allocates no
+ * memory. Arguments and results are those of lightning_prefill_backward.
+ * A request whose workspace would exceed the array returns
+ * LA_ERR_UNSUPPORTED before any launch. All calls on one device share the
+ * array: calls that could run at the same time (on different streams) must
+ * use lightning_prefill_backward with their own workspaces instead.
+ */
+la_status lightning_prefill_backward_noalloc(const void *q, const void *k, const void *v, const void *d_o,
+                                             la_dtype dtype, const float *slopes, int batch, int heads,
+                                             int seq, int dim, int block, const float *state_in,
+                                             const float *d_state_out, void *dq, void *dk, void *dv,
+                                             float *d_state_in, void *stream, int variant);
+
+/* Bytes of scratch lightning_prefill_backward_noalloc has. Host only. */
+size_t lightning_prefill_backward_noalloc_capacity(void);
+
 /* Bytes of workspace lightning_prefill_backward needs for these arguments
  * (three copies of a [batch][heads][seq][dim] tensor for the tensor-core
  * kernels, 0 for the CUDA-core ones or an invalid request). Host only. */

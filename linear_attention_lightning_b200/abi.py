@@ -33,6 +33,9 @@ _SIGNATURES = {
     "lightning_prefill_backward": ([_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _sz, _vp, _i], _i),
     "lightning_prefill_backward_workspace_size": ([_i, _i, _i, _i, _i, _i, _i], _sz),
+    "lightning_prefill_backward_noalloc": ([_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp,
+                                            _vp, _vp, _vp, _i], _i),
+    "lightning_prefill_backward_noalloc_capacity": ([], _sz),
     "lightning_decode": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp], _i),
     "lightning_device_status": ([_vp], _i),
     "lightning_status_string": ([_i], ctypes.c_char_p),
@@ -121,6 +124,16 @@ def lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, d
     return load().lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block,
                                              state_in, d_state_out, dq, dk, dv, d_state_in, workspace,
                                              workspace_bytes, stream, variant)
+
+
+def lightning_prefill_backward_noalloc(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in,
+                                       d_state_out, dq, dk, dv, d_state_in, stream, variant):
+    return load().lightning_prefill_backward_noalloc(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block,
+                                                     state_in, d_state_out, dq, dk, dv, d_state_in, stream, variant)
+
+
+def lightning_prefill_backward_noalloc_capacity():
+    return load().lightning_prefill_backward_noalloc_capacity()
 
 
 def lightning_prefill_backward_workspace_size(dtype, batch, heads, seq, dim, block, variant):

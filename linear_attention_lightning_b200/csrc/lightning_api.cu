@@ -193,6 +193,11 @@ struct BackwardArgs {
     size_t workspace_bytes;
 };
 
+// Scratch of lightning_prefill_backward_noalloc: a fixed device array, so that
+// entry point needs no workspace from the caller and allocates nothing.
+constexpr size_t kNoAllocScratchBytes = (size_t)64 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 // Which kernels a backward request runs (LA_VARIANT_SIMT or _TCGEN05_PAIR), or -1.
 int choose_backward_variant(la_dtype dtype, int dim, int block, int requested) {
     const bool pair_ok = la::pair_supports(dtype == LA_DTYPE_BF16, dim, block);
@@ -438,6 +443,30 @@ la_status lightning_prefill_backward(const void *q, const void *k, const void *v
     if (st != LA_OK) return st;
     return run_backward(a, static_cast<cudaStream_t>(stream), chosen);
 }
+
+la_status lightning_prefill_backward_noalloc(const void *q, const void *k, const void *v, const void *d_o,
+                                             la_dtype dtype, const float *slopes, int batch, int heads, int seq,
+                                             int dim, int block, const float *state_in, const float *d_state_out,
+                                             void *dq, void *dk, void *dv, float *d_state_in, void *stream,
+                                             int variant) {
+    la_status st = check_prefill_shape(dtype, batch, heads, seq, dim, block);
+    if (st != LA_OK) return st;
+    const int chosen = choose_backward_variant(dtype, dim, block, variant);
+    const size_t need = chosen < 0 ? 0 : backward_workspace_bytes(dtype, batch, heads, seq, dim, chosen);
+    if (need > kNoAllocScratchBytes)
+        return fail(LA_ERR_UNSUPPORTED, "the request needs %zu bytes of scratch; the built-in scratch holds %zu",
+                    need, kNoAllocScratchBytes);
+    void *scratch = nullptr;
+    if (need > 0 && batch > 0 && seq > 0) {
+        // the scratch array's address in the current device's context
+        const cudaError_t e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    }
+    return lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in,
+                                      d_state_out, dq, dk, dv, d_state_in, scratch, need, stream, variant);
+}
+
+size_t lightning_prefill_backward_noalloc_capacity(void) { return kNoAllocScratchBytes; }
 
 size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int heads, int seq, int dim,
                                                  int block, int variant) {
