@@ -452,8 +452,8 @@ def run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, plain_ms):
 
 def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     """lightning_prefill_backward on the workload (AUTO: the CTA-pair tensor-core
-    kernels where they apply), timed like the main leg: dQ on (dO, V, K), dV and
-    dK on token-reversed copies, plus the reversals."""
+    kernel where it applies), timed like the main leg: dQ causal on (dO, V, K),
+    dV and dK anti-causal on (K, Q, dO) and (V, dO, Q)."""
     import torch
     from linear_attention_lightning_b200 import abi
     q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
@@ -494,7 +494,12 @@ def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     gbs = by / (ms / 1e3) / 1e9
     # three passes of the block recurrence: 3 x (4Bd + 4d^2) per (token, head)
     tf = 3 * prefill_flops(w.batch, w.heads, w.seq, w.dim, w.block)["formula"] / (ms / 1e3) / 1e12
-    kernel = "pair (3 passes + token reversals)" if need > 0 else "simt (3 passes)"
+    import linear_attention_lightning_b200 as la
+    try:
+        la.prefill_variant(w.dtype, w.batch, w.heads, w.seq, w.dim, w.block, "pair")
+        kernel = "pair (dQ causal, dV and dK anti-causal)"
+    except ValueError:
+        kernel = "simt (3 passes)"
     return {"kernel": kernel, "steps": steps, "ms_per_step": round(ms, 3),
             "tokens_per_s": round(world * w.batch * w.seq / (ms / 1e3), 1),
             "workspace_bytes": need,

@@ -160,7 +160,7 @@ la_status lightning_prefill_snapshots(const void *q, const void *k, const void *
  * backward in time on (K, Q, dO) and (V, dO, Q) with state R.
  * Kernels (variant): LA_VARIANT_TCGEN05_PAIR runs the passes on the CTA-pair
  * tensor-core kernel (bf16, dim 128, block 256; the backward-in-time passes
- * read token-reversed operand copies kept in the workspace);
+ * run it anti-causally, blocks from last to first);
  * LA_VARIANT_SIMT runs them on CUDA cores in fp32 (any dtype, dim 64 or 128,
  * any block, no workspace); LA_VARIANT_AUTO takes the tensor-core kernels
  * where they apply. LA_VARIANT_TCGEN05 is not a backward variant.
@@ -173,8 +173,8 @@ la_status lightning_prefill_snapshots(const void *q, const void *k, const void *
  *   d_state_in    [batch][heads][dim][dim] float32, or NULL to skip.
  *   workspace, workspace_bytes
  *                 scratch of at least lightning_prefill_backward_workspace_size
- *                 bytes (0 for the CUDA-core kernels), 16-byte aligned,
- *                 overlapping nothing else; contents undefined afterwards.
+ *                 bytes (0 for every current kernel, so NULL/0 is fine);
+ *                 when needed: 16-byte aligned, overlapping nothing else.
  * All device pointers, caller-owned, 16-byte aligned. No output may overlap
  * an input or another output; a short or overlapping workspace is rejected
  * (all LA_ERR_INVALID_ARG). Shape rules as for lightning_prefill.
@@ -188,9 +188,10 @@ la_status lightning_prefill_backward(const void *q, const void *k, const void *v
 /*
  * lightning_prefill_backward without a workspace argument. The pages have no
  * counterpart to this entry point; it is a convenience of this library. It
- * takes its scratch from a fixed device array inside the library (its size:
- * lightning_prefill_backward_noalloc_capacity(), 64 MiB) and allocates no
- * memory. Arguments and results are those of lightning_prefill_backward.
+ * takes any scratch the chosen kernels need from a fixed device array inside
+ * the library (its size: lightning_prefill_backward_noalloc_capacity(),
+ * 64 MiB) and allocates no memory; the current kernels need none. Arguments
+ * and results are those of lightning_prefill_backward.
  * A request whose workspace would exceed the array returns
  * LA_ERR_UNSUPPORTED before any launch. All calls on one device share the
  * array: calls that could run at the same time (on different streams) must
@@ -206,8 +207,7 @@ la_status lightning_prefill_backward_noalloc(const void *q, const void *k, const
 size_t lightning_prefill_backward_noalloc_capacity(void);
 
 /* Bytes of workspace lightning_prefill_backward needs for these arguments
- * (three copies of a [batch][heads][seq][dim] tensor for the tensor-core
- * kernels, 0 for the CUDA-core ones or an invalid request). Host only. */
+ * (0 for every current kernel and for an invalid request). Host only. */
 size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int heads, int seq, int dim,
                                                  int block, int variant);
 

@@ -14,7 +14,6 @@
 #include "decode.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_pair.cuh"
-#include "reverse_rows.cuh"
 #include "prefill_tc.cuh"
 
 namespace {
@@ -209,10 +208,10 @@ int choose_backward_variant(la_dtype dtype, int dim, int block, int requested) {
     }
 }
 
-// Workspace of the tensor-core backward: three token-reversed operand copies.
+// Workspace a backward request needs: none of the current kernels needs any.
 size_t backward_workspace_bytes(la_dtype dtype, int batch, int heads, int seq, int dim, int variant) {
-    if (variant != LA_VARIANT_TCGEN05_PAIR) return 0;
-    return 3 * (size_t)batch * heads * seq * dim * elem_bytes(dtype);
+    (void)dtype; (void)batch; (void)heads; (void)seq; (void)dim; (void)variant;
+    return 0;
 }
 
 la_status check_backward_pointers(const BackwardArgs &a) {
@@ -265,44 +264,21 @@ la_status check_backward_workspace(const BackwardArgs &a, size_t need) {
     return LA_OK;
 }
 
-la_status launch_reverse(const void *src, void *dst, long long bh, int seq, int row_bytes, cudaStream_t stream) {
-    const int row_words = row_bytes / 16;
-    const int blocks = 148 * la::kRevBlocksPerSm;
-    if (dst) {
-        la::reverse_rows_kernel<<<blocks, la::kRevThreads, 0, stream>>>(
-            static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), bh * seq, seq, row_words);
-    } else {
-        la::reverse_rows_inplace_kernel<<<blocks, la::kRevThreads, 0, stream>>>(
-            static_cast<uint4 *>(const_cast<void *>(src)), bh, seq, row_words);
-    }
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? ok() : cuda_fail(e, "token reversal launch");
-}
-
-// The tensor-core backward: the dQ pass runs the CTA-pair prefill kernel
-// forward on (dO, V, K); the dV and dK passes run it on token-reversed copies
-// (in the workspace) and put their outputs back in order.
+// The tensor-core backward: the three passes on the CTA-pair kernel. dQ runs
+// causal on (dO, V, K) with the carried state S_in^T; dV and dK run
+// anti-causal (blocks from last to first, state anchored at each block's last
+// token) on (K, Q, dO) with carried state dS_out, whose final state is dS_in,
+// and on (V, dO, Q) with dS_out^T.
 la_status run_backward_pair(const BackwardArgs &a, cudaStream_t stream) {
-    const long long bh = (long long)a.batch * a.heads;
-    const size_t bytes = (size_t)bh * a.seq * a.dim * 2;
-    const int row_bytes = a.dim * 2;
-    uint8_t *w0 = static_cast<uint8_t *>(a.workspace), *w1 = w0 + bytes, *w2 = w1 + bytes;
     const la::Snapshots none{nullptr, 0, 0};
     la_status st = la::launch_pair(a.d_o, a.v, a.k, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.dq, nullptr,
-                                   none, la::pair::PairPass{1, 0, 0}, stream, &g_last_error);
+                                   none, la::pair::PairPass{1, 0}, stream, &g_last_error);
     if (st != LA_OK) return st;
-    if ((st = launch_reverse(a.k, w0, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
-    if ((st = launch_reverse(a.q, w1, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
-    if ((st = launch_reverse(a.d_o, w2, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
-    st = la::launch_pair(w0, w1, w2, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dv, a.d_state_in, none,
-                         la::pair::PairPass{0, 1, 1}, stream, &g_last_error);
+    st = la::launch_pair(a.k, a.q, a.d_o, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dv, a.d_state_in,
+                         none, la::pair::PairPass{0, 1}, stream, &g_last_error);
     if (st != LA_OK) return st;
-    if ((st = launch_reverse(a.dv, nullptr, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
-    if ((st = launch_reverse(a.v, w0, bh, a.seq, row_bytes, stream)) != LA_OK) return st;
-    st = la::launch_pair(w0, w2, w1, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dk, nullptr, none,
-                         la::pair::PairPass{1, 1, 0}, stream, &g_last_error);
-    if (st != LA_OK) return st;
-    return launch_reverse(a.dk, nullptr, bh, a.seq, row_bytes, stream);
+    return la::launch_pair(a.v, a.d_o, a.q, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dk, nullptr,
+                           none, la::pair::PairPass{1, 1}, stream, &g_last_error);
 }
 
 // The gradients as three passes of the block recurrence (see lightning.h):
@@ -352,7 +328,7 @@ la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
     }
     if (variant == LA_VARIANT_TCGEN05_PAIR)
         return la::launch_pair(a.q, a.k, a.v, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.o, a.state_out,
-                               a.sn, la::pair::PairPass{0, 0, 0}, stream, &g_last_error);
+                               a.sn, la::pair::PairPass{0, 0}, stream, &g_last_error);
     if (variant == LA_VARIANT_TCGEN05) return la::launch_tc(a.q, a.k, a.v, a.slopes, a.batch, a.heads,
                                                            a.seq, a.block, a.state_in, a.o, a.state_out,
                                                            a.sn, stream, &g_last_error);

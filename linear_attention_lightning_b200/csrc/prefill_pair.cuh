@@ -157,8 +157,10 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
 
 // fp32 P columns [col0, col0 + 128) of this thread's row -> fp16 P ⊙ D in
 // [dst0, dst0 + 64). Row i (block position) against keys j0 .. j0+127.
+// Causal: key j counts for j <= i with e^{-s(i-j)}; anti-causal (upper): for
+// j >= i with e^{-s(j-i)}. tab[u] = e^{-s(15-u)}, step = e^{-s}.
 __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uint32_t dst0, int i, int j0,
-                                          float sl2, float step, const float (&tab)[16]) {
+                                          float sl2, float step, const float (&tab)[16], bool upper) {
     // 32 fp32 columns per iteration -> 16 fp16 pair columns; the destination
     // [dst0 + 16 q, dst0 + 16 q + 16) lies inside columns already read
 #pragma unroll 1
@@ -172,7 +174,26 @@ __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uin
             const int jb = j0 + 32 * q + 16 * g;
             const int dlast = i - (jb + 15);
             float p[16];
-            if (dlast >= 0) {
+            if (upper) {
+                if (jb >= i) {
+                    const float wb = ptx::ex2(-sl2 * (float)(jb - i));
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[16 * g + u]) * tab[15 - u]) * wb;
+                } else if (jb + 15 < i) {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) p[u] = 0.f;
+                } else {
+                    // keys from the diagonal (u = i - jb) upward
+                    const int d0 = i - jb;
+                    float w = 1.f;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const bool live = u >= d0;
+                        p[u] = live ? __uint_as_float(v[16 * g + u]) * w : 0.f;
+                        w = live ? w * step : w;
+                    }
+                }
+            } else if (dlast >= 0) {
                 const float wb = ptx::ex2(-sl2 * (float)dlast);
 #pragma unroll
                 for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[16 * g + u]) * tab[u]) * wb;
@@ -211,14 +232,14 @@ __device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scal
     }
 }
 
-// How one launch treats its states. The forward prefill is {0, 0, 0}; the
-// passes of the backward computation (lightning_api.cu) read the carried
-// state transposed, let the first token see it with e^0 instead of e^{-s},
-// or write the final state one decay step further on.
+// How one launch runs. The forward prefill is {0, 0}; the passes of the
+// backward computation (lightning_api.cu) read the carried state transposed,
+// or run anti-causal.
 struct PairPass {
-    int state_in_t;      // 1: state_in holds the transpose of the carried state
-    int state_shift;     // 1: block 0 sees the carried state one step closer
-    int state_out_step;  // 1: state_out = e^{-s} times the final state
+    int state_in_t;  // 1: state_in holds the transpose of the carried state
+    int anti;        // 1: anti-causal: blocks from last to first, query i sees keys j >= i
+                     //    with e^{-s(j-i)}, the carried state anchored at each block's last
+                     //    token (query factor e^{-s(m-1-i)}, key factor e^{-s(j+1)})
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -243,6 +264,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const float s = slopes[bh % heads];
     const float sl2 = s * kLog2e;
     const int nblk = (seq + kBlock - 1) / kBlock;
+    // block index of the t-th block visited, and its length
+    auto tb = [&](int t) { return pp.anti ? nblk - 1 - t : t; };
+    auto blen = [&](int t) { return min(kBlock, seq - tb(t) * kBlock); };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(&c.bars[i], 1);
@@ -289,7 +313,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 uint8_t *dst = c.smem + kOffStage + st * kStageBytes;
                 uint64_t *bar = &c.bars[VK_LOADED + st];
                 ptx::mbar_arrive_expect_tx(bar, kStageBytes);
-                const int row0 = t * kBlock;
+                const int row0 = tb(t) * kBlock;
                 ptx::tma_load_3d(dst, &tm_v, bar, 64 * rank, row0, bh);                      // V keys 0..127
                 ptx::tma_load_3d(dst + kBoxBytes, &tm_v, bar, 64 * rank, row0 + kRows, bh);  // V keys 128..255
                 ptx::tma_load_3d(dst + 2 * kBoxBytes, &tm_k, bar, 64 * rank, row0, bh);      // K dims half, keys 0..127
@@ -302,8 +326,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // Q and K sub-tiles of block t, once block t-1's Q K^T ran and its Qd was built
                 if (t > 0) ok = wait_bar(c, QK_DONE, (uint32_t)(t - 1) & 1u) && wait_bar(c, QD_LOCAL, (uint32_t)(t - 1) & 1u);
                 if (!ok) break;
-                const int row = t * kBlock + kRows * (int)rank;
-                const int krow = t * kBlock + 64 * (int)rank;
+                const int row = tb(t) * kBlock + kRows * (int)rank;
+                const int krow = tb(t) * kBlock + 64 * (int)rank;
                 uint64_t *qkbar = &c.bars[QK_LOADED];
                 ptx::mbar_arrive_expect_tx(qkbar, 4 * kBoxBytes);
                 ptx::tma_load_3d(c.smem + kOffQ, &tm_q, qkbar, 0, row, bh);
@@ -415,7 +439,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int u = 0; u < 16; ++u) tab[u] = ptx::ex2(-sl2 * (float)(15 - u));
         for (int t = 0; t < nblk; ++t) {
             const uint32_t par = t & 1;
-            const int m = min(kBlock, seq - t * kBlock);
+            const int m = blen(t);
             if (grp == 0) {
                 // K ⊙ d_k (fp16) for this CTA's key-dim half and V widened to fp16, keys r
                 // and 128 + r. The
@@ -430,7 +454,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int u = 0; u < 4; ++u) {
                     // u = 0, 1: K rows r and 128 + r scaled by d_k; u = 2, 3: V rows widened
                     const int h = u & 1, j = kRows * h + r;
-                    const float sc = u >= 2 ? 1.f : (j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f);
+                    const float sc = u >= 2   ? 1.f
+                                     : j >= m ? 0.f
+                                              : ptx::ex2(-sl2 * (float)(pp.anti ? j + 1 : m - 1 - j));
                     scale_row_to_f16((u >= 2 ? vt : kd) + h * kBoxBytes + r * 128, r, sc);
                 }
                 ptx::fence_proxy_async_smem();
@@ -441,7 +467,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // Qd S MMA (which precedes its dS MMA) has read the region
                 if (t > 0 && !group_wait(c, DS_FULL, (uint32_t)(t - 1) & 1u, leader, bar_id)) goto ab_done;
                 if (!group_wait(c, QK_LOADED, par, leader, bar_id)) goto ab_done;
-                const float dq = ptx::ex2(-sl2 * (float)(i + 1 - (t == 0 ? pp.state_shift : 0)));
+                const float dq = pp.anti ? (i < m ? ptx::ex2(-sl2 * (float)(m - 1 - i)) : 0.f)
+                                         : ptx::ex2(-sl2 * (float)(i + 1));
                 const uint8_t *qrow = c.smem + kOffQ + r * 128;
 #pragma unroll 1
                 for (int hb = 0; hb < 4; ++hb) {
@@ -467,19 +494,21 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     arrive_leader(&c.bars[QD_READY]);
                 }
             }
-            // P ⊙ D -> fp16 for keys [128 grp, 128 grp + 128)
+            // P ⊙ D -> fp16 for keys [128 grp, 128 grp + 128); the quadrant the mask
+            // zeroes (causal: rows 0..127 x keys 128..255; anti-causal: rows
+            // 128..255 x keys 0..127) is only cleared
             if (!group_wait(c, P_FULL + grp, par, leader, bar_id)) goto ab_done;
             ptx::tc_fence_after();
-            if (grp == 1 && rank == 0) {
-                // rows 0..127 against keys 128..255: every entry is masked
+            if (pp.anti ? (grp == 0 && rank == 1) : (grp == 1 && rank == 0)) {
+                // every entry of this quadrant is masked
                 uint32_t zero[16];
 #pragma unroll
                 for (int u = 0; u < 16; ++u) zero[u] = 0u;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) ptx::tmem_st16(trow + kColPHi + 16 * q, zero);
+                for (int q = 0; q < 4; ++q) ptx::tmem_st16(trow + (grp == 0 ? kColP : kColPHi) + 16 * q, zero);
             } else {
                 convert_p(trow, grp == 0 ? kColP : kColPHi, grp == 0 ? kColP : kColPHi, i, kRows * grp, sl2,
-                          step, tab);
+                          step, tab, pp.anti != 0);
             }
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
@@ -499,7 +528,6 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int vcol = 64 * (int)rank + (l & 63);
         const int khalf = l >> 6;
         const size_t sb = (size_t)bh * kDim * kDim;
-        const float fout = pp.state_out_step ? ptx::ex2(-sl2) : 1.f;
         // fp16 state operand: K-major rows = value column (l & 63), 64 key dims per box
         uint8_t *srow = c.smem + kOffS + khalf * 8192 + (l & 63) * 128;
         // one 32-value half of this thread's state row: operand copy, optional
@@ -524,7 +552,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (state_out) {
 #pragma unroll
                     for (int q = 0; q < 32; ++q)
-                        state_out[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q] * fout;
+                        state_out[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q];
                 }
             } else {
                 uint32_t lo[16], hi[16];
@@ -562,8 +590,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // position to block 0's end when t = -1)
                 const float dnext =
                     last ? 0.f
-                         : ptx::ex2(-sl2 * (float)(min(kBlock, seq - (t + 1) * kBlock) - (t < 0 ? pp.state_shift : 0)));
-                float *snap = t >= 0 ? snapshot_at(sn, bh, t * kBlock + min(kBlock, seq - t * kBlock), kDim) : nullptr;
+                         : ptx::ex2(-sl2 * (float)blen(t + 1));
+                float *snap = t >= 0 && !pp.anti ? snapshot_at(sn, bh, t * kBlock + blen(t), kDim) : nullptr;
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     float sv[32];
@@ -622,7 +650,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ptx::fence_proxy_async_smem();
                     ptx::named_bar_sync(kBarW3, 128);
                     if (leader) {
-                        ptx::tma_store_3d(&tm_o, c.smem + kOffE, 64 * hh, t * kBlock + kRows * (int)rank, bh);
+                        ptx::tma_store_3d(&tm_o, c.smem + kOffE, 64 * hh, tb(t) * kBlock + kRows * (int)rank, bh);
                         ptx::bulk_commit();
                     }
                 }

@@ -187,10 +187,6 @@ def _backward(variant=abi.LA_VARIANT_AUTO, **kw):
     (dict(dv=DQ + 1024), abi.LA_ERR_INVALID_ARG),        # two outputs overlap
     (dict(d_state_in=DSO), abi.LA_ERR_INVALID_ARG),      # overlaps d_state_out
     (dict(d_state_in=S0 + 16), abi.LA_ERR_INVALID_ARG),  # overlaps state_in
-    (dict(ws=None), abi.LA_ERR_INVALID_ARG),              # the tensor-core kernels need a workspace
-    (dict(ws_bytes=1024), abi.LA_ERR_INVALID_ARG),        # too short
-    (dict(ws=WS + 8), abi.LA_ERR_INVALID_ARG),            # misaligned
-    (dict(ws=DQ), abi.LA_ERR_INVALID_ARG),                # overlaps an output
     (dict(variant=abi.LA_VARIANT_TCGEN05), abi.LA_ERR_INVALID_ARG),
     (dict(variant=7), abi.LA_ERR_INVALID_ARG),
     (dict(variant=abi.LA_VARIANT_TCGEN05_PAIR, block=128), abi.LA_ERR_UNSUPPORTED),
@@ -202,13 +198,11 @@ def test_backward_argument_errors(kw, status):
 
 def test_backward_workspace_size():
     ws = abi.lightning_prefill_backward_workspace_size
-    # three token-reversed bf16 copies for the tensor-core kernels, nothing for the CUDA cores
-    assert ws(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_AUTO) == 3 * 64 * 131072 * 128 * 2
-    assert ws(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_SIMT) == 0
-    assert ws(abi.LA_DTYPE_F32, 1, 2, 100, 64, 64, abi.LA_VARIANT_AUTO) == 0
-    assert ws(abi.LA_DTYPE_BF16, 1, 2, 100, 128, 128, abi.LA_VARIANT_TCGEN05_PAIR) == 0  # unsupported
-    # a CUDA-core request needs no workspace at all
-    assert _backward(variant=abi.LA_VARIANT_SIMT, ws=None, ws_bytes=0, batch=0) == abi.LA_OK
+    # no kernel needs a workspace: the anti-causal passes read their operands in place
+    for dt, blk, var in ((abi.LA_DTYPE_BF16, 256, abi.LA_VARIANT_AUTO), (abi.LA_DTYPE_BF16, 256, abi.LA_VARIANT_SIMT),
+                         (abi.LA_DTYPE_F32, 64, abi.LA_VARIANT_AUTO)):
+        assert ws(dt, 1, 64, 131072, 128, blk, var) == 0
+    assert _backward(ws=None, ws_bytes=0, batch=0) == abi.LA_OK
 
 
 def test_backward_trivial_calls_need_no_gpu():

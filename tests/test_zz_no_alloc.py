@@ -14,16 +14,18 @@ def _built():
     abi.load()
 
 
-def test_capacity_and_oversize_requests_are_rejected_before_any_launch():
-    cap = abi.lightning_prefill_backward_noalloc_capacity()
-    assert cap == 64 << 20
-    # the long-context shape needs 6.44 GB of scratch: rejected on the host
-    fake = [0x10000000 * (i + 1) for i in range(12)]
+def test_capacity_and_bad_requests_are_rejected_before_any_launch():
+    assert abi.lightning_prefill_backward_noalloc_capacity() == 64 << 20
+    # argument checks run on the host, before the scratch is looked up or anything launches
+    fake = [0x10000000 * (i + 1) for i in range(8)]
     st = abi.lightning_prefill_backward_noalloc(fake[0], fake[1], fake[2], fake[3], abi.LA_DTYPE_BF16, fake[4],
-                                                1, 64, 131072, 128, 256, None, None, fake[5], fake[6], fake[7],
+                                                1, 64, 131072, 96, 256, None, None, fake[5], fake[6], fake[7],
                                                 None, None, abi.LA_VARIANT_AUTO)
     assert st == abi.LA_ERR_UNSUPPORTED
-    assert "scratch" in abi.last_error_message()
+    st = abi.lightning_prefill_backward_noalloc(fake[0], fake[1], fake[2], fake[3], abi.LA_DTYPE_BF16, fake[4],
+                                                1, 64, 131072, 128, 256, None, None, fake[0], fake[6], fake[7],
+                                                None, None, abi.LA_VARIANT_AUTO)
+    assert st == abi.LA_ERR_INVALID_ARG  # dq overlaps q
 
 
 @pytest.mark.gpu
