@@ -6,8 +6,8 @@ shares no code with it.
 
 The arithmetic lives in ``lightning_oracle.c`` (three forms of the same
 result: F1 definition, F2 token recurrence, F3 blockwise, plus one decode
-step, the state snapshots of a prefix cache and the gradients of one
-prefill; see that file's header for
+step, the state snapshots of a prefix cache, the gradients of one prefill
+and the normalisation and gating of the output; see that file's header for
 the formulas and their sources on the "MINIMAX SIGNAL LAB · M1" page, §03
 Lightning Attention). This module only
 marshals numpy arrays into it.
@@ -43,6 +43,8 @@ def _load():
         lib.la_oracle_snapshots.restype = ctypes.c_int
         lib.la_oracle_backward.argtypes = [vp, vp, vp, vp, ip, fp, ip, ip, ip, ip, fp, fp, dp, dp, dp, dp]
         lib.la_oracle_backward.restype = ctypes.c_int
+        lib.la_oracle_norm_gate.argtypes = [vp, vp, ip, fp, ctypes.c_double, ip, ip, ip, ip, ip, dp]
+        lib.la_oracle_norm_gate.restype = ctypes.c_int
         lib.la_oracle_max_threads.restype = ctypes.c_int
         lib.la_oracle_set_threads.argtypes = [ip]
         _lib = lib
@@ -151,6 +153,30 @@ def backward(q, k, v, d_o, slopes, state_in=None, d_state_out=None):
     if rc != 0:
         raise RuntimeError("oracle backward failed (rc=%d)" % rc)
     return dq, dk, dv, ds_in
+
+
+def norm_gate(o, g, gamma, eps, per_head):
+    """RMS normalisation then sigmoid gating of an attention output.
+
+    o: [batch, heads, seq, dim]; g: [batch, seq, heads*dim] (same dtype);
+    gamma: [heads*dim]. Returns y float64 [batch, seq, heads*dim]."""
+    o = np.ascontiguousarray(o)
+    g = np.ascontiguousarray(g)
+    code = _dtype_code(o)
+    if _dtype_code(g) != code:
+        raise TypeError("o and g must share a dtype")
+    b, h, L, d = o.shape
+    if g.shape != (b, L, h * d):
+        raise ValueError("g must have shape [batch, seq, heads*dim]")
+    gamma = np.ascontiguousarray(gamma, dtype=np.float32)
+    if gamma.shape != (h * d,):
+        raise ValueError("gamma must have shape [heads*dim]")
+    y = np.empty((b, L, h * d), dtype=np.float64)
+    rc = _load().la_oracle_norm_gate(_ptr(o), _ptr(g), code, _ptr(gamma), float(eps), b, h, L, d,
+                                     1 if per_head else 0, _ptr(y))
+    if rc != 0:
+        raise RuntimeError("oracle norm_gate failed (rc=%d)" % rc)
+    return y
 
 
 def decode(q, k, v, slopes, state):

@@ -35,7 +35,8 @@
  *   F3 la_oracle_blockwise  : the block formulas of §03 for a given B.
  * plus la_oracle_decode, one recurrent step for a single new token,
  * la_oracle_snapshots, the state after every `interval` tokens (F2's state),
- * and la_oracle_backward, the gradients of one prefill.
+ * la_oracle_backward, the gradients of one prefill, and la_oracle_norm_gate,
+ * the normalisation and gating of the attention output.
  *
  * Layouts: q, k, v, o are [batch][heads][seq][dim] contiguous (o for decode
  * is [batch][heads][dim]); states are [batch][heads][dim(k)][dim(v)].
@@ -314,6 +315,46 @@ int la_oracle_backward(const void *q, const void *k, const void *v, const void *
         free(S); free(R); free(Q); free(K); free(V); free(G);
     }
     return fail;
+}
+
+/* Normalisation and gating of the attention output. "MINIMAX SIGNAL LAB ·
+ * M1", §03 Lightning Attention: the figure adds the intra- and inter-block
+ * outputs, then normalises and gates them; the pages print no formula. The
+ * reading taken: an RMS normalisation with a learned per-channel weight, then
+ * an elementwise sigmoid gate,
+ *   y[b][l][n] = gamma[n] * x[n] / sqrt(mean_{n' in group(n)} x[n']^2 + eps)
+ *                * 1 / (1 + e^{-g[b][l][n]})
+ * over the token's channels n = h*dim + c, x[n] = o[b][h][l][c]; the RMS is
+ * taken per head (group = the head's dim channels, per_head = 1) or over all
+ * heads*dim channels of the token (per_head = 0).
+ * o: [batch][heads][seq][dim]; g and y: [batch][seq][heads*dim]; gamma:
+ * [heads*dim] float32; o and g have one dtype; y is float64. */
+int la_oracle_norm_gate(const void *o, const void *g, int dtype, const float *gamma, double eps, int batch,
+                        int heads, int seq, int dim, int per_head, double *y) {
+    if (!o || !g || !gamma || !y) return 1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16) return 1;
+    if (batch < 0 || heads <= 0 || seq < 0 || dim <= 0 || eps < 0.0) return 1;
+    const size_t N = (size_t)heads * dim, L = (size_t)seq, d = (size_t)dim;
+    const long T = (long)batch * seq;
+#pragma omp parallel for schedule(static)
+    for (long tk = 0; tk < T; ++tk) {
+        const size_t b = (size_t)tk / L, l = (size_t)tk % L;
+        const size_t group = per_head ? d : N;
+        for (size_t g0 = 0; g0 < N; g0 += group) {
+            double ss = 0.0;
+            for (size_t n = g0; n < g0 + group; ++n) {
+                const double x = widen(o, dtype, ((b * heads + n / d) * L + l) * d + n % d);
+                ss += x * x;
+            }
+            const double inv = 1.0 / sqrt(ss / (double)group + eps);
+            for (size_t n = g0; n < g0 + group; ++n) {
+                const double x = widen(o, dtype, ((b * heads + n / d) * L + l) * d + n % d);
+                const double gv = widen(g, dtype, (size_t)tk * N + n);
+                y[(size_t)tk * N + n] = (double)gamma[n] * x * inv / (1.0 + exp(-gv));
+            }
+        }
+    }
+    return 0;
 }
 
 /* F3: the blockwise method, block by block, as the block formulas state it. */

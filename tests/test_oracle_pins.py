@@ -295,3 +295,47 @@ def test_backward_of_an_empty_sequence_passes_the_state_gradient():
     dq, dk, dv, ds_in = oracle.backward(z, z, z, z, SLOPES_MIX[:2], None, ds_out)
     assert dq.shape == (b, h, 0, d)
     np.testing.assert_array_equal(ds_in, ds_out.astype(np.float64))
+
+
+def _sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x.astype(np.float64)))
+
+
+@pytest.mark.parametrize("per_head", [True, False])
+def test_norm_gate_closed_forms(per_head):
+    b, h, L, d = 2, 3, 5, 4
+    g = _rand((b, L, h * d), 60)
+    gamma = _rand((h * d,), 61)
+    # constant channels c: every group's rms is |c|, so y = gamma * sign(c) * |c| / sqrt(c^2 + eps) * sigmoid(g)
+    for c, eps in ((0.75, 0.0), (-2.0, 0.5)):
+        o = np.full((b, h, L, d), c, np.float32)
+        y = oracle.norm_gate(o, g, gamma, eps, per_head)
+        want = gamma.astype(np.float64) * c / np.sqrt(c * c + eps) * _sigmoid(g)
+        _close(y, want, 1e-12)
+    # a zero gate halves; a large positive gate passes the normalised value through
+    o = _rand((b, h, L, d), 62)
+    y0 = oracle.norm_gate(o, np.zeros_like(g), gamma, 1e-6, per_head)
+    y1 = oracle.norm_gate(o, np.full_like(g, 60.0), gamma, 1e-6, per_head)
+    _close(y0, 0.5 * y1, 1e-12)
+
+
+@pytest.mark.parametrize("per_head", [True, False])
+def test_norm_gate_is_scale_invariant_and_groups_as_stated(per_head):
+    b, h, L, d = 1, 4, 3, 8
+    o = _rand((b, h, L, d), 63)
+    g = _rand((b, L, h * d), 64)
+    gamma = np.ones((h * d,), np.float32)
+    y = oracle.norm_gate(o, g, gamma, 0.0, per_head)
+    _close(oracle.norm_gate(o * np.float32(4.0), g, gamma, 0.0, per_head), y, 1e-12)
+    # with gamma = 1 and eps = 0, every group of the normalised output has mean square 1
+    x = y / _sigmoid(g)
+    grp = d if per_head else h * d
+    ms = np.mean(x.reshape(b, L, (h * d) // grp, grp) ** 2, axis=-1)
+    _close(ms, np.ones_like(ms), 1e-12)
+    # token channel n = head * dim + c reads o[b, head, l, c]
+    if per_head:
+        one = np.zeros_like(o)
+        one[0, 2, 1, 5] = 3.0
+        yy = oracle.norm_gate(one, np.full_like(g, 60.0), gamma, 1e-30, True)  # eps > 0: zero heads stay 0
+        assert abs(yy[0, 1, 2 * d + 5] - np.sqrt(d)) < 1e-9
+        assert np.count_nonzero(yy[0, 1]) == 1
