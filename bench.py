@@ -344,6 +344,9 @@ def run_ours(args):
     snaps = (run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, ms_per_step)
              if args.snapshot_interval > 0 and w.seq >= args.snapshot_interval else None)
 
+    # normalisation and gating of the prefill's output
+    ng = run_norm_gate_leg(w, dev, stream, o, dcode, args, world) if args.norm_gate_steps > 0 else None
+
     # gradients of the same prefill (dq, dk, dv, d state_in)
     bwd = run_backward_leg(w, dev, stream, inp, dcode, args, world) if args.backward_steps > 0 else None
 
@@ -365,6 +368,7 @@ def run_ours(args):
         "decode": dec,
         "e2e": e2e,
         "snapshots": snaps,
+        "norm_gate": ng,
         "backward": bwd,
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
@@ -448,6 +452,40 @@ def run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, plain_ms):
     return {"interval": interval, "count": n, "steps": steps, "ms_per_step": round(ms, 4),
             "overhead_vs_plain_pct": round(100.0 * (ms / plain_ms - 1.0), 2),
             "snapshot_bytes_per_step": int(snaps.numel() * 4)}
+
+
+def run_norm_gate_leg(w, dev, stream, o, dcode, args, world):
+    """lightning_norm_gate on the prefill's output: RMS over each token's
+    heads*dim channels, sigmoid gate; timed like the main leg."""
+    import torch
+    from linear_attention_lightning_b200 import abi
+    g = torch.Generator(device=dev).manual_seed(w.seed + 2000)
+    gate = torch.randn((w.batch, w.seq, w.heads * w.dim), generator=g, device=dev).to(o.dtype)
+    gamma = torch.ones(w.heads * w.dim, device=dev)
+    y = torch.empty((w.batch, w.seq, w.heads * w.dim), dtype=o.dtype, device=dev)
+    sp = stream.cuda_stream
+
+    def step():
+        abi.check(abi.lightning_norm_gate(o.data_ptr(), gate.data_ptr(), dcode, gamma.data_ptr(), 1e-6, w.batch,
+                                          w.heads, w.seq, w.dim, 0, y.data_ptr(), sp))
+
+    for _ in range(args.warmup):
+        step()
+    steps = args.norm_gate_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    by = 3 * o.numel() * o.element_size() + gamma.numel() * 4  # o, gate read; y written
+    gbs = by / (ms / 1e3) / 1e9
+    return {"steps": steps, "ms_per_step": round(ms, 4), "per": "token (heads*dim channels)",
+            "tokens_per_s": round(world * w.batch * w.seq / (ms / 1e3), 1),
+            "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s")}
 
 
 def run_backward_leg(w, dev, stream, inp, dcode, args, world):
@@ -556,6 +594,8 @@ def parse_args(argv=None):
     p.add_argument("--decode-steps", type=int, default=1000)
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--norm-gate-steps", type=int, default=20,
+                   help="timed steps of the norm-and-gate epilogue leg (0 skips it)")
     p.add_argument("--backward-steps", type=int, default=10,
                    help="timed steps of the gradient leg (0 skips it)")
     p.add_argument("--snapshot-interval", type=int, default=16384,

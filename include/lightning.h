@@ -211,6 +211,28 @@ size_t lightning_prefill_backward_noalloc_capacity(void);
 size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int heads, int seq, int dim,
                                                  int block, int variant);
 
+/*
+ * Normalisation and gating of the attention output. Source: "MINIMAX SIGNAL
+ * LAB · M1", §03 Lightning Attention: the figure sums the intra- and
+ * inter-block outputs, then normalises and gates them; the pages print no
+ * formula. The reading implemented: RMS normalisation with a learned
+ * per-channel weight, then an elementwise sigmoid gate,
+ *   y[b][l][n] = gamma[n] x[n] / sqrt(mean_{group} x^2 + eps) * 1 / (1 + e^{-gate[b][l][n]})
+ * over the token's channels n = h*dim + c, x[n] = o[b][h][l][c]. The mean
+ * runs over the head's dim channels (per_head != 0) or over all heads*dim
+ * channels of the token (per_head == 0).
+ *
+ *   o      [batch][heads][seq][dim], dtype (lightning_prefill's output).
+ *   gate   [batch][seq][heads*dim], dtype (the gate projection's output).
+ *   gamma  [heads*dim] float32.   eps: finite, >= 0.
+ *   y      [batch][seq][heads*dim], dtype; written; must not overlap o, gate
+ *          or gamma.
+ * dim 64 or 128; heads*dim at most 16384 (bf16) or 8192 (f32) channels, else
+ * LA_ERR_UNSUPPORTED. Device pointers, caller-owned, 16-byte aligned.
+ */
+la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, const float *gamma, float eps,
+                              int batch, int heads, int seq, int dim, int per_head, void *y, void *stream);
+
 /* Number of snapshots lightning_prefill_snapshots writes per (batch, head):
  * seq / interval, or -1 if seq < 0 or interval < 1. Host only. */
 int lightning_prefill_snapshot_count(int seq, int interval);

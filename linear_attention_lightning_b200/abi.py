@@ -30,6 +30,7 @@ _SIGNATURES = {
     "lightning_prefill_snapshots": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp,
                                      _i], _i),
     "lightning_prefill_snapshot_count": ([_i, _i], _i),
+    "lightning_norm_gate": ([_vp, _vp, _i, _vp, ctypes.c_float, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "lightning_prefill_backward": ([_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _sz, _vp, _i], _i),
     "lightning_prefill_backward_workspace_size": ([_i, _i, _i, _i, _i, _i, _i], _sz),
@@ -138,6 +139,10 @@ def lightning_prefill_backward_noalloc_capacity():
 
 def lightning_prefill_backward_workspace_size(dtype, batch, heads, seq, dim, block, variant):
     return load().lightning_prefill_backward_workspace_size(dtype, batch, heads, seq, dim, block, variant)
+
+
+def lightning_norm_gate(o, gate, dtype, gamma, eps, batch, heads, seq, dim, per_head, y, stream):
+    return load().lightning_norm_gate(o, gate, dtype, gamma, eps, batch, heads, seq, dim, per_head, y, stream)
 
 
 def lightning_prefill_snapshot_count(seq, interval):

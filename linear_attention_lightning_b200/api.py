@@ -138,6 +138,30 @@ def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, d_o: tor
     return dq, dk, dv, ds_in
 
 
+def norm_gate(o: torch.Tensor, gate: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+              per_head: bool = False, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """lightning_norm_gate: RMS-normalise the attention output o [batch, heads,
+    seq, dim] per token (or per head) and gate it with sigmoid(gate); returns y
+    [batch, seq, heads*dim]."""
+    if o.dtype not in _DTYPES:
+        raise ValueError("o must be float32 or bfloat16")
+    if o.dim() != 4:
+        raise ValueError("o must be [batch, heads, seq, dim]")
+    b, h, L, d = o.shape
+    _need_cuda("o", o, o.dtype)
+    _need_cuda("gate", gate, o.dtype)
+    if tuple(gate.shape) != (b, L, h * d):
+        raise ValueError("gate must be [batch, seq, heads*dim]")
+    _need_cuda("gamma", gamma, torch.float32)
+    if tuple(gamma.shape) != (h * d,):
+        raise ValueError("gamma must be [heads*dim]")
+    if y is None:
+        y = torch.empty((b, L, h * d), dtype=o.dtype, device=o.device)
+    abi.check(abi.lightning_norm_gate(_ptr(o), _ptr(gate), _DTYPES[o.dtype], _ptr(gamma), float(eps), b, h, L, d,
+                                      1 if per_head else 0, _ptr(y), _stream(stream)))
+    return y
+
+
 def prefill_variant(dtype: torch.dtype, batch: int, heads: int, seq: int, dim: int, block: int,
                     variant: str = "auto") -> str:
     """Which kernel lightning_prefill would run: "simt", "tcgen05" or "pair"."""

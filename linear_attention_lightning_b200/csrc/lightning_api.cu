@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_simt.cuh"
+#include "norm_gate.cuh"
 #include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
 
@@ -160,6 +161,64 @@ la_status launch_simt(const PrefillArgs &a, cudaStream_t stream) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "prefill_simt launch");
     return ok();
+}
+
+struct NgArgs {
+    const void *o, *gate;
+    const float *gamma;
+    float eps;
+    int batch, heads, seq, dim, per_head;
+    void *y;
+    long long tokens;
+    cudaStream_t stream;
+};
+
+// 3-D tensor map without swizzle over a tensor of 16- or 32-bit elements.
+bool make_plain_map(CUtensorMap *map, const void *base, bool bf16, const cuuint64_t (&dims)[3],
+                    const cuuint64_t (&strides)[2], const cuuint32_t (&box)[3], std::string *err) {
+    auto fn = la::tc::encode_fn(err);
+    if (!fn) return false;
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *err = "cuTensorMapEncodeTiled failed (CUresult " + std::to_string((int)r) + ")";
+        return false;
+    }
+    return true;
+}
+
+template <typename T, int U>
+la_status launch_norm_gate(const NgArgs &a) {
+    const size_t eb = sizeof(T);
+    const long long n_ch = (long long)a.heads * a.dim;
+    long long tile = (long long)la::kNgTileBytes / (n_ch * (long long)eb);
+    tile = tile < 1 ? 1 : (tile > 64 ? 64 : tile);
+    const bool bf16 = sizeof(T) == 2;
+    CUtensorMap mo, mg;
+    // o: [batch*heads][seq][dim], box = one tile of tokens for every head of a batch
+    const cuuint64_t odims[3] = {(cuuint64_t)a.dim, (cuuint64_t)a.seq, (cuuint64_t)a.batch * a.heads};
+    const cuuint64_t ostr[2] = {(cuuint64_t)a.dim * eb, (cuuint64_t)a.seq * a.dim * eb};
+    const cuuint32_t obox[3] = {(cuuint32_t)a.dim, (cuuint32_t)tile, (cuuint32_t)a.heads};
+    // gate: [batch*seq][heads][dim], box = one tile of tokens
+    const cuuint64_t gdims[3] = {(cuuint64_t)a.dim, (cuuint64_t)a.heads, (cuuint64_t)a.batch * a.seq};
+    const cuuint64_t gstr[2] = {(cuuint64_t)a.dim * eb, (cuuint64_t)n_ch * eb};
+    const cuuint32_t gbox[3] = {(cuuint32_t)a.dim, (cuuint32_t)a.heads, (cuuint32_t)tile};
+    if (!make_plain_map(&mo, a.o, bf16, odims, ostr, obox, &g_last_error) ||
+        !make_plain_map(&mg, a.gate, bf16, gdims, gstr, gbox, &g_last_error))
+        return LA_ERR_CUDA;
+    auto kern = la::norm_gate_kernel<T, U>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)la::kNgSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(norm_gate)");
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long tiles = (long long)a.batch * ((a.seq + tile - 1) / tile);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    kern<<<grid, la::kNgThreads, la::kNgSmemBytes, a.stream>>>(mo, mg, a.gamma, a.eps, a.batch, a.heads, a.seq, a.dim,
+                                                              a.per_head, (int)tile, static_cast<T *>(a.y));
+    e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "norm_gate launch");
 }
 
 // One launch of the CUDA-core kernel as a pass of the backward computation.
@@ -450,6 +509,47 @@ size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int 
     const int chosen = choose_backward_variant(dtype, dim, block, variant);
     return chosen < 0 ? 0 : backward_workspace_bytes(dtype, batch, heads, seq, dim, chosen);
 }
+
+la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, const float *gamma, float eps,
+                              int batch, int heads, int seq, int dim, int per_head, void *y, void *stream) {
+    if (dtype != LA_DTYPE_F32 && dtype != LA_DTYPE_BF16)
+        return fail(LA_ERR_INVALID_ARG, "dtype %d is neither LA_DTYPE_F32 nor LA_DTYPE_BF16", (int)dtype);
+    if (batch < 0 || heads < 1 || seq < 0)
+        return fail(LA_ERR_INVALID_ARG, "need batch >= 0, heads >= 1, seq >= 0 (got %d, %d, %d)", batch, heads, seq);
+    if (!(eps >= 0.f) || eps > 3.0e38f) return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    if (dim != 64 && dim != 128) return fail(LA_ERR_UNSUPPORTED, "dim %d unsupported (64 or 128)", dim);
+    const size_t eb = elem_bytes(dtype);
+    const long long max_ch = (long long)la::kNgThreads * la::kNgMaxChunks * (long long)(16 / eb);
+    if ((long long)heads * dim > max_ch)
+        return fail(LA_ERR_UNSUPPORTED, "heads*dim %lld exceeds %lld channels per token",
+                    (long long)heads * dim, max_ch);
+    const long long tokens = (long long)batch * seq;
+    if (tokens == 0) return ok();
+    if (!o || !gate || !gamma || !y) return fail(LA_ERR_INVALID_ARG, "o, gate, gamma and y must be non-NULL");
+    const void *ptrs[] = {o, gate, gamma, y};
+    const char *names[] = {"o", "gate", "gamma", "y"};
+    for (int i = 0; i < 4; ++i)
+        if (!aligned16(ptrs[i])) return fail(LA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+    const size_t bytes = (size_t)tokens * heads * dim * eb;
+    const Range ry = range_of(y, bytes);
+    if (overlaps(ry, range_of(o, bytes)) || overlaps(ry, range_of(gate, bytes)) ||
+        overlaps(ry, range_of(gamma, sizeof(float) * heads * dim)))
+        return fail(LA_ERR_INVALID_ARG, "y overlaps o, gate or gamma");
+    // chunks of 16 bytes per thread, and resident CTAs on every SM, each walking the tokens
+    const long long chunks_per_thread = ((long long)heads * dim * (long long)eb / 16 + la::kNgThreads - 1) / la::kNgThreads;
+    const int U = chunks_per_thread <= 1 ? 1 : chunks_per_thread <= 2 ? 2 : 4;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const NgArgs args{o, gate, gamma, eps, batch, heads, seq, dim, per_head ? 1 : 0, y, tokens, st};
+    la_status rs;
+    if (dtype == LA_DTYPE_BF16)
+        rs = U == 1 ? launch_norm_gate<__nv_bfloat16, 1>(args) : U == 2 ? launch_norm_gate<__nv_bfloat16, 2>(args)
+                    : launch_norm_gate<__nv_bfloat16, 4>(args);
+    else
+        rs = U == 1 ? launch_norm_gate<float, 1>(args) : U == 2 ? launch_norm_gate<float, 2>(args)
+                    : launch_norm_gate<float, 4>(args);
+    return rs;
+}
+
 
 int lightning_prefill_snapshot_count(int seq, int interval) {
     if (seq < 0 || interval < 1) return -1;

@@ -208,3 +208,37 @@ def test_backward_workspace_size():
 def test_backward_trivial_calls_need_no_gpu():
     assert _backward(batch=0) == abi.LA_OK
     assert _backward(seq=0, d_state_in=None) == abi.LA_OK
+
+
+G_, GM, Y_ = (0x10000000 * (i + 20) for i in range(3))
+
+
+def _norm_gate(**kw):
+    a = dict(o=O, gate=G_, dtype=abi.LA_DTYPE_BF16, gamma=GM, eps=1e-6, batch=1, heads=64, seq=16, dim=128,
+             per_head=0, y=Y_)
+    a.update(kw)
+    return abi.lightning_norm_gate(a["o"], a["gate"], a["dtype"], a["gamma"], a["eps"], a["batch"], a["heads"],
+                                   a["seq"], a["dim"], a["per_head"], a["y"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype=3), abi.LA_ERR_INVALID_ARG),
+    (dict(heads=0), abi.LA_ERR_INVALID_ARG),
+    (dict(seq=-1), abi.LA_ERR_INVALID_ARG),
+    (dict(eps=-1.0), abi.LA_ERR_INVALID_ARG),
+    (dict(eps=float("nan")), abi.LA_ERR_INVALID_ARG),
+    (dict(dim=32), abi.LA_ERR_UNSUPPORTED),
+    (dict(heads=129), abi.LA_ERR_UNSUPPORTED),                           # 16512 bf16 channels per token
+    (dict(heads=65, dtype=abi.LA_DTYPE_F32), abi.LA_ERR_UNSUPPORTED),    # 8320 f32 channels
+    (dict(gate=None), abi.LA_ERR_INVALID_ARG),
+    (dict(y=Y_ + 4), abi.LA_ERR_INVALID_ARG),
+    (dict(y=O + 1024), abi.LA_ERR_INVALID_ARG),                          # overlaps o
+])
+def test_norm_gate_argument_errors(kw, status):
+    assert _norm_gate(**kw) == status
+    assert abi.last_error_message() != ""
+
+
+def test_norm_gate_empty_needs_no_gpu():
+    assert _norm_gate(batch=0) == abi.LA_OK
+    assert _norm_gate(seq=0, o=None, y=None) == abi.LA_OK
