@@ -6,8 +6,9 @@ shares no code with it.
 
 The arithmetic lives in ``lightning_oracle.c`` (three forms of the same
 result: F1 definition, F2 token recurrence, F3 blockwise, plus one decode
-step, the state snapshots of a prefix cache, the gradients of one prefill
-and the normalisation and gating of the output; see that file's header for
+step, the state snapshots of a prefix cache, the gradients of one prefill,
+the normalisation and gating of the output and one decode step of the
+softmax GQA layer; see that file's header for
 the formulas and their sources on the "MINIMAX SIGNAL LAB · M1" page, §03
 Lightning Attention). This module only
 marshals numpy arrays into it.
@@ -45,6 +46,9 @@ def _load():
         lib.la_oracle_backward.restype = ctypes.c_int
         lib.la_oracle_norm_gate.argtypes = [vp, vp, ip, fp, ctypes.c_double, ip, ip, ip, ip, ip, dp]
         lib.la_oracle_norm_gate.restype = ctypes.c_int
+        lib.la_oracle_gqa_decode.argtypes = [vp, vp, vp, vp, vp, ip, vp, ip, ip, ip, ip, ip, ip, ctypes.c_double,
+                                             ctypes.c_double, dp]
+        lib.la_oracle_gqa_decode.restype = ctypes.c_int
         lib.la_oracle_max_threads.restype = ctypes.c_int
         lib.la_oracle_set_threads.argtypes = [ip]
         _lib = lib
@@ -177,6 +181,46 @@ def norm_gate(o, g, gamma, eps, per_head):
     if rc != 0:
         raise RuntimeError("oracle norm_gate failed (rc=%d)" % rc)
     return y
+
+
+def gqa_decode(q, k_new, v_new, k_cache, v_cache, pos, rot, base, scale):
+    """One decode step of the softmax GQA layer (RoPE on the first `rot` dims).
+
+    q: [batch, heads, dim]; k_new, v_new: [batch, kv_heads, dim]; caches:
+    [batch, kv_heads, cap, dim] (rotated keys; positions < pos[b] filled);
+    pos: [batch] int. Returns o float64 [batch, heads, dim]."""
+    q, k_new, v_new, k_cache, v_cache = (np.ascontiguousarray(x) for x in (q, k_new, v_new, k_cache, v_cache))
+    code = _dtype_code(q)
+    for x in (k_new, v_new, k_cache, v_cache):
+        if _dtype_code(x) != code:
+            raise TypeError("all gqa inputs must share a dtype")
+    b, h, d = q.shape
+    bk, hk, cap, dk = k_cache.shape
+    if (bk, dk) != (b, d) or k_new.shape != (b, hk, d) or v_new.shape != (b, hk, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("inconsistent gqa shapes")
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    if pos.shape != (b,):
+        raise ValueError("pos must have shape [batch]")
+    o = np.empty((b, h, d), dtype=np.float64)
+    rc = _load().la_oracle_gqa_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), code,
+                                      _ptr(pos), b, h, hk, d, cap, int(rot), float(base), float(scale), _ptr(o))
+    if rc != 0:
+        raise RuntimeError("oracle gqa_decode failed (rc=%d)" % rc)
+    return o
+
+
+def rope(x, pos, rot, base):
+    """RoPE of the last axis of x (float64 reference of the oracle's rotation,
+    used by tests to fill key caches): x [..., dim] at position pos."""
+    x = np.asarray(x, dtype=np.float64)
+    half = rot // 2
+    i = np.arange(half, dtype=np.float64)
+    ang = float(pos) * np.power(float(base), -2.0 * i / rot)
+    out = x.copy()
+    cs, sn = np.cos(ang), np.sin(ang)
+    out[..., :half] = x[..., :half] * cs - x[..., half:rot] * sn
+    out[..., half:rot] = x[..., half:rot] * cs + x[..., :half] * sn
+    return out
 
 
 def decode(q, k, v, slopes, state):

@@ -35,8 +35,9 @@
  *   F3 la_oracle_blockwise  : the block formulas of §03 for a given B.
  * plus la_oracle_decode, one recurrent step for a single new token,
  * la_oracle_snapshots, the state after every `interval` tokens (F2's state),
- * la_oracle_backward, the gradients of one prefill, and la_oracle_norm_gate,
- * the normalisation and gating of the attention output.
+ * la_oracle_backward, the gradients of one prefill, la_oracle_norm_gate, the
+ * normalisation and gating of the attention output, and la_oracle_gqa_decode,
+ * one decode step of the softmax attention layer of the hybrid model.
  *
  * Layouts: q, k, v, o are [batch][heads][seq][dim] contiguous (o for decode
  * is [batch][heads][dim]); states are [batch][heads][dim(k)][dim(v)].
@@ -355,6 +356,86 @@ int la_oracle_norm_gate(const void *o, const void *g, int dtype, const float *ga
         }
     }
     return 0;
+}
+
+/* Rotary position embedding on the first `rot` dims of a head, rotate-half
+ * pairing: for i < rot/2 the pair (x[i], x[i + rot/2]) turns by pos * theta_i,
+ * theta_i = base^{-2i/rot}; dims from rot on are unchanged. */
+static void rope_head(const double *x, double *out, int dim, int rot, double base, long pos) {
+    const int half = rot / 2;
+    for (int c = 0; c < dim; ++c) out[c] = x[c];
+    for (int i = 0; i < half; ++i) {
+        const double ang = (double)pos * pow(base, -2.0 * i / (double)rot);
+        const double cs = cos(ang), sn = sin(ang);
+        out[i] = x[i] * cs - x[i + half] * sn;
+        out[i + half] = x[i + half] * cs + x[i] * sn;
+    }
+}
+
+/* One decode step of the softmax attention layer that M1 places after every
+ * seven Lightning layers ("MINIMAX SIGNAL LAB · M1", §02: 64 query heads x 128,
+ * softmax K/V 8 x 128, RoPE on 64 of the 128 dims in the softmax layers only;
+ * §04: the softmax layers keep a bf16 KV cache that grows with the context).
+ * Readings (the pages print no formula): grouped-query attention, query head
+ * h reads KV head h / (heads / kv_heads); scores scaled by `scale`; RoPE as in
+ * rope_head with the token's position; the cache holds rotated keys.
+ * Per sequence b the new token sits at position pos[b]: its key (rotated) and
+ * value join the cache there, and each query head attends to positions
+ * 0 .. pos[b]:  o = sum_p softmax_p(scale * rope(q) . k_p) v_p.
+ * q: [batch][heads][dim]; k_new, v_new: [batch][kv_heads][dim]; caches:
+ * [batch][kv_heads][cap][dim] with positions < pos[b] filled; o: float64
+ * [batch][heads][dim]. All inputs share `dtype`. */
+int la_oracle_gqa_decode(const void *q, const void *k_new, const void *v_new, const void *k_cache,
+                         const void *v_cache, int dtype, const int *pos, int batch, int heads, int kv_heads,
+                         int dim, int cap, int rot, double base, double scale, double *o) {
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !o) return 1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16) return 1;
+    if (batch < 0 || kv_heads <= 0 || heads % kv_heads != 0 || dim <= 0 || rot < 0 || rot > dim || rot % 2)
+        return 1;
+    for (int b = 0; b < batch; ++b)
+        if (pos[b] < 0 || pos[b] >= cap) return 1;
+    const int group = heads / kv_heads;
+    const size_t d = (size_t)dim;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < (long)batch * heads; ++bh) {
+        const int b = (int)(bh / heads), h = (int)(bh % heads), hk = h / group;
+        const long P = pos[b];
+        double *x = malloc(sizeof(double) * d * 4), *sc = malloc(sizeof(double) * (size_t)(P + 1));
+        if (!x || !sc) {
+            fail = 1;
+            free(x); free(sc);
+            continue;
+        }
+        double *qr = x, *kr = x + d, *tmp = x + 2 * d, *acc = x + 3 * d;
+        for (size_t c = 0; c < d; ++c) tmp[c] = widen(q, dtype, (size_t)bh * d + c);
+        rope_head(tmp, qr, dim, rot, base, P);
+        const size_t kv = (size_t)b * kv_heads + hk;
+        double mx = -INFINITY;
+        for (long p = 0; p <= P; ++p) {
+            if (p < P) {
+                for (size_t c = 0; c < d; ++c) kr[c] = widen(k_cache, dtype, (kv * cap + p) * d + c);
+            } else {
+                for (size_t c = 0; c < d; ++c) tmp[c] = widen(k_new, dtype, kv * d + c);
+                rope_head(tmp, kr, dim, rot, base, P);
+            }
+            double dot = 0.0;
+            for (size_t c = 0; c < d; ++c) dot += qr[c] * kr[c];
+            sc[p] = scale * dot;
+            if (sc[p] > mx) mx = sc[p];
+        }
+        double den = 0.0;
+        for (size_t c = 0; c < d; ++c) acc[c] = 0.0;
+        for (long p = 0; p <= P; ++p) {
+            const double w = exp(sc[p] - mx);
+            den += w;
+            for (size_t c = 0; c < d; ++c)
+                acc[c] += w * (p < P ? widen(v_cache, dtype, (kv * cap + p) * d + c) : widen(v_new, dtype, kv * d + c));
+        }
+        for (size_t c = 0; c < d; ++c) o[(size_t)bh * d + c] = acc[c] / den;
+        free(x); free(sc);
+    }
+    return fail;
 }
 
 /* F3: the blockwise method, block by block, as the block formulas state it. */

@@ -339,3 +339,79 @@ def test_norm_gate_is_scale_invariant_and_groups_as_stated(per_head):
         yy = oracle.norm_gate(one, np.full_like(g, 60.0), gamma, 1e-30, True)  # eps > 0: zero heads stay 0
         assert abs(yy[0, 1, 2 * d + 5] - np.sqrt(d)) < 1e-9
         assert np.count_nonzero(yy[0, 1]) == 1
+
+
+def _gqa_case(b=2, h=8, hk=2, d=16, cap=12, seed=70):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((b, h, d)).astype(np.float32)
+    kn = rng.standard_normal((b, hk, d)).astype(np.float32)
+    vn = rng.standard_normal((b, hk, d)).astype(np.float32)
+    kc = rng.standard_normal((b, hk, cap, d)).astype(np.float32)
+    vc = rng.standard_normal((b, hk, cap, d)).astype(np.float32)
+    return q, kn, vn, kc, vc
+
+
+def test_rope_is_a_rotation_of_relative_position():
+    rng = np.random.default_rng(71)
+    x, y = rng.standard_normal(16), rng.standard_normal(16)
+    np.testing.assert_allclose(oracle.rope(x, 0, 8, 1e4), x, rtol=0, atol=0)        # position 0: identity
+    np.testing.assert_allclose(np.linalg.norm(oracle.rope(x, 777, 8, 1e4)), np.linalg.norm(x), rtol=1e-13)
+    np.testing.assert_array_equal(oracle.rope(x, 55, 8, 1e4)[8:], x[8:])           # dims past rot untouched
+    a = oracle.rope(x, 40, 8, 1e4) @ oracle.rope(y, 13, 8, 1e4)
+    b = oracle.rope(x, 1040, 8, 1e4) @ oracle.rope(y, 1013, 8, 1e4)
+    assert abs(a - b) < 1e-10                                                      # only m - n matters
+
+
+def test_gqa_decode_special_cases():
+    q, kn, vn, kc, vc = _gqa_case()
+    b, h, d = q.shape
+    hk = kn.shape[1]
+    # position 0: the only key is the new one, so o is its value for every query head
+    o = oracle.gqa_decode(q, kn, vn, kc, vc, np.zeros(b, np.int32), 8, 1e4, 0.25)
+    for hh in range(h):
+        np.testing.assert_allclose(o[:, hh], vn[:, hh // (h // hk)].astype(np.float64), rtol=0, atol=1e-14)
+    # identical keys everywhere: softmax is uniform, o = mean of the values
+    kcu = np.zeros_like(kc)
+    knu = np.zeros_like(kn)
+    pos = np.array([5, 9], np.int32)
+    o = oracle.gqa_decode(q, knu, vn, kcu, vc, pos, 8, 1e4, 0.25)
+    for bb in range(b):
+        for hh in range(h):
+            g = hh // (h // hk)
+            want = (vc[bb, g, :pos[bb]].astype(np.float64).sum(0) + vn[bb, g]) / (pos[bb] + 1)
+            np.testing.assert_allclose(o[bb, hh], want, rtol=1e-12, atol=1e-12)
+    # one key aligned with a large query: softmax saturates on it
+    qq = np.zeros_like(q)
+    qq[:, :, 12] = 50.0                       # dim 12 lies past the rotated dims
+    kca = np.zeros_like(kc)
+    kca[:, :, 3, 12] = 50.0
+    o = oracle.gqa_decode(qq, np.zeros_like(kn), vn, kca, vc, pos, 8, 1e4, 1.0)
+    for hh in range(h):
+        np.testing.assert_allclose(o[:, hh], vc[:, hh // (h // hk), 3].astype(np.float64), rtol=0, atol=1e-9)
+
+
+def test_gqa_decode_matches_a_numpy_softmax_with_grouping():
+    # brute force on a tiny case: numpy softmax over explicitly assembled keys
+    q, kn, vn, kc, vc = _gqa_case(b=1, h=4, hk=2, d=8, cap=6, seed=72)
+    pos = np.array([4], np.int32)
+    o = oracle.gqa_decode(q, kn, vn, kc, vc, pos, 4, 100.0, 0.3)
+    for hh in range(4):
+        g = hh // 2
+        keys = np.concatenate([kc[0, g, :4].astype(np.float64), oracle.rope(kn[0, g], 4, 4, 100.0)[None]], 0)
+        vals = np.concatenate([vc[0, g, :4].astype(np.float64), vn[0, g].astype(np.float64)[None]], 0)
+        s = 0.3 * keys @ oracle.rope(q[0, hh], 4, 4, 100.0)
+        w = np.exp(s - s.max())
+        np.testing.assert_allclose(o[0, hh], (w / w.sum()) @ vals, rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_decode_rotates_query_and_new_key_alike():
+    # cached keys zero: only the new key scores, with rope(q, P) . rope(k, P) = q . k at any P,
+    # so o = (sum_{p<P} v_p + e^{s} v_new) / (P + e^{s}), s = scale * q . k
+    q, kn, vn, kc, vc = _gqa_case(b=1, h=4, hk=1, d=16, cap=40, seed=73)
+    z = np.zeros_like(kc)
+    for P in (0, 7, 39):
+        o = oracle.gqa_decode(q, kn, vn, z, vc, np.array([P], np.int32), 16, 500.0, 0.2)
+        for hh in range(4):
+            s = 0.2 * float(q[0, hh].astype(np.float64) @ kn[0, 0].astype(np.float64))
+            want = (vc[0, 0, :P].astype(np.float64).sum(0) + np.exp(s) * vn[0, 0]) / (P + np.exp(s))
+            np.testing.assert_allclose(o[0, hh], want, rtol=1e-12, atol=1e-12)
