@@ -347,6 +347,9 @@ def run_ours(args):
     # normalisation and gating of the prefill's output
     ng = run_norm_gate_leg(w, dev, stream, o, dcode, args, world) if args.norm_gate_steps > 0 else None
 
+    # decode step of the softmax GQA layer the hybrid model interleaves
+    gqa = run_gqa_leg(dev, stream, args, world) if args.gqa_steps > 0 else None
+
     # gradients of the same prefill (dq, dk, dv, d state_in)
     bwd = run_backward_leg(w, dev, stream, inp, dcode, args, world) if args.backward_steps > 0 else None
 
@@ -369,6 +372,7 @@ def run_ours(args):
         "e2e": e2e,
         "snapshots": snaps,
         "norm_gate": ng,
+        "gqa_decode": gqa,
         "backward": bwd,
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
@@ -488,6 +492,55 @@ def run_norm_gate_leg(w, dev, stream, o, dcode, args, world):
             "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s")}
 
 
+GQA_BATCH, GQA_HEADS, GQA_KV_HEADS, GQA_CAP = 8, 64, 8, 131072
+
+
+def run_gqa_leg(dev, stream, args, world):
+    """lightning_gqa_decode: 8 sequences at the last position of a 131072-token
+    bf16 cache, 64 query heads over 8 KV heads, RoPE on 64 dims; timed like the
+    main leg. The step reads each sequence's whole cache once."""
+    import torch
+    import linear_attention_lightning_b200 as la
+    from linear_attention_lightning_b200 import abi
+    b, h, hk, cap, d = GQA_BATCH, GQA_HEADS, GQA_KV_HEADS, GQA_CAP, 128
+    g = torch.Generator(device=dev).manual_seed(3000)
+    mk = lambda *shape: torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+    q, kn, vn = mk(b, h, d), mk(b, hk, d), mk(b, hk, d)
+    kc, vc = mk(b, hk, cap, d), mk(b, hk, cap, d)
+    pos = torch.full((b,), cap - 1, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    need = abi.lightning_gqa_decode_workspace_size(b, h, cap)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    sp = stream.cuda_stream
+
+    def step():
+        abi.check(abi.lightning_gqa_decode(q.data_ptr(), kn.data_ptr(), vn.data_ptr(), kc.data_ptr(), vc.data_ptr(),
+                                           abi.LA_DTYPE_BF16, pos.data_ptr(), b, h, hk, d, cap, 64, 1e4,
+                                           1.0 / d ** 0.5, o.data_ptr(), ws.data_ptr(), need, sp))
+
+    for _ in range(args.warmup):
+        step()
+    steps = args.gqa_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    # algorithmic bytes: the cache read for positions 0..cap-1 (K and V), the new k, v
+    # written, q read and o written
+    by = 2 * b * hk * cap * d * 2 + 2 * b * hk * d * 2 + 2 * b * h * d * 2
+    gbs = by / (ms / 1e3) / 1e9
+    return {"config": {"batch": b, "heads": h, "kv_heads": hk, "context": cap, "dim": d, "rot": 64,
+                       "dtype": "bf16"},
+            "steps": steps, "us_per_step": round(ms * 1e3, 2), "launches_per_step": 3,
+            "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s"),
+            "l2": "cache %.1f GB per step > L2" % (by / 1e9)}
+
+
 def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     """lightning_prefill_backward on the workload (AUTO: the CTA-pair tensor-core
     kernel where it applies), timed like the main leg: dQ causal on (dO, V, K),
@@ -594,6 +647,8 @@ def parse_args(argv=None):
     p.add_argument("--decode-steps", type=int, default=1000)
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--gqa-steps", type=int, default=20,
+                   help="timed steps of the softmax GQA decode leg (0 skips it)")
     p.add_argument("--norm-gate-steps", type=int, default=20,
                    help="timed steps of the norm-and-gate epilogue leg (0 skips it)")
     p.add_argument("--backward-steps", type=int, default=10,

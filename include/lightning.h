@@ -36,7 +36,9 @@
  *     is launched; launch failures return LA_ERR_CUDA. No device-side trap
  *     or abort is ever used: a device-side wait that runs out of its
  *     iteration budget records LA_ERR_TIMEOUT in a device status word, read
- *     back by lightning_device_status().
+ *     back by lightning_device_status(); so does LA_ERR_INVALID_ARG for a
+ *     device-side argument the host cannot see (a decode position outside
+ *     its cache), whose work is then skipped.
  *   - A human-readable reason for the last failure on the calling thread is
  *     returned by lightning_last_error_message().
  */
@@ -257,6 +259,41 @@ la_status lightning_decode(const void *q, const void *k, const void *v, la_dtype
 /* Synchronises `stream`, returns the device status word (LA_OK or
  * LA_ERR_TIMEOUT) recorded by kernels since the last call, and clears it. */
 la_status lightning_device_status(void *stream);
+
+/*
+ * One decode step of the softmax attention layer that M1 places after every
+ * seven Lightning layers. Source: "MINIMAX SIGNAL LAB · M1", §02 (64 query
+ * heads x 128; softmax K/V 8 x 128; RoPE on 64 of the 128 dims, in the
+ * softmax layers only) and §04 (those layers keep a KV cache that grows with
+ * the context). The pages print no formula; the readings: grouped-query
+ * attention (query head h reads KV head h / (heads / kv_heads)), scores
+ * scaled by `scale` (1/sqrt(dim) in the model), rotate-half RoPE on the first
+ * `rot` dims with theta_i = rope_base^{-2i/rot}, a cache of rotated keys.
+ * For sequence b the new token sits at position pos[b]: its rotated key and
+ * its value are written into the caches there, and
+ *   o[b][h] = sum_{p <= pos[b]} softmax_p(scale * rope(q[b][h], pos[b]) . k_p) v_p.
+ *
+ *   q                [batch][heads][dim], dtype.
+ *   k_new, v_new     [batch][kv_heads][dim], dtype.
+ *   k_cache, v_cache [batch][kv_heads][cap][dim], dtype; positions < pos[b]
+ *                    read, position pos[b] written.
+ *   pos              DEVICE int32 [batch], 0 <= pos[b] < cap; an out-of-range
+ *                    position skips that sequence (o = 0) and is reported as
+ *                    LA_ERR_INVALID_ARG by lightning_device_status().
+ *   dim 128; heads / kv_heads at most 8; rot even, 0 <= rot <= dim.
+ *   o                [batch][heads][dim], dtype; written.
+ *   workspace        lightning_gqa_decode_workspace_size(batch, heads, cap)
+ *                    bytes, 16-byte aligned.
+ * Device pointers, caller-owned, 16-byte aligned; the caches, o and the
+ * workspace must not overlap any other buffer. CUDA cores, fp32 arithmetic.
+ */
+la_status lightning_gqa_decode(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                               la_dtype dtype, const int *pos, int batch, int heads, int kv_heads, int dim, int cap,
+                               int rot, double rope_base, float scale, void *o, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
+/* Workspace bytes of lightning_gqa_decode (0 for an invalid request). Host only. */
+size_t lightning_gqa_decode_workspace_size(int batch, int heads, int cap);
 
 /* Static description of a status code. */
 const char *lightning_status_string(int status);

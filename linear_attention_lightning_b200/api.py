@@ -162,6 +162,39 @@ def norm_gate(o: torch.Tensor, gate: torch.Tensor, gamma: torch.Tensor, eps: flo
     return y
 
 
+def gqa_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
+               v_cache: torch.Tensor, pos: torch.Tensor, rot: int = 64, rope_base: float = 10000.0,
+               scale: Optional[float] = None, o: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """lightning_gqa_decode: one decode step of the softmax GQA layer. Writes the
+    new rotated key and value into the caches at pos[b] and returns o
+    [batch, heads, dim]. scale defaults to 1/sqrt(dim)."""
+    if q.dtype not in _DTYPES:
+        raise ValueError("q must be float32 or bfloat16")
+    b, h, d = q.shape
+    bk, hk, cap, dk = k_cache.shape
+    if (bk, dk) != (b, d) or tuple(k_new.shape) != (b, hk, d) or tuple(v_new.shape) != (b, hk, d) \
+            or v_cache.shape != k_cache.shape:
+        raise ValueError("inconsistent shapes: q [b, heads, dim], k/v_new [b, kv_heads, dim], caches [b, kv_heads, cap, dim]")
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need_cuda(name, t, q.dtype)
+    _need_cuda("pos", pos, torch.int32)
+    if tuple(pos.shape) != (b,):
+        raise ValueError("pos must be [batch]")
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if o is None:
+        o = torch.empty_like(q)
+    need = abi.lightning_gqa_decode_workspace_size(b, h, cap)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    abi.check(abi.lightning_gqa_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                       _DTYPES[q.dtype], _ptr(pos), b, h, hk, d, cap, int(rot), float(rope_base),
+                                       float(scale), _ptr(o), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
 def prefill_variant(dtype: torch.dtype, batch: int, heads: int, seq: int, dim: int, block: int,
                     variant: str = "auto") -> str:
     """Which kernel lightning_prefill would run: "simt", "tcgen05" or "pair"."""

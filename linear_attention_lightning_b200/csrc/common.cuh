@@ -10,6 +10,9 @@ namespace la {
 // Device status word: kernels set LA_ERR_TIMEOUT here when a bounded wait
 // gives up. Read and cleared by lightning_device_status().
 __device__ unsigned int g_device_status;
+// flag in the status word: a kernel met an out-of-range device-side argument
+// (a decode position outside the cache) and skipped the work it governs
+constexpr unsigned int kBadDeviceArgFlag = 1u;
 
 constexpr float kLog2e = 1.4426950408889634f;
 

@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill_simt.cuh"
+#include "gqa_decode.cuh"
 #include "norm_gate.cuh"
 #include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
@@ -219,6 +220,75 @@ la_status launch_norm_gate(const NgArgs &a) {
                                                               a.per_head, (int)tile, static_cast<T *>(a.y));
     e = cudaGetLastError();
     return e == cudaSuccess ? ok() : cuda_fail(e, "norm_gate launch");
+}
+
+// Workspace of one GQA decode step: per (sequence, query head, chunk) the
+// running max, the sum and the weighted values of the chunk's softmax.
+struct GqaLayout {
+    int splits;
+    size_t m_off, l_off, o_off, q_off, bytes;
+};
+
+GqaLayout gqa_layout(int batch, int heads, int cap) {
+    GqaLayout g;
+    g.splits = (cap + la::kGqaChunk - 1) / la::kGqaChunk;
+    const size_t n = (size_t)batch * heads * g.splits;
+    auto up16 = [](size_t x) { return (x + 15) / 16 * 16; };
+    g.m_off = 0;
+    g.l_off = up16(n * 4);
+    g.o_off = g.l_off + up16(n * 4);
+    g.q_off = g.o_off + n * la::kGqaDim * 4;                           // rotated queries
+    g.bytes = g.q_off + (size_t)batch * heads * la::kGqaDim * 4;
+    return g;
+}
+
+template <typename T>
+la_status run_gqa_decode(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                         const int *pos, int batch, int heads, int kv_heads, int cap, int rot, double base,
+                         float scale, void *o, void *workspace, cudaStream_t stream) {
+    const GqaLayout g = gqa_layout(batch, heads, cap);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *pm = reinterpret_cast<float *>(ws + g.m_off), *pl = reinterpret_cast<float *>(ws + g.l_off);
+    float *po = reinterpret_cast<float *>(ws + g.o_off), *qr = reinterpret_cast<float *>(ws + g.q_off);
+    la::gqa_append_kernel<T><<<dim3(batch, kv_heads), la::kGqaDim, 0, stream>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k_new), static_cast<const T *>(v_new),
+        static_cast<T *>(k_cache), static_cast<T *>(v_cache), pos, heads, kv_heads, cap, rot, base, scale, qr);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "gqa append launch");
+    // the caches as 2-D tensors [batch*kv_heads*cap][dim], 128-byte swizzled boxes of one tile of positions
+    const bool bf16 = sizeof(T) == 2;
+    const cuuint64_t rows = (cuuint64_t)batch * kv_heads * cap;
+    CUtensorMap mk, mv;
+    {
+        auto fn = la::tc::encode_fn(&g_last_error);
+        if (!fn) return LA_ERR_CUDA;
+        const cuuint64_t dims[2] = {(cuuint64_t)la::kGqaDim, rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)la::kGqaDim * sizeof(T)};
+        const cuuint32_t box[2] = {la::kGqaBoxRowBytes / (cuuint32_t)sizeof(T),
+                                   (cuuint32_t)(la::kGqaTileBytes / (la::kGqaDim * sizeof(T)))};
+        const cuuint32_t estr[2] = {1, 1};
+        for (int i = 0; i < 2; ++i) {
+            CUresult r = fn(i == 0 ? &mk : &mv, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                            2, i == 0 ? k_cache : v_cache, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) {
+                g_last_error = "cuTensorMapEncodeTiled failed for a cache (CUresult " + std::to_string((int)r) + ")";
+                return LA_ERR_CUDA;
+            }
+        }
+    }
+    e = cudaFuncSetAttribute(la::gqa_partial_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)la::kGqaSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gqa_partial)");
+    la::gqa_partial_kernel<T><<<dim3(g.splits, kv_heads, batch), la::kGqaThreads, la::kGqaSmemBytes, stream>>>(
+        mk, mv, qr, pos, heads, kv_heads, cap, g.splits, pm, pl, po);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "gqa partial launch");
+    la::gqa_combine_kernel<T><<<(unsigned)((size_t)batch * heads), la::kGqaDim, 0, stream>>>(pm, pl, po, g.splits,
+                                                                                         static_cast<T *>(o));
+    e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "gqa combine launch");
 }
 
 // One launch of the CUDA-core kernel as a pass of the backward computation.
@@ -551,6 +621,58 @@ la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, c
 }
 
 
+size_t lightning_gqa_decode_workspace_size(int batch, int heads, int cap) {
+    if (batch < 0 || heads < 1 || cap < 1) return 0;
+    return gqa_layout(batch, heads, cap).bytes;
+}
+
+la_status lightning_gqa_decode(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+                               la_dtype dtype, const int *pos, int batch, int heads, int kv_heads, int dim, int cap,
+                               int rot, double rope_base, float scale, void *o, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+    if (dtype != LA_DTYPE_F32 && dtype != LA_DTYPE_BF16)
+        return fail(LA_ERR_INVALID_ARG, "dtype %d is neither LA_DTYPE_F32 nor LA_DTYPE_BF16", (int)dtype);
+    if (batch < 0 || heads < 1 || kv_heads < 1 || cap < 1 || heads % kv_heads != 0)
+        return fail(LA_ERR_INVALID_ARG, "need batch >= 0, cap >= 1 and kv_heads dividing heads (got %d, %d, %d, %d)",
+                    batch, cap, heads, kv_heads);
+    if (dim != la::kGqaDim) return fail(LA_ERR_UNSUPPORTED, "dim %d unsupported (128)", dim);
+    if (heads / kv_heads > la::kGqaMaxGroup)
+        return fail(LA_ERR_UNSUPPORTED, "at most %d query heads per KV head (got %d)", la::kGqaMaxGroup,
+                    heads / kv_heads);
+    if (rot < 0 || rot > dim || (rot & 1)) return fail(LA_ERR_INVALID_ARG, "rot must be even, 0 <= rot <= dim");
+    if (!(rope_base > 0.0) || rope_base > 1e300) return fail(LA_ERR_INVALID_ARG, "rope_base must be finite and > 0");
+    if (!(scale == scale) || scale > 3e38f || scale < -3e38f) return fail(LA_ERR_INVALID_ARG, "scale must be finite");
+    if (batch == 0) return ok();
+    const GqaLayout g = gqa_layout(batch, heads, cap);
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !pos || !o)
+        return fail(LA_ERR_INVALID_ARG, "q, k_new, v_new, the caches, pos and o must be non-NULL");
+    if (!workspace || workspace_bytes < g.bytes)
+        return fail(LA_ERR_INVALID_ARG, "workspace needs %zu bytes (got %zu)", g.bytes,
+                    workspace ? workspace_bytes : (size_t)0);
+    const void *ptrs[] = {q, k_new, v_new, k_cache, v_cache, pos, o, workspace};
+    const char *names[] = {"q", "k_new", "v_new", "k_cache", "v_cache", "pos", "o", "workspace"};
+    for (int i = 0; i < 8; ++i)
+        if (!aligned16(ptrs[i])) return fail(LA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+    const size_t eb = elem_bytes(dtype);
+    const size_t nq = (size_t)batch * heads * dim * eb, nkv = (size_t)batch * kv_heads * dim * eb;
+    const size_t ncache = (size_t)batch * kv_heads * cap * dim * eb;
+    const Range rq = range_of(q, nq), rkn = range_of(k_new, nkv), rvn = range_of(v_new, nkv);
+    const Range rkc = range_of(k_cache, ncache), rvc = range_of(v_cache, ncache), rp = range_of(pos, 4 * batch);
+    const Range ro = range_of(o, nq), rw = range_of(workspace, g.bytes);
+    const Range all[] = {rq, rkn, rvn, rkc, rvc, rp, ro, rw};
+    const int written[] = {3, 4, 6, 7};  // the caches, o and the workspace
+    for (int wi : written)
+        for (int j = 0; j < 8; ++j)
+            if (j != wi && overlaps(all[wi], all[j]))
+                return fail(LA_ERR_INVALID_ARG, "%s overlaps %s", names[wi], names[j]);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dtype == LA_DTYPE_BF16)
+        return run_gqa_decode<__nv_bfloat16>(q, k_new, v_new, k_cache, v_cache, pos, batch, heads, kv_heads, cap, rot,
+                                             rope_base, scale, o, workspace, st);
+    return run_gqa_decode<float>(q, k_new, v_new, k_cache, v_cache, pos, batch, heads, kv_heads, cap, rot, rope_base,
+                                 scale, o, workspace, st);
+}
+
 int lightning_prefill_snapshot_count(int seq, int interval) {
     if (seq < 0 || interval < 1) return -1;
     return seq / interval;
@@ -626,7 +748,9 @@ la_status lightning_device_status(void *stream) {
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
     e = cudaMemcpyToSymbol(la::g_device_status, &zero, sizeof zero);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
-    if (word != 0) return fail(LA_ERR_TIMEOUT, "a device-side wait gave up (status word 0x%x)", word);
+    if (word & LA_ERR_TIMEOUT) return fail(LA_ERR_TIMEOUT, "a device-side wait gave up (status word 0x%x)", word);
+    if (word & la::kBadDeviceArgFlag)
+        return fail(LA_ERR_INVALID_ARG, "a kernel met an out-of-range device-side argument (status word 0x%x)", word);
     return ok();
 }
 

@@ -242,3 +242,42 @@ def test_norm_gate_argument_errors(kw, status):
 def test_norm_gate_empty_needs_no_gpu():
     assert _norm_gate(batch=0) == abi.LA_OK
     assert _norm_gate(seq=0, o=None, y=None) == abi.LA_OK
+
+
+def _gqa(**kw):
+    a = dict(q=Q, kn=K, vn=V, kc=0x10000000 * 30, vc=0x10000000 * 40, dtype=abi.LA_DTYPE_BF16, pos=SL, batch=2,
+             heads=64, kv=8, dim=128, cap=1024, rot=64, base=1e4, scale=0.088, o=O, ws=WS, ws_bytes=1 << 26)
+    a.update(kw)
+    return abi.lightning_gqa_decode(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["dtype"], a["pos"], a["batch"],
+                                    a["heads"], a["kv"], a["dim"], a["cap"], a["rot"], a["base"], a["scale"], a["o"],
+                                    a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype=9), abi.LA_ERR_INVALID_ARG),
+    (dict(kv=7), abi.LA_ERR_INVALID_ARG),               # does not divide 64
+    (dict(cap=0), abi.LA_ERR_INVALID_ARG),
+    (dict(dim=64), abi.LA_ERR_UNSUPPORTED),
+    (dict(kv=4), abi.LA_ERR_UNSUPPORTED),               # 16 query heads per KV head
+    (dict(rot=63), abi.LA_ERR_INVALID_ARG),
+    (dict(rot=130), abi.LA_ERR_INVALID_ARG),
+    (dict(base=0.0), abi.LA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), abi.LA_ERR_INVALID_ARG),
+    (dict(pos=None), abi.LA_ERR_INVALID_ARG),
+    (dict(ws_bytes=64), abi.LA_ERR_INVALID_ARG),        # workspace too small
+    (dict(o=Q), abi.LA_ERR_INVALID_ARG),                # o is q
+    (dict(kc=0x10000000 * 40), abi.LA_ERR_INVALID_ARG), # k_cache is v_cache
+    (dict(vc=0x10000000 * 40 + 8), abi.LA_ERR_INVALID_ARG),
+])
+def test_gqa_decode_argument_errors(kw, status):
+    assert _gqa(**kw) == status
+    assert abi.last_error_message() != ""
+
+
+def test_gqa_workspace_size_and_empty_batch():
+    # per (sequence, query head, 2048-position chunk): max, sum, 128 weighted values;
+    # per (sequence, query head): the rotated, scaled query
+    n = 2 * 64 * 1
+    assert abi.lightning_gqa_decode_workspace_size(2, 64, 1024) == n * 4 + n * 4 + n * 128 * 4 + 2 * 64 * 128 * 4
+    assert abi.lightning_gqa_decode_workspace_size(0, 64, 1024) == 0
+    assert _gqa(batch=0) == abi.LA_OK
