@@ -77,31 +77,49 @@ def roofline(bound, achieved, peak, unit, traffic=None):
             "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic}
 
 
-def kernel_source_digest():
-    """Digest of the CUDA sources, to tell whether stored ncu counters still
-    describe the kernels being timed."""
+KERNEL_SOURCES = {  # traffic.json key suffix -> the header that holds the kernel
+    "pair": "prefill_pair.cuh", "tcgen05": "prefill_tc.cuh", "simt": "prefill_simt.cuh",
+    "backward_pair": "prefill_pair.cuh", "decode": "decode.cuh", "norm_gate": "norm_gate.cuh",
+    "gqa_partial": "gqa_decode.cuh",
+}
+
+
+def kernel_source_digest(header):
+    """Digest of one kernel's header and every local header it includes, to
+    tell whether stored ncu counters still describe the kernel being timed."""
     import hashlib
-    h = hashlib.sha256()
+    import re
     csrc = os.path.join(ROOT, "linear_attention_lightning_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+    seen, todo = [], [os.path.normpath(os.path.join(csrc, header))]
+    while todo:
+        path = todo.pop()
+        if path in seen:
+            continue
+        seen.append(path)
+        with open(path, "rb") as f:
+            text = f.read()
+        for inc in re.findall(rb'#include "([^"]+)"', text):
+            todo.append(os.path.normpath(os.path.join(os.path.dirname(path), inc.decode())))
+    h = hashlib.sha256()
+    for path in sorted(seen):
+        with open(path, "rb") as f:
+            h.update(os.path.relpath(path, ROOT).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload, variant):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernels changed since it was captured."""
+def measured_traffic(workload, kernel, field="dram_bytes_per_launch"):
+    """DRAM bytes from the committed ncu summary, or None when the kernel's
+    sources changed since it was captured."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
-    if t.get("kernel_source_digest") != kernel_source_digest():
+    entry = t.get("launches", {}).get("%s/%s" % (workload, kernel))
+    if entry is None or entry.get("kernel_source_digest") != kernel_source_digest(KERNEL_SOURCES[kernel]):
         return None
-    entry = t.get("launches", {}).get("%s/%s" % (workload, variant))
-    return None if entry is None else entry.get("dram_bytes_per_launch")
+    return entry.get(field)
 
 
 def summarize_clocks(rows):
@@ -390,7 +408,7 @@ def run_decode(dw, dev, stream, peaks, args):
     import torch
     from linear_attention_lightning_b200 import abi, inputs
     steps = args.decode_steps
-    inp = inputs.workload_inputs(dw, dev, steps=steps)
+    inp = inputs.workload_inputs(dw, dev, steps=max(steps, 3))  # 3 warm-up tokens at least
     state = inp["state"]
     qs, ks, vs, sl = inp["q"], inp["k"], inp["v"], inp["slopes"]
     o = torch.empty((dw.batch, dw.heads, dw.dim), dtype=dw.dtype, device=dev)
@@ -418,7 +436,7 @@ def run_decode(dw, dev, stream, peaks, args):
     del tok
     return {"workload": dw.name, "steps": steps, "us_per_step": round(1e3 * ms / steps, 3),
             "value": round(gbs, 1), "unit": "GB/s (state + token bytes)",
-            "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s"),
+            "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s", measured_traffic(dw.name, "decode")),
             "l2": "state 268 MB > L2; consecutive steps, no flush"}
 
 
@@ -489,7 +507,7 @@ def run_norm_gate_leg(w, dev, stream, o, dcode, args, world):
     gbs = by / (ms / 1e3) / 1e9
     return {"steps": steps, "ms_per_step": round(ms, 4), "per": "token (heads*dim channels)",
             "tokens_per_s": round(world * w.batch * w.seq / (ms / 1e3), 1),
-            "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s")}
+            "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s", measured_traffic(w.name, "norm_gate"))}
 
 
 GQA_BATCH, GQA_HEADS, GQA_KV_HEADS, GQA_CAP = 8, 64, 8, 131072
@@ -502,7 +520,7 @@ def run_gqa_leg(dev, stream, args, world):
     import torch
     import linear_attention_lightning_b200 as la
     from linear_attention_lightning_b200 import abi
-    b, h, hk, cap, d = GQA_BATCH, GQA_HEADS, GQA_KV_HEADS, GQA_CAP, 128
+    b, h, hk, cap, d = GQA_BATCH, GQA_HEADS, GQA_KV_HEADS, args.gqa_context, 128
     g = torch.Generator(device=dev).manual_seed(3000)
     mk = lambda *shape: torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
     q, kn, vn = mk(b, h, d), mk(b, hk, d), mk(b, hk, d)
@@ -537,7 +555,8 @@ def run_gqa_leg(dev, stream, args, world):
     return {"config": {"batch": b, "heads": h, "kv_heads": hk, "context": cap, "dim": d, "rot": 64,
                        "dtype": "bf16"},
             "steps": steps, "us_per_step": round(ms * 1e3, 2), "launches_per_step": 3,
-            "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s"),
+            "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s",
+                                 measured_traffic("gqa_%d" % cap, "gqa_partial")),
             "l2": "cache %.1f GB per step > L2" % (by / 1e9)}
 
 
@@ -594,7 +613,8 @@ def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     return {"kernel": kernel, "steps": steps, "ms_per_step": round(ms, 3),
             "tokens_per_s": round(world * w.batch * w.seq / (ms / 1e3), 1),
             "workspace_bytes": need,
-            "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s"),
+            "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s",
+                                 measured_traffic(w.name, "backward_pair", "dram_bytes_per_step")),
             "tflops_formula": round(tf, 2),
             "frac_bf16_peak_formula": round(tf / peaks["bf16_tflops"], 4)}
 
@@ -649,6 +669,8 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--gqa-steps", type=int, default=20,
                    help="timed steps of the softmax GQA decode leg (0 skips it)")
+    p.add_argument("--gqa-context", type=int, default=GQA_CAP,
+                   help="cached tokens per sequence in the GQA decode leg")
     p.add_argument("--norm-gate-steps", type=int, default=20,
                    help="timed steps of the norm-and-gate epilogue leg (0 skips it)")
     p.add_argument("--backward-steps", type=int, default=10,
@@ -658,6 +680,8 @@ def parse_args(argv=None):
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be at least 3")
+    if a.gqa_context < 1:
+        p.error("--gqa-context must be positive")
     return a
 
 

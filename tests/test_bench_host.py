@@ -58,21 +58,43 @@ def test_warmup_floor():
 
 
 def test_stored_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
-    digest = bench.kernel_source_digest()
+    import shutil
+    shutil.copytree(os.path.join(bench.ROOT, "linear_attention_lightning_b200", "csrc"),
+                    tmp_path / "linear_attention_lightning_b200" / "csrc")
+    shutil.copytree(os.path.join(bench.ROOT, "include"), tmp_path / "include")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "traffic.json").write_text(json.dumps({
-        "kernel_source_digest": digest,
-        "launches": {"w/tcgen05": {"dram_bytes_per_launch": 123}}}))
-    csrc = os.path.join(bench.ROOT, "linear_attention_lightning_b200", "csrc")
-    pkg = tmp_path / "linear_attention_lightning_b200"
-    pkg.mkdir()
-    os.symlink(csrc, pkg / "csrc")
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench.measured_traffic("w", "tcgen05") == 123
-    (prof / "traffic.json").write_text(json.dumps({
-        "kernel_source_digest": "stale", "launches": {"w/tcgen05": {"dram_bytes_per_launch": 123}}}))
-    assert bench.measured_traffic("w", "tcgen05") is None
+
+    def store():
+        (prof / "traffic.json").write_text(json.dumps({"launches": {
+            "w/pair": {"kernel_source_digest": bench.kernel_source_digest("prefill_pair.cuh"),
+                       "dram_bytes_per_launch": 123},
+            "w/norm_gate": {"kernel_source_digest": bench.kernel_source_digest("norm_gate.cuh"),
+                            "dram_bytes_per_launch": 456}}}))
+
+    store()
+    assert bench.measured_traffic("w", "pair") == 123
+    assert bench.measured_traffic("w", "norm_gate") == 456
+    assert bench.measured_traffic("w", "decode") is None  # never captured
+    csrc = tmp_path / "linear_attention_lightning_b200" / "csrc"
+    # a change to one kernel voids its own counters only
+    with open(csrc / "norm_gate.cuh", "a") as f:
+        f.write("// edit\n")
+    assert bench.measured_traffic("w", "norm_gate") is None
+    assert bench.measured_traffic("w", "pair") == 123
+    # a change to a shared header voids every kernel that includes it
+    store()
+    with open(csrc / "common.cuh", "a") as f:
+        f.write("// edit\n")
+    assert bench.measured_traffic("w", "pair") is None
+    assert bench.measured_traffic("w", "norm_gate") is None
+    # the public header is part of the pair kernel's sources
+    store()
+    with open(tmp_path / "include" / "lightning.h", "a") as f:
+        f.write("// edit\n")
+    assert bench.measured_traffic("w", "pair") is None
+    assert bench.measured_traffic("w", "norm_gate") == 456
 
 
 def _rank_main(rank, port, q):
