@@ -7,8 +7,8 @@ shares no code with it.
 The arithmetic lives in ``lightning_oracle.c`` (three forms of the same
 result: F1 definition, F2 token recurrence, F3 blockwise, plus one decode
 step, the state snapshots of a prefix cache, the gradients of one prefill,
-the normalisation and gating of the output and one decode step of the
-softmax GQA layer; see that file's header for
+the normalisation and gating of the output, and one decode step and one
+prefill of the softmax GQA layer; see that file's header for
 the formulas and their sources on the "MINIMAX SIGNAL LAB · M1" page, §03
 Lightning Attention). This module only
 marshals numpy arrays into it.
@@ -49,6 +49,9 @@ def _load():
         lib.la_oracle_gqa_decode.argtypes = [vp, vp, vp, vp, vp, ip, vp, ip, ip, ip, ip, ip, ip, ctypes.c_double,
                                              ctypes.c_double, dp]
         lib.la_oracle_gqa_decode.restype = ctypes.c_int
+        lib.la_oracle_gqa_prefill.argtypes = [vp, vp, vp, vp, vp, ip, ip, ip, ip, ip, ip, ip, ip, ip,
+                                              ctypes.c_double, ctypes.c_double, vp, ctypes.c_longlong, dp]
+        lib.la_oracle_gqa_prefill.restype = ctypes.c_int
         lib.la_oracle_max_threads.restype = ctypes.c_int
         lib.la_oracle_set_threads.argtypes = [ip]
         _lib = lib
@@ -206,6 +209,39 @@ def gqa_decode(q, k_new, v_new, k_cache, v_cache, pos, rot, base, scale):
                                       _ptr(pos), b, h, hk, d, cap, int(rot), float(base), float(scale), _ptr(o))
     if rc != 0:
         raise RuntimeError("oracle gqa_decode failed (rc=%d)" % rc)
+    return o
+
+
+def gqa_prefill(q, k_new, v_new, k_cache, v_cache, start, rot, base, scale, rows=None):
+    """The softmax GQA layer over `seq` new tokens at positions start ..
+    start+seq-1 (RoPE on the first `rot` dims, causal).
+
+    q: [batch, heads, seq, dim]; k_new, v_new: [batch, kv_heads, seq, dim];
+    caches: [batch, kv_heads, cap, dim] (rotated keys; positions < start
+    filled). rows: None for every output (returns o float64 [batch, heads,
+    seq, dim]) or indices (b*heads + h)*seq + i (returns [len(rows), dim])."""
+    q, k_new, v_new, k_cache, v_cache = (np.ascontiguousarray(x) for x in (q, k_new, v_new, k_cache, v_cache))
+    code = _dtype_code(q)
+    for x in (k_new, v_new, k_cache, v_cache):
+        if _dtype_code(x) != code:
+            raise TypeError("all gqa inputs must share a dtype")
+    b, h, L, d = q.shape
+    bk, hk, cap, dk = k_cache.shape
+    if (bk, dk) != (b, d) or k_new.shape != (b, hk, L, d) or v_new.shape != k_new.shape or \
+            v_cache.shape != k_cache.shape:
+        raise ValueError("inconsistent gqa shapes")
+    if rows is None:
+        o = np.empty((b, h, L, d), dtype=np.float64)
+        rp, n = None, 0
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1)
+        o = np.empty((rows.size, d), dtype=np.float64)
+        rp, n = _ptr(rows), rows.size
+    rc = _load().la_oracle_gqa_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), code,
+                                       int(start), b, h, hk, L, d, cap, int(rot), float(base), float(scale), rp, n,
+                                       _ptr(o))
+    if rc != 0:
+        raise RuntimeError("oracle gqa_prefill failed (rc=%d)" % rc)
     return o
 
 

@@ -36,13 +36,15 @@
  * plus la_oracle_decode, one recurrent step for a single new token,
  * la_oracle_snapshots, the state after every `interval` tokens (F2's state),
  * la_oracle_backward, the gradients of one prefill, la_oracle_norm_gate, the
- * normalisation and gating of the attention output, and la_oracle_gqa_decode,
- * one decode step of the softmax attention layer of the hybrid model.
+ * normalisation and gating of the attention output, la_oracle_gqa_decode,
+ * one decode step of the softmax attention layer of the hybrid model, and
+ * la_oracle_gqa_prefill, the same layer over a run of new tokens.
  *
  * Layouts: q, k, v, o are [batch][heads][seq][dim] contiguous (o for decode
  * is [batch][heads][dim]); states are [batch][heads][dim(k)][dim(v)].
- * Parallelism: OpenMP over (batch, head) only; the arithmetic inside one
- * head is a plain sequential loop.
+ * Parallelism: OpenMP over (batch, head) only (over output rows for the
+ * softmax layer's prefill); the arithmetic inside one head or row is a plain
+ * sequential loop.
  */
 #include <math.h>
 #include <stdint.h>
@@ -529,4 +531,103 @@ int la_oracle_decode(const void *q, const void *k, const void *v, int dtype, con
         }
     }
     return 0;
+}
+
+/* The softmax GQA layer over a run of `seq` new tokens per sequence, at
+ * positions start .. start+seq-1 (§02 and §04 of "MINIMAX SIGNAL LAB · M1" as
+ * for la_oracle_gqa_decode, whose readings this follows: query head h reads
+ * KV head h / (heads / kv_heads), rotate-half RoPE on the first `rot` dims at
+ * the token's position, scores scaled by `scale`, causal order). Token i of
+ * sequence b, query head h, sits at position P = start + i and attends to
+ * every position p <= P:
+ *   o = sum_{p <= P} softmax_p(scale * rope(q_i, P) . key_p) val_p,
+ *   key_p = k_cache[p] (already rotated), val_p = v_cache[p]          for p < start,
+ *   key_p = rope(k_new[p - start], p), val_p = v_new[p - start]        for p >= start.
+ * q: [batch][heads][seq][dim]; k_new, v_new: [batch][kv_heads][seq][dim];
+ * caches: [batch][kv_heads][cap][dim] with positions < start filled. All
+ * inputs share `dtype`. rows: the outputs to compute, as indices
+ * (b * heads + h) * seq + i, or NULL for all batch*heads*seq of them in that
+ * order; o: float64 [nrows][dim]. The angles are those of rope_head. */
+int la_oracle_gqa_prefill(const void *q, const void *k_new, const void *v_new, const void *k_cache,
+                          const void *v_cache, int dtype, int start, int batch, int heads, int kv_heads, int seq,
+                          int dim, int cap, int rot, double base, double scale, const long long *rows,
+                          long long nrows, double *o) {
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !o) return 1;
+    if (dtype != ORACLE_F32 && dtype != ORACLE_BF16) return 1;
+    if (batch < 0 || seq < 0 || start < 0 || kv_heads <= 0 || heads % kv_heads != 0 || dim <= 0 || rot < 0 ||
+        rot > dim || rot % 2 || (long long)start + seq > cap)
+        return 1;
+    const long long total = (long long)batch * heads * seq;
+    if (!rows) nrows = total;
+    if (nrows < 0) return 1;
+    for (long long n = 0; rows && n < nrows; ++n)
+        if (rows[n] < 0 || rows[n] >= total) return 1;
+    const int group = heads / kv_heads, half = rot / 2;
+    const size_t d = (size_t)dim;
+    /* cos and sin of every new position's angles, as rope_head takes them */
+    double *cs = malloc(sizeof(double) * ((size_t)seq * half + 1)), *sn = malloc(sizeof(double) * ((size_t)seq * half + 1));
+    if (!cs || !sn) {
+        free(cs); free(sn);
+        return 1;
+    }
+    for (int i = 0; i < seq; ++i)
+        for (int c = 0; c < half; ++c) {
+            const double ang = (double)(start + i) * pow(base, -2.0 * c / (double)rot);
+            cs[(size_t)i * half + c] = cos(ang);
+            sn[(size_t)i * half + c] = sin(ang);
+        }
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long n = 0; n < nrows; ++n) {
+        const long long r = rows ? rows[n] : n;
+        const int i = (int)(r % seq), h = (int)((r / seq) % heads), b = (int)(r / ((long long)seq * heads));
+        const size_t kv = (size_t)b * kv_heads + h / group;
+        const long P = (long)start + i;
+        double *x = malloc(sizeof(double) * d * 4), *sc = malloc(sizeof(double) * (size_t)(P + 1));
+        if (!x || !sc) {
+            fail = 1;
+            free(x); free(sc);
+            continue;
+        }
+        double *qr = x, *kr = x + d, *tmp = x + 2 * d, *acc = x + 3 * d;
+        /* rotate a head row given at tmp by the angles of new token t into out */
+#define ROPE_NEW(out, t)                                                                  \
+        do {                                                                              \
+            for (size_t c_ = 0; c_ < d; ++c_) (out)[c_] = tmp[c_];                        \
+            for (int c_ = 0; c_ < half; ++c_) {                                           \
+                const double cv = cs[(size_t)(t) * half + c_], sv = sn[(size_t)(t) * half + c_]; \
+                (out)[c_] = tmp[c_] * cv - tmp[c_ + half] * sv;                           \
+                (out)[c_ + half] = tmp[c_ + half] * cv + tmp[c_] * sv;                    \
+            }                                                                             \
+        } while (0)
+        for (size_t c = 0; c < d; ++c) tmp[c] = widen(q, dtype, (size_t)r * d + c);
+        ROPE_NEW(qr, i);
+        double mx = -INFINITY;
+        for (long p = 0; p <= P; ++p) {
+            if (p < start) {
+                for (size_t c = 0; c < d; ++c) kr[c] = widen(k_cache, dtype, (kv * cap + p) * d + c);
+            } else {
+                for (size_t c = 0; c < d; ++c) tmp[c] = widen(k_new, dtype, (kv * seq + (p - start)) * d + c);
+                ROPE_NEW(kr, p - start);
+            }
+            double dot = 0.0;
+            for (size_t c = 0; c < d; ++c) dot += qr[c] * kr[c];
+            sc[p] = scale * dot;
+            if (sc[p] > mx) mx = sc[p];
+        }
+#undef ROPE_NEW
+        double den = 0.0;
+        for (size_t c = 0; c < d; ++c) acc[c] = 0.0;
+        for (long p = 0; p <= P; ++p) {
+            const double w = exp(sc[p] - mx);
+            den += w;
+            for (size_t c = 0; c < d; ++c)
+                acc[c] += w * (p < start ? widen(v_cache, dtype, (kv * cap + p) * d + c)
+                                         : widen(v_new, dtype, (kv * seq + (p - start)) * d + c));
+        }
+        for (size_t c = 0; c < d; ++c) o[(size_t)n * d + c] = acc[c] / den;
+        free(x); free(sc);
+    }
+    free(cs); free(sn);
+    return fail;
 }

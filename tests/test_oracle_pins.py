@@ -415,3 +415,89 @@ def test_gqa_decode_rotates_query_and_new_key_alike():
             s = 0.2 * float(q[0, hh].astype(np.float64) @ kn[0, 0].astype(np.float64))
             want = (vc[0, 0, :P].astype(np.float64).sum(0) + np.exp(s) * vn[0, 0]) / (P + np.exp(s))
             np.testing.assert_allclose(o[0, hh], want, rtol=1e-12, atol=1e-12)
+
+
+def _gqa_prefill_case(b=2, h=4, hk=2, L=6, d=16, cap=20, seed=80):
+    rng = np.random.default_rng(seed)
+    f = lambda *s: rng.standard_normal(s).astype(np.float32)
+    return f(b, h, L, d), f(b, hk, L, d), f(b, hk, L, d), f(b, hk, cap, d), f(b, hk, cap, d)
+
+
+def test_gqa_prefill_matches_a_numpy_causal_softmax():
+    # brute force: every key and value of the sequence assembled explicitly, one masked
+    # score matrix per head, numpy softmax along keys
+    q, kn, vn, kc, vc = _gqa_prefill_case()
+    start, rot, base, scale = 5, 8, 100.0, 0.3
+    o = oracle.gqa_prefill(q, kn, vn, kc, vc, start, rot, base, scale)
+    b, h, L, d = q.shape
+    hk = kn.shape[1]
+    for bb in range(b):
+        for hh in range(h):
+            g = hh // (h // hk)
+            keys = np.concatenate([kc[bb, g, :start].astype(np.float64),
+                                   np.stack([oracle.rope(kn[bb, g, i], start + i, rot, base) for i in range(L)])])
+            vals = np.concatenate([vc[bb, g, :start], vn[bb, g]]).astype(np.float64)
+            qr = np.stack([oracle.rope(q[bb, hh, i], start + i, rot, base) for i in range(L)])
+            s = scale * qr @ keys.T                                   # [L, start + L]
+            s[np.arange(start + L)[None, :] > (start + np.arange(L))[:, None]] = -np.inf
+            w = np.exp(s - s.max(1, keepdims=True))
+            np.testing.assert_allclose(o[bb, hh], (w / w.sum(1, keepdims=True)) @ vals, rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_prefill_is_a_chain_of_decode_steps():
+    # token i of a prefill is the decode step at position start + i over a cache that holds
+    # the earlier new tokens (rotated keys) after the given prefix
+    q, kn, vn, kc, vc = _gqa_prefill_case(b=1, h=4, hk=1, L=5, d=16, cap=12, seed=81)
+    start, rot, base, scale = 3, 16, 500.0, 0.25
+    o = oracle.gqa_prefill(q, kn, vn, kc, vc, start, rot, base, scale)
+    kcc, vcc = kc.copy(), vc.copy()
+    for i in range(q.shape[2]):
+        od = oracle.gqa_decode(q[:, :, i], kn[:, :, i], vn[:, :, i], kcc, vcc, np.array([start + i], np.int32),
+                               rot, base, scale)
+        # the decode step reads the earlier keys back from a float32 cache
+        np.testing.assert_allclose(o[:, :, i], od, rtol=0, atol=2e-6)
+        kcc[0, 0, start + i] = oracle.rope(kn[0, 0, i], start + i, rot, base).astype(np.float32)
+        vcc[0, 0, start + i] = vn[0, 0, i]
+    # one token: exactly the decode step
+    o1 = oracle.gqa_prefill(q[:, :, :1], kn[:, :, :1], vn[:, :, :1], kc, vc, start, rot, base, scale)
+    od = oracle.gqa_decode(q[:, :, 0], kn[:, :, 0], vn[:, :, 0], kc, vc, np.array([start], np.int32), rot, base, scale)
+    np.testing.assert_allclose(o1[:, :, 0], od, rtol=1e-13, atol=1e-13)
+
+
+def test_gqa_prefill_is_causal_and_rows_are_independent():
+    q, kn, vn, kc, vc = _gqa_prefill_case(seed=82)
+    args = (4, 8, 1e4, 0.2)
+    o = oracle.gqa_prefill(q, kn, vn, kc, vc, *args)
+    q2, kn2, vn2 = q.copy(), kn.copy(), vn.copy()
+    q2[:, :, 3:] += 1.0
+    kn2[:, :, 3:] -= 2.0
+    vn2[:, :, 3:] *= 3.0
+    o2 = oracle.gqa_prefill(q2, kn2, vn2, kc, vc, *args)
+    np.testing.assert_array_equal(o[:, :, :3], o2[:, :, :3])     # earlier tokens never see later ones
+    assert np.abs(o[:, :, 3:] - o2[:, :, 3:]).max() > 1e-3
+    b, h, L, d = q.shape
+    rows = np.array([0, 7, L * 3 + 2, b * h * L - 1])
+    np.testing.assert_array_equal(oracle.gqa_prefill(q, kn, vn, kc, vc, *args, rows=rows), o.reshape(-1, d)[rows])
+
+
+def test_gqa_prefill_with_identical_keys_averages_the_prefix():
+    q, kn, vn, kc, vc = _gqa_prefill_case(seed=83)
+    start = 7
+    o = oracle.gqa_prefill(q, np.zeros_like(kn), vn, np.zeros_like(kc), vc, start, 8, 1e4, 0.5)
+    b, h, L, d = q.shape
+    hk = kn.shape[1]
+    for hh in range(h):
+        g = hh // (h // hk)
+        vals = np.concatenate([vc[:, g, :start], vn[:, g]], 1).astype(np.float64)
+        for i in range(L):
+            np.testing.assert_allclose(o[:, hh, i], vals[:, :start + i + 1].mean(1), rtol=1e-12, atol=1e-12)
+
+
+def test_gqa_prefill_rejects_bad_arguments():
+    q, kn, vn, kc, vc = _gqa_prefill_case(L=6, cap=20)
+    with pytest.raises(RuntimeError):
+        oracle.gqa_prefill(q, kn, vn, kc, vc, 15, 8, 1e4, 0.5)   # start + seq > cap
+    with pytest.raises(RuntimeError):
+        oracle.gqa_prefill(q, kn, vn, kc, vc, 0, 7, 1e4, 0.5)    # odd rot
+    with pytest.raises(RuntimeError):
+        oracle.gqa_prefill(q, kn, vn, kc, vc, 0, 8, 1e4, 0.5, rows=[10 ** 6])
