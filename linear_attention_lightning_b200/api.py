@@ -195,6 +195,38 @@ def gqa_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cach
     return o
 
 
+def gqa_prefill(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, start: int = 0, rot: int = 64, rope_base: float = 10000.0,
+                scale: Optional[float] = None, o: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """lightning_gqa_prefill: the softmax GQA layer over seq new tokens at
+    positions start .. start+seq-1. Writes their rotated keys and values into
+    the caches and returns o [batch, heads, seq, dim]. bf16 only; scale
+    defaults to 1/sqrt(dim)."""
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q must be bfloat16")
+    b, h, L, d = q.shape
+    bk, hk, cap, dk = k_cache.shape
+    if (bk, dk) != (b, d) or tuple(k_new.shape) != (b, hk, L, d) or tuple(v_new.shape) != (b, hk, L, d) \
+            or v_cache.shape != k_cache.shape:
+        raise ValueError("inconsistent shapes: q [b, heads, seq, dim], k/v_new [b, kv_heads, seq, dim], "
+                         "caches [b, kv_heads, cap, dim]")
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need_cuda(name, t, q.dtype)
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    if o is None:
+        o = torch.empty_like(q)
+    need = abi.lightning_gqa_prefill_workspace_size(b, h, L, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    abi.check(abi.lightning_gqa_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                        _DTYPES[q.dtype], int(start), b, h, hk, L, d, cap, int(rot),
+                                        float(rope_base), float(scale), _ptr(o), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
 def prefill_variant(dtype: torch.dtype, batch: int, heads: int, seq: int, dim: int, block: int,
                     variant: str = "auto") -> str:
     """Which kernel lightning_prefill would run: "simt", "tcgen05" or "pair"."""

@@ -1,0 +1,540 @@
+// Prefill of the softmax attention layer that M1 places after every seven
+// Lightning layers ("MINIMAX SIGNAL LAB · M1", §02: 64 query heads x 128,
+// softmax K/V 8 x 128, RoPE on 64 of the 128 dims in the softmax layers only;
+// §04: those layers keep a bf16 KV cache). Readings as for the decode step:
+// grouped-query attention (query head h reads KV head h / (heads/kv_heads)),
+// scores scaled by `scale`, rotate-half RoPE on the first `rot` dims, the
+// cache holds rotated keys. `seq` new tokens per sequence sit at positions
+// start .. start+seq-1; token i attends causally to positions 0 .. start+i:
+//   o_i = sum_{p <= start+i} softmax_p(scale * rope(q_i) . k_p) v_p.
+//
+// Two kernels:
+//   gqp_rope_kernel     one CTA per (token, sequence): the token's angles once
+//                       (double), then q rotated into a bf16 workspace and the
+//                       rotated key and the value written into the cache.
+//   gqp_attn_kernel     causal softmax attention on the tensor cores (tcgen05,
+//                       TMEM accumulators, TMA-fed), one CTA per 256 query rows
+//                       of one query head, as two 128-row tiles t = 0, 1.
+//
+// Attention, per key tile j of 128 positions (K_j, V_j from the cache):
+//   S_t = Q_t K_j^T         SS MMA bf16, M128 N128 K128 -> TMEM (fp32)
+//   softmax warpgroup t:    row max, P_t = 2^(S_t * scale * log2 e - m) as bf16
+//                           written over the first 64 columns of S_t in TMEM
+//                           (the row sum l adds the same rounded values);
+//                           the running max m is raised only when a row's max
+//                           grows by more than 2^8, and O_t is then rescaled
+//                           in TMEM before the next P V (P stays <= 2^8)
+//   O_t += P_t V_j          TS MMA bf16 (A = P from TMEM), M128 N128 K128
+// The MMA thread issues PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), ... so each
+// tile's softmax overlaps the other tile's MMAs. MMAs issued by one thread run
+// in order, so QK_t(j+1) writes S_t only after PV_t(j) has read P_t, and the
+// commit that announces S_t(j+1) also covers PV_t(j) (O_t is complete when the
+// softmax warpgroup reads it). The epilogue scales O_t by 1/l, rounds it to
+// bf16 into the Q_t tile's shared memory and stores it with TMA.
+// Key tiles end at position start+seq-1: the key and value tensor maps stop
+// there, so TMA reads zeros past it and no cache row beyond the sequence is
+// ever read.
+//
+// Warp roles: warp 0 TMA, warp 1 MMA, warp 2 TMEM, warps 4-7 and 8-11 the
+// softmax warpgroups of tiles 0 and 1. Every wait is bounded.
+// Shared memory: Q_0, Q_1 (32 KB each, also the output staging), 2 stages of
+// K and of V (32 KB each), barriers. TMEM: [0,128) S_0/P_0, [128,256) S_1/P_1,
+// [256,384) O_0, [384,512) O_1.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <string>
+
+#include "common.cuh"
+#include "prefill_tc.cuh"
+#include "tc_ptx.cuh"
+
+namespace la {
+namespace gqp {
+
+constexpr int kThreads = 384;
+constexpr int kDim = 128;
+constexpr int kRows = 128;                       // query rows per tile, positions per key tile
+constexpr int kQRows = 2 * kRows;                // query rows per CTA
+constexpr uint32_t kBoxBytes = 16384;            // 128 rows x 64 bf16 (128-byte rows)
+constexpr uint32_t kTileBytes = 2 * kBoxBytes;   // 128 rows x 128 dims
+constexpr int kStages = 2;
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
+constexpr int kNumBars = 16;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;  // + slack to align the base to 1024
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 256;       // + 128 t
+
+constexpr int Q_FULL = 0, K_FULL = 1 /* 2 */, K_EMPTY = 3 /* 2 */, V_FULL = 5 /* 2 */, V_EMPTY = 7 /* 2 */,
+              S_FULL = 9 /* 2 */, P_FULL = 11 /* 2 */, O_FINAL = 13 /* 2 */, DRAIN = 15;
+
+// the running max is raised only past this margin (log2 units): P <= 2^8
+constexpr float kRescaleMargin = 8.f;
+constexpr float kLog2eF = 1.4426950408889634f;
+
+__host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool a_mn, bool b_mn) {
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+constexpr uint32_t kIdescQK = idesc(128, 128, 1, false, false);  // Q (K-major) x K (K-major), bf16
+constexpr uint32_t kIdescPV = idesc(128, 128, 1, false, true);   // P (TMEM) x V (MN-major), bf16
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// --------------------------------------------------------------------- RoPE
+
+// grid (seq, batch), 256 threads. q_rot[b][h][i] = rope(q[b][h][i], start+i);
+// k_cache[b][g][start+i] = rope(k_new[b][g][i], start+i); v_cache[..] = v_new.
+// Elements travel in pairs (rot % 4 == 0 keeps a pair on one side of the
+// rotation); angles in double, rotation in fp32, results rounded to bf16.
+__global__ void __launch_bounds__(256)
+gqp_rope_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k_new,
+                const __nv_bfloat16 *__restrict__ v_new, __nv_bfloat16 *__restrict__ k_cache,
+                __nv_bfloat16 *__restrict__ v_cache, __nv_bfloat16 *__restrict__ q_rot, int heads, int kv_heads,
+                int seq, int start, int cap, int rot, double base) {
+    __shared__ float cs[kDim / 2], sn[kDim / 2];
+    const int i = blockIdx.x, b = blockIdx.y, pos = start + i, half = rot / 2;
+    for (int c = threadIdx.x; c < half; c += blockDim.x) {
+        double s, co;
+        sincos((double)pos * pow(base, -2.0 * c / (double)rot), &s, &co);
+        cs[c] = (float)co;
+        sn[c] = (float)s;
+    }
+    __syncthreads();
+    constexpr int kPairs = kDim / 2;
+    const int rows = heads + 2 * kv_heads;
+    for (int u = threadIdx.x; u < rows * kPairs; u += blockDim.x) {
+        const int hr = u / kPairs, c = 2 * (u - hr * kPairs);
+        const uint32_t *src;
+        uint32_t *dst;
+        if (hr < heads) {
+            const size_t row = ((size_t)b * heads + hr) * seq + i;
+            src = reinterpret_cast<const uint32_t *>(q + row * kDim);
+            dst = reinterpret_cast<uint32_t *>(q_rot + row * kDim);
+        } else if (hr < heads + kv_heads) {
+            const size_t g = (size_t)b * kv_heads + (hr - heads);
+            src = reinterpret_cast<const uint32_t *>(k_new + (g * seq + i) * kDim);
+            dst = reinterpret_cast<uint32_t *>(k_cache + (g * cap + pos) * kDim);
+        } else {
+            const size_t g = (size_t)b * kv_heads + (hr - heads - kv_heads);
+            reinterpret_cast<uint32_t *>(v_cache + (g * cap + pos) * kDim)[c / 2] =
+                reinterpret_cast<const uint32_t *>(v_new + (g * seq + i) * kDim)[c / 2];
+            continue;
+        }
+        const uint32_t x = src[c / 2];
+        if (c >= rot) {
+            dst[c / 2] = x;
+            continue;
+        }
+        const bool lo = c < half;
+        const int a = lo ? c : c - half;  // angle index of this pair's first element
+        const uint32_t y = src[(lo ? c + half : c - half) / 2];
+        const float sg = lo ? -1.f : 1.f;
+        const float r0 = fmaf(sg * ptx::bf16_lo(y), sn[a], ptx::bf16_lo(x) * cs[a]);
+        const float r1 = fmaf(sg * ptx::bf16_hi(y), sn[a + 1], ptx::bf16_hi(x) * cs[a + 1]);
+        dst[c / 2] = ptx::pack_bf16(r0, r1);
+    }
+}
+
+// ---------------------------------------------------------------- attention
+
+// 32 lanes x 128 consecutive 32-bit columns (four x32 loads, one wait by the caller)
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+#define GQP_LD32(Q)                                                                                        \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                                 \
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"                                 \
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                \
+                 : "=r"(r[32 * Q + 0]), "=r"(r[32 * Q + 1]), "=r"(r[32 * Q + 2]), "=r"(r[32 * Q + 3]),     \
+                   "=r"(r[32 * Q + 4]), "=r"(r[32 * Q + 5]), "=r"(r[32 * Q + 6]), "=r"(r[32 * Q + 7]),     \
+                   "=r"(r[32 * Q + 8]), "=r"(r[32 * Q + 9]), "=r"(r[32 * Q + 10]), "=r"(r[32 * Q + 11]),   \
+                   "=r"(r[32 * Q + 12]), "=r"(r[32 * Q + 13]), "=r"(r[32 * Q + 14]), "=r"(r[32 * Q + 15]), \
+                   "=r"(r[32 * Q + 16]), "=r"(r[32 * Q + 17]), "=r"(r[32 * Q + 18]), "=r"(r[32 * Q + 19]), \
+                   "=r"(r[32 * Q + 20]), "=r"(r[32 * Q + 21]), "=r"(r[32 * Q + 22]), "=r"(r[32 * Q + 23]), \
+                   "=r"(r[32 * Q + 24]), "=r"(r[32 * Q + 25]), "=r"(r[32 * Q + 26]), "=r"(r[32 * Q + 27]), \
+                   "=r"(r[32 * Q + 28]), "=r"(r[32 * Q + 29]), "=r"(r[32 * Q + 30]), "=r"(r[32 * Q + 31])  \
+                 : "r"(taddr + 32u * Q)                                                                    \
+                 : "memory")
+    GQP_LD32(0);
+    GQP_LD32(1);
+    GQP_LD32(2);
+    GQP_LD32(3);
+#undef GQP_LD32
+}
+
+struct Ctx {
+    uint8_t *smem;
+    uint32_t sbase;
+    uint64_t *bars;
+    volatile int *abort;
+    uint32_t tmem;
+};
+
+__device__ __forceinline__ bool wait_bar(const Ctx &c, int idx, uint32_t parity) {
+    return ptx::mbar_wait(&c.bars[idx], parity, c.abort);
+}
+// one thread of the warpgroup waits, the others learn the outcome at the named barrier
+__device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parity, bool leader, int bar_id) {
+    const bool ok = leader ? wait_bar(c, idx, parity) : true;
+    return ptx::named_bar_and(bar_id, 128, ok);
+}
+
+// Work of one CTA: query rows i0 .. i0+255 of head h of sequence b.
+struct Work {
+    int bh, bkv, i0, n[2];  // n[t]: key tiles that query tile t reads (0: tile absent)
+};
+
+__device__ __forceinline__ Work work_of(int heads, int kv_heads, int batch, int seq, int start) {
+    const int group = heads / kv_heads, nkv = batch * kv_heads;
+    const int npairs = (seq + kQRows - 1) / kQRows;
+    const int x = blockIdx.x;
+    const int hq = x % group, rest = x / group;
+    const int bkv = rest % nkv;
+    const int pi = npairs - 1 - rest / nkv;  // the longest rows first
+    const int b = bkv / kv_heads, g = bkv - b * kv_heads;
+    Work w;
+    w.bh = b * heads + g * group + hq;
+    w.bkv = bkv;
+    w.i0 = kQRows * pi;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int r0 = w.i0 + kRows * t;
+        w.n[t] = r0 < seq ? (start + min(r0 + kRows - 1, seq - 1)) / kRows + 1 : 0;
+    }
+    return w;
+}
+
+// tm_q: q_rot [batch*heads][seq][128]; tm_k, tm_v: caches [batch*kv_heads][start+seq][128]
+// (row stride cap); tm_o: o [batch*heads][seq][128]. All 128-byte swizzled boxes of 64 x 128.
+__global__ void __launch_bounds__(kThreads, 1)
+gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, int batch,
+                int heads, int kv_heads, int seq, int start, float sl2) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = ptx::smem_addr(smem_raw);
+    const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
+    Ctx c;
+    c.smem = smem_raw + pad;
+    c.sbase = raw_addr + pad;
+    c.bars = reinterpret_cast<uint64_t *>(c.smem + kOffBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c.smem + kOffMisc);
+    c.abort = reinterpret_cast<volatile int *>(c.smem + kOffMisc + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Work w = work_of(heads, kv_heads, batch, seq, start);
+    const int nmax = max(w.n[0], w.n[1]);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(&c.bars[i], 1);
+        ptx::mbar_init(&c.bars[P_FULL], 4);      // one arrival per softmax warp
+        ptx::mbar_init(&c.bars[P_FULL + 1], 4);
+        *c.abort = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tensormap(&tm_q);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+        ptx::prefetch_tensormap(&tm_o);
+    }
+    if (warp == 2) {
+        ptx::tmem_alloc(tmem_slot, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    c.tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            uint64_t *qbar = &c.bars[Q_FULL];
+            ptx::mbar_arrive_expect_tx(qbar, (w.n[1] > 0 ? 2 : 1) * kTileBytes);
+            for (int t = 0; t < 2; ++t) {
+                if (w.n[t] == 0) continue;
+                uint8_t *dst = c.smem + kOffQ + t * kTileBytes;
+                ptx::tma_load_3d(dst, &tm_q, qbar, 0, w.i0 + kRows * t, w.bh);
+                ptx::tma_load_3d(dst + kBoxBytes, &tm_q, qbar, 64, w.i0 + kRows * t, w.bh);
+            }
+            int k_issued = 0, v_issued = 0;
+            for (int j = 0; j < nmax && ok; ++j) {
+                const int st = j & 1;
+                const uint32_t epar = ((uint32_t)(j >> 1) & 1u) ^ 1u;  // phase of the stage's previous use
+                if (j >= kStages && !wait_bar(c, K_EMPTY + st, epar)) { ok = false; break; }
+                uint64_t *kb = &c.bars[K_FULL + st];
+                uint8_t *kd = c.smem + kOffK + st * kTileBytes;
+                ptx::mbar_arrive_expect_tx(kb, kTileBytes);
+                ptx::tma_load_3d(kd, &tm_k, kb, 0, kRows * j, w.bkv);
+                ptx::tma_load_3d(kd + kBoxBytes, &tm_k, kb, 64, kRows * j, w.bkv);
+                k_issued = j + 1;
+                if (j >= kStages && !wait_bar(c, V_EMPTY + st, epar)) { ok = false; break; }
+                uint64_t *vb = &c.bars[V_FULL + st];
+                uint8_t *vd = c.smem + kOffV + st * kTileBytes;
+                ptx::mbar_arrive_expect_tx(vb, kTileBytes);
+                ptx::tma_load_3d(vd, &tm_v, vb, 0, kRows * j, w.bkv);
+                ptx::tma_load_3d(vd + kBoxBytes, &tm_v, vb, 64, kRows * j, w.bkv);
+                v_issued = j + 1;
+            }
+            // let every copy issued land before the CTA may exit (earlier ones were consumed)
+            volatile int never = 0;
+            ptx::mbar_wait(qbar, 0, &never);
+            for (int j = k_issued > kStages ? k_issued - kStages : 0; j < k_issued; ++j)
+                ptx::mbar_wait(&c.bars[K_FULL + (j & 1)], (uint32_t)(j >> 1) & 1u, &never);
+            for (int j = v_issued > kStages ? v_issued - kStages : 0; j < v_issued; ++j)
+                ptx::mbar_wait(&c.bars[V_FULL + (j & 1)], (uint32_t)(j >> 1) & 1u, &never);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t tm = c.tmem;
+            const uint64_t dq0 = sdesc(c.sbase + kOffQ, 16u, 1024u);
+            const uint64_t dk0 = sdesc(c.sbase + kOffK, 16u, 1024u);
+            const uint64_t dv0 = sdesc(c.sbase + kOffV, kBoxBytes, 1024u);
+            int k_ready = -1, v_ready = -1;
+            bool ok = wait_bar(c, Q_FULL, 0);
+            if (ok) ptx::tc_fence_after();
+            // S_t = Q_t K_j^T
+            auto qk = [&](int t, int j) -> bool {
+                if (j > k_ready) {
+                    if (!wait_bar(c, K_FULL + (j & 1), (uint32_t)(j >> 1) & 1u)) return false;
+                    ptx::tc_fence_after();
+                    k_ready = j;
+                }
+                const uint64_t dq = dq0 + (uint64_t)((t * kTileBytes) >> 4);
+                const uint64_t dk = dk0 + (uint64_t)(((j & 1) * kTileBytes) >> 4);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
+                    ptx::mma_ss(tm + kColS + 128u * t, dq + koff, dk + koff, kIdescQK, k > 0);
+                }
+                ptx::mma_commit(&c.bars[S_FULL + t]);
+                if (t == 1 || j >= w.n[1]) ptx::mma_commit(&c.bars[K_EMPTY + (j & 1)]);  // last reader of K_j
+                return true;
+            };
+            // O_t += P_t V_j
+            auto pv = [&](int t, int j) -> bool {
+                if (j > v_ready) {
+                    if (!wait_bar(c, V_FULL + (j & 1), (uint32_t)(j >> 1) & 1u)) return false;
+                    v_ready = j;
+                }
+                if (!wait_bar(c, P_FULL + t, (uint32_t)j & 1u)) return false;
+                ptx::tc_fence_after();
+                const uint64_t dv = dv0 + (uint64_t)(((j & 1) * kTileBytes) >> 4);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    ptx::mma_ts(tm + kColO + 128u * t, tm + kColS + 128u * t + 8u * k,
+                                dv + (uint64_t)(k * (2048 >> 4)), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+                if (t == 1 || j >= w.n[1]) ptx::mma_commit(&c.bars[V_EMPTY + (j & 1)]);  // last reader of V_j
+                if (j == w.n[t] - 1) ptx::mma_commit(&c.bars[O_FINAL + t]);
+                return true;
+            };
+            for (int t = 0; t < 2 && ok; ++t)
+                if (w.n[t] > 0) ok = qk(t, 0);
+            for (int j = 0; j < nmax && ok; ++j) {
+#pragma unroll 1
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (j >= w.n[t]) continue;
+                    ok = pv(t, j);
+                    if (ok && j + 1 < w.n[t]) ok = qk(t, j + 1);
+                }
+            }
+            ptx::mma_commit(&c.bars[DRAIN]);
+            volatile int never = 0;
+            ptx::mbar_wait(&c.bars[DRAIN], 0, &never);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax warpgroups
+        const int t = (warp - 4) >> 2;             // query tile
+        const int r = threadIdx.x & 127;           // TMEM lane = row of the tile
+        const bool leader = r == 0;
+        const int bar_id = 1 + t;
+        const uint32_t trow = c.tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const uint32_t cs_ = kColS + 128u * t, co_ = kColO + 128u * t;
+        const int nt = w.n[t];
+        const int pmin = start + w.i0 + kRows * t;  // position of the tile's first row
+        const int qpos = pmin + r;
+        float m = -INFINITY, l = 0.f;               // running max (log2 units) and sum
+        bool done = nt > 0;
+        for (int j = 0; j < nt; ++j) {
+            if (!group_wait(c, S_FULL + t, (uint32_t)j & 1u, leader, bar_id)) { done = false; break; }
+            ptx::tc_fence_after();
+            uint32_t v[128];
+            tmem_ld128(trow + cs_, v);
+            ptx::tmem_ld_wait();
+            if (kRows * j + kRows - 1 > pmin) {     // the tile reaches past some row's position
+                const int lim = qpos - kRows * j;   // last live column of this row
+#pragma unroll
+                for (int u = 0; u < 128; ++u)
+                    if (u > lim) v[u] = 0xff800000u;  // -inf
+            }
+            float mx0 = __uint_as_float(v[0]), mx1 = __uint_as_float(v[1]);
+            float mx2 = __uint_as_float(v[2]), mx3 = __uint_as_float(v[3]);
+#pragma unroll
+            for (int u = 4; u < 128; u += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(v[u]));
+                mx1 = fmaxf(mx1, __uint_as_float(v[u + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(v[u + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(v[u + 3]));
+            }
+            const float mnew = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+            // raise the running max (warp-uniformly: the TMEM accesses are collective)
+            if (__any_sync(0xffffffffu, mnew > m + kRescaleMargin)) {
+                const float alpha = ptx::ex2(m - mnew);   // 0 on the first tile
+                l *= alpha;
+                m = mnew;
+                if (j > 0) {
+#pragma unroll 1
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t a[32];
+                        ptx::tmem_ld32(trow + co_ + 32u * q, a);
+                        ptx::tmem_ld_wait();
+                        uint32_t b0[16], b1[16];
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) {
+                            b0[u] = __float_as_uint(__uint_as_float(a[u]) * alpha);
+                            b1[u] = __float_as_uint(__uint_as_float(a[16 + u]) * alpha);
+                        }
+                        ptx::tmem_st16(trow + co_ + 32u * q, b0);
+                        ptx::tmem_st16(trow + co_ + 32u * q + 16u, b1);
+                    }
+                }
+            }
+            // P = 2^(S sl2 - m), bf16 pairs over the first 64 columns of S
+            const float nm = -m;
+            float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const float p0 = ptx::ex2(fmaf(__uint_as_float(v[32 * q + 2 * u]), sl2, nm));
+                    const float p1 = ptx::ex2(fmaf(__uint_as_float(v[32 * q + 2 * u + 1]), sl2, nm));
+                    pk[u] = ptx::pack_bf16(p0, p1);
+                    // the sum takes the rounded weights the P V product uses, so that o stays an
+                    // exact weighted mean of the values
+                    l0 += ptx::bf16_lo(pk[u]);
+                    l1 += ptx::bf16_hi(pk[u]);
+                }
+                ptx::tmem_st16(trow + cs_ + 16u * q, pk);
+            }
+            l += l0 + l1;
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&c.bars[P_FULL + t]);
+        }
+        if (done) done = group_wait(c, O_FINAL + t, 0, leader, bar_id);
+        if (done) {
+            // O / l -> bf16 -> this tile's Q buffer (128B-swizzled, as TMA reads it) -> TMA store;
+            // rows past seq are clipped by the store
+            ptx::tc_fence_after();
+            const float inv = 1.f / l;
+            uint8_t *tile = c.smem + kOffQ + t * kTileBytes;
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                uint32_t a0[32], a1[32];
+                ptx::tmem_ld32(trow + co_ + 64u * hb, a0);
+                ptx::tmem_ld32(trow + co_ + 64u * hb + 32u, a1);
+                ptx::tmem_ld_wait();
+                uint8_t *row = tile + hb * kBoxBytes + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint32_t *x = ch < 4 ? &a0[8 * ch] : &a1[8 * (ch - 4)];
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        pk[u] = ptx::pack_bf16(__uint_as_float(x[2 * u]) * inv, __uint_as_float(x[2 * u + 1]) * inv);
+                    *reinterpret_cast<uint4 *>(row + ((ch ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::named_bar_sync(bar_id, 128);
+            if (leader) {
+                ptx::tma_store_3d(&tm_o, tile, 0, w.i0 + kRows * t, w.bh);
+                ptx::tma_store_3d(&tm_o, tile + kBoxBytes, 64, w.i0 + kRows * t, w.bh);
+                ptx::bulk_commit();
+                ptx::bulk_wait_all();  // output stores complete before the CTA exits
+            }
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(c.tmem, kTmemCols);
+    }
+}
+
+}  // namespace gqp
+
+// [outer][rows][128] bf16 with `stride_rows` rows between consecutive outer
+// indices (rows <= stride_rows), as a 3-D tensor map of 64 x 128 boxes with
+// the 128-byte swizzle; rows past `rows` read as zeros and are clipped on store.
+inline bool gqp_make_map(CUtensorMap *map, const void *base, long long rows, long long stride_rows,
+                         long long outer, std::string *err) {
+    auto fn = tc::encode_fn(err);
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)gqp::kDim, (cuuint64_t)rows, (cuuint64_t)outer};
+    cuuint64_t strides[2] = {(cuuint64_t)gqp::kDim * 2, (cuuint64_t)stride_rows * gqp::kDim * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)gqp::kRows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *err = "cuTensorMapEncodeTiled failed (CUresult " + std::to_string((int)r) + ")";
+        return false;
+    }
+    return true;
+}
+
+// q, o: [batch][heads][seq][128]; k_new, v_new: [batch][kv_heads][seq][128];
+// caches [batch][kv_heads][cap][128]; q_rot: workspace of q's size. bf16 throughout.
+inline la_status launch_gqa_prefill(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                                    void *v_cache, int start, int batch, int heads, int kv_heads, int seq, int cap,
+                                    int rot, double base, float scale, void *o, void *q_rot, cudaStream_t stream,
+                                    std::string *err) {
+    using bf = __nv_bfloat16;
+    gqp::gqp_rope_kernel<<<dim3((unsigned)seq, (unsigned)batch), 256, 0, stream>>>(
+        static_cast<const bf *>(q), static_cast<const bf *>(k_new), static_cast<const bf *>(v_new),
+        static_cast<bf *>(k_cache), static_cast<bf *>(v_cache), static_cast<bf *>(q_rot), heads, kv_heads, seq,
+        start, cap, rot, base);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        *err = std::string("gqa prefill rope launch: ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    const long long bh = (long long)batch * heads, bkv = (long long)batch * kv_heads;
+    CUtensorMap mq, mk, mv, mo;
+    if (!gqp_make_map(&mq, q_rot, seq, seq, bh, err) || !gqp_make_map(&mk, k_cache, (long long)start + seq, cap, bkv, err) ||
+        !gqp_make_map(&mv, v_cache, (long long)start + seq, cap, bkv, err) || !gqp_make_map(&mo, o, seq, seq, bh, err))
+        return LA_ERR_CUDA;
+    e = cudaFuncSetAttribute(gqp::gqp_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gqp::kSmemBytes);
+    if (e != cudaSuccess) {
+        *err = std::string("cudaFuncSetAttribute(gqa prefill attention): ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    const long long ctas = bh * ((seq + gqp::kQRows - 1) / gqp::kQRows);
+    gqp::gqp_attn_kernel<<<(unsigned)ctas, gqp::kThreads, gqp::kSmemBytes, stream>>>(
+        mq, mk, mv, mo, batch, heads, kv_heads, seq, start, scale * gqp::kLog2eF);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        *err = std::string("gqa prefill attention launch: ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    err->clear();
+    return LA_OK;
+}
+
+}  // namespace la

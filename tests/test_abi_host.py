@@ -281,3 +281,48 @@ def test_gqa_workspace_size_and_empty_batch():
     assert abi.lightning_gqa_decode_workspace_size(2, 64, 1024) == n * 4 + n * 4 + n * 128 * 4 + 2 * 64 * 128 * 4
     assert abi.lightning_gqa_decode_workspace_size(0, 64, 1024) == 0
     assert _gqa(batch=0) == abi.LA_OK
+
+
+def _gqp(**kw):
+    # sizes: q, o 2 x 64 x 512 x 128 bf16 = 16 MiB; caches 2 x 8 x 1024 x 128 bf16 = 4 MiB (fake addresses 256 MiB apart)
+    a = dict(q=Q, kn=K, vn=V, kc=0x10000000 * 30, vc=0x10000000 * 40, dtype=abi.LA_DTYPE_BF16, start=100, batch=2,
+             heads=64, kv=8, seq=512, dim=128, cap=1024, rot=64, base=1e4, scale=0.088, o=O, ws=WS, ws_bytes=1 << 26)
+    a.update(kw)
+    return abi.lightning_gqa_prefill(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["dtype"], a["start"], a["batch"],
+                                     a["heads"], a["kv"], a["seq"], a["dim"], a["cap"], a["rot"], a["base"],
+                                     a["scale"], a["o"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype=9), abi.LA_ERR_INVALID_ARG),
+    (dict(dtype=abi.LA_DTYPE_F32), abi.LA_ERR_UNSUPPORTED),   # bf16 only
+    (dict(kv=7), abi.LA_ERR_INVALID_ARG),                     # does not divide 64
+    (dict(start=-1), abi.LA_ERR_INVALID_ARG),
+    (dict(seq=-3), abi.LA_ERR_INVALID_ARG),
+    (dict(start=600), abi.LA_ERR_INVALID_ARG),                # start + seq > cap
+    (dict(dim=64), abi.LA_ERR_UNSUPPORTED),
+    (dict(rot=62), abi.LA_ERR_INVALID_ARG),                   # not a multiple of 4
+    (dict(rot=132), abi.LA_ERR_INVALID_ARG),
+    (dict(base=-1.0), abi.LA_ERR_INVALID_ARG),
+    (dict(scale=0.0), abi.LA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), abi.LA_ERR_INVALID_ARG),
+    (dict(batch=70000, start=0, seq=1, cap=2), abi.LA_ERR_UNSUPPORTED),
+    (dict(kn=None), abi.LA_ERR_INVALID_ARG),
+    (dict(q=Q + 8), abi.LA_ERR_INVALID_ARG),                  # not 16-byte aligned
+    (dict(ws_bytes=1 << 20), abi.LA_ERR_INVALID_ARG),         # workspace too small
+    (dict(o=Q + (1 << 20)), abi.LA_ERR_INVALID_ARG),          # o overlaps q
+    (dict(ws=0x10000000 * 30 + 4096), abi.LA_ERR_INVALID_ARG),  # workspace overlaps k_cache
+    (dict(vc=0x10000000 * 30 + 1024), abi.LA_ERR_INVALID_ARG),  # caches overlap
+])
+def test_gqa_prefill_argument_errors(kw, status):
+    assert _gqp(**kw) == status
+    assert abi.last_error_message() != ""
+
+
+def test_gqa_prefill_workspace_size_and_empty_calls():
+    # the rotated queries, bf16, q's shape
+    assert abi.lightning_gqa_prefill_workspace_size(2, 64, 512, 128) == 2 * 64 * 512 * 128 * 2
+    assert abi.lightning_gqa_prefill_workspace_size(2, 64, 512, 64) == 0
+    assert abi.lightning_gqa_prefill_workspace_size(-1, 64, 512, 128) == 0
+    assert _gqp(batch=0) == abi.LA_OK
+    assert _gqp(seq=0, q=None, o=None, ws=None) == abi.LA_OK
