@@ -368,6 +368,9 @@ def run_ours(args):
     # decode step of the softmax GQA layer the hybrid model interleaves
     gqa = run_gqa_leg(dev, stream, args, world) if args.gqa_steps > 0 else None
 
+    # prefill of the softmax GQA layer at the same context length
+    gqp = run_gqa_prefill_leg(dev, stream, args, world) if args.gqa_prefill_steps > 0 else None
+
     # gradients of the same prefill (dq, dk, dv, d state_in)
     bwd = run_backward_leg(w, dev, stream, inp, dcode, args, world) if args.backward_steps > 0 else None
 
@@ -391,6 +394,7 @@ def run_ours(args):
         "snapshots": snaps,
         "norm_gate": ng,
         "gqa_decode": gqa,
+        "gqa_prefill": gqp,
         "backward": bwd,
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
@@ -560,6 +564,52 @@ def run_gqa_leg(dev, stream, args, world):
             "l2": "cache %.1f GB per step > L2" % (by / 1e9)}
 
 
+def run_gqa_prefill_leg(dev, stream, args, world):
+    """lightning_gqa_prefill: one sequence of args.gqa_prefill_seq new tokens
+    (empty cache), 64 query heads over 8 KV heads, RoPE on 64 dims, bf16;
+    timed like the main leg. Causal FLOPs: 4 d per (query, key <= query) pair
+    and query head (Q K^T and P V)."""
+    import torch
+    from linear_attention_lightning_b200 import abi
+    b, h, hk, L, d = 1, GQA_HEADS, GQA_KV_HEADS, args.gqa_prefill_seq, 128
+    g = torch.Generator(device=dev).manual_seed(3100)
+    mk = lambda *shape: torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+    q, kn, vn = mk(b, h, L, d), mk(b, hk, L, d), mk(b, hk, L, d)
+    kc = torch.empty((b, hk, L, d), dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    o = torch.empty_like(q)
+    need = abi.lightning_gqa_prefill_workspace_size(b, h, L, d)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    sp = stream.cuda_stream
+
+    def step():
+        abi.check(abi.lightning_gqa_prefill(q.data_ptr(), kn.data_ptr(), vn.data_ptr(), kc.data_ptr(), vc.data_ptr(),
+                                            abi.LA_DTYPE_BF16, 0, b, h, hk, L, d, L, 64, 1e4, 1.0 / d ** 0.5,
+                                            o.data_ptr(), ws.data_ptr(), need, sp))
+
+    for _ in range(args.warmup):
+        step()
+    steps = args.gqa_prefill_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    peaks = load_peaks()
+    causal = 4.0 * d * h * b * L * (L + 1) / 2
+    tf = causal / (ms / 1e3) / 1e12
+    return {"config": {"batch": b, "heads": h, "kv_heads": hk, "seq": L, "dim": d, "rot": 64, "dtype": "bf16"},
+            "steps": steps, "ms_per_step": round(ms, 3), "launches_per_step": 2,
+            "tokens_per_s": round(world * b * L / (ms / 1e3), 1),
+            "tflops_causal": round(tf, 2),
+            "roofline": roofline("tensor", tf, peaks["bf16_tflops"], "TFLOP/s"),
+            "flops": "causal: 4 d per (query, key <= query) pair and query head; the step includes the RoPE launch"}
+
+
 def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     """lightning_prefill_backward on the workload (AUTO: the CTA-pair tensor-core
     kernel where it applies), timed like the main leg: dQ causal on (dO, V, K),
@@ -671,6 +721,10 @@ def parse_args(argv=None):
                    help="timed steps of the softmax GQA decode leg (0 skips it)")
     p.add_argument("--gqa-context", type=int, default=GQA_CAP,
                    help="cached tokens per sequence in the GQA decode leg")
+    p.add_argument("--gqa-prefill-steps", type=int, default=3,
+                   help="timed steps of the softmax GQA prefill leg (0 skips it)")
+    p.add_argument("--gqa-prefill-seq", type=int, default=131072,
+                   help="new tokens of the GQA prefill leg")
     p.add_argument("--norm-gate-steps", type=int, default=20,
                    help="timed steps of the norm-and-gate epilogue leg (0 skips it)")
     p.add_argument("--backward-steps", type=int, default=10,
