@@ -24,7 +24,8 @@
 //                           the running max m is raised only when a row's max
 //                           grows by more than 2^8, and O_t is then rescaled
 //                           in TMEM before the next P V (P stays <= 2^8)
-//   O_t += P_t V_j          TS MMA bf16 (A = P from TMEM), M128 N128 K128
+//   O_t += P_t V_j          TS MMA bf16 (A = P from TMEM), M128 N128 K128, in two
+//                           halves of 64 keys, each as soon as its half of P is written
 // The MMA thread issues PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), ... so each
 // tile's softmax overlaps the other tile's MMAs. MMAs issued by one thread run
 // in order, so QK_t(j+1) writes S_t only after PV_t(j) has read P_t, and the
@@ -35,8 +36,9 @@
 // there, so TMA reads zeros past it and no cache row beyond the sequence is
 // ever read.
 //
-// Warp roles: warp 0 TMA, warp 1 MMA, warp 2 TMEM, warps 4-7 and 8-11 the
-// softmax warpgroups of tiles 0 and 1. Every wait is bounded.
+// Warp roles: warp 0 TMA, warp 1 MMA (the whole warp follows the waits, one elected lane
+// issues), warp 2 TMEM, warps 4-7 and 8-11 the softmax warpgroups of tiles 0 and 1; the
+// control warps hand most of their registers to the softmax warps. Every wait is bounded.
 // Shared memory: Q_0, Q_1 (32 KB each, also the output staging), 2 stages of
 // K and of V (32 KB each), barriers. TMEM: [0,128) S_0/P_0, [128,256) S_1/P_1,
 // [256,384) O_0, [384,512) O_1.
@@ -65,15 +67,22 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + 2 * kTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
 constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
-constexpr int kNumBars = 16;
+constexpr int kNumBars = 18;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;  // + slack to align the base to 1024
+
+// registers per thread after the split: the control warpgroup gives its share to the two
+// softmax warpgroups. The launcher checks the kernel's allocation (threads x registers) holds
+// the split, since a setmaxnreg.inc beyond it would wait forever.
+constexpr int kCtrlRegs = 56, kSoftmaxRegs = 224;
+constexpr int kSplitRegs = 4 * 32 * kCtrlRegs + 8 * 32 * kSoftmaxRegs;
+static_assert(kSplitRegs <= kThreads * ((65536 / kThreads) & ~7), "register split above the launch's");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;       // + 128 t
 
 constexpr int Q_FULL = 0, K_FULL = 1 /* 2 */, K_EMPTY = 3 /* 2 */, V_FULL = 5 /* 2 */, V_EMPTY = 7 /* 2 */,
-              S_FULL = 9 /* 2 */, P_FULL = 11 /* 2 */, O_FINAL = 13 /* 2 */, DRAIN = 15;
+              S_FULL = 9 /* 2 */, P_FULL = 11 /* 2 x 2: tile, half */, O_FINAL = 15 /* 2 */, DRAIN = 17;
 
 // the running max is raised only past this margin (log2 units): P <= 2^8
 constexpr float kRescaleMargin = 8.f;
@@ -182,10 +191,49 @@ struct Ctx {
 __device__ __forceinline__ bool wait_bar(const Ctx &c, int idx, uint32_t parity) {
     return ptx::mbar_wait(&c.bars[idx], parity, c.abort);
 }
-// one thread of the warpgroup waits, the others learn the outcome at the named barrier
-__device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parity, bool leader, int bar_id) {
-    const bool ok = leader ? wait_bar(c, idx, parity) : true;
-    return ptx::named_bar_and(bar_id, 128, ok);
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// P = 2^(S sl2 - m) for keys 64 H .. 64 H + 63 of one row of scores: bf16 pairs into TMEM
+// columns [taddr + 32 H, taddr + 32 H + 32); returns the sum of the rounded weights.
+template <int H>
+__device__ __forceinline__ float p_half(const uint32_t (&v)[128], float sl2, float m, uint32_t taddr) {
+    const float2 sl = make_float2(sl2, sl2), nm = make_float2(-m, -m), one = make_float2(1.f, 1.f);
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int q = 2 * H; q < 2 * H + 2; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const float2 x = fma2(make_float2(__uint_as_float(v[32 * q + 2 * u]), __uint_as_float(v[32 * q + 2 * u + 1])),
+                                  sl, nm);
+            pk[u] = ptx::pack_bf16(ptx::ex2(x.x), ptx::ex2(x.y));
+            acc = fma2(make_float2(ptx::bf16_lo(pk[u]), ptx::bf16_hi(pk[u])), one, acc);
+        }
+        ptx::tmem_st16(taddr + 16u * q, pk);
+    }
+    return acc.x + acc.y;
+}
+
+// one lane of a converged warp (the lowest active one)
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+    return pred != 0;
 }
 
 // Work of one CTA: query rows i0 .. i0+255 of head h of sequence b.
@@ -234,8 +282,7 @@ gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(&c.bars[i], 1);
-        ptx::mbar_init(&c.bars[P_FULL], 4);      // one arrival per softmax warp
-        ptx::mbar_init(&c.bars[P_FULL + 1], 4);
+        for (int i = 0; i < 4; ++i) ptx::mbar_init(&c.bars[P_FULL + i], 4);  // one arrival per softmax warp
         *c.abort = 0;
         ptx::fence_mbar_init();
     }
@@ -254,105 +301,125 @@ gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ptx::tc_fence_after();
     c.tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            bool ok = true;
-            uint64_t *qbar = &c.bars[Q_FULL];
-            ptx::mbar_arrive_expect_tx(qbar, (w.n[1] > 0 ? 2 : 1) * kTileBytes);
-            for (int t = 0; t < 2; ++t) {
-                if (w.n[t] == 0) continue;
-                uint8_t *dst = c.smem + kOffQ + t * kTileBytes;
-                ptx::tma_load_3d(dst, &tm_q, qbar, 0, w.i0 + kRows * t, w.bh);
-                ptx::tma_load_3d(dst + kBoxBytes, &tm_q, qbar, 64, w.i0 + kRows * t, w.bh);
+    // registers: the control warps (TMA, MMA, TMEM) give theirs to the softmax warps
+    // (4 x 32 x 56 + 8 x 32 x 224 = 384 x 168, the launch's allocation)
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+        if (warp == 0) {
+            // ------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                bool ok = true;
+                uint64_t *qbar = &c.bars[Q_FULL];
+                ptx::mbar_arrive_expect_tx(qbar, (w.n[1] > 0 ? 2 : 1) * kTileBytes);
+                for (int t = 0; t < 2; ++t) {
+                    if (w.n[t] == 0) continue;
+                    uint8_t *dst = c.smem + kOffQ + t * kTileBytes;
+                    ptx::tma_load_3d(dst, &tm_q, qbar, 0, w.i0 + kRows * t, w.bh);
+                    ptx::tma_load_3d(dst + kBoxBytes, &tm_q, qbar, 64, w.i0 + kRows * t, w.bh);
+                }
+                int k_issued = 0, v_issued = 0;
+                for (int j = 0; j < nmax && ok; ++j) {
+                    const int st = j & 1;
+                    const uint32_t epar = ((uint32_t)(j >> 1) & 1u) ^ 1u;  // phase of the stage's previous use
+                    if (j >= kStages && !wait_bar(c, K_EMPTY + st, epar)) { ok = false; break; }
+                    uint64_t *kb = &c.bars[K_FULL + st];
+                    uint8_t *kd = c.smem + kOffK + st * kTileBytes;
+                    ptx::mbar_arrive_expect_tx(kb, kTileBytes);
+                    ptx::tma_load_3d(kd, &tm_k, kb, 0, kRows * j, w.bkv);
+                    ptx::tma_load_3d(kd + kBoxBytes, &tm_k, kb, 64, kRows * j, w.bkv);
+                    k_issued = j + 1;
+                    if (j >= kStages && !wait_bar(c, V_EMPTY + st, epar)) { ok = false; break; }
+                    uint64_t *vb = &c.bars[V_FULL + st];
+                    uint8_t *vd = c.smem + kOffV + st * kTileBytes;
+                    ptx::mbar_arrive_expect_tx(vb, kTileBytes);
+                    ptx::tma_load_3d(vd, &tm_v, vb, 0, kRows * j, w.bkv);
+                    ptx::tma_load_3d(vd + kBoxBytes, &tm_v, vb, 64, kRows * j, w.bkv);
+                    v_issued = j + 1;
+                }
+                // let every copy issued land before the CTA may exit (earlier ones were consumed)
+                volatile int never = 0;
+                ptx::mbar_wait(qbar, 0, &never);
+                for (int j = k_issued > kStages ? k_issued - kStages : 0; j < k_issued; ++j)
+                    ptx::mbar_wait(&c.bars[K_FULL + (j & 1)], (uint32_t)(j >> 1) & 1u, &never);
+                for (int j = v_issued > kStages ? v_issued - kStages : 0; j < v_issued; ++j)
+                    ptx::mbar_wait(&c.bars[V_FULL + (j & 1)], (uint32_t)(j >> 1) & 1u, &never);
             }
-            int k_issued = 0, v_issued = 0;
-            for (int j = 0; j < nmax && ok; ++j) {
-                const int st = j & 1;
-                const uint32_t epar = ((uint32_t)(j >> 1) & 1u) ^ 1u;  // phase of the stage's previous use
-                if (j >= kStages && !wait_bar(c, K_EMPTY + st, epar)) { ok = false; break; }
-                uint64_t *kb = &c.bars[K_FULL + st];
-                uint8_t *kd = c.smem + kOffK + st * kTileBytes;
-                ptx::mbar_arrive_expect_tx(kb, kTileBytes);
-                ptx::tma_load_3d(kd, &tm_k, kb, 0, kRows * j, w.bkv);
-                ptx::tma_load_3d(kd + kBoxBytes, &tm_k, kb, 64, kRows * j, w.bkv);
-                k_issued = j + 1;
-                if (j >= kStages && !wait_bar(c, V_EMPTY + st, epar)) { ok = false; break; }
-                uint64_t *vb = &c.bars[V_FULL + st];
-                uint8_t *vd = c.smem + kOffV + st * kTileBytes;
-                ptx::mbar_arrive_expect_tx(vb, kTileBytes);
-                ptx::tma_load_3d(vd, &tm_v, vb, 0, kRows * j, w.bkv);
-                ptx::tma_load_3d(vd + kBoxBytes, &tm_v, vb, 64, kRows * j, w.bkv);
-                v_issued = j + 1;
-            }
-            // let every copy issued land before the CTA may exit (earlier ones were consumed)
-            volatile int never = 0;
-            ptx::mbar_wait(qbar, 0, &never);
-            for (int j = k_issued > kStages ? k_issued - kStages : 0; j < k_issued; ++j)
-                ptx::mbar_wait(&c.bars[K_FULL + (j & 1)], (uint32_t)(j >> 1) & 1u, &never);
-            for (int j = v_issued > kStages ? v_issued - kStages : 0; j < v_issued; ++j)
-                ptx::mbar_wait(&c.bars[V_FULL + (j & 1)], (uint32_t)(j >> 1) & 1u, &never);
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t tm = c.tmem;
-            const uint64_t dq0 = sdesc(c.sbase + kOffQ, 16u, 1024u);
-            const uint64_t dk0 = sdesc(c.sbase + kOffK, 16u, 1024u);
-            const uint64_t dv0 = sdesc(c.sbase + kOffV, kBoxBytes, 1024u);
-            int k_ready = -1, v_ready = -1;
-            bool ok = wait_bar(c, Q_FULL, 0);
-            if (ok) ptx::tc_fence_after();
-            // S_t = Q_t K_j^T
-            auto qk = [&](int t, int j) -> bool {
-                if (j > k_ready) {
-                    if (!wait_bar(c, K_FULL + (j & 1), (uint32_t)(j >> 1) & 1u)) return false;
-                    ptx::tc_fence_after();
-                    k_ready = j;
-                }
-                const uint64_t dq = dq0 + (uint64_t)((t * kTileBytes) >> 4);
-                const uint64_t dk = dk0 + (uint64_t)(((j & 1) * kTileBytes) >> 4);
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            // the whole warp follows the waits; one elected lane issues the MMAs and commits
+            {
+                const uint32_t tm = c.tmem;
+                const uint64_t dq0 = sdesc(c.sbase + kOffQ, 16u, 1024u);
+                const uint64_t dk0 = sdesc(c.sbase + kOffK, 16u, 1024u);
+                const uint64_t dv0 = sdesc(c.sbase + kOffV, kBoxBytes, 1024u);
+                int k_ready = -1, v_ready = -1;
+                bool ok = wait_bar(c, Q_FULL, 0);
+                if (ok) ptx::tc_fence_after();
+                // S_t = Q_t K_j^T
+                auto qk = [&](int t, int j) -> bool {
+                    if (j > k_ready) {
+                        if (!wait_bar(c, K_FULL + (j & 1), (uint32_t)(j >> 1) & 1u)) return false;
+                        ptx::tc_fence_after();
+                        k_ready = j;
+                    }
+                    const uint64_t dq = dq0 + (uint64_t)((t * kTileBytes) >> 4);
+                    const uint64_t dk = dk0 + (uint64_t)(((j & 1) * kTileBytes) >> 4);
+                    if (elect_one()) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
-                    ptx::mma_ss(tm + kColS + 128u * t, dq + koff, dk + koff, kIdescQK, k > 0);
-                }
-                ptx::mma_commit(&c.bars[S_FULL + t]);
-                if (t == 1 || j >= w.n[1]) ptx::mma_commit(&c.bars[K_EMPTY + (j & 1)]);  // last reader of K_j
-                return true;
-            };
-            // O_t += P_t V_j
-            auto pv = [&](int t, int j) -> bool {
-                if (j > v_ready) {
-                    if (!wait_bar(c, V_FULL + (j & 1), (uint32_t)(j >> 1) & 1u)) return false;
-                    v_ready = j;
-                }
-                if (!wait_bar(c, P_FULL + t, (uint32_t)j & 1u)) return false;
-                ptx::tc_fence_after();
-                const uint64_t dv = dv0 + (uint64_t)(((j & 1) * kTileBytes) >> 4);
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
+                            ptx::mma_ss(tm + kColS + 128u * t, dq + koff, dk + koff, kIdescQK, k > 0);
+                        }
+                        ptx::mma_commit(&c.bars[S_FULL + t]);
+                        if (t == 1 || j >= w.n[1]) ptx::mma_commit(&c.bars[K_EMPTY + (j & 1)]);  // last reader of K_j
+                    }
+                    __syncwarp();
+                    return true;
+                };
+                // O_t += P_t V_j
+                auto pv = [&](int t, int j) -> bool {
+                    if (j > v_ready) {
+                        if (!wait_bar(c, V_FULL + (j & 1), (uint32_t)(j >> 1) & 1u)) return false;
+                        v_ready = j;
+                    }
+                    const uint64_t dv = dv0 + (uint64_t)(((j & 1) * kTileBytes) >> 4);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    ptx::mma_ts(tm + kColO + 128u * t, tm + kColS + 128u * t + 8u * k,
-                                dv + (uint64_t)(k * (2048 >> 4)), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
-                if (t == 1 || j >= w.n[1]) ptx::mma_commit(&c.bars[V_EMPTY + (j & 1)]);  // last reader of V_j
-                if (j == w.n[t] - 1) ptx::mma_commit(&c.bars[O_FINAL + t]);
-                return true;
-            };
-            for (int t = 0; t < 2 && ok; ++t)
-                if (w.n[t] > 0) ok = qk(t, 0);
-            for (int j = 0; j < nmax && ok; ++j) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        // keys 64 hh .. 64 hh + 63, as soon as their half of P is in TMEM
+                        if (!wait_bar(c, P_FULL + 2 * t + hh, (uint32_t)j & 1u)) return false;
+                        ptx::tc_fence_after();
+                        if (elect_one()) {
+#pragma unroll
+                            for (int k = 4 * hh; k < 4 * hh + 4; ++k)
+                                ptx::mma_ts(tm + kColO + 128u * t, tm + kColS + 128u * t + 8u * k,
+                                            dv + (uint64_t)(k * (2048 >> 4)), kIdescPV, (j > 0 || k > 0) ? 1u : 0u);
+                            if (hh == 1) {
+                                if (t == 1 || j >= w.n[1]) ptx::mma_commit(&c.bars[V_EMPTY + (j & 1)]);  // last reader of V_j
+                                if (j == w.n[t] - 1) ptx::mma_commit(&c.bars[O_FINAL + t]);
+                            }
+                        }
+                        __syncwarp();
+                    }
+                    return true;
+                };
+                for (int t = 0; t < 2 && ok; ++t)
+                    if (w.n[t] > 0) ok = qk(t, 0);
+                for (int j = 0; j < nmax && ok; ++j) {
 #pragma unroll 1
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (j >= w.n[t]) continue;
-                    ok = pv(t, j);
-                    if (ok && j + 1 < w.n[t]) ok = qk(t, j + 1);
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j >= w.n[t]) continue;
+                        ok = pv(t, j);
+                        if (ok && j + 1 < w.n[t]) ok = qk(t, j + 1);
+                    }
                 }
+                if (elect_one()) ptx::mma_commit(&c.bars[DRAIN]);
+                __syncwarp();
+                volatile int never = 0;
+                ptx::mbar_wait(&c.bars[DRAIN], 0, &never);
             }
-            ptx::mma_commit(&c.bars[DRAIN]);
-            volatile int never = 0;
-            ptx::mbar_wait(&c.bars[DRAIN], 0, &never);
         }
-    } else if (warp >= 4) {
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // ------------------------------------------------------------ softmax warpgroups
         const int t = (warp - 4) >> 2;             // query tile
         const int r = threadIdx.x & 127;           // TMEM lane = row of the tile
@@ -366,27 +433,26 @@ gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         float m = -INFINITY, l = 0.f;               // running max (log2 units) and sum
         bool done = nt > 0;
         for (int j = 0; j < nt; ++j) {
-            if (!group_wait(c, S_FULL + t, (uint32_t)j & 1u, leader, bar_id)) { done = false; break; }
+            // every thread waits itself: the lanes of a warp poll together and agree
+            if (!ptx::mbar_wait(&c.bars[S_FULL + t], (uint32_t)j & 1u, c.abort)) { done = false; break; }
             ptx::tc_fence_after();
             uint32_t v[128];
             tmem_ld128(trow + cs_, v);
             ptx::tmem_ld_wait();
-            if (kRows * j + kRows - 1 > pmin) {     // the tile reaches past some row's position
+            const bool masked = kRows * j + kRows - 1 > pmin;  // the tile reaches past some row's position
+            if (masked) {
                 const int lim = qpos - kRows * j;   // last live column of this row
 #pragma unroll
                 for (int u = 0; u < 128; ++u)
                     if (u > lim) v[u] = 0xff800000u;  // -inf
             }
             float mx0 = __uint_as_float(v[0]), mx1 = __uint_as_float(v[1]);
-            float mx2 = __uint_as_float(v[2]), mx3 = __uint_as_float(v[3]);
 #pragma unroll
-            for (int u = 4; u < 128; u += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(v[u]));
-                mx1 = fmaxf(mx1, __uint_as_float(v[u + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(v[u + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(v[u + 3]));
+            for (int u = 2; u < 126; u += 4) {
+                mx0 = max3(mx0, __uint_as_float(v[u]), __uint_as_float(v[u + 1]));
+                mx1 = max3(mx1, __uint_as_float(v[u + 2]), __uint_as_float(v[u + 3]));
             }
-            const float mnew = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+            const float mnew = fmaxf(m, max3(mx0, mx1, fmaxf(__uint_as_float(v[126]), __uint_as_float(v[127]))) * sl2);
             // raise the running max (warp-uniformly: the TMEM accesses are collective)
             if (__any_sync(0xffffffffu, mnew > m + kRescaleMargin)) {
                 const float alpha = ptx::ex2(m - mnew);   // 0 on the first tile
@@ -409,31 +475,21 @@ gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
-            // P = 2^(S sl2 - m), bf16 pairs over the first 64 columns of S
-            const float nm = -m;
-            float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const float p0 = ptx::ex2(fmaf(__uint_as_float(v[32 * q + 2 * u]), sl2, nm));
-                    const float p1 = ptx::ex2(fmaf(__uint_as_float(v[32 * q + 2 * u + 1]), sl2, nm));
-                    pk[u] = ptx::pack_bf16(p0, p1);
-                    // the sum takes the rounded weights the P V product uses, so that o stays an
-                    // exact weighted mean of the values
-                    l0 += ptx::bf16_lo(pk[u]);
-                    l1 += ptx::bf16_hi(pk[u]);
-                }
-                ptx::tmem_st16(trow + cs_ + 16u * q, pk);
-            }
-            l += l0 + l1;
+            // P = 2^(S sl2 - m) as bf16 pairs over the first 64 columns of S, in two halves of
+            // 64 keys: the P V of the first half runs while the second is computed
+            l += p_half<0>(v, sl2, m, trow + cs_);
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&c.bars[P_FULL + t]);
+            if (lane == 0) ptx::mbar_arrive(&c.bars[P_FULL + 2 * t]);
+            l += p_half<1>(v, sl2, m, trow + cs_);
+            ptx::tmem_st_wait();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&c.bars[P_FULL + 2 * t + 1]);
         }
-        if (done) done = group_wait(c, O_FINAL + t, 0, leader, bar_id);
+        if (done) done = ptx::mbar_wait(&c.bars[O_FINAL + t], 0, c.abort);
+        done = ptx::named_bar_and(bar_id, 128, done);  // the four warps agree before the epilogue
         if (done) {
             // O / l -> bf16 -> this tile's Q buffer (128B-swizzled, as TMA reads it) -> TMA store;
             // rows past seq are clipped by the store
@@ -523,6 +579,13 @@ inline la_status launch_gqa_prefill(const void *q, const void *k_new, const void
     e = cudaFuncSetAttribute(gqp::gqp_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gqp::kSmemBytes);
     if (e != cudaSuccess) {
         *err = std::string("cudaFuncSetAttribute(gqa prefill attention): ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, gqp::gqp_attn_kernel);
+    if (e != cudaSuccess || fa.numRegs * gqp::kThreads < gqp::kSplitRegs) {
+        // the warps' register split would wait for registers the launch never holds
+        *err = "gqa prefill attention: register allocation below the kernel's split";
         return LA_ERR_CUDA;
     }
     const long long ctas = bh * ((seq + gqp::kQRows - 1) / gqp::kQRows);
