@@ -31,7 +31,8 @@
 // Q ⊙ d_q, S and K ⊙ d_k rounded to fp16; V widened to fp16 exactly; fp32
 // accumulation; the fp32 state stays in TMEM for the whole sequence.
 //
-// Warp roles (per CTA): warp 0 TMA, warp 1 MMA (even CTA only), warp 2 TMEM,
+// Warp roles (per CTA): warp 0 TMA, warp 1 MMA (even CTA only; the whole warp follows
+// the waits and one elected lane issues), warp 2 TMEM,
 // warp 3 forwards "Q/K landed" to the even CTA; warpgroup A (warps 4-7) writes
 // K ⊙ d_k and widens V, then turns keys 0..127 of P into fp16 P ⊙ D;
 // warpgroup B (warps 8-11) builds Qd, then does keys 128..255 of P;
@@ -130,6 +131,13 @@ __device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
 // output stores), which costs thousands of cycles per hand-off.
 __device__ __forceinline__ void arrive_leader(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(map_to_rank(bar, 0)) : "memory");
+}
+
+// one lane of a converged warp (the lowest active one)
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+    return pred != 0;
 }
 
 struct Ctx {
@@ -357,7 +365,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (even CTA)
-        if (lane == 0 && rank == 0) {
+        // the whole warp follows the waits; one elected lane issues the MMAs and commits
+        if (rank == 0) {
             const uint32_t tm = c.tmem;
             const uint64_t dq = sdesc(c.sbase + kOffQ, 16u, 1024u);
             const uint64_t dk = sdesc(c.sbase + kOffK, 16u, 1024u);
@@ -376,52 +385,69 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     if (!ok) break;
                     ptx::tc_fence_after();
                     const uint64_t dkh = dk + (uint64_t)(h * (kBoxBytes / 2) >> 4);
+                    if (elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
-                        ptx::mma_ss_2(tm + kColP + kColPHi * h, dq + koff, dkh + koff, kIdescQK, k > 0);
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
+                            ptx::mma_ss_2(tm + kColP + kColPHi * h, dq + koff, dkh + koff, kIdescQK, k > 0);
+                        }
+                        ptx::mma_commit_2_mc(&c.bars[P_FULL + h], 0x3);
                     }
-                    ptx::mma_commit_2_mc(&c.bars[P_FULL + h], 0x3);
+                    __syncwarp();
                 }
                 if (!ok) break;
-                ptx::mma_commit_2_mc(&c.bars[QK_DONE], 0x3);
+                if (elect_one()) ptx::mma_commit_2_mc(&c.bars[QK_DONE], 0x3);
+                __syncwarp();
                 // O = Qd S_{t-1}
                 ok = wait_pair(c, QD_READY, par) && wait_pair(c, S_READY, par) && wait_pair(c, O_FREE, fpar);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                if (elect_one()) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint64_t koff = (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4);
-                    ptx::mma_ts_2(tm + kColO, tm + kColQd + 8u * k, ds + koff, kIdescQS, k > 0);
+                    for (int k = 0; k < 8; ++k) {
+                        const uint64_t koff = (uint64_t)(((k >> 2) * 8192 + (k & 3) * 32) >> 4);
+                        ptx::mma_ts_2(tm + kColO, tm + kColQd + 8u * k, ds + koff, kIdescQS, k > 0);
+                    }
                 }
+                __syncwarp();
                 // S^T += V^T (K ⊙ d_k), onto e^{-s m} S^T prepared in TMEM
                 ok = wait_pair(c, VK_READY, par) && wait_pair(c, DS_FREE, par);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                if (elect_one()) {
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const uint64_t koff = (uint64_t)(k * (2048 >> 4));
-                    ptx::mma_ss_2(tm + kColDS, vdesc + koff, kddesc + koff, kIdescDS, 1);
+                    for (int k = 0; k < 16; ++k) {
+                        const uint64_t koff = (uint64_t)(k * (2048 >> 4));
+                        ptx::mma_ss_2(tm + kColDS, vdesc + koff, kddesc + koff, kIdescDS, 1);
+                    }
+                    // S_t is complete and S_{t-1} (the operand copy) is no longer read
+                    ptx::mma_commit_2_mc(&c.bars[DS_FULL], 0x3);
                 }
-                // S_t is complete and S_{t-1} (the operand copy) is no longer read
-                ptx::mma_commit_2_mc(&c.bars[DS_FULL], 0x3);
+                __syncwarp();
                 // O += P V, one key half at a time
 #pragma unroll 1
                 for (int h = 0; h < 2 && ok; ++h) {
                     ok = wait_pair(c, P_CONV + h, par);
                     if (!ok) break;
                     ptx::tc_fence_after();
+                    if (elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        ptx::mma_ts_2(tm + kColO, tm + kColPHi * h + 8u * k,
-                                      vdesc + (uint64_t)((8 * h + k) * (2048 >> 4)), kIdescPV, 1);
-                    ptx::mma_commit_2_mc(&c.bars[P_FREE + h], 0x3);
+                        for (int k = 0; k < 8; ++k)
+                            ptx::mma_ts_2(tm + kColO, tm + kColPHi * h + 8u * k,
+                                          vdesc + (uint64_t)((8 * h + k) * (2048 >> 4)), kIdescPV, 1);
+                        ptx::mma_commit_2_mc(&c.bars[P_FREE + h], 0x3);
+                    }
+                    __syncwarp();
                 }
                 if (!ok) break;
-                ptx::mma_commit_2_mc(&c.bars[O_FULL], 0x3);
-                ptx::mma_commit_2_mc(&c.bars[VK_EMPTY + (t & 1)], 0x3);
+                if (elect_one()) {
+                    ptx::mma_commit_2_mc(&c.bars[O_FULL], 0x3);
+                    ptx::mma_commit_2_mc(&c.bars[VK_EMPTY + (t & 1)], 0x3);
+                }
+                __syncwarp();
             }
-            ptx::mma_commit_2_mc(&c.bars[DRAIN], 0x1);
+            if (elect_one()) ptx::mma_commit_2_mc(&c.bars[DRAIN], 0x1);
+            __syncwarp();
             volatile int never = 0;
             ptx::mbar_wait(&c.bars[DRAIN], 0, &never);
         }
