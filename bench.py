@@ -80,7 +80,7 @@ def roofline(bound, achieved, peak, unit, traffic=None):
 KERNEL_SOURCES = {  # traffic.json key suffix -> the header that holds the kernel
     "pair": "prefill_pair.cuh", "tcgen05": "prefill_tc.cuh", "simt": "prefill_simt.cuh",
     "backward_pair": "prefill_pair.cuh", "decode": "decode.cuh", "norm_gate": "norm_gate.cuh",
-    "gqa_partial": "gqa_decode.cuh",
+    "gqa_partial": "gqa_decode.cuh", "gqp_attn": "gqa_prefill.cuh",
 }
 
 
@@ -607,6 +607,7 @@ def run_gqa_prefill_leg(dev, stream, args, world):
             "tokens_per_s": round(world * b * L / (ms / 1e3), 1),
             "tflops_causal": round(tf, 2),
             "roofline": roofline("tensor", tf, peaks["bf16_tflops"], "TFLOP/s"),
+            "dram_bytes_per_launch": measured_traffic("gqa_prefill_%d" % L, "gqp_attn"),
             "flops": "causal: 4 d per (query, key <= query) pair and query head; the step includes the RoPE launch"}
 
 
