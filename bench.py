@@ -80,7 +80,7 @@ def roofline(bound, achieved, peak, unit, traffic=None):
 KERNEL_SOURCES = {  # traffic.json key suffix -> the header that holds the kernel
     "pair": "prefill_pair.cuh", "tcgen05": "prefill_tc.cuh", "simt": "prefill_simt.cuh",
     "backward_pair": "prefill_pair.cuh", "decode": "decode.cuh", "norm_gate": "norm_gate.cuh",
-    "gqa_partial": "gqa_decode.cuh", "gqp_attn": "gqa_prefill.cuh",
+    "gqa_partial": "gqa_decode_tc.cuh", "gqp_attn": "gqa_prefill.cuh",
 }
 
 

@@ -285,7 +285,10 @@ la_status lightning_device_status(void *stream);
  *   workspace        lightning_gqa_decode_workspace_size(batch, heads, cap)
  *                    bytes, 16-byte aligned.
  * Device pointers, caller-owned, 16-byte aligned; the caches, o and the
- * workspace must not overlap any other buffer. CUDA cores, fp32 arithmetic.
+ * workspace must not overlap any other buffer. Three launches (cache append
+ * and query rotation, chunk partials, merge). bf16: the chunk partials on the
+ * tensor cores (tcgen05; the rotated queries and the weights rounded to bf16,
+ * fp32 softmax and accumulation); float32: CUDA cores, fp32 arithmetic.
  */
 la_status lightning_gqa_decode(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
                                la_dtype dtype, const int *pos, int batch, int heads, int kv_heads, int dim, int cap,

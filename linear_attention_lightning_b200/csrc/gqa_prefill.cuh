@@ -74,7 +74,7 @@ constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;  // + slack to align the b
 // registers per thread after the split: the control warpgroup gives its share to the two
 // softmax warpgroups. The launcher checks the kernel's allocation (threads x registers) holds
 // the split, since a setmaxnreg.inc beyond it would wait forever.
-constexpr int kCtrlRegs = 56, kSoftmaxRegs = 224;
+constexpr int kCtrlRegs = 80, kSoftmaxRegs = 200;
 constexpr int kSplitRegs = 4 * 32 * kCtrlRegs + 8 * 32 * kSoftmaxRegs;
 static_assert(kSplitRegs <= kThreads * ((65536 / kThreads) & ~7), "register split above the launch's");
 
@@ -156,6 +156,17 @@ gqp_rope_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__rest
 }
 
 // ---------------------------------------------------------------- attention
+
+// 32 lanes x 16 consecutive 32-bit columns
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
 
 // 32 lanes x 128 consecutive 32-bit columns (four x32 loads, one wait by the caller)
 __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
@@ -454,35 +465,40 @@ gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             const float mnew = fmaxf(m, max3(mx0, mx1, fmaxf(__uint_as_float(v[126]), __uint_as_float(v[127]))) * sl2);
             // raise the running max (warp-uniformly: the TMEM accesses are collective)
-            if (__any_sync(0xffffffffu, mnew > m + kRescaleMargin)) {
-                const float alpha = ptx::ex2(m - mnew);   // 0 on the first tile
+            const bool raise = __any_sync(0xffffffffu, mnew > m + kRescaleMargin);
+            float alpha = 1.f;
+            if (raise) {
+                alpha = ptx::ex2(m - mnew);   // 0 on the first tile
                 l *= alpha;
                 m = mnew;
-                if (j > 0) {
-#pragma unroll 1
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t a[32];
-                        ptx::tmem_ld32(trow + co_ + 32u * q, a);
-                        ptx::tmem_ld_wait();
-                        uint32_t b0[16], b1[16];
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) {
-                            b0[u] = __float_as_uint(__uint_as_float(a[u]) * alpha);
-                            b1[u] = __float_as_uint(__uint_as_float(a[16 + u]) * alpha);
-                        }
-                        ptx::tmem_st16(trow + co_ + 32u * q, b0);
-                        ptx::tmem_st16(trow + co_ + 32u * q + 16u, b1);
-                    }
-                }
             }
             // P = 2^(S sl2 - m) as bf16 pairs over the first 64 columns of S, in two halves of
             // 64 keys: the P V of the first half runs while the second is computed
-            l += p_half<0>(v, sl2, m, trow + cs_);
-            ptx::tmem_st_wait();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&c.bars[P_FULL + 2 * t]);
-            l += p_half<1>(v, sl2, m, trow + cs_);
+            if (!raise || j == 0) {
+                l += p_half<0>(v, sl2, m, trow + cs_);
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&c.bars[P_FULL + 2 * t]);
+                l += p_half<1>(v, sl2, m, trow + cs_);
+            } else {
+                // O is rescaled once the scores are no longer needed, before either half of P V
+                l += p_half<0>(v, sl2, m, trow + cs_);
+                l += p_half<1>(v, sl2, m, trow + cs_);
+#pragma unroll 1
+                for (int q = 0; q < 8; ++q) {
+                    uint32_t a[16];
+                    tmem_ld16(trow + co_ + 16u * q, a);
+                    ptx::tmem_ld_wait();
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) a[u] = __float_as_uint(__uint_as_float(a[u]) * alpha);
+                    ptx::tmem_st16(trow + co_ + 16u * q, a);
+                }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&c.bars[P_FULL + 2 * t]);
+            }
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
             __syncwarp();

@@ -15,6 +15,7 @@
 #include "prefill_simt.cuh"
 #include "gqa_decode.cuh"
 #include "gqa_prefill.cuh"
+#include "gqa_decode_tc.cuh"
 #include "norm_gate.cuh"
 #include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
@@ -256,8 +257,28 @@ la_status run_gqa_decode(const void *q, const void *k_new, const void *v_new, vo
         static_cast<T *>(k_cache), static_cast<T *>(v_cache), pos, heads, kv_heads, cap, rot, base, scale, qr);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "gqa append launch");
-    // the caches as 2-D tensors [batch*kv_heads*cap][dim], 128-byte swizzled boxes of one tile of positions
     const bool bf16 = sizeof(T) == 2;
+    if (bf16) {
+        // bf16 cache: the chunks' partial softmax on the tensor cores
+        CUtensorMap tk, tv;
+        const long long bkv = (long long)batch * kv_heads;
+        if (!la::gqp_make_map(&tk, k_cache, cap, cap, bkv, &g_last_error) ||
+            !la::gqp_make_map(&tv, v_cache, cap, cap, bkv, &g_last_error))
+            return LA_ERR_CUDA;
+        e = cudaFuncSetAttribute(la::gqd::gqd_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)la::gqd::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gqd_partial)");
+        la::gqd::gqd_partial_kernel<<<dim3(g.splits, kv_heads, batch), la::gqd::kThreads, la::gqd::kSmemBytes,
+                                      stream>>>(tk, tv, qr, pos, heads, kv_heads, cap, g.splits, pm, pl, po);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "gqd partial launch");
+        la::gqa_combine_kernel<T><<<(unsigned)((size_t)batch * heads), la::kGqaDim, 0, stream>>>(
+            pm, pl, po, g.splits, static_cast<T *>(o));
+        e = cudaGetLastError();
+        return e == cudaSuccess ? ok() : cuda_fail(e, "gqa combine launch");
+    }
+    // f32 cache: CUDA cores. The caches as 2-D tensors [batch*kv_heads*cap][dim], 128-byte
+    // swizzled boxes of one tile of positions
     const cuuint64_t rows = (cuuint64_t)batch * kv_heads * cap;
     CUtensorMap mk, mv;
     {
