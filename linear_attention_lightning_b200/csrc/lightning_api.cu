@@ -611,7 +611,7 @@ la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, c
     if (!(eps >= 0.f) || eps > 3.0e38f) return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
     if (dim != 64 && dim != 128) return fail(LA_ERR_UNSUPPORTED, "dim %d unsupported (64 or 128)", dim);
     const size_t eb = elem_bytes(dtype);
-    const long long max_ch = (long long)la::kNgThreads * la::kNgMaxChunks * (long long)(16 / eb);
+    const long long max_ch = (long long)la::kNgGroup * la::kNgMaxChunks * (long long)(16 / eb);
     if ((long long)heads * dim > max_ch)
         return fail(LA_ERR_UNSUPPORTED, "heads*dim %lld exceeds %lld channels per token",
                     (long long)heads * dim, max_ch);
@@ -628,17 +628,17 @@ la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, c
         overlaps(ry, range_of(gamma, sizeof(float) * heads * dim)))
         return fail(LA_ERR_INVALID_ARG, "y overlaps o, gate or gamma");
     // chunks of 16 bytes per thread, and resident CTAs on every SM, each walking the tokens
-    const long long chunks_per_thread = ((long long)heads * dim * (long long)eb / 16 + la::kNgThreads - 1) / la::kNgThreads;
-    const int U = chunks_per_thread <= 1 ? 1 : chunks_per_thread <= 2 ? 2 : 4;
+    const long long chunks_per_thread = ((long long)heads * dim * (long long)eb / 16 + la::kNgGroup - 1) / la::kNgGroup;
+    const int U = chunks_per_thread <= 1 ? 1 : chunks_per_thread <= 2 ? 2 : chunks_per_thread <= 4 ? 4 : 8;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const NgArgs args{o, gate, gamma, eps, batch, heads, seq, dim, per_head ? 1 : 0, y, tokens, st};
     la_status rs;
     if (dtype == LA_DTYPE_BF16)
         rs = U == 1 ? launch_norm_gate<__nv_bfloat16, 1>(args) : U == 2 ? launch_norm_gate<__nv_bfloat16, 2>(args)
-                    : launch_norm_gate<__nv_bfloat16, 4>(args);
+           : U == 4 ? launch_norm_gate<__nv_bfloat16, 4>(args) : launch_norm_gate<__nv_bfloat16, 8>(args);
     else
         rs = U == 1 ? launch_norm_gate<float, 1>(args) : U == 2 ? launch_norm_gate<float, 2>(args)
-                    : launch_norm_gate<float, 4>(args);
+           : U == 4 ? launch_norm_gate<float, 4>(args) : launch_norm_gate<float, 8>(args);
     return rs;
 }
 

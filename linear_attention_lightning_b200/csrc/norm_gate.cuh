@@ -11,10 +11,13 @@
 // tiles of `tile` consecutive tokens of one batch through a kNgStages-deep TMA
 // pipeline in shared memory: one 3-D box brings a tile's o for every head
 // (o is [batch*heads][seq][dim]), one more the tile's gate; two tiles stay in
-// flight while the sixteen warps work on the third. Each thread takes U 16-byte
-// chunks of a token's row; a head's chunks sit in dim/E consecutive lanes of
-// one warp (E values per chunk), so per-head sums are warp shuffles and
-// per-token sums one block reduction. y is written straight from registers
+// flight while the warps work on the third. The CTA's two groups of 256
+// threads take alternate tokens of a tile, each on its own named barrier, so
+// two tokens' reductions are in flight per SM. In a group each thread takes U
+// 16-byte chunks of a token's row; a head's chunks sit in dim/E consecutive
+// lanes of one warp (E values per chunk), so per-head sums are warp shuffles
+// and per-token sums one group reduction (one barrier a token: the partial
+// sums alternate between two buffers). y is written straight from registers
 // with streaming stores (a token's row is contiguous in y).
 #pragma once
 
@@ -26,7 +29,8 @@
 namespace la {
 
 constexpr int kNgThreads = 512;
-constexpr int kNgMaxChunks = 4;                 // heads*dim <= kNgThreads * kNgMaxChunks * (16 / sizeof(T))
+constexpr int kNgGroup = 256;                   // threads per token group (two groups per CTA)
+constexpr int kNgMaxChunks = 8;                 // heads*dim <= kNgGroup * kNgMaxChunks * (16 / sizeof(T))
 constexpr int kNgStages = 3;
 constexpr uint32_t kNgTileBytes = 32768;        // one tile of o (and one of gate) at most
 constexpr uint32_t kNgSmemBytes = kNgStages * 2 * kNgTileBytes + 64 + 128;
@@ -85,7 +89,9 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
     const int tiles_per_batch = (seq + tile - 1) / tile;
     const long long total = (long long)batch * tiles_per_batch;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    __shared__ float red[kNgThreads / 32];
+    const int grp = threadIdx.x / kNgGroup, gtid = threadIdx.x % kNgGroup, gwarp = gtid >> 5;
+    __shared__ float red[2][2][kNgGroup / 32];  // [group][buffer][warp]
+    int nred = 0;                                // this group's reductions so far (picks the buffer)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kNgStages; ++s) {
@@ -123,11 +129,11 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
         const int tcount = min(tile, seq - l0);
         const T *os = reinterpret_cast<const T *>(smem + s * 2 * kNgTileBytes);
         const T *gs = reinterpret_cast<const T *>(smem + s * 2 * kNgTileBytes + kNgTileBytes);
-        for (int t = 0; t < tcount; ++t) {
+        for (int t = grp; t < tcount; t += 2) {
             float x[U][8], ss[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int k = threadIdx.x + kNgThreads * u;
+                const int k = gtid + kNgGroup * u;
                 ss[u] = 0.f;
                 if (k < chunks) {
                     const int n0 = k * E, h = n0 / dim, c0 = n0 - h * dim;
@@ -146,19 +152,22 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
                 for (int u = 0; u < U; ++u) tsum += ss[u];
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, off);
-                if (lane == 0) red[warp] = tsum;
-                __syncthreads();
+                // buffers alternate over the group's tokens: a group's next write to one
+                // follows its next barrier, which every thread reaches only after reading it
+                float *rb = red[grp][nred & 1];
+                ++nred;
+                if (lane == 0) rb[gwarp] = tsum;
+                ptx::named_bar_sync(1 + grp, kNgGroup);
                 float all = 0.f;
 #pragma unroll
-                for (int w = 0; w < kNgThreads / 32; ++w) all += red[w];
-                __syncthreads();  // red[] is rewritten for the next token
+                for (int w = 0; w < kNgGroup / 32; ++w) all += rb[w];
 #pragma unroll
                 for (int u = 0; u < U; ++u) ss[u] = all;
             }
             T *yrow = y + ((long long)b * seq + l0 + t) * n_ch;
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int k = threadIdx.x + kNgThreads * u;
+                const int k = gtid + kNgGroup * u;
                 if (k < chunks) {
                     const int n0 = k * E;
                     const float inv = rsqrtf(ss[u] * inv_group + eps);
