@@ -261,6 +261,16 @@ la_status lightning_decode(const void *q, const void *k, const void *v, la_dtype
 la_status lightning_device_status(void *stream);
 
 /*
+ * Test hook for the failure-detection path (the pages have no counterpart):
+ * enqueues on `stream` one CTA whose bounded mbarrier wait, the one every
+ * kernel of the library uses, is never satisfied. The wait runs out, the
+ * kernel records LA_ERR_TIMEOUT in the device status word and returns; the
+ * context stays usable. Returns LA_OK once the kernel is enqueued (or
+ * LA_ERR_CUDA if the launch fails).
+ */
+la_status lightning_selftest_wait_timeout(void *stream);
+
+/*
  * One decode step of the softmax attention layer that M1 places after every
  * seven Lightning layers. Source: "MINIMAX SIGNAL LAB · M1", §02 (64 query
  * heads x 128; softmax K/V 8 x 128; RoPE on 64 of the 128 dims, in the

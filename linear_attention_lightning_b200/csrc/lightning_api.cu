@@ -16,6 +16,7 @@
 #include "gqa_decode.cuh"
 #include "gqa_prefill.cuh"
 #include "gqa_decode_tc.cuh"
+#include "selftest.cuh"
 #include "norm_gate.cuh"
 #include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
@@ -822,6 +823,12 @@ la_status lightning_device_status(void *stream) {
     if (word & la::kBadDeviceArgFlag)
         return fail(LA_ERR_INVALID_ARG, "a kernel met an out-of-range device-side argument (status word 0x%x)", word);
     return ok();
+}
+
+la_status lightning_selftest_wait_timeout(void *stream) {
+    la::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ok() : cuda_fail(e, "self-test launch");
 }
 
 const char *lightning_status_string(int status) {

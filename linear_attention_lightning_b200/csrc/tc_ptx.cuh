@@ -12,7 +12,7 @@
 namespace la {
 namespace ptx {
 
-constexpr uint32_t kWaitLimit = 1u << 22;     // a few seconds of polling at worst
+constexpr uint32_t kWaitLimit = 1u << 18;     // about a second of polling (a few us per suspended poll)
 constexpr unsigned int kTimeoutFlag = 4u;       // LA_ERR_TIMEOUT
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
