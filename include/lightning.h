@@ -162,7 +162,9 @@ la_status lightning_prefill_snapshots(const void *q, const void *k, const void *
  * backward in time on (K, Q, dO) and (V, dO, Q) with state R.
  * Kernels (variant): LA_VARIANT_TCGEN05_PAIR runs the passes on the CTA-pair
  * tensor-core kernel (bf16, dim 128, block 256; the backward-in-time passes
- * run it anti-causally, blocks from last to first);
+ * run it anti-causally, blocks from last to first; the three passes run side
+ * by side: dV and dK on two library-owned streams per device, forked from and
+ * joined back into `stream` with events, so the call keeps `stream`'s order);
  * LA_VARIANT_SIMT runs them on CUDA cores in fp32 (any dtype, dim 64 or 128,
  * any block, no workspace); LA_VARIANT_AUTO takes the tensor-core kernels
  * where they apply. LA_VARIANT_TCGEN05 is not a backward variant.

@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "../../include/lightning.h"
@@ -421,16 +422,66 @@ la_status check_backward_workspace(const BackwardArgs &a, size_t need) {
 // anti-causal (blocks from last to first, state anchored at each block's last
 // token) on (K, Q, dO) with carried state dS_out, whose final state is dS_in,
 // and on (V, dO, Q) with dS_out^T.
+// Two auxiliary streams per device, created on first use and kept for the process:
+// the backward passes run side by side on them.
+cudaError_t aux_streams(cudaStream_t (&out)[2]) {
+    static std::mutex mu;
+    static cudaStream_t streams[64][2] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < 2; ++i)
+        if (!streams[dev][i]) {
+            e = cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking);
+            if (e != cudaSuccess) return e;
+        }
+    out[0] = streams[dev][0];
+    out[1] = streams[dev][1];
+    return cudaSuccess;
+}
+
+// The three passes read the same inputs and write disjoint outputs, and each launch fills
+// only 2 SMs per (batch, head): dV and dK go to two auxiliary streams forked from and joined
+// back into `stream` with events, so that a pass's CTA pairs start on the SMs the others
+// leave free. Enqueue order on `stream` is kept (the fork waits for everything before it,
+// and everything after waits for the join), and the pattern can be captured into a graph.
 la_status run_backward_pair(const BackwardArgs &a, cudaStream_t stream) {
     const la::Snapshots none{nullptr, 0, 0};
-    la_status st = la::launch_pair(a.d_o, a.v, a.k, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.dq, nullptr,
-                                   none, la::pair::PairPass{1, 0}, stream, &g_last_error);
-    if (st != LA_OK) return st;
-    st = la::launch_pair(a.k, a.q, a.d_o, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dv, a.d_state_in,
-                         none, la::pair::PairPass{0, 1}, stream, &g_last_error);
-    if (st != LA_OK) return st;
-    return la::launch_pair(a.v, a.d_o, a.q, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dk, nullptr,
-                           none, la::pair::PairPass{1, 1}, stream, &g_last_error);
+    cudaStream_t aux[2];
+    cudaError_t e = aux_streams(aux);
+    if (e != cudaSuccess) return cuda_fail(e, "creating the backward's auxiliary streams");
+    cudaEvent_t fork, join[2];
+    e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+    for (int i = 0; i < 2; ++i)
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&join[i], cudaEventDisableTiming);
+    la_status st = LA_OK;
+    if (e != cudaSuccess) st = cuda_fail(e, "cudaEventCreate");
+    if (st == LA_OK) {
+        e = cudaEventRecord(fork, stream);
+        for (int i = 0; i < 2 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(aux[i], fork, 0);
+        if (e != cudaSuccess) st = cuda_fail(e, "forking the backward passes");
+    }
+    if (st == LA_OK)
+        st = la::launch_pair(a.k, a.q, a.d_o, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dv, a.d_state_in,
+                             none, la::pair::PairPass{0, 1}, aux[0], &g_last_error);
+    if (st == LA_OK)
+        st = la::launch_pair(a.v, a.d_o, a.q, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dk, nullptr,
+                             none, la::pair::PairPass{1, 1}, aux[1], &g_last_error);
+    if (st == LA_OK)
+        st = la::launch_pair(a.d_o, a.v, a.k, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.dq, nullptr, none,
+                             la::pair::PairPass{1, 0}, stream, &g_last_error);
+    // join even after a failed launch, so that `stream` never runs ahead of work already enqueued
+    for (int i = 0; i < 2; ++i) {
+        cudaError_t r = cudaEventRecord(join[i], aux[i]);
+        if (r == cudaSuccess) r = cudaStreamWaitEvent(stream, join[i], 0);
+        if (r != cudaSuccess && st == LA_OK) st = cuda_fail(r, "joining the backward passes");
+    }
+    cudaEventDestroy(fork);
+    for (int i = 0; i < 2; ++i) cudaEventDestroy(join[i]);
+    return st;
 }
 
 // The gradients as three passes of the block recurrence (see lightning.h):

@@ -88,7 +88,7 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
     const uint32_t box_bytes = (uint32_t)tile * n_ch * sizeof(T);
     const int tiles_per_batch = (seq + tile - 1) / tile;
     const long long total = (long long)batch * tiles_per_batch;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     const int grp = threadIdx.x / kNgGroup, gtid = threadIdx.x % kNgGroup, gwarp = gtid >> 5;
     __shared__ float red[2][2][kNgGroup / 32];  // [group][buffer][warp]
     int nred = 0;                                // this group's reductions so far (picks the buffer)
