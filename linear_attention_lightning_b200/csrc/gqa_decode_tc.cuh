@@ -201,7 +201,7 @@ gqd_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     } else if (warp == 4) {
         // ------------------------------------------------------------ softmax: lane g = head g
         const uint32_t trow = tmem;  // warp 4 reads TMEM lanes 0..31
-        float m = -INFINITY, l = 0.f;  // running max (log2 units), sum of the rounded weights
+        float m = -INFINITY, l = 0.f;  // running max (log2 units), sum of the weights
         bool done = nt > 0;
         for (int j = 0; j < nt; ++j) {
             if (!ptx::mbar_wait(&bars[S_FULL + (j & 1)], (uint32_t)(j >> 1) & 1u, abort)) { done = false; break; }
