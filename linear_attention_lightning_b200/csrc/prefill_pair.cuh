@@ -159,8 +159,20 @@ __device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parit
     const bool ok = leader ? wait_bar(c, idx, parity) : true;
     return ptx::named_bar_and(bar_id, 128, ok);
 }
+// two fp32 products in one instruction (each rounded as a plain multiply)
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
-    return ptx::pack_f16(ptx::bf16_lo(w) * scale, ptx::bf16_hi(w) * scale);
+    const float2 r = mul2(make_float2(ptx::bf16_lo(w), ptx::bf16_hi(w)), make_float2(scale, scale));
+    return ptx::pack_f16(r.x, r.y);
 }
 
 // fp32 P columns [col0, col0 + 128) of this thread's row -> fp16 P ⊙ D in
@@ -186,7 +198,13 @@ __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uin
                 if (jb >= i) {
                     const float wb = ptx::ex2(-sl2 * (float)(jb - i));
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[16 * g + u]) * tab[15 - u]) * wb;
+                    for (int u = 0; u < 16; u += 2) {
+                        const float2 t = mul2(make_float2(__uint_as_float(v[16 * g + u]), __uint_as_float(v[16 * g + u + 1])),
+                                              make_float2(tab[15 - u], tab[14 - u]));
+                        const float2 r2 = mul2(t, make_float2(wb, wb));
+                        p[u] = r2.x;
+                        p[u + 1] = r2.y;
+                    }
                 } else if (jb + 15 < i) {
 #pragma unroll
                     for (int u = 0; u < 16; ++u) p[u] = 0.f;
@@ -204,7 +222,13 @@ __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uin
             } else if (dlast >= 0) {
                 const float wb = ptx::ex2(-sl2 * (float)dlast);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[16 * g + u]) * tab[u]) * wb;
+                for (int u = 0; u < 16; u += 2) {
+                    const float2 t = mul2(make_float2(__uint_as_float(v[16 * g + u]), __uint_as_float(v[16 * g + u + 1])),
+                                          make_float2(tab[u], tab[u + 1]));
+                    const float2 r2 = mul2(t, make_float2(wb, wb));
+                    p[u] = r2.x;
+                    p[u + 1] = r2.y;
+                }
             } else if (i < jb) {
 #pragma unroll
                 for (int u = 0; u < 16; ++u) p[u] = 0.f;
@@ -583,9 +607,13 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             } else {
                 uint32_t lo[16], hi[16];
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    lo[q] = __float_as_uint(sv[q] * dnext);
-                    hi[q] = __float_as_uint(sv[16 + q] * dnext);
+                for (int q = 0; q < 16; q += 2) {
+                    const float2 a = mul2(make_float2(sv[q], sv[q + 1]), make_float2(dnext, dnext));
+                    const float2 bb = mul2(make_float2(sv[16 + q], sv[17 + q]), make_float2(dnext, dnext));
+                    lo[q] = __float_as_uint(a.x);
+                    lo[q + 1] = __float_as_uint(a.y);
+                    hi[q] = __float_as_uint(bb.x);
+                    hi[q + 1] = __float_as_uint(bb.y);
                 }
                 __syncwarp();
                 ptx::tmem_st16(trow + kColDS + 32 * hh, lo);
