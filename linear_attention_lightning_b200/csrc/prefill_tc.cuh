@@ -101,14 +101,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-// K-major operand (rows of 128 dims = two 64-dim boxes): k-step k of 16 dims
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int k) {
-    return sdesc(tile + (uint32_t)(k >> 2) * kBoxBytes + (uint32_t)(k & 3) * 32u, 16u, 1024u);
-}
-// MN-major operand (rows = the K dimension, 128 B per row): k-step of 16 rows
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int k) {
-    return sdesc(tile + (uint32_t)k * 2048u, kBoxBytes, 1024u);
-}
 
 // Rotation of the five Q/K sub-tile slots between blocks. Slots are reused in
 // the order they are released: Q slots free early (after their P tiles are
