@@ -110,3 +110,39 @@ def test_m1_prefill_8k_backward_sampled_heads(variant):
     torch.cuda.synchronize()
     heads = [0, 40, 63]
     _check([t[:, heads] for t in got], _oracle_backward(inp, heads_idx=heads), w.dtype)
+
+
+def test_backward_captures_into_a_cuda_graph():
+    # the tensor-core passes fork onto the library's side streams and join back with events;
+    # captured into a graph and replayed, they give the same gradients as the direct call
+    import linear_attention_lightning_b200 as la
+    torch.manual_seed(0)
+    b, h, L, d, block = 1, 4, 700, 128, 256
+    dev = torch.device("cuda")
+    mk = lambda: (torch.randn(b, h, L, d, device=dev) / d ** 0.5).to(torch.bfloat16)
+    q, k, v, d_o = mk(), mk(), mk(), mk()
+    sl = torch.rand(h, device=dev) * 0.05 + 0.001
+    s0 = torch.randn(b, h, d, d, device=dev) * 0.1
+    dso = torch.randn(b, h, d, d, device=dev) * 0.1
+    ref = la.prefill_backward(q, k, v, d_o, sl, block, s0, dso)
+    torch.cuda.synchronize()
+    outs = [torch.empty_like(q) for _ in range(3)] + [torch.empty_like(dso)]
+    from linear_attention_lightning_b200 import abi
+    need = abi.lightning_prefill_backward_workspace_size(abi.LA_DTYPE_BF16, b, h, L, d, block, abi.LA_VARIANT_AUTO)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            abi.check(abi.lightning_prefill_backward(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), d_o.data_ptr(), abi.LA_DTYPE_BF16, sl.data_ptr(), b, h, L,
+                d, block, s0.data_ptr(), dso.data_ptr(), outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(),
+                outs[3].data_ptr(), ws.data_ptr(), need, side.cuda_stream, abi.LA_VARIANT_AUTO))
+    for x in outs:
+        x.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    for got, want in zip(outs, ref):
+        assert torch.equal(got, want)
+    assert abi.lightning_device_status(torch.cuda.current_stream().cuda_stream) == abi.LA_OK
