@@ -680,7 +680,10 @@ def run_backward_leg(w, dev, stream, inp, dcode, args, world):
 
 def run_e2e(w, dev, stream, inp, variant, args, world):
     """Same prefill through the public API with host buffers: every step copies
-    q, k, v from pinned host memory and reads o and the state back."""
+    q, k, v from pinned host memory and reads o and the state back. Steps are
+    pipelined over two device buffer sets: step i's inputs copy in on one
+    stream while step i-1 computes and its outputs copy out on another (the
+    two PCIe directions have their own copy engines)."""
     import torch
     import linear_attention_lightning_b200 as la
     steps = args.e2e_steps
@@ -689,31 +692,64 @@ def run_e2e(w, dev, stream, inp, variant, args, world):
     hv = inp["v"].cpu().pin_memory()
     ho = torch.empty_like(hq).pin_memory()
     hs = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32).pin_memory()
-    dq, dk, dv = (torch.empty_like(inp["q"]) for _ in range(3))
+    sets = [[torch.empty_like(inp["q"]) for _ in range(3)] for _ in range(2)]
+    outs = [(torch.empty_like(inp["q"]), torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32,
+                                                      device=dev)) for _ in range(2)]
     h2d = 3 * hq.numel() * hq.element_size()
     d2h = ho.numel() * ho.element_size() + hs.numel() * 4
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event()
 
-    def one():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        o, s = la.prefill(dq, dk, dv, inp["slopes"], w.block, inp["state_in"], variant=variant)
-        ho.copy_(o, non_blocking=True)
-        hs.copy_(s, non_blocking=True)
+    def run(n):
+        copied = [None, None]  # per buffer set: inputs landed
+        computed = [None, None]  # per buffer set: compute done (inputs free, outputs ready)
+        read = [None, None]      # per buffer set: outputs copied out
+        for i in range(n):
+            b = i % 2
+            dq, dk, dv = sets[b]
+            o, s_ = outs[b]
+            with torch.cuda.stream(s_in):
+                if computed[b] is not None:
+                    s_in.wait_event(computed[b])   # the compute two steps back read this set
+                dq.copy_(hq, non_blocking=True)
+                dk.copy_(hk, non_blocking=True)
+                dv.copy_(hv, non_blocking=True)
+                copied[b] = ev()
+                copied[b].record(s_in)
+            stream.wait_event(copied[b])
+            if read[b] is not None:
+                stream.wait_event(read[b])         # its outputs from two steps back were read
+            la.prefill(dq, dk, dv, inp["slopes"], w.block, inp["state_in"], variant=variant, o=o, state_out=s_,
+                       stream=stream)
+            computed[b] = ev()
+            computed[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[b])
+                ho.copy_(o, non_blocking=True)
+                hs.copy_(s_, non_blocking=True)
+                read[b] = ev()
+                read[b].record(s_out)
+        stream.wait_stream(s_out)
+        stream.wait_stream(s_in)
 
-    one()
+    run(1)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     e0.record(stream)
-    for _ in range(steps):
-        one()
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    run(steps)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     value = world * w.batch * w.seq * steps / (ms / 1e3)
+    # the last step's host output is the device prefill's on the same inputs
+    ref_o, _ = la.prefill(inp["q"], inp["k"], inp["v"], inp["slopes"], w.block, inp["state_in"], variant=variant)
+    same = bool(torch.equal(ho, ref_o.cpu()))
     return {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps}
+            "d2h_bytes_per_step": d2h, "steps": steps, "output_matches_device_call": same,
+            "pipeline": "two buffer sets; inputs in on one stream, outputs out on another"}
 
 
 def parse_args(argv=None):
@@ -724,7 +760,7 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=PREFILL_WORKLOAD)
     p.add_argument("--decode-steps", type=int, default=1000)
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--gqa-steps", type=int, default=20,
                    help="timed steps of the softmax GQA decode leg (0 skips it)")
