@@ -179,9 +179,19 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
                         const float4 g4 = __ldg(reinterpret_cast<const float4 *>(gamma + n0 + e));
                         gm[e] = g4.x; gm[e + 1] = g4.y; gm[e + 2] = g4.z; gm[e + 3] = g4.w;
                     }
-                    // sigmoid with the fast divide: a few ulp, far inside the output's rounding
+                    if (sizeof(T) == 2) {
+                        // bf16: sigmoid(g) = 1/2 + tanh(g/2)/2 with the SFU's tanh (one SFU op)
 #pragma unroll
-                    for (int e = 0; e < E; ++e) out[e] = __fdividef(gm[e] * x[u][e] * inv, 1.f + __expf(-gv[e]));
+                        for (int e = 0; e < E; ++e) {
+                            float th;
+                            asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(0.5f * gv[e]));
+                            out[e] = gm[e] * x[u][e] * inv * fmaf(0.5f, th, 0.5f);
+                        }
+                    } else {
+                        // sigmoid with the fast divide: a few ulp, far inside the output's rounding
+#pragma unroll
+                        for (int e = 0; e < E; ++e) out[e] = __fdividef(gm[e] * x[u][e] * inv, 1.f + __expf(-gv[e]));
+                    }
                     __stcs(reinterpret_cast<uint4 *>(yrow + n0), V::pack(out));
                 }
             }
