@@ -77,3 +77,25 @@ def test_gqa_decode_rejects_an_out_of_range_position_on_the_device():
     assert torch.equal(kc[0], kc0[0]) and torch.equal(vc[0], vc0[0])  # nothing written for it
     assert torch.count_nonzero(o[0]) == 0
     assert abi.lightning_device_status(stream) == abi.LA_OK          # the word was cleared
+
+
+def test_gqa_decode_never_lets_cache_rows_past_pos_into_the_result():
+    # rows past pos[b] hold NaN: masked weights are 0, and 0 x NaN would still be NaN, so the
+    # kernel must keep those rows out of every sum (the tensor-core path zeroes them in shared
+    # memory before P V)
+    b, h, hk, cap = 3, 16, 2, 2500
+    positions = [300, 2047, 2100]          # inside the first chunk, its last slot, the second chunk
+    q, kn, vn, kc, vc = _inputs(b, h, hk, cap, torch.bfloat16, 83)
+    for bb, p in enumerate(positions):
+        kc[bb, :, p + 1:] = float("nan")
+        vc[bb, :, p + 1:] = float("nan")
+    kc0, vc0 = kc.clone(), vc.clone()
+    conv = inputs.to_oracle
+    ref = oracle.gqa_decode(conv(q), conv(kn), conv(vn), conv(kc0), conv(vc0), np.array(positions, np.int32), 64,
+                            10000.0, 1.0 / np.sqrt(128.0))
+    o = la.gqa_decode(q, kn, vn, kc, vc, torch.tensor(positions, dtype=torch.int32, device=DEV))
+    torch.cuda.synchronize()
+    got = to_f64(o)
+    assert np.all(np.isfinite(got))
+    e = rel_err(got, ref, bf16_out=1)
+    assert e <= TOL[torch.bfloat16], e
