@@ -379,6 +379,10 @@ def run_ours(args):
     # prefill of the softmax GQA layer at the same context length
     gqp = run_gqa_prefill_leg(dev, stream, args, world) if args.gqa_prefill_steps > 0 else None
 
+    # one block of the hybrid model's attention: 7 Lightning layers and 1 softmax layer
+    hyb = (run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world)
+           if args.hybrid_steps > 0 and w.dtype == torch.bfloat16 and w.dim == 128 else None)
+
     # gradients of the same prefill (dq, dk, dv, d state_in)
     bwd = run_backward_leg(w, dev, stream, inp, dcode, args, world) if args.backward_steps > 0 else None
 
@@ -403,6 +407,7 @@ def run_ours(args):
         "norm_gate": ng,
         "gqa_decode": gqa,
         "gqa_prefill": gqp,
+        "hybrid_block": hyb,
         "backward": bwd,
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
@@ -619,6 +624,68 @@ def run_gqa_prefill_leg(dev, stream, args, world):
             "flops": "causal: 4 d per (query, key <= query) pair and query head; the step includes the RoPE launch"}
 
 
+def run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world):
+    """One block of the hybrid model's attention at the workload's shape: seven
+    Lightning layers (prefill, then normalisation and gating of its output) and
+    one softmax GQA layer (64 query heads over 8 KV heads, RoPE on 64 dims) on
+    the same tokens, through the library's entry points; timed like the main
+    leg. The layers reuse one set of inputs (timing only)."""
+    import torch
+    from linear_attention_lightning_b200 import abi
+    q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
+    b, L, d = w.batch, w.seq, w.dim
+    o = torch.empty_like(q)
+    s_out = torch.empty((b, w.heads, d, d), dtype=torch.float32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(w.seed + 4000)
+    gate = torch.randn((b, L, w.heads * d), generator=g, device=dev).to(q.dtype)
+    gamma = torch.ones(w.heads * d, device=dev)
+    y = torch.empty((b, L, w.heads * d), dtype=q.dtype, device=dev)
+    hq, hk = GQA_HEADS, GQA_KV_HEADS
+    kn = torch.randn((b, hk, L, d), generator=g, device=dev).to(q.dtype)
+    vn = torch.randn((b, hk, L, d), generator=g, device=dev).to(q.dtype)
+    kc, vc = torch.empty_like(kn), torch.empty_like(vn)
+    og = torch.empty((b, hq, L, d), dtype=q.dtype, device=dev)
+    need = abi.lightning_gqa_prefill_workspace_size(b, hq, L, d)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    sp = stream.cuda_stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+
+    def step(mark=False):
+        if mark:
+            ev[0].record(stream)
+        for _ in range(7):
+            abi.check(abi.lightning_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), b,
+                                               w.heads, L, d, w.block, None if s0 is None else s0.data_ptr(),
+                                               o.data_ptr(), s_out.data_ptr(), None, 0, sp, vcode))
+            abi.check(abi.lightning_norm_gate(o.data_ptr(), gate.data_ptr(), dcode, gamma.data_ptr(), 1e-6, b,
+                                              w.heads, L, d, 0, y.data_ptr(), sp))
+        if mark:
+            ev[1].record(stream)
+        abi.check(abi.lightning_gqa_prefill(q.data_ptr(), kn.data_ptr(), vn.data_ptr(), kc.data_ptr(), vc.data_ptr(),
+                                            dcode, 0, b, hq, hk, L, d, L, 64, 1e4, 1.0 / d ** 0.5, og.data_ptr(),
+                                            ws.data_ptr(), need, sp))
+        if mark:
+            ev[2].record(stream)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    steps = args.hybrid_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        step(mark=(i == steps - 1))
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    lightning_ms, softmax_ms = ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])
+    return {"layers": "7 x (Lightning prefill + norm and gate) + 1 x softmax GQA prefill", "steps": steps,
+            "ms_per_step": round(ms, 3), "tokens_per_s": round(world * b * L / (ms / 1e3), 1),
+            "lightning_ms": round(lightning_ms, 3), "softmax_ms": round(softmax_ms, 3),
+            "softmax_share": round(softmax_ms / (lightning_ms + softmax_ms), 4)}
+
+
 def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     """lightning_prefill_backward on the workload (AUTO: the CTA-pair tensor-core
     kernel where it applies), timed like the main leg: dQ causal on (dO, V, K),
@@ -770,6 +837,8 @@ def parse_args(argv=None):
                    help="timed steps of the softmax GQA prefill leg (0 skips it)")
     p.add_argument("--gqa-prefill-seq", type=int, default=131072,
                    help="new tokens of the GQA prefill leg")
+    p.add_argument("--hybrid-steps", type=int, default=2,
+                   help="timed steps of the hybrid-block leg, 7 Lightning + 1 softmax layer (0 skips it)")
     p.add_argument("--norm-gate-steps", type=int, default=20,
                    help="timed steps of the norm-and-gate epilogue leg (0 skips it)")
     p.add_argument("--backward-steps", type=int, default=10,
