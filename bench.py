@@ -383,6 +383,8 @@ def run_ours(args):
     hyb = (run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world)
            if args.hybrid_steps > 0 and w.dtype == torch.bfloat16 and w.dim == 128 else None)
 
+    hyd = run_hybrid_decode_leg(dev, stream, args, world) if args.hybrid_steps > 0 and args.gqa_steps > 0 else None
+
     # gradients of the same prefill (dq, dk, dv, d state_in)
     bwd = run_backward_leg(w, dev, stream, inp, dcode, args, world) if args.backward_steps > 0 else None
 
@@ -408,6 +410,7 @@ def run_ours(args):
         "gqa_decode": gqa,
         "gqa_prefill": gqp,
         "hybrid_block": hyb,
+        "hybrid_decode": hyd,
         "backward": bwd,
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
@@ -684,6 +687,52 @@ def run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world):
             "ms_per_step": round(ms, 3), "tokens_per_s": round(world * b * L / (ms / 1e3), 1),
             "lightning_ms": round(lightning_ms, 3), "softmax_ms": round(softmax_ms, 3),
             "softmax_share": round(softmax_ms / (lightning_ms + softmax_ms), 4)}
+
+
+def run_hybrid_decode_leg(dev, stream, args, world):
+    """One decode step of the hybrid block for GQA_BATCH sequences at a context of
+    args.gqa_context tokens: seven Lightning decode steps (64 heads x 128, fp32
+    states) and one softmax GQA decode step (64 query heads over 8 KV heads,
+    bf16 cache), through the library's entry points."""
+    import torch
+    from linear_attention_lightning_b200 import abi, inputs
+    b, h, hk, cap, d = GQA_BATCH, GQA_HEADS, GQA_KV_HEADS, args.gqa_context, 128
+    g = torch.Generator(device=dev).manual_seed(3200)
+    mk = lambda *shape: torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+    states = [torch.randn((b, h, d, d), generator=g, device=dev) * 0.1 for _ in range(7)]
+    sl = inputs.slopes(h, device=dev)
+    ql, kl, vl = mk(b, h, d), mk(b, h, d), mk(b, h, d)
+    ol = torch.empty_like(ql)
+    q, kn, vn = mk(b, h, d), mk(b, hk, d), mk(b, hk, d)
+    kc, vc = mk(b, hk, cap, d), mk(b, hk, cap, d)
+    pos = torch.full((b,), cap - 1, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    need = abi.lightning_gqa_decode_workspace_size(b, h, cap)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    sp = stream.cuda_stream
+
+    def step():
+        for st in states:
+            abi.check(abi.lightning_decode(ql.data_ptr(), kl.data_ptr(), vl.data_ptr(), abi.LA_DTYPE_BF16, sl.data_ptr(),
+                                           b, h, d, st.data_ptr(), ol.data_ptr(), sp))
+        abi.check(abi.lightning_gqa_decode(q.data_ptr(), kn.data_ptr(), vn.data_ptr(), kc.data_ptr(), vc.data_ptr(),
+                                           abi.LA_DTYPE_BF16, pos.data_ptr(), b, h, hk, d, cap, 64, 1e4,
+                                           1.0 / d ** 0.5, o.data_ptr(), ws.data_ptr(), need, sp))
+
+    for _ in range(args.warmup):
+        step()
+    steps = args.gqa_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    return {"layers": "7 x Lightning decode + 1 x softmax GQA decode", "sequences": b, "context": cap,
+            "steps": steps, "us_per_step": round(ms * 1e3, 2), "tokens_per_s": round(world * b / (ms / 1e3), 1)}
 
 
 def run_backward_leg(w, dev, stream, inp, dcode, args, world):
