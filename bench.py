@@ -242,7 +242,7 @@ def oracle_sample(w, tokens, heads, threads=None, h0=0):
     return time.perf_counter() - t0, tokens * heads
 
 
-def cpu_baseline(w, budget_s=15.0):
+def cpu_baseline(w, budget_s=25.0):
     """The oracle on a bounded sample of the workload, sized to about budget_s
     of CPU work: groups of up to one head per core (inputs and the float64
     output of a whole head group stay a few GB), each up to the full sequence."""
