@@ -594,7 +594,7 @@ def run_gqa_prefill_leg(dev, stream, args, world):
     kc = torch.empty((b, hk, L, d), dtype=torch.bfloat16, device=dev)
     vc = torch.empty_like(kc)
     o = torch.empty_like(q)
-    need = abi.lightning_gqa_prefill_workspace_size(b, h, L, d)
+    need = abi.lightning_gqa_prefill_workspace_size(abi.LA_DTYPE_BF16, b, h, L, d)
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
     sp = stream.cuda_stream
 
@@ -648,7 +648,7 @@ def run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world):
     vn = torch.randn((b, hk, L, d), generator=g, device=dev).to(q.dtype)
     kc, vc = torch.empty_like(kn), torch.empty_like(vn)
     og = torch.empty((b, hq, L, d), dtype=q.dtype, device=dev)
-    need = abi.lightning_gqa_prefill_workspace_size(b, hq, L, d)
+    need = abi.lightning_gqa_prefill_workspace_size(dcode, b, hq, L, d)
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
     sp = stream.cuda_stream
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]

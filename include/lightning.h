@@ -319,21 +319,22 @@ size_t lightning_gqa_decode_workspace_size(int batch, int heads, int cap);
  *   o[b][h][i] = sum_{p <= start+i} softmax_p(scale * rope(q[b][h][i], start+i) . k_p) v_p,
  * k_p, v_p the cache rows (positions < start as given, the rest as written).
  *
- *   q                [batch][heads][seq][dim], bf16.
- *   k_new, v_new     [batch][kv_heads][seq][dim], bf16.
- *   k_cache, v_cache [batch][kv_heads][cap][dim], bf16; positions < start
+ *   q                [batch][heads][seq][dim], dtype.
+ *   k_new, v_new     [batch][kv_heads][seq][dim], dtype.
+ *   k_cache, v_cache [batch][kv_heads][cap][dim], dtype; positions < start
  *                    read, positions start .. start+seq-1 written, the rest
  *                    neither read nor written. start + seq <= cap.
- *   dtype            LA_DTYPE_BF16 (LA_DTYPE_F32 is LA_ERR_UNSUPPORTED).
+ *   dtype            LA_DTYPE_BF16 (tensor cores) or LA_DTYPE_F32 (CUDA cores).
  *   dim 128; rot a multiple of 4, 0 <= rot <= dim; scale finite and > 0;
  *   batch <= 65535.
- *   o                [batch][heads][seq][dim], bf16; written.
- *   workspace        lightning_gqa_prefill_workspace_size(batch, heads, seq,
- *                    dim) bytes (the rotated queries), 16-byte aligned.
+ *   o                [batch][heads][seq][dim], dtype; written.
+ *   workspace        lightning_gqa_prefill_workspace_size(dtype, batch, heads,
+ *                    seq, dim) bytes (the rotated queries), 16-byte aligned.
  * Device pointers, caller-owned, 16-byte aligned; the caches, o and the
  * workspace must not overlap any other buffer. seq == 0 or batch == 0 launches
- * nothing. Two launches: the rotation, then the attention on the tensor cores
- * (tcgen05; bf16 operands, fp32 accumulation and softmax, P rounded to bf16).
+ * nothing. Two launches: the rotation, then the attention: bf16 on the tensor
+ * cores (tcgen05; bf16 operands, fp32 accumulation and softmax, P rounded to
+ * bf16); float32 on CUDA cores (fp32 throughout, exact online softmax).
  */
 la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
                                 la_dtype dtype, int start, int batch, int heads, int kv_heads, int seq, int dim,
@@ -341,7 +342,7 @@ la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_
                                 size_t workspace_bytes, void *stream);
 
 /* Workspace bytes of lightning_gqa_prefill (0 for an invalid request). Host only. */
-size_t lightning_gqa_prefill_workspace_size(int batch, int heads, int seq, int dim);
+size_t lightning_gqa_prefill_workspace_size(la_dtype dtype, int batch, int heads, int seq, int dim);
 
 /* Static description of a status code. */
 const char *lightning_status_string(int status);

@@ -36,7 +36,7 @@ _SIGNATURES = {
     "lightning_gqa_decode_workspace_size": ([_i, _i, _i], _sz),
     "lightning_gqa_prefill": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.c_double,
                                ctypes.c_float, _vp, _vp, _sz, _vp], _i),
-    "lightning_gqa_prefill_workspace_size": ([_i, _i, _i, _i], _sz),
+    "lightning_gqa_prefill_workspace_size": ([_i, _i, _i, _i, _i], _sz),
     "lightning_prefill_backward": ([_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _sz, _vp, _i], _i),
     "lightning_prefill_backward_workspace_size": ([_i, _i, _i, _i, _i, _i, _i], _sz),
@@ -168,8 +168,8 @@ def lightning_gqa_prefill(q, k_new, v_new, k_cache, v_cache, dtype, start, batch
                                         dim, cap, rot, rope_base, scale, o, workspace, workspace_bytes, stream)
 
 
-def lightning_gqa_prefill_workspace_size(batch, heads, seq, dim):
-    return load().lightning_gqa_prefill_workspace_size(batch, heads, seq, dim)
+def lightning_gqa_prefill_workspace_size(dtype, batch, heads, seq, dim):
+    return load().lightning_gqa_prefill_workspace_size(dtype, batch, heads, seq, dim)
 
 
 def lightning_prefill_snapshot_count(seq, interval):

@@ -201,10 +201,10 @@ def gqa_prefill(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """lightning_gqa_prefill: the softmax GQA layer over seq new tokens at
     positions start .. start+seq-1. Writes their rotated keys and values into
-    the caches and returns o [batch, heads, seq, dim]. bf16 only; scale
-    defaults to 1/sqrt(dim)."""
-    if q.dtype != torch.bfloat16:
-        raise ValueError("q must be bfloat16")
+    the caches and returns o [batch, heads, seq, dim]. bf16 (tensor cores) or
+    float32 (CUDA cores); scale defaults to 1/sqrt(dim)."""
+    if q.dtype not in _DTYPES:
+        raise ValueError("q must be float32 or bfloat16")
     b, h, L, d = q.shape
     bk, hk, cap, dk = k_cache.shape
     if (bk, dk) != (b, d) or tuple(k_new.shape) != (b, hk, L, d) or tuple(v_new.shape) != (b, hk, L, d) \
@@ -217,7 +217,7 @@ def gqa_prefill(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
         scale = 1.0 / float(d) ** 0.5
     if o is None:
         o = torch.empty_like(q)
-    need = abi.lightning_gqa_prefill_workspace_size(b, h, L, d)
+    need = abi.lightning_gqa_prefill_workspace_size(_DTYPES[q.dtype], b, h, L, d)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     abi.check(abi.lightning_gqa_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),

@@ -619,3 +619,167 @@ inline la_status launch_gqa_prefill(const void *q, const void *k_new, const void
 }
 
 }  // namespace la
+
+// ------------------------------------------------------------------ float32 path (CUDA cores)
+namespace la {
+namespace gqs {
+
+constexpr int kThreads = 128;
+constexpr int kQRows = 16;   // query rows per CTA (8 threads per row)
+constexpr int kKeys = 64;    // keys per tile
+constexpr int kDim = 128;
+constexpr int kKPitch = kDim + 1;  // padded key rows: the 8 threads of a row read 8 different banks
+constexpr uint32_t kSmemBytes = (kQRows * kDim + kKeys * kKPitch + kKeys * kDim + kQRows * kKeys) * 4;
+
+// grid (seq, batch), 256 threads: q_rot = rope(q), cache rows start+i <- rope(k_new), v_new.
+// float32 throughout; angles in double.
+__global__ void __launch_bounds__(256)
+gqs_rope_kernel(const float *__restrict__ q, const float *__restrict__ k_new, const float *__restrict__ v_new,
+                float *__restrict__ k_cache, float *__restrict__ v_cache, float *__restrict__ q_rot, int heads,
+                int kv_heads, int seq, int start, int cap, int rot, double base) {
+    __shared__ float cs[kDim / 2], sn[kDim / 2];
+    const int i = blockIdx.x, b = blockIdx.y, pos = start + i, half = rot / 2;
+    for (int c = threadIdx.x; c < half; c += blockDim.x) {
+        double s, co;
+        sincos((double)pos * pow(base, -2.0 * c / (double)rot), &s, &co);
+        cs[c] = (float)co;
+        sn[c] = (float)s;
+    }
+    __syncthreads();
+    const int rows = heads + 2 * kv_heads;
+    for (int u = threadIdx.x; u < rows * kDim; u += blockDim.x) {
+        const int hr = u / kDim, c = u - hr * kDim;
+        const float *src;
+        float *dst;
+        if (hr < heads) {
+            const size_t row = ((size_t)b * heads + hr) * seq + i;
+            src = q + row * kDim;
+            dst = q_rot + row * kDim;
+        } else if (hr < heads + kv_heads) {
+            const size_t g = (size_t)b * kv_heads + (hr - heads);
+            src = k_new + (g * seq + i) * kDim;
+            dst = k_cache + (g * cap + pos) * kDim;
+        } else {
+            const size_t g = (size_t)b * kv_heads + (hr - heads - kv_heads);
+            v_cache[(g * cap + pos) * kDim + c] = v_new[(g * seq + i) * kDim + c];
+            continue;
+        }
+        if (c >= rot) {
+            dst[c] = src[c];
+        } else if (c < half) {
+            dst[c] = fmaf(-src[c + half], sn[c], src[c] * cs[c]);
+        } else {
+            dst[c] = fmaf(src[c - half], sn[c - half], src[c] * cs[c - half]);
+        }
+    }
+}
+
+// grid (ceil(seq / 16), heads, batch), 128 threads; dynamic shared memory kSmemBytes.
+// Thread t takes row r = t / 8 of the CTA's 16 query rows: scores for keys t%8, t%8 + 8, ...
+// of each 64-key tile, then output dims 16 (t%8) .. 16 (t%8) + 15. Exact online softmax in
+// fp32 (the running max is raised on every increase); keys past start+seq are never read.
+__global__ void __launch_bounds__(kThreads)
+gqs_attn_kernel(const float *__restrict__ q_rot, const float *__restrict__ k_cache, const float *__restrict__ v_cache,
+                float *__restrict__ o, int heads, int kv_heads, int seq, int start, int cap, float scale) {
+    extern __shared__ float sm[];
+    float *qs = sm, *ks = qs + kQRows * kDim, *vs = ks + kKeys * kKPitch, *ps = vs + kKeys * kDim;
+    const int i0 = blockIdx.x * kQRows, h = blockIdx.y, b = blockIdx.z;
+    const int group = heads / kv_heads;
+    const size_t bh = (size_t)b * heads + h, kv = (size_t)b * kv_heads + h / group;
+    const int t = threadIdx.x, r = t >> 3, j8 = t & 7;
+    const int qpos = start + i0 + r;                       // this row's position
+    const int kend = min(start + i0 + kQRows, start + seq);  // keys 0 .. kend-1 are needed
+    for (int e = t; e < kQRows * kDim; e += kThreads) {
+        const int rr = e / kDim;
+        qs[e] = i0 + rr < seq ? q_rot[(bh * seq + i0 + rr) * kDim + e % kDim] : 0.f;
+    }
+    float m = -INFINITY, l = 0.f, acc[16];
+#pragma unroll
+    for (int d = 0; d < 16; ++d) acc[d] = 0.f;
+    for (int k0 = 0; k0 < kend; k0 += kKeys) {
+        __syncthreads();  // the previous tile's keys, values and weights are no longer read
+        for (int e = t; e < kKeys * kDim; e += kThreads) {
+            const int kk = e / kDim, c = e % kDim;
+            const bool live = k0 + kk < kend;
+            ks[kk * kKPitch + c] = live ? k_cache[(kv * cap + k0 + kk) * kDim + c] : 0.f;
+            vs[kk * kDim + c] = live ? v_cache[(kv * cap + k0 + kk) * kDim + c] : 0.f;
+        }
+        __syncthreads();
+        float sc[8];
+        float mt = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int kk = j8 + 8 * u;
+            float dot = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < kDim; ++c) dot = fmaf(qs[r * kDim + c], ks[kk * kKPitch + c], dot);
+            sc[u] = (k0 + kk <= qpos && k0 + kk < kend) ? dot * scale : -INFINITY;
+            mt = fmaxf(mt, sc[u]);
+        }
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        const float mnew = fmaxf(m, mt);
+        const float alpha = mnew == -INFINITY ? 1.f : __expf(m - mnew);  // 0 on a row's first live tile
+        float ls = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float p = sc[u] == -INFINITY ? 0.f : __expf(sc[u] - mnew);
+            ps[r * kKeys + j8 + 8 * u] = p;
+            ls += p;
+        }
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+        l = l * alpha + ls;
+        m = mnew;
+        __syncwarp();
+#pragma unroll
+        for (int d = 0; d < 16; ++d) acc[d] *= alpha;
+        for (int kk = 0; kk < kKeys; ++kk) {
+            const float p = ps[r * kKeys + kk];
+            const float *vrow = vs + kk * kDim + 16 * j8;
+#pragma unroll
+            for (int d = 0; d < 16; ++d) acc[d] = fmaf(p, vrow[d], acc[d]);
+        }
+    }
+    if (i0 + r < seq) {
+        const float inv = 1.f / l;
+        float *dst = o + (bh * seq + i0 + r) * kDim + 16 * j8;
+#pragma unroll
+        for (int d = 0; d < 16; ++d) dst[d] = acc[d] * inv;
+    }
+}
+
+}  // namespace gqs
+
+inline la_status launch_gqa_prefill_f32(const void *q, const void *k_new, const void *v_new, void *k_cache,
+                                        void *v_cache, int start, int batch, int heads, int kv_heads, int seq,
+                                        int cap, int rot, double base, float scale, void *o, void *q_rot,
+                                        cudaStream_t stream, std::string *err) {
+    gqs::gqs_rope_kernel<<<dim3((unsigned)seq, (unsigned)batch), 256, 0, stream>>>(
+        static_cast<const float *>(q), static_cast<const float *>(k_new), static_cast<const float *>(v_new),
+        static_cast<float *>(k_cache), static_cast<float *>(v_cache), static_cast<float *>(q_rot), heads, kv_heads,
+        seq, start, cap, rot, base);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        *err = std::string("gqa prefill rope launch: ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    e = cudaFuncSetAttribute(gqs::gqs_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gqs::kSmemBytes);
+    if (e != cudaSuccess) {
+        *err = std::string("cudaFuncSetAttribute(gqa prefill f32): ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    gqs::gqs_attn_kernel<<<dim3((unsigned)((seq + gqs::kQRows - 1) / gqs::kQRows), (unsigned)heads, (unsigned)batch),
+                           gqs::kThreads, gqs::kSmemBytes, stream>>>(
+        static_cast<const float *>(q_rot), static_cast<const float *>(k_cache), static_cast<const float *>(v_cache),
+        static_cast<float *>(o), heads, kv_heads, seq, start, cap, scale);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        *err = std::string("gqa prefill f32 attention launch: ") + cudaGetErrorString(e);
+        return LA_ERR_CUDA;
+    }
+    err->clear();
+    return LA_OK;
+}
+
+}  // namespace la

@@ -747,9 +747,10 @@ la_status lightning_gqa_decode(const void *q, const void *k_new, const void *v_n
                                  scale, o, workspace, st);
 }
 
-size_t lightning_gqa_prefill_workspace_size(int batch, int heads, int seq, int dim) {
-    if (batch < 0 || heads < 1 || seq < 0 || dim != la::gqp::kDim) return 0;
-    return (size_t)batch * heads * seq * dim * 2;
+size_t lightning_gqa_prefill_workspace_size(la_dtype dtype, int batch, int heads, int seq, int dim) {
+    if ((dtype != LA_DTYPE_F32 && dtype != LA_DTYPE_BF16) || batch < 0 || heads < 1 || seq < 0 || dim != la::gqp::kDim)
+        return 0;
+    return (size_t)batch * heads * seq * dim * elem_bytes(dtype);  // the rotated queries
 }
 
 la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
@@ -764,7 +765,6 @@ la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_
                     batch, seq, start, cap, heads, kv_heads);
     if ((long long)start + seq > cap) return fail(LA_ERR_INVALID_ARG, "start + seq (%lld) exceeds cap %d",
                                                    (long long)start + seq, cap);
-    if (dtype != LA_DTYPE_BF16) return fail(LA_ERR_UNSUPPORTED, "the GQA prefill takes bf16 inputs only");
     if (dim != la::gqp::kDim) return fail(LA_ERR_UNSUPPORTED, "dim %d unsupported (128)", dim);
     if (rot < 0 || rot > dim || (rot & 3)) return fail(LA_ERR_INVALID_ARG, "rot must be a multiple of 4, 0 <= rot <= dim");
     if (!(rope_base > 0.0) || rope_base > 1e300) return fail(LA_ERR_INVALID_ARG, "rope_base must be finite and > 0");
@@ -773,7 +773,7 @@ la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_
     if (batch == 0 || seq == 0) return ok();
     const long long ctas = (long long)batch * heads * ((seq + la::gqp::kQRows - 1) / la::gqp::kQRows);
     if (ctas > 0x7fffffffLL) return fail(LA_ERR_UNSUPPORTED, "problem too large for one launch");
-    const size_t need = lightning_gqa_prefill_workspace_size(batch, heads, seq, dim);
+    const size_t need = lightning_gqa_prefill_workspace_size(dtype, batch, heads, seq, dim);
     if (!q || !k_new || !v_new || !k_cache || !v_cache || !o)
         return fail(LA_ERR_INVALID_ARG, "q, k_new, v_new, the caches and o must be non-NULL");
     if (!workspace || workspace_bytes < need)
@@ -782,8 +782,9 @@ la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_
     const char *names[] = {"q", "k_new", "v_new", "k_cache", "v_cache", "o", "workspace"};
     for (int i = 0; i < 7; ++i)
         if (!aligned16(ptrs[i])) return fail(LA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
-    const size_t nq = (size_t)batch * heads * seq * dim * 2, nkv = (size_t)batch * kv_heads * seq * dim * 2;
-    const size_t ncache = (size_t)batch * kv_heads * cap * dim * 2;
+    const size_t eb = elem_bytes(dtype);
+    const size_t nq = (size_t)batch * heads * seq * dim * eb, nkv = (size_t)batch * kv_heads * seq * dim * eb;
+    const size_t ncache = (size_t)batch * kv_heads * cap * dim * eb;
     const Range all[] = {range_of(q, nq), range_of(k_new, nkv), range_of(v_new, nkv), range_of(k_cache, ncache),
                          range_of(v_cache, ncache), range_of(o, nq), range_of(workspace, need)};
     const int written[] = {3, 4, 5, 6};  // the caches, o and the workspace
@@ -791,6 +792,10 @@ la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_
         for (int j = 0; j < 7; ++j)
             if (j != wi && overlaps(all[wi], all[j]))
                 return fail(LA_ERR_INVALID_ARG, "%s overlaps %s", names[wi], names[j]);
+    if (dtype == LA_DTYPE_F32)
+        return la::launch_gqa_prefill_f32(q, k_new, v_new, k_cache, v_cache, start, batch, heads, kv_heads, seq, cap,
+                                          rot, rope_base, scale, o, workspace, static_cast<cudaStream_t>(stream),
+                                          &g_last_error);
     return la::launch_gqa_prefill(q, k_new, v_new, k_cache, v_cache, start, batch, heads, kv_heads, seq, cap, rot,
                                   rope_base, scale, o, workspace, static_cast<cudaStream_t>(stream), &g_last_error);
 }

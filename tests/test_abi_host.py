@@ -295,7 +295,6 @@ def _gqp(**kw):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(dtype=9), abi.LA_ERR_INVALID_ARG),
-    (dict(dtype=abi.LA_DTYPE_F32), abi.LA_ERR_UNSUPPORTED),   # bf16 only
     (dict(kv=7), abi.LA_ERR_INVALID_ARG),                     # does not divide 64
     (dict(start=-1), abi.LA_ERR_INVALID_ARG),
     (dict(seq=-3), abi.LA_ERR_INVALID_ARG),
@@ -321,8 +320,11 @@ def test_gqa_prefill_argument_errors(kw, status):
 
 def test_gqa_prefill_workspace_size_and_empty_calls():
     # the rotated queries, bf16, q's shape
-    assert abi.lightning_gqa_prefill_workspace_size(2, 64, 512, 128) == 2 * 64 * 512 * 128 * 2
-    assert abi.lightning_gqa_prefill_workspace_size(2, 64, 512, 64) == 0
-    assert abi.lightning_gqa_prefill_workspace_size(-1, 64, 512, 128) == 0
+    bf, f32 = abi.LA_DTYPE_BF16, abi.LA_DTYPE_F32
+    assert abi.lightning_gqa_prefill_workspace_size(bf, 2, 64, 512, 128) == 2 * 64 * 512 * 128 * 2
+    assert abi.lightning_gqa_prefill_workspace_size(f32, 2, 64, 512, 128) == 2 * 64 * 512 * 128 * 4
+    assert abi.lightning_gqa_prefill_workspace_size(bf, 2, 64, 512, 64) == 0
+    assert abi.lightning_gqa_prefill_workspace_size(bf, -1, 64, 512, 128) == 0
+    assert abi.lightning_gqa_prefill_workspace_size(7, 2, 64, 512, 128) == 0
     assert _gqp(batch=0) == abi.LA_OK
     assert _gqp(seq=0, q=None, o=None, ws=None) == abi.LA_OK

@@ -21,13 +21,21 @@ TOL_V = 2e-2
 TOL_RMS = 1e-2
 
 
-def check(got, ref, v_rms):
+# float32 inputs: fp32 throughout (rotation, scores, exact softmax, accumulation)
+TOL_V_F32 = 1e-4
+TOL_RMS_F32 = 1e-4
+
+
+def check(got, ref, v_rms, dtype=torch.bfloat16):
     got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
-    diff = np.maximum(np.abs(got - ref) - half_ulp_bf16(np.maximum(np.abs(got), np.abs(ref))), 0.0)
+    diff = np.abs(got - ref)
+    if dtype == torch.bfloat16:
+        diff = np.maximum(diff - half_ulp_bf16(np.maximum(np.abs(got), np.abs(ref))), 0.0)
+    tv, tr = (TOL_V, TOL_RMS) if dtype == torch.bfloat16 else (TOL_V_F32, TOL_RMS_F32)
     e = float(diff.max()) / v_rms
-    assert e <= TOL_V, "max error %.3g rms(v) > %.3g" % (e, TOL_V)
+    assert e <= tv, "max error %.3g rms(v) > %.3g" % (e, tv)
     er = float(np.sqrt(np.mean((got - ref) ** 2)) / np.sqrt(np.mean(ref ** 2)))
-    assert er <= TOL_RMS, "rms error %.3g rms(o) > %.3g" % (er, TOL_RMS)
+    assert er <= tr, "rms error %.3g rms(o) > %.3g" % (er, tr)
     return e
 
 
@@ -36,23 +44,23 @@ GUARD = 1024          # bf16 elements of guard band on each side of o (16-byte m
 SENTINEL = -77.0
 
 
-def _inputs(b, h, hk, L, cap, seed, q_scale=1.0):
+def _inputs(b, h, hk, L, cap, seed, q_scale=1.0, dtype=torch.bfloat16):
     g = torch.Generator(device=DEV).manual_seed(seed)
     d = 128
-    mk = lambda *shape: torch.randn(shape, generator=g, device=DEV).to(torch.bfloat16)
-    q = (torch.randn((b, h, L, d), generator=g, device=DEV) * q_scale).to(torch.bfloat16)
+    mk = lambda *shape: torch.randn(shape, generator=g, device=DEV).to(dtype)
+    q = (torch.randn((b, h, L, d), generator=g, device=DEV) * q_scale).to(dtype)
     return q, mk(b, hk, L, d), mk(b, hk, L, d), mk(b, hk, cap, d), mk(b, hk, cap, d)
 
 
-def _guarded_o(shape):
+def _guarded_o(shape, dtype=torch.bfloat16):
     n = int(np.prod(shape))
-    buf = torch.full((n + 2 * GUARD,), SENTINEL, dtype=torch.bfloat16, device=DEV)
+    buf = torch.full((n + 2 * GUARD,), SENTINEL, dtype=dtype, device=DEV)
     return buf, buf[GUARD:GUARD + n].view(shape)
 
 
 def _run(b, h, hk, L, start, cap, rot, seed, scale=None, q_scale=1.0, poison_tail=False, base=10000.0,
-         rows=None):
-    q, kn, vn, kc, vc = _inputs(b, h, hk, L, cap, seed, q_scale)
+         rows=None, dtype=torch.bfloat16):
+    q, kn, vn, kc, vc = _inputs(b, h, hk, L, cap, seed, q_scale, dtype)
     if poison_tail and start + L < cap:
         # rows past the sequence hold NaN: the kernel must never read them
         kc[:, :, start + L:] = float("nan")
@@ -61,7 +69,7 @@ def _run(b, h, hk, L, start, cap, rot, seed, scale=None, q_scale=1.0, poison_tai
     conv = inputs.to_oracle
     sc = 1.0 / np.sqrt(128.0) if scale is None else scale
     ref = oracle.gqa_prefill(conv(q), conv(kn), conv(vn), conv(kc0), conv(vc0), start, rot, base, sc, rows=rows)
-    buf, o = _guarded_o(q.shape)
+    buf, o = _guarded_o(q.shape, dtype)
     la.gqa_prefill(q, kn, vn, kc, vc, start=start, rot=rot, rope_base=base, scale=sc, o=o)
     torch.cuda.synchronize()
     assert torch.all(buf[:GUARD] == SENTINEL) and torch.all(buf[-GUARD:] == SENTINEL), "o guard band written"
@@ -72,8 +80,8 @@ def _run(b, h, hk, L, start, cap, rot, seed, scale=None, q_scale=1.0, poison_tai
         ref = ref.reshape(-1, 128)
     assert np.all(np.isfinite(got))
     v_rms = float(torch.sqrt(torch.mean(torch.cat([vn.float().flatten(), vc0[:, :, :start].float().flatten()]) ** 2)))
-    e = check(got, ref, v_rms)
-    print("gqa_prefill b%d h%d kv%d L%d start%d rot%d: max error %.3g rms(v)" % (b, h, hk, L, start, rot, e))
+    e = check(got, ref, v_rms, dtype)
+    print("gqa_prefill %s b%d h%d kv%d L%d start%d rot%d: max error %.3g rms(v)" % (str(dtype)[6:], b, h, hk, L, start, rot, e))
     # cache rows start .. start+L-1 hold the rotated keys and the values; the rest is untouched
     span = slice(start, start + L)
     for bb in range(b):
@@ -84,13 +92,16 @@ def _run(b, h, hk, L, start, cap, rot, seed, scale=None, q_scale=1.0, poison_tai
             if want is not None:
                 # the rotated key within the bf16 rounding of the cache (plus fp32 rotation noise)
                 got_k = to_f64(kc[bb, g, span])
-                slack = np.abs(got_k - want) - half_ulp_bf16(np.maximum(np.abs(got_k), np.abs(want)))
+                slack = np.abs(got_k - want)
+                if dtype == torch.bfloat16:
+                    slack = slack - half_ulp_bf16(np.maximum(np.abs(got_k), np.abs(want)))
                 assert slack.max() <= 1e-5 * np.sqrt(np.mean(want ** 2)), slack.max()
     assert torch.equal(vc[:, :, span], vn)
     keep = torch.ones(cap, dtype=torch.bool, device=DEV)
     keep[span] = False
-    assert torch.equal(kc[:, :, keep].view(torch.int16), kc0[:, :, keep].view(torch.int16))
-    assert torch.equal(vc[:, :, keep].view(torch.int16), vc0[:, :, keep].view(torch.int16))
+    iv = torch.int16 if dtype == torch.bfloat16 else torch.int32
+    assert torch.equal(kc[:, :, keep].view(iv), kc0[:, :, keep].view(iv))
+    assert torch.equal(vc[:, :, keep].view(iv), vc0[:, :, keep].view(iv))
     return e
 
 
@@ -176,3 +187,23 @@ def test_gqa_prefill_leaves_the_device_status_clean():
     assert abi.lightning_device_status(stream) == abi.LA_OK
     _run(1, 8, 2, 64, 10, 80, 64, seed=99)
     assert abi.lightning_device_status(stream) == abi.LA_OK
+
+
+F32_CASES = [
+    # (batch, heads, kv_heads, seq, start, cap, rot)
+    (1, 8, 2, 1, 0, 1, 64),
+    (2, 8, 4, 300, 37, 400, 64),
+    (1, 16, 2, 257, 0, 257, 128),
+    (1, 8, 8, 129, 200, 400, 0),
+]
+
+
+@pytest.mark.parametrize("case", F32_CASES, ids=lambda c: "b%d_h%d_kv%d_L%d_s%d_rot%d" % (c[0], c[1], c[2], c[3], c[4],
+                                                                                             c[6]))
+def test_gqa_prefill_float32_matches_the_oracle(case):
+    b, h, hk, L, start, cap, rot = case
+    _run(b, h, hk, L, start, cap, rot, seed=190 + L, dtype=torch.float32)
+
+
+def test_gqa_prefill_float32_never_reads_cache_rows_past_the_sequence():
+    _run(1, 8, 2, 100, 20, 400, 64, seed=191, poison_tail=True, dtype=torch.float32)
