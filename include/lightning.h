@@ -292,7 +292,8 @@ la_status lightning_selftest_wait_timeout(void *stream);
  *   pos              DEVICE int32 [batch], 0 <= pos[b] < cap; an out-of-range
  *                    position skips that sequence (o = 0) and is reported as
  *                    LA_ERR_INVALID_ARG by lightning_device_status().
- *   dim 128; heads / kv_heads at most 8; rot even, 0 <= rot <= dim.
+ *   dim 128; heads / kv_heads at most 32 (bf16) or 8 (float32); rot even,
+ *   0 <= rot <= dim.
  *   o                [batch][heads][dim], dtype; written.
  *   workspace        lightning_gqa_decode_workspace_size(batch, heads, cap)
  *                    bytes, 16-byte aligned.

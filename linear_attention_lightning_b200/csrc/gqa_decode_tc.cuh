@@ -4,7 +4,7 @@
 // the scores and the weighted values as tcgen05 MMAs.
 //
 // One CTA per (chunk of kGqaChunk positions, KV head, sequence). The group's
-// query heads (at most 8) are the first rows of a 128-row Q tile; the other
+// query heads (at most 32, one softmax lane each) are the first rows of a 128-row Q tile; the other
 // rows are zero, so the MMAs do 16x the useful work, which the step can afford
 // (it is bound by reading the cache). Per key tile j of 128 positions:
 //   S_j = Q K_j^T      SS MMA bf16, M128 N128 K128 -> TMEM, double-buffered

@@ -710,8 +710,11 @@ la_status lightning_gqa_decode(const void *q, const void *k_new, const void *v_n
         return fail(LA_ERR_INVALID_ARG, "need batch >= 0, cap >= 1 and kv_heads dividing heads (got %d, %d, %d, %d)",
                     batch, cap, heads, kv_heads);
     if (dim != la::kGqaDim) return fail(LA_ERR_UNSUPPORTED, "dim %d unsupported (128)", dim);
-    if (heads / kv_heads > la::kGqaMaxGroup)
-        return fail(LA_ERR_UNSUPPORTED, "at most %d query heads per KV head (got %d)", la::kGqaMaxGroup,
+    // bf16: the group's heads are rows handled by one 32-lane softmax warp; float32: the
+    // CUDA-core kernel keeps kGqaMaxGroup heads in registers
+    const int max_group = dtype == LA_DTYPE_BF16 ? 32 : la::kGqaMaxGroup;
+    if (heads / kv_heads > max_group)
+        return fail(LA_ERR_UNSUPPORTED, "at most %d query heads per KV head for this dtype (got %d)", max_group,
                     heads / kv_heads);
     if (rot < 0 || rot > dim || (rot & 1)) return fail(LA_ERR_INVALID_ARG, "rot must be even, 0 <= rot <= dim");
     if (!(rope_base > 0.0) || rope_base > 1e300) return fail(LA_ERR_INVALID_ARG, "rope_base must be finite and > 0");

@@ -258,7 +258,8 @@ def _gqa(**kw):
     (dict(kv=7), abi.LA_ERR_INVALID_ARG),               # does not divide 64
     (dict(cap=0), abi.LA_ERR_INVALID_ARG),
     (dict(dim=64), abi.LA_ERR_UNSUPPORTED),
-    (dict(kv=4), abi.LA_ERR_UNSUPPORTED),               # 16 query heads per KV head
+    (dict(kv=4, dtype=abi.LA_DTYPE_F32), abi.LA_ERR_UNSUPPORTED),  # 16 query heads per KV head, float32
+    (dict(kv=1), abi.LA_ERR_UNSUPPORTED),               # 64 query heads per KV head
     (dict(rot=63), abi.LA_ERR_INVALID_ARG),
     (dict(rot=130), abi.LA_ERR_INVALID_ARG),
     (dict(base=0.0), abi.LA_ERR_INVALID_ARG),

@@ -99,3 +99,12 @@ def test_gqa_decode_never_lets_cache_rows_past_pos_into_the_result():
     assert np.all(np.isfinite(got))
     e = rel_err(got, ref, bf16_out=1)
     assert e <= TOL[torch.bfloat16], e
+
+
+@pytest.mark.parametrize("case", [(1, 32, 2, 1500, [1499]), (2, 64, 2, 2100, [2099, 700])],
+                         ids=["group16", "group32"])
+def test_gqa_decode_bf16_groups_up_to_32(case):
+    # the tensor-core path takes a KV head's query group as the rows of its tile, one softmax
+    # lane per head: groups up to 32
+    b, h, hk, cap, positions = case
+    _run_and_check(b, h, hk, cap, positions, 64, torch.bfloat16, seed=84)
