@@ -379,6 +379,9 @@ def run_ours(args):
     # prefill of the softmax GQA layer at the same context length
     gqp = run_gqa_prefill_leg(dev, stream, args, world) if args.gqa_prefill_steps > 0 else None
 
+    # the batched workload: many short sequences with carried-in states
+    bat = run_batched_leg(dev, stream, peaks, args, world) if args.batched_steps > 0 else None
+
     # one block of the hybrid model's attention: 7 Lightning layers and 1 softmax layer
     hyb = (run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world)
            if args.hybrid_steps > 0 and w.dtype == torch.bfloat16 and w.dim == 128 else None)
@@ -409,6 +412,7 @@ def run_ours(args):
         "norm_gate": ng,
         "gqa_decode": gqa,
         "gqa_prefill": gqp,
+        "batched_prefill": bat,
         "hybrid_block": hyb,
         "hybrid_decode": hyd,
         "backward": bwd,
@@ -735,6 +739,48 @@ def run_hybrid_decode_leg(dev, stream, args, world):
             "steps": steps, "us_per_step": round(ms * 1e3, 2), "tokens_per_s": round(world * b / (ms / 1e3), 1)}
 
 
+def run_batched_leg(dev, stream, peaks, args, world):
+    """The prefill on the batched workload with carried-in states (16 sequences
+    x 64 heads x 4096 tokens, fp32 state_in): many short sequences instead of
+    one long one; timed like the main leg."""
+    import torch
+    import linear_attention_lightning_b200 as la
+    from linear_attention_lightning_b200 import abi, inputs
+    bw = inputs.WORKLOADS["batched_prefill_state"]
+    inp = inputs.workload_inputs(bw, dev)
+    q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
+    o = torch.empty_like(q)
+    s_out = torch.empty((bw.batch, bw.heads, bw.dim, bw.dim), dtype=torch.float32, device=dev)
+    variant = la.prefill_variant(bw.dtype, bw.batch, bw.heads, bw.seq, bw.dim, bw.block)
+    vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05,
+             "pair": abi.LA_VARIANT_TCGEN05_PAIR}[variant]
+    sp = stream.cuda_stream
+
+    def step():
+        abi.check(abi.lightning_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), abi.LA_DTYPE_BF16, sl.data_ptr(),
+                                           bw.batch, bw.heads, bw.seq, bw.dim, bw.block, s0.data_ptr(), o.data_ptr(),
+                                           s_out.data_ptr(), None, 0, sp, vcode))
+
+    for _ in range(args.warmup):
+        step()
+    steps = args.batched_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    by = prefill_bytes(bw.batch, bw.heads, bw.seq, bw.dim, 2, state_in=True, state_out=True)
+    gbs = by / (ms / 1e3) / 1e9
+    fl = prefill_flops(bw.batch, bw.heads, bw.seq, bw.dim, bw.block)["formula"] / (ms / 1e3) / 1e12
+    return {"workload": bw.name, "kernel": variant, "steps": steps, "ms_per_step": round(ms, 4),
+            "tokens_per_s": round(world * bw.batch * bw.seq / (ms / 1e3), 1), "tflops_formula": round(fl, 2),
+            "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s", measured_traffic(bw.name, variant))}
+
+
 def run_backward_leg(w, dev, stream, inp, dcode, args, world):
     """lightning_prefill_backward on the workload (AUTO: the CTA-pair tensor-core
     kernel where it applies), timed like the main leg: dQ causal on (dO, V, K),
@@ -886,6 +932,8 @@ def parse_args(argv=None):
                    help="timed steps of the softmax GQA prefill leg (0 skips it)")
     p.add_argument("--gqa-prefill-seq", type=int, default=131072,
                    help="new tokens of the GQA prefill leg")
+    p.add_argument("--batched-steps", type=int, default=5,
+                   help="timed steps of the batched-prefill leg, 16 x 64 heads x 4096 tokens (0 skips it)")
     p.add_argument("--hybrid-steps", type=int, default=2,
                    help="timed steps of the hybrid-block leg, 7 Lightning + 1 softmax layer (0 skips it)")
     p.add_argument("--norm-gate-steps", type=int, default=20,
