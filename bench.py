@@ -379,8 +379,10 @@ def run_ours(args):
     # prefill of the softmax GQA layer at the same context length
     gqp = run_gqa_prefill_leg(dev, stream, args, world) if args.gqa_prefill_steps > 0 else None
 
-    # the batched workload: many short sequences with carried-in states
-    bat = run_batched_leg(dev, stream, peaks, args, world) if args.batched_steps > 0 else None
+    # the other prefill workloads: many short sequences with carried-in states; 8192 tokens
+    others = ({n: run_workload_leg(n, dev, stream, peaks, args, world)
+               for n in ("batched_prefill_state", "m1_prefill_8k") if n != w.name}
+              if args.batched_steps > 0 else None)
 
     # one block of the hybrid model's attention: 7 Lightning layers and 1 softmax layer
     hyb = (run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world)
@@ -412,7 +414,7 @@ def run_ours(args):
         "norm_gate": ng,
         "gqa_decode": gqa,
         "gqa_prefill": gqp,
-        "batched_prefill": bat,
+        "other_workloads": others,
         "hybrid_block": hyb,
         "hybrid_decode": hyd,
         "backward": bwd,
@@ -739,14 +741,14 @@ def run_hybrid_decode_leg(dev, stream, args, world):
             "steps": steps, "us_per_step": round(ms * 1e3, 2), "tokens_per_s": round(world * b / (ms / 1e3), 1)}
 
 
-def run_batched_leg(dev, stream, peaks, args, world):
-    """The prefill on the batched workload with carried-in states (16 sequences
-    x 64 heads x 4096 tokens, fp32 state_in): many short sequences instead of
-    one long one; timed like the main leg."""
+def run_workload_leg(name, dev, stream, peaks, args, world):
+    """The prefill on another named workload (the batched one with carried-in
+    states: 16 sequences x 64 heads x 4096 tokens; the 8192-token one), timed
+    like the main leg."""
     import torch
     import linear_attention_lightning_b200 as la
     from linear_attention_lightning_b200 import abi, inputs
-    bw = inputs.WORKLOADS["batched_prefill_state"]
+    bw = inputs.WORKLOADS[name]
     inp = inputs.workload_inputs(bw, dev)
     q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
     o = torch.empty_like(q)
@@ -758,8 +760,9 @@ def run_batched_leg(dev, stream, peaks, args, world):
 
     def step():
         abi.check(abi.lightning_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), abi.LA_DTYPE_BF16, sl.data_ptr(),
-                                           bw.batch, bw.heads, bw.seq, bw.dim, bw.block, s0.data_ptr(), o.data_ptr(),
-                                           s_out.data_ptr(), None, 0, sp, vcode))
+                                           bw.batch, bw.heads, bw.seq, bw.dim, bw.block,
+                                           None if s0 is None else s0.data_ptr(), o.data_ptr(), s_out.data_ptr(), None,
+                                           0, sp, vcode))
 
     for _ in range(args.warmup):
         step()
@@ -773,7 +776,7 @@ def run_batched_leg(dev, stream, peaks, args, world):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
-    by = prefill_bytes(bw.batch, bw.heads, bw.seq, bw.dim, 2, state_in=True, state_out=True)
+    by = prefill_bytes(bw.batch, bw.heads, bw.seq, bw.dim, 2, state_in=s0 is not None, state_out=True)
     gbs = by / (ms / 1e3) / 1e9
     fl = prefill_flops(bw.batch, bw.heads, bw.seq, bw.dim, bw.block)["formula"] / (ms / 1e3) / 1e12
     return {"workload": bw.name, "kernel": variant, "steps": steps, "ms_per_step": round(ms, 4),
@@ -933,7 +936,7 @@ def parse_args(argv=None):
     p.add_argument("--gqa-prefill-seq", type=int, default=131072,
                    help="new tokens of the GQA prefill leg")
     p.add_argument("--batched-steps", type=int, default=5,
-                   help="timed steps of the batched-prefill leg, 16 x 64 heads x 4096 tokens (0 skips it)")
+                   help="timed steps of the other prefill workloads' legs (0 skips them)")
     p.add_argument("--hybrid-steps", type=int, default=2,
                    help="timed steps of the hybrid-block leg, 7 Lightning + 1 softmax layer (0 skips it)")
     p.add_argument("--norm-gate-steps", type=int, default=20,
