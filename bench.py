@@ -85,15 +85,16 @@ KERNEL_SOURCES = {  # traffic.json key suffix -> the header that holds the kerne
 
 
 def kernel_source_digest(header):
-    """Digest of one kernel's header and every local header it includes, to
-    tell whether stored ncu counters still describe the kernel being timed."""
+    """Digest of one kernel's header and every kernel source it includes (the
+    files under csrc/; the public header holds only declarations), to tell
+    whether stored ncu counters still describe the kernel being timed."""
     import hashlib
     import re
     csrc = os.path.join(ROOT, "linear_attention_lightning_b200", "csrc")
     seen, todo = [], [os.path.normpath(os.path.join(csrc, header))]
     while todo:
         path = todo.pop()
-        if path in seen:
+        if path in seen or os.path.dirname(path) != os.path.normpath(csrc):
             continue
         seen.append(path)
         with open(path, "rb") as f:

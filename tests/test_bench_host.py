@@ -89,11 +89,11 @@ def test_stored_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
         f.write("// edit\n")
     assert bench.measured_traffic("w", "pair") is None
     assert bench.measured_traffic("w", "norm_gate") is None
-    # the public header is part of the pair kernel's sources
+    # the public header (declarations only) is not part of any kernel's sources
     store()
     with open(tmp_path / "include" / "lightning.h", "a") as f:
         f.write("// edit\n")
-    assert bench.measured_traffic("w", "pair") is None
+    assert bench.measured_traffic("w", "pair") == 123
     assert bench.measured_traffic("w", "norm_gate") == 456
 
 
