@@ -32,6 +32,9 @@
 // commit that announces S_t(j+1) also covers PV_t(j) (O_t is complete when the
 // softmax warpgroup reads it). The epilogue scales O_t by 1/l, rounds it to
 // bf16 into the Q_t tile's shared memory and stores it with TMA.
+// CTAs go KV head by KV head (query head fastest, then the query rows from the longest
+// down), so the CTAs resident at a time read one KV head's keys and values, which L2 holds
+// (67 MB at 131072 positions); heavy-first within a KV head keeps the tail short.
 // Key tiles end at position start+seq-1: the key and value tensor maps stop
 // there, so TMA reads zeros past it and no cache row beyond the sequence is
 // ever read.
@@ -259,8 +262,8 @@ __device__ __forceinline__ Work work_of(int heads, int kv_heads, int batch, int 
     const int npairs = (seq + kQRows - 1) / kQRows;
     const int x = blockIdx.x;
     const int hq = x % group, rest = x / group;
-    const int bkv = rest % nkv;
-    const int pi = npairs - 1 - rest / nkv;  // the longest rows first
+    const int pi = npairs - 1 - rest % npairs;  // the longest rows first, within a KV head
+    const int bkv = rest / npairs;
     const int b = bkv / kv_heads, g = bkv - b * kv_heads;
     Work w;
     w.bh = b * heads + g * group + hq;
