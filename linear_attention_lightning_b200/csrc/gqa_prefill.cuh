@@ -258,7 +258,7 @@ struct Work {
 };
 
 __device__ __forceinline__ Work work_of(int heads, int kv_heads, int batch, int seq, int start) {
-    const int group = heads / kv_heads, nkv = batch * kv_heads;
+    const int group = heads / kv_heads;
     const int npairs = (seq + kQRows - 1) / kQRows;
     const int x = blockIdx.x;
     const int hq = x % group, rest = x / group;

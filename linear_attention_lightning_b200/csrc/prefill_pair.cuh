@@ -266,7 +266,9 @@ __device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scal
 
 // How one launch runs. The forward prefill is {0, 0}; the passes of the
 // backward computation (lightning_api.cu) read the carried state transposed,
-// or run anti-causal.
+// or run anti-causal. The direction is a template argument of the kernel, so
+// that the causal instantiation carries no anti-causal code (a smaller hot
+// loop for the instruction cache).
 struct PairPass {
     int state_in_t;  // 1: state_in holds the transpose of the carried state
     int anti;        // 1: anti-causal: blocks from last to first, query i sees keys j >= i
@@ -274,6 +276,7 @@ struct PairPass {
                      //    token (query factor e^{-s(m-1-i)}, key factor e^{-s(j+1)})
 };
 
+template <bool kAnti>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v,
@@ -297,7 +300,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const float sl2 = s * kLog2e;
     const int nblk = (seq + kBlock - 1) / kBlock;
     // block index of the t-th block visited, and its length
-    auto tb = [&](int t) { return pp.anti ? nblk - 1 - t : t; };
+    auto tb = [&](int t) { return kAnti ? nblk - 1 - t : t; };
     auto blen = [&](int t) { return min(kBlock, seq - tb(t) * kBlock); };
 
     if (threadIdx.x == 0) {
@@ -506,7 +509,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const int h = u & 1, j = kRows * h + r;
                     const float sc = u >= 2   ? 1.f
                                      : j >= m ? 0.f
-                                              : ptx::ex2(-sl2 * (float)(pp.anti ? j + 1 : m - 1 - j));
+                                              : ptx::ex2(-sl2 * (float)(kAnti ? j + 1 : m - 1 - j));
                     scale_row_to_f16((u >= 2 ? vt : kd) + h * kBoxBytes + r * 128, r, sc);
                 }
                 ptx::fence_proxy_async_smem();
@@ -517,7 +520,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // Qd S MMA (which precedes its dS MMA) has read the region
                 if (t > 0 && !group_wait(c, DS_FULL, (uint32_t)(t - 1) & 1u, leader, bar_id)) goto ab_done;
                 if (!group_wait(c, QK_LOADED, par, leader, bar_id)) goto ab_done;
-                const float dq = pp.anti ? (i < m ? ptx::ex2(-sl2 * (float)(m - 1 - i)) : 0.f)
+                const float dq = kAnti ? (i < m ? ptx::ex2(-sl2 * (float)(m - 1 - i)) : 0.f)
                                          : ptx::ex2(-sl2 * (float)(i + 1));
                 const uint8_t *qrow = c.smem + kOffQ + r * 128;
 #pragma unroll 1
@@ -549,7 +552,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // 128..255 x keys 0..127) is only cleared
             if (!group_wait(c, P_FULL + grp, par, leader, bar_id)) goto ab_done;
             ptx::tc_fence_after();
-            if (pp.anti ? (grp == 0 && rank == 1) : (grp == 1 && rank == 0)) {
+            if (kAnti ? (grp == 0 && rank == 1) : (grp == 1 && rank == 0)) {
                 // every entry of this quadrant is masked
                 uint32_t zero[16];
 #pragma unroll
@@ -558,7 +561,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int q = 0; q < 4; ++q) ptx::tmem_st16(trow + (grp == 0 ? kColP : kColPHi) + 16 * q, zero);
             } else {
                 convert_p(trow, grp == 0 ? kColP : kColPHi, grp == 0 ? kColP : kColPHi, i, kRows * grp, sl2,
-                          step, tab, pp.anti != 0);
+                          step, tab, kAnti);
             }
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
@@ -645,7 +648,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const float dnext =
                     last ? 0.f
                          : ptx::ex2(-sl2 * (float)blen(t + 1));
-                float *snap = t >= 0 && !pp.anti ? snapshot_at(sn, bh, t * kBlock + blen(t), kDim) : nullptr;
+                float *snap = t >= 0 && !kAnti ? snapshot_at(sn, bh, t * kBlock + blen(t), kDim) : nullptr;
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     float sv[32];
@@ -739,8 +742,8 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
         !tc::make_map(&mk64, k, seq, bh, err, 64) || !tc::make_map(&mv, v, seq, bh, err) ||
         !tc::make_map(&mo, o, seq, bh, err))
         return LA_ERR_CUDA;
-    cudaError_t e = cudaFuncSetAttribute(pair::prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)pair::kSmemBytes);
+    const auto kernel = pp.anti ? pair::prefill_pair_kernel<true> : pair::prefill_pair_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pair::kSmemBytes);
     if (e != cudaSuccess) {
         *err = std::string("cudaFuncSetAttribute(prefill_pair): ") + cudaGetErrorString(e);
         return LA_ERR_CUDA;
@@ -757,7 +760,7 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, pair::prefill_pair_kernel, mq, mk, mk64, mv, mo, slopes, heads, seq, state_in,
+    e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mk64, mv, mo, slopes, heads, seq, state_in,
                            state_out, sn, pp);
     if (e != cudaSuccess) {
         *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
