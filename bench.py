@@ -80,7 +80,7 @@ def roofline(bound, achieved, peak, unit, traffic=None):
 KERNEL_SOURCES = {  # traffic.json key suffix -> the header that holds the kernel
     "pair": "prefill_pair.cuh", "tcgen05": "prefill_tc.cuh", "simt": "prefill_simt.cuh",
     "backward_pair": "prefill_pair.cuh", "decode": "decode.cuh", "norm_gate": "norm_gate.cuh",
-    "gqa_partial": "gqa_decode_tc.cuh", "gqp_attn": "gqa_prefill.cuh",
+    "gqa_partial": "gqa_decode_tc.cuh", "gqp_attn": "gqa_prefill.cuh", "prefill_norm_gate": "prefill_pair.cuh",
 }
 
 
@@ -374,6 +374,10 @@ def run_ours(args):
     # normalisation and gating of the prefill's output
     ng = run_norm_gate_leg(w, dev, stream, o, dcode, args, world) if args.norm_gate_steps > 0 else None
 
+    # the same prefill with the per-head normalisation and gate fused into its epilogue
+    png = (run_prefill_norm_gate_leg(w, dev, stream, inp, dcode, args, world)
+           if args.norm_gate_steps > 0 and variant == "pair" else None)
+
     # decode step of the softmax GQA layer the hybrid model interleaves
     gqa = run_gqa_leg(dev, stream, args, world) if args.gqa_steps > 0 else None
 
@@ -413,6 +417,7 @@ def run_ours(args):
         "e2e": e2e,
         "snapshots": snaps,
         "norm_gate": ng,
+        "prefill_norm_gate": png,
         "gqa_decode": gqa,
         "gqa_prefill": gqp,
         "other_workloads": others,
@@ -535,6 +540,64 @@ def run_norm_gate_leg(w, dev, stream, o, dcode, args, world):
     return {"steps": steps, "ms_per_step": round(ms, 4), "per": "token (heads*dim channels)",
             "tokens_per_s": round(world * w.batch * w.seq / (ms / 1e3), 1),
             "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s", measured_traffic(w.name, "norm_gate"))}
+
+
+def run_prefill_norm_gate_leg(w, dev, stream, inp, dcode, args, world):
+    """lightning_prefill_norm_gate (the per-head normalisation and gate fused into
+    the prefill's epilogue, o never written) against the two calls it replaces
+    (lightning_prefill_ex, then lightning_norm_gate with the per-head mean),
+    alternating, each timed like the main leg."""
+    import torch
+    from linear_attention_lightning_b200 import abi
+    q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
+    g = torch.Generator(device=dev).manual_seed(w.seed + 2000)
+    gate = torch.randn((w.batch, w.seq, w.heads * w.dim), generator=g, device=dev).to(q.dtype)
+    gamma = torch.ones(w.heads * w.dim, device=dev)
+    y = torch.empty((w.batch, w.seq, w.heads * w.dim), dtype=q.dtype, device=dev)
+    o = torch.empty_like(q)
+    s_out = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32, device=dev)
+    sp = stream.cuda_stream
+    s0p = None if s0 is None else s0.data_ptr()
+
+    def fused():
+        abi.check(abi.lightning_prefill_norm_gate(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads, w.seq, w.dim,
+            w.block, s0p, gate.data_ptr(), gamma.data_ptr(), 1e-6, y.data_ptr(), s_out.data_ptr(), sp))
+
+    def two_calls():
+        abi.check(abi.lightning_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch,
+                                           w.heads, w.seq, w.dim, w.block, s0p, o.data_ptr(), s_out.data_ptr(),
+                                           None, 0, sp, abi.LA_VARIANT_TCGEN05_PAIR))
+        abi.check(abi.lightning_norm_gate(o.data_ptr(), gate.data_ptr(), dcode, gamma.data_ptr(), 1e-6, w.batch,
+                                          w.heads, w.seq, w.dim, 1, y.data_ptr(), sp))
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+
+    steps = max(1, min(args.norm_gate_steps, 10))
+    f_ms, t_ms = [], []
+    for _ in range(2):
+        f_ms.append(timed(fused, steps))
+        t_ms.append(timed(two_calls, steps))
+    ms, ms2 = min(f_ms), min(t_ms)
+    n = q.numel() * q.element_size()
+    by = 5 * n + gamma.numel() * 4 + (0 if s0 is None else 2 * s0.numel() * 4)  # q, k, v, gate in; y out
+    gbs = by / (ms / 1e3) / 1e9
+    return {"steps": steps, "ms_per_step": round(ms, 4), "two_calls_ms_per_step": round(ms2, 4),
+            "speedup_vs_two_calls": round(ms2 / ms, 3), "per": "head (dim channels)",
+            "tokens_per_s": round(world * w.batch * w.seq / (ms / 1e3), 1), "algorithmic_bytes": by,
+            "roofline": roofline("hbm", gbs, load_peaks()["hbm_gbs"], "GB/s",
+                                 measured_traffic(w.name, "prefill_norm_gate"))}
 
 
 GQA_BATCH, GQA_HEADS, GQA_KV_HEADS, GQA_CAP = 8, 64, 8, 131072

@@ -237,6 +237,33 @@ size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int 
 la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, const float *gamma, float eps,
                               int batch, int heads, int seq, int dim, int per_head, void *y, void *stream);
 
+/*
+ * A prefill whose output goes through the normalisation and gating above with
+ * the per-head mean (per_head != 0), fused into the prefill's output epilogue:
+ * o is never written to memory. Source: "MINIMAX SIGNAL LAB · M1", §03
+ * Lightning Attention (the figure's sum of the intra- and inter-block outputs,
+ * then normalisation and gate; the same reading as lightning_norm_gate).
+ *   y[b][l][h*128 + c] = gamma[h*128 + c] o[b][h][l][c]
+ *                        / sqrt(mean_c o[b][h][l][c]^2 + eps) * sigmoid(gate[b][l][h*128 + c])
+ * with o the result lightning_prefill defines (before its rounding to bf16;
+ * the normalised value is formed from o rounded to bf16 and the fp32 mean).
+ *
+ *   q, k, v, slopes, state_in, state_out: as for lightning_prefill.
+ *   gate   [batch][seq][heads*128] bf16; read only.
+ *   gamma  [heads*128] float32.   eps: finite, >= 0.
+ *   y      [batch][seq][heads*128] bf16; written; must not overlap any input,
+ *          the states, gate or gamma.
+ * Runs on the CTA-pair tensor-core kernel only: bf16, dim 128, block 256;
+ * other shapes or dtypes return LA_ERR_UNSUPPORTED before any launch (the
+ * whole-token mean needs every head of a token, which one head's kernel does
+ * not see: use lightning_prefill then lightning_norm_gate). Device pointers,
+ * caller-owned, 16-byte aligned; asynchronous on `stream`.
+ */
+la_status lightning_prefill_norm_gate(const void *q, const void *k, const void *v, la_dtype dtype,
+                                      const float *slopes, int batch, int heads, int seq, int dim, int block,
+                                      const float *state_in, const void *gate, const float *gamma, float eps,
+                                      void *y, float *state_out, void *stream);
+
 /* Number of snapshots lightning_prefill_snapshots writes per (batch, head):
  * seq / interval, or -1 if seq < 0 or interval < 1. Host only. */
 int lightning_prefill_snapshot_count(int seq, int interval);

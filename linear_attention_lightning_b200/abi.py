@@ -31,6 +31,8 @@ _SIGNATURES = {
                                      _i], _i),
     "lightning_prefill_snapshot_count": ([_i, _i], _i),
     "lightning_norm_gate": ([_vp, _vp, _i, _vp, ctypes.c_float, _i, _i, _i, _i, _i, _vp, _vp], _i),
+    "lightning_prefill_norm_gate": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, ctypes.c_float,
+                                     _vp, _vp, _vp], _i),
     "lightning_gqa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_double,
                               ctypes.c_float, _vp, _vp, _sz, _vp], _i),
     "lightning_gqa_decode_workspace_size": ([_i, _i, _i], _sz),
@@ -150,6 +152,12 @@ def lightning_prefill_backward_workspace_size(dtype, batch, heads, seq, dim, blo
 
 def lightning_norm_gate(o, gate, dtype, gamma, eps, batch, heads, seq, dim, per_head, y, stream):
     return load().lightning_norm_gate(o, gate, dtype, gamma, eps, batch, heads, seq, dim, per_head, y, stream)
+
+
+def lightning_prefill_norm_gate(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, gate, gamma, eps,
+                                y, state_out, stream):
+    return load().lightning_prefill_norm_gate(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in,
+                                              gate, gamma, eps, y, state_out, stream)
 
 
 def lightning_gqa_decode(q, k_new, v_new, k_cache, v_cache, dtype, pos, batch, heads, kv_heads, dim, cap, rot,

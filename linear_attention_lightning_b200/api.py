@@ -162,6 +162,41 @@ def norm_gate(o: torch.Tensor, gate: torch.Tensor, gamma: torch.Tensor, eps: flo
     return y
 
 
+def prefill_norm_gate(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor, block: int,
+                      gate: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+                      state_in: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                      state_out: Optional[torch.Tensor] = None, want_state: bool = True,
+                      stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """lightning_prefill_norm_gate: the prefill with the per-head normalisation and
+    gate fused into its epilogue; returns (y [batch, seq, heads*dim], state_out)."""
+    if q.dtype not in _DTYPES:
+        raise ValueError("q must be float32 or bfloat16")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share one [batch, heads, seq, dim] shape")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(name, t, q.dtype)
+    b, h, L, d = q.shape
+    _need_cuda("slopes", slopes, torch.float32)
+    _need_cuda("gate", gate, q.dtype)
+    if tuple(gate.shape) != (b, L, h * d):
+        raise ValueError("gate must be [batch, seq, heads*dim]")
+    _need_cuda("gamma", gamma, torch.float32)
+    if tuple(gamma.shape) != (h * d,):
+        raise ValueError("gamma must be [heads*dim]")
+    if state_in is not None:
+        _need_cuda("state_in", state_in, torch.float32)
+        if tuple(state_in.shape) != (b, h, d, d):
+            raise ValueError("state_in must be [batch, heads, dim, dim]")
+    if y is None:
+        y = torch.empty((b, L, h * d), dtype=q.dtype, device=q.device)
+    if state_out is None and want_state:
+        state_out = torch.empty((b, h, d, d), dtype=torch.float32, device=q.device)
+    abi.check(abi.lightning_prefill_norm_gate(
+        _ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(slopes), b, h, L, d, int(block), _ptr(state_in),
+        _ptr(gate), _ptr(gamma), float(eps), _ptr(y), _ptr(state_out), _stream(stream)))
+    return y, state_out
+
+
 def gqa_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
                v_cache: torch.Tensor, pos: torch.Tensor, rot: int = 64, rope_base: float = 10000.0,
                scale: Optional[float] = None, o: Optional[torch.Tensor] = None,

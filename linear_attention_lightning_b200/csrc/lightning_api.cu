@@ -654,6 +654,43 @@ size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int 
     return chosen < 0 ? 0 : backward_workspace_bytes(dtype, batch, heads, seq, dim, chosen);
 }
 
+la_status lightning_prefill_norm_gate(const void *q, const void *k, const void *v, la_dtype dtype,
+                                      const float *slopes, int batch, int heads, int seq, int dim, int block,
+                                      const float *state_in, const void *gate, const float *gamma, float eps,
+                                      void *y, float *state_out, void *stream) {
+    la_status st = check_prefill_shape(dtype, batch, heads, seq, dim, block);
+    if (st != LA_OK) return st;
+    if (!la::pair_supports(dtype == LA_DTYPE_BF16, dim, block))
+        return fail(LA_ERR_UNSUPPORTED,
+                    "the fused normalisation runs on the CTA-pair kernel: bf16, dim 128, block 256 (got dtype %d, "
+                    "dim %d, block %d)",
+                    (int)dtype, dim, block);
+    if (!(eps >= 0.f) || eps > 3.0e38f) return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    const PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, y, state_out,
+                        la::Snapshots{nullptr, 0, 0}};
+    st = check_prefill_pointers(a);
+    if (st != LA_OK) return st;
+    const size_t n_tok = (size_t)batch * heads * seq * dim;
+    if (n_tok > 0) {
+        if (!gate || !gamma) return fail(LA_ERR_INVALID_ARG, "gate and gamma must be non-NULL when seq > 0");
+        if (!aligned16(gate) || !aligned16(gamma))
+            return fail(LA_ERR_INVALID_ARG, "gate and gamma must be 16-byte aligned");
+        const Range ry = range_of(y, n_tok * 2);
+        if (overlaps(ry, range_of(gate, n_tok * 2)) || overlaps(ry, range_of(gamma, sizeof(float) * heads * dim)))
+            return fail(LA_ERR_INVALID_ARG, "y overlaps gate or gamma");
+        if (state_out) {
+            const Range rs = range_of(state_out, (size_t)batch * heads * dim * dim * 4);
+            if (overlaps(rs, range_of(gate, n_tok * 2)) || overlaps(rs, range_of(gamma, sizeof(float) * heads * dim)))
+                return fail(LA_ERR_INVALID_ARG, "state_out overlaps gate or gamma");
+        }
+    }
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (batch == 0 || seq == 0) return run_prefill(a, cs, LA_VARIANT_TCGEN05_PAIR);
+    const la::pair::PairNormGate ng{static_cast<const __nv_bfloat16 *>(gate), gamma, eps};
+    return la::launch_pair(q, k, v, slopes, batch, heads, seq, state_in, y, state_out, a.sn, la::pair::PairPass{0, 0},
+                           cs, &g_last_error, &ng);
+}
+
 la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, const float *gamma, float eps,
                               int batch, int heads, int seq, int dim, int per_head, void *y, void *stream) {
     if (dtype != LA_DTYPE_F32 && dtype != LA_DTYPE_BF16)

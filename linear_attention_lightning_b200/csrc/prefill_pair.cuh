@@ -81,7 +81,8 @@ constexpr uint32_t kOffE = kOffS + kSBytes;                    // output staging
 constexpr uint32_t kOffBar = kOffE + kBoxBytes;
 constexpr int kNumBars = 24;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+constexpr uint32_t kOffGamma = kOffMisc + 64;                  // fused norm + gate: gamma of the head
+constexpr uint32_t kSmemBytes = kOffGamma + kDim * 4 + 1024;
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColP = 0, kColPHi = 128, kColO = 256, kColDS = 384, kColQd = 448;
@@ -91,7 +92,7 @@ constexpr uint32_t kColP = 0, kColPHi = 128, kColO = 256, kColDS = 384, kColQd =
 constexpr int QK_LOADED = 0, VK_LOADED = 1 /* 2 */, P_FULL = 3 /* 2 */, QK_DONE = 5, O_FULL = 6,
               DS_FULL = 7, VK_EMPTY = 8 /* 2 */, P_FREE = 10 /* 2 */, QD_LOCAL = 12, QK_FULL = 13,
               QD_READY = 14, S_READY = 15, O_FREE = 16, VK_READY = 17, DS_FREE = 18, P_CONV = 19 /* 2 */,
-              DRAIN = 21;
+              DRAIN = 21, G_FULL = 22 /* fused norm + gate: a gate half landed in the staging tile */;
 
 constexpr int kBarA = 1, kBarB = 3, kBarW3 = 2;  // named barriers of the three warpgroups
 
@@ -264,6 +265,15 @@ __device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scal
     }
 }
 
+// Normalisation and gating fused into the output epilogue (per-head RMS
+// reading): y[b][l][h*128 + c] = gamma[h*128 + c] o_c / sqrt(mean_c o_c^2 + eps)
+// * sigmoid(gate[b][l][h*128 + c]), written token-major in place of o.
+struct PairNormGate {
+    const __nv_bfloat16 *gate;  // [batch][seq][heads*128]
+    const float *gamma;         // [heads*128]
+    float eps;
+};
+
 // How one launch runs. The forward prefill is {0, 0}; the passes of the
 // backward computation (lightning_api.cu) read the carried state transposed,
 // or run anti-causal. The direction is a template argument of the kernel, so
@@ -276,13 +286,13 @@ struct PairPass {
                      //    token (query factor e^{-s(m-1-i)}, key factor e^{-s(j+1)})
 };
 
-template <bool kAnti>
+template <bool kAnti, bool kNormGate>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_o,
+                    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ slopes, int heads, int seq, const float *state_in,
-                    float *state_out, Snapshots sn, PairPass pp) {
+                    float *state_out, Snapshots sn, PairPass pp, PairNormGate ng) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_addr(smem_raw);
     const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -323,6 +333,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::prefetch_tensormap(&tm_k64);
         ptx::prefetch_tensormap(&tm_v);
         ptx::prefetch_tensormap(&tm_o);
+        if (kNormGate) ptx::prefetch_tensormap(&tm_g);
     }
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -583,6 +594,21 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const size_t sb = (size_t)bh * kDim * kDim;
         // fp16 state operand: K-major rows = value column (l & 63), 64 key dims per box
         uint8_t *srow = c.smem + kOffS + khalf * 8192 + (l & 63) * 128;
+        // fused norm + gate: this head's gamma in shared memory (visible to the group
+        // after the first publish's barrier); the gate reaches the output staging tile
+        // by TMA, 64 channels x 128 tokens at a time
+        const int nb = bh / heads, nh = bh - nb * heads;
+        const float *gsm = reinterpret_cast<const float *>(c.smem + kOffGamma);
+        if (kNormGate) reinterpret_cast<float *>(c.smem + kOffGamma)[l] = ng.gamma[(size_t)nh * kDim + l];
+        // gate half hh of block t into the staging tile, once the previous store has read it
+        int g_issued = 0;  // gate loads issued (leader): the k-th completes G_FULL's phase k
+        auto load_gate = [&](int t, int hh) {
+            ++g_issued;
+            ptx::bulk_wait_read();
+            ptx::mbar_arrive_expect_tx(&c.bars[G_FULL], kBoxBytes);
+            ptx::tma_load_4d(c.smem + kOffE, &tm_g, &c.bars[G_FULL], 64 * hh, nh, tb(t) * kBlock + kRows * (int)rank,
+                             nb);
+        };
         // one 32-value half of this thread's state row: operand copy, optional
         // prefix-cache snapshot and state_out, then the decayed value back into
         // TMEM for the next MMA
@@ -637,6 +663,11 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int t = -1; t < nblk; ++t) {
             const uint32_t par = t & 1;
             const bool last = t + 1 == nblk;
+            if (kNormGate && t >= 0 && leader) {
+                // this block's gate rows into L2 now; the epilogue loads them a block later
+                ptx::tma_prefetch_4d(&tm_g, 0, nh, tb(t) * kBlock + kRows * (int)rank, nb);
+                ptx::tma_prefetch_4d(&tm_g, 64, nh, tb(t) * kBlock + kRows * (int)rank, nb);
+            }
             // S_t is in TMEM once the state MMA is done
             if (t >= 0) {
                 if (!group_wait(c, DS_FULL, par, leader, kBarW3)) goto w3_done;
@@ -671,12 +702,14 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 publish(last);
             }
             if (t < 0) continue;
+            if (kNormGate && leader) load_gate(t, 0);
             // O rows of this CTA: TMEM (fp32) -> bf16 -> staging (128B-swizzled) -> TMA
             // store, 64 value columns at a time; rows past seq are clipped by TMA
             if (!group_wait(c, O_FULL, par, leader, kBarW3)) goto w3_done;
             ptx::tc_fence_after();
             {
                 uint32_t pk[64];  // the whole output row as bf16 pairs
+                float ss = 0.f;   // fused norm + gate: the row's sum of squares (fp32 values)
 #pragma unroll
                 for (int cb = 0; cb < 4; cb += 2) {
                     // two loads in flight per wait: O_FREE is on the path to the next block's first MMA
@@ -686,35 +719,83 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ptx::tmem_ld_wait();
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
-                        pk[16 * cb + u] = ptx::pack_bf16(__uint_as_float(a0[2 * u]), __uint_as_float(a0[2 * u + 1]));
-                        pk[16 * cb + 16 + u] = ptx::pack_bf16(__uint_as_float(a1[2 * u]), __uint_as_float(a1[2 * u + 1]));
+                        const float x0 = __uint_as_float(a0[2 * u]), x1 = __uint_as_float(a0[2 * u + 1]);
+                        const float y0 = __uint_as_float(a1[2 * u]), y1 = __uint_as_float(a1[2 * u + 1]);
+                        pk[16 * cb + u] = ptx::pack_bf16(x0, x1);
+                        pk[16 * cb + 16 + u] = ptx::pack_bf16(y0, y1);
+                        if (kNormGate) {
+                            ss = fmaf(x0, x0, ss);
+                            ss = fmaf(x1, x1, ss);
+                            ss = fmaf(y0, y0, ss);
+                            ss = fmaf(y1, y1, ss);
+                        }
                     }
                 }
                 ptx::tc_fence_before();
                 ptx::named_bar_sync(kBarW3, 128);
                 if (leader) arrive_leader(&c.bars[O_FREE]);
                 uint8_t *erow = c.smem + kOffE + l * 128;
+                const float rstd = kNormGate ? rsqrtf(ss * (1.f / kDim) + ng.eps) : 0.f;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    // the previous store must have finished reading the staging buffer
-                    if (leader) ptx::bulk_wait_read();
-                    ptx::named_bar_sync(kBarW3, 128);
+                    if (kNormGate) {
+                        // y = gamma o rstd sigmoid(g) on this half's 64 columns, written over the
+                        // gate row in the staging tile; sigmoid(g) = 1/2 + tanh(g/2)/2 (SFU tanh)
+                        if (hh == 1 && leader) load_gate(t, 1);
+                        if (!group_wait(c, G_FULL, (uint32_t)hh, leader, kBarW3)) goto w3_done;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        *reinterpret_cast<uint4 *>(erow + ((ch ^ (l & 7)) << 4)) =
-                            make_uint4(pk[32 * hh + 4 * ch], pk[32 * hh + 4 * ch + 1], pk[32 * hh + 4 * ch + 2],
-                                       pk[32 * hh + 4 * ch + 3]);
+                        for (int ch = 0; ch < 8; ++ch) {
+                            uint4 *slot = reinterpret_cast<uint4 *>(erow + ((ch ^ (l & 7)) << 4));
+                            const uint4 g4 = *slot;
+                            const float4 ga = *reinterpret_cast<const float4 *>(gsm + 64 * hh + 8 * ch);
+                            const float4 gb = *reinterpret_cast<const float4 *>(gsm + 64 * hh + 8 * ch + 4);
+                            const float gm[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                            const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+                            uint32_t yw[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const uint32_t w = pk[32 * hh + 4 * ch + e];
+                                float th0, th1;
+                                asm("tanh.approx.f32 %0, %1;" : "=f"(th0) : "f"(0.5f * ptx::bf16_lo(gw[e])));
+                                asm("tanh.approx.f32 %0, %1;" : "=f"(th1) : "f"(0.5f * ptx::bf16_hi(gw[e])));
+                                yw[e] = ptx::pack_bf16(gm[2 * e] * ptx::bf16_lo(w) * rstd * fmaf(0.5f, th0, 0.5f),
+                                                       gm[2 * e + 1] * ptx::bf16_hi(w) * rstd * fmaf(0.5f, th1, 0.5f));
+                            }
+                            *slot = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+                        }
+                    } else {
+                        // the previous store must have finished reading the staging buffer
+                        if (leader) ptx::bulk_wait_read();
+                        ptx::named_bar_sync(kBarW3, 128);
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch)
+                            *reinterpret_cast<uint4 *>(erow + ((ch ^ (l & 7)) << 4)) =
+                                make_uint4(pk[32 * hh + 4 * ch], pk[32 * hh + 4 * ch + 1], pk[32 * hh + 4 * ch + 2],
+                                           pk[32 * hh + 4 * ch + 3]);
+                    }
                     ptx::fence_proxy_async_smem();
                     ptx::named_bar_sync(kBarW3, 128);
                     if (leader) {
-                        ptx::tma_store_3d(&tm_o, c.smem + kOffE, 64 * hh, tb(t) * kBlock + kRows * (int)rank, bh);
+                        if (kNormGate)  // y is token-major: [batch][seq][heads][128]
+                            ptx::tma_store_4d(&tm_o, c.smem + kOffE, 64 * hh, nh, tb(t) * kBlock + kRows * (int)rank,
+                                              nb);
+                        else
+                            ptx::tma_store_3d(&tm_o, c.smem + kOffE, 64 * hh, tb(t) * kBlock + kRows * (int)rank, bh);
                         ptx::bulk_commit();
                     }
                 }
             }
         }
     w3_done:;
-        if (leader) ptx::bulk_wait_all();  // output stores complete before the CTA exits
+        if (leader) {
+            ptx::bulk_wait_all();  // output stores complete before the CTA exits
+            // and the last gate load (if a wait for it was cut short): the k-th load
+            // completes phase k, and the loads go one at a time
+            if (kNormGate && g_issued > 0) {
+                volatile int never = 0;
+                ptx::mbar_wait(&c.bars[G_FULL], (uint32_t)(g_issued - 1) & 1u, &never);
+            }
+        }
     }
 
     ptx::tc_fence_before();
@@ -732,17 +813,51 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 // The CTA-pair kernel covers bf16 inputs, head dim 128 and blocks of 256.
 inline bool pair_supports(bool bf16, int dim, int block) { return bf16 && dim == 128 && block == 256; }
 
+// Tensor map of a token-major output y [batch][seq][heads][128] (bf16), boxes of
+// 64 channels of one head x 128 tokens (rows past seq are clipped on store).
+inline bool make_token_major_map(CUtensorMap *map, void *y, int batch, int heads, int seq, std::string *err) {
+    auto fn = tc::encode_fn(err);
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)pair::kDim, (cuuint64_t)heads, (cuuint64_t)seq, (cuuint64_t)batch};
+    cuuint64_t strides[3] = {(cuuint64_t)pair::kDim * 2, (cuuint64_t)heads * pair::kDim * 2,
+                             (cuuint64_t)seq * heads * pair::kDim * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)pair::kRows, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, y, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *err = "cuTensorMapEncodeTiled (token-major output) failed (CUresult " + std::to_string((int)r) + ")";
+        return false;
+    }
+    return true;
+}
+
+// ng != nullptr: the forward prefill with the normalisation and gating fused into
+// its epilogue; o is then the token-major y.
 inline la_status launch_pair(const void *q, const void *k, const void *v, const float *slopes, int batch,
                              int heads, int seq, const float *state_in, void *o, float *state_out, Snapshots sn,
                              pair::PairPass pp,
-                             cudaStream_t stream, std::string *err) {
+                             cudaStream_t stream, std::string *err, const pair::PairNormGate *ng = nullptr) {
     const long long bh = (long long)batch * heads;
-    CUtensorMap mq, mk, mk64, mv, mo;
+    if (ng && pp.anti) {
+        *err = "the fused normalisation runs on the forward (causal) pass only";
+        return LA_ERR_UNSUPPORTED;
+    }
+    CUtensorMap mq, mk, mk64, mv, mo, mg;
     if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
         !tc::make_map(&mk64, k, seq, bh, err, 64) || !tc::make_map(&mv, v, seq, bh, err) ||
-        !tc::make_map(&mo, o, seq, bh, err))
+        !(ng ? make_token_major_map(&mo, o, batch, heads, seq, err) : tc::make_map(&mo, o, seq, bh, err)))
         return LA_ERR_CUDA;
-    const auto kernel = pp.anti ? pair::prefill_pair_kernel<true> : pair::prefill_pair_kernel<false>;
+    if (ng) {
+        if (!make_token_major_map(&mg, const_cast<__nv_bfloat16 *>(ng->gate), batch, heads, seq, err))
+            return LA_ERR_CUDA;
+    } else {
+        mg = mo;  // unused
+    }
+    const auto kernel = ng        ? pair::prefill_pair_kernel<false, true>
+                        : pp.anti ? pair::prefill_pair_kernel<true, false>
+                                  : pair::prefill_pair_kernel<false, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pair::kSmemBytes);
     if (e != cudaSuccess) {
         *err = std::string("cudaFuncSetAttribute(prefill_pair): ") + cudaGetErrorString(e);
@@ -760,8 +875,9 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mk64, mv, mo, slopes, heads, seq, state_in,
-                           state_out, sn, pp);
+    const pair::PairNormGate ngv = ng ? *ng : pair::PairNormGate{nullptr, nullptr, 0.f};
+    e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mk64, mv, mo, mg, slopes, heads, seq, state_in,
+                           state_out, sn, pp, ngv);
     if (e != cudaSuccess) {
         *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
         return LA_ERR_CUDA;

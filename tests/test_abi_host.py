@@ -244,6 +244,42 @@ def test_norm_gate_empty_needs_no_gpu():
     assert _norm_gate(seq=0, o=None, y=None) == abi.LA_OK
 
 
+def _prefill_norm_gate(**kw):
+    a = dict(GOOD, gate=G_, gamma=GM, eps=1e-6, y=Y_)
+    a.update(kw)
+    return abi.lightning_prefill_norm_gate(a["q"], a["k"], a["v"], a["dtype"], a["slopes"], a["batch"], a["heads"],
+                                           a["seq"], a["dim"], a["block"], a["state_in"], a["gate"], a["gamma"],
+                                           a["eps"], a["y"], a["state_out"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype=5), abi.LA_ERR_INVALID_ARG),
+    (dict(heads=0), abi.LA_ERR_INVALID_ARG),
+    (dict(seq=-2), abi.LA_ERR_INVALID_ARG),
+    (dict(dtype=abi.LA_DTYPE_F32), abi.LA_ERR_UNSUPPORTED),      # the CTA-pair kernel only
+    (dict(block=128), abi.LA_ERR_UNSUPPORTED),
+    (dict(dim=64), abi.LA_ERR_UNSUPPORTED),
+    (dict(eps=-1.0), abi.LA_ERR_INVALID_ARG),
+    (dict(eps=float("inf")), abi.LA_ERR_INVALID_ARG),
+    (dict(y=None), abi.LA_ERR_INVALID_ARG),
+    (dict(gate=None), abi.LA_ERR_INVALID_ARG),
+    (dict(gamma=None), abi.LA_ERR_INVALID_ARG),
+    (dict(gate=G_ + 2), abi.LA_ERR_INVALID_ARG),                  # misaligned
+    (dict(y=Q + 512), abi.LA_ERR_INVALID_ARG),                    # y overlaps q
+    (dict(y=G_ + 1024), abi.LA_ERR_INVALID_ARG),                  # y overlaps the gate
+    (dict(gamma=Y_ + 64), abi.LA_ERR_INVALID_ARG),                # y overlaps gamma
+    (dict(state_out=G_ + 256), abi.LA_ERR_INVALID_ARG),           # state_out overlaps the gate
+])
+def test_prefill_norm_gate_argument_errors(kw, status):
+    assert _prefill_norm_gate(**kw) == status
+    assert abi.last_error_message() != ""
+
+
+def test_prefill_norm_gate_trivial_calls_need_no_gpu():
+    assert _prefill_norm_gate(batch=0) == abi.LA_OK
+    assert _prefill_norm_gate(seq=0, state_out=None, y=None, gate=None, gamma=None) == abi.LA_OK
+
+
 def _gqa(**kw):
     a = dict(q=Q, kn=K, vn=V, kc=0x10000000 * 30, vc=0x10000000 * 40, dtype=abi.LA_DTYPE_BF16, pos=SL, batch=2,
              heads=64, kv=8, dim=128, cap=1024, rot=64, base=1e4, scale=0.088, o=O, ws=WS, ws_bytes=1 << 26)
