@@ -9,7 +9,7 @@ import oracle
 import linear_attention_lightning_b200 as la
 from linear_attention_lightning_b200 import abi, inputs
 
-from parity import TOL, guarded_empty, guards_intact, oracle_prefill, rel_err, to_f64
+from parity import TOL, guarded_empty, guards_intact, half_ulp_bf16, oracle_prefill, rel_err, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -38,6 +38,29 @@ def _oracle_y(o64, gate, gamma, heads_idx=None):
     return oracle.norm_gate(o64.astype(np.float32), g, np.ascontiguousarray(gm.reshape(-1)), EPS, True)
 
 
+def _y_err_in_o_units(y, y_ref, o64, gate, gamma, heads_idx=None):
+    """The error of y carried back to o: |y - y_ref| (less half a bf16 ulp of y) divided by
+    dy/do = |gamma| sigmoid(g) / sqrt(mean o^2 + eps) at the reference, over rms(o).
+
+    y normalises each head's row to unit rms, so an error of o that is small against
+    rms(o) (the prefill's bound, 2e-2 rms(o) for bf16 inputs) becomes large against y
+    on rows whose own rms is small; the fused kernel's y is held to the prefill's bound
+    on o through the exact normalisation. (The normalisation's own fp32 arithmetic and
+    the SFU sigmoid add far less.)"""
+    b, h, L, d = o64.shape
+    g = gate.float().cpu().numpy().reshape(b, L, -1, d)
+    gm = gamma.cpu().numpy().reshape(-1, d)
+    if heads_idx is not None:
+        g, gm = g[:, :, heads_idx], gm[heads_idx]
+    o = np.transpose(o64, (0, 2, 1, 3))                           # [b, L, h, d]
+    rstd = 1.0 / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + EPS)
+    dydo = np.abs(gm)[None, None] / (1.0 + np.exp(-g.astype(np.float64))) * rstd
+    got = np.asarray(y, np.float64).reshape(b, L, h, d)
+    ref = np.asarray(y_ref, np.float64).reshape(b, L, h, d)
+    diff = np.maximum(np.abs(got - ref) - half_ulp_bf16(np.maximum(np.abs(got), np.abs(ref))), 0.0)
+    return float(np.max(diff / dydo)) / float(np.sqrt(np.mean(o64 * o64)))
+
+
 def _run(b, h, L, state_in, seed):
     inp = inputs.prefill_inputs(b, h, L, 128, torch.bfloat16, state_in, seed=seed, device=DEV)
     gate, gamma = _gate_gamma(b, h, L, 128, seed + 1000)
@@ -48,9 +71,11 @@ def _run(b, h, L, state_in, seed):
     assert guards_intact(back, y.numel()), "prefill_norm_gate wrote outside y"
     o64, s64 = oracle_prefill(inp)
     if L > 0:
-        e = rel_err(to_f64(y), _oracle_y(o64, gate, gamma), bf16_out=1)
-        print("prefill_norm_gate b%d h%d L%d: y error %.3g rms" % (b, h, L, e))
-        assert e <= TOL[torch.bfloat16], "y error %.3g rms > %.3g" % (e, TOL[torch.bfloat16])
+        ref = _oracle_y(o64, gate, gamma)
+        e = _y_err_in_o_units(to_f64(y), ref, o64, gate, gamma)
+        print("prefill_norm_gate b%d h%d L%d: error %.3g rms(o) through dy/do (%.3g rms(y) as is)"
+              % (b, h, L, e, rel_err(to_f64(y), ref, bf16_out=1)))
+        assert e <= TOL[torch.bfloat16], "y error %.3g rms(o) through dy/do > %.3g" % (e, TOL[torch.bfloat16])
     es = rel_err(to_f64(s_out), s64)
     assert es <= TOL[torch.bfloat16], "state_out error %.3g rms" % es
     return inp, gate, gamma, y, s_out
@@ -109,8 +134,9 @@ def test_prefill_norm_gate_8k_workload_sampled_heads():
     o64, s64 = oracle_prefill(inp, heads_idx=heads)
     ref = _oracle_y(o64, gate, gamma, heads_idx=heads)
     got = to_f64(y).reshape(w.batch, w.seq, w.heads, w.dim)[:, :, heads].reshape(ref.shape)
-    e = rel_err(got, ref, bf16_out=1)
-    print("prefill_norm_gate 8k sampled heads: y error %.3g rms" % e)
+    e = _y_err_in_o_units(got, ref, o64, gate, gamma, heads_idx=heads)
+    print("prefill_norm_gate 8k sampled heads: error %.3g rms(o) through dy/do (%.3g rms(y) as is)"
+          % (e, rel_err(got, ref, bf16_out=1)))
     assert e <= TOL[torch.bfloat16]
     assert rel_err(to_f64(s_out[:, heads]), s64) <= TOL[torch.bfloat16]
 
