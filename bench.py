@@ -376,7 +376,7 @@ def run_ours(args):
 
     # the same prefill with the per-head normalisation and gate fused into its epilogue
     png = (run_prefill_norm_gate_leg(w, dev, stream, inp, dcode, args, world)
-           if args.norm_gate_steps > 0 and variant == "pair" else None)
+           if args.fused_norm_gate_steps > 0 and variant == "pair" else None)
 
     # decode step of the softmax GQA layer the hybrid model interleaves
     gqa = run_gqa_leg(dev, stream, args, world) if args.gqa_steps > 0 else None
@@ -584,7 +584,7 @@ def run_prefill_norm_gate_leg(w, dev, stream, inp, dcode, args, world):
         torch.cuda.synchronize()
         return max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
 
-    steps = max(1, min(args.norm_gate_steps, 10))
+    steps = max(1, min(args.fused_norm_gate_steps, 10))
     f_ms, t_ms = [], []
     for _ in range(2):
         f_ms.append(timed(fused, steps))
@@ -1005,6 +1005,8 @@ def parse_args(argv=None):
                    help="timed steps of the hybrid-block leg, 7 Lightning + 1 softmax layer (0 skips it)")
     p.add_argument("--norm-gate-steps", type=int, default=20,
                    help="timed steps of the norm-and-gate epilogue leg (0 skips it)")
+    p.add_argument("--fused-norm-gate-steps", type=int, default=10,
+                   help="timed steps of the prefill with the per-head norm + gate fused in (0: skip)")
     p.add_argument("--backward-steps", type=int, default=10,
                    help="timed steps of the gradient leg (0 skips it)")
     p.add_argument("--snapshot-interval", type=int, default=16384,
