@@ -122,3 +122,15 @@ def test_max_over_ranks_on_two_gloo_ranks():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert out == [(0, 2, 11.0), (1, 2, 11.0)]
+
+
+def test_every_stored_traffic_entry_names_a_known_kernel():
+    # each stored counter is looked up by (workload, kernel) and checked against that
+    # kernel's source digest, so its kernel must be one bench.py knows the header of
+    stored = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))["launches"]
+    assert stored
+    for key, entry in stored.items():
+        workload, _, kernel = key.partition("/")
+        assert workload and kernel in bench.KERNEL_SOURCES, key
+        assert len(entry["kernel_source_digest"]) == 16, key
+        assert any(f in entry for f in ("dram_bytes_per_launch", "dram_bytes_per_step")), key
