@@ -72,3 +72,55 @@ def guards_intact(back, n, guard=4096) -> bool:
     head = back[:guard].cpu()
     tail = back[guard + n:].cpu()
     return bool(torch.all(head == sentinel)) and bool(torch.all(tail == sentinel))
+
+
+# The per-head normalisation and gate after a prefill (the fused call's reference).
+NG_EPS = 1e-6
+
+
+def oracle_norm_gate_of(o64, gate, gamma, heads_idx=None):
+    """norm_gate of the oracle's float64 prefill output (per-head mean), on the
+    heads heads_idx (all when None). The oracle's norm_gate reads float32: o is
+    rounded once to float32 (relative 2^-24, far below the bound) and the bf16
+    gate widens exactly."""
+    b, h, L, d = o64.shape
+    g = gate.float().cpu().numpy().reshape(b, L, -1, d)
+    gm = gamma.cpu().numpy().reshape(-1, d)
+    if heads_idx is not None:
+        g, gm = g[:, :, heads_idx], gm[heads_idx]
+    g = np.ascontiguousarray(g.reshape(b, L, h * d))
+    return oracle.norm_gate(o64.astype(np.float32), g, np.ascontiguousarray(gm.reshape(-1)), NG_EPS, True)
+
+
+# Absolute error allowed for sigmoid(g) = 1/2 + tanh(g/2)/2 formed with the SFU's tanh
+# approximation: twice the ~2.5e-4 measured against the exact function.
+SIGMOID_ABS_ERR = 5e-4
+
+
+def norm_gate_y_err_in_o_units(y, y_ref, o64, gate, gamma, heads_idx=None):
+    """The error of y carried back to o, over rms(o): (|y - y_ref| - allowance) / dy/do,
+    dy/do = |gamma| sigmoid(g) / sqrt(mean o^2 + eps) at the reference.
+
+    y normalises each head's row to unit rms, so an error of o that is small against
+    rms(o) (the prefill's bound, 2e-2 rms(o) for bf16 inputs) becomes large against y
+    on rows whose own rms is small; the fused kernel's y is held to the prefill's bound
+    on o through the exact normalisation. The allowance excludes, as the bound on o
+    does, the rounding of the formats (half a bf16 ulp of y, and half a bf16 ulp of o
+    through dy/do: y is formed from o rounded to bf16, as in the two-call path), and
+    the sigmoid's absolute error times |gamma o / rms(o_row)|, which dividing by
+    sigmoid(g) would otherwise magnify where g is very negative."""
+    b, h, L, d = o64.shape
+    g = gate.float().cpu().numpy().reshape(b, L, -1, d)
+    gm = gamma.cpu().numpy().reshape(-1, d)
+    if heads_idx is not None:
+        g, gm = g[:, :, heads_idx], gm[heads_idx]
+    o = np.transpose(o64, (0, 2, 1, 3))                           # [b, L, h, d]
+    rstd = 1.0 / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + NG_EPS)
+    sig = 1.0 / (1.0 + np.exp(-g.astype(np.float64)))
+    dydo = np.abs(gm)[None, None] * sig * rstd
+    got = np.asarray(y, np.float64).reshape(b, L, h, d)
+    ref = np.asarray(y_ref, np.float64).reshape(b, L, h, d)
+    allow = (half_ulp_bf16(np.maximum(np.abs(got), np.abs(ref))) + dydo * half_ulp_bf16(o)
+             + np.abs(gm)[None, None] * np.abs(o) * rstd * SIGMOID_ABS_ERR)
+    diff = np.maximum(np.abs(got - ref) - allow, 0.0)
+    return float(np.max(diff / dydo)) / float(np.sqrt(np.mean(o64 * o64)))
