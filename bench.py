@@ -138,18 +138,102 @@ def summarize_clocks(rows):
             "reasons": sorted(reasons), "samples": len(loaded)}
 
 
+class NvmlPoller:
+    """Reads one GPU's SM clock, power draw and clock-event reasons through NVML every
+    `period` seconds from a thread, in the rows summarize_clocks takes. Queries only: no
+    setting of the GPU is changed. A timed region of tens of milliseconds falls between
+    the samples of nvidia-smi's 200 ms loop; this one lands several inside it. Any NVML
+    failure leaves it empty (ok False), and the caller falls back to nvidia-smi."""
+
+    REASONS = (("hw_slowdown", "HwSlowdown"), ("hw_thermal_slowdown", "HwThermalSlowdown"),
+               ("sw_thermal_slowdown", "SwThermalSlowdown"), ("sw_power_cap", "SwPowerCap"))
+
+    def __init__(self, bus_id=None, index=0, period=0.002, nvml=None):
+        self.bus_id, self.index, self.period, self.nv = bus_id, index, period, nvml
+        self.rows = []
+        self.ok = False
+        self._stop = threading.Event()
+        self._thread = None
+        self._sample = None
+
+    def start(self):
+        try:
+            nv = self.nv
+            if nv is None:
+                import pynvml as nv
+                self.nv = nv
+            nv.nvmlInit()
+            self.ok = True  # initialised: stop() shuts NVML down again
+            h = (nv.nvmlDeviceGetHandleByPciBusId(self.bus_id) if self.bus_id
+                 else nv.nvmlDeviceGetHandleByIndex(self.index))
+            reasons = (getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                       or nv.nvmlDeviceGetCurrentClocksThrottleReasons)
+            bits = {name: (getattr(nv, "nvmlClocksEventReason" + suffix, None)
+                           or getattr(nv, "nvmlClocksThrottleReason" + suffix)) for name, suffix in self.REASONS}
+            sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+            def sample():
+                r = int(reasons(h))
+                row = {"sm_mhz": float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), "sm_max_mhz": sm_max,
+                       "power_w": nv.nvmlDeviceGetPowerUsage(h) / 1000.0}
+                for name, bit in bits.items():
+                    row[name] = "Active" if r & int(bit) else "Not Active"
+                return row
+
+            sample()  # a query that is not available fails here, before the thread starts
+            self._sample = sample
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception:
+            self.stop()
+            self.ok = False
+        return self
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.rows.append(self._sample())
+            except Exception:
+                return
+            self._stop.wait(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+            self._thread = None
+        if self.ok and self.nv is not None:
+            try:
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
+
+
+def pci_bus_id_of(dev):
+    """The PCI bus id of a torch CUDA device ("00000000:1B:00.0"), or None: NVML's
+    device order need not follow CUDA_VISIBLE_DEVICES, the bus id does not depend on it."""
+    try:
+        import torch
+        p = torch.cuda.get_device_properties(dev)
+        return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        return None
+
+
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples clocks and throttle reasons while the timed region runs: NVML every 2 ms
+    (NvmlPoller), with nvidia-smi's loop as the fallback when NVML is not available."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, bus_id=None, nvml=None):
         self.gpu_index = gpu_index
         self.rows = []
         self.proc = None
         self.thread = None
+        self.poller = NvmlPoller(bus_id=bus_id, index=gpu_index, nvml=nvml)
 
     def __enter__(self):
         try:
@@ -161,6 +245,7 @@ class ClockSampler:
             self.thread.start()
         except OSError:
             self.proc = None
+        self.poller.start()
         return self
 
     def _read(self):
@@ -177,6 +262,7 @@ class ClockSampler:
                 continue
 
     def __exit__(self, *exc):
+        self.poller.stop()  # at the end of the timed region
         if self.proc is not None:
             time.sleep(0.3)
             self.proc.terminate()
@@ -189,7 +275,13 @@ class ClockSampler:
         return False
 
     def summary(self):
-        return summarize_clocks(self.rows)
+        if len(self.poller.rows) >= 3:
+            out = summarize_clocks(self.poller.rows)
+            out["source"] = "nvml every 2 ms over the timed region"
+        else:
+            out = summarize_clocks(self.rows)
+            out["source"] = "nvidia-smi -lms 200"
+        return out
 
 
 # ---------------------------------------------------------------- ranks
@@ -336,7 +428,7 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(local_rank, bus_id=pci_bus_id_of(dev)) as clk:
         barrier(world)
         torch.cuda.synchronize()
         ev[0].record(stream)

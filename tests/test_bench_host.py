@@ -134,3 +134,66 @@ def test_every_stored_traffic_entry_names_a_known_kernel():
         assert workload and kernel in bench.KERNEL_SOURCES, key
         assert len(entry["kernel_source_digest"]) == 16, key
         assert any(f in entry for f in ("dram_bytes_per_launch", "dram_bytes_per_step")), key
+
+
+class _FakeNvml:
+    """Stands in for pynvml: one GPU at bus 00000000:1B:00.0, SM clock 1965 of 1965 MHz,
+    800 W, the power cap the only active clock-event reason. Records what it is asked."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonSwPowerCap = 0x4
+
+    def __init__(self, fail_init=False):
+        self.fail_init, self.calls, self.inited = fail_init, [], 0
+
+    def nvmlInit(self):
+        if self.fail_init:
+            raise RuntimeError("no driver")
+        self.inited += 1
+
+    def nvmlShutdown(self):
+        self.inited -= 1
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus):
+        self.calls.append(("bus", bus))
+        return "gpu"
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        self.calls.append(("index", i))
+        return "gpu"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 800000
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x4 | 0x1  # power cap, plus a reason the bench does not report (idle)
+
+
+def test_clock_sampler_reads_nvml_over_the_timed_region():
+    import time
+    nv = _FakeNvml()
+    with bench.ClockSampler(0, bus_id="00000000:1B:00.0", nvml=nv) as clk:
+        time.sleep(0.03)
+    s = clk.summary()
+    assert ("bus", "00000000:1B:00.0") in nv.calls and nv.inited == 0
+    assert s["source"].startswith("nvml") and s["samples"] >= 3
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0 and s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_falls_back_when_nvml_is_unavailable():
+    nv = _FakeNvml(fail_init=True)
+    with bench.ClockSampler(0, nvml=nv) as clk:
+        pass
+    s = clk.summary()
+    assert s["source"].startswith("nvidia-smi") and not clk.poller.ok
+    # no nvidia-smi on a host without a GPU either: reported as not sampled, not invented
+    if not clk.rows:
+        assert s["reasons"] == ["not sampled"] and s["sm_mhz"] is None
