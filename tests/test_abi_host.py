@@ -365,3 +365,22 @@ def test_gqa_prefill_workspace_size_and_empty_calls():
     assert abi.lightning_gqa_prefill_workspace_size(7, 2, 64, 512, 128) == 0
     assert _gqp(batch=0) == abi.LA_OK
     assert _gqp(seq=0, q=None, o=None, ws=None) == abi.LA_OK
+
+
+def test_the_header_is_c_and_matches_the_library(tmp_path):
+    # a plain C program against include/lightning.h, linked with the library
+    import os
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    libdir = os.path.dirname(abi.LIBRARY)
+    exe = str(tmp_path / "abi_from_c")
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                    os.path.join(here, "c", "abi_from_c.c"), "-o", exe, "-L", libdir, "-llightning",
+                    "-Wl,-rpath," + libdir], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
