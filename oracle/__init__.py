@@ -15,6 +15,10 @@ marshals numpy arrays into it.
 
 Inputs are numpy arrays: float32, or uint16 holding bfloat16 bit patterns.
 Outputs are float64.
+
+LA_ORACLE_LIBRARY, when set, names a compiled oracle to load instead of building
+this one: the mutation tests point it at copies with a planted mistake, to show
+that the pins reject them.
 """
 import ctypes
 import os
@@ -30,7 +34,7 @@ _lib = None
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(_build())
+        lib = ctypes.CDLL(os.environ.get("LA_ORACLE_LIBRARY") or _build())
         vp, ip, fp, dp = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
         for name in ("la_oracle_definition", "la_oracle_recurrence"):
             fn = getattr(lib, name)
