@@ -197,3 +197,28 @@ def test_clock_sampler_falls_back_when_nvml_is_unavailable():
     # no nvidia-smi on a host without a GPU either: reported as not sampled, not invented
     if not clk.rows:
         assert s["reasons"] == ["not sampled"] and s["sm_mhz"] is None
+
+
+def test_reference_arm_prints_one_contract_line_on_rank_zero_only():
+    # the reference arm times the oracle on the host cores: one JSON line with the
+    # contract's keys on rank 0, nothing (and exit 0) on the other ranks
+    import subprocess
+    import sys
+    cmd = [sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+           "--warmup", "3"]
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, env=env, cwd=bench.ROOT)
+    assert r.returncode == 0 and r.stdout.strip() == "", r.stderr[-500:]
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE")}
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=env, cwd=bench.ROOT)
+    assert r.returncode == 0, r.stderr[-500:]
+    lines = [x for x in r.stdout.splitlines() if x.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["steps"] == 1 and d["value"] > 0
+    assert d["config"]["workload"] == bench.PREFILL_WORKLOAD
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
