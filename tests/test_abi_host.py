@@ -384,3 +384,33 @@ def test_the_header_is_c_and_matches_the_library(tmp_path):
                     "-Wl,-rpath," + libdir], check=True)
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+
+
+def test_the_binding_has_no_cpu_path():
+    # every entry point refuses host tensors instead of computing on the CPU
+    import torch
+    import linear_attention_lightning_b200 as la
+    x = torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16)
+    sl = torch.ones(2)
+    calls = [
+        lambda: la.prefill(x, x, x, sl, 256),
+        lambda: la.prefill_snapshots(x, x, x, sl, 256, 256),
+        lambda: la.prefill_backward(x, x, x, x, sl, 256),
+        lambda: la.prefill_norm_gate(x, x, x, sl, 256, torch.zeros((1, 8, 256), dtype=torch.bfloat16),
+                                     torch.ones(256)),
+        lambda: la.norm_gate(x, torch.zeros((1, 8, 256), dtype=torch.bfloat16), torch.ones(256)),
+        lambda: la.decode(x[:, :, 0], x[:, :, 0], x[:, :, 0], sl, torch.zeros((1, 2, 128, 128))),
+        lambda: la.gqa_decode(x[:, :, 0], x[:, :1, 0], x[:, :1, 0], x[:, :1], x[:, :1],
+                              torch.zeros(1, dtype=torch.int32)),
+        lambda: la.gqa_prefill(x, x[:, :1], x[:, :1], x[:, :1], x[:, :1]),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
+
+
+def test_a_missing_library_raises(monkeypatch, tmp_path):
+    monkeypatch.setattr(abi, "LIBRARY", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(abi, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        abi.load()
