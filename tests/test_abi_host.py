@@ -414,3 +414,81 @@ def test_a_missing_library_raises(monkeypatch, tmp_path):
     monkeypatch.setattr(abi, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         abi.load()
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor on a machine without a GPU: the binding's checks
+    read only shape, dtype, device and contiguity, and must reject a bad argument
+    before anything is allocated or called."""
+
+    def __init__(self, shape, dtype, index=0):
+        import torch
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+        self.device = torch.device("cuda", index)
+        self.is_cuda = True
+
+    def dim(self):
+        return len(self.shape)
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):  # pragma: no cover - never reached: the checks raise first
+        raise AssertionError("a pointer was taken before the arguments were checked")
+
+
+def _fake_args():
+    import torch
+    b, h, L, d = 1, 2, 8, 128
+    bf = torch.bfloat16
+    return {
+        "q": _FakeCuda((b, h, L, d), bf), "k": _FakeCuda((b, h, L, d), bf), "v": _FakeCuda((b, h, L, d), bf),
+        "slopes": _FakeCuda((h,), torch.float32), "state": _FakeCuda((b, h, d, d), torch.float32),
+        "o": _FakeCuda((b, h, L, d), bf), "gate": _FakeCuda((b, L, h * d), bf),
+        "gamma": _FakeCuda((h * d,), torch.float32), "y": _FakeCuda((b, L, h * d), bf),
+    }
+
+
+@pytest.mark.parametrize("case", [
+    "short_slopes", "long_slopes", "o_shape", "o_dtype", "state_out_shape", "state_in_other_gpu",
+    "q_other_gpu", "o_other_gpu", "snapshots_shape", "y_shape", "decode_o_shape", "decode_state_shape",
+    "decode_slopes",
+])
+def test_the_binding_checks_every_tensor_before_calling(monkeypatch, case):
+    # a short slopes vector, an undersized output, or a tensor on another GPU would let
+    # the kernel read or write out of bounds or touch a peer's memory: the binding
+    # must refuse them, since the C layer sees raw pointers only
+    import torch
+    import linear_attention_lightning_b200.api as api
+    monkeypatch.setattr(api, "_current_device", lambda: 0)
+    a = _fake_args()
+    q, k, v, sl, st, o = a["q"], a["k"], a["v"], a["slopes"], a["state"], a["o"]
+    bad_st = _FakeCuda((1, 2, 128, 64), torch.float32)
+    calls = {
+        "short_slopes": lambda: api.prefill(q, k, v, _FakeCuda((1,), torch.float32), 256, o=o, state_out=st),
+        "long_slopes": lambda: api.prefill(q, k, v, _FakeCuda((3,), torch.float32), 256, o=o, state_out=st),
+        "o_shape": lambda: api.prefill(q, k, v, sl, 256, o=_FakeCuda((1, 2, 4, 128), torch.bfloat16)),
+        "o_dtype": lambda: api.prefill(q, k, v, sl, 256, o=_FakeCuda((1, 2, 8, 128), torch.float32)),
+        "state_out_shape": lambda: api.prefill(q, k, v, sl, 256, o=o, state_out=bad_st),
+        "state_in_other_gpu": lambda: api.prefill(q, k, v, sl, 256, state_in=_FakeCuda(st.shape, torch.float32, 1)),
+        "q_other_gpu": lambda: api.prefill(_FakeCuda(q.shape, torch.bfloat16, 1), k, v, sl, 256),
+        "o_other_gpu": lambda: api.prefill(q, k, v, sl, 256, o=_FakeCuda(o.shape, torch.bfloat16, 1)),
+        "snapshots_shape": lambda: api.prefill_snapshots(q, k, v, sl, 256, 4, o=o, state_out=st,
+                                                         snapshots=_FakeCuda((1, 2, 1, 128, 128), torch.float32)),
+        "y_shape": lambda: api.prefill_norm_gate(q, k, v, sl, 256, a["gate"], a["gamma"],
+                                                 y=_FakeCuda((1, 8, 128), torch.bfloat16)),
+        "decode_o_shape": lambda: api.decode(_FakeCuda((1, 2, 128), torch.bfloat16),
+                                             _FakeCuda((1, 2, 128), torch.bfloat16),
+                                             _FakeCuda((1, 2, 128), torch.bfloat16), sl, st,
+                                             o=_FakeCuda((1, 1, 128), torch.bfloat16)),
+        "decode_state_shape": lambda: api.decode(_FakeCuda((1, 2, 128), torch.bfloat16),
+                                                 _FakeCuda((1, 2, 128), torch.bfloat16),
+                                                 _FakeCuda((1, 2, 128), torch.bfloat16), sl, bad_st),
+        "decode_slopes": lambda: api.decode(_FakeCuda((1, 2, 128), torch.bfloat16),
+                                            _FakeCuda((1, 2, 128), torch.bfloat16),
+                                            _FakeCuda((1, 2, 128), torch.bfloat16),
+                                            _FakeCuda((1,), torch.float32), st),
+    }
+    with pytest.raises(ValueError):
+        calls[case]()
