@@ -6,10 +6,16 @@ One step = one lightning_prefill call over the long-context workload
 (batch 1, 64 heads, 131072 tokens, head dim 128, block 256, bf16 q/k/v/o,
 fp32 state), inputs resident in HBM. The same run also times the decode
 workload (64 sequences x 64 heads x 128, fp32 states, 1000 consecutive
-single-token steps) and the end-to-end path with host buffers. Rank 0 prints
-one JSON line. With --gpus N (under torchrun) every rank runs an independent
-replica of the workload ("replicas only": the path has no exchange step);
-times are the max over ranks.
+single-token steps) and the end-to-end path with host buffers; these go into
+the contract line, which rank 0 prints last. Auxiliary legs (snapshots, the
+norm-and-gate epilogue, the softmax GQA layer, the other workloads, the
+hybrid block, the backward) come before it, one JSON line each
+({"aux": name, "result": ...}). After every timed region the library's status
+word is checked on every rank: a leg whose kernels recorded a failure is no
+measurement (the prefill and decode legs then end the run; an auxiliary leg
+is reported as failed). With --gpus N (under torchrun) every rank runs an
+independent replica of the workload ("replicas only": the path has no
+exchange step); times are the max over ranks.
 
 `--impl reference` times the float64 CPU oracle on the host cores on a
 bounded sample of the same workload (rank 0 only).
@@ -57,6 +63,17 @@ def decode_bytes(batch, heads, dim, elem_bytes=2):
     """Algorithmic HBM bytes of one decode step: the fp32 state read and
     written once, q, k, v read and o written once."""
     return batch * heads * (2 * dim * dim * 4 + 4 * dim * elem_bytes)
+
+
+def workload_config(w, world):
+    """The contract line's config, the same for both arms: the workload by name
+    and sizes, how the run is spread over GPUs, and how L2 is kept out of the
+    timing (every step streams more than L2 holds)."""
+    by = prefill_bytes(w.batch, w.heads, w.seq, w.dim, 2 if "bf16" in str(w.dtype) else 4,
+                       state_in=w.state_in, state_out=True)
+    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": w.seq, "dim": w.dim,
+            "block": w.block, "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (%.1f GB per step)" % (by / 1e9)}
 
 
 def load_peaks():
@@ -315,6 +332,48 @@ def max_over_ranks(value, world, device="cpu"):
     return float(t.item())
 
 
+class LegFailed(RuntimeError):
+    """A timed leg whose kernels recorded a failure in the status word."""
+
+
+def check_device_status(leg, abi, stream_handle, world, device="cpu"):
+    """After a timed region: the library's status word must be clean on every
+    rank. A kernel whose bounded wait ran out returns early, and its time would
+    read as a fast step, so such a leg is no measurement. Collective (every
+    rank takes the same step), then raises on every rank if any rank failed."""
+    st = abi.lightning_last_device_status(stream_handle)
+    worst = max_over_ranks(0.0 if st == abi.LA_OK else float(st), world, device)
+    if worst:
+        raise LegFailed("%s: a kernel recorded %s during the timed region" % (leg, abi.status_string(int(worst))))
+
+
+def timed(leg, step, steps, warmup, stream, world, device):
+    """`warmup` untimed calls, then `steps` calls between CUDA events on
+    `stream`, bracketed by a barrier and a synchronisation; the status word is
+    checked afterwards. Returns milliseconds per step, the max over ranks."""
+    import torch
+    from linear_attention_lightning_b200 import abi
+    for _ in range(warmup):
+        step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device) / steps
+    check_device_status(leg, abi, stream.cuda_stream, world, device)
+    return ms
+
+
+def aux_line(name, result):
+    """One auxiliary leg's result as its own JSON line, printed before the
+    contract line so that the contract line stays short."""
+    return json.dumps({"aux": name, "result": result})
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_sample(w, tokens, heads, threads=None, h0=0):
@@ -384,8 +443,7 @@ def run_reference(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1000 * tot / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": w.seq,
-                       "dim": w.dim, "block": w.block, "inputs": "bf16 q,k,v widened to float64"},
+            "config": workload_config(w, world), "inputs": "bf16 q,k,v widened to float64",
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
                              "kind": "oracle",
                              "sample": "%d of %d heads x %d tokens per step" % (heads, w.heads, tokens)},
@@ -417,6 +475,7 @@ def run_ours(args):
     vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05,
              "pair": abi.LA_VARIANT_TCGEN05_PAIR}[variant]
     dcode = abi.LA_DTYPE_BF16 if w.dtype == torch.bfloat16 else abi.LA_DTYPE_F32
+    launches_per_step = 1   # kernels one lightning_prefill_ex call launches
 
     def step():
         abi.check(abi.lightning_prefill_ex(
@@ -440,6 +499,7 @@ def run_ours(args):
     per_launch_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     total_ms = ev[0].elapsed_time(ev[-1])
     total_ms = max_over_ranks(total_ms, world, dev)
+    check_device_status("prefill", abi, sp, world, dev)
     ms_per_step = total_ms / args.steps
     tokens = w.batch * w.seq
     value = world * tokens * args.steps / (total_ms / 1e3)
@@ -454,51 +514,57 @@ def run_ours(args):
 
     # decode: 1000 consecutive single-token steps over fp32 states
     dw = inputs.WORKLOADS[DECODE_WORKLOAD]
-    dec = run_decode(dw, dev, stream, peaks, args) if args.decode_steps > 0 else None
+    dec = run_decode(dw, dev, stream, peaks, args, world) if args.decode_steps > 0 else None
 
     # end to end: host buffers, copies inside the timed region
     e2e = run_e2e(w, dev, stream, inp, variant, args, world) if args.e2e_steps > 0 else None
 
+    # Auxiliary legs, each printed on a line of its own before the contract line.
+    # A leg whose kernels recorded a failure is reported as failed (on every rank
+    # alike) and the run goes on; the contract line lists the failed legs.
+    failed = []
+
+    def aux(name, enabled, fn):
+        if not enabled:
+            return
+        try:
+            r = fn()
+        except LegFailed as exc:
+            failed.append(name)
+            r = {"failed": str(exc)}
+        if rank == 0:
+            print(aux_line(name, r), flush=True)
+
     # the same prefill keeping prefix-cache snapshots of the state
-    snaps = (run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, ms_per_step)
-             if args.snapshot_interval > 0 and w.seq >= args.snapshot_interval else None)
-
+    aux("snapshots", args.snapshot_interval > 0 and w.seq >= args.snapshot_interval,
+        lambda: run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, ms_per_step))
     # normalisation and gating of the prefill's output
-    ng = run_norm_gate_leg(w, dev, stream, o, dcode, args, world) if args.norm_gate_steps > 0 else None
-
+    aux("norm_gate", args.norm_gate_steps > 0, lambda: run_norm_gate_leg(w, dev, stream, o, dcode, args, world))
     # the same prefill with the per-head normalisation and gate fused into its epilogue
-    png = (run_prefill_norm_gate_leg(w, dev, stream, inp, dcode, args, world)
-           if args.fused_norm_gate_steps > 0 and variant == "pair" else None)
-
-    # decode step of the softmax GQA layer the hybrid model interleaves
-    gqa = run_gqa_leg(dev, stream, args, world) if args.gqa_steps > 0 else None
-
-    # prefill of the softmax GQA layer at the same context length
-    gqp = run_gqa_prefill_leg(dev, stream, args, world) if args.gqa_prefill_steps > 0 else None
-
+    aux("prefill_norm_gate", args.fused_norm_gate_steps > 0 and variant == "pair",
+        lambda: run_prefill_norm_gate_leg(w, dev, stream, inp, dcode, args, world))
+    # decode step and prefill of the softmax GQA layer the hybrid model interleaves
+    aux("gqa_decode", args.gqa_steps > 0, lambda: run_gqa_leg(dev, stream, args, world))
+    aux("gqa_prefill", args.gqa_prefill_steps > 0, lambda: run_gqa_prefill_leg(dev, stream, args, world))
     # the other prefill workloads: many short sequences with carried-in states; 8192 tokens
-    others = ({n: run_workload_leg(n, dev, stream, peaks, args, world)
-               for n in ("batched_prefill_state", "m1_prefill_8k") if n != w.name}
-              if args.batched_steps > 0 else None)
-
+    for n in ("batched_prefill_state", "m1_prefill_8k"):
+        aux("other_workloads/" + n, args.batched_steps > 0 and n != w.name,
+            lambda n=n: run_workload_leg(n, dev, stream, peaks, args, world))
     # one block of the hybrid model's attention: 7 Lightning layers and 1 softmax layer
-    hyb = (run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world)
-           if args.hybrid_steps > 0 and w.dtype == torch.bfloat16 and w.dim == 128 else None)
-
-    hyd = run_hybrid_decode_leg(dev, stream, args, world) if args.hybrid_steps > 0 and args.gqa_steps > 0 else None
-
+    aux("hybrid_block", args.hybrid_steps > 0 and w.dtype == torch.bfloat16 and w.dim == 128,
+        lambda: run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world))
+    aux("hybrid_decode", args.hybrid_steps > 0 and args.gqa_steps > 0,
+        lambda: run_hybrid_decode_leg(dev, stream, args, world))
     # gradients of the same prefill (dq, dk, dv, d state_in)
-    bwd = run_backward_leg(w, dev, stream, inp, dcode, args, world) if args.backward_steps > 0 else None
+    aux("backward", args.backward_steps > 0, lambda: run_backward_leg(w, dev, stream, inp, dcode, args, world))
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": w.seq,
-                   "dim": w.dim, "block": w.block, "kernel": variant,
-                   "parallelism": "replicas" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (%.1f GB per step)" % (by / 1e9)},
+        "config": workload_config(w, world),
+        "kernel": variant,
         "tflops": {"formula": round(tflops["formula"], 2), "causal": round(tflops["causal"], 2),
                    "peak_bf16": peaks["bf16_tflops"],
                    "frac_formula": round(tflops["formula"] / peaks["bf16_tflops"], 4),
@@ -507,16 +573,8 @@ def run_ours(args):
         "roofline": roofline("hbm", gbs, peaks["hbm_gbs"], "GB/s", traffic),
         "decode": dec,
         "e2e": e2e,
-        "snapshots": snaps,
-        "norm_gate": ng,
-        "prefill_norm_gate": png,
-        "gqa_decode": gqa,
-        "gqa_prefill": gqp,
-        "other_workloads": others,
-        "hybrid_block": hyb,
-        "hybrid_decode": hyd,
-        "backward": bwd,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step,
+        "aux_legs_failed": failed,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -528,7 +586,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_decode(dw, dev, stream, peaks, args):
+def run_decode(dw, dev, stream, peaks, args, world=1):
     import torch
     from linear_attention_lightning_b200 import abi, inputs
     steps = args.decode_steps
@@ -549,12 +607,15 @@ def run_decode(dw, dev, stream, peaks, args):
         one(t)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
     e0.record(stream)
     for t in range(steps):
         one(t)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    check_device_status("decode", abi, sp, world, dev)
     by = decode_bytes(dw.batch, dw.heads, dw.dim)
     gbs = by * steps / (ms / 1e3) / 1e9
     del tok
@@ -583,18 +644,8 @@ def run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, plain_ms):
             w.block, None if s0 is None else s0.data_ptr(), o.data_ptr(), s_out.data_ptr(), interval,
             snaps.data_ptr(), sp, vcode))
 
-    for _ in range(args.warmup):
-        step()
     steps = max(1, min(args.steps, 10))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    ms = timed("snapshots", step, steps, args.warmup, stream, world, dev)
     return {"interval": interval, "count": n, "steps": steps, "ms_per_step": round(ms, 4),
             "overhead_vs_plain_pct": round(100.0 * (ms / plain_ms - 1.0), 2),
             "snapshot_bytes_per_step": int(snaps.numel() * 4)}
@@ -615,18 +666,8 @@ def run_norm_gate_leg(w, dev, stream, o, dcode, args, world):
         abi.check(abi.lightning_norm_gate(o.data_ptr(), gate.data_ptr(), dcode, gamma.data_ptr(), 1e-6, w.batch,
                                           w.heads, w.seq, w.dim, 0, y.data_ptr(), sp))
 
-    for _ in range(args.warmup):
-        step()
     steps = args.norm_gate_steps
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    ms = timed("norm_gate", step, steps, args.warmup, stream, world, dev)
     by = 3 * o.numel() * o.element_size() + gamma.numel() * 4  # o, gate read; y written
     gbs = by / (ms / 1e3) / 1e9
     return {"steps": steps, "ms_per_step": round(ms, 4), "per": "token (heads*dim channels)",
@@ -663,24 +704,11 @@ def run_prefill_norm_gate_leg(w, dev, stream, inp, dcode, args, world):
         abi.check(abi.lightning_norm_gate(o.data_ptr(), gate.data_ptr(), dcode, gamma.data_ptr(), 1e-6, w.batch,
                                           w.heads, w.seq, w.dim, 1, y.data_ptr(), sp))
 
-    def timed(fn, steps):
-        for _ in range(args.warmup):
-            fn()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(steps):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        return max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
-
     steps = max(1, min(args.fused_norm_gate_steps, 10))
     f_ms, t_ms = [], []
     for _ in range(2):
-        f_ms.append(timed(fused, steps))
-        t_ms.append(timed(two_calls, steps))
+        f_ms.append(timed("prefill_norm_gate", fused, steps, args.warmup, stream, world, dev))
+        t_ms.append(timed("prefill_norm_gate/two_calls", two_calls, steps, args.warmup, stream, world, dev))
     ms, ms2 = min(f_ms), min(t_ms)
     n = q.numel() * q.element_size()
     by = 5 * n + gamma.numel() * 4 + (0 if s0 is None else 2 * s0.numel() * 4)  # q, k, v, gate in; y out
@@ -718,18 +746,8 @@ def run_gqa_leg(dev, stream, args, world):
                                            abi.LA_DTYPE_BF16, pos.data_ptr(), b, h, hk, d, cap, 64, 1e4,
                                            1.0 / d ** 0.5, o.data_ptr(), ws.data_ptr(), need, sp))
 
-    for _ in range(args.warmup):
-        step()
     steps = args.gqa_steps
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    ms = timed("gqa_decode", step, steps, args.warmup, stream, world, dev)
     # algorithmic bytes: the cache read for positions 0..cap-1 (K and V), the new k, v
     # written, q read and o written
     by = 2 * b * hk * cap * d * 2 + 2 * b * hk * d * 2 + 2 * b * h * d * 2
@@ -765,18 +783,8 @@ def run_gqa_prefill_leg(dev, stream, args, world):
                                             abi.LA_DTYPE_BF16, 0, b, h, hk, L, d, L, 64, 1e4, 1.0 / d ** 0.5,
                                             o.data_ptr(), ws.data_ptr(), need, sp))
 
-    for _ in range(args.warmup):
-        step()
     steps = args.gqa_prefill_steps
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    ms = timed("gqa_prefill", step, steps, args.warmup, stream, world, dev)
     peaks = load_peaks()
     causal = 4.0 * d * h * b * L * (L + 1) / 2
     tf = causal / (ms / 1e3) / 1e12
@@ -844,6 +852,7 @@ def run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    check_device_status("hybrid_block", abi, sp, world, dev)
     lightning_ms, softmax_ms = ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2])
     return {"layers": "7 x (Lightning prefill + norm and gate) + 1 x softmax GQA prefill", "steps": steps,
             "ms_per_step": round(ms, 3), "tokens_per_s": round(world * b * L / (ms / 1e3), 1),
@@ -881,18 +890,8 @@ def run_hybrid_decode_leg(dev, stream, args, world):
                                            abi.LA_DTYPE_BF16, pos.data_ptr(), b, h, hk, d, cap, 64, 1e4,
                                            1.0 / d ** 0.5, o.data_ptr(), ws.data_ptr(), need, sp))
 
-    for _ in range(args.warmup):
-        step()
     steps = args.gqa_steps
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    ms = timed("hybrid_decode", step, steps, args.warmup, stream, world, dev)
     return {"layers": "7 x Lightning decode + 1 x softmax GQA decode", "sequences": b, "context": cap,
             "steps": steps, "us_per_step": round(ms * 1e3, 2), "tokens_per_s": round(world * b / (ms / 1e3), 1)}
 
@@ -920,18 +919,8 @@ def run_workload_leg(name, dev, stream, peaks, args, world):
                                            None if s0 is None else s0.data_ptr(), o.data_ptr(), s_out.data_ptr(), None,
                                            0, sp, vcode))
 
-    for _ in range(args.warmup):
-        step()
     steps = args.batched_steps
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    ms = timed("other_workloads/%s" % bw.name, step, steps, args.warmup, stream, world, dev)
     by = prefill_bytes(bw.batch, bw.heads, bw.seq, bw.dim, 2, state_in=s0 is not None, state_out=True)
     gbs = by / (ms / 1e3) / 1e9
     fl = prefill_flops(bw.batch, bw.heads, bw.seq, bw.dim, bw.block)["formula"] / (ms / 1e3) / 1e12
@@ -963,18 +952,8 @@ def run_backward_leg(w, dev, stream, inp, dcode, args, world):
             w.seq, w.dim, w.block, None if s0 is None else s0.data_ptr(), d_so.data_ptr(), dq.data_ptr(),
             dk.data_ptr(), dv.data_ptr(), ds_in.data_ptr(), ws.data_ptr(), need, sp, variant))
 
-    for _ in range(args.warmup):
-        step()
     steps = args.backward_steps
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    ms = timed("backward", step, steps, args.warmup, stream, world, dev)
     peaks = load_peaks()
     eb = 2 if q.dtype == torch.bfloat16 else 4
     # algorithmic bytes: q, k, v, dO read and dq, dk, dv written once, plus the
@@ -1064,6 +1043,8 @@ def run_e2e(w, dev, stream, inp, variant, args, world):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    from linear_attention_lightning_b200 import abi
+    check_device_status("e2e", abi, stream.cuda_stream, world, dev)
     value = world * w.batch * w.seq * steps / (ms / 1e3)
     # the last step's host output is the device prefill's on the same inputs
     ref_o, _ = la.prefill(inp["q"], inp["k"], inp["v"], inp["slopes"], w.block, inp["state_in"], variant=variant)

@@ -35,10 +35,11 @@
  *   - Argument errors are detected on the host and returned before anything
  *     is launched; launch failures return LA_ERR_CUDA. No device-side trap
  *     or abort is ever used: a device-side wait that runs out of its
- *     iteration budget records LA_ERR_TIMEOUT in a device status word, read
- *     back by lightning_device_status(); so does LA_ERR_INVALID_ARG for a
- *     device-side argument the host cannot see (a decode position outside
- *     its cache), whose work is then skipped.
+ *     iteration budget records LA_ERR_TIMEOUT in a status word; so does
+ *     LA_ERR_INVALID_ARG for a device-side argument the host cannot see (a
+ *     decode position outside its cache), whose work is then skipped. The
+ *     next launching call returns that status instead of launching, and
+ *     lightning_last_device_status() returns it on demand (see there).
  *   - A human-readable reason for the last failure on the calling thread is
  *     returned by lightning_last_error_message().
  */
@@ -285,8 +286,30 @@ la_status lightning_decode(const void *q, const void *k, const void *v, la_dtype
                            const float *slopes, int batch, int heads, int dim, float *state,
                            void *o, void *stream);
 
-/* Synchronises `stream`, returns the device status word (LA_OK or
- * LA_ERR_TIMEOUT) recorded by kernels since the last call, and clears it. */
+/*
+ * Failures that kernels record on the device. Source: none in the pages; this
+ * is the library's own failure reporting. A kernel whose bounded wait runs out
+ * records LA_ERR_TIMEOUT, and one that meets an out-of-range device-side
+ * argument records LA_ERR_INVALID_ARG, in a status word; no kernel traps.
+ *
+ * The word is one per process (managed memory), shared by every device,
+ * stream and thread. It is reported in two ways:
+ *   - on the next launching call: every entry point that launches work looks
+ *     at the word, without synchronising anything, just before its first
+ *     launch; if an earlier kernel recorded a failure, the call clears the
+ *     word, launches nothing and returns that status (lightning_last_error_message
+ *     says so). Calls that launch nothing (argument errors, empty problems,
+ *     host-only queries) do not look.
+ *   - on demand: lightning_last_device_status synchronises `stream`, then
+ *     returns the recorded status (LA_OK if none) and clears the word.
+ * Because the word is shared, a failure recorded by a kernel on one stream or
+ * device is returned by whichever call looks first, from any thread, and a
+ * kernel still running when a call looks may record a failure that only the
+ * call after it sees.
+ */
+la_status lightning_last_device_status(void *stream);
+
+/* The same as lightning_last_device_status (kept under its earlier name). */
 la_status lightning_device_status(void *stream);
 
 /*

@@ -47,6 +47,7 @@ _SIGNATURES = {
     "lightning_prefill_backward_noalloc_capacity": ([], _sz),
     "lightning_decode": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp], _i),
     "lightning_device_status": ([_vp], _i),
+    "lightning_last_device_status": ([_vp], _i),
     "lightning_selftest_wait_timeout": ([_vp], _i),
     "lightning_status_string": ([_i], ctypes.c_char_p),
     "lightning_last_error_message": ([], ctypes.c_char_p),
@@ -190,6 +191,10 @@ def lightning_decode(q, k, v, dtype, slopes, batch, heads, dim, state, o, stream
 
 def lightning_device_status(stream):
     return load().lightning_device_status(stream)
+
+
+def lightning_last_device_status(stream):
+    return load().lightning_last_device_status(stream)
 
 
 def lightning_selftest_wait_timeout(stream):

@@ -7,9 +7,13 @@
 
 namespace la {
 
-// Device status word: kernels set LA_ERR_TIMEOUT here when a bounded wait
-// gives up. Read and cleared by lightning_device_status().
-__device__ unsigned int g_device_status;
+// Status word: kernels set LA_ERR_TIMEOUT here when a bounded wait gives up,
+// and kBadDeviceArgFlag when they meet an out-of-range device-side argument.
+// It lives in managed memory, one word for the process, so that the host can
+// read it without synchronising anything: every launching entry point looks
+// at it before it launches, and lightning_last_device_status() reads it after
+// synchronising a stream. Kernels of every device and stream share it.
+__managed__ unsigned int g_device_status;
 // flag in the status word: a kernel met an out-of-range device-side argument
 // (a decode position outside the cache) and skipped the work it governs
 constexpr unsigned int kBadDeviceArgFlag = 1u;

@@ -45,6 +45,26 @@ la_status cuda_fail(cudaError_t e, const char *what) {
     return fail(LA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// The status a kernel recorded in the status word, as an la_status (LA_OK for 0).
+la_status status_of_word(unsigned int word) {
+    if (word & LA_ERR_TIMEOUT)
+        return fail(LA_ERR_TIMEOUT, "a device-side wait of an earlier kernel gave up (status word 0x%x)", word);
+    if (word & la::kBadDeviceArgFlag)
+        return fail(LA_ERR_INVALID_ARG,
+                    "an earlier kernel met an out-of-range device-side argument (status word 0x%x)", word);
+    return LA_OK;
+}
+
+// Called by every entry point just before its first launch (never on a path
+// that launches nothing, so that host-only calls need no CUDA context): a
+// failure an earlier kernel recorded is returned now, the word is cleared, and
+// nothing is launched. The word is read without any synchronisation; a kernel
+// still running may record a failure after this look, and the next call sees it.
+la_status earlier_failure() {
+    if (__atomic_load_n(&la::g_device_status, __ATOMIC_ACQUIRE) == 0u) return LA_OK;
+    return status_of_word(__atomic_exchange_n(&la::g_device_status, 0u, __ATOMIC_ACQ_REL));
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct Range {
@@ -502,10 +522,10 @@ la_status run_backward_typed(const BackwardArgs &a, cudaStream_t stream) {
 }
 
 la_status run_backward(const BackwardArgs &a, cudaStream_t stream, int variant) {
-    if (a.batch == 0) return ok();
+    if (a.batch == 0 || (a.seq == 0 && !a.d_state_in)) return ok();
+    if (const la_status early = earlier_failure()) return early;
     if (a.seq == 0) {
         // no token: the state passes through, and so does its gradient
-        if (!a.d_state_in) return ok();
         const size_t n = (size_t)a.batch * a.heads * a.dim * a.dim;
         la::state_passthrough_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0,
                                        stream>>>(a.d_state_out, a.d_state_in, n);
@@ -520,9 +540,9 @@ la_status run_backward(const BackwardArgs &a, cudaStream_t stream, int variant) 
 }
 
 la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
-    if (a.batch == 0) return ok();
+    if (a.batch == 0 || (a.seq == 0 && !a.state_out)) return ok();
+    if (const la_status early = earlier_failure()) return early;
     if (a.seq == 0) {
-        if (!a.state_out) return ok();
         const size_t n = (size_t)a.batch * a.heads * a.dim * a.dim;
         la::state_passthrough_kernel<<<(unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0,
                                        stream>>>(a.state_in, a.state_out, n);
@@ -686,6 +706,7 @@ la_status lightning_prefill_norm_gate(const void *q, const void *k, const void *
     }
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (batch == 0 || seq == 0) return run_prefill(a, cs, LA_VARIANT_TCGEN05_PAIR);
+    if (const la_status early = earlier_failure()) return early;
     const la::pair::PairNormGate ng{static_cast<const __nv_bfloat16 *>(gate), gamma, eps};
     return la::launch_pair(q, k, v, slopes, batch, heads, seq, state_in, y, state_out, a.sn, la::pair::PairPass{0, 0},
                            cs, &g_last_error, &ng);
@@ -719,6 +740,7 @@ la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, c
     // chunks of 16 bytes per thread, and resident CTAs on every SM, each walking the tokens
     const long long chunks_per_thread = ((long long)heads * dim * (long long)eb / 16 + la::kNgGroup - 1) / la::kNgGroup;
     const int U = chunks_per_thread <= 1 ? 1 : chunks_per_thread <= 2 ? 2 : chunks_per_thread <= 4 ? 4 : 8;
+    if (const la_status early = earlier_failure()) return early;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const NgArgs args{o, gate, gamma, eps, batch, heads, seq, dim, per_head ? 1 : 0, y, tokens, st};
     la_status rs;
@@ -779,6 +801,7 @@ la_status lightning_gqa_decode(const void *q, const void *k_new, const void *v_n
         for (int j = 0; j < 8; ++j)
             if (j != wi && overlaps(all[wi], all[j]))
                 return fail(LA_ERR_INVALID_ARG, "%s overlaps %s", names[wi], names[j]);
+    if (const la_status early = earlier_failure()) return early;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dtype == LA_DTYPE_BF16)
         return run_gqa_decode<__nv_bfloat16>(q, k_new, v_new, k_cache, v_cache, pos, batch, heads, kv_heads, cap, rot,
@@ -832,6 +855,7 @@ la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_
         for (int j = 0; j < 7; ++j)
             if (j != wi && overlaps(all[wi], all[j]))
                 return fail(LA_ERR_INVALID_ARG, "%s overlaps %s", names[wi], names[j]);
+    if (const la_status early = earlier_failure()) return early;
     if (dtype == LA_DTYPE_F32)
         return la::launch_gqa_prefill_f32(q, k_new, v_new, k_cache, v_cache, start, batch, heads, kv_heads, seq, cap,
                                           rot, rope_base, scale, o, workspace, static_cast<cudaStream_t>(stream),
@@ -899,6 +923,7 @@ la_status lightning_decode(const void *q, const void *k, const void *v, la_dtype
         if (overlaps(ro, r)) return fail(LA_ERR_INVALID_ARG, "o overlaps an input");
         if (overlaps(rs, r)) return fail(LA_ERR_INVALID_ARG, "state overlaps an input");
     }
+    if (const la_status early = earlier_failure()) return early;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dtype == LA_DTYPE_BF16)
         return dim == 64 ? launch_decode<__nv_bfloat16, 64>(q, k, v, slopes, batch, heads, state, o, s)
@@ -907,19 +932,14 @@ la_status lightning_decode(const void *q, const void *k, const void *v, la_dtype
                      : launch_decode<float, 128>(q, k, v, slopes, batch, heads, state, o, s);
 }
 
-la_status lightning_device_status(void *stream) {
+la_status lightning_last_device_status(void *stream) {
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-    unsigned int word = 0, zero = 0;
-    e = cudaMemcpyFromSymbol(&word, la::g_device_status, sizeof word);
-    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
-    e = cudaMemcpyToSymbol(la::g_device_status, &zero, sizeof zero);
-    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
-    if (word & LA_ERR_TIMEOUT) return fail(LA_ERR_TIMEOUT, "a device-side wait gave up (status word 0x%x)", word);
-    if (word & la::kBadDeviceArgFlag)
-        return fail(LA_ERR_INVALID_ARG, "a kernel met an out-of-range device-side argument (status word 0x%x)", word);
-    return ok();
+    const la_status st = status_of_word(__atomic_exchange_n(&la::g_device_status, 0u, __ATOMIC_ACQ_REL));
+    return st == LA_OK ? ok() : st;
 }
+
+la_status lightning_device_status(void *stream) { return lightning_last_device_status(stream); }
 
 la_status lightning_selftest_wait_timeout(void *stream) {
     la::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();

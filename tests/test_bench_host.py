@@ -222,3 +222,63 @@ def test_reference_arm_prints_one_contract_line_on_rank_zero_only():
     assert d["config"]["workload"] == bench.PREFILL_WORKLOAD
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+class _FakeAbi:
+    """Stands in for the binding: a status word that reads `status` once."""
+    LA_OK, LA_ERR_TIMEOUT = 0, 4
+
+    def __init__(self, status):
+        self.status, self.asked = status, 0
+
+    def lightning_last_device_status(self, stream):
+        self.asked += 1
+        return self.status
+
+    def status_string(self, st):
+        return {0: "LA_OK", 4: "LA_ERR_TIMEOUT: a device-side wait gave up"}[st]
+
+
+def test_a_leg_whose_kernels_recorded_a_failure_is_not_a_measurement():
+    # a kernel whose bounded wait ran out returns early: its time would read as a fast step
+    ok = _FakeAbi(0)
+    bench.check_device_status("decode", ok, 0, 1)
+    assert ok.asked == 1
+    with pytest.raises(bench.LegFailed, match="decode: a kernel recorded LA_ERR_TIMEOUT"):
+        bench.check_device_status("decode", _FakeAbi(4), 0, 1)
+
+
+def _status_rank_main(rank, port, q):
+    os.environ.update(RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    r, world, _ = bench.dist_setup(2)
+    # only rank 1's kernels recorded a failure; both ranks must fail the leg alike
+    try:
+        bench.check_device_status("backward", _FakeAbi(4 if r == 1 else 0), 0, world)
+        q.put((r, "passed"))
+    except bench.LegFailed:
+        q.put((r, "failed"))
+    bench.barrier(world)   # both ranks are still in step
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_a_failure_on_one_rank_fails_the_leg_on_every_rank():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_status_rank_main, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert out == [(0, "failed"), (1, "failed")]
+
+
+def test_auxiliary_legs_go_on_lines_of_their_own():
+    line = json.loads(bench.aux_line("backward", {"ms_per_step": 1.0}))
+    assert line == {"aux": "backward", "result": {"ms_per_step": 1.0}}
