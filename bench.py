@@ -475,13 +475,17 @@ def run_ours(args):
     vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05,
              "pair": abi.LA_VARIANT_TCGEN05_PAIR}[variant]
     dcode = abi.LA_DTYPE_BF16 if w.dtype == torch.bfloat16 else abi.LA_DTYPE_F32
-    launches_per_step = 1   # kernels one lightning_prefill_ex call launches
+    # kernels one lightning_prefill_ex call launches: the CTA-pair kernel, then its
+    # range guard's second pass (which returns at once for heads it need not redo)
+    launches_per_step = 2 if variant == "pair" else 1
+    need = abi.lightning_prefill_workspace_size(w.batch, w.heads, w.seq, w.dim, w.block)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 
     def step():
         abi.check(abi.lightning_prefill_ex(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads,
             w.seq, w.dim, w.block, None if s0 is None else s0.data_ptr(), o.data_ptr(),
-            s_out.data_ptr(), None, 0, sp, vcode))
+            s_out.data_ptr(), ws.data_ptr(), need, sp, vcode))
 
     for _ in range(args.warmup):
         step()
@@ -636,13 +640,15 @@ def run_snapshots(w, dev, stream, inp, vcode, dcode, args, world, plain_ms):
     o = torch.empty_like(q)
     s_out = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32, device=dev)
     snaps = torch.empty((w.batch, w.heads, n, w.dim, w.dim), dtype=torch.float32, device=dev)
+    need = abi.lightning_prefill_workspace_size(w.batch, w.heads, w.seq, w.dim, w.block)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     sp = stream.cuda_stream
 
     def step():
         abi.check(abi.lightning_prefill_snapshots(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads, w.seq, w.dim,
             w.block, None if s0 is None else s0.data_ptr(), o.data_ptr(), s_out.data_ptr(), interval,
-            snaps.data_ptr(), sp, vcode))
+            snaps.data_ptr(), ws.data_ptr(), need, sp, vcode))
 
     steps = max(1, min(args.steps, 10))
     ms = timed("snapshots", step, steps, args.warmup, stream, world, dev)
@@ -691,16 +697,19 @@ def run_prefill_norm_gate_leg(w, dev, stream, inp, dcode, args, world):
     s_out = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32, device=dev)
     sp = stream.cuda_stream
     s0p = None if s0 is None else s0.data_ptr()
+    need = abi.lightning_prefill_workspace_size(w.batch, w.heads, w.seq, w.dim, w.block)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 
     def fused():
         abi.check(abi.lightning_prefill_norm_gate(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads, w.seq, w.dim,
-            w.block, s0p, gate.data_ptr(), gamma.data_ptr(), 1e-6, y.data_ptr(), s_out.data_ptr(), sp))
+            w.block, s0p, gate.data_ptr(), gamma.data_ptr(), 1e-6, y.data_ptr(), s_out.data_ptr(), ws.data_ptr(),
+            need, sp))
 
     def two_calls():
         abi.check(abi.lightning_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch,
                                            w.heads, w.seq, w.dim, w.block, s0p, o.data_ptr(), s_out.data_ptr(),
-                                           None, 0, sp, abi.LA_VARIANT_TCGEN05_PAIR))
+                                           ws.data_ptr(), need, sp, abi.LA_VARIANT_TCGEN05_PAIR))
         abi.check(abi.lightning_norm_gate(o.data_ptr(), gate.data_ptr(), dcode, gamma.data_ptr(), 1e-6, w.batch,
                                           w.heads, w.seq, w.dim, 1, y.data_ptr(), sp))
 
@@ -820,6 +829,8 @@ def run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world):
     og = torch.empty((b, hq, L, d), dtype=q.dtype, device=dev)
     need = abi.lightning_gqa_prefill_workspace_size(dcode, b, hq, L, d)
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    lneed = abi.lightning_prefill_workspace_size(b, w.heads, L, d, w.block)
+    lws = torch.empty(max(lneed, 16), dtype=torch.uint8, device=dev)
     sp = stream.cuda_stream
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
 
@@ -829,7 +840,7 @@ def run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world):
         for _ in range(7):
             abi.check(abi.lightning_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), b,
                                                w.heads, L, d, w.block, None if s0 is None else s0.data_ptr(),
-                                               o.data_ptr(), s_out.data_ptr(), None, 0, sp, vcode))
+                                               o.data_ptr(), s_out.data_ptr(), lws.data_ptr(), lneed, sp, vcode))
             abi.check(abi.lightning_norm_gate(o.data_ptr(), gate.data_ptr(), dcode, gamma.data_ptr(), 1e-6, b,
                                               w.heads, L, d, 0, y.data_ptr(), sp))
         if mark:
@@ -911,13 +922,15 @@ def run_workload_leg(name, dev, stream, peaks, args, world):
     variant = la.prefill_variant(bw.dtype, bw.batch, bw.heads, bw.seq, bw.dim, bw.block)
     vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05,
              "pair": abi.LA_VARIANT_TCGEN05_PAIR}[variant]
+    need = abi.lightning_prefill_workspace_size(bw.batch, bw.heads, bw.seq, bw.dim, bw.block)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     sp = stream.cuda_stream
 
     def step():
         abi.check(abi.lightning_prefill_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), abi.LA_DTYPE_BF16, sl.data_ptr(),
                                            bw.batch, bw.heads, bw.seq, bw.dim, bw.block,
-                                           None if s0 is None else s0.data_ptr(), o.data_ptr(), s_out.data_ptr(), None,
-                                           0, sp, vcode))
+                                           None if s0 is None else s0.data_ptr(), o.data_ptr(), s_out.data_ptr(),
+                                           ws.data_ptr(), need, sp, vcode))
 
     steps = args.batched_steps
     ms = timed("other_workloads/%s" % bw.name, step, steps, args.warmup, stream, world, dev)
@@ -978,6 +991,11 @@ def run_backward_leg(w, dev, stream, inp, dcode, args, world):
             "frac_bf16_peak_formula": round(tf / peaks["bf16_tflops"], 4)}
 
 
+def abi_ws_bytes(w):
+    from linear_attention_lightning_b200 import abi
+    return abi.lightning_prefill_workspace_size(w.batch, w.heads, w.seq, w.dim, w.block)
+
+
 def run_e2e(w, dev, stream, inp, variant, args, world):
     """Same prefill through the public API with host buffers: every step copies
     q, k, v from pinned host memory and reads o and the state back. Steps are
@@ -995,6 +1013,7 @@ def run_e2e(w, dev, stream, inp, variant, args, world):
     sets = [[torch.empty_like(inp["q"]) for _ in range(3)] for _ in range(2)]
     outs = [(torch.empty_like(inp["q"]), torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32,
                                                       device=dev)) for _ in range(2)]
+    wsp = torch.empty(max(abi_ws_bytes(w), 16), dtype=torch.uint8, device=dev)
     h2d = 3 * hq.numel() * hq.element_size()
     d2h = ho.numel() * ho.element_size() + hs.numel() * 4
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
@@ -1020,7 +1039,7 @@ def run_e2e(w, dev, stream, inp, variant, args, world):
             if read[b] is not None:
                 stream.wait_event(read[b])         # its outputs from two steps back were read
             la.prefill(dq, dk, dv, inp["slopes"], w.block, inp["state_in"], variant=variant, o=o, state_out=s_,
-                       stream=stream)
+                       workspace=wsp, stream=stream)
             computed[b] = ev()
             computed[b].record(stream)
             with torch.cuda.stream(s_out):

@@ -99,10 +99,31 @@ int lightning_abi_version(void);
  *              NULL to skip. May be the same pointer as state_in (in-place
  *              carry); any other overlap is rejected.
  *   workspace, workspace_bytes
- *              scratch; the current kernels need none
- *              (lightning_prefill_workspace_size returns 0), so NULL/0 is fine.
+ *              device scratch, caller-owned, 16-byte aligned, overlapping no
+ *              other buffer, of at least lightning_prefill_workspace_size
+ *              bytes: 32 bytes per (batch, head) for the CTA-pair tensor-core
+ *              kernel (its range guard, below), none for the other kernels
+ *              (NULL/0 is fine there). Too little returns LA_ERR_INVALID_ARG.
+ *              Its contents need no initialisation; calls that share one
+ *              workspace must not run at the same time.
  *   stream     cudaStream_t as void*.
  * seq == 0 writes state_out = state_in (or zeros) and nothing else.
+ *
+ * Input range of the tensor-core kernels. They round the operands they form
+ * (P ⊙ D, Q ⊙ d_q, K ⊙ d_k, V and the carried state) to fp16, whose range is
+ * narrower than bf16's. The CTA-pair kernel guards against that: while it
+ * runs it bounds every such operand of each (batch, head) from the largest
+ * row norms of q and k, the largest |v| and the largest |state_in| element;
+ * a head whose operands could pass 2^15, or whose row norms fall below 2^-8,
+ * is recomputed by a second launch with q, k and v scaled by powers of two
+ * (exact) so that they sit in fp16's normal range, and scaled back. Its
+ * results meet the error bound for any scale of q, k, v and state_in within
+ * about 2^-36 .. 2^44, provided the values inside one (batch, head) span less
+ * than about 2^14 (a few rows 2^8 above the rest, with |q.k| above 65504, are
+ * covered). Inputs holding inf or NaN give non-finite results. The
+ * single-CTA kernel (LA_VARIANT_TCGEN05) has no guard: its operands must stay
+ * inside fp16's range (|q.k|, |q|, |k|, |v| and the state below 65504) and its
+ * row norms near or above 2^-8 for the bound to hold.
  */
 la_status lightning_prefill(const void *q, const void *k, const void *v, la_dtype dtype,
                             const float *slopes, int batch, int heads, int seq, int dim,
@@ -123,7 +144,9 @@ la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_d
 int lightning_prefill_selected_variant(la_dtype dtype, int batch, int heads, int seq, int dim,
                                        int block, int variant);
 
-/* Bytes of workspace lightning_prefill needs for these sizes (currently 0). */
+/* Bytes of workspace lightning_prefill (with AUTO, bf16 inputs) needs for these
+ * sizes: 32 * batch * heads for the CTA-pair kernel (dim 128, block 256), 0
+ * otherwise. Enough for every variant and dtype. Host only. */
 size_t lightning_prefill_workspace_size(int batch, int heads, int seq, int dim, int block);
 
 /*
@@ -132,7 +155,7 @@ size_t lightning_prefill_workspace_size(int batch, int heads, int seq, int dim, 
  * state S_t; the page's note that prefix caching and speculative decoding are
  * where such states are hard to serve) and §04 (the fp32 state per head).
  *
- * Same arguments and results as lightning_prefill_ex (workspace: none), plus
+ * Same arguments and results as lightning_prefill_ex (workspace included), plus
  *   interval   snapshot spacing in tokens: a positive multiple of `block`.
  *   snapshots  [batch][heads][n][dim][dim] float32, n = seq / interval
  *              (lightning_prefill_snapshot_count); snapshot i is the state after
@@ -147,7 +170,8 @@ size_t lightning_prefill_workspace_size(int batch, int heads, int seq, int dim, 
 la_status lightning_prefill_snapshots(const void *q, const void *k, const void *v, la_dtype dtype,
                                       const float *slopes, int batch, int heads, int seq, int dim,
                                       int block, const float *state_in, void *o, float *state_out,
-                                      int interval, float *snapshots, void *stream, int variant);
+                                      int interval, float *snapshots, void *workspace, size_t workspace_bytes,
+                                      void *stream, int variant);
 
 /*
  * Gradients of one prefill, for training through the layer. The pages print
@@ -178,8 +202,10 @@ la_status lightning_prefill_snapshots(const void *q, const void *k, const void *
  *   d_state_in    [batch][heads][dim][dim] float32, or NULL to skip.
  *   workspace, workspace_bytes
  *                 scratch of at least lightning_prefill_backward_workspace_size
- *                 bytes (0 for every current kernel, so NULL/0 is fine);
- *                 when needed: 16-byte aligned, overlapping nothing else.
+ *                 bytes: the range guard's records of the three tensor-core
+ *                 passes (96 bytes per (batch, head); see lightning_prefill),
+ *                 none on CUDA cores (NULL/0 is fine there); 16-byte aligned,
+ *                 overlapping nothing else, no initialisation needed.
  * All device pointers, caller-owned, 16-byte aligned. No output may overlap
  * an input or another output; a short or overlapping workspace is rejected
  * (all LA_ERR_INVALID_ARG). Shape rules as for lightning_prefill.
@@ -191,16 +217,24 @@ la_status lightning_prefill_backward(const void *q, const void *k, const void *v
                                      size_t workspace_bytes, void *stream, int variant);
 
 /*
- * lightning_prefill_backward without a workspace argument. The pages have no
- * counterpart to this entry point; it is a convenience of this library. It
- * takes any scratch the chosen kernels need from a fixed device array inside
- * the library (its size: lightning_prefill_backward_noalloc_capacity(),
- * 64 MiB) and allocates no memory; the current kernels need none. Arguments
- * and results are those of lightning_prefill_backward.
- * A request whose workspace would exceed the array returns
- * LA_ERR_UNSUPPORTED before any launch. All calls on one device share the
- * array: calls that could run at the same time (on different streams) must
- * use lightning_prefill_backward with their own workspaces instead.
+ * lightning_prefill_backward for callers that cannot allocate device memory
+ * themselves: a runtime whose allocator owns all of the device's memory and
+ * hands out none at the point of the call, or a plugin inside another
+ * framework that may not call cudaMalloc. The pages have no counterpart to
+ * this entry point. It allocates nothing: the scratch the tensor-core passes
+ * need (the range guard's records, 96 bytes per (batch, head)) comes from a
+ * fixed array inside the library, 4 MiB on every device that loads it, kept
+ * until the process exits (lightning_prefill_backward_noalloc_capacity()).
+ * Arguments and results are those of lightning_prefill_backward; argument
+ * errors come in the same order, then a request that needs more scratch than
+ * the array holds (more than 43690 batch x heads) returns LA_ERR_UNSUPPORTED,
+ * all before any launch.
+ * The first call on a device looks up the array's address on that device
+ * (with that device current): make that first call before any stream capture.
+ * Every call on a device shares the array, which keeps the last call's
+ * contents (nothing in it needs to start at zero): calls that overlap in time
+ * on the GPU (on different streams) race on it, so such callers must use
+ * lightning_prefill_backward with a workspace of their own.
  */
 la_status lightning_prefill_backward_noalloc(const void *q, const void *k, const void *v, const void *d_o,
                                              la_dtype dtype, const float *slopes, int batch, int heads,
@@ -254,6 +288,8 @@ la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, c
  *   gamma  [heads*128] float32.   eps: finite, >= 0.
  *   y      [batch][seq][heads*128] bf16; written; must not overlap any input,
  *          the states, gate or gamma.
+ *   workspace, workspace_bytes: as for lightning_prefill (the CTA-pair
+ *          kernel's range guard: 32 bytes per (batch, head)).
  * Runs on the CTA-pair tensor-core kernel only: bf16, dim 128, block 256;
  * other shapes or dtypes return LA_ERR_UNSUPPORTED before any launch (the
  * whole-token mean needs every head of a token, which one head's kernel does
@@ -263,7 +299,8 @@ la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, c
 la_status lightning_prefill_norm_gate(const void *q, const void *k, const void *v, la_dtype dtype,
                                       const float *slopes, int batch, int heads, int seq, int dim, int block,
                                       const float *state_in, const void *gate, const float *gamma, float eps,
-                                      void *y, float *state_out, void *stream);
+                                      void *y, float *state_out, void *workspace, size_t workspace_bytes,
+                                      void *stream);
 
 /* Number of snapshots lightning_prefill_snapshots writes per (batch, head):
  * seq / interval, or -1 if seq < 0 or interval < 1. Host only. */

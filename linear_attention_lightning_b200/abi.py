@@ -28,11 +28,11 @@ _SIGNATURES = {
     "lightning_prefill_selected_variant": ([_i, _i, _i, _i, _i, _i, _i], _i),
     "lightning_prefill_workspace_size": ([_i, _i, _i, _i, _i], _sz),
     "lightning_prefill_snapshots": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp,
-                                     _i], _i),
+                                     _sz, _vp, _i], _i),
     "lightning_prefill_snapshot_count": ([_i, _i], _i),
     "lightning_norm_gate": ([_vp, _vp, _i, _vp, ctypes.c_float, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "lightning_prefill_norm_gate": ([_vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, ctypes.c_float,
-                                     _vp, _vp, _vp], _i),
+                                     _vp, _vp, _vp, _sz, _vp], _i),
     "lightning_gqa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_double,
                               ctypes.c_float, _vp, _vp, _sz, _vp], _i),
     "lightning_gqa_decode_workspace_size": ([_i, _i, _i], _sz),
@@ -125,9 +125,10 @@ def lightning_prefill_workspace_size(batch, heads, seq, dim, block):
 
 
 def lightning_prefill_snapshots(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out,
-                                interval, snapshots, stream, variant):
+                                interval, snapshots, workspace, workspace_bytes, stream, variant):
     return load().lightning_prefill_snapshots(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in,
-                                              o, state_out, interval, snapshots, stream, variant)
+                                              o, state_out, interval, snapshots, workspace, workspace_bytes, stream,
+                                              variant)
 
 
 def lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in,
@@ -156,9 +157,9 @@ def lightning_norm_gate(o, gate, dtype, gamma, eps, batch, heads, seq, dim, per_
 
 
 def lightning_prefill_norm_gate(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, gate, gamma, eps,
-                                y, state_out, stream):
+                                y, state_out, workspace, workspace_bytes, stream):
     return load().lightning_prefill_norm_gate(q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in,
-                                              gate, gamma, eps, y, state_out, stream)
+                                              gate, gamma, eps, y, state_out, workspace, workspace_bytes, stream)
 
 
 def lightning_gqa_decode(q, k_new, v_new, k_cache, v_cache, dtype, pos, batch, heads, kv_heads, dim, cap, rot,

@@ -106,11 +106,11 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Ten
 def prefill_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes: torch.Tensor, block: int,
                       interval: int, state_in: Optional[torch.Tensor] = None, o: Optional[torch.Tensor] = None,
                       state_out: Optional[torch.Tensor] = None, snapshots: Optional[torch.Tensor] = None,
-                      want_state: bool = True, variant: str = "auto",
+                      want_state: bool = True, variant: str = "auto", workspace: Optional[torch.Tensor] = None,
                       stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor], torch.Tensor]:
     """lightning_prefill_snapshots: returns (o, state_out, snapshots); snapshots is
     [batch, heads, seq // interval, dim, dim] float32, the state after each
-    interval tokens."""
+    interval tokens. The workspace is allocated with torch unless given."""
     b, h, L, d = _qkv(q, k, v)
     _need_cuda("slopes", slopes, torch.float32, (h,))
     _state("state_in", state_in, b, h, d)
@@ -129,10 +129,11 @@ def prefill_snapshots(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes:
         snapshots = torch.empty((b, h, n, d, d), dtype=torch.float32, device=q.device)
     else:
         _need_cuda("snapshots", snapshots, torch.float32, (b, h, n, d, d))
+    workspace = _workspace(abi.lightning_prefill_workspace_size(b, h, L, d, int(block)), workspace, q.device)
     abi.check(abi.lightning_prefill_snapshots(
         _ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(slopes), b, h, L, d, int(block),
         _ptr(state_in), _ptr(o), _ptr(state_out), int(interval), _ptr(snapshots) if n > 0 else None,
-        _stream(stream), _VARIANTS[variant]))
+        _ptr(workspace), _nbytes(workspace), _stream(stream), _VARIANTS[variant]))
     return o, state_out, snapshots
 
 
@@ -188,9 +189,11 @@ def prefill_norm_gate(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes:
                       gate: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
                       state_in: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
                       state_out: Optional[torch.Tensor] = None, want_state: bool = True,
+                      workspace: Optional[torch.Tensor] = None,
                       stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """lightning_prefill_norm_gate: the prefill with the per-head normalisation and
-    gate fused into its epilogue; returns (y [batch, seq, heads*dim], state_out)."""
+    gate fused into its epilogue; returns (y [batch, seq, heads*dim], state_out).
+    The workspace is allocated with torch unless given."""
     b, h, L, d = _qkv(q, k, v)
     _need_cuda("slopes", slopes, torch.float32, (h,))
     _need_cuda("gate", gate, q.dtype, (b, L, h * d))
@@ -204,9 +207,11 @@ def prefill_norm_gate(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slopes:
         state_out = torch.empty((b, h, d, d), dtype=torch.float32, device=q.device)
     else:
         _state("state_out", state_out, b, h, d)
+    workspace = _workspace(abi.lightning_prefill_workspace_size(b, h, L, d, int(block)), workspace, q.device)
     abi.check(abi.lightning_prefill_norm_gate(
         _ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], _ptr(slopes), b, h, L, d, int(block), _ptr(state_in),
-        _ptr(gate), _ptr(gamma), float(eps), _ptr(y), _ptr(state_out), _stream(stream)))
+        _ptr(gate), _ptr(gamma), float(eps), _ptr(y), _ptr(state_out), _ptr(workspace), _nbytes(workspace),
+        _stream(stream)))
     return y, state_out
 
 

@@ -2,8 +2,8 @@
 //
 // Argument checking happens here, before any launch; every check failure
 // returns a status and records a message for lightning_last_error_message().
-// The library allocates nothing: all tensors, and the (currently unused)
-// workspace, belong to the caller.
+// The library allocates nothing: all tensors, and the workspace (the range
+// guard's per-head records of the tensor-core prefill), belong to the caller.
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -91,7 +91,27 @@ struct PrefillArgs {
     void *o;
     float *state_out;
     la::Snapshots sn;  // prefix-cache snapshots; sn.ptr == nullptr: none
+    void *workspace;
+    size_t workspace_bytes;
 };
+
+// Workspace a prefill request needs: the range guard's records for the CTA-pair
+// kernel, none for the others.
+size_t prefill_workspace_bytes(int batch, int heads, int variant) {
+    return variant == LA_VARIANT_TCGEN05_PAIR ? la::pair_workspace_bytes((long long)batch * heads) : 0;
+}
+
+// A workspace of at least `need` bytes, 16-byte aligned, overlapping none of `others`.
+la_status check_workspace(const void *ws, size_t bytes, size_t need, const Range *others, int n_others) {
+    if (need == 0) return LA_OK;
+    if (!ws || bytes < need)
+        return fail(LA_ERR_INVALID_ARG, "this call needs %zu bytes of workspace (got %zu)", need, ws ? bytes : (size_t)0);
+    if (!aligned16(ws)) return fail(LA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    const Range rw = range_of(ws, need);
+    for (int i = 0; i < n_others; ++i)
+        if (overlaps(rw, others[i])) return fail(LA_ERR_INVALID_ARG, "workspace overlaps an input or an output");
+    return LA_OK;
+}
 
 // Shape / dtype checks shared by the launcher and the variant query.
 la_status check_prefill_shape(la_dtype dtype, int batch, int heads, int seq, int dim, int block) {
@@ -170,6 +190,22 @@ la_status check_snapshots(const PrefillArgs &a) {
     for (const Range &r : others)
         if (overlaps(rs, r)) return fail(LA_ERR_INVALID_ARG, "snapshots overlaps an input, o or a state");
     return LA_OK;
+}
+
+// The workspace of a prefill request (after check_prefill_pointers and, for
+// snapshots, check_snapshots).
+la_status check_prefill_workspace(const PrefillArgs &a, int variant) {
+    if (a.batch == 0 || a.seq == 0) return LA_OK;
+    const size_t eb = elem_bytes(a.dtype);
+    const size_t n_tok = (size_t)a.batch * a.heads * a.seq * a.dim;
+    const size_t n_state = (size_t)a.batch * a.heads * a.dim * a.dim;
+    const Range others[] = {range_of(a.q, n_tok * eb), range_of(a.k, n_tok * eb), range_of(a.v, n_tok * eb),
+                            range_of(a.o, n_tok * eb), range_of(a.slopes, sizeof(float) * a.heads),
+                            range_of(a.state_in, a.state_in ? n_state * 4 : 0),
+                            range_of(a.state_out, a.state_out ? n_state * 4 : 0),
+                            range_of(a.sn.ptr, a.sn.ptr ? n_state * (size_t)a.sn.count * 4 : 0)};
+    return check_workspace(a.workspace, a.workspace_bytes, prefill_workspace_bytes(a.batch, a.heads, variant), others,
+                           8);
 }
 
 template <typename T, int D>
@@ -366,9 +402,31 @@ struct BackwardArgs {
 };
 
 // Scratch of lightning_prefill_backward_noalloc: a fixed device array, so that
-// entry point needs no workspace from the caller and allocates nothing.
-constexpr size_t kNoAllocScratchBytes = (size_t)64 << 20;
+// entry point needs no workspace from the caller and allocates nothing. 4 MiB
+// hold the three passes' range-guard records for 43690 (batch, head) pairs.
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// The array's device address, looked up once per device with that device current.
+// In host code `g_noalloc_scratch` names a host-side stand-in, not the device
+// memory, so a kernel must be given this address instead.
+la_status noalloc_scratch(void **out) {
+    static std::mutex mu;
+    static void *addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(LA_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return LA_OK;
+}
 
 // Which kernels a backward request runs (LA_VARIANT_SIMT or _TCGEN05_PAIR), or -1.
 int choose_backward_variant(la_dtype dtype, int dim, int block, int requested) {
@@ -381,10 +439,11 @@ int choose_backward_variant(la_dtype dtype, int dim, int block, int requested) {
     }
 }
 
-// Workspace a backward request needs: none of the current kernels needs any.
+// Workspace a backward request needs: the range guard's records of the three
+// tensor-core passes (dV, dK, dQ, one region each); none on CUDA cores.
 size_t backward_workspace_bytes(la_dtype dtype, int batch, int heads, int seq, int dim, int variant) {
-    (void)dtype; (void)batch; (void)heads; (void)seq; (void)dim; (void)variant;
-    return 0;
+    (void)dtype; (void)seq; (void)dim;
+    return variant == LA_VARIANT_TCGEN05_PAIR ? 3 * la::pair_workspace_bytes((long long)batch * heads) : 0;
 }
 
 la_status check_backward_pointers(const BackwardArgs &a) {
@@ -469,6 +528,8 @@ cudaError_t aux_streams(cudaStream_t (&out)[2]) {
 // and everything after waits for the join), and the pattern can be captured into a graph.
 la_status run_backward_pair(const BackwardArgs &a, cudaStream_t stream) {
     const la::Snapshots none{nullptr, 0, 0};
+    la::rg::RangeRec *rec = static_cast<la::rg::RangeRec *>(a.workspace);
+    const size_t per_pass = (size_t)a.batch * a.heads;
     cudaStream_t aux[2];
     cudaError_t e = aux_streams(aux);
     if (e != cudaSuccess) return cuda_fail(e, "creating the backward's auxiliary streams");
@@ -486,13 +547,13 @@ la_status run_backward_pair(const BackwardArgs &a, cudaStream_t stream) {
     }
     if (st == LA_OK)
         st = la::launch_pair(a.k, a.q, a.d_o, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dv, a.d_state_in,
-                             none, la::pair::PairPass{0, 1}, aux[0], &g_last_error);
+                             none, la::pair::PairPass{0, 1}, rec, aux[0], &g_last_error);
     if (st == LA_OK)
         st = la::launch_pair(a.v, a.d_o, a.q, a.slopes, a.batch, a.heads, a.seq, a.d_state_out, a.dk, nullptr,
-                             none, la::pair::PairPass{1, 1}, aux[1], &g_last_error);
+                             none, la::pair::PairPass{1, 1}, rec + per_pass, aux[1], &g_last_error);
     if (st == LA_OK)
         st = la::launch_pair(a.d_o, a.v, a.k, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.dq, nullptr, none,
-                             la::pair::PairPass{1, 0}, stream, &g_last_error);
+                             la::pair::PairPass{1, 0}, rec + 2 * per_pass, stream, &g_last_error);
     // join even after a failed launch, so that `stream` never runs ahead of work already enqueued
     for (int i = 0; i < 2; ++i) {
         cudaError_t r = cudaEventRecord(join[i], aux[i]);
@@ -551,7 +612,8 @@ la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
     }
     if (variant == LA_VARIANT_TCGEN05_PAIR)
         return la::launch_pair(a.q, a.k, a.v, a.slopes, a.batch, a.heads, a.seq, a.state_in, a.o, a.state_out,
-                               a.sn, la::pair::PairPass{0, 0}, stream, &g_last_error);
+                               a.sn, la::pair::PairPass{0, 0}, static_cast<la::rg::RangeRec *>(a.workspace), stream,
+                               &g_last_error);
     if (variant == LA_VARIANT_TCGEN05) return la::launch_tc(a.q, a.k, a.v, a.slopes, a.batch, a.heads,
                                                            a.seq, a.block, a.state_in, a.o, a.state_out,
                                                            a.sn, stream, &g_last_error);
@@ -575,7 +637,7 @@ la_status launch_decode(const void *q, const void *k, const void *v, const float
 
 extern "C" {
 
-int lightning_abi_version(void) { return 1; }
+int lightning_abi_version(void) { return 2; }
 
 }  // extern "C"
 
@@ -602,6 +664,8 @@ la_status prefill_entry(const PrefillArgs &a, void *stream, int variant, bool wi
         st = check_snapshots(a);
         if (st != LA_OK) return st;
     }
+    st = check_prefill_workspace(a, chosen);
+    if (st != LA_OK) return st;
     return run_prefill(a, static_cast<cudaStream_t>(stream), chosen);
 }
 
@@ -613,10 +677,8 @@ la_status lightning_prefill_ex(const void *q, const void *k, const void *v, la_d
                                const float *slopes, int batch, int heads, int seq, int dim, int block,
                                const float *state_in, void *o, float *state_out, void *workspace,
                                size_t workspace_bytes, void *stream, int variant) {
-    (void)workspace;
-    (void)workspace_bytes;
     const PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out,
-                        la::Snapshots{nullptr, 0, 0}};
+                        la::Snapshots{nullptr, 0, 0}, workspace, workspace_bytes};
     return prefill_entry(a, stream, variant, false);
 }
 
@@ -648,18 +710,25 @@ la_status lightning_prefill_backward_noalloc(const void *q, const void *k, const
                                              int dim, int block, const float *state_in, const float *d_state_out,
                                              void *dq, void *dk, void *dv, float *d_state_in, void *stream,
                                              int variant) {
+    // the same argument checks, in the same order, as lightning_prefill_backward
     la_status st = check_prefill_shape(dtype, batch, heads, seq, dim, block);
     if (st != LA_OK) return st;
     const int chosen = choose_backward_variant(dtype, dim, block, variant);
-    const size_t need = chosen < 0 ? 0 : backward_workspace_bytes(dtype, batch, heads, seq, dim, chosen);
+    if (chosen < 0)  // its own message for an unknown or unsupported variant
+        return lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in,
+                                          d_state_out, dq, dk, dv, d_state_in, nullptr, 0, stream, variant);
+    const BackwardArgs a{q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in, d_state_out,
+                         dq, dk, dv, d_state_in, nullptr, 0};
+    st = check_backward_pointers(a);
+    if (st != LA_OK) return st;
+    const size_t need = backward_workspace_bytes(dtype, batch, heads, seq, dim, chosen);
     if (need > kNoAllocScratchBytes)
         return fail(LA_ERR_UNSUPPORTED, "the request needs %zu bytes of scratch; the built-in scratch holds %zu",
                     need, kNoAllocScratchBytes);
     void *scratch = nullptr;
     if (need > 0 && batch > 0 && seq > 0) {
-        // the scratch array's address in the current device's context
-        const cudaError_t e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        st = noalloc_scratch(&scratch);
+        if (st != LA_OK) return st;
     }
     return lightning_prefill_backward(q, k, v, d_o, dtype, slopes, batch, heads, seq, dim, block, state_in,
                                       d_state_out, dq, dk, dv, d_state_in, scratch, need, stream, variant);
@@ -677,7 +746,8 @@ size_t lightning_prefill_backward_workspace_size(la_dtype dtype, int batch, int 
 la_status lightning_prefill_norm_gate(const void *q, const void *k, const void *v, la_dtype dtype,
                                       const float *slopes, int batch, int heads, int seq, int dim, int block,
                                       const float *state_in, const void *gate, const float *gamma, float eps,
-                                      void *y, float *state_out, void *stream) {
+                                      void *y, float *state_out, void *workspace, size_t workspace_bytes,
+                                      void *stream) {
     la_status st = check_prefill_shape(dtype, batch, heads, seq, dim, block);
     if (st != LA_OK) return st;
     if (!la::pair_supports(dtype == LA_DTYPE_BF16, dim, block))
@@ -687,7 +757,7 @@ la_status lightning_prefill_norm_gate(const void *q, const void *k, const void *
                     (int)dtype, dim, block);
     if (!(eps >= 0.f) || eps > 3.0e38f) return fail(LA_ERR_INVALID_ARG, "eps must be finite and >= 0");
     const PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, y, state_out,
-                        la::Snapshots{nullptr, 0, 0}};
+                        la::Snapshots{nullptr, 0, 0}, workspace, workspace_bytes};
     st = check_prefill_pointers(a);
     if (st != LA_OK) return st;
     const size_t n_tok = (size_t)batch * heads * seq * dim;
@@ -703,13 +773,18 @@ la_status lightning_prefill_norm_gate(const void *q, const void *k, const void *
             if (overlaps(rs, range_of(gate, n_tok * 2)) || overlaps(rs, range_of(gamma, sizeof(float) * heads * dim)))
                 return fail(LA_ERR_INVALID_ARG, "state_out overlaps gate or gamma");
         }
+        st = check_prefill_workspace(a, LA_VARIANT_TCGEN05_PAIR);
+        if (st != LA_OK) return st;
+        const Range rw = range_of(workspace, prefill_workspace_bytes(batch, heads, LA_VARIANT_TCGEN05_PAIR));
+        if (overlaps(rw, range_of(gate, n_tok * 2)) || overlaps(rw, range_of(gamma, sizeof(float) * heads * dim)))
+            return fail(LA_ERR_INVALID_ARG, "workspace overlaps gate or gamma");
     }
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     if (batch == 0 || seq == 0) return run_prefill(a, cs, LA_VARIANT_TCGEN05_PAIR);
     if (const la_status early = earlier_failure()) return early;
     const la::pair::PairNormGate ng{static_cast<const __nv_bfloat16 *>(gate), gamma, eps};
     return la::launch_pair(q, k, v, slopes, batch, heads, seq, state_in, y, state_out, a.sn, la::pair::PairPass{0, 0},
-                           cs, &g_last_error, &ng);
+                           static_cast<la::rg::RangeRec *>(workspace), cs, &g_last_error, &ng);
 }
 
 la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, const float *gamma, float eps,
@@ -872,10 +947,11 @@ int lightning_prefill_snapshot_count(int seq, int interval) {
 la_status lightning_prefill_snapshots(const void *q, const void *k, const void *v, la_dtype dtype,
                                       const float *slopes, int batch, int heads, int seq, int dim, int block,
                                       const float *state_in, void *o, float *state_out, int interval,
-                                      float *snapshots, void *stream, int variant) {
+                                      float *snapshots, void *workspace, size_t workspace_bytes, void *stream,
+                                      int variant) {
     const int count = interval > 0 && seq >= 0 ? seq / interval : 0;
     const PrefillArgs a{q, k, v, dtype, slopes, batch, heads, seq, dim, block, state_in, o, state_out,
-                        la::Snapshots{count > 0 ? snapshots : nullptr, interval, count}};
+                        la::Snapshots{count > 0 ? snapshots : nullptr, interval, count}, workspace, workspace_bytes};
     return prefill_entry(a, stream, variant, true);
 }
 
@@ -894,8 +970,9 @@ int lightning_prefill_selected_variant(la_dtype dtype, int batch, int heads, int
 }
 
 size_t lightning_prefill_workspace_size(int batch, int heads, int seq, int dim, int block) {
-    (void)batch; (void)heads; (void)seq; (void)dim; (void)block;
-    return 0;
+    if (check_prefill_shape(LA_DTYPE_BF16, batch, heads, seq, dim, block) != LA_OK) return 0;
+    // the largest any kernel takes for these sizes (bf16 inputs)
+    return prefill_workspace_bytes(batch, heads, choose_variant(LA_DTYPE_BF16, dim, block, LA_VARIANT_AUTO));
 }
 
 la_status lightning_decode(const void *q, const void *k, const void *v, la_dtype dtype, const float *slopes,

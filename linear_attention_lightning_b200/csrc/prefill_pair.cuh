@@ -61,6 +61,7 @@
 #include "../../include/lightning.h"
 #include "common.cuh"
 #include "prefill_tc.cuh"
+#include "range_guard.cuh"
 #include "tc_ptx.cuh"
 
 namespace la {
@@ -79,10 +80,12 @@ constexpr uint32_t kOffS = kOffStage + 2 * kStageBytes;
 constexpr uint32_t kSBytes = 2 * 8192;                         // 2 boxes of 64 rows x 128 B
 constexpr uint32_t kOffE = kOffS + kSBytes;                    // output staging: 128 rows x 64 bf16
 constexpr uint32_t kOffBar = kOffE + kBoxBytes;
-constexpr int kNumBars = 24;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kNumBars = 27;
+constexpr uint32_t kOffMisc = (kOffBar + kNumBars * 8 + 15) & ~15u;
 constexpr uint32_t kOffGamma = kOffMisc + 64;                  // fused norm + gate: gamma of the head
 constexpr uint32_t kSmemBytes = kOffGamma + kDim * 4 + 1024;
+static_assert(kOffMisc % 16 == 0 && kOffGamma % 16 == 0, "gamma is read with 16-byte loads");
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColP = 0, kColPHi = 128, kColO = 256, kColDS = 384, kColQd = 448;
@@ -92,7 +95,16 @@ constexpr uint32_t kColP = 0, kColPHi = 128, kColO = 256, kColDS = 384, kColQd =
 constexpr int QK_LOADED = 0, VK_LOADED = 1 /* 2 */, P_FULL = 3 /* 2 */, QK_DONE = 5, O_FULL = 6,
               DS_FULL = 7, VK_EMPTY = 8 /* 2 */, P_FREE = 10 /* 2 */, QD_LOCAL = 12, QK_FULL = 13,
               QD_READY = 14, S_READY = 15, O_FREE = 16, VK_READY = 17, DS_FREE = 18, P_CONV = 19 /* 2 */,
-              DRAIN = 21, G_FULL = 22 /* fused norm + gate: a gate half landed in the staging tile */;
+              DRAIN = 21, G_FULL = 22 /* fused norm + gate: a gate half landed in the staging tile */,
+              // range guard (pass 1 only): SCAN_FIN: warpgroups A and B put their maxima of
+              // k, v and q in shared memory; SIN_DONE: warpgroup 3 put its maximum of state_in;
+              // PEER: the other CTA's maxima landed here; RANGE_DONE: the head's verdict is set
+              SCAN_FIN = 23, SIN_DONE = 24, PEER = 25, RANGE_DONE = 26;
+
+// shared-memory words after the barriers
+// (the maxima as float bits, which order like unsigned integers for values >= 0)
+constexpr uint32_t kMiscTmem = 0, kMiscAbort = 4, kMiscMq = 8, kMiscMk = 12, kMiscMv = 16, kMiscSin = 20,
+                   kMiscPeer = 24 /* 4 floats */, kMiscFlag = 40;
 
 constexpr int kBarA = 1, kBarB = 3, kBarW3 = 2;  // named barriers of the three warpgroups
 
@@ -179,9 +191,11 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
 // fp32 P columns [col0, col0 + 128) of this thread's row -> fp16 P ⊙ D in
 // [dst0, dst0 + 64). Row i (block position) against keys j0 .. j0+127.
 // Causal: key j counts for j <= i with e^{-s(i-j)}; anti-causal (upper): for
-// j >= i with e^{-s(j-i)}. tab[u] = e^{-s(15-u)}, step = e^{-s}.
+// j >= i with e^{-s(j-i)}. tab[u] = pscale e^{-s(15-u)}, step = e^{-s};
+// pscale is the range guard's factor for P (1 in the plain kernel).
 __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uint32_t dst0, int i, int j0,
-                                          float sl2, float step, const float (&tab)[16], bool upper) {
+                                          float sl2, float step, const float (&tab)[16], bool upper,
+                                          float pscale) {
     // 32 fp32 columns per iteration -> 16 fp16 pair columns; the destination
     // [dst0 + 16 q, dst0 + 16 q + 16) lies inside columns already read
 #pragma unroll 1
@@ -212,7 +226,7 @@ __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uin
                 } else {
                     // keys from the diagonal (u = i - jb) upward
                     const int d0 = i - jb;
-                    float w = 1.f;
+                    float w = pscale;
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
                         const bool live = u >= d0;
@@ -235,7 +249,7 @@ __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uin
                 for (int u = 0; u < 16; ++u) p[u] = 0.f;
             } else {
                 const int d0 = i - jb;
-                float w = 1.f;
+                float w = pscale;
 #pragma unroll
                 for (int u = 15; u >= 0; --u) {
                     const bool live = u <= d0;
@@ -251,11 +265,19 @@ __device__ __forceinline__ void convert_p(uint32_t taddr_row, uint32_t col0, uin
     }
 }
 
-// scale one 128-byte swizzled row (64 16-bit values) in place: bf16 -> fp16 x scale
-__device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scale) {
+// scale one 128-byte swizzled row (64 16-bit values) in place: bf16 -> fp16 x scale.
+// kMeasure: also fold the row's largest |value| (bf16, as read) into mx.
+template <bool kMeasure>
+__device__ __forceinline__ void scale_row_to_f16(uint8_t *row, int r, float scale, uint32_t &mx) {
     uint4 x[8];
 #pragma unroll
     for (int ch = 0; ch < 8; ++ch) x[ch] = *reinterpret_cast<const uint4 *>(row + ((ch ^ (r & 7)) << 4));
+    if (kMeasure) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+            mx = rg::maxabs_bf16x2(mx, rg::maxabs_bf16x2(rg::maxabs_bf16x2(x[ch].x, x[ch].y),
+                                                         rg::maxabs_bf16x2(x[ch].z, x[ch].w)));
+    }
 #pragma unroll
     for (int ch = 0; ch < 8; ++ch) {
         uint4 y;
@@ -286,22 +308,62 @@ struct PairPass {
                      //    token (query factor e^{-s(m-1-i)}, key factor e^{-s(j+1)})
 };
 
-template <bool kAnti, bool kNormGate>
+// kScaled = false: the plain kernel (pass 1 of the range guard), which also
+// measures every (batch, head) and records its bounds and verdict in rec[bh].
+// kScaled = true: pass 2, which returns at once for a head pass 1 did not flag
+// and otherwise recomputes it with the guard's power-of-two operand scales.
+template <bool kAnti, bool kNormGate, bool kScaled>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ slopes, int heads, int seq, const float *state_in,
-                    float *state_out, Snapshots sn, PairPass pp, PairNormGate ng) {
+                    float *state_out, Snapshots sn, PairPass pp, PairNormGate ng, rg::RangeRec *rec,
+                    const __nv_bfloat16 *qg, const __nv_bfloat16 *kg) {
     extern __shared__ uint8_t smem_raw[];
+    // operand scales: q, k, v, P = q k, the carried state, its inverse, and o's inverse
+    float f_q = 1.f, f_k = 1.f, f_v = 1.f, f_p = 1.f, f_s = 1.f, f_su = 1.f, f_o = 1.f;
+    if constexpr (kScaled) {
+        const int bh0 = blockIdx.x >> 1;
+        const rg::RangeRec r = rec[bh0];
+        if (!r.flag) return;  // both CTAs of the pair read the same record and leave together
+        // the head's largest row norms of q and k, fp32 sums: this CTA takes every other
+        // row, then the two CTAs exchange through the output staging tile (first written
+        // after the set-up's cluster barrier, which the other CTA reaches only after its read)
+        const uint32_t a0 = ptx::smem_addr(smem_raw);
+        uint8_t *sm = smem_raw + (((a0 + 1023u) & ~1023u) - a0);
+        float *red = reinterpret_cast<float *>(sm + kOffE);
+        float *mine = reinterpret_cast<float *>(sm + kOffE + 64);
+        const uint32_t crank = cluster_rank();
+        const size_t hb = (size_t)bh0 * seq * kDim;
+        const float sq = rg::head_max_row_sumsq(qg + hb, seq, (int)crank, 2, red);
+        const float sk = rg::head_max_row_sumsq(kg + hb, seq, (int)crank, 2, red);
+        if (threadIdx.x == 0) {
+            mine[0] = sq;
+            mine[1] = sk;
+        }
+        cluster_sync();
+        float pq, pk;
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pq) : "r"(map_to_rank(mine, crank ^ 1u)) : "memory");
+        asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pk) : "r"(map_to_rank(mine + 1, crank ^ 1u)) : "memory");
+        const float nq = sqrtf(fmaxf(sq, pq)), nk = sqrtf(fmaxf(sk, pk));
+        const rg::Exps e = rg::scale_exponents(nq, nk, r.mv, r.msin, slopes[bh0 % heads], seq);
+        f_q = rg::pow2(e.a);
+        f_k = rg::pow2(e.b);
+        f_v = rg::pow2(e.c);
+        f_p = rg::pow2(e.a + e.b);
+        f_s = rg::pow2(e.b + e.c);
+        f_su = rg::pow2(-(e.b + e.c));
+        f_o = rg::pow2(-(e.a + e.b + e.c));
+    }
     const uint32_t raw_addr = ptx::smem_addr(smem_raw);
     const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
     Ctx c;
     c.smem = smem_raw + pad;
     c.sbase = raw_addr + pad;
     c.bars = reinterpret_cast<uint64_t *>(c.smem + kOffBar);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c.smem + kOffMisc);
-    c.abort = reinterpret_cast<volatile int *>(c.smem + kOffMisc + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c.smem + kOffMisc + kMiscTmem);
+    c.abort = reinterpret_cast<volatile int *>(c.smem + kOffMisc + kMiscAbort);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -324,7 +386,12 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::mbar_init(&c.bars[DS_FREE], 2);
         ptx::mbar_init(&c.bars[P_CONV], 2);
         ptx::mbar_init(&c.bars[P_CONV + 1], 2);
+        ptx::mbar_init(&c.bars[SCAN_FIN], 2);  // warpgroups A and B
+        *reinterpret_cast<uint32_t *>(c.smem + kOffMisc + kMiscMq) = 0u;
+        *reinterpret_cast<uint32_t *>(c.smem + kOffMisc + kMiscMk) = 0u;
+        *reinterpret_cast<uint32_t *>(c.smem + kOffMisc + kMiscMv) = 0u;
         *c.abort = 0;
+        *reinterpret_cast<uint32_t *>(c.smem + kOffMisc + kMiscSin) = 0u;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -399,6 +466,42 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int t = 0; t < nblk; ++t) {
                 if (!wait_bar(c, QK_LOADED, (uint32_t)t & 1u)) break;
                 arrive_leader(&c.bars[QK_FULL]);
+            }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ range guard (pass 1)
+        // Lane 0 combines this CTA's maxima (warpgroups A and B measure k, v and q as they
+        // convert them; warpgroup 3 measures state_in) with the other CTA's, and sets the
+        // head's verdict.
+        if (!kScaled && lane == 0) {
+            const uint32_t *misc = reinterpret_cast<const uint32_t *>(c.smem + kOffMisc);
+            float *peer = reinterpret_cast<float *>(c.smem + kOffMisc + kMiscPeer);
+            bool ok = wait_bar(c, SCAN_FIN, 0) && wait_bar(c, SIN_DONE, 0);
+            if (ok) {
+                // this CTA's maxima to the other CTA
+                const float v4[4] = {__uint_as_float(misc[kMiscMq / 4]), __uint_as_float(misc[kMiscMk / 4]),
+                                     __uint_as_float(misc[kMiscMv / 4]), __uint_as_float(misc[kMiscSin / 4])};
+                const uint32_t other = rank ^ 1u;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(map_to_rank(peer + i, other)), "f"(v4[i])
+                                 : "memory");
+                asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                                 map_to_rank(&c.bars[PEER], other))
+                             : "memory");
+                ok = ptx::mbar_wait_cluster(&c.bars[PEER], 0, c.abort);
+                if (ok) {
+                    rg::RangeRec r;
+                    r.mq = fmaxf(v4[0], peer[0]);
+                    r.mk = fmaxf(v4[1], peer[1]);
+                    r.mv = fmaxf(v4[2], peer[2]);
+                    r.msin = fmaxf(v4[3], peer[3]);
+                    r.flag = rg::plain_ok(r, s, seq) ? 0 : 1;
+                    r.pad[0] = r.pad[1] = r.pad[2] = 0;
+                    *reinterpret_cast<volatile int *>(c.smem + kOffMisc + kMiscFlag) = r.flag;
+                    if (rank == 0) rec[bh] = r;
+                    ptx::mbar_arrive(&c.bars[RANGE_DONE]);
+                }
             }
         }
     } else if (warp == 1) {
@@ -500,7 +603,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float step = ptx::ex2(-sl2);
         float tab[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) tab[u] = ptx::ex2(-sl2 * (float)(15 - u));
+        for (int u = 0; u < 16; ++u) tab[u] = ptx::ex2(-sl2 * (float)(15 - u)) * f_p;
+        // pass 1: the largest |x| this thread converts (bf16 pairs; group A: k in mx0 and
+        // v in mx1, group B: q in mx0), for the range guard
+        uint32_t mx0 = 0u, mx1 = 0u;
         for (int t = 0; t < nblk; ++t) {
             const uint32_t par = t & 1;
             const int m = blen(t);
@@ -518,10 +624,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int u = 0; u < 4; ++u) {
                     // u = 0, 1: K rows r and 128 + r scaled by d_k; u = 2, 3: V rows widened
                     const int h = u & 1, j = kRows * h + r;
-                    const float sc = u >= 2   ? 1.f
+                    const float sc = u >= 2   ? f_v
                                      : j >= m ? 0.f
-                                              : ptx::ex2(-sl2 * (float)(kAnti ? j + 1 : m - 1 - j));
-                    scale_row_to_f16((u >= 2 ? vt : kd) + h * kBoxBytes + r * 128, r, sc);
+                                              : ptx::ex2(-sl2 * (float)(kAnti ? j + 1 : m - 1 - j)) * f_k;
+                    scale_row_to_f16<!kScaled>((u >= 2 ? vt : kd) + h * kBoxBytes + r * 128, r, sc, u >= 2 ? mx1 : mx0);
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::named_bar_sync(bar_id, 128);
@@ -531,8 +637,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // Qd S MMA (which precedes its dS MMA) has read the region
                 if (t > 0 && !group_wait(c, DS_FULL, (uint32_t)(t - 1) & 1u, leader, bar_id)) goto ab_done;
                 if (!group_wait(c, QK_LOADED, par, leader, bar_id)) goto ab_done;
-                const float dq = kAnti ? (i < m ? ptx::ex2(-sl2 * (float)(m - 1 - i)) : 0.f)
-                                         : ptx::ex2(-sl2 * (float)(i + 1));
+                const float dq = (kAnti ? (i < m ? ptx::ex2(-sl2 * (float)(m - 1 - i)) : 0.f)
+                                          : ptx::ex2(-sl2 * (float)(i + 1))) * f_q;
                 const uint8_t *qrow = c.smem + kOffQ + r * 128;
 #pragma unroll 1
                 for (int hb = 0; hb < 4; ++hb) {
@@ -542,6 +648,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         const int chunk = 4 * (hb & 1) + cc;
                         const uint4 q4 = *reinterpret_cast<const uint4 *>(qrow + (hb >> 1) * kBoxBytes +
                                                                           ((chunk ^ (r & 7)) << 4));
+                        if (!kScaled)
+                            mx0 = rg::maxabs_bf16x2(mx0, rg::maxabs_bf16x2(rg::maxabs_bf16x2(q4.x, q4.y),
+                                                                           rg::maxabs_bf16x2(q4.z, q4.w)));
                         out[4 * cc + 0] = bf16x2_to_f16x2(q4.x, dq);
                         out[4 * cc + 1] = bf16x2_to_f16x2(q4.y, dq);
                         out[4 * cc + 2] = bf16x2_to_f16x2(q4.z, dq);
@@ -572,14 +681,26 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int q = 0; q < 4; ++q) ptx::tmem_st16(trow + (grp == 0 ? kColP : kColPHi) + 16 * q, zero);
             } else {
                 convert_p(trow, grp == 0 ? kColP : kColPHi, grp == 0 ? kColP : kColPHi, i, kRows * grp, sl2,
-                          step, tab, kAnti);
+                          step, tab, kAnti, f_p);
             }
             ptx::tmem_st_wait();
             ptx::tc_fence_before();
             ptx::named_bar_sync(bar_id, 128);
             if (leader) arrive_leader(&c.bars[P_CONV + grp]);
         }
-    ab_done:;
+    ab_done:
+        if (!kScaled) {
+            // the group's maxima into shared memory for the range guard's verdict
+            const auto as_float = [](uint32_t w) { return fmaxf(fabsf(rg::bf_lo(w)), fabsf(rg::bf_hi(w))); };
+            const float m0 = rg::warp_max_nonneg(as_float(mx0)), m1 = rg::warp_max_nonneg(as_float(mx1));
+            if (lane == 0) {
+                uint32_t *misc = reinterpret_cast<uint32_t *>(c.smem + kOffMisc);
+                atomicMax(misc + (grp == 0 ? kMiscMk : kMiscMq) / 4, __float_as_uint(m0));
+                if (grp == 0) atomicMax(misc + kMiscMv / 4, __float_as_uint(m1));
+            }
+            ptx::named_bar_sync(bar_id, 128);
+            if (leader) ptx::mbar_arrive(&c.bars[SCAN_FIN]);
+        }
     } else if (warp >= 12) {
         // ------------------------------------------------------------ warpgroup 3
         // The fp32 state S^T lives in TMEM [384, 448) in the 2x2 layout of the
@@ -612,7 +733,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // one 32-value half of this thread's state row: operand copy, optional
         // prefix-cache snapshot and state_out, then the decayed value back into
         // TMEM for the next MMA
-        auto carry_half = [&](const float (&sv)[32], int hh, float dnext, bool last, float *snap) {
+        auto carry_half = [&](const float (&sv)[32], int hh, float dnext, bool last, float *snap, bool write_state) {
 #pragma unroll
             for (int cq = 0; cq < 4; ++cq) {
                 const int ch = 4 * hh + cq;
@@ -625,13 +746,13 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             if (snap) {
 #pragma unroll
-                for (int q = 0; q < 32; ++q) snap[(size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q];
+                for (int q = 0; q < 32; ++q) snap[(size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q] * f_su;
             }
             if (last) {
-                if (state_out) {
+                if (write_state) {
 #pragma unroll
                     for (int q = 0; q < 32; ++q)
-                        state_out[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q];
+                        state_out[sb + (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol] = sv[q] * f_su;
                 }
             } else {
                 uint32_t lo[16], hi[16];
@@ -673,6 +794,13 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (!group_wait(c, DS_FULL, par, leader, kBarW3)) goto w3_done;
                 ptx::tc_fence_after();
             }
+            // pass 1 writes the final state only for a head the range guard passed, so that
+            // an in-place carry (state_out == state_in) is still intact for pass 2
+            bool write_state = state_out != nullptr;
+            if (!kScaled && last && write_state) {
+                if (!group_wait(c, RANGE_DONE, 0, leader, kBarW3)) goto w3_done;
+                write_state = *reinterpret_cast<volatile int *>(c.smem + kOffMisc + kMiscFlag) == 0;
+            }
             {
                 // decay from block t's end to block t+1's end (from the carried state's
                 // position to block 0's end when t = -1)
@@ -680,6 +808,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     last ? 0.f
                          : ptx::ex2(-sl2 * (float)blen(t + 1));
                 float *snap = t >= 0 && !kAnti ? snapshot_at(sn, bh, t * kBlock + blen(t), kDim) : nullptr;
+                float msin = 0.f;  // pass 1: the largest |state_in| element of this thread
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     float sv[32];
@@ -691,15 +820,25 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         for (int q = 0; q < 32; ++q) sv[q] = __uint_as_float(d[q]);
                     } else {
 #pragma unroll
-                        for (int q = 0; q < 32; ++q)
-                            sv[q] = state_in ? state_in[sb + (pp.state_in_t
-                                                                  ? (size_t)vcol * kDim + (64 * khalf + 32 * hh + q)
-                                                                  : (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol)]
-                                             : 0.f;
+                        for (int q = 0; q < 32; ++q) {
+                            const float x = state_in ? state_in[sb + (pp.state_in_t
+                                                                        ? (size_t)vcol * kDim + (64 * khalf + 32 * hh + q)
+                                                                        : (size_t)(64 * khalf + 32 * hh + q) * kDim + vcol)]
+                                                     : 0.f;
+                            msin = fmaxf(msin, fabsf(x));
+                            sv[q] = x * f_s;
+                        }
                     }
-                    carry_half(sv, hh, dnext, last, snap);
+                    carry_half(sv, hh, dnext, last, snap, write_state);
                 }
                 publish(last);
+                if (!kScaled && t < 0) {
+                    // the carried-in state's bound for the range guard
+                    const float m = rg::warp_max_nonneg(msin);
+                    if ((l & 31) == 0) atomicMax(reinterpret_cast<uint32_t *>(c.smem + kOffMisc + kMiscSin), __float_as_uint(m));
+                    ptx::named_bar_sync(kBarW3, 128);
+                    if (leader) ptx::mbar_arrive(&c.bars[SIN_DONE]);
+                }
             }
             if (t < 0) continue;
             if (kNormGate && leader) load_gate(t, 0);
@@ -719,8 +858,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ptx::tmem_ld_wait();
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
-                        const float x0 = __uint_as_float(a0[2 * u]), x1 = __uint_as_float(a0[2 * u + 1]);
-                        const float y0 = __uint_as_float(a1[2 * u]), y1 = __uint_as_float(a1[2 * u + 1]);
+                        const float x0 = __uint_as_float(a0[2 * u]) * f_o, x1 = __uint_as_float(a0[2 * u + 1]) * f_o;
+                        const float y0 = __uint_as_float(a1[2 * u]) * f_o, y1 = __uint_as_float(a1[2 * u + 1]) * f_o;
                         pk[16 * cb + u] = ptx::pack_bf16(x0, x1);
                         pk[16 * cb + 16 + u] = ptx::pack_bf16(y0, y1);
                         if (kNormGate) {
@@ -833,16 +972,27 @@ inline bool make_token_major_map(CUtensorMap *map, void *y, int batch, int heads
     return true;
 }
 
+// Workspace of one CTA-pair prefill: the range guard's record per (batch, head).
+inline size_t pair_workspace_bytes(long long batch_heads) {
+    return (size_t)batch_heads * sizeof(rg::RangeRec);
+}
+
 // ng != nullptr: the forward prefill with the normalisation and gating fused into
-// its epilogue; o is then the token-major y.
+// its epilogue; o is then the token-major y. Two launches on `stream`: the plain
+// kernel, which measures every (batch, head) into rec (pair_workspace_bytes of
+// the caller's workspace), then pass 2, which recomputes the heads it flagged.
 inline la_status launch_pair(const void *q, const void *k, const void *v, const float *slopes, int batch,
                              int heads, int seq, const float *state_in, void *o, float *state_out, Snapshots sn,
-                             pair::PairPass pp,
+                             pair::PairPass pp, rg::RangeRec *rec,
                              cudaStream_t stream, std::string *err, const pair::PairNormGate *ng = nullptr) {
     const long long bh = (long long)batch * heads;
     if (ng && pp.anti) {
         *err = "the fused normalisation runs on the forward (causal) pass only";
         return LA_ERR_UNSUPPORTED;
+    }
+    if (!rec) {
+        *err = "the CTA-pair prefill needs its workspace (the range guard's records)";
+        return LA_ERR_INVALID_ARG;
     }
     CUtensorMap mq, mk, mk64, mv, mo, mg;
     if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
@@ -855,14 +1005,14 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     } else {
         mg = mo;  // unused
     }
-    const auto kernel = ng        ? pair::prefill_pair_kernel<false, true>
-                        : pp.anti ? pair::prefill_pair_kernel<true, false>
-                                  : pair::prefill_pair_kernel<false, false>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pair::kSmemBytes);
-    if (e != cudaSuccess) {
-        *err = std::string("cudaFuncSetAttribute(prefill_pair): ") + cudaGetErrorString(e);
-        return LA_ERR_CUDA;
-    }
+    using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                            const float *, int, int, const float *, float *, Snapshots, pair::PairPass,
+                            pair::PairNormGate, rg::RangeRec *, const __nv_bfloat16 *, const __nv_bfloat16 *);
+    const Kernel passes[2] = {
+        ng ? pair::prefill_pair_kernel<false, true, false>
+           : pp.anti ? pair::prefill_pair_kernel<true, false, false> : pair::prefill_pair_kernel<false, false, false>,
+        ng ? pair::prefill_pair_kernel<false, true, true>
+           : pp.anti ? pair::prefill_pair_kernel<true, false, true> : pair::prefill_pair_kernel<false, false, true>};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(bh * 2));
     cfg.blockDim = dim3(pair::kThreads);
@@ -876,11 +1026,20 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const pair::PairNormGate ngv = ng ? *ng : pair::PairNormGate{nullptr, nullptr, 0.f};
-    e = cudaLaunchKernelEx(&cfg, kernel, mq, mk, mk64, mv, mo, mg, slopes, heads, seq, state_in,
-                           state_out, sn, pp, ngv);
-    if (e != cudaSuccess) {
-        *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
-        return LA_ERR_CUDA;
+    for (int pass = 0; pass < 2; ++pass) {
+        cudaError_t e = cudaFuncSetAttribute(passes[pass], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)pair::kSmemBytes);
+        if (e != cudaSuccess) {
+            *err = std::string("cudaFuncSetAttribute(prefill_pair): ") + cudaGetErrorString(e);
+            return LA_ERR_CUDA;
+        }
+        e = cudaLaunchKernelEx(&cfg, passes[pass], mq, mk, mk64, mv, mo, mg, slopes, heads, seq, state_in,
+                               state_out, sn, pp, ngv, rec, static_cast<const __nv_bfloat16 *>(q),
+                               static_cast<const __nv_bfloat16 *>(k));
+        if (e != cudaSuccess) {
+            *err = std::string("prefill_pair launch: ") + cudaGetErrorString(e);
+            return LA_ERR_CUDA;
+        }
     }
     err->clear();
     return LA_OK;

@@ -22,13 +22,14 @@ static void check(int cond, const char *what) {
 static const void *fake(int i) { return (const void *)(uintptr_t)(0x10000000u * (unsigned)(i + 1)); }
 
 int main(void) {
-    check(lightning_abi_version() == 1, "ABI version 1");
+    check(lightning_abi_version() == 2, "ABI version 2");
     for (int s = LA_OK; s <= LA_ERR_TIMEOUT; ++s)
         check(lightning_status_string(s) != NULL && strlen(lightning_status_string(s)) > 0, "status strings");
 
     check(lightning_prefill_snapshot_count(131072, 16384) == 8, "snapshot count");
     check(lightning_prefill_snapshot_count(-1, 16) == -1, "snapshot count of a bad length");
-    check(lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 0, "prefill needs no workspace");
+    check(lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 64 * 32,
+          "the CTA-pair prefill's workspace: 32 bytes per (batch, head)");
     check(lightning_prefill_backward_noalloc_capacity() > 0, "no-alloc backward capacity");
     check(lightning_gqa_decode_workspace_size(8, 64, 131072) > 0, "GQA decode workspace");
     check(lightning_prefill_selected_variant(LA_DTYPE_BF16, 1, 64, 131072, 128, 256, LA_VARIANT_AUTO) ==
@@ -44,10 +45,13 @@ int main(void) {
                             NULL, 0, NULL) == LA_ERR_UNSUPPORTED, "dim 96 unsupported");
     check(lightning_prefill(fake(0), fake(1), fake(2), LA_DTYPE_BF16, slopes, 1, 2, 16, 128, 256, NULL, (void *)fake(0),
                             state_out, NULL, 0, NULL) == LA_ERR_INVALID_ARG, "o overlapping q");
+    check(lightning_prefill(fake(0), fake(1), fake(2), LA_DTYPE_BF16, slopes, 1, 2, 16, 128, 256, NULL, o, state_out,
+                            NULL, 0, NULL) == LA_ERR_INVALID_ARG, "the CTA-pair prefill without its workspace");
     check(lightning_decode(fake(0), fake(1), fake(2), (la_dtype)7, slopes, 1, 2, 128, state, o, NULL) ==
               LA_ERR_INVALID_ARG, "bad dtype");
     check(lightning_prefill_norm_gate(fake(0), fake(1), fake(2), LA_DTYPE_F32, slopes, 1, 2, 16, 128, 256, NULL,
-                                      fake(7), (const float *)fake(8), 1e-6f, (void *)fake(9), NULL, NULL) ==
+                                      fake(7), (const float *)fake(8), 1e-6f, (void *)fake(9), NULL, NULL, 0,
+                                      NULL) ==
               LA_ERR_UNSUPPORTED, "fused norm + gate needs bf16");
     /* nothing to do: returns before touching the device */
     check(lightning_prefill(fake(0), fake(1), fake(2), LA_DTYPE_BF16, slopes, 0, 2, 16, 128, 256, NULL, o, state_out,

@@ -27,21 +27,27 @@ def test_every_declared_function_is_exported():
 
 
 def test_version_and_status_strings():
-    assert abi.lightning_abi_version() == 1
+    assert abi.lightning_abi_version() == 2
     for st in range(5):
         assert abi.status_string(st).startswith("LA_")
     assert abi.status_string(99) == "unknown status"
 
 
-def test_workspace_is_zero():
-    assert abi.lightning_prefill_workspace_size(16, 64, 4096, 128, 256) == 0
+def test_prefill_workspace_holds_the_range_guard_records():
+    # 32 bytes per (batch, head) for the CTA-pair kernel (block 256, dim 128); none otherwise
+    assert abi.lightning_prefill_workspace_size(16, 64, 4096, 128, 256) == 16 * 64 * 32
+    assert abi.lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 64 * 32
+    assert abi.lightning_prefill_workspace_size(1, 2, 256, 64, 64) == 0
+    assert abi.lightning_prefill_workspace_size(1, 2, 256, 128, 128) == 0
+    assert abi.lightning_prefill_workspace_size(-1, 2, 256, 128, 256) == 0
 
 
 # Fake, well-aligned, non-overlapping "device" addresses: every call below must
 # be rejected (or finish trivially) before any CUDA call is made.
 Q, K, V, O, SL, S0, S1 = (0x10000000 * (i + 1) for i in range(7))
+PWS = 0x10000000 * 40  # fake prefill workspace
 GOOD = dict(q=Q, k=K, v=V, dtype=abi.LA_DTYPE_BF16, slopes=SL, batch=1, heads=2, seq=16, dim=128,
-            block=256, state_in=S0, o=O, state_out=S1)
+            block=256, state_in=S0, o=O, state_out=S1, pws=PWS, pws_bytes=4096)
 
 
 def _prefill(variant=abi.LA_VARIANT_AUTO, **kw):
@@ -49,7 +55,7 @@ def _prefill(variant=abi.LA_VARIANT_AUTO, **kw):
     a.update(kw)
     return abi.lightning_prefill_ex(a["q"], a["k"], a["v"], a["dtype"], a["slopes"], a["batch"],
                                     a["heads"], a["seq"], a["dim"], a["block"], a["state_in"], a["o"],
-                                    a["state_out"], None, 0, None, variant)
+                                    a["state_out"], a["pws"], a["pws_bytes"], None, variant)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -67,6 +73,10 @@ def _prefill(variant=abi.LA_VARIANT_AUTO, **kw):
     (dict(o=Q + 256), abi.LA_ERR_INVALID_ARG),          # o overlaps q
     (dict(state_out=V), abi.LA_ERR_INVALID_ARG),        # state overlaps v
     (dict(state_out=S0 + 4096), abi.LA_ERR_INVALID_ARG),  # partial overlap with state_in
+    (dict(pws=None, pws_bytes=0), abi.LA_ERR_INVALID_ARG),  # the CTA-pair kernel needs its workspace
+    (dict(pws_bytes=32), abi.LA_ERR_INVALID_ARG),           # 2 heads need 64 bytes
+    (dict(pws=PWS + 8), abi.LA_ERR_INVALID_ARG),            # misaligned workspace
+    (dict(pws=V + 64), abi.LA_ERR_INVALID_ARG),             # workspace overlaps v
 ])
 def test_prefill_argument_errors(kw, status):
     assert _prefill(**kw) == status
@@ -125,7 +135,8 @@ def _prefill_snapshots(interval=256, snapshots=SN, variant=abi.LA_VARIANT_AUTO, 
     a.update(kw)
     return abi.lightning_prefill_snapshots(a["q"], a["k"], a["v"], a["dtype"], a["slopes"], a["batch"],
                                            a["heads"], a["seq"], a["dim"], a["block"], a["state_in"], a["o"],
-                                           a["state_out"], interval, snapshots, None, variant)
+                                           a["state_out"], interval, snapshots, a["pws"], a["pws_bytes"], None,
+                                           variant)
 
 
 def test_snapshot_count():
@@ -198,11 +209,15 @@ def test_backward_argument_errors(kw, status):
 
 def test_backward_workspace_size():
     ws = abi.lightning_prefill_backward_workspace_size
-    # no kernel needs a workspace: the anti-causal passes read their operands in place
-    for dt, blk, var in ((abi.LA_DTYPE_BF16, 256, abi.LA_VARIANT_AUTO), (abi.LA_DTYPE_BF16, 256, abi.LA_VARIANT_SIMT),
-                         (abi.LA_DTYPE_F32, 64, abi.LA_VARIANT_AUTO)):
+    # the three tensor-core passes keep one range-guard record (32 bytes) per (batch, head)
+    # each; the CUDA-core passes need no workspace
+    assert ws(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_AUTO) == 3 * 64 * 32
+    assert ws(abi.LA_DTYPE_BF16, 2, 64, 131072, 128, 256, abi.LA_VARIANT_TCGEN05_PAIR) == 3 * 2 * 64 * 32
+    for dt, blk, var in ((abi.LA_DTYPE_BF16, 256, abi.LA_VARIANT_SIMT), (abi.LA_DTYPE_F32, 64, abi.LA_VARIANT_AUTO)):
         assert ws(dt, 1, 64, 131072, 128, blk, var) == 0
     assert _backward(ws=None, ws_bytes=0, batch=0) == abi.LA_OK
+    assert _backward(ws=None, ws_bytes=0) == abi.LA_ERR_INVALID_ARG          # the tensor-core passes need it
+    assert _backward(ws_bytes=3 * 2 * 32 - 16) == abi.LA_ERR_INVALID_ARG     # 2 heads need 192 bytes
 
 
 def test_backward_trivial_calls_need_no_gpu():
@@ -249,7 +264,7 @@ def _prefill_norm_gate(**kw):
     a.update(kw)
     return abi.lightning_prefill_norm_gate(a["q"], a["k"], a["v"], a["dtype"], a["slopes"], a["batch"], a["heads"],
                                            a["seq"], a["dim"], a["block"], a["state_in"], a["gate"], a["gamma"],
-                                           a["eps"], a["y"], a["state_out"], None)
+                                           a["eps"], a["y"], a["state_out"], a["pws"], a["pws_bytes"], None)
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -114,6 +114,6 @@ def test_prefill_norm_gate_rejects_what_the_pair_kernel_does_not_take():
         rc = abi.lightning_prefill_norm_gate(
             inp["q"].data_ptr(), inp["k"].data_ptr(), inp["v"].data_ptr(), 0 if dtype == torch.float32 else 1,
             inp["slopes"].data_ptr(), 1, 2, 64, 128, block, None, gate.data_ptr(), gamma.data_ptr(), EPS,
-            y.data_ptr(), None, stream)
+            y.data_ptr(), None, None, 0, stream)
         assert rc == abi.LA_ERR_UNSUPPORTED
     assert abi.lightning_device_status(stream) == abi.LA_OK
