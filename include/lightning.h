@@ -112,18 +112,21 @@ int lightning_abi_version(void);
  * Input range of the tensor-core kernels. They round the operands they form
  * (P ⊙ D, Q ⊙ d_q, K ⊙ d_k, V and the carried state) to fp16, whose range is
  * narrower than bf16's. The CTA-pair kernel guards against that: while it
- * runs it bounds every such operand of each (batch, head) from the largest
- * row norms of q and k, the largest |v| and the largest |state_in| element;
- * a head whose operands could pass 2^15, or whose row norms fall below 2^-8,
- * is recomputed by a second launch with q, k and v scaled by powers of two
- * (exact) so that they sit in fp16's normal range, and scaled back. Its
- * results meet the error bound for any scale of q, k, v and state_in within
- * about 2^-36 .. 2^44, provided the values inside one (batch, head) span less
- * than about 2^14 (a few rows 2^8 above the rest, with |q.k| above 65504, are
- * covered). Inputs holding inf or NaN give non-finite results. The
- * single-CTA kernel (LA_VARIANT_TCGEN05) has no guard: its operands must stay
- * inside fp16's range (|q.k|, |q|, |k|, |v| and the state below 65504) and its
- * row norms near or above 2^-8 for the bound to hold.
+ * runs it takes, per (batch, head), the largest |q|, |k|, |v| and |state_in|
+ * element, which bound every such operand; a head whose operands could pass
+ * 2^15, or whose maxima fall below 2^-9, is recomputed by a second launch with
+ * q, k and v scaled by powers of two (exact) chosen from the head's largest
+ * row norms of q and k, so that the operands sit in fp16's normal range, and
+ * the results scaled back. The results then meet the error bound for any
+ * scale of q, k, v and state_in whose row norms lie within about
+ * 2^-36 .. 2^44, provided the values inside one (batch, head) span less than
+ * about 2^14 (for example a few rows 2^8 above the rest, with |q.k| above
+ * 65504, are covered). Inputs holding inf or NaN give non-finite results.
+ * The single-CTA kernel (LA_VARIANT_TCGEN05) has no guard: its operands must
+ * stay inside fp16's range (|q.k|, |q|, |k|, |v| and the state below 65504)
+ * and its inputs' elements near or above 2^-9 in magnitude for the bound to
+ * hold (scales 2^-10 .. 2^8 of the workloads' inputs, one tensor at a time,
+ * are tested).
  */
 la_status lightning_prefill(const void *q, const void *k, const void *v, la_dtype dtype,
                             const float *slopes, int batch, int heads, int seq, int dim,
