@@ -101,7 +101,7 @@ int lightning_abi_version(void);
  *   workspace, workspace_bytes
  *              device scratch, caller-owned, 16-byte aligned, overlapping no
  *              other buffer, of at least lightning_prefill_workspace_size
- *              bytes: 32 bytes per (batch, head) for the CTA-pair tensor-core
+ *              bytes: 48 bytes per (batch, head) for the CTA-pair tensor-core
  *              kernel (its range guard, below), none for the other kernels
  *              (NULL/0 is fine there). Too little returns LA_ERR_INVALID_ARG.
  *              Its contents need no initialisation; calls that share one
@@ -148,7 +148,7 @@ int lightning_prefill_selected_variant(la_dtype dtype, int batch, int heads, int
                                        int block, int variant);
 
 /* Bytes of workspace lightning_prefill (with AUTO, bf16 inputs) needs for these
- * sizes: 32 * batch * heads for the CTA-pair kernel (dim 128, block 256), 0
+ * sizes: 48 * batch * heads for the CTA-pair kernel (dim 128, block 256), 0
  * otherwise. Enough for every variant and dtype. Host only. */
 size_t lightning_prefill_workspace_size(int batch, int heads, int seq, int dim, int block);
 
@@ -206,7 +206,7 @@ la_status lightning_prefill_snapshots(const void *q, const void *k, const void *
  *   workspace, workspace_bytes
  *                 scratch of at least lightning_prefill_backward_workspace_size
  *                 bytes: the range guard's records of the three tensor-core
- *                 passes (96 bytes per (batch, head); see lightning_prefill),
+ *                 passes (144 bytes per (batch, head); see lightning_prefill),
  *                 none on CUDA cores (NULL/0 is fine there); 16-byte aligned,
  *                 overlapping nothing else, no initialisation needed.
  * All device pointers, caller-owned, 16-byte aligned. No output may overlap
@@ -225,12 +225,12 @@ la_status lightning_prefill_backward(const void *q, const void *k, const void *v
  * hands out none at the point of the call, or a plugin inside another
  * framework that may not call cudaMalloc. The pages have no counterpart to
  * this entry point. It allocates nothing: the scratch the tensor-core passes
- * need (the range guard's records, 96 bytes per (batch, head)) comes from a
+ * need (the range guard's records, 144 bytes per (batch, head)) comes from a
  * fixed array inside the library, 4 MiB on every device that loads it, kept
  * until the process exits (lightning_prefill_backward_noalloc_capacity()).
  * Arguments and results are those of lightning_prefill_backward; argument
  * errors come in the same order, then a request that needs more scratch than
- * the array holds (more than 43690 batch x heads) returns LA_ERR_UNSUPPORTED,
+ * the array holds (more than 29127 batch x heads) returns LA_ERR_UNSUPPORTED,
  * all before any launch.
  * The first call on a device looks up the array's address on that device
  * (with that device current): make that first call before any stream capture.
@@ -292,7 +292,7 @@ la_status lightning_norm_gate(const void *o, const void *gate, la_dtype dtype, c
  *   y      [batch][seq][heads*128] bf16; written; must not overlap any input,
  *          the states, gate or gamma.
  *   workspace, workspace_bytes: as for lightning_prefill (the CTA-pair
- *          kernel's range guard: 32 bytes per (batch, head)).
+ *          kernel's range guard: 48 bytes per (batch, head)).
  * Runs on the CTA-pair tensor-core kernel only: bf16, dim 128, block 256;
  * other shapes or dtypes return LA_ERR_UNSUPPORTED before any launch (the
  * whole-token mean needs every head of a token, which one head's kernel does

@@ -403,7 +403,7 @@ struct BackwardArgs {
 
 // Scratch of lightning_prefill_backward_noalloc: a fixed device array, so that
 // entry point needs no workspace from the caller and allocates nothing. 4 MiB
-// hold the three passes' range-guard records for 43690 (batch, head) pairs.
+// hold the three passes' range-guard records for 29127 (batch, head) pairs.
 constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

@@ -172,6 +172,16 @@ __device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parit
     const bool ok = leader ? wait_bar(c, idx, parity) : true;
     return ptx::named_bar_and(bar_id, 128, ok);
 }
+// two fp32 sums in one instruction (each rounded as a plain add)
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
 // two fp32 products in one instruction (each rounded as a plain multiply)
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
     float2 d;
@@ -321,12 +331,20 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     float *state_out, Snapshots sn, PairPass pp, PairNormGate ng, rg::RangeRec *rec,
                     const __nv_bfloat16 *qg, const __nv_bfloat16 *kg) {
     extern __shared__ uint8_t smem_raw[];
+    // pass 1: pass 2 may be scheduled now (it waits for this grid's completion before
+    // reading anything), so that its launch overlaps this one
+    if (!kScaled && threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;");
     // operand scales: q, k, v, P = q k, the carried state, its inverse, and o's inverse
     float f_q = 1.f, f_k = 1.f, f_v = 1.f, f_p = 1.f, f_s = 1.f, f_su = 1.f, f_o = 1.f;
     if constexpr (kScaled) {
+        // pass 2 is launched as pass 1's programmatic dependent: wait until pass 1 has
+        // completed and its records are visible
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         const int bh0 = blockIdx.x >> 1;
-        const rg::RangeRec r = rec[bh0];
-        if (!r.flag) return;  // both CTAs of the pair read the same record and leave together
+        const rg::RangePart r = rg::combine(rec[bh0].part[0], rec[bh0].part[1]);
+        const bool flag = !rg::plain_ok(r, slopes[bh0 % heads], seq);
+        if (threadIdx.x == 0 && (blockIdx.x & 1) == 0) rec[bh0].flag = flag ? 1 : 0;
+        if (!flag) return;  // both CTAs of the pair read the same record and leave together
         // the head's largest row norms of q and k, fp32 sums: this CTA takes every other
         // row, then the two CTAs exchange through the output staging tile (first written
         // after the set-up's cluster barrier, which the other CTA reaches only after its read)
@@ -470,10 +488,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------ range guard (pass 1)
-        // Lane 0 combines this CTA's maxima (warpgroups A and B measure k, v and q as they
-        // convert them; warpgroup 3 measures state_in) with the other CTA's, and sets the
-        // head's verdict.
-        if (!kScaled && lane == 0) {
+        // With the state carried in place (state_out == state_in), lane 0 combines this
+        // CTA's maxima with the other CTA's and sets the verdict here, so that the final
+        // state of a head pass 2 will recompute is not overwritten (pass 2 reads it).
+        if (!kScaled && lane == 0 && state_out != nullptr && state_out == state_in) {
             const uint32_t *misc = reinterpret_cast<const uint32_t *>(c.smem + kOffMisc);
             float *peer = reinterpret_cast<float *>(c.smem + kOffMisc + kMiscPeer);
             bool ok = wait_bar(c, SCAN_FIN, 0) && wait_bar(c, SIN_DONE, 0);
@@ -491,15 +509,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                              : "memory");
                 ok = ptx::mbar_wait_cluster(&c.bars[PEER], 0, c.abort);
                 if (ok) {
-                    rg::RangeRec r;
-                    r.mq = fmaxf(v4[0], peer[0]);
-                    r.mk = fmaxf(v4[1], peer[1]);
-                    r.mv = fmaxf(v4[2], peer[2]);
-                    r.msin = fmaxf(v4[3], peer[3]);
-                    r.flag = rg::plain_ok(r, s, seq) ? 0 : 1;
-                    r.pad[0] = r.pad[1] = r.pad[2] = 0;
-                    *reinterpret_cast<volatile int *>(c.smem + kOffMisc + kMiscFlag) = r.flag;
-                    if (rank == 0) rec[bh] = r;
+                    const rg::RangePart r = rg::combine(rg::RangePart{v4[0], v4[1], v4[2], v4[3]},
+                                                        rg::RangePart{peer[0], peer[1], peer[2], peer[3]});
+                    *reinterpret_cast<volatile int *>(c.smem + kOffMisc + kMiscFlag) = rg::plain_ok(r, s, seq) ? 0 : 1;
                     ptx::mbar_arrive(&c.bars[RANGE_DONE]);
                 }
             }
@@ -699,7 +711,18 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (grp == 0) atomicMax(misc + kMiscMv / 4, __float_as_uint(m1));
             }
             ptx::named_bar_sync(bar_id, 128);
-            if (leader) ptx::mbar_arrive(&c.bars[SCAN_FIN]);
+            if (leader) {
+                // this CTA's share of the head's maxima, for pass 2
+                const uint32_t *misc = reinterpret_cast<const uint32_t *>(c.smem + kOffMisc);
+                rg::RangePart &part = rec[bh].part[rank];
+                if (grp == 0) {
+                    part.mk = __uint_as_float(misc[kMiscMk / 4]);
+                    part.mv = __uint_as_float(misc[kMiscMv / 4]);
+                } else {
+                    part.mq = __uint_as_float(misc[kMiscMq / 4]);
+                }
+                ptx::mbar_arrive(&c.bars[SCAN_FIN]);
+            }
         }
     } else if (warp >= 12) {
         // ------------------------------------------------------------ warpgroup 3
@@ -794,10 +817,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (!group_wait(c, DS_FULL, par, leader, kBarW3)) goto w3_done;
                 ptx::tc_fence_after();
             }
-            // pass 1 writes the final state only for a head the range guard passed, so that
-            // an in-place carry (state_out == state_in) is still intact for pass 2
+            // with the state carried in place (state_out == state_in), pass 1 writes the final
+            // state only for a head the range guard passed, so that pass 2 can still read it
             bool write_state = state_out != nullptr;
-            if (!kScaled && last && write_state) {
+            if (!kScaled && last && write_state && state_out == state_in) {
                 if (!group_wait(c, RANGE_DONE, 0, leader, kBarW3)) goto w3_done;
                 write_state = *reinterpret_cast<volatile int *>(c.smem + kOffMisc + kMiscFlag) == 0;
             }
@@ -837,7 +860,11 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float m = rg::warp_max_nonneg(msin);
                     if ((l & 31) == 0) atomicMax(reinterpret_cast<uint32_t *>(c.smem + kOffMisc + kMiscSin), __float_as_uint(m));
                     ptx::named_bar_sync(kBarW3, 128);
-                    if (leader) ptx::mbar_arrive(&c.bars[SIN_DONE]);
+                    if (leader) {
+                        rec[bh].part[rank].msin = __uint_as_float(*reinterpret_cast<const uint32_t *>(
+                            c.smem + kOffMisc + kMiscSin));
+                        ptx::mbar_arrive(&c.bars[SIN_DONE]);
+                    }
                 }
             }
             if (t < 0) continue;
@@ -875,11 +902,13 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (leader) arrive_leader(&c.bars[O_FREE]);
                 uint8_t *erow = c.smem + kOffE + l * 128;
                 const float rstd = kNormGate ? rsqrtf(ss * (1.f / kDim) + ng.eps) : 0.f;
+                const float hr = 0.5f * rstd;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     if (kNormGate) {
                         // y = gamma o rstd sigmoid(g) on this half's 64 columns, written over the
-                        // gate row in the staging tile; sigmoid(g) = 1/2 + tanh(g/2)/2 (SFU tanh)
+                        // gate row in the staging tile, as (gamma rstd / 2) o (1 + tanh(g/2)) in
+                        // paired fp32 operations (SFU tanh)
                         if (hh == 1 && leader) load_gate(t, 1);
                         if (!group_wait(c, G_FULL, (uint32_t)hh, leader, kBarW3)) goto w3_done;
 #pragma unroll
@@ -894,11 +923,15 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const uint32_t w = pk[32 * hh + 4 * ch + e];
+                                const float2 ga = mul2(make_float2(ptx::bf16_lo(gw[e]), ptx::bf16_hi(gw[e])),
+                                                       make_float2(0.5f, 0.5f));
                                 float th0, th1;
-                                asm("tanh.approx.f32 %0, %1;" : "=f"(th0) : "f"(0.5f * ptx::bf16_lo(gw[e])));
-                                asm("tanh.approx.f32 %0, %1;" : "=f"(th1) : "f"(0.5f * ptx::bf16_hi(gw[e])));
-                                yw[e] = ptx::pack_bf16(gm[2 * e] * ptx::bf16_lo(w) * rstd * fmaf(0.5f, th0, 0.5f),
-                                                       gm[2 * e + 1] * ptx::bf16_hi(w) * rstd * fmaf(0.5f, th1, 0.5f));
+                                asm("tanh.approx.f32 %0, %1;" : "=f"(th0) : "f"(ga.x));
+                                asm("tanh.approx.f32 %0, %1;" : "=f"(th1) : "f"(ga.y));
+                                const float2 cg = mul2(make_float2(gm[2 * e], gm[2 * e + 1]), make_float2(hr, hr));
+                                const float2 a = mul2(cg, make_float2(ptx::bf16_lo(w), ptx::bf16_hi(w)));
+                                const float2 yv = mul2(a, add2(make_float2(th0, th1), make_float2(1.f, 1.f)));
+                                yw[e] = ptx::pack_bf16(yv.x, yv.y);
                             }
                             *slot = make_uint4(yw[0], yw[1], yw[2], yw[3]);
                         }
@@ -972,7 +1005,7 @@ inline bool make_token_major_map(CUtensorMap *map, void *y, int batch, int heads
     return true;
 }
 
-// Workspace of one CTA-pair prefill: the range guard's record per (batch, head).
+// Workspace of one CTA-pair prefill: the range guard's record per (batch, head), 48 bytes.
 inline size_t pair_workspace_bytes(long long batch_heads) {
     return (size_t)batch_heads * sizeof(rg::RangeRec);
 }
@@ -1018,15 +1051,18 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     cfg.blockDim = dim3(pair::kThreads);
     cfg.dynamicSmemBytes = pair::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // pass 2 is pass 1's programmatic dependent (it starts with griddepcontrol.wait)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
     const pair::PairNormGate ngv = ng ? *ng : pair::PairNormGate{nullptr, nullptr, 0.f};
     for (int pass = 0; pass < 2; ++pass) {
+        cfg.numAttrs = pass == 0 ? 1 : 2;
         cudaError_t e = cudaFuncSetAttribute(passes[pass], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)pair::kSmemBytes);
         if (e != cudaSuccess) {

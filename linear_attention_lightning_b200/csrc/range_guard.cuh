@@ -10,18 +10,20 @@
 // by 2^(b+c)) scales o by 2^(a+b+c) and the state by 2^(b+c) exactly, with no
 // rounding: the guard picks such exponents per (batch, head).
 //
-// Pass 1 (the plain kernel) also measures each (batch, head) while it runs, on
-// warps that have no other work: the largest |q|, |k| and |v| element and the
-// largest |state_in| element. These bound every fp16 operand: |Q ⊙ d_q| <= max|q|,
+// Pass 1 (the plain kernel) also measures each (batch, head) while it runs, in
+// the warps that convert the operands (one packed max per word already in a
+// register): the largest |q|, |k| and |v| element and the largest |state_in|
+// element. These bound every fp16 operand: |Q ⊙ d_q| <= max|q|,
 // |K ⊙ d_k| <= max|k|, |V| <= max|v|, |P ⊙ D| <= d max|q| max|k| (d = 128), and
 // each state element |S| <= max|S_in| + max|k| max|v| W, W = the sum over the
 // call's tokens of the decay = min(L, 1 / (1 - e^{-s})). A head whose bounds
 // keep every operand below 2^15 and its maxima at or above 2^-9 (so that the
 // operands' bulk stays in fp16's normal range) is done. Any other head is
-// flagged; a second launch (pass 2) recomputes exactly those heads with
-// power-of-two scales, and leaves the others alone. Pass 1 does not write the
-// final state of a flagged head, so an in-place state carry stays intact for
-// pass 2.
+// flagged; a second launch (pass 2) takes the verdict and recomputes exactly the
+// flagged heads with power-of-two scales, leaving the others alone. Pass 1 learns
+// the verdict itself only when the state is carried in place (state_out ==
+// state_in): its two CTAs then exchange their maxima, and it does not write the
+// final state of a flagged head, which pass 2 still has to read.
 //
 // Pass 2 first measures the flagged head's largest row norms of q and k (a
 // tighter bound on |P ⊙ D| = |q_i . k_j| <= ||q_i|| ||k_j|| than the elementwise
@@ -34,17 +36,26 @@
 namespace la {
 namespace rg {
 
-// One record per (batch, head) in the caller's workspace, written by pass 1 and
-// read by pass 2: the measured maxima and the verdict.
-struct RangeRec {
+// The maxima one CTA of a pair measured, over its share of the head's q, k, v and
+// state_in (the pair's two shares together cover them).
+struct RangePart {
     float mq;    // largest |q| element
     float mk;    // largest |k| element
     float mv;    // largest |v| element
     float msin;  // largest |state_in| element (0 without a carried-in state)
-    int flag;    // 1: recompute with scaled operands (pass 2)
+};
+// One record per (batch, head) in the caller's workspace: pass 1 writes the two
+// parts, pass 2 combines them, decides, and writes the verdict.
+struct RangeRec {
+    RangePart part[2];
+    int flag;    // written by pass 2: 1 if the head took the scaled recomputation
     int pad[3];
 };
-static_assert(sizeof(RangeRec) == 32, "RangeRec is 32 bytes");
+static_assert(sizeof(RangeRec) == 48, "RangeRec is 48 bytes");
+
+__device__ __forceinline__ RangePart combine(const RangePart &a, const RangePart &b) {
+    return RangePart{fmaxf(a.mq, b.mq), fmaxf(a.mk, b.mk), fmaxf(a.mv, b.mv), fmaxf(a.msin, b.msin)};
+}
 
 constexpr float kHi = 32768.f;            // 2^15: every fp16 operand stays below this (fp16 max 65504)
 constexpr float kLoElem = 0.001953125f;   // 2^-9: elementwise maxima below this are scaled up
@@ -92,7 +103,7 @@ __device__ __forceinline__ bool finite(float x) { return x == x && fabsf(x) <= 3
 // Pass 1's verdict: true when the plain kernel's fp16 operands all stay below
 // 2^15 and its maxima at or above 2^-9. Non-finite maxima (inputs holding inf
 // or NaN) keep pass 1's result: scaling cannot make such a result finite.
-__device__ __forceinline__ bool plain_ok(const RangeRec &r, float s, int seq) {
+__device__ __forceinline__ bool plain_ok(const RangePart &r, float s, int seq) {
     if (!finite(r.mq) || !finite(r.mk) || !finite(r.mv) || !finite(r.msin)) return true;
     const float W = decay_window(s, seq);
     const bool hi = fmaxf(fmaxf(r.mq, r.mk), r.mv) <= kHi * 0.5f && 128.f * r.mq * r.mk <= kHi &&

@@ -28,8 +28,8 @@ int main(void) {
 
     check(lightning_prefill_snapshot_count(131072, 16384) == 8, "snapshot count");
     check(lightning_prefill_snapshot_count(-1, 16) == -1, "snapshot count of a bad length");
-    check(lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 64 * 32,
-          "the CTA-pair prefill's workspace: 32 bytes per (batch, head)");
+    check(lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 64 * 48,
+          "the CTA-pair prefill's workspace: 48 bytes per (batch, head)");
     check(lightning_prefill_backward_noalloc_capacity() > 0, "no-alloc backward capacity");
     check(lightning_gqa_decode_workspace_size(8, 64, 131072) > 0, "GQA decode workspace");
     check(lightning_prefill_selected_variant(LA_DTYPE_BF16, 1, 64, 131072, 128, 256, LA_VARIANT_AUTO) ==

@@ -34,9 +34,9 @@ def test_version_and_status_strings():
 
 
 def test_prefill_workspace_holds_the_range_guard_records():
-    # 32 bytes per (batch, head) for the CTA-pair kernel (block 256, dim 128); none otherwise
-    assert abi.lightning_prefill_workspace_size(16, 64, 4096, 128, 256) == 16 * 64 * 32
-    assert abi.lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 64 * 32
+    # 48 bytes per (batch, head) for the CTA-pair kernel (block 256, dim 128); none otherwise
+    assert abi.lightning_prefill_workspace_size(16, 64, 4096, 128, 256) == 16 * 64 * 48
+    assert abi.lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 64 * 48
     assert abi.lightning_prefill_workspace_size(1, 2, 256, 64, 64) == 0
     assert abi.lightning_prefill_workspace_size(1, 2, 256, 128, 128) == 0
     assert abi.lightning_prefill_workspace_size(-1, 2, 256, 128, 256) == 0
@@ -74,7 +74,7 @@ def _prefill(variant=abi.LA_VARIANT_AUTO, **kw):
     (dict(state_out=V), abi.LA_ERR_INVALID_ARG),        # state overlaps v
     (dict(state_out=S0 + 4096), abi.LA_ERR_INVALID_ARG),  # partial overlap with state_in
     (dict(pws=None, pws_bytes=0), abi.LA_ERR_INVALID_ARG),  # the CTA-pair kernel needs its workspace
-    (dict(pws_bytes=32), abi.LA_ERR_INVALID_ARG),           # 2 heads need 64 bytes
+    (dict(pws_bytes=48), abi.LA_ERR_INVALID_ARG),           # 2 heads need 96 bytes (48 each)
     (dict(pws=PWS + 8), abi.LA_ERR_INVALID_ARG),            # misaligned workspace
     (dict(pws=V + 64), abi.LA_ERR_INVALID_ARG),             # workspace overlaps v
 ])
@@ -209,15 +209,15 @@ def test_backward_argument_errors(kw, status):
 
 def test_backward_workspace_size():
     ws = abi.lightning_prefill_backward_workspace_size
-    # the three tensor-core passes keep one range-guard record (32 bytes) per (batch, head)
+    # the three tensor-core passes keep one range-guard record (48 bytes) per (batch, head)
     # each; the CUDA-core passes need no workspace
-    assert ws(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_AUTO) == 3 * 64 * 32
-    assert ws(abi.LA_DTYPE_BF16, 2, 64, 131072, 128, 256, abi.LA_VARIANT_TCGEN05_PAIR) == 3 * 2 * 64 * 32
+    assert ws(abi.LA_DTYPE_BF16, 1, 64, 131072, 128, 256, abi.LA_VARIANT_AUTO) == 3 * 64 * 48
+    assert ws(abi.LA_DTYPE_BF16, 2, 64, 131072, 128, 256, abi.LA_VARIANT_TCGEN05_PAIR) == 3 * 2 * 64 * 48
     for dt, blk, var in ((abi.LA_DTYPE_BF16, 256, abi.LA_VARIANT_SIMT), (abi.LA_DTYPE_F32, 64, abi.LA_VARIANT_AUTO)):
         assert ws(dt, 1, 64, 131072, 128, blk, var) == 0
     assert _backward(ws=None, ws_bytes=0, batch=0) == abi.LA_OK
     assert _backward(ws=None, ws_bytes=0) == abi.LA_ERR_INVALID_ARG          # the tensor-core passes need it
-    assert _backward(ws_bytes=3 * 2 * 32 - 16) == abi.LA_ERR_INVALID_ARG     # 2 heads need 192 bytes
+    assert _backward(ws_bytes=3 * 2 * 48 - 16) == abi.LA_ERR_INVALID_ARG     # 2 heads need 288 bytes
 
 
 def test_backward_trivial_calls_need_no_gpu():

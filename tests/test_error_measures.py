@@ -46,13 +46,28 @@ def test_format_rounding_and_the_sigmoid_allowance_read_zero():
     ob = torch.tensor(o64).to(torch.bfloat16).double().numpy()
     yb = torch.tensor(oracle_norm_gate_of(ob, gate, gamma)).to(torch.bfloat16).double().numpy()
     assert norm_gate_y_err_in_o_units(yb, y_ref, o64, gate, gamma) == 0.0
-    # a sigmoid off by 2.5e-4 everywhere (the SFU approximation's size) is allowed; by 5e-3, not
+    # a sigmoid off by the documented bound of the SFU approximation everywhere is allowed
+    # (2^-12 + 2^-24: tanh.approx.f32's relative error of at most 2^-11, halved, plus the
+    # fma's rounding); off by 5e-3, not
     b, h, L, d = o64.shape
     gf = gate.float().numpy().reshape(b, L, h, d)
     o = np.transpose(o64, (0, 2, 1, 3))
     rstd = 1.0 / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + 1e-6)
     gm = gamma.numpy().reshape(h, d)[None, None]
-    for off, ok in ((2.5e-4, True), (5e-3, False)):
+    for off, ok in ((2.0 ** -12, True), (5e-3, False)):
         y_off = (gm * o * rstd * (1.0 / (1.0 + np.exp(-gf)) + off)).reshape(b, L, h * d)
         e = norm_gate_y_err_in_o_units(y_off, y_ref, o64, gate, gamma)
         assert (e == 0.0) == ok, (off, e)
+
+
+def test_the_per_head_reading_sees_an_error_in_one_head_against_that_head():
+    from parity import y_err_per_head
+    o64, gate, gamma = _case(2)
+    y_ref = oracle_norm_gate_of(o64, gate, gamma)
+    b, L, hd = y_ref.shape
+    y_bad = y_ref.copy().reshape(b, L, 2, hd // 2)
+    rms1 = float(np.sqrt(np.mean(y_bad[:, :, 1] ** 2)))
+    y_bad[0, 3, 1, 5] += 0.1 * rms1
+    e = y_err_per_head(y_bad.reshape(b, L, hd), y_ref, 2)
+    assert 0.09 <= e <= 0.101, e
+    assert y_err_per_head(y_ref, y_ref, 2) == 0.0

@@ -9,7 +9,7 @@ import linear_attention_lightning_b200 as la
 from linear_attention_lightning_b200 import abi, inputs
 
 from parity import (NG_EPS, TOL, guarded_empty, guards_intact, norm_gate_y_err_in_o_units as _y_err_in_o_units,
-                    oracle_norm_gate_of as _oracle_y, oracle_prefill, rel_err, to_f64)
+                    oracle_norm_gate_of as _oracle_y, oracle_prefill, rel_err, to_f64, y_err_per_head)
 
 pytestmark = pytest.mark.gpu
 
@@ -36,9 +36,11 @@ def _run(b, h, L, state_in, seed):
     if L > 0:
         ref = _oracle_y(o64, gate, gamma)
         e = _y_err_in_o_units(to_f64(y), ref, o64, gate, gamma)
-        print("prefill_norm_gate b%d h%d L%d: error %.3g rms(o) through dy/do (%.3g rms(y) as is)"
-              % (b, h, L, e, rel_err(to_f64(y), ref, bf16_out=1)))
+        ep = y_err_per_head(to_f64(y), ref, h)
+        print("prefill_norm_gate b%d h%d L%d: error %.3g rms(o) through dy/do, %.3g rms(y) per head as is"
+              % (b, h, L, e, ep))
         assert e <= TOL[torch.bfloat16], "y error %.3g rms(o) through dy/do > %.3g" % (e, TOL[torch.bfloat16])
+        assert ep <= TOL[torch.bfloat16], "y error %.3g rms(y) per head > %.3g" % (ep, TOL[torch.bfloat16])
     es = rel_err(to_f64(s_out), s64)
     assert es <= TOL[torch.bfloat16], "state_out error %.3g rms" % es
     return inp, gate, gamma, y, s_out
@@ -98,9 +100,11 @@ def test_prefill_norm_gate_8k_workload_sampled_heads():
     ref = _oracle_y(o64, gate, gamma, heads_idx=heads)
     got = to_f64(y).reshape(w.batch, w.seq, w.heads, w.dim)[:, :, heads].reshape(ref.shape)
     e = _y_err_in_o_units(got, ref, o64, gate, gamma, heads_idx=heads)
-    print("prefill_norm_gate 8k sampled heads: error %.3g rms(o) through dy/do (%.3g rms(y) as is)"
-          % (e, rel_err(got, ref, bf16_out=1)))
+    ep = y_err_per_head(got, ref, len(heads))
+    print("prefill_norm_gate 8k sampled heads: error %.3g rms(o) through dy/do, %.3g rms(y) per head as is"
+          % (e, ep))
     assert e <= TOL[torch.bfloat16]
+    assert ep <= TOL[torch.bfloat16], "y error %.3g rms(y) per head" % ep
     assert rel_err(to_f64(s_out[:, heads]), s64) <= TOL[torch.bfloat16]
 
 

@@ -8,7 +8,7 @@ while it runs and recomputes, with power-of-two operand scales, the heads whose
 operands would leave fp16's range. These tests scale q, k, v and the carried
 state by powers of two (exact in bf16), put |q . k| above 65504 on a few rows,
 and hold every result to the bound of the workloads (max |err| <= 2e-2 rms).
-The guard's records (32 bytes per (batch, head) in the workspace) show which
+The guard's records (48 bytes per (batch, head) in the workspace) show which
 heads took the second pass."""
 import numpy as np
 import pytest
@@ -47,7 +47,7 @@ def _prefill_with_records(inp, block=256, variant="pair", state_out=None, in_pla
     o, s = la.prefill(q, inp["k"], inp["v"], inp["slopes"], block, s_in, state_out=state_out, variant=variant,
                       workspace=ws)
     torch.cuda.synchronize()
-    flags = ws[:need].view(torch.int32).view(b * h, 8)[:, 4].cpu().numpy() if need else None
+    flags = ws[:need].view(torch.int32).view(b * h, 12)[:, 8].cpu().numpy() if need else None
     return o, s, flags
 
 

@@ -39,14 +39,14 @@ def test_capacity_and_bad_requests_are_rejected_before_any_launch():
                                                 1, 64, 16, 128, 256, None, None, fake[5], fake[6], fake[7],
                                                 None, None, abi.LA_VARIANT_TCGEN05)
     assert st == abi.LA_ERR_INVALID_ARG  # not a backward variant
-    # more (batch, head) pairs than the array holds records for: 3 x 700 x 64 x 32 bytes > 4 MiB
+    # more (batch, head) pairs than the array holds records for: 3 x 456 x 64 x 48 bytes > 4 MiB
     st = abi.lightning_prefill_backward_noalloc(fake[0], fake[1], fake[2], fake[3], abi.LA_DTYPE_BF16, fake[4],
-                                                700, 64, 16, 128, 256, None, None, fake[5], fake[6], fake[7],
+                                                456, 64, 16, 128, 256, None, None, fake[5], fake[6], fake[7],
                                                 None, None, abi.LA_VARIANT_AUTO)
     assert st == abi.LA_ERR_UNSUPPORTED and "scratch" in abi.last_error_message()
-    assert abi.lightning_prefill_backward_workspace_size(abi.LA_DTYPE_BF16, 700, 64, 16, 128, 256,
+    assert abi.lightning_prefill_backward_workspace_size(abi.LA_DTYPE_BF16, 456, 64, 16, 128, 256,
                                                          abi.LA_VARIANT_AUTO) > CAPACITY
-    assert abi.lightning_prefill_backward_workspace_size(abi.LA_DTYPE_BF16, 682, 64, 16, 128, 256,
+    assert abi.lightning_prefill_backward_workspace_size(abi.LA_DTYPE_BF16, 455, 64, 16, 128, 256,
                                                          abi.LA_VARIANT_AUTO) <= CAPACITY
 
 
