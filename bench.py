@@ -785,12 +785,13 @@ def run_gqa_prefill_leg(dev, stream, args, world):
     o = torch.empty_like(q)
     need = abi.lightning_gqa_prefill_workspace_size(abi.LA_DTYPE_BF16, b, h, L, d)
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    start = torch.zeros((b,), dtype=torch.int32, device=dev)
     sp = stream.cuda_stream
 
     def step():
         abi.check(abi.lightning_gqa_prefill(q.data_ptr(), kn.data_ptr(), vn.data_ptr(), kc.data_ptr(), vc.data_ptr(),
-                                            abi.LA_DTYPE_BF16, 0, b, h, hk, L, d, L, 64, 1e4, 1.0 / d ** 0.5,
-                                            o.data_ptr(), ws.data_ptr(), need, sp))
+                                            abi.LA_DTYPE_BF16, start.data_ptr(), b, h, hk, L, d, L, 64, 1e4,
+                                            1.0 / d ** 0.5, o.data_ptr(), ws.data_ptr(), need, sp))
 
     steps = args.gqa_prefill_steps
     ms = timed("gqa_prefill", step, steps, args.warmup, stream, world, dev)
@@ -831,6 +832,7 @@ def run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world):
     ws = torch.empty(need, dtype=torch.uint8, device=dev)
     lneed = abi.lightning_prefill_workspace_size(b, w.heads, L, d, w.block)
     lws = torch.empty(max(lneed, 16), dtype=torch.uint8, device=dev)
+    gstart = torch.zeros((b,), dtype=torch.int32, device=dev)
     sp = stream.cuda_stream
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
 
@@ -846,8 +848,8 @@ def run_hybrid_leg(w, dev, stream, inp, vcode, dcode, args, world):
         if mark:
             ev[1].record(stream)
         abi.check(abi.lightning_gqa_prefill(q.data_ptr(), kn.data_ptr(), vn.data_ptr(), kc.data_ptr(), vc.data_ptr(),
-                                            dcode, 0, b, hq, hk, L, d, L, 64, 1e4, 1.0 / d ** 0.5, og.data_ptr(),
-                                            ws.data_ptr(), need, sp))
+                                            dcode, gstart.data_ptr(), b, hq, hk, L, d, L, 64, 1e4, 1.0 / d ** 0.5,
+                                            og.data_ptr(), ws.data_ptr(), need, sp))
         if mark:
             ev[2].record(stream)
 

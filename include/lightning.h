@@ -402,33 +402,43 @@ la_status lightning_gqa_decode(const void *q, const void *k_new, const void *v_n
 size_t lightning_gqa_decode_workspace_size(int batch, int heads, int cap);
 
 /*
- * Prefill of the same softmax attention layer: `seq` new tokens per sequence
- * at positions start .. start+seq-1, one `start` for the whole batch. Source
- * and readings as for lightning_gqa_decode; the causal order is that of the
- * decode step applied to each new token in turn. The new tokens' rotated keys
- * and their values are written into the caches at positions start+i, and
- *   o[b][h][i] = sum_{p <= start+i} softmax_p(scale * rope(q[b][h][i], start+i) . k_p) v_p,
- * k_p, v_p the cache rows (positions < start as given, the rest as written).
+ * Prefill of the same softmax attention layer: `seq` new tokens per sequence,
+ * sequence b's at positions start[b] .. start[b]+seq-1 (each sequence with a
+ * cached prefix of its own length). Source and readings as for
+ * lightning_gqa_decode (and §04: the KV cache grows per sequence); the causal
+ * order is that of the decode step applied to each new token in turn. The new
+ * tokens' rotated keys and their values are written into the caches at
+ * positions start[b]+i, and
+ *   o[b][h][i] = sum_{p <= start[b]+i} softmax_p(scale * rope(q[b][h][i], start[b]+i) . k_p) v_p,
+ * k_p, v_p the cache rows (positions < start[b] as given, the rest as written).
  *
  *   q                [batch][heads][seq][dim], dtype.
  *   k_new, v_new     [batch][kv_heads][seq][dim], dtype.
- *   k_cache, v_cache [batch][kv_heads][cap][dim], dtype; positions < start
- *                    read, positions start .. start+seq-1 written, the rest
- *                    neither read nor written. start + seq <= cap.
+ *   k_cache, v_cache [batch][kv_heads][cap][dim], dtype; positions < start[b]
+ *                    read, positions start[b] .. start[b]+seq-1 written, the
+ *                    rest never written (the last key tile a query reads may
+ *                    reach past start[b]+seq-1; those rows enter no result,
+ *                    whatever they hold).
+ *   start            DEVICE int32 [batch], 0 <= start[b] <= cap - seq. A
+ *                    start[b] outside that range skips sequence b (its caches
+ *                    and o are not written) and is reported as
+ *                    LA_ERR_INVALID_ARG through the status word (see
+ *                    lightning_last_device_status); the other sequences run.
  *   dtype            LA_DTYPE_BF16 (tensor cores) or LA_DTYPE_F32 (CUDA cores).
  *   dim 128; rot a multiple of 4, 0 <= rot <= dim; scale finite and > 0;
- *   batch <= 65535.
+ *   seq <= cap; batch <= 65535.
  *   o                [batch][heads][seq][dim], dtype; written.
  *   workspace        lightning_gqa_prefill_workspace_size(dtype, batch, heads,
  *                    seq, dim) bytes (the rotated queries), 16-byte aligned.
  * Device pointers, caller-owned, 16-byte aligned; the caches, o and the
- * workspace must not overlap any other buffer. seq == 0 or batch == 0 launches
- * nothing. Two launches: the rotation, then the attention: bf16 on the tensor
- * cores (tcgen05; bf16 operands, fp32 accumulation and softmax, P rounded to
- * bf16); float32 on CUDA cores (fp32 throughout, exact online softmax).
+ * workspace must not overlap any other buffer (start included). seq == 0 or
+ * batch == 0 launches nothing. Two launches: the rotation, then the attention:
+ * bf16 on the tensor cores (tcgen05; bf16 operands, fp32 accumulation and
+ * softmax, P rounded to bf16); float32 on CUDA cores (fp32 throughout, exact
+ * online softmax).
  */
 la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
-                                la_dtype dtype, int start, int batch, int heads, int kv_heads, int seq, int dim,
+                                la_dtype dtype, const int *start, int batch, int heads, int kv_heads, int seq, int dim,
                                 int cap, int rot, double rope_base, float scale, void *o, void *workspace,
                                 size_t workspace_bytes, void *stream);
 

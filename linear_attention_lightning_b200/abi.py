@@ -36,7 +36,7 @@ _SIGNATURES = {
     "lightning_gqa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, ctypes.c_double,
                               ctypes.c_float, _vp, _vp, _sz, _vp], _i),
     "lightning_gqa_decode_workspace_size": ([_i, _i, _i], _sz),
-    "lightning_gqa_prefill": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.c_double,
+    "lightning_gqa_prefill": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, ctypes.c_double,
                                ctypes.c_float, _vp, _vp, _sz, _vp], _i),
     "lightning_gqa_prefill_workspace_size": ([_i, _i, _i, _i, _i], _sz),
     "lightning_prefill_backward": ([_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,

@@ -249,13 +249,14 @@ def gqa_decode(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cach
 
 
 def gqa_prefill(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
-                v_cache: torch.Tensor, start: int = 0, rot: int = 64, rope_base: float = 10000.0,
+                v_cache: torch.Tensor, start=0, rot: int = 64, rope_base: float = 10000.0,
                 scale: Optional[float] = None, o: Optional[torch.Tensor] = None,
                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """lightning_gqa_prefill: the softmax GQA layer over seq new tokens at
-    positions start .. start+seq-1. Writes their rotated keys and values into
-    the caches and returns o [batch, heads, seq, dim]. bf16 (tensor cores) or
-    float32 (CUDA cores); scale defaults to 1/sqrt(dim)."""
+    """lightning_gqa_prefill: the softmax GQA layer over seq new tokens of each
+    sequence b at positions start[b] .. start[b]+seq-1. Writes their rotated keys
+    and values into the caches and returns o [batch, heads, seq, dim]. `start` is
+    an int (the same for every sequence) or a CUDA int32 tensor [batch]. bf16
+    (tensor cores) or float32 (CUDA cores); scale defaults to 1/sqrt(dim)."""
     if q.dtype not in _DTYPES:
         raise ValueError("q must be float32 or bfloat16")
     if q.dim() != 4 or k_cache.dim() != 4:
@@ -268,6 +269,10 @@ def gqa_prefill(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
                          "caches [b, kv_heads, cap, dim]")
     for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache), ("v_cache", v_cache)):
         _need_cuda(name, t, q.dtype)
+    if isinstance(start, torch.Tensor):
+        _need_cuda("start", start, torch.int32, (b,))
+    else:
+        start = torch.full((b,), int(start), dtype=torch.int32, device=q.device)
     if scale is None:
         scale = 1.0 / float(d) ** 0.5
     if o is None:
@@ -277,7 +282,7 @@ def gqa_prefill(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
     need = abi.lightning_gqa_prefill_workspace_size(_DTYPES[q.dtype], b, h, L, d)
     workspace = _workspace(max(need, 16), workspace, q.device)
     abi.check(abi.lightning_gqa_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
-                                        _DTYPES[q.dtype], int(start), b, h, hk, L, d, cap, int(rot),
+                                        _DTYPES[q.dtype], _ptr(start), b, h, hk, L, d, cap, int(rot),
                                         float(rope_base), float(scale), _ptr(o), _ptr(workspace),
                                         _nbytes(workspace), _stream(stream)))
     return o

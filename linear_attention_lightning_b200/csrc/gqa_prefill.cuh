@@ -4,9 +4,10 @@
 // §04: those layers keep a bf16 KV cache). Readings as for the decode step:
 // grouped-query attention (query head h reads KV head h / (heads/kv_heads)),
 // scores scaled by `scale`, rotate-half RoPE on the first `rot` dims, the
-// cache holds rotated keys. `seq` new tokens per sequence sit at positions
-// start .. start+seq-1; token i attends causally to positions 0 .. start+i:
-//   o_i = sum_{p <= start+i} softmax_p(scale * rope(q_i) . k_p) v_p.
+// cache holds rotated keys. `seq` new tokens of sequence b sit at positions
+// start[b] .. start[b]+seq-1 (each sequence with its own cached prefix); token i
+// attends causally to positions 0 .. start[b]+i:
+//   o_i = sum_{p <= start[b]+i} softmax_p(scale * rope(q_i) . k_p) v_p.
 //
 // Two kernels:
 //   gqp_rope_kernel     one CTA per (token, sequence): the token's angles once
@@ -35,9 +36,11 @@
 // CTAs go KV head by KV head (query head fastest, then the query rows from the longest
 // down), so the CTAs resident at a time read one KV head's keys and values, which L2 holds
 // (67 MB at 131072 positions); heavy-first within a KV head keeps the tail short.
-// Key tiles end at position start+seq-1: the key and value tensor maps stop
-// there, so TMA reads zeros past it and no cache row beyond the sequence is
-// ever read.
+// A query tile reads the key tiles up to its last row's position. Only the
+// last of them can reach past position start[b]+seq-1, into cache rows this
+// call neither wrote nor was given: their scores are masked, and their value
+// rows are zeroed in shared memory before P V (a masked weight is 0, but
+// 0 x NaN is NaN).
 //
 // Warp roles: warp 0 TMA, warp 1 MMA (the whole warp follows the waits, one elected lane
 // issues), warp 2 TMEM, warps 4-7 and 8-11 the softmax warpgroups of tiles 0 and 1; the
@@ -105,17 +108,23 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 
 // --------------------------------------------------------------------- RoPE
 
-// grid (seq, batch), 256 threads. q_rot[b][h][i] = rope(q[b][h][i], start+i);
-// k_cache[b][g][start+i] = rope(k_new[b][g][i], start+i); v_cache[..] = v_new.
+// grid (seq, batch), 256 threads. q_rot[b][h][i] = rope(q[b][h][i], start[b]+i);
+// k_cache[b][g][start[b]+i] = rope(k_new[b][g][i], start[b]+i); v_cache[..] = v_new.
+// A start[b] outside 0 .. cap-seq skips sequence b and is reported in the status word.
 // Elements travel in pairs (rot % 4 == 0 keeps a pair on one side of the
 // rotation); angles in double, rotation in fp32, results rounded to bf16.
 __global__ void __launch_bounds__(256)
 gqp_rope_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k_new,
                 const __nv_bfloat16 *__restrict__ v_new, __nv_bfloat16 *__restrict__ k_cache,
                 __nv_bfloat16 *__restrict__ v_cache, __nv_bfloat16 *__restrict__ q_rot, int heads, int kv_heads,
-                int seq, int start, int cap, int rot, double base) {
+                int seq, const int *__restrict__ start, int cap, int rot, double base) {
     __shared__ float cs[kDim / 2], sn[kDim / 2];
-    const int i = blockIdx.x, b = blockIdx.y, pos = start + i, half = rot / 2;
+    const int i = blockIdx.x, b = blockIdx.y, st = start[b], half = rot / 2;
+    if (st < 0 || st > cap - seq) {
+        if (i == 0 && threadIdx.x == 0) atomicOr(&g_device_status, kBadDeviceArgFlag);
+        return;
+    }
+    const int pos = st + i;
     for (int c = threadIdx.x; c < half; c += blockDim.x) {
         double s, co;
         sincos((double)pos * pow(base, -2.0 * c / (double)rot), &s, &co);
@@ -257,7 +266,8 @@ struct Work {
     int bh, bkv, i0, n[2];  // n[t]: key tiles that query tile t reads (0: tile absent)
 };
 
-__device__ __forceinline__ Work work_of(int heads, int kv_heads, int batch, int seq, int start) {
+__device__ __forceinline__ Work work_of(int heads, int kv_heads, int batch, int seq, const int *start,
+                                        int *start_b) {
     const int group = heads / kv_heads;
     const int npairs = (seq + kQRows - 1) / kQRows;
     const int x = blockIdx.x;
@@ -269,20 +279,25 @@ __device__ __forceinline__ Work work_of(int heads, int kv_heads, int batch, int 
     w.bh = b * heads + g * group + hq;
     w.bkv = bkv;
     w.i0 = kQRows * pi;
+    *start_b = start[b];
+    const int st = *start_b;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int r0 = w.i0 + kRows * t;
-        w.n[t] = r0 < seq ? (start + min(r0 + kRows - 1, seq - 1)) / kRows + 1 : 0;
+        w.n[t] = r0 < seq ? (st + min(r0 + kRows - 1, seq - 1)) / kRows + 1 : 0;
     }
     return w;
 }
 
-// tm_q: q_rot [batch*heads][seq][128]; tm_k, tm_v: caches [batch*kv_heads][start+seq][128]
-// (row stride cap); tm_o: o [batch*heads][seq][128]. All 128-byte swizzled boxes of 64 x 128.
+// tm_q: q_rot [batch*heads][seq][128]; tm_k, tm_v: caches [batch*kv_heads][cap][128];
+// tm_o: o [batch*heads][seq][128]. All 128-byte swizzled boxes of 64 x 128. Sequence b
+// reads cache rows 0 .. start[b]+seq-1 only: its last key tile may reach past them, and
+// those value rows are zeroed in shared memory before P V (their weights are 0, but the
+// rows may hold anything, and 0 x NaN is NaN); the scores of those keys are masked.
 __global__ void __launch_bounds__(kThreads, 1)
 gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, int batch,
-                int heads, int kv_heads, int seq, int start, float sl2) {
+                int heads, int kv_heads, int seq, const int *__restrict__ start, int cap, float sl2) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = ptx::smem_addr(smem_raw);
     const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
@@ -293,8 +308,11 @@ gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c.smem + kOffMisc);
     c.abort = reinterpret_cast<volatile int *>(c.smem + kOffMisc + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const Work w = work_of(heads, kv_heads, batch, seq, start);
+    int st = 0;  // this sequence's start
+    const Work w = work_of(heads, kv_heads, batch, seq, start, &st);
+    if (st < 0 || st > cap - seq) return;  // reported by the RoPE launch; nothing allocated yet
     const int nmax = max(w.n[0], w.n[1]);
+    const int kend = st + seq;  // cache rows 0 .. kend-1 hold this sequence's keys
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(&c.bars[i], 1);
@@ -397,6 +415,18 @@ gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (j > v_ready) {
                         if (!wait_bar(c, V_FULL + (j & 1), (uint32_t)(j >> 1) & 1u)) return false;
                         v_ready = j;
+                        const int live = kend - kRows * j;  // rows of this value tile inside the sequence
+                        if (live < kRows) {
+                            // the rows past the sequence: zeros, as the whole warp stores them
+                            uint8_t *vd = c.smem + kOffV + (j & 1) * kTileBytes;
+                            for (int u = lane; u < (kRows - live) * 16; u += 32) {
+                                const int row = live + (u >> 4), box = (u >> 3) & 1, ch = u & 7;
+                                *reinterpret_cast<uint4 *>(vd + box * kBoxBytes + row * 128 + ch * 16) =
+                                    make_uint4(0u, 0u, 0u, 0u);
+                            }
+                            ptx::fence_proxy_async_smem();
+                            __syncwarp();
+                        }
                     }
                     const uint64_t dv = dv0 + (uint64_t)(((j & 1) * kTileBytes) >> 4);
 #pragma unroll
@@ -444,7 +474,7 @@ gqp_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t trow = c.tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         const uint32_t cs_ = kColS + 128u * t, co_ = kColO + 128u * t;
         const int nt = w.n[t];
-        const int pmin = start + w.i0 + kRows * t;  // position of the tile's first row
+        const int pmin = st + w.i0 + kRows * t;     // position of the tile's first row
         const int qpos = pmin + r;
         float m = -INFINITY, l = 0.f;               // running max (log2 units) and sum
         bool done = nt > 0;
@@ -579,7 +609,7 @@ inline bool gqp_make_map(CUtensorMap *map, const void *base, long long rows, lon
 // q, o: [batch][heads][seq][128]; k_new, v_new: [batch][kv_heads][seq][128];
 // caches [batch][kv_heads][cap][128]; q_rot: workspace of q's size. bf16 throughout.
 inline la_status launch_gqa_prefill(const void *q, const void *k_new, const void *v_new, void *k_cache,
-                                    void *v_cache, int start, int batch, int heads, int kv_heads, int seq, int cap,
+                                    void *v_cache, const int *start, int batch, int heads, int kv_heads, int seq, int cap,
                                     int rot, double base, float scale, void *o, void *q_rot, cudaStream_t stream,
                                     std::string *err) {
     using bf = __nv_bfloat16;
@@ -594,8 +624,8 @@ inline la_status launch_gqa_prefill(const void *q, const void *k_new, const void
     }
     const long long bh = (long long)batch * heads, bkv = (long long)batch * kv_heads;
     CUtensorMap mq, mk, mv, mo;
-    if (!gqp_make_map(&mq, q_rot, seq, seq, bh, err) || !gqp_make_map(&mk, k_cache, (long long)start + seq, cap, bkv, err) ||
-        !gqp_make_map(&mv, v_cache, (long long)start + seq, cap, bkv, err) || !gqp_make_map(&mo, o, seq, seq, bh, err))
+    if (!gqp_make_map(&mq, q_rot, seq, seq, bh, err) || !gqp_make_map(&mk, k_cache, cap, cap, bkv, err) ||
+        !gqp_make_map(&mv, v_cache, cap, cap, bkv, err) || !gqp_make_map(&mo, o, seq, seq, bh, err))
         return LA_ERR_CUDA;
     e = cudaFuncSetAttribute(gqp::gqp_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gqp::kSmemBytes);
     if (e != cudaSuccess) {
@@ -611,7 +641,7 @@ inline la_status launch_gqa_prefill(const void *q, const void *k_new, const void
     }
     const long long ctas = bh * ((seq + gqp::kQRows - 1) / gqp::kQRows);
     gqp::gqp_attn_kernel<<<(unsigned)ctas, gqp::kThreads, gqp::kSmemBytes, stream>>>(
-        mq, mk, mv, mo, batch, heads, kv_heads, seq, start, scale * gqp::kLog2eF);
+        mq, mk, mv, mo, batch, heads, kv_heads, seq, start, cap, scale * gqp::kLog2eF);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
         *err = std::string("gqa prefill attention launch: ") + cudaGetErrorString(e);
@@ -634,14 +664,20 @@ constexpr int kDim = 128;
 constexpr int kKPitch = kDim + 1;  // padded key rows: the 8 threads of a row read 8 different banks
 constexpr uint32_t kSmemBytes = (kQRows * kDim + kKeys * kKPitch + kKeys * kDim + kQRows * kKeys) * 4;
 
-// grid (seq, batch), 256 threads: q_rot = rope(q), cache rows start+i <- rope(k_new), v_new.
-// float32 throughout; angles in double.
+// grid (seq, batch), 256 threads: q_rot = rope(q), cache rows start[b]+i <- rope(k_new), v_new.
+// float32 throughout; angles in double. A start[b] outside 0 .. cap-seq skips sequence b and is
+// reported in the status word.
 __global__ void __launch_bounds__(256)
 gqs_rope_kernel(const float *__restrict__ q, const float *__restrict__ k_new, const float *__restrict__ v_new,
                 float *__restrict__ k_cache, float *__restrict__ v_cache, float *__restrict__ q_rot, int heads,
-                int kv_heads, int seq, int start, int cap, int rot, double base) {
+                int kv_heads, int seq, const int *__restrict__ start, int cap, int rot, double base) {
     __shared__ float cs[kDim / 2], sn[kDim / 2];
-    const int i = blockIdx.x, b = blockIdx.y, pos = start + i, half = rot / 2;
+    const int i = blockIdx.x, b = blockIdx.y, st = start[b], half = rot / 2;
+    if (st < 0 || st > cap - seq) {
+        if (i == 0 && threadIdx.x == 0) atomicOr(&g_device_status, kBadDeviceArgFlag);
+        return;
+    }
+    const int pos = st + i;
     for (int c = threadIdx.x; c < half; c += blockDim.x) {
         double s, co;
         sincos((double)pos * pow(base, -2.0 * c / (double)rot), &s, &co);
@@ -680,18 +716,21 @@ gqs_rope_kernel(const float *__restrict__ q, const float *__restrict__ k_new, co
 // grid (ceil(seq / 16), heads, batch), 128 threads; dynamic shared memory kSmemBytes.
 // Thread t takes row r = t / 8 of the CTA's 16 query rows: scores for keys t%8, t%8 + 8, ...
 // of each 64-key tile, then output dims 16 (t%8) .. 16 (t%8) + 15. Exact online softmax in
-// fp32 (the running max is raised on every increase); keys past start+seq are never read.
+// fp32 (the running max is raised on every increase); keys past start[b]+seq are never read.
 __global__ void __launch_bounds__(kThreads)
 gqs_attn_kernel(const float *__restrict__ q_rot, const float *__restrict__ k_cache, const float *__restrict__ v_cache,
-                float *__restrict__ o, int heads, int kv_heads, int seq, int start, int cap, float scale) {
+                float *__restrict__ o, int heads, int kv_heads, int seq, const int *__restrict__ start, int cap,
+                float scale) {
     extern __shared__ float sm[];
     float *qs = sm, *ks = qs + kQRows * kDim, *vs = ks + kKeys * kKPitch, *ps = vs + kKeys * kDim;
     const int i0 = blockIdx.x * kQRows, h = blockIdx.y, b = blockIdx.z;
     const int group = heads / kv_heads;
     const size_t bh = (size_t)b * heads + h, kv = (size_t)b * kv_heads + h / group;
     const int t = threadIdx.x, r = t >> 3, j8 = t & 7;
-    const int qpos = start + i0 + r;                       // this row's position
-    const int kend = min(start + i0 + kQRows, start + seq);  // keys 0 .. kend-1 are needed
+    const int st = start[b];
+    if (st < 0 || st > cap - seq) return;  // reported by the RoPE launch
+    const int qpos = st + i0 + r;                    // this row's position
+    const int kend = min(st + i0 + kQRows, st + seq);  // keys 0 .. kend-1 are needed
     for (int e = t; e < kQRows * kDim; e += kThreads) {
         const int rr = e / kDim;
         qs[e] = i0 + rr < seq ? q_rot[(bh * seq + i0 + rr) * kDim + e % kDim] : 0.f;
@@ -755,7 +794,7 @@ gqs_attn_kernel(const float *__restrict__ q_rot, const float *__restrict__ k_cac
 }  // namespace gqs
 
 inline la_status launch_gqa_prefill_f32(const void *q, const void *k_new, const void *v_new, void *k_cache,
-                                        void *v_cache, int start, int batch, int heads, int kv_heads, int seq,
+                                        void *v_cache, const int *start, int batch, int heads, int kv_heads, int seq,
                                         int cap, int rot, double base, float scale, void *o, void *q_rot,
                                         cudaStream_t stream, std::string *err) {
     gqs::gqs_rope_kernel<<<dim3((unsigned)seq, (unsigned)batch), 256, 0, stream>>>(

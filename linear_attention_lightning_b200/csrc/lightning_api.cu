@@ -892,17 +892,16 @@ size_t lightning_gqa_prefill_workspace_size(la_dtype dtype, int batch, int heads
 }
 
 la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
-                                la_dtype dtype, int start, int batch, int heads, int kv_heads, int seq, int dim,
+                                la_dtype dtype, const int *start, int batch, int heads, int kv_heads, int seq, int dim,
                                 int cap, int rot, double rope_base, float scale, void *o, void *workspace,
                                 size_t workspace_bytes, void *stream) {
     if (dtype != LA_DTYPE_F32 && dtype != LA_DTYPE_BF16)
         return fail(LA_ERR_INVALID_ARG, "dtype %d is neither LA_DTYPE_F32 nor LA_DTYPE_BF16", (int)dtype);
-    if (batch < 0 || seq < 0 || start < 0 || heads < 1 || kv_heads < 1 || cap < 1 || heads % kv_heads != 0)
+    if (batch < 0 || seq < 0 || heads < 1 || kv_heads < 1 || cap < 1 || heads % kv_heads != 0)
         return fail(LA_ERR_INVALID_ARG,
-                    "need batch, seq, start >= 0, cap >= 1 and kv_heads dividing heads (got %d, %d, %d, %d, %d, %d)",
-                    batch, seq, start, cap, heads, kv_heads);
-    if ((long long)start + seq > cap) return fail(LA_ERR_INVALID_ARG, "start + seq (%lld) exceeds cap %d",
-                                                   (long long)start + seq, cap);
+                    "need batch, seq >= 0, cap >= 1 and kv_heads dividing heads (got %d, %d, %d, %d, %d)", batch, seq,
+                    cap, heads, kv_heads);
+    if (seq > cap) return fail(LA_ERR_INVALID_ARG, "seq %d exceeds cap %d", seq, cap);
     if (dim != la::gqp::kDim) return fail(LA_ERR_UNSUPPORTED, "dim %d unsupported (128)", dim);
     if (rot < 0 || rot > dim || (rot & 3)) return fail(LA_ERR_INVALID_ARG, "rot must be a multiple of 4, 0 <= rot <= dim");
     if (!(rope_base > 0.0) || rope_base > 1e300) return fail(LA_ERR_INVALID_ARG, "rope_base must be finite and > 0");
@@ -912,22 +911,23 @@ la_status lightning_gqa_prefill(const void *q, const void *k_new, const void *v_
     const long long ctas = (long long)batch * heads * ((seq + la::gqp::kQRows - 1) / la::gqp::kQRows);
     if (ctas > 0x7fffffffLL) return fail(LA_ERR_UNSUPPORTED, "problem too large for one launch");
     const size_t need = lightning_gqa_prefill_workspace_size(dtype, batch, heads, seq, dim);
-    if (!q || !k_new || !v_new || !k_cache || !v_cache || !o)
-        return fail(LA_ERR_INVALID_ARG, "q, k_new, v_new, the caches and o must be non-NULL");
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !o || !start)
+        return fail(LA_ERR_INVALID_ARG, "q, k_new, v_new, the caches, start and o must be non-NULL");
     if (!workspace || workspace_bytes < need)
         return fail(LA_ERR_INVALID_ARG, "workspace needs %zu bytes (got %zu)", need, workspace ? workspace_bytes : (size_t)0);
-    const void *ptrs[] = {q, k_new, v_new, k_cache, v_cache, o, workspace};
-    const char *names[] = {"q", "k_new", "v_new", "k_cache", "v_cache", "o", "workspace"};
-    for (int i = 0; i < 7; ++i)
+    const void *ptrs[] = {q, k_new, v_new, k_cache, v_cache, o, workspace, start};
+    const char *names[] = {"q", "k_new", "v_new", "k_cache", "v_cache", "o", "workspace", "start"};
+    for (int i = 0; i < 8; ++i)
         if (!aligned16(ptrs[i])) return fail(LA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
     const size_t eb = elem_bytes(dtype);
     const size_t nq = (size_t)batch * heads * seq * dim * eb, nkv = (size_t)batch * kv_heads * seq * dim * eb;
     const size_t ncache = (size_t)batch * kv_heads * cap * dim * eb;
     const Range all[] = {range_of(q, nq), range_of(k_new, nkv), range_of(v_new, nkv), range_of(k_cache, ncache),
-                         range_of(v_cache, ncache), range_of(o, nq), range_of(workspace, need)};
+                         range_of(v_cache, ncache), range_of(o, nq), range_of(workspace, need),
+                         range_of(start, sizeof(int) * batch)};
     const int written[] = {3, 4, 5, 6};  // the caches, o and the workspace
     for (int wi : written)
-        for (int j = 0; j < 7; ++j)
+        for (int j = 0; j < 8; ++j)
             if (j != wi && overlaps(all[wi], all[j]))
                 return fail(LA_ERR_INVALID_ARG, "%s overlaps %s", names[wi], names[j]);
     if (const la_status early = earlier_failure()) return early;

@@ -335,9 +335,12 @@ def test_gqa_workspace_size_and_empty_batch():
     assert _gqa(batch=0) == abi.LA_OK
 
 
+ST = 0x10000000 * 50  # fake device start[batch] array
+
+
 def _gqp(**kw):
     # sizes: q, o 2 x 64 x 512 x 128 bf16 = 16 MiB; caches 2 x 8 x 1024 x 128 bf16 = 4 MiB (fake addresses 256 MiB apart)
-    a = dict(q=Q, kn=K, vn=V, kc=0x10000000 * 30, vc=0x10000000 * 40, dtype=abi.LA_DTYPE_BF16, start=100, batch=2,
+    a = dict(q=Q, kn=K, vn=V, kc=0x10000000 * 30, vc=0x10000000 * 40, dtype=abi.LA_DTYPE_BF16, start=ST, batch=2,
              heads=64, kv=8, seq=512, dim=128, cap=1024, rot=64, base=1e4, scale=0.088, o=O, ws=WS, ws_bytes=1 << 26)
     a.update(kw)
     return abi.lightning_gqa_prefill(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["dtype"], a["start"], a["batch"],
@@ -348,16 +351,18 @@ def _gqp(**kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(dtype=9), abi.LA_ERR_INVALID_ARG),
     (dict(kv=7), abi.LA_ERR_INVALID_ARG),                     # does not divide 64
-    (dict(start=-1), abi.LA_ERR_INVALID_ARG),
+    (dict(start=None), abi.LA_ERR_INVALID_ARG),               # the device start array is required
+    (dict(start=ST + 4), abi.LA_ERR_INVALID_ARG),             # not 16-byte aligned
+    (dict(o=ST), abi.LA_ERR_INVALID_ARG),                     # o overlaps start
     (dict(seq=-3), abi.LA_ERR_INVALID_ARG),
-    (dict(start=600), abi.LA_ERR_INVALID_ARG),                # start + seq > cap
+    (dict(seq=1025), abi.LA_ERR_INVALID_ARG),                 # seq > cap
     (dict(dim=64), abi.LA_ERR_UNSUPPORTED),
     (dict(rot=62), abi.LA_ERR_INVALID_ARG),                   # not a multiple of 4
     (dict(rot=132), abi.LA_ERR_INVALID_ARG),
     (dict(base=-1.0), abi.LA_ERR_INVALID_ARG),
     (dict(scale=0.0), abi.LA_ERR_INVALID_ARG),
     (dict(scale=float("nan")), abi.LA_ERR_INVALID_ARG),
-    (dict(batch=70000, start=0, seq=1, cap=2), abi.LA_ERR_UNSUPPORTED),
+    (dict(batch=70000, seq=1, cap=2), abi.LA_ERR_UNSUPPORTED),
     (dict(kn=None), abi.LA_ERR_INVALID_ARG),
     (dict(q=Q + 8), abi.LA_ERR_INVALID_ARG),                  # not 16-byte aligned
     (dict(ws_bytes=1 << 20), abi.LA_ERR_INVALID_ARG),         # workspace too small

@@ -207,3 +207,68 @@ def test_gqa_prefill_float32_matches_the_oracle(case):
 
 def test_gqa_prefill_float32_never_reads_cache_rows_past_the_sequence():
     _run(1, 8, 2, 100, 20, 400, 64, seed=191, poison_tail=True, dtype=torch.float32)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gqa_prefill_sequences_with_unequal_prefixes(dtype):
+    # each sequence continues its own cached prefix (start[b] on the device): the pages'
+    # KV cache grows per sequence ("MINIMAX SIGNAL LAB · M1", §04). Cache rows past each
+    # sequence's end hold NaN: the last key tile a query reads may reach them, and they
+    # must enter no result.
+    b, h, hk, L, cap, rot, base = 4, 16, 4, 300, 1500, 64, 10000.0
+    starts = [0, 37, 1000, 1200]
+    q, kn, vn, kc, vc = _inputs(b, h, hk, L, cap, 301, dtype=dtype)
+    for bb, st in enumerate(starts):
+        kc[bb, :, st + L:] = float("nan")
+        vc[bb, :, st + L:] = float("nan")
+    kc0, vc0 = kc.clone(), vc.clone()
+    sc = 1.0 / np.sqrt(128.0)
+    buf, o = _guarded_o(q.shape, dtype)
+    la.gqa_prefill(q, kn, vn, kc, vc, start=torch.tensor(starts, dtype=torch.int32, device=DEV), rot=rot,
+                   rope_base=base, scale=sc, o=o)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:GUARD] == SENTINEL) and torch.all(buf[-GUARD:] == SENTINEL), "o guard band written"
+    conv = inputs.to_oracle
+    iv = torch.int16 if dtype == torch.bfloat16 else torch.int32
+    for bb, st in enumerate(starts):
+        sl = slice(bb, bb + 1)
+        ref = oracle.gqa_prefill(conv(q[sl]), conv(kn[sl]), conv(vn[sl]), conv(kc0[sl]), conv(vc0[sl]), st, rot,
+                                 base, sc)
+        got = to_f64(o[sl])
+        assert np.all(np.isfinite(got)), "sequence %d" % bb
+        v_rms = float(torch.sqrt(torch.mean(torch.cat([vn[sl].float().flatten(),
+                                                       vc0[sl, :, :st].float().flatten()]) ** 2)))
+        e = check(got.reshape(-1, 128), ref.reshape(-1, 128), v_rms, dtype)
+        print("gqa_prefill %s, sequence %d at start %d: max error %.3g rms(v)" % (str(dtype)[6:], bb, st, e))
+        # this sequence's new rows are written; every other row keeps its contents (NaN included)
+        assert torch.equal(vc[bb, :, st:st + L], vn[bb])
+        keep = torch.ones(cap, dtype=torch.bool, device=DEV)
+        keep[st:st + L] = False
+        assert torch.equal(kc[bb][:, keep].view(iv), kc0[bb][:, keep].view(iv))
+        assert torch.equal(vc[bb][:, keep].view(iv), vc0[bb][:, keep].view(iv))
+    assert abi.lightning_last_device_status(torch.cuda.current_stream().cuda_stream) == abi.LA_OK
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gqa_prefill_skips_and_reports_a_start_outside_the_cache(dtype):
+    b, h, hk, L, cap = 3, 8, 2, 200, 600
+    starts = [5, 450, 100]            # 450 + 200 > 600: sequence 1 does not fit
+    q, kn, vn, kc, vc = _inputs(b, h, hk, L, cap, 302, dtype=dtype)
+    kc0, vc0 = kc.clone(), vc.clone()
+    o = torch.full_like(q, SENTINEL)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert abi.lightning_last_device_status(stream) == abi.LA_OK
+    la.gqa_prefill(q, kn, vn, kc, vc, start=torch.tensor(starts, dtype=torch.int32, device=DEV), rot=64, o=o)
+    assert abi.lightning_last_device_status(stream) == abi.LA_ERR_INVALID_ARG
+    iv = torch.int16 if dtype == torch.bfloat16 else torch.int32
+    assert torch.equal(kc[1].view(iv), kc0[1].view(iv)) and torch.equal(vc[1].view(iv), vc0[1].view(iv))
+    assert torch.all(o[1] == SENTINEL)       # nothing written for the sequence that does not fit
+    conv = inputs.to_oracle
+    for bb in (0, 2):
+        sl = slice(bb, bb + 1)
+        ref = oracle.gqa_prefill(conv(q[sl]), conv(kn[sl]), conv(vn[sl]), conv(kc0[sl]), conv(vc0[sl]), starts[bb],
+                                 64, 10000.0, 1.0 / np.sqrt(128.0))
+        v_rms = float(torch.sqrt(torch.mean(torch.cat([vn[sl].float().flatten(),
+                                                       vc0[sl, :, :starts[bb]].float().flatten()]) ** 2)))
+        check(to_f64(o[sl]).reshape(-1, 128), ref.reshape(-1, 128), v_rms, dtype)
+    assert abi.lightning_last_device_status(stream) == abi.LA_OK
