@@ -69,7 +69,7 @@ def workload_config(w, world):
     """The contract line's config, the same for both arms: the workload by name
     and sizes, how the run is spread over GPUs, and how L2 is kept out of the
     timing (every step streams more than L2 holds)."""
-    by = prefill_bytes(w.batch, w.heads, w.seq, w.dim, 2 if "bf16" in str(w.dtype) else 4,
+    by = prefill_bytes(w.batch, w.heads, w.seq, w.dim, 2 if str(w.dtype) == "torch.bfloat16" else 4,
                        state_in=w.state_in, state_out=True)
     return {"workload": w.name, "batch": w.batch, "heads": w.heads, "seq_len": w.seq, "dim": w.dim,
             "block": w.block, "parallelism": "replicas" if world > 1 else "single GPU",
@@ -475,9 +475,9 @@ def run_ours(args):
     vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05,
              "pair": abi.LA_VARIANT_TCGEN05_PAIR}[variant]
     dcode = abi.LA_DTYPE_BF16 if w.dtype == torch.bfloat16 else abi.LA_DTYPE_F32
-    # kernels one lightning_prefill_ex call launches: the CTA-pair kernel, then its
+    # kernels one lightning_prefill_ex call launches: a tensor-core kernel, then its
     # range guard's second pass (which returns at once for heads it need not redo)
-    launches_per_step = 2 if variant == "pair" else 1
+    launches_per_step = 2 if variant in ("pair", "tcgen05") else 1
     need = abi.lightning_prefill_workspace_size(w.batch, w.heads, w.seq, w.dim, w.block)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 

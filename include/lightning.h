@@ -101,8 +101,8 @@ int lightning_abi_version(void);
  *   workspace, workspace_bytes
  *              device scratch, caller-owned, 16-byte aligned, overlapping no
  *              other buffer, of at least lightning_prefill_workspace_size
- *              bytes: 48 bytes per (batch, head) for the CTA-pair tensor-core
- *              kernel (its range guard, below), none for the other kernels
+ *              bytes: 48 bytes per (batch, head) for either tensor-core
+ *              kernel (its range guard, below), none for the CUDA-core kernel
  *              (NULL/0 is fine there). Too little returns LA_ERR_INVALID_ARG.
  *              Its contents need no initialisation; calls that share one
  *              workspace must not run at the same time.
@@ -111,8 +111,8 @@ int lightning_abi_version(void);
  *
  * Input range of the tensor-core kernels. They round the operands they form
  * (P ⊙ D, Q ⊙ d_q, K ⊙ d_k, V and the carried state) to fp16, whose range is
- * narrower than bf16's. The CTA-pair kernel guards against that: while it
- * runs it takes, per (batch, head), the largest |q|, |k|, |v| and |state_in|
+ * narrower than bf16's. Both tensor-core kernels guard against that: while
+ * they run they take, per (batch, head), the largest |q|, |k|, |v| and |state_in|
  * element, which bound every such operand; a head whose operands could pass
  * 2^15, or whose maxima fall below 2^-9, is recomputed by a second launch with
  * q, k and v scaled by powers of two (exact) chosen from the head's largest
@@ -122,11 +122,10 @@ int lightning_abi_version(void);
  * 2^-36 .. 2^44, provided the values inside one (batch, head) span less than
  * about 2^14 (for example a few rows 2^8 above the rest, with |q.k| above
  * 65504, are covered). Inputs holding inf or NaN give non-finite results.
- * The single-CTA kernel (LA_VARIANT_TCGEN05) has no guard: its operands must
- * stay inside fp16's range (|q.k|, |q|, |k|, |v| and the state below 65504)
- * and its inputs' elements near or above 2^-9 in magnitude for the bound to
- * hold (scales 2^-10 .. 2^8 of the workloads' inputs, one tensor at a time,
- * are tested).
+ * Every call of a tensor-core kernel is two launches on `stream`: the kernel,
+ * then the guard's second pass, which returns at once for heads it need not
+ * redo. With state_out == state_in, the single-CTA kernel runs each head's
+ * two CTAs as a thread-block cluster of two.
  */
 la_status lightning_prefill(const void *q, const void *k, const void *v, la_dtype dtype,
                             const float *slopes, int batch, int heads, int seq, int dim,

@@ -98,7 +98,9 @@ struct PrefillArgs {
 // Workspace a prefill request needs: the range guard's records for the CTA-pair
 // kernel, none for the others.
 size_t prefill_workspace_bytes(int batch, int heads, int variant) {
-    return variant == LA_VARIANT_TCGEN05_PAIR ? la::pair_workspace_bytes((long long)batch * heads) : 0;
+    if (variant == LA_VARIANT_TCGEN05_PAIR) return la::pair_workspace_bytes((long long)batch * heads);
+    if (variant == LA_VARIANT_TCGEN05) return la::tc_workspace_bytes((long long)batch * heads);
+    return 0;
 }
 
 // A workspace of at least `need` bytes, 16-byte aligned, overlapping none of `others`.
@@ -616,7 +618,8 @@ la_status run_prefill(const PrefillArgs &a, cudaStream_t stream, int variant) {
                                &g_last_error);
     if (variant == LA_VARIANT_TCGEN05) return la::launch_tc(a.q, a.k, a.v, a.slopes, a.batch, a.heads,
                                                            a.seq, a.block, a.state_in, a.o, a.state_out,
-                                                           a.sn, stream, &g_last_error);
+                                                           a.sn, static_cast<la::rg::RangeRec *>(a.workspace),
+                                                           stream, &g_last_error);
     if (a.dtype == LA_DTYPE_BF16)
         return a.dim == 64 ? launch_simt<__nv_bfloat16, 64>(a, stream)
                            : launch_simt<__nv_bfloat16, 128>(a, stream);

@@ -122,20 +122,9 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// shared::cluster address of the same shared-memory location in CTA `rank`
-__device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
-    uint32_t out;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(ptx::smem_addr(p)), "r"(rank));
-    return out;
-}
+using ptx::cluster_rank;
+using ptx::cluster_sync;
+using ptx::map_to_rank;
 // Arrive on the even CTA's copy of barrier `bar`. Every hand-off to the MMA
 // thread concerns data in the arriving CTA's own shared memory or TMEM, made
 // visible to the tensor core by the async-proxy or tcgen05 fence that precedes
@@ -172,26 +161,8 @@ __device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parit
     const bool ok = leader ? wait_bar(c, idx, parity) : true;
     return ptx::named_bar_and(bar_id, 128, ok);
 }
-// two fp32 sums in one instruction (each rounded as a plain add)
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-// two fp32 products in one instruction (each rounded as a plain multiply)
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
+using ptx::add2;
+using ptx::mul2;
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
     const float2 r = mul2(make_float2(ptx::bf16_lo(w), ptx::bf16_hi(w)), make_float2(scale, scale));

@@ -43,6 +43,15 @@
 // TMEM (512 columns x 128 lanes of 32 bit):
 //   [0,128) P_aa | Qd_a   [128,256) P_ba | Qd_b   [256,384) P_bb | dS
 //   [384,448) O_a   [448,512) O_b
+//
+// Range guard (range_guard.cuh). The plain kernel is pass 1: its conversion
+// warps also take the largest |q|, |k| (both CTAs of a head convert all of Q and
+// K) and warpgroup 3 the largest |v| element (this CTA's value half) and
+// |state_in| element of its half; at its end warpgroup 3 writes them as this
+// CTA's part of the head's record. Pass 2, launched as its programmatic dependent, decides
+// per head and recomputes the flagged heads with power-of-two operand scales.
+// With the state carried in place the two CTAs of a head run as a cluster of
+// two, exchange their parts, and pass 1 withholds a flagged head's final state.
 #pragma once
 
 #include <cuda.h>
@@ -52,6 +61,7 @@
 
 #include "../../include/lightning.h"
 #include "common.cuh"
+#include "range_guard.cuh"
 #include "tc_ptx.cuh"
 
 namespace la {
@@ -69,9 +79,10 @@ constexpr uint32_t kOffQK = 0;
 constexpr uint32_t kOffV = kOffQK + kQKSlots * kQKSlotBytes;
 constexpr uint32_t kOffS = kOffV + kVSlots * kVSlotBytes;
 constexpr uint32_t kOffBar = kOffS + kBoxBytes;
-constexpr int kNumBars = 36;
+constexpr int kNumBars = 38;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;   // + slack to align the base to 1024
+static_assert(kSmemBytes <= 232448, "fits the 227 KB of opt-in shared memory");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColP0 = 0, kColP1 = 128, kColP2 = 256;
@@ -82,7 +93,15 @@ __device__ __forceinline__ uint32_t p_col(int tile) { return tile == 0 ? kColP0 
 // barrier indices
 constexpr int FULL_QK = 0, EMPTY_QK = 5, FULL_V = 10, EMPTY_V = 13, P_FULL = 16, P_CONV = 19,
               P_FREE = 22, O_FULL = 25, O_FREE = 27, V_CONV = 29, KD_READY = 31, DS_FULL = 32,
-              DS_FREE = 33, S_READY = 34, DRAIN = 35;
+              DS_FREE = 33, S_READY = 34, DRAIN = 35,
+              // range guard (pass 1 only): SCAN_FIN: the two conversion warpgroups put
+              // their maxima in shared memory; PEER: the other CTA's part landed here
+              // (state carried in place)
+              SCAN_FIN = 36, PEER = 37;
+// shared-memory words after the barriers
+constexpr uint32_t kMiscTmem = 0, kMiscAbort = 4, kMiscMq = 8, kMiscMk = 12, kMiscMv = 16, kMiscSin = 20,
+                   kMiscPeer = 24 /* 4 floats */, kMiscFlag = 40;
+static_assert(kMiscFlag + 4 <= 64, "misc words fit their 64 bytes");
 
 // named barriers: 1 / 3 = the two conversion warpgroups, 2 = warpgroup 3
 constexpr int kBarConv = 1, kBarWG3 = 2, kBarConv2 = 3;
@@ -150,35 +169,77 @@ __device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parit
 
 // bf16x2 word -> f16x2 word of the values times `scale`
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
-    return ptx::pack_f16(ptx::bf16_lo(w) * scale, ptx::bf16_hi(w) * scale);
+    const float2 r = ptx::mul2(make_float2(ptx::bf16_lo(w), ptx::bf16_hi(w)), make_float2(scale, scale));
+    return ptx::pack_f16(r.x, r.y);
 }
 
-template <int NSUB>
+// kScaled = false: the plain kernel (pass 1 of the range guard), which also
+// measures every (batch, head) into rec[bh].part[half].
+// kScaled = true: pass 2, which returns at once for a head whose parts pass the
+// guard and otherwise recomputes it with power-of-two operand scales.
+template <int NSUB, bool kScaled>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ slopes, int heads,
-                  int seq, const float *state_in, __nv_bfloat16 *o, float *state_out, Snapshots sn) {
+                  int seq, const float *state_in, __nv_bfloat16 *o, float *state_out, Snapshots sn,
+                  rg::RangeRec *rec, const __nv_bfloat16 *qg, const __nv_bfloat16 *kg) {
     constexpr int B = kRows * NSUB;
     constexpr int kLastTile = 2 * NSUB - 2;  // index of the block's last P tile
     extern __shared__ uint8_t smem_raw[];
+    // pass 1: pass 2 may be scheduled now (it waits for this grid's completion before
+    // reading anything), so that its launch overlaps this one
+    if (!kScaled && threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;");
     const uint32_t raw_addr = ptx::smem_addr(smem_raw);
     const uint32_t pad = ((raw_addr + 1023u) & ~1023u) - raw_addr;
     Ctx c;
     c.smem = smem_raw + pad;
     c.sbase = raw_addr + pad;
     c.bars = reinterpret_cast<uint64_t *>(c.smem + kOffBar);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c.smem + kOffMisc);
-    c.abort = reinterpret_cast<volatile int *>(c.smem + kOffMisc + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(c.smem + kOffMisc + kMiscTmem);
+    c.abort = reinterpret_cast<volatile int *>(c.smem + kOffMisc + kMiscAbort);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(c.smem + kOffMisc);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x >> 1, half = blockIdx.x & 1;
     const float s = slopes[bh % heads];
     const float sl2 = s * kLog2e;  // e^{-s n} = 2^{-sl2 n}
+    // state carried in place: pass 1 runs the head's two CTAs as a cluster of two
+    // (rank = half) and they exchange their parts of the record
+    const bool in_place = state_out != nullptr && state_out == state_in;
+    // operand scales: q, k, v, P = q k, the carried state, its inverse, and o's inverse
+    float f_q = 1.f, f_k = 1.f, f_v = 1.f, f_p = 1.f, f_s = 1.f, f_su = 1.f, f_o = 1.f;
+    if constexpr (kScaled) {
+        // wait until pass 1 has completed and its records are visible
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        const rg::RangePart r = rg::combine(rec[bh].part[0], rec[bh].part[1]);
+        const bool flag = !rg::plain_ok(r, s, seq);
+        if (threadIdx.x == 0 && half == 0) rec[bh].flag = flag ? 1 : 0;
+        if (!flag) return;  // the whole CTA leaves before any set-up
+        // the head's largest row norms of q and k (fp32 sums over every row; the
+        // state operand's tile, first written after the set-up, holds the reduction)
+        float *red = reinterpret_cast<float *>(c.smem + kOffS);
+        const size_t hb = (size_t)bh * seq * kDim;
+        const float nq = sqrtf(rg::head_max_row_sumsq(qg + hb, seq, 0, 1, red));
+        const float nk = sqrtf(rg::head_max_row_sumsq(kg + hb, seq, 0, 1, red));
+        const rg::Exps e = rg::scale_exponents(nq, nk, r.mv, r.msin, s, seq);
+        f_q = rg::pow2(e.a);
+        f_k = rg::pow2(e.b);
+        f_v = rg::pow2(e.c);
+        f_p = rg::pow2(e.a + e.b);
+        f_s = rg::pow2(e.b + e.c);
+        f_su = rg::pow2(-(e.b + e.c));
+        f_o = rg::pow2(-(e.a + e.b + e.c));
+    }
     const int nblk = (seq + B - 1) / B;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNumBars; ++i) ptx::mbar_init(&c.bars[i], 1);
+        ptx::mbar_init(&c.bars[SCAN_FIN], 2);  // both conversion warpgroups
         *c.abort = 0;
+        misc[kMiscMq / 4] = 0u;
+        misc[kMiscMk / 4] = 0u;
+        misc[kMiscMv / 4] = 0u;
+        misc[kMiscSin / 4] = 0u;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -192,6 +253,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     ptx::tc_fence_before();
     __syncthreads();
+    // the other CTA's barriers are initialised before either CTA writes into them
+    if (!kScaled && in_place) ptx::cluster_sync();
     ptx::tc_fence_after();
     c.tmem = *tmem_slot;
 
@@ -376,7 +439,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const float step = ptx::ex2(-sl2);  // e^{-s}
         float tab[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) tab[u] = ptx::ex2(-sl2 * (float)(15 - u));
+        for (int u = 0; u < 16; ++u) tab[u] = ptx::ex2(-sl2 * (float)(15 - u)) * f_p;
+        uint32_t mxq = 0u, mxk = 0u;  // pass 1: packed maxima of |q| and |k| this thread converted
         uint32_t qk_par = 0;
         SlotMap<NSUB> sm;
         sm.init();
@@ -409,7 +473,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             if (dlast >= 0) {
                                 const float wb = ptx::ex2(-sl2 * (float)dlast);
 #pragma unroll
-                                for (int u = 0; u < 16; ++u) p[u] = (__uint_as_float(v[u]) * tab[u]) * wb;
+                                for (int u = 0; u < 16; u += 2) {
+                                    const float2 t2 = ptx::mul2(make_float2(__uint_as_float(v[u]), __uint_as_float(v[u + 1])),
+                                                                make_float2(tab[u], tab[u + 1]));
+                                    const float2 r2 = ptx::mul2(t2, make_float2(wb, wb));
+                                    p[u] = r2.x;
+                                    p[u + 1] = r2.y;
+                                }
                             } else if (i < jb) {
                                 // every key of the group is after row i: masked
 #pragma unroll
@@ -417,7 +487,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             } else {
                                 // the group holds the diagonal key jb + d0: walk down from it
                                 const int d0 = i - jb;
-                                float w = 1.f;
+                                float w = f_p;
 #pragma unroll
                                 for (int u = 15; u >= 0; --u) {
                                     const bool live = u <= d0;
@@ -437,7 +507,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const int qslot = tile == 0 ? sm.q0 : sm.q1;
                     if (!group_wait(c, FULL_QK + qslot, (qk_par >> qslot) & 1u, leader, bar_id, 128))
                         goto conv_done;
-                    const float dq = ptx::ex2(-sl2 * (float)(i + 1));
+                    const float dq = ptx::ex2(-sl2 * (float)(i + 1)) * f_q;
                     const uint8_t *qrow = c.smem + kOffQK + qslot * kQKSlotBytes + r * 128;
 #pragma unroll
                     for (int hb = 0; hb < 4; ++hb) {
@@ -447,6 +517,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             const int chunk = 4 * (hb & 1) + cc;
                             const uint4 q4 = *reinterpret_cast<const uint4 *>(
                                 qrow + (hb >> 1) * kBoxBytes + ((chunk ^ (r & 7)) << 4));
+                            if (!kScaled)
+                                mxq = rg::maxabs_bf16x2(mxq, rg::maxabs_bf16x2(rg::maxabs_bf16x2(q4.x, q4.y),
+                                                                               rg::maxabs_bf16x2(q4.z, q4.w)));
                             out[4 * cc + 0] = bf16x2_to_f16x2(q4.x, dq);
                             out[4 * cc + 1] = bf16x2_to_f16x2(q4.y, dq);
                             out[4 * cc + 2] = bf16x2_to_f16x2(q4.z, dq);
@@ -477,12 +550,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     // full-barrier wait: makes the TMA bytes visible to these threads
                     if (!group_wait(c, FULL_QK + kslot, (qk_par >> kslot) & 1u, leader, bar_id, 128)) goto conv_done;
                     const int j = sub * kRows + r;
-                    const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) : 0.f;
+                    const float dk = j < m ? ptx::ex2(-sl2 * (float)(m - 1 - j)) * f_k : 0.f;
                     uint8_t *krow = c.smem + kOffQK + kslot * kQKSlotBytes + r * 128;
                     uint4 x[16];
 #pragma unroll
                     for (int ch = 0; ch < 16; ++ch)
                         x[ch] = *reinterpret_cast<const uint4 *>(krow + (ch >> 3) * kBoxBytes + (((ch & 7) ^ (r & 7)) << 4));
+                    if (!kScaled) {
+#pragma unroll
+                        for (int ch = 0; ch < 16; ++ch)
+                            mxk = rg::maxabs_bf16x2(mxk, rg::maxabs_bf16x2(rg::maxabs_bf16x2(x[ch].x, x[ch].y),
+                                                                           rg::maxabs_bf16x2(x[ch].z, x[ch].w)));
+                    }
 #pragma unroll
                     for (int ch = 0; ch < 16; ++ch) {
                         uint4 y;
@@ -498,7 +577,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             qk_par ^= sm.used_mask();
             sm.advance();
         }
-    conv_done:;
+    conv_done:
+        if (!kScaled) {
+            // the group's maxima into shared memory for the record (rows past seq read
+            // as zeros and change no maximum)
+            const auto as_float = [](uint32_t w) { return fmaxf(fabsf(rg::bf_lo(w)), fabsf(rg::bf_hi(w))); };
+            const float mq = rg::warp_max_nonneg(as_float(mxq)), mk = rg::warp_max_nonneg(as_float(mxk));
+            if (lane == 0) {
+                atomicMax(misc + kMiscMq / 4, __float_as_uint(mq));
+                atomicMax(misc + kMiscMk / 4, __float_as_uint(mk));
+            }
+            ptx::named_bar_sync(bar_id, 128);
+            if (leader) ptx::mbar_arrive(&c.bars[SCAN_FIN]);
+        }
     } else if (warp >= 12) {
         // ------------------------------------------------------------ warpgroup 3
         const int r = threadIdx.x - 384;  // row of V / K sub-tiles, key-dim row of S, output row
@@ -506,11 +597,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
         float S[64];
         const size_t sbase = (size_t)bh * kDim * kDim + (size_t)r * kDim + 64 * half;
+        float msin = 0.f;     // pass 1: the largest |state_in| element of this thread
+        uint32_t mxv = 0u;    // pass 1: packed maximum of |v| this thread converted
         if (state_in) {
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
                 const float4 x = *reinterpret_cast<const float4 *>(state_in + sbase + 4 * q);
-                S[4 * q] = x.x; S[4 * q + 1] = x.y; S[4 * q + 2] = x.z; S[4 * q + 3] = x.w;
+                if (!kScaled) msin = fmaxf(msin, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
+                S[4 * q] = x.x * f_s; S[4 * q + 1] = x.y * f_s; S[4 * q + 2] = x.z * f_s; S[4 * q + 3] = x.w * f_s;
             }
         } else {
 #pragma unroll
@@ -551,8 +645,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     // then hit 8 different bank groups instead of one
                     uint4 *pv = reinterpret_cast<uint4 *>(vrow + ((ch ^ (r & 7)) << 4));
                     uint4 x = *pv;
-                    x.x = bf16x2_to_f16x2(x.x, 1.f); x.y = bf16x2_to_f16x2(x.y, 1.f);
-                    x.z = bf16x2_to_f16x2(x.z, 1.f); x.w = bf16x2_to_f16x2(x.w, 1.f);
+                    if (!kScaled)
+                        mxv = rg::maxabs_bf16x2(mxv, rg::maxabs_bf16x2(rg::maxabs_bf16x2(x.x, x.y),
+                                                                       rg::maxabs_bf16x2(x.z, x.w)));
+                    x.x = bf16x2_to_f16x2(x.x, f_v); x.y = bf16x2_to_f16x2(x.y, f_v);
+                    x.z = bf16x2_to_f16x2(x.z, f_v); x.w = bf16x2_to_f16x2(x.w, f_v);
                     *pv = x;
                 }
                 ptx::fence_proxy_async_smem();
@@ -582,7 +679,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                 for (int q = 0; q < 16; ++q)
                     *reinterpret_cast<float4 *>(snap + (size_t)r * kDim + 64 * half + 4 * q) =
-                        make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+                        make_float4(S[4 * q] * f_su, S[4 * q + 1] * f_su, S[4 * q + 2] * f_su, S[4 * q + 3] * f_su);
             }
 
             // outputs of this block: O (TMEM, fp32) -> bf16 -> global, 32 columns at a time
@@ -606,10 +703,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
                             dst[4 * hh + q] = make_uint4(
-                                ptx::pack_bf16(__uint_as_float(a[8 * q + 0]), __uint_as_float(a[8 * q + 1])),
-                                ptx::pack_bf16(__uint_as_float(a[8 * q + 2]), __uint_as_float(a[8 * q + 3])),
-                                ptx::pack_bf16(__uint_as_float(a[8 * q + 4]), __uint_as_float(a[8 * q + 5])),
-                                ptx::pack_bf16(__uint_as_float(a[8 * q + 6]), __uint_as_float(a[8 * q + 7])));
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 0]) * f_o, __uint_as_float(a[8 * q + 1]) * f_o),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 2]) * f_o, __uint_as_float(a[8 * q + 3]) * f_o),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 4]) * f_o, __uint_as_float(a[8 * q + 5]) * f_o),
+                                ptx::pack_bf16(__uint_as_float(a[8 * q + 6]) * f_o, __uint_as_float(a[8 * q + 7]) * f_o));
                     }
                 }
             }
@@ -617,17 +714,69 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             sm.advance();
             vtile += NSUB;
         }
-        if (state_out) {
+        {
+            bool write_state = state_out != nullptr;
+            if (!kScaled) {
+                // range guard, pass 1: this warpgroup's maxima join the conversion
+                // warpgroups' in shared memory, and the leader writes the CTA's part of
+                // the head's record once those have arrived (they finished converting
+                // before this block's outputs were ready, so the wait is short)
+                const float mv = rg::warp_max_nonneg(fmaxf(fabsf(rg::bf_lo(mxv)), fabsf(rg::bf_hi(mxv))));
+                const float ms = rg::warp_max_nonneg(msin);
+                if (lane == 0) {
+                    atomicMax(misc + kMiscMv / 4, __float_as_uint(mv));
+                    atomicMax(misc + kMiscSin / 4, __float_as_uint(ms));
+                }
+                ptx::named_bar_sync(kBarWG3, 128);
+                bool ok = true;
+                if (leader) {
+                    ok = wait_bar(c, SCAN_FIN, 0);
+                    if (ok) {
+                        const rg::RangePart mine{__uint_as_float(misc[kMiscMq / 4]), __uint_as_float(misc[kMiscMk / 4]),
+                                                 __uint_as_float(misc[kMiscMv / 4]), __uint_as_float(misc[kMiscSin / 4])};
+                        rec[bh].part[half] = mine;
+                        if (in_place) {
+                            // with the state carried in place, the two CTAs exchange their parts
+                            // and decide here: a flagged head's final state is not written
+                            // (pass 2 still reads it as state_in)
+                            float *peer = reinterpret_cast<float *>(c.smem + kOffMisc + kMiscPeer);
+                            const uint32_t other = (uint32_t)half ^ 1u;
+                            const float v4[4] = {mine.mq, mine.mk, mine.mv, mine.msin};
 #pragma unroll
-            for (int q = 0; q < 16; ++q)
-                *reinterpret_cast<float4 *>(state_out + sbase + 4 * q) =
-                    make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+                            for (int i = 0; i < 4; ++i)
+                                asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ptx::map_to_rank(peer + i, other)),
+                                             "f"(v4[i])
+                                             : "memory");
+                            asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                                             ptx::map_to_rank(&c.bars[PEER], other))
+                                         : "memory");
+                            ok = ptx::mbar_wait_cluster(&c.bars[PEER], 0, c.abort);
+                            if (ok) {
+                                const rg::RangePart r =
+                                    rg::combine(mine, rg::RangePart{peer[0], peer[1], peer[2], peer[3]});
+                                misc[kMiscFlag / 4] = rg::plain_ok(r, s, seq) ? 0u : 1u;
+                            }
+                        }
+                    }
+                }
+                // the leader's result (and the flag, written before this barrier) to the group
+                if (!ptx::named_bar_and(kBarWG3, 128, ok)) goto wg3_done;
+                if (in_place) write_state = write_state && misc[kMiscFlag / 4] == 0u;
+            }
+            if (write_state) {
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    *reinterpret_cast<float4 *>(state_out + sbase + 4 * q) =
+                        make_float4(S[4 * q] * f_su, S[4 * q + 1] * f_su, S[4 * q + 2] * f_su, S[4 * q + 3] * f_su);
+            }
         }
     wg3_done:;
     }
 
     ptx::tc_fence_before();
     __syncthreads();
+    // neither CTA of a cluster leaves while the other may still write into its shared memory
+    if (!kScaled && in_place) ptx::cluster_sync();
     if (warp == 2) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(c.tmem, kTmemCols);
@@ -681,26 +830,60 @@ inline bool make_map(CUtensorMap *map, const void *base, int seq, long long bh, 
 
 }  // namespace tc
 
+// Workspace of one single-CTA prefill: the range guard's record per (batch, head), 48 bytes.
+inline size_t tc_workspace_bytes(long long batch_heads) { return (size_t)batch_heads * sizeof(rg::RangeRec); }
+
+// Two launches on `stream`: the plain kernel, which measures every (batch, head)
+// into rec (tc_workspace_bytes of the caller's workspace), then pass 2, its
+// programmatic dependent, which recomputes the heads the guard flags.
 inline la_status launch_tc(const void *q, const void *k, const void *v, const float *slopes, int batch,
                            int heads, int seq, int block, const float *state_in, void *o, float *state_out,
-                           Snapshots sn, cudaStream_t stream, std::string *err) {
+                           Snapshots sn, rg::RangeRec *rec, cudaStream_t stream, std::string *err) {
     const long long bh = (long long)batch * heads;
+    if (!rec) {
+        *err = "the single-CTA prefill needs its workspace (the range guard's records)";
+        return LA_ERR_INVALID_ARG;
+    }
     CUtensorMap mq, mk, mv;
     if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
         !tc::make_map(&mv, v, seq, bh, err))
         return LA_ERR_CUDA;
-    auto kern = block == 256 ? tc::prefill_tc_kernel<2> : tc::prefill_tc_kernel<1>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes);
-    if (e != cudaSuccess) {
-        *err = std::string("cudaFuncSetAttribute(prefill_tc): ") + cudaGetErrorString(e);
-        return LA_ERR_CUDA;
-    }
-    kern<<<(unsigned)(bh * 2), tc::kThreads, tc::kSmemBytes, stream>>>(
-        mq, mk, mv, slopes, heads, seq, state_in, static_cast<__nv_bfloat16 *>(o), state_out, sn);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) {
-        *err = std::string("prefill_tc launch: ") + cudaGetErrorString(e);
-        return LA_ERR_CUDA;
+    using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, const float *, int, int, const float *,
+                            __nv_bfloat16 *, float *, Snapshots, rg::RangeRec *, const __nv_bfloat16 *,
+                            const __nv_bfloat16 *);
+    const Kernel passes[2] = {block == 256 ? tc::prefill_tc_kernel<2, false> : tc::prefill_tc_kernel<1, false>,
+                              block == 256 ? tc::prefill_tc_kernel<2, true> : tc::prefill_tc_kernel<1, true>};
+    // the state carried in place: pass 1 runs each head's two CTAs as a cluster of two
+    const bool in_place = state_out != nullptr && state_out == state_in;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(bh * 2));
+    cfg.blockDim = dim3(tc::kThreads);
+    cfg.dynamicSmemBytes = tc::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute cluster, pdl;
+    cluster.id = cudaLaunchAttributeClusterDimension;
+    cluster.val.clusterDim.x = 2;
+    cluster.val.clusterDim.y = 1;
+    cluster.val.clusterDim.z = 1;
+    // pass 2 is pass 1's programmatic dependent (it starts with griddepcontrol.wait)
+    pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl.val.programmaticStreamSerializationAllowed = 1;
+    for (int pass = 0; pass < 2; ++pass) {
+        cfg.attrs = pass == 0 ? &cluster : &pdl;
+        cfg.numAttrs = pass == 0 ? (in_place ? 1 : 0) : 1;
+        cudaError_t e = cudaFuncSetAttribute(passes[pass], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)tc::kSmemBytes);
+        if (e != cudaSuccess) {
+            *err = std::string("cudaFuncSetAttribute(prefill_tc): ") + cudaGetErrorString(e);
+            return LA_ERR_CUDA;
+        }
+        e = cudaLaunchKernelEx(&cfg, passes[pass], mq, mk, mv, slopes, heads, seq, state_in,
+                               static_cast<__nv_bfloat16 *>(o), state_out, sn, rec, static_cast<const __nv_bfloat16 *>(q),
+                               static_cast<const __nv_bfloat16 *>(k));
+        if (e != cudaSuccess) {
+            *err = std::string("prefill_tc launch: ") + cudaGetErrorString(e);
+            return LA_ERR_CUDA;
+        }
     }
     err->clear();
     return LA_OK;

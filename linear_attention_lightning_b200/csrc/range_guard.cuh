@@ -36,8 +36,9 @@
 namespace la {
 namespace rg {
 
-// The maxima one CTA of a pair measured, over its share of the head's q, k, v and
-// state_in (the pair's two shares together cover them).
+// The maxima one of a head's two CTAs measured, over its share of the head's q, k,
+// v and state_in (the two shares together cover them: the CTA pair splits the
+// rows, the single-CTA kernel's two CTAs the value columns).
 struct RangePart {
     float mq;    // largest |q| element
     float mk;    // largest |k| element
@@ -71,18 +72,6 @@ __device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
 }
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// Largest |x| over `bytes` of bf16 values (a multiple of 512), 16 bytes per lane
-// per step, consecutive lanes on consecutive chunks.
-__device__ __forceinline__ float tile_max_abs(const uint8_t *tile, int bytes, int lane) {
-    uint32_t m = 0u;
-#pragma unroll 4
-    for (int off = lane * 16; off < bytes; off += 512) {
-        const uint4 x = *reinterpret_cast<const uint4 *>(tile + off);
-        m = maxabs_bf16x2(m, maxabs_bf16x2(maxabs_bf16x2(x.x, x.y), maxabs_bf16x2(x.z, x.w)));
-    }
-    return fmaxf(fabsf(bf_lo(m)), fabsf(bf_hi(m)));
-}
 
 // Largest value over the warp (non-negative floats order like their bits; a
 // NaN, 0x7fc00000 and above, counts as the largest).

@@ -30,6 +30,8 @@ int main(void) {
     check(lightning_prefill_snapshot_count(-1, 16) == -1, "snapshot count of a bad length");
     check(lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 64 * 48,
           "the CTA-pair prefill's workspace: 48 bytes per (batch, head)");
+    check(lightning_prefill_workspace_size(1, 64, 131072, 128, 128) == 64 * 48,
+          "the single-CTA prefill's workspace: 48 bytes per (batch, head)");
     check(lightning_prefill_backward_noalloc_capacity() > 0, "no-alloc backward capacity");
     check(lightning_gqa_decode_workspace_size(8, 64, 131072) > 0, "GQA decode workspace");
     check(lightning_prefill_selected_variant(LA_DTYPE_BF16, 1, 64, 131072, 128, 256, LA_VARIANT_AUTO) ==
@@ -47,6 +49,8 @@ int main(void) {
                             state_out, NULL, 0, NULL) == LA_ERR_INVALID_ARG, "o overlapping q");
     check(lightning_prefill(fake(0), fake(1), fake(2), LA_DTYPE_BF16, slopes, 1, 2, 16, 128, 256, NULL, o, state_out,
                             NULL, 0, NULL) == LA_ERR_INVALID_ARG, "the CTA-pair prefill without its workspace");
+    check(lightning_prefill(fake(0), fake(1), fake(2), LA_DTYPE_BF16, slopes, 1, 2, 16, 128, 128, NULL, o, state_out,
+                            NULL, 0, NULL) == LA_ERR_INVALID_ARG, "the single-CTA prefill without its workspace");
     check(lightning_decode(fake(0), fake(1), fake(2), (la_dtype)7, slopes, 1, 2, 128, state, o, NULL) ==
               LA_ERR_INVALID_ARG, "bad dtype");
     check(lightning_prefill_norm_gate(fake(0), fake(1), fake(2), LA_DTYPE_F32, slopes, 1, 2, 16, 128, 256, NULL,

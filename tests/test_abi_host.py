@@ -34,11 +34,12 @@ def test_version_and_status_strings():
 
 
 def test_prefill_workspace_holds_the_range_guard_records():
-    # 48 bytes per (batch, head) for the CTA-pair kernel (block 256, dim 128); none otherwise
+    # 48 bytes per (batch, head) for the tensor-core kernels (dim 128: the CTA pair at
+    # block 256, the single-CTA kernel at block 128); none for the CUDA-core kernel
     assert abi.lightning_prefill_workspace_size(16, 64, 4096, 128, 256) == 16 * 64 * 48
     assert abi.lightning_prefill_workspace_size(1, 64, 131072, 128, 256) == 64 * 48
     assert abi.lightning_prefill_workspace_size(1, 2, 256, 64, 64) == 0
-    assert abi.lightning_prefill_workspace_size(1, 2, 256, 128, 128) == 0
+    assert abi.lightning_prefill_workspace_size(1, 2, 256, 128, 128) == 2 * 48
     assert abi.lightning_prefill_workspace_size(-1, 2, 256, 128, 256) == 0
 
 
@@ -86,6 +87,16 @@ def test_prefill_argument_errors(kw, status):
 def test_prefill_trivial_calls_need_no_gpu():
     assert _prefill(batch=0) == abi.LA_OK
     assert _prefill(seq=0, state_out=None) == abi.LA_OK
+
+
+@pytest.mark.parametrize("block", [128, 256])
+def test_single_cta_kernel_needs_its_workspace(block):
+    tc = abi.LA_VARIANT_TCGEN05
+    assert _prefill(variant=tc, block=block, pws=None, pws_bytes=0) == abi.LA_ERR_INVALID_ARG
+    assert "workspace" in abi.last_error_message()
+    assert _prefill(variant=tc, block=block, pws_bytes=48) == abi.LA_ERR_INVALID_ARG  # 2 heads need 96
+    # the CUDA-core kernel takes none
+    assert _prefill(variant=abi.LA_VARIANT_SIMT, block=block, pws=None, pws_bytes=0, batch=0) == abi.LA_OK
 
 
 def test_unknown_variant_and_unsupported_tensor_core_requests():

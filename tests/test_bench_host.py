@@ -23,6 +23,14 @@ def test_prefill_work_matches_the_stated_figures():
     assert abs(by - 8.594e9) / 8.594e9 < 1e-3
 
 
+def test_config_states_the_bytes_a_step_streams():
+    from linear_attention_lightning_b200 import inputs
+    c = bench.workload_config(inputs.WORKLOADS["m1_prefill_128k"], 1)
+    assert c["l2"] == "inputs larger than L2 (8.6 GB per step)"  # bf16 q, k, v, o + fp32 state
+    assert c["parallelism"] == "single GPU"
+    assert bench.workload_config(inputs.WORKLOADS["m1_prefill_128k"], 4)["parallelism"] == "replicas"
+
+
 def test_decode_bytes():
     # state read + written (2 * 4 * d^2) plus four bf16 vectors per (seq, head)
     assert bench.decode_bytes(1, 1, 128) == 2 * 4 * 128 * 128 + 4 * 128 * 2

@@ -3,9 +3,10 @@
 The tensor-core kernels round the operands they form to fp16 (range 2^-24 ..
 65504) while bf16 inputs span fp32's range; the pages put no normalisation on
 q or k before Q_t K_t^T ("MINIMAX SIGNAL LAB · M1", §03 Lightning Attention).
-The CTA-pair kernel carries a range guard: it measures every (batch, head)
-while it runs and recomputes, with power-of-two operand scales, the heads whose
-operands would leave fp16's range. These tests scale q, k, v and the carried
+Both tensor-core kernels (the CTA pair and the single-CTA kernel) carry a
+range guard: they measure every (batch, head) while they run and recompute,
+with power-of-two operand scales, the heads whose operands would leave fp16's
+range. These tests scale q, k, v and the carried
 state by powers of two (exact in bf16), put |q . k| above 65504 on a few rows,
 and hold every result to the bound of the workloads (max |err| <= 2e-2 rms).
 The guard's records (48 bytes per (batch, head) in the workspace) show which
@@ -25,6 +26,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 HEADS = [0, 9, 31, 63]     # fast to slow decay
 BF = torch.bfloat16
+# (variant, block): the CTA pair, and the single-CTA kernel at both of its block sizes
+KERNELS = [("pair", 256), ("tcgen05", 256), ("tcgen05", 128)]
 
 
 def _scaled(inp, eq=0, ek=0, ev=0, es=0):
@@ -73,17 +76,17 @@ def test_one_input_scaled_8k(variant, which, e):
     inp = _scaled(inputs.workload_inputs(w, DEV), **{"e" + which: e})
     o, s, flags = _prefill_with_records(inp, variant=variant)
     e_o, e_s = _check(inp, o, s)
-    if variant == "pair":
-        print("%s x 2^%d: o %.2e, state %.2e rms; %d of 64 heads took the scaled pass" % (
-            which, e, e_o, e_s, int(flags.sum())))
+    print("%s %s x 2^%d: o %.2e, state %.2e rms; %d of 64 heads took the scaled pass" % (
+        variant, which, e, e_o, e_s, int(flags.sum())))
 
 
-def test_the_workload_itself_takes_no_second_pass():
+@pytest.mark.parametrize("variant,block", KERNELS)
+def test_the_workload_itself_takes_no_second_pass(variant, block):
     # at the workloads' own scale every head passes the guard: the plain kernel's result stands
     for name in ("m1_prefill_8k", "batched_prefill_state"):
         w = inputs.WORKLOADS[name]
         inp = inputs.workload_inputs(w, DEV)
-        _, _, flags = _prefill_with_records(inp)
+        _, _, flags = _prefill_with_records(inp, block=block, variant=variant)
         assert flags.sum() == 0, name
 
 
@@ -95,10 +98,11 @@ def test_the_workload_itself_takes_no_second_pass():
     (-20, 0, 12, 0),
     (16, -16, 0, 0),
 ])
-def test_joint_scales_with_a_carried_state(eq, ek, ev, es):
+@pytest.mark.parametrize("variant,block", KERNELS)
+def test_joint_scales_with_a_carried_state(variant, block, eq, ek, ev, es):
     inp = inputs.prefill_inputs(2, 64, 1000, 128, BF, True, seed=61, device=DEV)
     inp = _scaled(inp, eq, ek, ev, es)
-    o, s, flags = _prefill_with_records(inp)
+    o, s, flags = _prefill_with_records(inp, block=block, variant=variant)
     _check(inp, o, s, heads=[0, 17, 40, 63])
     assert flags.sum() == 2 * 64, "every head is outside fp16's window and must take the scaled pass"
 
@@ -126,31 +130,40 @@ def _outlier_rows(inp, rows, mag=2.0 ** 8.5):
 
 
 @pytest.mark.parametrize("with_state", [False, True])
-def test_q_dot_k_above_65504_on_a_few_rows(with_state):
+@pytest.mark.parametrize("variant,block", KERNELS)
+def test_q_dot_k_above_65504_on_a_few_rows(variant, block, with_state):
     inp = inputs.prefill_inputs(1, 64, 8192, 128, BF, with_state, seed=62, device=DEV)
     inp = _outlier_rows(inp, rows=[5, 3000, 8000])
     qk = (inp["q"][0, :, [5, 3000, 8000]].float() * inp["k"][0, :, [5, 3000, 8000]].float()).sum(-1)
     assert float(qk.abs().min()) > 65504.0
-    o, s, flags = _prefill_with_records(inp)
+    o, s, flags = _prefill_with_records(inp, block=block, variant=variant)
     e_o, e_s = _check(inp, o, s)
     assert flags.sum() == 64
-    print("|q.k| = %.0f on 3 rows: o %.2e, state %.2e rms" % (float(qk.abs().max()), e_o, e_s))
+    print("%s B%d |q.k| = %.0f on 3 rows: o %.2e, state %.2e rms" % (variant, block, float(qk.abs().max()), e_o, e_s))
 
 
-def test_a_flagged_head_keeps_an_in_place_state_carry_intact():
-    # pass 1 must not overwrite state_in (== state_out) for a head it hands to pass 2
+@pytest.mark.parametrize("variant,block", KERNELS)
+def test_a_flagged_head_keeps_an_in_place_state_carry_intact(variant, block):
+    # pass 1 must not overwrite state_in (== state_out) for a head it hands to pass 2;
+    # heads 0-3 are scaled out of fp16's window, heads 4-7 stay in it (their state is
+    # carried by pass 1 alone)
     inp = inputs.prefill_inputs(1, 8, 700, 128, BF, True, seed=63, device=DEV)
-    inp = _scaled(inp, 9, 9, 0, 0)
+    for name in ("q", "k"):
+        x = inp[name].float()
+        x[:, :4] *= 2.0 ** 9
+        inp[name] = x.to(BF)
     ref = oracle_prefill(inp, heads_idx=list(range(8)))
     s_carry = inp["state_in"].clone()
-    o, s, flags = _prefill_with_records(dict(inp, state_in=s_carry), in_place=True)
-    assert flags.sum() == 8
+    o, s, flags = _prefill_with_records(dict(inp, state_in=s_carry), block=block, variant=variant, in_place=True)
+    assert list(flags) == [1, 1, 1, 1, 0, 0, 0, 0]
     _check(inp, o, s, heads=list(range(8)), ref=ref)
 
 
-def test_snapshots_of_a_scaled_input():
+@pytest.mark.parametrize("variant,block", KERNELS)
+def test_snapshots_of_a_scaled_input(variant, block):
     inp = _scaled(inputs.prefill_inputs(1, 4, 1024, 128, BF, True, seed=64, device=DEV), 8, 8, -8, 0)
-    o, s, snaps = la.prefill_snapshots(inp["q"], inp["k"], inp["v"], inp["slopes"], 256, 512, inp["state_in"])
+    o, s, snaps = la.prefill_snapshots(inp["q"], inp["k"], inp["v"], inp["slopes"], block, 512, inp["state_in"],
+                                       variant=variant)
     torch.cuda.synchronize()
     conv = inputs.to_oracle
     ref = oracle.snapshots(conv(inp["k"]), conv(inp["v"]), inp["slopes"].cpu().numpy(), 512,
