@@ -21,6 +21,7 @@ exchange step); times are the max over ranks.
 bounded sample of the same workload (rank 0 only).
 """
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -471,20 +472,24 @@ def run_ours(args):
     q, k, v, sl, s0 = inp["q"], inp["k"], inp["v"], inp["slopes"], inp["state_in"]
     o = torch.empty_like(q)
     s_out = torch.empty((w.batch, w.heads, w.dim, w.dim), dtype=torch.float32, device=dev)
-    variant = la.prefill_variant(w.dtype, w.batch, w.heads, w.seq, w.dim, w.block)
+    # the main leg may time another block length or kernel than the library picks
+    # for the workload (--block, --variant); the other legs keep the workload's own
+    wm = dataclasses.replace(w, block=args.block) if args.block else w
+    variant = (la.prefill_variant(wm.dtype, wm.batch, wm.heads, wm.seq, wm.dim, wm.block) if args.variant == "auto"
+               else args.variant)
     vcode = {"simt": abi.LA_VARIANT_SIMT, "tcgen05": abi.LA_VARIANT_TCGEN05,
              "pair": abi.LA_VARIANT_TCGEN05_PAIR}[variant]
     dcode = abi.LA_DTYPE_BF16 if w.dtype == torch.bfloat16 else abi.LA_DTYPE_F32
     # kernels one lightning_prefill_ex call launches: a tensor-core kernel, then its
     # range guard's second pass (which returns at once for heads it need not redo)
     launches_per_step = 2 if variant in ("pair", "tcgen05") else 1
-    need = abi.lightning_prefill_workspace_size(w.batch, w.heads, w.seq, w.dim, w.block)
+    need = abi.lightning_prefill_workspace_size(wm.batch, wm.heads, wm.seq, wm.dim, wm.block)
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 
     def step():
         abi.check(abi.lightning_prefill_ex(
-            q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), w.batch, w.heads,
-            w.seq, w.dim, w.block, None if s0 is None else s0.data_ptr(), o.data_ptr(),
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), dcode, sl.data_ptr(), wm.batch, wm.heads,
+            wm.seq, wm.dim, wm.block, None if s0 is None else s0.data_ptr(), o.data_ptr(),
             s_out.data_ptr(), ws.data_ptr(), need, sp, vcode))
 
     for _ in range(args.warmup):
@@ -508,13 +513,13 @@ def run_ours(args):
     tokens = w.batch * w.seq
     value = world * tokens * args.steps / (total_ms / 1e3)
 
-    fl = prefill_flops(w.batch, w.heads, w.seq, w.dim, w.block)
-    by = prefill_bytes(w.batch, w.heads, w.seq, w.dim, 2 if w.dtype == torch.bfloat16 else 4,
+    fl = prefill_flops(wm.batch, wm.heads, wm.seq, wm.dim, wm.block)
+    by = prefill_bytes(wm.batch, wm.heads, wm.seq, wm.dim, 2 if wm.dtype == torch.bfloat16 else 4,
                        state_in=s0 is not None, state_out=True)
     avg_launch_s = statistics.mean(per_launch_ms) / 1e3
     gbs = by / avg_launch_s / 1e9
     tflops = {kk: vv / avg_launch_s / 1e12 for kk, vv in fl.items()}
-    traffic = measured_traffic(w.name, variant)
+    traffic = measured_traffic(w.name, variant) if wm.block == w.block else None
 
     # decode: 1000 consecutive single-token steps over fp32 states
     dw = inputs.WORKLOADS[DECODE_WORKLOAD]
@@ -567,7 +572,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": workload_config(w, world),
+        "config": workload_config(wm, world),
         "kernel": variant,
         "tflops": {"formula": round(tflops["formula"], 2), "causal": round(tflops["causal"], 2),
                    "peak_bf16": peaks["bf16_tflops"],
@@ -1103,6 +1108,10 @@ def parse_args(argv=None):
                    help="timed steps of the prefill with the per-head norm + gate fused in (0: skip)")
     p.add_argument("--backward-steps", type=int, default=10,
                    help="timed steps of the gradient leg (0 skips it)")
+    p.add_argument("--variant", choices=["auto", "pair", "tcgen05", "simt"], default="auto",
+                   help="prefill kernel of the main leg (auto: the library's choice for the workload)")
+    p.add_argument("--block", type=int, default=0,
+                   help="block length of the main leg (0: the workload's own)")
     p.add_argument("--snapshot-interval", type=int, default=16384,
                    help="tokens between prefix-cache state snapshots in the snapshot leg (0 skips it)")
     a = p.parse_args(argv)
