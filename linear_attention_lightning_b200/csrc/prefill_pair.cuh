@@ -12,21 +12,20 @@
 // the pair and B operands by columns, so no product is computed twice.
 // CTA c owns
 //   - rows 128c .. 128c+127 of every block (its Q sub-tile) and the keys
-//     64c .. 64c+63 and 128+64c .. 128+64c+63 (its K sub-tile: its share of
-//     each key half's B operand),
+//     128c .. 128c+127 (its K sub-tile: its half of the B operand of Q K^T),
 //   - value columns 64c .. 64c+63 (its half of V, of the state and of the
 //     state operand), and
 //   - the key-dimension half 64c .. 64c+63 of K ⊙ d_k for the state MMA.
 // Per block:
-//   QK   SS, M256 N128 K128, bf16, twice: keys 0..127 and 128..255
-//                                      P (128 rows x 256 keys per SM, fp32 in TMEM)
+//   QK   SS, M256 N256 K128, bf16       P (128 rows x 256 keys per SM, fp32 in TMEM)
 //   QS   TS, M256 N128 K128, f16       O  = Qd S_{t-1}   (Qd = Q ⊙ d_q, fp16 in TMEM)
 //   dS   SS, M128 N128 K256, f16       S^T += V^T (K ⊙ d_k) onto e^{-s m} S^T (each
 //                                      SM: its 64 value columns x all 128 key dims)
 //   PV   TS, M256 N128 K128, f16, twice: O += P V per key half (P ⊙ D, fp16)
-// Splitting P by key halves pipelines the chain Q K^T -> P ⊙ D -> P V: one
-// half is converted while the tensor core works on the other, and the next
-// block's first half of Q K^T runs as soon as this block's first P V is done.
+// Q K^T runs as one group of 8 MMAs over all 256 keys; its two key halves of P
+// are then converted by two warpgroups side by side, and P V takes each half as
+// soon as it is converted. (Q K^T as two N = 128 groups, one per half, re-read Q
+// from shared memory and took twice the MMA instructions, for no gain.)
 // Precision as in the single-CTA kernel: Q K^T on the bf16 inputs; P ⊙ D,
 // Q ⊙ d_q, S and K ⊙ d_k rounded to fp16; V widened to fp16 exactly; fp32
 // accumulation; the fp32 state stays in TMEM for the whole sequence.
@@ -44,8 +43,7 @@
 // per-block sequence below is ordered so that this holds.
 //
 // Shared memory per CTA (1024-aligned, 128B-swizzled):
-//   Q sub-tile 32 KB, K sub-tile 32 KB (per 64-dim box: rows 0..63 keys
-//   64c.., rows 64..127 keys 128+64c..),
+//   Q sub-tile 32 KB, K sub-tile 32 KB (keys 128c .. 128c+127),
 //   2 stages x (V half for 256 keys 32 KB + K half-dims for 256 keys 32 KB),
 //   fp16 state operand 16 KB (rows = this CTA's 64 value columns),
 //   output staging 16 KB (half a row block of O, written out by TMA).
@@ -80,7 +78,7 @@ constexpr uint32_t kOffS = kOffStage + 2 * kStageBytes;
 constexpr uint32_t kSBytes = 2 * 8192;                         // 2 boxes of 64 rows x 128 B
 constexpr uint32_t kOffE = kOffS + kSBytes;                    // output staging: 128 rows x 64 bf16
 constexpr uint32_t kOffBar = kOffE + kBoxBytes;
-constexpr int kNumBars = 27;
+constexpr int kNumBars = 26;
 constexpr uint32_t kOffMisc = (kOffBar + kNumBars * 8 + 15) & ~15u;
 constexpr uint32_t kOffGamma = kOffMisc + 64;                  // fused norm + gate: gamma of the head
 constexpr uint32_t kSmemBytes = kOffGamma + kDim * 4 + 1024;
@@ -91,15 +89,15 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColP = 0, kColPHi = 128, kColO = 256, kColDS = 384, kColQd = 448;
 
 // barriers: local ones first, then the ones only the even CTA's MMA thread waits on
-// (P_FULL, P_CONV, P_FREE: one per key half, index + half)
-constexpr int QK_LOADED = 0, VK_LOADED = 1 /* 2 */, P_FULL = 3 /* 2 */, QK_DONE = 5, O_FULL = 6,
-              DS_FULL = 7, VK_EMPTY = 8 /* 2 */, P_FREE = 10 /* 2 */, QD_LOCAL = 12, QK_FULL = 13,
-              QD_READY = 14, S_READY = 15, O_FREE = 16, VK_READY = 17, DS_FREE = 18, P_CONV = 19 /* 2 */,
-              DRAIN = 21, G_FULL = 22 /* fused norm + gate: a gate half landed in the staging tile */,
+// (P_CONV, P_FREE: one per key half, index + half)
+constexpr int QK_LOADED = 0, VK_LOADED = 1 /* 2 */, P_FULL = 3, QK_DONE = 4, O_FULL = 5,
+              DS_FULL = 6, VK_EMPTY = 7 /* 2 */, P_FREE = 9 /* 2 */, QD_LOCAL = 11, QK_FULL = 12,
+              QD_READY = 13, S_READY = 14, O_FREE = 15, VK_READY = 16, DS_FREE = 17, P_CONV = 18 /* 2 */,
+              DRAIN = 20, G_FULL = 21 /* fused norm + gate: a gate half landed in the staging tile */,
               // range guard (pass 1 only): SCAN_FIN: warpgroups A and B put their maxima of
               // k, v and q in shared memory; SIN_DONE: warpgroup 3 put its maximum of state_in;
               // PEER: the other CTA's maxima landed here; RANGE_DONE: the head's verdict is set
-              SCAN_FIN = 23, SIN_DONE = 24, PEER = 25, RANGE_DONE = 26;
+              SCAN_FIN = 22, SIN_DONE = 23, PEER = 24, RANGE_DONE = 25;
 
 // shared-memory words after the barriers
 // (the maxima as float bits, which order like unsigned integers for values >= 0)
@@ -112,7 +110,7 @@ __host__ __device__ constexpr uint32_t idesc(int M, int N, uint32_t fmt, bool a_
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr uint32_t kIdescQK = idesc(256, 128, 1, false, false);  // Q (K-major) x K (K-major), bf16
+constexpr uint32_t kIdescQK = idesc(256, 256, 1, false, false);  // Q (K-major) x K (K-major), bf16
 constexpr uint32_t kIdescQS = idesc(256, 128, 0, false, false);  // Qd (TMEM) x S (K-major), f16
 constexpr uint32_t kIdescPV = idesc(256, 128, 0, false, true);   // P (TMEM) x V (MN-major), f16
 constexpr uint32_t kIdescDS = idesc(128, 128, 0, true, true);    // V^T (MN-major) x Kd (MN-major), f16
@@ -296,7 +294,7 @@ struct PairPass {
 template <bool kAnti, bool kNormGate, bool kScaled>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_k64, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_g,
                     const float *__restrict__ slopes, int heads, int seq, const float *state_in,
                     float *state_out, Snapshots sn, PairPass pp, PairNormGate ng, rg::RangeRec *rec,
@@ -386,7 +384,6 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (warp == 0 && lane == 0) {
         ptx::prefetch_tensormap(&tm_q);
         ptx::prefetch_tensormap(&tm_k);
-        ptx::prefetch_tensormap(&tm_k64);
         ptx::prefetch_tensormap(&tm_v);
         ptx::prefetch_tensormap(&tm_o);
         if (kNormGate) ptx::prefetch_tensormap(&tm_g);
@@ -429,17 +426,13 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (t > 0) ok = wait_bar(c, QK_DONE, (uint32_t)(t - 1) & 1u) && wait_bar(c, QD_LOCAL, (uint32_t)(t - 1) & 1u);
                 if (!ok) break;
                 const int row = tb(t) * kBlock + kRows * (int)rank;
-                const int krow = tb(t) * kBlock + 64 * (int)rank;
                 uint64_t *qkbar = &c.bars[QK_LOADED];
                 ptx::mbar_arrive_expect_tx(qkbar, 4 * kBoxBytes);
                 ptx::tma_load_3d(c.smem + kOffQ, &tm_q, qkbar, 0, row, bh);
                 ptx::tma_load_3d(c.smem + kOffQ + kBoxBytes, &tm_q, qkbar, 64, row, bh);
-#pragma unroll 1
-                for (int x = 0; x < 2; ++x) {
-                    uint8_t *kdst = c.smem + kOffK + x * kBoxBytes;
-                    ptx::tma_load_3d(kdst, &tm_k64, qkbar, 64 * x, krow, bh);                  // keys 64c..
-                    ptx::tma_load_3d(kdst + kBoxBytes / 2, &tm_k64, qkbar, 64 * x, krow + kRows, bh);  // 128+64c..
-                }
+                // K sub-tile: keys 128c .. 128c+127, this CTA's half of the N = 256 B operand
+                ptx::tma_load_3d(c.smem + kOffK, &tm_k, qkbar, 0, row, bh);
+                ptx::tma_load_3d(c.smem + kOffK + kBoxBytes, &tm_k, qkbar, 64, row, bh);
                 qk_issued = t + 1;
                 if (t + 1 < nblk) ok = load_vk(t + 1);
             }
@@ -501,25 +494,19 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t par = t & 1, fpar = par ^ 1u;
                 const uint64_t vdesc = dstage + (uint64_t)((uint32_t)(t & 1) * (kStageBytes >> 4));
                 const uint64_t kddesc = vdesc + (uint64_t)((2 * kBoxBytes) >> 4);
-                // P = Q K^T, one key half at a time, each once the previous
-                // block's P V for that half has read its columns
-#pragma unroll 1
-                for (int h = 0; h < 2 && ok; ++h) {
-                    ok = (h > 0 || wait_pair(c, QK_FULL, par)) && wait_bar(c, P_FREE + h, fpar);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                    const uint64_t dkh = dk + (uint64_t)(h * (kBoxBytes / 2) >> 4);
-                    if (elect_one()) {
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
-                            ptx::mma_ss_2(tm + kColP + kColPHi * h, dq + koff, dkh + koff, kIdescQK, k > 0);
-                        }
-                        ptx::mma_commit_2_mc(&c.bars[P_FULL + h], 0x3);
-                    }
-                    __syncwarp();
-                }
+                // P = Q K^T for all 256 keys, once the previous block's P V has read P
+                ok = wait_pair(c, QK_FULL, par) && wait_bar(c, P_FREE, fpar) && wait_bar(c, P_FREE + 1, fpar);
                 if (!ok) break;
+                ptx::tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint64_t koff = (uint64_t)(((k >> 2) * kBoxBytes + (k & 3) * 32) >> 4);
+                        ptx::mma_ss_2(tm + kColP, dq + koff, dk + koff, kIdescQK, k > 0);
+                    }
+                    ptx::mma_commit_2_mc(&c.bars[P_FULL], 0x3);
+                }
+                __syncwarp();
                 if (elect_one()) ptx::mma_commit_2_mc(&c.bars[QK_DONE], 0x3);
                 __syncwarp();
                 // O = Qd S_{t-1}
@@ -653,7 +640,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // P ⊙ D -> fp16 for keys [128 grp, 128 grp + 128); the quadrant the mask
             // zeroes (causal: rows 0..127 x keys 128..255; anti-causal: rows
             // 128..255 x keys 0..127) is only cleared
-            if (!group_wait(c, P_FULL + grp, par, leader, bar_id)) goto ab_done;
+            if (!group_wait(c, P_FULL, par, leader, bar_id)) goto ab_done;
             ptx::tc_fence_after();
             if (kAnti ? (grp == 0 && rank == 1) : (grp == 1 && rank == 0)) {
                 // every entry of this quadrant is masked
@@ -998,9 +985,9 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
         *err = "the CTA-pair prefill needs its workspace (the range guard's records)";
         return LA_ERR_INVALID_ARG;
     }
-    CUtensorMap mq, mk, mk64, mv, mo, mg;
+    CUtensorMap mq, mk, mv, mo, mg;
     if (!tc::make_map(&mq, q, seq, bh, err) || !tc::make_map(&mk, k, seq, bh, err) ||
-        !tc::make_map(&mk64, k, seq, bh, err, 64) || !tc::make_map(&mv, v, seq, bh, err) ||
+        !tc::make_map(&mv, v, seq, bh, err) ||
         !(ng ? make_token_major_map(&mo, o, batch, heads, seq, err) : tc::make_map(&mo, o, seq, bh, err)))
         return LA_ERR_CUDA;
     if (ng) {
@@ -1009,7 +996,7 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
     } else {
         mg = mo;  // unused
     }
-    using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+    using Kernel = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
                             const float *, int, int, const float *, float *, Snapshots, pair::PairPass,
                             pair::PairNormGate, rg::RangeRec *, const __nv_bfloat16 *, const __nv_bfloat16 *);
     const Kernel passes[2] = {
@@ -1040,7 +1027,7 @@ inline la_status launch_pair(const void *q, const void *k, const void *v, const 
             *err = std::string("cudaFuncSetAttribute(prefill_pair): ") + cudaGetErrorString(e);
             return LA_ERR_CUDA;
         }
-        e = cudaLaunchKernelEx(&cfg, passes[pass], mq, mk, mk64, mv, mo, mg, slopes, heads, seq, state_in,
+        e = cudaLaunchKernelEx(&cfg, passes[pass], mq, mk, mv, mo, mg, slopes, heads, seq, state_in,
                                state_out, sn, pp, ngv, rec, static_cast<const __nv_bfloat16 *>(q),
                                static_cast<const __nv_bfloat16 *>(k));
         if (e != cudaSuccess) {

@@ -808,15 +808,14 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn(std::string *err) {
 }
 
 // [batch*heads][seq][128] bf16 viewed as a 3-D tensor; boxes of 64 dims x
-// box_rows rows, 128-byte swizzle; rows past seq read as zeros and are
-// clipped on store.
-inline bool make_map(CUtensorMap *map, const void *base, int seq, long long bh, std::string *err,
-                     int box_rows = kRows) {
+// 128 rows, 128-byte swizzle; rows past seq read as zeros and are clipped on
+// store.
+inline bool make_map(CUtensorMap *map, const void *base, int seq, long long bh, std::string *err) {
     auto fn = encode_fn(err);
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kDim, (cuuint64_t)seq, (cuuint64_t)bh};
     cuuint64_t strides[2] = {(cuuint64_t)kDim * 2, (cuuint64_t)seq * kDim * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)kRows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
