@@ -31,6 +31,12 @@ def test_config_states_the_bytes_a_step_streams():
     assert bench.workload_config(inputs.WORKLOADS["m1_prefill_128k"], 4)["parallelism"] == "replicas"
 
 
+def test_long_tensor_bound_legs_are_held_to_the_sustained_peak():
+    peaks = {"bf16_tflops": 1656.8, "bf16_tflops_sustained": 1388.7}
+    assert bench.tensor_peak(peaks, 0.72) == (1388.7, "sustained")   # 3 steps of 240 ms
+    assert bench.tensor_peak(peaks, 0.036) == (1656.8, "burst")      # 20 steps of 1.8 ms
+
+
 def test_decode_bytes():
     # state read + written (2 * 4 * d^2) plus four bf16 vectors per (seq, head)
     assert bench.decode_bytes(1, 1, 128) == 2 * 4 * 128 * 128 + 4 * 128 * 2
