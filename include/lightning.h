@@ -42,6 +42,12 @@
  *     lightning_last_device_status() returns it on demand (see there).
  *   - A human-readable reason for the last failure on the calling thread is
  *     returned by lightning_last_error_message().
+ *   - lightning_prefill, lightning_prefill_ex, lightning_decode and
+ *     lightning_prefill_backward may be recorded into a CUDA graph by stream
+ *     capture. Their launches use only `stream` (the backward also uses the
+ *     library's side streams, forked from and joined to it with events), so
+ *     replaying the graph repeats the call. The host-side argument checks and
+ *     the status-word check run once, when the call is recorded.
  */
 #ifndef LIGHTNING_H
 #define LIGHTNING_H
