@@ -29,17 +29,6 @@ constexpr int kGqaChunk = 2048;        // positions per CTA
 constexpr int kGqaDim = 128;
 constexpr int kGqaMaxGroup = 8;        // query heads per KV head
 
-// d = a * b + c on two fp32 lanes at once (one paired FMA: two IEEE fp32 FMAs)
-__device__ __forceinline__ float2 gqa_fma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-
 template <typename T> __device__ __forceinline__ void gqa_store(T *p, float x);
 template <> __device__ __forceinline__ void gqa_store<float>(float *p, float x) { *p = x; }
 template <> __device__ __forceinline__ void gqa_store<__nv_bfloat16>(__nv_bfloat16 *p, float x) {
@@ -216,8 +205,8 @@ gqa_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
                     for (int e4 = 0; e4 < EV; e4 += 4) {
                         const float4 qv = *reinterpret_cast<const float4 *>(&qs[g][c * EV + e4]);
-                        dot2[g] = gqa_fma2(make_float2(qv.x, qv.y), make_float2(kf[e4], kf[e4 + 1]), dot2[g]);
-                        dot2[g] = gqa_fma2(make_float2(qv.z, qv.w), make_float2(kf[e4 + 2], kf[e4 + 3]), dot2[g]);
+                        dot2[g] = ptx::fma2(make_float2(qv.x, qv.y), make_float2(kf[e4], kf[e4 + 1]), dot2[g]);
+                        dot2[g] = ptx::fma2(make_float2(qv.z, qv.w), make_float2(kf[e4 + 2], kf[e4 + 3]), dot2[g]);
                     }
             }
             float dot[G];
@@ -291,9 +280,9 @@ gqa_partial_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             const float wv[G] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float2 lo = gqa_fma2(make_float2(wv[g], wv[g]), make_float2(vf[0], vf[1]),
+                const float2 lo = ptx::fma2(make_float2(wv[g], wv[g]), make_float2(vf[0], vf[1]),
                                            make_float2(acc[g][0], acc[g][1]));
-                const float2 hi = gqa_fma2(make_float2(wv[g], wv[g]), make_float2(vf[2], vf[3]),
+                const float2 hi = ptx::fma2(make_float2(wv[g], wv[g]), make_float2(vf[2], vf[3]),
                                            make_float2(acc[g][2], acc[g][3]));
                 acc[g][0] = lo.x; acc[g][1] = lo.y; acc[g][2] = hi.x; acc[g][3] = hi.y;
             }

@@ -215,15 +215,7 @@ __device__ __forceinline__ bool wait_bar(const Ctx &c, int idx, uint32_t parity)
     return ptx::mbar_wait(&c.bars[idx], parity, c.abort);
 }
 
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
+using ptx::fma2;
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;

@@ -159,7 +159,6 @@ __device__ __forceinline__ bool group_wait(const Ctx &c, int idx, uint32_t parit
     const bool ok = leader ? wait_bar(c, idx, parity) : true;
     return ptx::named_bar_and(bar_id, 128, ok);
 }
-using ptx::add2;
 using ptx::mul2;
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w, float scale) {
@@ -865,8 +864,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int hh = 0; hh < 2; ++hh) {
                     if (kNormGate) {
                         // y = gamma o rstd sigmoid(g) on this half's 64 columns, written over the
-                        // gate row in the staging tile, as (gamma rstd / 2) o (1 + tanh(g/2)) in
-                        // paired fp32 operations (SFU tanh)
+                        // gate row in the staging tile, as a + a tanh(g/2) with a = (gamma rstd / 2) o,
+                        // in paired fp32 operations (SFU tanh)
                         if (hh == 1 && leader) load_gate(t, 1);
                         if (!group_wait(c, G_FULL, (uint32_t)hh, leader, kBarW3)) goto w3_done;
 #pragma unroll
@@ -888,7 +887,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                 asm("tanh.approx.f32 %0, %1;" : "=f"(th1) : "f"(ga.y));
                                 const float2 cg = mul2(make_float2(gm[2 * e], gm[2 * e + 1]), make_float2(hr, hr));
                                 const float2 a = mul2(cg, make_float2(ptx::bf16_lo(w), ptx::bf16_hi(w)));
-                                const float2 yv = mul2(a, add2(make_float2(th0, th1), make_float2(1.f, 1.f)));
+                                const float2 yv = ptx::fma2(a, make_float2(th0, th1), a);  // a (1 + tanh)
                                 yw[e] = ptx::pack_bf16(yv.x, yv.y);
                             }
                             *slot = make_uint4(yw[0], yw[1], yw[2], yw[3]);
