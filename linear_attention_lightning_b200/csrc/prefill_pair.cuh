@@ -832,7 +832,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ptx::tc_fence_after();
             {
                 uint32_t pk[64];  // the whole output row as bf16 pairs
-                float ss = 0.f;   // fused norm + gate: the row's sum of squares (fp32 values)
+                float2 ss2 = make_float2(0.f, 0.f);  // fused norm + gate: the row's sum of squares, in two parts
 #pragma unroll
                 for (int cb = 0; cb < 4; cb += 2) {
                     // two loads in flight per wait: O_FREE is on the path to the next block's first MMA
@@ -847,10 +847,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         pk[16 * cb + u] = ptx::pack_bf16(x0, x1);
                         pk[16 * cb + 16 + u] = ptx::pack_bf16(y0, y1);
                         if (kNormGate) {
-                            ss = fmaf(x0, x0, ss);
-                            ss = fmaf(x1, x1, ss);
-                            ss = fmaf(y0, y0, ss);
-                            ss = fmaf(y1, y1, ss);
+                            ss2 = ptx::fma2(make_float2(x0, x1), make_float2(x0, x1), ss2);
+                            ss2 = ptx::fma2(make_float2(y0, y1), make_float2(y0, y1), ss2);
                         }
                     }
                 }
@@ -858,7 +856,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::named_bar_sync(kBarW3, 128);
                 if (leader) arrive_leader(&c.bars[O_FREE]);
                 uint8_t *erow = c.smem + kOffE + l * 128;
-                const float rstd = kNormGate ? rsqrtf(ss * (1.f / kDim) + ng.eps) : 0.f;
+                const float rstd = kNormGate ? rsqrtf((ss2.x + ss2.y) * (1.f / kDim) + ng.eps) : 0.f;
                 const float hr = 0.5f * rstd;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
