@@ -259,18 +259,12 @@ la_status launch_norm_gate(const NgArgs &a) {
     long long tile = (long long)la::kNgTileBytes / (n_ch * (long long)eb);
     tile = tile < 1 ? 1 : (tile > 64 ? 64 : tile);
     const bool bf16 = sizeof(T) == 2;
-    CUtensorMap mo, mg;
+    CUtensorMap mo;
     // o: [batch*heads][seq][dim], box = one tile of tokens for every head of a batch
     const cuuint64_t odims[3] = {(cuuint64_t)a.dim, (cuuint64_t)a.seq, (cuuint64_t)a.batch * a.heads};
     const cuuint64_t ostr[2] = {(cuuint64_t)a.dim * eb, (cuuint64_t)a.seq * a.dim * eb};
     const cuuint32_t obox[3] = {(cuuint32_t)a.dim, (cuuint32_t)tile, (cuuint32_t)a.heads};
-    // gate: [batch*seq][heads][dim], box = one tile of tokens
-    const cuuint64_t gdims[3] = {(cuuint64_t)a.dim, (cuuint64_t)a.heads, (cuuint64_t)a.batch * a.seq};
-    const cuuint64_t gstr[2] = {(cuuint64_t)a.dim * eb, (cuuint64_t)n_ch * eb};
-    const cuuint32_t gbox[3] = {(cuuint32_t)a.dim, (cuuint32_t)a.heads, (cuuint32_t)tile};
-    if (!make_plain_map(&mo, a.o, bf16, odims, ostr, obox, &g_last_error) ||
-        !make_plain_map(&mg, a.gate, bf16, gdims, gstr, gbox, &g_last_error))
-        return LA_ERR_CUDA;
+    if (!make_plain_map(&mo, a.o, bf16, odims, ostr, obox, &g_last_error)) return LA_ERR_CUDA;
     auto kern = la::norm_gate_kernel<T, U>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)la::kNgSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(norm_gate)");
@@ -278,8 +272,9 @@ la_status launch_norm_gate(const NgArgs &a) {
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long tiles = (long long)a.batch * ((a.seq + tile - 1) / tile);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    kern<<<grid, la::kNgThreads, la::kNgSmemBytes, a.stream>>>(mo, mg, a.gamma, a.eps, a.batch, a.heads, a.seq, a.dim,
-                                                              a.per_head, (int)tile, static_cast<T *>(a.y));
+    kern<<<grid, la::kNgThreads, la::kNgSmemBytes, a.stream>>>(mo, static_cast<const T *>(a.gate), a.gamma, a.eps,
+                                                              a.batch, a.heads, a.seq, a.dim, a.per_head, (int)tile,
+                                                              static_cast<T *>(a.y));
     e = cudaGetLastError();
     return e == cudaSuccess ? ok() : cuda_fail(e, "norm_gate launch");
 }

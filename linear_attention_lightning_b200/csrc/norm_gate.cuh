@@ -10,8 +10,10 @@
 // Bound by HBM: o, g read and y written once. A persistent CTA per SM streams
 // tiles of `tile` consecutive tokens of one batch through a kNgStages-deep TMA
 // pipeline in shared memory: one 3-D box brings a tile's o for every head
-// (o is [batch*heads][seq][dim]), one more the tile's gate; two tiles stay in
-// flight while the warps work on the third. The CTA's two groups of 256
+// (o is [batch*heads][seq][dim]); two tiles stay in flight while the warps work
+// on the third. The tile's gate rows, contiguous in g, are prefetched into L2 by
+// one bulk copy when its o is requested, and read from there with 16-byte loads
+// (a token's gate row is contiguous, as is its y row). The CTA's two groups of 256
 // threads take alternate tokens of a tile, each on its own named barrier, so
 // two tokens' reductions are in flight per SM. In a group each thread takes U
 // 16-byte chunks of a token's row; a head's chunks sit in dim/E consecutive
@@ -32,8 +34,14 @@ constexpr int kNgThreads = 512;
 constexpr int kNgGroup = 256;                   // threads per token group (two groups per CTA)
 constexpr int kNgMaxChunks = 8;                 // heads*dim <= kNgGroup * kNgMaxChunks * (16 / sizeof(T))
 constexpr int kNgStages = 3;
-constexpr uint32_t kNgTileBytes = 32768;        // one tile of o (and one of gate) at most
-constexpr uint32_t kNgSmemBytes = kNgStages * 2 * kNgTileBytes + 64 + 128;
+constexpr uint32_t kNgTileBytes = 65536;        // one tile of o at most
+constexpr uint32_t kNgSmemBytes = kNgStages * kNgTileBytes + 64 + 128;
+
+// Bulk prefetch of `bytes` contiguous bytes into L2 (address and size multiples of 16).
+__device__ __forceinline__ void ng_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
 
 template <typename T> struct NgVec;
 template <> struct NgVec<float> {
@@ -70,7 +78,7 @@ template <> struct NgVec<__nv_bfloat16> {
 // tile: tokens per tile (tile * heads * dim * sizeof(T) <= kNgTileBytes).
 template <typename T, int U>
 __global__ void __launch_bounds__(kNgThreads, 1)
-norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_g,
+norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const T *__restrict__ g,
                  const float *__restrict__ gamma, float eps, int batch, int heads, int seq, int dim, int per_head,
                  int tile, T *__restrict__ y) {
     using V = NgVec<T>;
@@ -78,7 +86,7 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
     extern __shared__ uint8_t ng_smem_raw[];
     const uint32_t raw = ptx::smem_addr(ng_smem_raw);
     uint8_t *smem = ng_smem_raw + (((raw + 127u) & ~127u) - raw);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kNgStages * 2 * kNgTileBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kNgStages * kNgTileBytes);
     uint64_t *empty = full + kNgStages;
     int *abort_flag = reinterpret_cast<int *>(empty + kNgStages);
 
@@ -101,7 +109,6 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
         *abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tensormap(&tm_o);
-        ptx::prefetch_tensormap(&tm_g);
     }
     __syncthreads();
 
@@ -112,10 +119,10 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
         const int s = (int)(it % kNgStages);
         if (it >= kNgStages && !ptx::mbar_wait(&empty[s], (uint32_t)((it / kNgStages - 1) & 1), abort_flag)) return;
         const int b = (int)(gt / tiles_per_batch), l0 = (int)(gt - (long long)b * tiles_per_batch) * tile;
-        uint8_t *os = smem + s * 2 * kNgTileBytes;
-        ptx::mbar_arrive_expect_tx(&full[s], 2 * box_bytes);
+        uint8_t *os = smem + s * kNgTileBytes;
+        ptx::mbar_arrive_expect_tx(&full[s], box_bytes);
         ptx::tma_load_3d(os, &tm_o, &full[s], 0, l0, b * heads);
-        ptx::tma_load_3d(os + kNgTileBytes, &tm_g, &full[s], 0, 0, b * seq + l0);
+        ng_prefetch_l2(g + ((long long)b * seq + l0) * n_ch, (uint32_t)(min(tile, seq - l0) * n_ch * sizeof(T)));
     };
     if (threadIdx.x == 0)
         for (int it = 0; it < kNgStages - 1; ++it) issue(it);
@@ -127,9 +134,20 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
         const long long gt = blockIdx.x + it * gridDim.x;
         const int b = (int)(gt / tiles_per_batch), l0 = (int)(gt - (long long)b * tiles_per_batch) * tile;
         const int tcount = min(tile, seq - l0);
-        const T *os = reinterpret_cast<const T *>(smem + s * 2 * kNgTileBytes);
-        const T *gs = reinterpret_cast<const T *>(smem + s * 2 * kNgTileBytes + kNgTileBytes);
+        const T *os = reinterpret_cast<const T *>(smem + s * kNgTileBytes);
         for (int t = grp; t < tcount; t += 2) {
+            // the token's gate chunks first, so that their loads (from L2) overlap the
+            // sums; at U = 8 (16-bit) they are loaded where used, to stay in registers
+            constexpr bool kEarlyGate = U * E <= 32;
+            const T *grow = g + ((long long)b * seq + l0 + t) * n_ch;
+            uint4 gw[U];
+            if (kEarlyGate) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int k = gtid + kNgGroup * u;
+                    if (k < chunks) gw[u] = __ldcs(reinterpret_cast<const uint4 *>(grow + k * E));
+                }
+            }
             float x[U][8], ss[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -172,7 +190,7 @@ norm_gate_kernel(const __grid_constant__ CUtensorMap tm_o, const __grid_constant
                     const int n0 = k * E;
                     const float inv = rsqrtf(ss[u] * inv_group + eps);
                     float gv[8], out[8];
-                    V::unpack(*reinterpret_cast<const uint4 *>(gs + (size_t)t * n_ch + n0), gv);
+                    V::unpack(kEarlyGate ? gw[u] : __ldcs(reinterpret_cast<const uint4 *>(grow + n0)), gv);
                     float gm[8];
 #pragma unroll
                     for (int e = 0; e < E; e += 4) {
