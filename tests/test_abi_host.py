@@ -257,8 +257,10 @@ def _norm_gate(**kw):
     (dict(heads=129), abi.LA_ERR_UNSUPPORTED),                           # 16512 bf16 channels per token
     (dict(heads=65, dtype=abi.LA_DTYPE_F32), abi.LA_ERR_UNSUPPORTED),    # 8320 f32 channels
     (dict(gate=None), abi.LA_ERR_INVALID_ARG),
+    (dict(gate=G_ + 8), abi.LA_ERR_INVALID_ARG),  # the kernel reads the gate by 16-byte loads and a bulk L2 prefetch
     (dict(y=Y_ + 4), abi.LA_ERR_INVALID_ARG),
     (dict(y=O + 1024), abi.LA_ERR_INVALID_ARG),                          # overlaps o
+    (dict(y=G_ + 1024), abi.LA_ERR_INVALID_ARG),                         # overlaps the gate
 ])
 def test_norm_gate_argument_errors(kw, status):
     assert _norm_gate(**kw) == status
