@@ -51,6 +51,25 @@ MUTATIONS = [
      "ROPE_NEW(qr, i);", "ROPE_NEW(qr, i + 1);", 0),
     ("gqa prefill: a query does not see its own key",
      "const long P = (long)start + i;", "const long P = (long)start + i - 1;", 0),
+    ("blockwise: query decay one step short",
+     "const double dq = exp(-s * (double)(i + 1)); /* query decay d_q[i] */",
+     "const double dq = exp(-s * (double)(i)); /* query decay d_q[i] */", 0),
+    ("backward: dk from the transposed gradient state",
+     "acc += R[r * d + c] * V[jj * d + c];", "acc += R[c * d + r] * V[jj * d + c];", 0),
+    ("backward: the state-in gradient not decayed",
+     "const double f = L > 0 ? decay : 1.0;", "const double f = 1.0;", 0),
+    ("decode: the output read from k",
+     "const double qr = widen(q, dtype, base + r);", "const double qr = widen(k, dtype, base + r);", 0),
+    ("norm_gate: eps added outside the square root",
+     "1.0 / sqrt(ss / (double)group + eps);", "1.0 / (sqrt(ss / (double)group) + eps);", 0),
+    ("norm_gate: the weight of the head's channel only",
+     "(double)gamma[n] * x * inv", "(double)gamma[n % d] * x * inv", 0),
+    ("rope: frequencies halved",
+     "pow(base, -2.0 * i / (double)rot)", "pow(base, -1.0 * i / (double)rot)", 0),
+    ("gqa decode: KV head by modulo instead of by group",
+     "hk = h / group;", "hk = h % kv_heads;", 0),
+    ("gqa prefill: scores not scaled",
+     "sc[p] = scale * dot;", "sc[p] = dot;", 1),
 ]
 
 
